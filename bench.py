@@ -1,0 +1,469 @@
+"""Benchmark of the mLSTM cell forward and decode step on B200.
+
+Default run (N = 1): the long-context forward (B=1, NH=8, S=16384, DH=256,
+bf16 q/k/v, fp32 gates and state) is the timed step; one step is one full
+forward over that batch (gate prologue, segment summaries, chunkwise outputs
+and final state).  The decode step workload (B=256, NH=8, DH=512, fp32 state,
+1024 consecutive tokens after a 512-token prefill) is timed in the same run and
+reported under "decode".  Inputs are seeded synthetic tensors of those shapes.
+
+Under torchrun (N > 1) every rank runs its own replica of the same workload on
+its own GPU (heads are independent, so the batch shards with no collective);
+the timed region is bracketed by barriers and device syncs and the max over
+ranks is reported.  ``--impl reference`` times the float64 CPU oracle instead
+(rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from linear_rnn_mlstm_b200 import binding as xb  # noqa: E402
+from linear_rnn_mlstm_b200 import synthetic as syn  # noqa: E402
+
+METRIC = "mLSTM fwd tokens/s & % bf16 TC peak; decode-step HBM GB/s vs peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ------------------------------------------------------------------ helpers
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {k: float(p[k]) for k in FALLBACK_PEAKS}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def fwd_flops(BH, S, DH, L):
+    """Useful flops of the chunkwise forward: inter retrieval and state update
+    (2*DH^2 each per token) and the causal-exact intra part ((L+1)*DH each for
+    scores and values per token on average)."""
+    return BH * S * (4.0 * DH * DH + 2.0 * (L + 1) * DH)
+
+
+def fwd_token_bytes(DH, qkv_bytes):
+    """Algorithmic HBM bytes per token: q, k, v, h in the q dtype, otilde fp32
+    per element, itilde and ftilde fp32."""
+    return 4 * DH * qkv_bytes + 4 * DH + 8
+
+
+def state_bytes(BH, DH):
+    return BH * 4 * (DH * DH + DH + 1)
+
+
+def kernel_algorithmic_bytes(name, w, plan):
+    """Bytes a launch of kernel `name` must move over one forward of `w`."""
+    BH, S, DH = w.B * w.NH, w.S, w.DH
+    qb = 2 if w.dtype == "bf16" else 4
+    if name.startswith("segment_output"):
+        return BH * S * fwd_token_bytes(DH, qb) + state_bytes(BH, DH)
+    if name.startswith("segment_summary"):
+        seg_tokens = BH * S * (plan["P"] - 1) / max(plan["P"], 1)
+        return seg_tokens * (2 * DH * qb + 8) + BH * (plan["P"] - 1) * 4 * (DH * DH + DH)
+    if name == "gate_prologue":
+        return BH * S * 12
+    return None
+
+
+def source_sha(kernel):
+    files = {"segment_output_simt": "fwd_simt.cu", "segment_summary_simt": "fwd_simt.cu",
+             "gate_prologue": "fwd_simt.cu", "step_rows": "step.cu", "step_state": "step.cu"}
+    fn = files.get(kernel)
+    if fn is None and kernel.endswith("_tc"):
+        fn = "fwd_tc.cu"
+    if fn is None:
+        return None
+    with open(os.path.join(ROOT, "linear_rnn_mlstm_b200", "csrc", fn), "rb") as f:
+        return hashlib.sha1(f.read()).hexdigest()
+
+
+def ncu_traffic(kernel, units):
+    """DRAM bytes per launch from the committed ncu summary, scaled to `units`
+    processed, if the kernel source is unchanged since the capture; else None."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f).get(kernel)
+    except Exception:
+        return None
+    if not rec or rec.get("source_sha") != source_sha(kernel):
+        return None
+    return rec["dram_bytes_per_unit"] * units
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 100 ms."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.samples = []
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(gpu_index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) == 7:
+                self.samples.append(parts)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for p in self.samples:
+            try:
+                sm.append(float(p[0]))
+                mx = float(p[1])
+            except ValueError:
+                continue
+            for nm, val in zip(names, p[3:]):
+                if val.lower().startswith("active"):
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def physical_gpu_index(local_rank):
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        items = [x.strip() for x in vis.split(",") if x.strip()]
+        if local_rank < len(items):
+            return items[local_rank]
+    return str(local_rank)
+
+
+# ------------------------------------------------------------ oracle (CPU)
+def cpu_baseline(w, max_tokens_per_head):
+    """The float64 oracle as it stands, on a bounded sample of workload `w`:
+    all heads, the first `max_tokens_per_head` tokens of each.  Returns the
+    baseline record (tokens/s)."""
+    import oracle
+    S = min(w.S, max_tokens_per_head)
+    inp = syn.fwd_inputs(w)
+    sub = {k: v[:, :, :S] for k, v in inp.items()}
+    t0 = time.perf_counter()
+    oracle.fwd(sub["q"], sub["k"], sub["v"], sub["i_pre"], sub["f_pre"], sub["o_pre"], w.fgate)
+    dt = time.perf_counter() - t0
+    toks = w.B * w.NH * S
+    cores = min(oracle.max_threads(), w.B * w.NH)
+    return {"value": toks / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"{w.B * w.NH} heads x first {S} tokens of the {w.name} workload "
+                      f"({toks} tokens, {dt:.2f} s wall)"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import oracle
+    w = syn.WORKLOADS[args.config]
+    S = min(w.S, args.ref_tokens)
+    inp = syn.fwd_inputs(w)
+    sub = {k: v[:, :, :S] for k, v in inp.items()}
+    run = lambda: oracle.fwd(sub["q"], sub["k"], sub["v"], sub["i_pre"], sub["f_pre"],
+                             sub["o_pre"], w.fgate)
+    for _ in range(args.warmup):
+        run()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        run()
+    dt = (time.perf_counter() - t0) / args.steps
+    toks = w.B * w.NH * S
+    value = toks / dt
+    cores = min(oracle.max_threads(), w.B * w.NH)
+    sample = f"{w.B * w.NH} heads x first {S} tokens of the {w.name} workload per step"
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": workload_config(w, args.chunk, args.gpus),
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(w, chunk, n):
+    return {"workload": f"{w.name} mLSTM fwd: B={w.B} NH={w.NH} S={w.S} DH={w.DH} {w.dtype} q/k/v, "
+                        f"{w.fgate} forget gate, chunk {chunk}",
+            "B": w.B, "NH": w.NH, "S": w.S, "DH": w.DH, "chunk": chunk,
+            "global_batch": w.B * n, "seq_len": w.S, "parallelism": f"replicas x{n} (heads independent)"}
+
+
+# ----------------------------------------------------------------- GPU arm
+def make_fwd_runner(x, w, chunk, dev, path):
+    BH = w.B * w.NH
+    h = torch.empty_like(x["q"])
+    C = torch.empty((w.B, w.NH, w.DH, w.DH), dtype=torch.float32, device=dev)
+    n = torch.empty((w.B, w.NH, w.DH), dtype=torch.float32, device=dev)
+    m = torch.empty((w.B, w.NH), dtype=torch.float32, device=dev)
+    dt = xb.BF16 if w.dtype == "bf16" else xb.F32
+    fg = xb.FGATE_EXP if w.fgate == "exp" else xb.FGATE_SIGMOID
+    st, nbytes = xb.xlstm_mlstm_fwd_workspace_size(w.B, w.NH, w.S, w.DH, chunk, dt, path)
+    assert st == xb.OK, xb.status_string(st)
+    ws = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev).cuda_stream
+    ptrs = [x[k].data_ptr() for k in ("q", "k", "v", "i_pre", "f_pre", "o_pre")]
+
+    def run():
+        s = xb.xlstm_mlstm_fwd(*ptrs, h.data_ptr(), None, None, None, C.data_ptr(), n.data_ptr(),
+                               m.data_ptr(), w.B, w.NH, w.S, w.DH, chunk, dt, fg, ws.data_ptr(),
+                               ws.numel(), stream, path)
+        if s != xb.OK:
+            raise xb.XlstmError(s, "xlstm_mlstm_fwd")
+    return run, (h, C, n, m), BH
+
+
+def time_region(fn, steps, dist_on, dev):
+    if dist_on:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        fn()
+    e1.record()
+    torch.cuda.synchronize(dev)
+    if dist_on:
+        torch.distributed.barrier()
+    ms = e0.elapsed_time(e1)
+    if dist_on:
+        t = torch.tensor([ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    return ms
+
+
+def plan_info(w, chunk, path):
+    # segments chosen by the library: recover P from the workspace size
+    BH, DH = w.B * w.NH, w.DH
+    dt = xb.BF16 if w.dtype == "bf16" else xb.F32
+    _, base = xb.xlstm_mlstm_fwd_workspace_size(w.B, w.NH, w.S, DH, chunk, dt, path, 1)
+    _, auto = xb.xlstm_mlstm_fwd_workspace_size(w.B, w.NH, w.S, DH, chunk, dt, path, 0)
+    per_seg = BH * (DH * DH + DH) * 4
+    P = 1 + max(0, round((auto - base) / per_seg))
+    return {"P": P}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--config", default="long", choices=sorted(syn.WORKLOADS))
+    ap.add_argument("--chunk", type=int, default=64)
+    ap.add_argument("--path", default="auto", choices=["auto", "simt", "tensor"])
+    ap.add_argument("--decode-steps", type=int, default=1024)
+    ap.add_argument("--skip-decode", action="store_true")
+    ap.add_argument("--skip-e2e", action="store_true")
+    ap.add_argument("--skip-cpu", action="store_true")
+    ap.add_argument("--ref-tokens", type=int, default=4096,
+                    help="tokens per head in each reference (oracle) step")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    dist_on = world > 1
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    if dist_on:
+        import datetime
+        torch.distributed.init_process_group("nccl", device_id=dev,
+                                             timeout=datetime.timedelta(seconds=300))
+    xb.load()
+    peaks, peak_src = load_peaks()
+    path = {"auto": xb.PATH_AUTO, "simt": xb.PATH_SIMT, "tensor": xb.PATH_TENSOR}[args.path]
+
+    # ------------------------------------------------------------ forward
+    w = syn.WORKLOADS[args.config]
+    inp = syn.fwd_inputs(w, seed=w.seed + rank)
+    x = {k: v.to(dev).contiguous() for k, v in inp.items()}
+    run, outs, BH = make_fwd_runner(x, w, args.chunk, dev, path)
+    sampler = ClockSampler(physical_gpu_index(local_rank)) if rank == 0 else None
+    for _ in range(args.warmup):
+        run()
+    torch.cuda.synchronize(dev)
+    xb.xlstm_profile_begin()
+    ms = time_region(run, args.steps, dist_on, dev)
+    _, kt = xb.xlstm_profile_end()
+    ms_step = ms / args.steps
+    tokens = w.B * w.NH * w.S
+    value = tokens * world / (ms_step * 1e-3)
+    launches = sum(v[0] for v in kt.values())
+    kernels = {k: {"launches": v[0], "avg_us": 1e3 * v[1] / max(v[0], 1),
+                   "share": v[1] / max(sum(u[1] for u in kt.values()), 1e-12)}
+               for k, v in kt.items()}
+    top = max(kt.items(), key=lambda kv: kv[1][1])[0] if kt else None
+    plan = plan_info(w, args.chunk, path)
+    alg = kernel_algorithmic_bytes(top, w, plan) if top else None
+    top_us = kernels[top]["avg_us"] if top else None
+    roofline = None
+    if alg:
+        achieved = alg / (top_us * 1e-6) / 1e9
+        roofline = {"kernel": top, "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
+                    "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
+                    "traffic": ncu_traffic(top, BH * w.S), "algorithmic_bytes": alg,
+                    "peak_source": f"{peak_src} (burst copy)"}
+    flops = fwd_flops(BH, w.S, w.DH, args.chunk)
+    tflops = flops / (ms_step * 1e-3) / 1e12
+    tc = {"useful_tflops": tflops, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+          "frac": tflops / peaks["bf16_tflops"], "useful_flops_per_step": flops,
+          "peak_source": f"{peak_src} (burst cuBLAS bf16)"}
+    step_bytes = tokens * fwd_token_bytes(w.DH, 2 if w.dtype == "bf16" else 4) + state_bytes(BH, w.DH)
+    whole = {"achieved_gbs": step_bytes / (ms_step * 1e-3) / 1e9,
+             "frac": step_bytes / (ms_step * 1e-3) / 1e9 / peaks["hbm_gbs"],
+             "algorithmic_bytes_per_step": step_bytes}
+
+    # ------------------------------------------------------------- end to end
+    e2e = None
+    if not args.skip_e2e:
+        pin = {k: v.pin_memory() for k, v in inp.items()}
+        h, C, n, m = outs
+        out_host = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in (h, C, n, m)]
+        dev_in = x
+
+        def e2e_step():
+            for k in dev_in:
+                dev_in[k].copy_(pin[k], non_blocking=True)
+            run()
+            for hst, dv in zip(out_host, (h, C, n, m)):
+                hst.copy_(dv, non_blocking=True)
+        for _ in range(2):
+            e2e_step()
+        ms_e2e = time_region(e2e_step, max(3, min(args.steps, 10)), dist_on, dev) / max(3, min(args.steps, 10))
+        h2d = sum(t.numel() * t.element_size() for t in pin.values())
+        d2h = sum(t.numel() * t.element_size() for t in out_host)
+        e2e = {"value": tokens * world / (ms_e2e * 1e-3), "unit": "tokens/s",
+               "ms_per_step": ms_e2e, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+    del x, outs, run
+
+    # ----------------------------------------------------------------- decode
+    decode = None
+    if not args.skip_decode:
+        decode = run_decode(args, dev, dist_on, rank, world, peaks, peak_src)
+
+    clocks = sampler.stop() if sampler else None
+
+    # ------------------------------------------------------------ CPU baseline
+    cpu = None
+    if rank == 0 and world == 1 and not args.skip_cpu:
+        cpu = cpu_baseline(w, w.S)
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "bf16" if (w.dtype == "bf16" and top and top.endswith("_tc")) else "f32",
+                "data": "synthetic (seeded N(0,1)-based draws of the workload shapes)",
+                "config": dict(workload_config(w, args.chunk, world),
+                               l2="inputs 406 MB > 126 MB L2; no flush" if w.name == "long"
+                               else "inputs may fit L2", segments=plan["P"],
+                               path=args.path),
+                "roofline": roofline, "tc": tc, "hbm_whole_step": whole,
+                "kernels": kernels, "gpu_launches": launches, "cpu_baseline": cpu, "e2e": e2e,
+                "clocks": clocks, "decode": decode}
+        print(json.dumps(line), flush=True)
+    if dist_on:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+def run_decode(args, dev, dist_on, rank, world, peaks, peak_src):
+    d = syn.DECODE
+    T = args.decode_steps
+    BH, DH = d.B * d.NH, d.DH
+    pre = syn.fwd_inputs(d.prefill(), seed=d.seed + rank)
+    x = {k: v.to(dev) for k, v in pre.items()}
+    _, C, n, m = xb.mlstm_fwd(x["q"], x["k"], x["v"], x["i_pre"], x["f_pre"], x["o_pre"],
+                              chunk=d.prefill_chunk, fgate=d.fgate)
+    del x
+    steps = []
+    for t in range(T):
+        s = syn.step_inputs(d, t, seed=d.seed + rank)
+        steps.append({k: v.to(dev, non_blocking=False) for k, v in s.items()})
+    h = torch.empty((d.B, d.NH, DH), dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream(dev).cuda_stream
+    fg = xb.FGATE_EXP if d.fgate == "exp" else xb.FGATE_SIGMOID
+    cur = [0]
+
+    def one():
+        s = steps[cur[0] % T]
+        cur[0] += 1
+        st = xb.xlstm_mlstm_step(s["q"].data_ptr(), s["k"].data_ptr(), s["v"].data_ptr(),
+                                 s["i_pre"].data_ptr(), s["f_pre"].data_ptr(), s["o_pre"].data_ptr(),
+                                 h.data_ptr(), C.data_ptr(), n.data_ptr(), m.data_ptr(),
+                                 d.B, d.NH, DH, xb.BF16, fg, stream)
+        if st != xb.OK:
+            raise xb.XlstmError(st, "xlstm_mlstm_step")
+    for _ in range(max(3, args.warmup)):
+        one()
+    torch.cuda.synchronize(dev)
+    cur[0] = 0
+    xb.xlstm_profile_begin()
+    ms = time_region(one, T, dist_on, dev)
+    _, kt = xb.xlstm_profile_end()
+    ms_step = ms / T
+    step_bytes = BH * (8.0 * DH * DH + 8 * DH + 8) + BH * DH * (3 * 2 + 4 + 2) + BH * 8
+    gbs = step_bytes / (ms_step * 1e-3) / 1e9
+    rows = kt.get("step_rows", (0, 0.0))
+    rows_us = 1e3 * rows[1] / max(rows[0], 1)
+    row_bytes = BH * (8.0 * DH * DH) + BH * DH * (3 * 2 + 4 + 2 + 4) + BH * 12
+    ach = row_bytes / (rows_us * 1e-6) / 1e9 if rows_us > 0 else None
+    return {"metric": "decode-step HBM GB/s", "value": gbs * world, "unit": "GB/s",
+            "per_gpu_frac": gbs / peaks["hbm_gbs"], "ms_per_step": ms_step, "steps": T,
+            "tokens_per_s": BH * world / (ms_step * 1e-3),
+            "algorithmic_bytes_per_step": step_bytes,
+            "roofline": {"kernel": "step_rows", "bound": "hbm", "achieved": ach,
+                         "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": (ach / peaks["hbm_gbs"]) if ach else None,
+                         "traffic": ncu_traffic("step_rows", BH), "peak_source": f"{peak_src} (burst copy)"},
+            "kernels": {k: {"launches": v[0], "avg_us": 1e3 * v[1] / max(v[0], 1)} for k, v in kt.items()},
+            "gpu_launches": sum(v[0] for v in kt.values()),
+            "config": f"decode: B={d.B} NH={d.NH} DH={DH} bf16 q/k/v, fp32 state (2 GiB, > L2), "
+                      f"prefill S={d.prefill_S} chunk {d.prefill_chunk}, {T} consecutive tokens"}
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,182 @@
+/*
+ * xlstm_mlstm.h -- C ABI of the B200 (sm_100a) mLSTM cell library.
+ *
+ * The operation is the mLSTM cell of "xLSTM: Extended Long Short-Term Memory":
+ * a matrix memory C (section 2.3) updated by the gated covariance rule (eq. (18)
+ * with the forget gate as decay rate and the input gate as learning rate), a
+ * normaliser state n whose dot product with the query is floored at 1.0
+ * (section 2.3), exponential input gating with the stabiliser state m
+ * (section 2.2, applied to mLSTM as section 2.3 says), and the output gate
+ * scaling the retrieved vector.  Per batch b and head h, with d = DH:
+ *
+ *   log i_t = itilde_t;  log f_t = log sigmoid(ftilde_t)  or  ftilde_t;
+ *   o_t = sigmoid(otilde_t) (per element);   khat_t = k_t / sqrt(d)
+ *   m_t  = max(log f_t + m_{t-1}, log i_t)
+ *   C'_t = exp(log f_t + m_{t-1} - m_t) C'_{t-1} + exp(log i_t - m_t) v_t khat_t^T
+ *   n'_t = exp(log f_t + m_{t-1} - m_t) n'_{t-1} + exp(log i_t - m_t) khat_t
+ *   h_t  = o_t * (C'_t q_t) / max(|n'_t^T q_t|, exp(-m_t))
+ *
+ * The state (C', n', m) is kept in stabilised units (C' = C exp(-m)); the
+ * floor exp(-m_t) is the section 2.3 bound of 1.0 expressed in those units.
+ * C' is [value row, key column].  Heads are independent (section 2.3: no
+ * memory mixing between heads).
+ *
+ * Conventions for every entry point
+ *  - Pointers are DEVICE pointers owned by the caller; the library keeps none
+ *    of them after the call returns and allocates no device memory.
+ *  - Tensors are dense, row-major (C order) with the shapes given, and every
+ *    pointer is 16-byte aligned (else XLSTM_ERR_ALIGN).
+ *  - Work is enqueued on the CUDA stream `cuda_stream` (a cudaStream_t; NULL =
+ *    the legacy default stream) on the current device, asynchronously; no call
+ *    synchronises.  The returned status covers argument validation and kernel
+ *    launch only.  Errors found on the device (a bounded wait that ran out) are
+ *    latched in a device status word read by xlstm_device_status().
+ *  - No entry point exits, aborts, traps or throws.
+ */
+#ifndef XLSTM_MLSTM_H
+#define XLSTM_MLSTM_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    XLSTM_OK = 0,
+    XLSTM_ERR_NULL = 1,        /* a required pointer is NULL                       */
+    XLSTM_ERR_SHAPE = 2,       /* a size is negative, DH unsupported, or too large */
+    XLSTM_ERR_DTYPE = 3,       /* dtype or forget-gate kind out of range           */
+    XLSTM_ERR_CHUNK = 4,       /* chunk size not supported for this dtype          */
+    XLSTM_ERR_ALIGN = 5,       /* a pointer is not 16-byte aligned                 */
+    XLSTM_ERR_CUDA = 6,        /* a CUDA runtime call or kernel launch failed      */
+    XLSTM_ERR_TIMEOUT = 7,     /* a bounded device-side wait ran out               */
+    XLSTM_ERR_WORKSPACE = 8,   /* workspace NULL or smaller than required          */
+    XLSTM_ERR_UNSUPPORTED = 9  /* option combination not supported                 */
+} xlstm_status;
+
+typedef enum { XLSTM_F32 = 0, XLSTM_BF16 = 1 } xlstm_dtype;          /* dtype of q, k, v, h */
+typedef enum { XLSTM_FGATE_SIGMOID = 0, XLSTM_FGATE_EXP = 1 } xlstm_fgate;
+
+/* Kernel family for the forward.  AUTO picks the tensor-core (tcgen05) kernels
+ * for bf16 inputs and the fp32 SIMT kernels for fp32 inputs.  SIMT forces the
+ * fp32-arithmetic kernels for either dtype (a second, independent path used by
+ * the tests). */
+typedef enum { XLSTM_PATH_AUTO = 0, XLSTM_PATH_SIMT = 1, XLSTM_PATH_TENSOR = 2 } xlstm_path;
+
+typedef struct {
+    int path;       /* xlstm_path                                                       */
+    int segments;   /* sequence segments per head for the two-level scan; 0 = automatic */
+} xlstm_fwd_options;
+
+/* ABI version of this header (bumped on any signature change). */
+#define XLSTM_ABI_VERSION 1
+int xlstm_abi_version(void);
+
+/* Human-readable name of a status; never NULL. */
+const char *xlstm_status_string(xlstm_status status);
+
+/*
+ * Bytes of device workspace xlstm_mlstm_fwd needs for these arguments (written
+ * to *bytes; may be 0).  The workspace holds per-chunk gate prefix sums and,
+ * when a head's sequence is split into segments that run in parallel, one
+ * summary state per segment (the two-level chunk-state scan).  Same validation
+ * as xlstm_mlstm_fwd.  Pure host function; touches no device.
+ */
+xlstm_status xlstm_mlstm_fwd_workspace_size(int B, int NH, int S, int DH, int chunk,
+                                            xlstm_dtype dt, size_t *bytes);
+xlstm_status xlstm_mlstm_fwd_workspace_size_ex(int B, int NH, int S, int DH, int chunk,
+                                               xlstm_dtype dt, const xlstm_fwd_options *opts,
+                                               size_t *bytes);
+
+/*
+ * Chunkwise-parallel forward (prefill) over S tokens.
+ *
+ *   q, k, v      [B, NH, S, DH]  dtype dt (float or bfloat16)
+ *   i_pre, f_pre [B, NH, S]      float   (input / forget gate pre-activations)
+ *   o_pre        [B, NH, S, DH]  float   (output gate pre-activation, per element)
+ *   h            [B, NH, S, DH]  dtype dt, output
+ *   C0 [B, NH, DH, DH], n0 [B, NH, DH], m0 [B, NH]  float, initial state in
+ *                stabilised units; each may be NULL, meaning zeros.
+ *   C_out, n_out, m_out  same shapes, final state; each may be NULL (not written).
+ *                They must not overlap C0, n0, m0 or any input (the same
+                pointer passed twice is rejected with XLSTM_ERR_UNSUPPORTED).
+ *   chunk        tokens per chunk of the chunkwise form: 64, 128 or 256 for
+ *                bf16; 1..1024 for f32.  S need not be a multiple of chunk.
+ *   DH           multiple of 16 in [16, 512].
+ *   fg           forget gate activation (sigmoid or exponential).
+ *   workspace    device buffer of at least xlstm_mlstm_fwd_workspace_size()
+ *                bytes (may be NULL when that size is 0); contents on entry
+ *                are ignored, on exit unspecified.
+ * S == 0 is allowed: h is untouched and the final state equals the initial one.
+ * B == 0 or NH == 0 is a no-op.
+ */
+xlstm_status xlstm_mlstm_fwd(const void *q, const void *k, const void *v,
+                             const float *i_pre, const float *f_pre, const float *o_pre,
+                             void *h,
+                             const float *C0, const float *n0, const float *m0,
+                             float *C_out, float *n_out, float *m_out,
+                             int B, int NH, int S, int DH, int chunk,
+                             xlstm_dtype dt, xlstm_fgate fg,
+                             void *workspace, size_t workspace_bytes, void *cuda_stream);
+
+/* As xlstm_mlstm_fwd, with explicit options (NULL = defaults). */
+xlstm_status xlstm_mlstm_fwd_ex(const void *q, const void *k, const void *v,
+                                const float *i_pre, const float *f_pre, const float *o_pre,
+                                void *h,
+                                const float *C0, const float *n0, const float *m0,
+                                float *C_out, float *n_out, float *m_out,
+                                int B, int NH, int S, int DH, int chunk,
+                                xlstm_dtype dt, xlstm_fgate fg,
+                                void *workspace, size_t workspace_bytes,
+                                const xlstm_fwd_options *opts, void *cuda_stream);
+
+/*
+ * One recurrent decode token for every (b, h), updating the resident state in
+ * place (section 2.5 of the paper: constant memory in the sequence length).
+ *
+ *   q, k, v      [B, NH, DH]      dtype dt
+ *   i_pre, f_pre [B, NH]          float
+ *   o_pre        [B, NH, DH]      float
+ *   h            [B, NH, DH]      dtype dt, output
+ *   C [B, NH, DH, DH], n [B, NH, DH], m [B, NH]  float, stabilised state,
+ *                read and overwritten with the state after this token.  This
+ *                is exactly the state xlstm_mlstm_fwd returns.
+ * DH: multiple of 16 in [16, 512].  B == 0 or NH == 0 is a no-op.
+ */
+xlstm_status xlstm_mlstm_step(const void *q, const void *k, const void *v,
+                              const float *i_pre, const float *f_pre, const float *o_pre,
+                              void *h, float *C, float *n, float *m,
+                              int B, int NH, int DH, xlstm_dtype dt, xlstm_fgate fg,
+                              void *cuda_stream);
+
+/*
+ * Synchronises `cuda_stream`, then reads and clears the device status word of
+ * the current device.  Returns XLSTM_OK, XLSTM_ERR_TIMEOUT if a kernel gave up
+ * a bounded wait since the last call, or XLSTM_ERR_CUDA.
+ */
+xlstm_status xlstm_device_status(void *cuda_stream);
+
+/*
+ * Per-kernel timing (tracing).  Between xlstm_profile_begin() and
+ * xlstm_profile_end(), every kernel this library launches, from any thread, is
+ * bracketed by a pair of CUDA events recorded on the stream it is launched
+ * on.  xlstm_profile_end() waits for those events and writes, per kernel
+ * name, the launch count and the summed device time, for at most `max`
+ * kernels into `out`; *count receives the number of distinct kernels.  The
+ * events cost one stream operation each and do not serialise streams.
+ */
+typedef struct {
+    char name[48];       /* kernel name, NUL-terminated */
+    int launches;
+    double total_ms;     /* sum of event-to-event times of its launches */
+} xlstm_kernel_time;
+
+xlstm_status xlstm_profile_begin(void);
+xlstm_status xlstm_profile_end(xlstm_kernel_time *out, int max, int *count);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* XLSTM_MLSTM_H */

@@ -1,0 +1,231 @@
+"""ctypes binding of ``libxlstm_mlstm.so``: argument marshalling only.
+
+The names mirror the C ABI in ``include/xlstm_mlstm.h``.  ``load()`` binds the
+library and raises if it is missing: there is no fallback path.  The
+convenience wrappers ``mlstm_fwd`` / ``mlstm_step`` take torch CUDA tensors,
+allocate outputs and workspace with torch (device memory is PyTorch's job
+here), pass raw pointers and the current CUDA stream, and turn a non-OK status
+into ``XlstmError``.  Every step of the computation runs in the library's
+kernels.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libxlstm_mlstm.so")
+
+OK, ERR_NULL, ERR_SHAPE, ERR_DTYPE, ERR_CHUNK, ERR_ALIGN, ERR_CUDA, ERR_TIMEOUT, \
+    ERR_WORKSPACE, ERR_UNSUPPORTED = range(10)
+F32, BF16 = 0, 1
+FGATE_SIGMOID, FGATE_EXP = 0, 1
+PATH_AUTO, PATH_SIMT, PATH_TENSOR = 0, 1, 2
+
+EXPORTED = ("xlstm_abi_version", "xlstm_status_string", "xlstm_mlstm_fwd_workspace_size",
+            "xlstm_mlstm_fwd_workspace_size_ex", "xlstm_mlstm_fwd", "xlstm_mlstm_fwd_ex",
+            "xlstm_mlstm_step", "xlstm_device_status", "xlstm_profile_begin", "xlstm_profile_end")
+
+
+class XlstmError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)} (status {status})")
+
+
+class FwdOptions(ctypes.Structure):
+    _fields_ = [("path", ctypes.c_int), ("segments", ctypes.c_int)]
+
+
+class KernelTime(ctypes.Structure):
+    _fields_ = [("name", ctypes.c_char * 48), ("launches", ctypes.c_int),
+                ("total_ms", ctypes.c_double)]
+
+
+_lock = threading.Lock()
+_lib = None
+
+
+def load(path: str = LIB_PATH):
+    """Load and bind the library.  Raises OSError if it has not been built."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(path):
+            raise OSError(f"{path} is missing: build it with `python -m linear_rnn_mlstm_b200.build`"
+                          " (the mLSTM ops have no other implementation)")
+        lib = ctypes.CDLL(path)
+        vp, fp, i, sz = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+        lib.xlstm_abi_version.restype = i
+        lib.xlstm_status_string.argtypes = [i]
+        lib.xlstm_status_string.restype = ctypes.c_char_p
+        lib.xlstm_mlstm_fwd_workspace_size.argtypes = [i] * 6 + [ctypes.POINTER(sz)]
+        lib.xlstm_mlstm_fwd_workspace_size.restype = i
+        lib.xlstm_mlstm_fwd_workspace_size_ex.argtypes = [i] * 6 + [ctypes.POINTER(FwdOptions),
+                                                                   ctypes.POINTER(sz)]
+        lib.xlstm_mlstm_fwd_workspace_size_ex.restype = i
+        fwd_args = [vp] * 3 + [fp] * 3 + [vp] + [fp] * 6 + [i] * 7 + [vp, sz]
+        lib.xlstm_mlstm_fwd.argtypes = fwd_args + [vp]
+        lib.xlstm_mlstm_fwd.restype = i
+        lib.xlstm_mlstm_fwd_ex.argtypes = fwd_args + [ctypes.POINTER(FwdOptions), vp]
+        lib.xlstm_mlstm_fwd_ex.restype = i
+        lib.xlstm_mlstm_step.argtypes = [vp] * 3 + [fp] * 3 + [vp] + [fp] * 3 + [i] * 5 + [vp]
+        lib.xlstm_mlstm_step.restype = i
+        lib.xlstm_device_status.argtypes = [vp]
+        lib.xlstm_device_status.restype = i
+        lib.xlstm_profile_begin.restype = i
+        lib.xlstm_profile_end.argtypes = [ctypes.POINTER(KernelTime), i, ctypes.POINTER(i)]
+        lib.xlstm_profile_end.restype = i
+        _lib = lib
+        return lib
+
+
+def status_string(status: int) -> str:
+    return load().xlstm_status_string(int(status)).decode()
+
+
+# ----------------------------------------------------- raw C entry points
+def xlstm_abi_version() -> int:
+    return load().xlstm_abi_version()
+
+
+def xlstm_mlstm_fwd_workspace_size(B, NH, S, DH, chunk, dt, path=PATH_AUTO, segments=0):
+    n = ctypes.c_size_t(0)
+    opts = FwdOptions(path, segments)
+    st = load().xlstm_mlstm_fwd_workspace_size_ex(B, NH, S, DH, chunk, dt, ctypes.byref(opts),
+                                                   ctypes.byref(n))
+    return st, n.value
+
+
+def xlstm_mlstm_fwd(q, k, v, i_pre, f_pre, o_pre, h, C0, n0, m0, C_out, n_out, m_out,
+                    B, NH, S, DH, chunk, dt, fg, workspace, workspace_bytes, stream,
+                    path=PATH_AUTO, segments=0):
+    """Pointers are ints (device addresses) or None; returns the status."""
+    opts = FwdOptions(path, segments)
+    return load().xlstm_mlstm_fwd_ex(q, k, v, i_pre, f_pre, o_pre, h, C0, n0, m0,
+                                     C_out, n_out, m_out, B, NH, S, DH, chunk, dt, fg,
+                                     workspace, workspace_bytes, ctypes.byref(opts), stream)
+
+
+def xlstm_mlstm_step(q, k, v, i_pre, f_pre, o_pre, h, C, n, m, B, NH, DH, dt, fg, stream):
+    return load().xlstm_mlstm_step(q, k, v, i_pre, f_pre, o_pre, h, C, n, m, B, NH, DH, dt, fg,
+                                   stream)
+
+
+def xlstm_device_status(stream) -> int:
+    return load().xlstm_device_status(stream)
+
+
+def xlstm_profile_begin() -> int:
+    return load().xlstm_profile_begin()
+
+
+def xlstm_profile_end(max_kernels: int = 32):
+    """Returns (status, {kernel name: (launches, total_ms)})."""
+    arr = (KernelTime * max_kernels)()
+    count = ctypes.c_int(0)
+    st = load().xlstm_profile_end(arr, max_kernels, ctypes.byref(count))
+    out = {}
+    for i in range(min(count.value, max_kernels)):
+        out[arr[i].name.decode()] = (arr[i].launches, arr[i].total_ms)
+    return st, out
+
+
+# ------------------------------------------------------ torch conveniences
+def _torch():
+    import torch
+    return torch
+
+
+def _dt(t):
+    torch = _torch()
+    if t.dtype == torch.bfloat16:
+        return BF16
+    if t.dtype == torch.float32:
+        return F32
+    raise TypeError(f"q/k/v must be float32 or bfloat16, got {t.dtype}")
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _check(t, name, shape, dtype, device):
+    if t is None:
+        return
+    if not t.is_cuda or t.device != device:
+        raise ValueError(f"{name} must be a CUDA tensor on {device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} has dtype {t.dtype}, expected {dtype}")
+
+
+def _stream(device):
+    return _torch().cuda.current_stream(device).cuda_stream
+
+
+def mlstm_fwd(q, k, v, i_pre, f_pre, o_pre, chunk=64, fgate="sigmoid", C0=None, n0=None,
+              m0=None, h=None, state_out=True, path=PATH_AUTO, segments=0, workspace=None):
+    """Chunkwise forward.  Returns (h, C, n, m) (state None unless state_out)."""
+    torch = _torch()
+    B, NH, S, DH = q.shape
+    dev = q.device
+    dtype = q.dtype
+    dt = _dt(q)
+    for t, nm in ((q, "q"), (k, "k"), (v, "v")):
+        _check(t, nm, (B, NH, S, DH), dtype, dev)
+    _check(i_pre, "i_pre", (B, NH, S), torch.float32, dev)
+    _check(f_pre, "f_pre", (B, NH, S), torch.float32, dev)
+    _check(o_pre, "o_pre", (B, NH, S, DH), torch.float32, dev)
+    _check(C0, "C0", (B, NH, DH, DH), torch.float32, dev)
+    _check(n0, "n0", (B, NH, DH), torch.float32, dev)
+    _check(m0, "m0", (B, NH), torch.float32, dev)
+    if h is None:
+        h = torch.empty((B, NH, S, DH), dtype=dtype, device=dev)
+    _check(h, "h", (B, NH, S, DH), dtype, dev)
+    C = n = m = None
+    if state_out:
+        C = torch.empty((B, NH, DH, DH), dtype=torch.float32, device=dev)
+        n = torch.empty((B, NH, DH), dtype=torch.float32, device=dev)
+        m = torch.empty((B, NH), dtype=torch.float32, device=dev)
+    fg = FGATE_EXP if fgate == "exp" else FGATE_SIGMOID
+    st, nbytes = xlstm_mlstm_fwd_workspace_size(B, NH, S, DH, chunk, dt, path, segments)
+    if st != OK:
+        raise XlstmError(st, "xlstm_mlstm_fwd_workspace_size")
+    if workspace is None or workspace.numel() < nbytes:
+        workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=dev)
+    st = xlstm_mlstm_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(i_pre), _ptr(f_pre), _ptr(o_pre),
+                         _ptr(h), _ptr(C0), _ptr(n0), _ptr(m0), _ptr(C), _ptr(n), _ptr(m),
+                         B, NH, S, DH, chunk, dt, fg, workspace.data_ptr(), workspace.numel(),
+                         _stream(dev), path, segments)
+    if st != OK:
+        raise XlstmError(st, "xlstm_mlstm_fwd")
+    return h, C, n, m
+
+
+def mlstm_step(q, k, v, i_pre, f_pre, o_pre, C, n, m, fgate="sigmoid", h=None):
+    """One decode token; (C, n, m) are updated in place.  Returns h."""
+    torch = _torch()
+    B, NH, DH = q.shape
+    dev, dtype, dt = q.device, q.dtype, _dt(q)
+    for t, nm in ((q, "q"), (k, "k"), (v, "v")):
+        _check(t, nm, (B, NH, DH), dtype, dev)
+    _check(i_pre, "i_pre", (B, NH), torch.float32, dev)
+    _check(f_pre, "f_pre", (B, NH), torch.float32, dev)
+    _check(o_pre, "o_pre", (B, NH, DH), torch.float32, dev)
+    _check(C, "C", (B, NH, DH, DH), torch.float32, dev)
+    _check(n, "n", (B, NH, DH), torch.float32, dev)
+    _check(m, "m", (B, NH), torch.float32, dev)
+    if h is None:
+        h = torch.empty((B, NH, DH), dtype=dtype, device=dev)
+    fg = FGATE_EXP if fgate == "exp" else FGATE_SIGMOID
+    st = xlstm_mlstm_step(_ptr(q), _ptr(k), _ptr(v), _ptr(i_pre), _ptr(f_pre), _ptr(o_pre),
+                          _ptr(h), _ptr(C), _ptr(n), _ptr(m), B, NH, DH, dt, fg, _stream(dev))
+    if st != OK:
+        raise XlstmError(st, "xlstm_mlstm_step")
+    return h

@@ -1,0 +1,254 @@
+// C ABI of the mLSTM library: argument validation, launch planning, dispatch.
+// The operation and every argument are documented in include/xlstm_mlstm.h.
+#include <stdint.h>
+#include <string.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "plan.h"
+#include "profile.h"
+
+namespace xlstm {
+
+__device__ unsigned int g_device_status = 0;
+
+constexpr int kNumSms = 148;               // B200
+constexpr int kMaxHeads = 65535;           // B * NH rides in a grid dimension
+
+static size_t align64(size_t x) { return (x + 63) & ~size_t(63); }
+
+bool make_fwd_plan(int B, int NH, int S, int DH, int L, int path, int forced_segments,
+                   int num_sms, FwdPlan *p) {
+    memset(p, 0, sizeof(*p));
+    p->B = B; p->NH = NH; p->S = S; p->DH = DH; p->L = L;
+    p->BH = B * NH;
+    p->path = path;
+    p->nchunks = S > 0 ? (S + L - 1) / L : 0;
+    if (path == XLSTM_PATH_TENSOR) {
+        p->rows = DH < 128 ? DH : 128;
+    } else {
+        p->rows = DH < 32 ? DH : 32;
+    }
+    p->ntiles = (DH + p->rows - 1) / p->rows;
+    if (p->nchunks == 0 || p->BH == 0) {
+        p->P = 0; p->cps = 0;
+        p->total_floats = 0;
+        return true;
+    }
+    int P;
+    if (forced_segments > 0) {
+        P = forced_segments;
+    } else {
+        const long per_set = (long)p->BH * p->ntiles;
+        const long target = 2L * num_sms;
+        P = (int)((target + per_set - 1) / per_set);
+    }
+    if (P < 1) P = 1;
+    if (P > p->nchunks) P = p->nchunks;
+    if (P > kMaxHeads) P = kMaxHeads;
+    p->cps = (p->nchunks + P - 1) / P;
+    p->P = (p->nchunks + p->cps - 1) / p->cps;
+
+    size_t off = 0;
+    p->off_bcum = off;  off = align64(off + (size_t)p->BH * S);
+    p->off_cstat = off; off = align64(off + (size_t)p->BH * p->nchunks * 2);
+    p->off_sstat = off; off = align64(off + (size_t)p->BH * p->P * 2);
+    p->off_summ = off;  off = align64(off + (size_t)p->BH * (p->P - 1) * ((size_t)DH * DH + DH));
+    p->total_floats = off;
+    return true;
+}
+
+// Copies (or zero-fills) the initial state into the final-state outputs: the
+// S == 0 forward.
+__global__ void state_passthrough_kernel(const float *C0, const float *n0, const float *m0,
+                                         float *C_out, float *n_out, float *m_out, int BH, int DH) {
+    const size_t nC = (size_t)BH * DH * DH, nn = (size_t)BH * DH;
+    const size_t stride = (size_t)gridDim.x * blockDim.x;
+    for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < nC; i += stride) {
+        if (C_out) C_out[i] = C0 ? C0[i] : 0.f;
+        if (i < nn && n_out) n_out[i] = n0 ? n0[i] : 0.f;
+        if (i < (size_t)BH && m_out) m_out[i] = m0 ? m0[i] : 0.f;
+    }
+}
+
+cudaError_t launch_state_passthrough(const FwdArgs &a, int BH, int DH, cudaStream_t st) {
+    if (!a.C_out && !a.n_out && !a.m_out) return cudaSuccess;
+    KernelTimer timer("state_passthrough", st);
+    state_passthrough_kernel<<<4 * kNumSms, 256, 0, st>>>(a.C0, a.n0, a.m0, a.C_out, a.n_out,
+                                                          a.m_out, BH, DH);
+    return cudaGetLastError();
+}
+
+}  // namespace xlstm
+
+using namespace xlstm;
+
+static bool misaligned(const void *p) { return ((uintptr_t)p & 15u) != 0; }
+
+static xlstm_status check_fwd_shape(int B, int NH, int S, int DH, int chunk, xlstm_dtype dt) {
+    if (dt != XLSTM_F32 && dt != XLSTM_BF16) return XLSTM_ERR_DTYPE;
+    if (B < 0 || NH < 0 || S < 0) return XLSTM_ERR_SHAPE;
+    if (DH < 16 || DH > 512 || DH % 16 != 0) return XLSTM_ERR_SHAPE;
+    if ((long long)B * NH > kMaxHeads) return XLSTM_ERR_SHAPE;
+    if ((long long)B * NH * S * DH > (1LL << 40)) return XLSTM_ERR_SHAPE;
+    if (dt == XLSTM_BF16) {
+        if (chunk != 64 && chunk != 128 && chunk != 256) return XLSTM_ERR_CHUNK;
+    } else {
+        if (chunk < 1 || chunk > 1024) return XLSTM_ERR_CHUNK;
+    }
+    return XLSTM_OK;
+}
+
+static int resolve_path(xlstm_dtype dt, int DH, int chunk, const xlstm_fwd_options *opts,
+                        xlstm_status *st) {
+    *st = XLSTM_OK;
+    const int want = opts ? opts->path : XLSTM_PATH_AUTO;
+    if (want == XLSTM_PATH_SIMT) return XLSTM_PATH_SIMT;
+    if (want == XLSTM_PATH_TENSOR) {
+        if (dt != XLSTM_BF16 || !tensor_path_supports(DH, chunk)) {
+            *st = XLSTM_ERR_UNSUPPORTED;
+            return 0;
+        }
+        return XLSTM_PATH_TENSOR;
+    }
+    if (want != XLSTM_PATH_AUTO) {
+        *st = XLSTM_ERR_UNSUPPORTED;
+        return 0;
+    }
+    if (dt == XLSTM_BF16 && tensor_path_supports(DH, chunk)) return XLSTM_PATH_TENSOR;
+    return XLSTM_PATH_SIMT;
+}
+
+extern "C" {
+
+int xlstm_abi_version(void) { return XLSTM_ABI_VERSION; }
+
+const char *xlstm_status_string(xlstm_status s) {
+    switch (s) {
+        case XLSTM_OK: return "ok";
+        case XLSTM_ERR_NULL: return "a required pointer is NULL";
+        case XLSTM_ERR_SHAPE: return "unsupported or inconsistent shape";
+        case XLSTM_ERR_DTYPE: return "unsupported dtype or forget-gate kind";
+        case XLSTM_ERR_CHUNK: return "unsupported chunk size for this dtype";
+        case XLSTM_ERR_ALIGN: return "a pointer is not 16-byte aligned";
+        case XLSTM_ERR_CUDA: return "CUDA runtime or launch error";
+        case XLSTM_ERR_TIMEOUT: return "a bounded device-side wait ran out";
+        case XLSTM_ERR_WORKSPACE: return "workspace missing or too small";
+        case XLSTM_ERR_UNSUPPORTED: return "unsupported option combination";
+    }
+    return "unknown status";
+}
+
+xlstm_status xlstm_mlstm_fwd_workspace_size_ex(int B, int NH, int S, int DH, int chunk,
+                                               xlstm_dtype dt, const xlstm_fwd_options *opts,
+                                               size_t *bytes) {
+    if (!bytes) return XLSTM_ERR_NULL;
+    xlstm_status st = check_fwd_shape(B, NH, S, DH, chunk, dt);
+    if (st != XLSTM_OK) return st;
+    const int path = resolve_path(dt, DH, chunk, opts, &st);
+    if (st != XLSTM_OK) return st;
+    FwdPlan p;
+    if (!make_fwd_plan(B, NH, S, DH, chunk, path, opts ? opts->segments : 0, kNumSms, &p))
+        return XLSTM_ERR_SHAPE;
+    *bytes = p.bytes();
+    return XLSTM_OK;
+}
+
+xlstm_status xlstm_mlstm_fwd_workspace_size(int B, int NH, int S, int DH, int chunk,
+                                            xlstm_dtype dt, size_t *bytes) {
+    return xlstm_mlstm_fwd_workspace_size_ex(B, NH, S, DH, chunk, dt, nullptr, bytes);
+}
+
+xlstm_status xlstm_mlstm_fwd_ex(const void *q, const void *k, const void *v,
+                                const float *i_pre, const float *f_pre, const float *o_pre,
+                                void *h, const float *C0, const float *n0, const float *m0,
+                                float *C_out, float *n_out, float *m_out,
+                                int B, int NH, int S, int DH, int chunk,
+                                xlstm_dtype dt, xlstm_fgate fg,
+                                void *workspace, size_t workspace_bytes,
+                                const xlstm_fwd_options *opts, void *cuda_stream) {
+    xlstm_status st = check_fwd_shape(B, NH, S, DH, chunk, dt);
+    if (st != XLSTM_OK) return st;
+    if (fg != XLSTM_FGATE_SIGMOID && fg != XLSTM_FGATE_EXP) return XLSTM_ERR_DTYPE;
+    if (opts && opts->segments < 0) return XLSTM_ERR_UNSUPPORTED;
+    const int path = resolve_path(dt, DH, chunk, opts, &st);
+    if (st != XLSTM_OK) return st;
+    if ((long long)B * NH == 0) return XLSTM_OK;
+    if (S > 0 && (!q || !k || !v || !i_pre || !f_pre || !o_pre || !h)) return XLSTM_ERR_NULL;
+    const void *ptrs[] = {q, k, v, i_pre, f_pre, o_pre, h, C0, n0, m0, C_out, n_out, m_out, workspace};
+    for (const void *p : ptrs)
+        if (misaligned(p)) return XLSTM_ERR_ALIGN;
+
+    if ((C_out && C_out == C0) || (n_out && n_out == n0) || (m_out && m_out == m0))
+        return XLSTM_ERR_UNSUPPORTED;
+    FwdPlan plan;
+    if (!make_fwd_plan(B, NH, S, DH, chunk, path, opts ? opts->segments : 0, kNumSms, &plan))
+        return XLSTM_ERR_SHAPE;
+    if (plan.bytes() > 0 && (!workspace || workspace_bytes < plan.bytes())) return XLSTM_ERR_WORKSPACE;
+
+    FwdArgs a;
+    a.q = q; a.k = k; a.v = v; a.i_pre = i_pre; a.f_pre = f_pre; a.o_pre = o_pre; a.h = h;
+    a.C0 = C0; a.n0 = n0; a.m0 = m0; a.C_out = C_out; a.n_out = n_out; a.m_out = m_out;
+    a.workspace = workspace;
+    a.status = nullptr;
+    if (cudaGetSymbolAddress((void **)&a.status, g_device_status) != cudaSuccess) return XLSTM_ERR_CUDA;
+    a.bf16 = dt == XLSTM_BF16;
+    a.fgate_exp = fg == XLSTM_FGATE_EXP;
+    cudaStream_t stream = (cudaStream_t)cuda_stream;
+    cudaError_t e;
+    if (S == 0) {
+        e = launch_state_passthrough(a, plan.BH, DH, stream);
+    } else if (path == XLSTM_PATH_TENSOR) {
+        e = launch_fwd_tensor(a, plan, stream);
+    } else {
+        e = launch_fwd_simt(a, plan, stream);
+    }
+    return e == cudaSuccess ? XLSTM_OK : XLSTM_ERR_CUDA;
+}
+
+xlstm_status xlstm_mlstm_fwd(const void *q, const void *k, const void *v,
+                             const float *i_pre, const float *f_pre, const float *o_pre,
+                             void *h, const float *C0, const float *n0, const float *m0,
+                             float *C_out, float *n_out, float *m_out,
+                             int B, int NH, int S, int DH, int chunk,
+                             xlstm_dtype dt, xlstm_fgate fg,
+                             void *workspace, size_t workspace_bytes, void *cuda_stream) {
+    return xlstm_mlstm_fwd_ex(q, k, v, i_pre, f_pre, o_pre, h, C0, n0, m0, C_out, n_out, m_out,
+                              B, NH, S, DH, chunk, dt, fg, workspace, workspace_bytes, nullptr,
+                              cuda_stream);
+}
+
+xlstm_status xlstm_mlstm_step(const void *q, const void *k, const void *v,
+                              const float *i_pre, const float *f_pre, const float *o_pre,
+                              void *h, float *C, float *n, float *m,
+                              int B, int NH, int DH, xlstm_dtype dt, xlstm_fgate fg,
+                              void *cuda_stream) {
+    if (dt != XLSTM_F32 && dt != XLSTM_BF16) return XLSTM_ERR_DTYPE;
+    if (fg != XLSTM_FGATE_SIGMOID && fg != XLSTM_FGATE_EXP) return XLSTM_ERR_DTYPE;
+    if (B < 0 || NH < 0 || DH < 16 || DH > 512 || DH % 16 != 0) return XLSTM_ERR_SHAPE;
+    if ((long long)B * NH > kMaxHeads) return XLSTM_ERR_SHAPE;
+    if ((long long)B * NH == 0) return XLSTM_OK;
+    if (!q || !k || !v || !i_pre || !f_pre || !o_pre || !h || !C || !n || !m) return XLSTM_ERR_NULL;
+    const void *ptrs[] = {q, k, v, i_pre, f_pre, o_pre, h, C, n, m};
+    for (const void *p : ptrs)
+        if (misaligned(p)) return XLSTM_ERR_ALIGN;
+    StepArgs a;
+    a.q = q; a.k = k; a.v = v; a.i_pre = i_pre; a.f_pre = f_pre; a.o_pre = o_pre; a.h = h;
+    a.C = C; a.n = n; a.m = m;
+    a.BH = B * NH; a.DH = DH;
+    a.bf16 = dt == XLSTM_BF16;
+    a.fgate_exp = fg == XLSTM_FGATE_EXP;
+    return launch_step(a, (cudaStream_t)cuda_stream) == cudaSuccess ? XLSTM_OK : XLSTM_ERR_CUDA;
+}
+
+xlstm_status xlstm_device_status(void *cuda_stream) {
+    cudaStream_t stream = (cudaStream_t)cuda_stream;
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return XLSTM_ERR_CUDA;
+    unsigned int word = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&word, g_device_status, sizeof(word)) != cudaSuccess) return XLSTM_ERR_CUDA;
+    if (word && cudaMemcpyToSymbol(g_device_status, &zero, sizeof(zero)) != cudaSuccess)
+        return XLSTM_ERR_CUDA;
+    return word ? XLSTM_ERR_TIMEOUT : XLSTM_OK;
+}
+
+}  // extern "C"

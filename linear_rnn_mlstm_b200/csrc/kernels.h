@@ -1,0 +1,43 @@
+// Internal launch interface between the C ABI (abi.cu) and the kernel files.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+
+#include "plan.h"
+
+namespace xlstm {
+
+struct FwdArgs {
+    const void *q, *k, *v;
+    const float *i_pre, *f_pre, *o_pre;
+    void *h;
+    const float *C0, *n0, *m0;
+    float *C_out, *n_out, *m_out;
+    void *workspace;
+    unsigned int *status;     // device status word of the current device
+    int bf16;
+    int fgate_exp;
+};
+
+struct StepArgs {
+    const void *q, *k, *v;
+    const float *i_pre, *f_pre, *o_pre;
+    void *h;
+    float *C, *n, *m;
+    int BH, DH;
+    int bf16;
+    int fgate_exp;
+};
+
+cudaError_t launch_gate_prologue(const FwdArgs &a, const FwdPlan &p, cudaStream_t st);
+cudaError_t launch_fwd_simt(const FwdArgs &a, const FwdPlan &p, cudaStream_t st);
+cudaError_t launch_fwd_tensor(const FwdArgs &a, const FwdPlan &p, cudaStream_t st);
+bool tensor_path_supports(int DH, int L);
+cudaError_t launch_state_passthrough(const FwdArgs &a, int BH, int DH, cudaStream_t st);
+cudaError_t launch_step(const StepArgs &a, cudaStream_t st);
+
+size_t simt_summary_smem(int DH, int rows);
+size_t simt_output_smem(int DH, int rows, int L);
+
+}  // namespace xlstm

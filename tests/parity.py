@@ -1,0 +1,52 @@
+"""Shared helpers of the GPU parity tests: run the CUDA path through the C ABI
+(via the binding) and the float64 oracle on the same seeded inputs, and
+measure the error the way the tolerances are stated."""
+import numpy as np
+import torch
+
+import oracle
+from linear_rnn_mlstm_b200 import binding as xb
+
+# Tolerances: max |dh| and relative L2 of h over the whole tensor.
+TOL = {"bf16": (2e-2, 1e-2), "f32": (1e-5, 1e-5)}
+STATE_REL_L2 = 1e-2        # final C', n' (bf16 inputs)
+STATE_M_ABS = 1e-4         # final m
+
+
+def errors(got, ref):
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    diff = got - ref
+    max_abs = float(np.max(np.abs(diff))) if diff.size else 0.0
+    denom = float(np.linalg.norm(ref))
+    rel = float(np.linalg.norm(diff)) / denom if denom > 0 else float(np.linalg.norm(diff))
+    return max_abs, rel
+
+
+def assert_close(got, ref, dtype, what="h"):
+    tol_abs, tol_rel = TOL[dtype]
+    max_abs, rel = errors(got, ref)
+    assert max_abs <= tol_abs and rel <= tol_rel, (
+        f"{what}: max|d|={max_abs:.3e} (tol {tol_abs}), relL2={rel:.3e} (tol {tol_rel})")
+    return max_abs, rel
+
+
+def to_cuda(inp):
+    return {k: v.cuda().contiguous() for k, v in inp.items()}
+
+
+def gpu_fwd(inp, chunk, fgate, path=xb.PATH_AUTO, segments=0, C0=None, n0=None, m0=None):
+    d = to_cuda(inp)
+    st = {}
+    for name, t in (("C0", C0), ("n0", n0), ("m0", m0)):
+        st[name] = None if t is None else torch.as_tensor(t, dtype=torch.float32).cuda().contiguous()
+    h, C, n, m = xb.mlstm_fwd(d["q"], d["k"], d["v"], d["i_pre"], d["f_pre"], d["o_pre"],
+                              chunk=chunk, fgate=fgate, path=path, segments=segments, **st)
+    torch.cuda.synchronize()
+    assert xb.xlstm_device_status(torch.cuda.current_stream().cuda_stream) == xb.OK
+    return (h.float().cpu().numpy(), C.cpu().numpy(), n.cpu().numpy(), m.cpu().numpy())
+
+
+def oracle_fwd(inp, fgate, C0=None, n0=None, m0=None):
+    return oracle.fwd(inp["q"], inp["k"], inp["v"], inp["i_pre"], inp["f_pre"], inp["o_pre"],
+                      fgate, C0, n0, m0)

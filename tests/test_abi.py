@@ -1,0 +1,119 @@
+"""Host-side checks of the C ABI: the library loads, exports every entry point
+the header declares, and rejects bad arguments before touching any device.
+No test here launches GPU work (fake device addresses are only ever passed
+where validation must reject them first)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from linear_rnn_mlstm_b200 import binding as xb
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "xlstm_mlstm.h")
+
+
+def _declared():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(xlstm_\w+)\s*\(", text)))
+
+
+def test_header_declares_expected_entry_points():
+    assert set(_declared()) == set(xb.EXPORTED)
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(xb.LIB_PATH)
+    missing = [name for name in _declared() if not hasattr(lib, name)]
+    assert not missing, missing
+
+
+def test_abi_version_and_status_strings():
+    assert xb.xlstm_abi_version() == 1
+    for s in range(10):
+        assert xb.status_string(s) and "unknown" not in xb.status_string(s)
+    assert "unknown" in xb.status_string(99)
+
+
+@pytest.mark.parametrize("args,expect", [
+    ((1, 1, 64, 64, 64, xb.BF16), xb.OK),
+    ((1, 1, 64, 64, 32, xb.BF16), xb.ERR_CHUNK),      # bf16 chunk must be 64/128/256
+    ((1, 1, 64, 64, 0, xb.F32), xb.ERR_CHUNK),
+    ((1, 1, 64, 64, 2048, xb.F32), xb.ERR_CHUNK),
+    ((1, 1, 64, 24, 64, xb.F32), xb.ERR_SHAPE),       # DH not a multiple of 16
+    ((1, 1, 64, 528, 64, xb.F32), xb.ERR_SHAPE),      # DH > 512
+    ((-1, 1, 64, 64, 64, xb.F32), xb.ERR_SHAPE),
+    ((1, 1, -5, 64, 64, xb.F32), xb.ERR_SHAPE),
+    ((300, 300, 64, 64, 64, xb.F32), xb.ERR_SHAPE),   # B * NH beyond one grid dimension
+    ((1, 1, 64, 64, 64, 7), xb.ERR_DTYPE),
+])
+def test_workspace_size_validation(args, expect):
+    st, _ = xb.xlstm_mlstm_fwd_workspace_size(*args)
+    assert st == expect
+
+
+def test_workspace_size_grows_with_segments_and_is_zero_for_empty():
+    st, n1 = xb.xlstm_mlstm_fwd_workspace_size(1, 2, 1024, 64, 64, xb.F32, xb.PATH_SIMT, 1)
+    st2, n4 = xb.xlstm_mlstm_fwd_workspace_size(1, 2, 1024, 64, 64, xb.F32, xb.PATH_SIMT, 4)
+    assert st == st2 == xb.OK and n4 > n1 > 0
+    # three extra segment summaries of DH*DH + DH floats per head, plus segment stats
+    assert n4 - n1 >= 3 * 2 * (64 * 64 + 64) * 4
+    st, n0 = xb.xlstm_mlstm_fwd_workspace_size(1, 2, 0, 64, 64, xb.F32)
+    assert st == xb.OK and n0 == 0
+
+
+FAKE = 1 << 40          # an aligned address; validation must reject before use
+
+
+def _fwd(**over):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, i_pre=FAKE, f_pre=FAKE, o_pre=FAKE, h=FAKE, C0=None,
+             n0=None, m0=None, C_out=None, n_out=None, m_out=None, B=1, NH=1, S=64, DH=64,
+             chunk=64, dt=xb.F32, fg=xb.FGATE_SIGMOID, workspace=FAKE, workspace_bytes=0,
+             stream=None)
+    a.update(over)
+    return xb.xlstm_mlstm_fwd(**a)
+
+
+@pytest.mark.parametrize("over,expect", [
+    (dict(q=None), xb.ERR_NULL),
+    (dict(o_pre=None), xb.ERR_NULL),
+    (dict(h=None), xb.ERR_NULL),
+    (dict(k=FAKE + 8), xb.ERR_ALIGN),
+    (dict(C0=FAKE + 4), xb.ERR_ALIGN),
+    (dict(fg=5), xb.ERR_DTYPE),
+    (dict(dt=xb.BF16, chunk=100), xb.ERR_CHUNK),
+    (dict(DH=40), xb.ERR_SHAPE),
+    (dict(workspace_bytes=16), xb.ERR_WORKSPACE),       # far smaller than required
+    (dict(workspace=None, workspace_bytes=1 << 30), xb.ERR_WORKSPACE),
+    (dict(segments=-1), xb.ERR_UNSUPPORTED),
+    (dict(path=7), xb.ERR_UNSUPPORTED),
+    (dict(path=xb.PATH_TENSOR, dt=xb.F32), xb.ERR_UNSUPPORTED),
+    (dict(B=0), xb.OK),                                  # no heads: a no-op
+    (dict(NH=0, q=None), xb.OK),
+])
+def test_fwd_rejects_bad_arguments_before_device_work(over, expect):
+    assert _fwd(**over) == expect
+
+
+def _step(**over):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, i_pre=FAKE, f_pre=FAKE, o_pre=FAKE, h=FAKE, C=FAKE, n=FAKE,
+             m=FAKE, B=1, NH=1, DH=64, dt=xb.BF16, fg=xb.FGATE_SIGMOID, stream=None)
+    a.update(over)
+    return xb.xlstm_mlstm_step(**a)
+
+
+@pytest.mark.parametrize("over,expect", [
+    (dict(C=None), xb.ERR_NULL),
+    (dict(m=None), xb.ERR_NULL),
+    (dict(v=FAKE + 2), xb.ERR_ALIGN),
+    (dict(dt=3), xb.ERR_DTYPE),
+    (dict(fg=-1), xb.ERR_DTYPE),
+    (dict(DH=8), xb.ERR_SHAPE),
+    (dict(DH=1024), xb.ERR_SHAPE),
+    (dict(B=-2), xb.ERR_SHAPE),
+    (dict(B=0), xb.OK),
+])
+def test_step_rejects_bad_arguments_before_device_work(over, expect):
+    assert _step(**over) == expect
