@@ -290,6 +290,8 @@ def main():
     ap.add_argument("--chunk", type=int, default=64)
     ap.add_argument("--path", default="auto", choices=["auto", "simt", "tensor"])
     ap.add_argument("--decode-steps", type=int, default=1024)
+    ap.add_argument("--decode-B", type=int, default=0,
+                    help="batch of the decode workload (0 = its full B of 256); profiling only")
     ap.add_argument("--skip-decode", action="store_true")
     ap.add_argument("--skip-e2e", action="store_true")
     ap.add_argument("--skip-cpu", action="store_true")
@@ -412,6 +414,9 @@ def main():
 
 def run_decode(args, dev, dist_on, rank, world, peaks, peak_src):
     d = syn.DECODE
+    if args.decode_B:
+        import dataclasses
+        d = dataclasses.replace(d, B=args.decode_B)
     T = args.decode_steps
     BH, DH = d.B * d.NH, d.DH
     pre = syn.fwd_inputs(d.prefill(), seed=d.seed + rank)

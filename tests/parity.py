@@ -7,28 +7,41 @@ import torch
 import oracle
 from linear_rnn_mlstm_b200 import binding as xb
 
-# Tolerances: max |dh| and relative L2 of h over the whole tensor.
-TOL = {"bf16": (2e-2, 1e-2), "f32": (1e-5, 1e-5)}
+# Tolerances on h: (max error, relative L2 over the whole tensor).  The max
+# error is taken per element in units of max(1, |h_ref|): absolute for
+# |h| <= 1, relative above.  A literal absolute bound is unattainable for a
+# bf16 output: |h| reaches several hundred on these workloads, where one bf16
+# ulp is far larger than 2e-2 (rounding the exact oracle output to bf16 alone
+# exceeds it).
+#
+# "f32_wide": fp32 inputs with wide input gates (itilde ~ N(0, 3)) and the
+# exponential forget gate.  There the stabiliser m reaches |m| ~ 10, so each
+# exponent such as log f + m_prev - m is formed from fp32 numbers whose ulp is
+# ~1e-6; that relative error enters the state once per token and compounds
+# over the sequence (<= 256 tokens here): 256 * 6e-7 ~ 1.5e-4 worst case.
+TOL = {"bf16": (2e-2, 1e-2), "f32": (1e-5, 1e-5), "f32_wide": (2e-4, 1e-4)}
 STATE_REL_L2 = 1e-2        # final C', n' (bf16 inputs)
 STATE_M_ABS = 1e-4         # final m
 
 
 def errors(got, ref):
+    """(max |got - ref| / max(1, |ref|), ||got - ref||_2 / ||ref||_2)."""
     got = np.asarray(got, dtype=np.float64)
     ref = np.asarray(ref, dtype=np.float64)
     diff = got - ref
-    max_abs = float(np.max(np.abs(diff))) if diff.size else 0.0
+    max_scaled = float(np.max(np.abs(diff) / np.maximum(1.0, np.abs(ref)))) if diff.size else 0.0
     denom = float(np.linalg.norm(ref))
     rel = float(np.linalg.norm(diff)) / denom if denom > 0 else float(np.linalg.norm(diff))
-    return max_abs, rel
+    return max_scaled, rel
 
 
 def assert_close(got, ref, dtype, what="h"):
     tol_abs, tol_rel = TOL[dtype]
-    max_abs, rel = errors(got, ref)
-    assert max_abs <= tol_abs and rel <= tol_rel, (
-        f"{what}: max|d|={max_abs:.3e} (tol {tol_abs}), relL2={rel:.3e} (tol {tol_rel})")
-    return max_abs, rel
+    max_scaled, rel = errors(got, ref)
+    assert max_scaled <= tol_abs and rel <= tol_rel, (
+        f"{what}: max|d|/max(1,|ref|)={max_scaled:.3e} (tol {tol_abs}), "
+        f"relL2={rel:.3e} (tol {tol_rel})")
+    return max_scaled, rel
 
 
 def to_cuda(inp):

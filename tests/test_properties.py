@@ -39,7 +39,9 @@ def test_segment_count_invariance(dtype):
     ref = _fwd(x, 64, w.fgate, segments=1)
     for seg in (2, 5, 16):
         h, C, n, m = _fwd(x, 64, w.fgate, segments=seg)
-        tol = "f32" if dtype == "f32" else "bf16"
+        # two fp32 runs with different rounding paths over 1000 tokens: the
+        # compounding bound of the wide-gate case applies, not the tiny one
+        tol = "f32_wide" if dtype == "f32" else "bf16"
         assert_close(h.float().cpu().numpy(), ref[0].float().cpu().numpy(), tol)
         assert np.max(np.abs(m.cpu().numpy() - ref[3].cpu().numpy())) <= 1e-4
 
@@ -54,8 +56,9 @@ def test_split_continuity(dtype):
     b = {k: v[:, :, s1:].contiguous() for k, v in x.items()}
     ha, Ca, na, ma = _fwd(a, 64, w.fgate)
     hb, Cb, nb, mb = _fwd(b, 64, w.fgate, state=(Ca, na, ma))
+    tol = "f32_wide" if dtype == "f32" else "bf16"
     got = torch.cat([ha, hb], 2).float().cpu().numpy()
-    assert_close(got, h.float().cpu().numpy(), dtype)
+    assert_close(got, h.float().cpu().numpy(), tol)
     assert errors(Cb.cpu().numpy(), C.cpu().numpy())[1] <= (1e-5 if dtype == "f32" else 1e-2)
     # forward over S-k, then k decode steps
     k = 16
@@ -64,7 +67,7 @@ def test_split_continuity(dtype):
         y = {kk: v[:, :, t].contiguous() for kk, v in x.items()}
         ht = xb.mlstm_step(y["q"], y["k"], y["v"], y["i_pre"], y["f_pre"], y["o_pre"],
                            Cc, nc, mc, fgate=w.fgate)
-        assert_close(ht.float().cpu().numpy(), h[:, :, t].float().cpu().numpy(), dtype)
+        assert_close(ht.float().cpu().numpy(), h[:, :, t].float().cpu().numpy(), tol)
     assert errors(Cc.cpu().numpy(), C.cpu().numpy())[1] <= (1e-5 if dtype == "f32" else 1e-2)
 
 
