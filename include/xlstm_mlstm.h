@@ -132,6 +132,38 @@ xlstm_status xlstm_mlstm_fwd_ex(const void *q, const void *k, const void *v,
                                 const xlstm_fwd_options *opts, void *cuda_stream);
 
 /*
+ * xlstm_mlstm_fwd without a workspace argument.  (The paper has no
+ * counterpart: this is a calling convention of this library.)
+ *
+ * For callers that cannot allocate device memory: code that reaches this
+ * library only through the C ABI and owns no device allocator (a plugin inside
+ * a runtime that owns all device memory), or a serving loop that must not call
+ * cudaMalloc, which can synchronise the device, fail under memory pressure or
+ * stall for an unbounded time.  Inputs and outputs are passed exactly as for
+ * xlstm_mlstm_fwd; the scratch comes from one device array inside the library
+ * of XLSTM_NOALLOC_SCRATCH_BYTES bytes, which every GPU that loads the library
+ * holds until the process exits.
+ *  - Calls whose xlstm_mlstm_fwd_workspace_size() exceeds that size return
+ *    XLSTM_ERR_WORKSPACE and launch nothing.  Nothing is allocated, ever.
+ *  - The first call on a device looks up the array's device address
+ *    (cudaGetSymbolAddress) with that device current; make that first call
+ *    before any stream capture.
+ *  - All calls share the one array: two calls whose kernels overlap on the GPU
+ *    (different streams, or different host threads) race on it and give wrong
+ *    results.  Serialise them, e.g. by issuing them on one stream.  The array
+ *    keeps the last call's contents; the forward overwrites whatever it reads,
+ *    so no clearing is needed.
+ */
+#define XLSTM_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+xlstm_status xlstm_mlstm_fwd_noalloc(const void *q, const void *k, const void *v,
+                                     const float *i_pre, const float *f_pre, const float *o_pre,
+                                     void *h,
+                                     const float *C0, const float *n0, const float *m0,
+                                     float *C_out, float *n_out, float *m_out,
+                                     int B, int NH, int S, int DH, int chunk,
+                                     xlstm_dtype dt, xlstm_fgate fg, void *cuda_stream);
+
+/*
  * One recurrent decode token for every (b, h), updating the resident state in
  * place (section 2.5 of the paper: constant memory in the sequence length).
  *

@@ -25,7 +25,9 @@ PATH_AUTO, PATH_SIMT, PATH_TENSOR = 0, 1, 2
 
 EXPORTED = ("xlstm_abi_version", "xlstm_status_string", "xlstm_mlstm_fwd_workspace_size",
             "xlstm_mlstm_fwd_workspace_size_ex", "xlstm_mlstm_fwd", "xlstm_mlstm_fwd_ex",
-            "xlstm_mlstm_step", "xlstm_device_status", "xlstm_profile_begin", "xlstm_profile_end")
+            "xlstm_mlstm_step", "xlstm_device_status", "xlstm_profile_begin", "xlstm_profile_end",
+            "xlstm_mlstm_fwd_noalloc")
+NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
 
 
 class XlstmError(RuntimeError):
@@ -75,6 +77,8 @@ def load(path: str = LIB_PATH):
         lib.xlstm_mlstm_step.restype = i
         lib.xlstm_device_status.argtypes = [vp]
         lib.xlstm_device_status.restype = i
+        lib.xlstm_mlstm_fwd_noalloc.argtypes = [vp] * 3 + [fp] * 3 + [vp] + [fp] * 6 + [i] * 7 + [vp]
+        lib.xlstm_mlstm_fwd_noalloc.restype = i
         lib.xlstm_profile_begin.restype = i
         lib.xlstm_profile_end.argtypes = [ctypes.POINTER(KernelTime), i, ctypes.POINTER(i)]
         lib.xlstm_profile_end.restype = i
@@ -107,6 +111,13 @@ def xlstm_mlstm_fwd(q, k, v, i_pre, f_pre, o_pre, h, C0, n0, m0, C_out, n_out, m
     return load().xlstm_mlstm_fwd_ex(q, k, v, i_pre, f_pre, o_pre, h, C0, n0, m0,
                                      C_out, n_out, m_out, B, NH, S, DH, chunk, dt, fg,
                                      workspace, workspace_bytes, ctypes.byref(opts), stream)
+
+
+def xlstm_mlstm_fwd_noalloc(q, k, v, i_pre, f_pre, o_pre, h, C0, n0, m0, C_out, n_out, m_out,
+                            B, NH, S, DH, chunk, dt, fg, stream):
+    """The forward with the library's built-in scratch (no workspace argument)."""
+    return load().xlstm_mlstm_fwd_noalloc(q, k, v, i_pre, f_pre, o_pre, h, C0, n0, m0,
+                                          C_out, n_out, m_out, B, NH, S, DH, chunk, dt, fg, stream)
 
 
 def xlstm_mlstm_step(q, k, v, i_pre, f_pre, o_pre, h, C, n, m, B, NH, DH, dt, fg, stream):
