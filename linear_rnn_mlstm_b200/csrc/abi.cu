@@ -36,14 +36,23 @@ bool make_fwd_plan(int B, int NH, int S, int DH, int L, int path, int forced_seg
         return true;
     }
     int P;
+    const long per_set = (long)p->BH * p->ntiles;
     if (forced_segments > 0) {
         P = forced_segments;
+    } else if (path == XLSTM_PATH_TENSOR) {
+        // one CTA per SM (shared memory and TMEM are sized for that): fill one wave
+        P = (int)(num_sms / per_set);
     } else {
-        const long per_set = (long)p->BH * p->ntiles;
         const long target = 2L * num_sms;
         P = (int)((target + per_set - 1) / per_set);
     }
     if (P < 1) P = 1;
+    if (path == XLSTM_PATH_TENSOR) {
+        // the per-CTA chunk tables hold a bounded number of chunks
+        const int cap = tensor_path_max_chunks_per_segment();
+        const int need = (p->nchunks + cap - 1) / cap;
+        if (P < need) P = need;
+    }
     if (P > p->nchunks) P = p->nchunks;
     if (P > kMaxHeads) P = kMaxHeads;
     p->cps = (p->nchunks + P - 1) / P;
@@ -51,6 +60,7 @@ bool make_fwd_plan(int B, int NH, int S, int DH, int L, int path, int forced_seg
 
     size_t off = 0;
     p->off_bcum = off;  off = align64(off + (size_t)p->BH * S);
+    p->off_pmax = off;  off = align64(off + (size_t)p->BH * S);
     p->off_cstat = off; off = align64(off + (size_t)p->BH * p->nchunks * 2);
     p->off_sstat = off; off = align64(off + (size_t)p->BH * p->P * 2);
     p->off_summ = off;  off = align64(off + (size_t)p->BH * (p->P - 1) * ((size_t)DH * DH + DH));

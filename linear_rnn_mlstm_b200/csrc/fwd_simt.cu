@@ -25,10 +25,11 @@ namespace xlstm {
 
 // ------------------------------------------------------------------ phase 0
 // One warp per (head, chunk): lf, the chunk-local inclusive prefix sum b, the
-// chunk total and the chunk maximum of u = li - b.
+// chunk-local inclusive prefix maximum of u = li - b, the chunk total and the
+// chunk maximum of u.
 __global__ void __launch_bounds__(256)
 gate_prologue_kernel(const float *__restrict__ i_pre, const float *__restrict__ f_pre,
-                     float *__restrict__ bcum, float2 *__restrict__ cstat,
+                     float *__restrict__ bcum, float *__restrict__ pmx, float2 *__restrict__ cstat,
                      int BH, int S, int L, int nchunks, int fgate_exp) {
     const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
@@ -48,13 +49,20 @@ gate_prologue_kernel(const float *__restrict__ i_pre, const float *__restrict__ 
             if (lane >= o) lf += y;
         }
         const float b = carry + lf;
+        float u = ok ? i_pre[base + tt] - b : -INFINITY;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {          // inclusive prefix max of u
+            const float y = __shfl_up_sync(0xffffffffu, u, o);
+            if (lane >= o) u = fmaxf(u, y);
+        }
+        u = fmaxf(u, umax);
         if (ok) {
             bcum[base + tt] = b;
-            umax = fmaxf(umax, i_pre[base + tt] - b);
+            pmx[base + tt] = u;
         }
         carry = __shfl_sync(0xffffffffu, b, 31);
+        umax = __shfl_sync(0xffffffffu, u, 31);
     }
-    umax = warp_max(umax);
     if (lane == 0) cstat[(size_t)bh * nchunks + c] = make_float2(carry, umax);
 }
 
@@ -185,7 +193,6 @@ segment_output_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, con
     float *gb = iden + 16;                  // [L]   b_t
     float *gu = gb + L;                     // [L]   u_t = li - b
     float *gm = gu + L;                     // [L]   m_t
-    __shared__ float s_m[2];
 
     const size_t tok_base = (size_t)bh * S;
     // ---- incoming state: initial state folded with the summaries of segments < g
@@ -384,7 +391,7 @@ cudaError_t launch_gate_prologue(const FwdArgs &a, const FwdPlan &p, cudaStream_
     const int warps = p.BH * p.nchunks;
     const int blocks = (warps + 7) / 8;
     KernelTimer timer("gate_prologue", st);
-    gate_prologue_kernel<<<blocks, 256, 0, st>>>(a.i_pre, a.f_pre, ws + p.off_bcum,
+    gate_prologue_kernel<<<blocks, 256, 0, st>>>(a.i_pre, a.f_pre, ws + p.off_bcum, ws + p.off_pmax,
                                                  (float2 *)(ws + p.off_cstat), p.BH, p.S, p.L,
                                                  p.nchunks, a.fgate_exp);
     return cudaGetLastError();

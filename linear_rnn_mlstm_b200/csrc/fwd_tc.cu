@@ -1,14 +1,1138 @@
-// Chunkwise mLSTM forward on the 5th-generation tensor cores (tcgen05).
+// Chunkwise mLSTM forward on the 5th-generation tensor cores (tcgen05, TMEM, TMA).
+//
+// Computes the same chunkwise-parallel form as the fp32 SIMT kernels (see
+// fwd_simt.cu for the notation) for bf16 q/k/v, chunk L = 64, DH in {128, 256},
+// with value rows tiled by 128 per CTA ("xLSTM: Extended Long Short-Term
+// Memory" section 2.3: retrieval by matrix multiplication, covariance update of
+// the matrix memory).  Per chunk of a segment, on the tensor cores:
+//
+//   S    = Q [K ; n'_prev hi ; n'_prev lo]^T           M=64,  N=72, K=DH (bf16)
+//   H~^T = Cs Q^T                                      M=128, N=64, K=DH (tf32, Cs in TMEM)
+//   H~^T += (w^ V)^T (Shi + Slo)^T  (scores masked s<=t) M=128, N=64, K=64 (bf16)
+//   Cs  += (w^ V)^T K                                  M=128, N=DH, K=64 (bf16)
+//
+// Cs is the CTA's 128 value rows of the state, resident in TMEM in fp32 for the
+// whole segment and lazily scaled, C' = Lambda Cs; w^_s = e^{u_s + b_L - m_next}
+// / (sqrt(d) Lambda_c) folds the gates, the key scaling and the lazy scale into
+// V.  With that choice the decayed intra-chunk weight factorises exactly,
+//   e^{b_t - b_s + itilde_s - m_t} / sqrt(d) = F_t w^_s,  F_t = g_t Lambda_prev,
+// and F_t is also the retrieval's row scale, so
+//   h_t = o_t F_t H~_t / max(|g_t n'_prev.q_t + F_t sum_s w^_s S_ts|, e^{-m_t})
+// needs no per-element exponential and the retrieval uses Q as loaded.  The
+// normaliser n' rides in two extra key rows of S (hi and lo bf16 parts); the
+// masked scores go to the MMA as hi + lo bf16 parts, since the intra term can
+// nearly cancel against the normaliser and one bf16 rounding there would be
+// amplified in h.
+//
+// Every wait is bounded (tc_ptx.cuh): on a timeout the kernel raises the device
+// status word and unwinds.
+#include <mutex>
+
 #include "common.cuh"
 #include "kernels.h"
+#include "profile.h"
+#include "tc_ptx.cuh"
 
 namespace xlstm {
 
-bool tensor_path_supports(int DH, int L) { (void)DH; (void)L; return false; }
+using namespace tc;
+
+namespace {
+
+constexpr int kL = 64;             // tokens per chunk on this path
+constexpr int kRows = 128;         // value rows per CTA
+constexpr int kKRows = 72;         // key-tile rows: 64 keys, n' hi, n' lo, 6 zero rows
+constexpr int kKBlock = kKRows * 128;   // bytes per 64-column block of the key tile
+constexpr int kThreads = 192;
+constexpr int kMaxCps = 256;       // chunks per segment the tables hold
+constexpr float kLnLambdaFloor = -40.f;  // rescale the TMEM state below this log scale
+constexpr float kLnChunkFloor = -60.f;   // smallest decay of the state's scale over one chunk (see below)
+
+__device__ __forceinline__ void named_sync_compute() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+#ifdef XLSTM_TC_TRACE
+// Timing trace of the pipeline steps (diagnostic builds only): 32 globaltimer
+// stamps per (CTA, chunk).
+__device__ unsigned long long *g_tc_trace = nullptr;
+#define TC_TRACE(cond, c, slot)                                                                    \
+    do {                                                                                           \
+        if (g_tc_trace && (cond)) {                                                                \
+            const size_t cta_ = ((size_t)blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x; \
+            g_tc_trace[(cta_ * kMaxCps + (c)) * 32 + (slot)] = globaltimer_ns();                   \
+        }                                                                                          \
+    } while (0)
+#else
+#define TC_TRACE(cond, c, slot) do { } while (0)
+#endif
+
+// A bounded wait taken by all 128 compute threads, with a group-uniform result.
+__device__ __forceinline__ bool compute_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                             unsigned int *status) {
+    return group_all<1, 128>(mbar_wait(bar, parity, abort_flag, status));
+}
+
+__device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
+    return p + ((1024u - (smem_u32(p) & 1023u)) & 1023u);
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t *>(&v);
+}
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// ------------------------------------------------------------ segment outputs
+template <int D>
+struct OutLayout {
+    static constexpr int kQ = 0;                          // Q  bf16 K-major: D/64 blocks x 8 KB
+    static constexpr int kKslot = (D / 64) * kKBlock;     // one key slot: D/64 blocks x 72 rows
+    static constexpr int kK = kQ + D * 128;
+    static constexpr int kV = kK + 2 * kKslot;            // V, scaled in place to w^ V: 2 blocks x 8 KB
+    static constexpr int kQt = kV + 16384;                // Q as fp32 (tf32 operand), K-major: D/32 blocks x 8 KB
+    static constexpr int kP = kQt + D * 256;              // masked scores, high bf16 part, K-major: 64 x 128 B
+    static constexpr int kPl = kP + 8192;                 // masked scores, low bf16 part
+    static constexpr int kHs = kPl + 8192;                // h tile for the TMA store: 2 blocks x 64 rows x 128 B
+    static constexpr int kF = kHs + 16384;                // float arrays (see kernel)
+    static constexpr int kNF = 16 * 64;
+    static constexpr int kTab = kF + kNF * 4;             // per-chunk tables
+    static constexpr int kBar = kTab + 5 * kMaxCps * 4;
+    static constexpr int kNumBars = 32;
+    static constexpr int kMisc = kBar + kNumBars * 8;     // tmem base, abort flag
+    static constexpr int kEnd = kMisc + 16;
+    static constexpr int kBytes = kEnd + 1024;            // slack for 1024-byte alignment
+};
+
+constexpr int kMaxSmemPerCta = 232448;   // 227 KB of opt-in shared memory per CTA on sm_100
+static_assert(OutLayout<256>::kBytes <= kMaxSmemPerCta, "output kernel shared memory");
+
+enum {
+    B_FULL_Q = 0, B_Q_FREE, B_FULL_K0, B_FULL_K1, B_K_FREE0, B_K_FREE1, B_FULL_V, B_V_FREE,
+    B_VHAT_READY, B_QT_READY, B_QT_FREE, B_S_FULL, B_S_FREE, B_P_READY, B_P_FREE,
+    B_H_FULL0, B_H_FULL1, B_H_FREE0, B_H_FREE1, B_NROW_READY0, B_NROW_READY1, B_RESC_DONE, B_DONE,
+    B_GATES_READY0, B_GATES_READY1, B_GATES_FREE0, B_GATES_FREE1,
+    B_FINV_READY0, B_FINV_READY1, B_FINV_FREE0, B_FINV_FREE1, B_INTRA_DONE, B_NUM
+};
+static_assert(B_NUM <= OutLayout<128>::kNumBars, "barrier slots");
+// Every barrier is waited by parity, so no producer may complete a barrier twice
+// ahead of a waiter.  Buffers that a producer can refill before the consumer of
+// the previous fill has waited are double-buffered with their own barriers
+// (key-slot normaliser rows, gate arrays, denominators, H accumulators).
+
+// Per-CTA tables built from the chunk statistics: for each chunk of the
+// segment, the stabiliser at its start, the state scale used by its retrieval,
+// the rescale factor applied before it (0 = none), ln(1/Lambda) after its
+// update, and whether it is a wide chunk.
+//
+// A chunk is wide when its largest input-gate term outweighs the decayed state
+// it starts from by more than e^60 (m_prev - max_s u_s < -60).  The factorised
+// intra weights F_t w^_s would then leave the fp32 range, so a wide chunk takes
+// exact weights instead: the score group forms e^{u_s + b_t - m_t} S_ts / sqrt(d)
+// per element, the retrieval operand is g_t q_t, and V is scaled by w^ only
+// after the intra-chunk MMA has read it (MMA order retrieval, intra, update).
+struct ChunkTab {
+    float *mprev, *lamret, *resc, *lnupd, *wide;
+};
+
+__device__ __forceinline__ float ldg_nc_early(const float *p) {
+    float v;
+    asm volatile("ld.global.nc.f32 %0, [%1];" : "=f"(v) : "l"(p));   // volatile: issued where written
+    return v;
+}
+
+// Warp roles: 0 TMA, 1 MMA (and TMEM owner), 2-5 operand group (gates, Q as
+// fp32, normaliser chain, w^ V, rescale, final state), 6-9 score group (masked
+// scores and the denominators; one warp per TMEM lane quadrant), 10-13 output
+// group (h; one warp per quadrant, the chunk's tokens in two passes of 32).
+// Each group has its own named barrier and one thread that polls mbarriers for
+// it.  14 warps: at most 4 per SM sub-partition, so 128 registers fit.
+constexpr int kOutThreads = 448;
+
+__device__ __forceinline__ void sync_ops() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+__device__ __forceinline__ void sync_sco() { asm volatile("bar.sync 2, 128;" ::: "memory"); }
+__device__ __forceinline__ void sync_out() { asm volatile("bar.sync 3, 128;" ::: "memory"); }
+__device__ __forceinline__ bool wait_ops(uint64_t *bar, uint32_t parity, volatile int *abort_flag, unsigned int *status) {
+    return group_wait<1, 128>(bar, parity, threadIdx.x == 64, abort_flag, status);
+}
+__device__ __forceinline__ bool wait_sco(uint64_t *bar, uint32_t parity, volatile int *abort_flag, unsigned int *status) {
+    return group_wait<2, 128>(bar, parity, threadIdx.x == 192, abort_flag, status);
+}
+__device__ __forceinline__ bool wait_out(uint64_t *bar, uint32_t parity, volatile int *abort_flag, unsigned int *status) {
+    return group_wait<3, 128>(bar, parity, threadIdx.x == 320, abort_flag, status);
+}
+
+template <int D>
+__global__ void __launch_bounds__(kOutThreads, 1)
+segment_output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
+                         const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_h,
+                         const float *__restrict__ i_pre, const float *__restrict__ o_pre,
+                         const float *__restrict__ C0, const float *__restrict__ n0, const float *__restrict__ m0,
+                         float *__restrict__ C_out, float *__restrict__ n_out, float *__restrict__ m_out,
+                         const float *__restrict__ bcum, const float *__restrict__ pmx,
+                         const float2 *__restrict__ cstat,
+                         const float2 *__restrict__ sstat, const float *__restrict__ summ,
+                         unsigned int *status, int S, int nchunks, int P, int cps) {
+    using Lay = OutLayout<D>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = align1024(smem_raw);
+    uint8_t *sQ = smem + Lay::kQ;
+    uint8_t *sK = smem + Lay::kK;
+    uint8_t *sV = smem + Lay::kV;
+    uint8_t *sQt = smem + Lay::kQt;
+    uint8_t *sP = smem + Lay::kP;
+    uint8_t *sPl = smem + Lay::kPl;
+    uint8_t *sHs = smem + Lay::kHs;
+    // per-token arrays, [2][64] by chunk parity, written by the operand group
+    float *fm = reinterpret_cast<float *>(smem + Lay::kF);   // m_t
+    float *fg = fm + 128;                                    // g_t = e^{b_t + m_prev - m_t}
+    float *fF = fg + 128;                                    // F_t = g_t * Lambda_prev (row scale of H)
+    float *fw = fF + 128;                                    // w^_s: weight folded into V (per key)
+    float *fpw = fw + 128;                                   // [64] normaliser weight (operand group only)
+    float *finv = fpw + 64;                                  // [2][64] F_t / denominator (score -> output)
+    float *fu = finv + 128;                                  // [2][64] u_s (wide chunks)
+    float *frun = fu + 128;                                  // [2][64] m_t - b_t (wide chunks)
+    ChunkTab tab;
+    tab.mprev = reinterpret_cast<float *>(smem + Lay::kTab);
+    tab.lamret = tab.mprev + kMaxCps;
+    tab.resc = tab.lamret + kMaxCps;
+    tab.lnupd = tab.resc + kMaxCps;
+    tab.wide = tab.lnupd + kMaxCps;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Lay::kBar);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + Lay::kMisc);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + Lay::kMisc + 4);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int tile = blockIdx.x, g = blockIdx.y, bh = blockIdx.z;
+    const int i0 = tile * kRows;
+    const int c0 = g * cps;
+    const int nch = min(nchunks, c0 + cps) - c0;
+    const size_t tok0 = (size_t)bh * S;
+    const float inv_sqrt_d = rsqrtf((float)D);
+    const int q4 = warp & 3;                                 // TMEM lane quadrant of this warp
+    const uint32_t lane_addr = ((uint32_t)(32 * q4)) << 16;
+    const bool is_ops = warp >= 2 && warp < 6;
+    const bool is_sco = warp >= 6 && warp < 10;
+    const bool is_out = warp >= 10;
+    const int ct = tid - 64;                                 // operand-group thread 0..127
+    const int st_ = tid - 192;                               // score-group thread 0..127
+    const int xt = tid - 320;                                // output-group thread 0..127
+
+    // ------------------------------------------------------------ set-up
+    if (tid == 0) {
+        for (int i = 0; i < B_NUM; ++i) mbar_init(&bars[i], i == B_Q_FREE ? 2 : 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, 512);
+        tc_fence_before();
+    }
+    float nreg[D / 128];                           // operand group: n' entries j = nj(r)
+    // key column of the operand group's r-th normaliser register (adjacent pairs for DH = 256)
+    auto nj = [&](int r) { return D == 256 ? 2 * (tid - 64) + r : (tid - 64); };
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = *tmem_slot;
+    const uint32_t t_state = tbase;                // columns [0, D)
+    const uint32_t t_S = tbase + 256;              // columns [256, 328)
+    const uint32_t t_H0 = tbase + 384;             // columns [384, 448) and [448, 512)
+
+    if (is_ops) {
+        // Incoming state: the initial state folded with the summaries of segments < g.
+        const float m_init = m0 ? m0[bh] : 0.f;
+        const int i = 32 * q4 + lane;
+        for (int jb = 0; jb < D; jb += 16) {
+            float v[16];
+            const float *c0row = C0 ? C0 + ((size_t)bh * D + i0 + i) * D + jb : nullptr;
+#pragma unroll
+            for (int e = 0; e < 16; ++e) v[e] = c0row ? c0row[e] : 0.f;
+            float mc = m_init;
+            for (int gp = 0; gp < g; ++gp) {
+                const float2 st = sstat[(size_t)bh * P + gp];
+                const float mn = fmaxf(st.x + mc, st.y);
+                const float al = expf(st.x + mc - mn), be = expf(st.y - mn);
+                const float *sm = summ + ((size_t)bh * (P - 1) + gp) * ((size_t)D * D + D) +
+                                  (size_t)(i0 + i) * D + jb;
+#pragma unroll
+                for (int e = 0; e < 16; ++e) v[e] = al * v[e] + be * sm[e];
+                mc = mn;
+            }
+            uint32_t r[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) r[e] = __float_as_uint(v[e]);
+            tmem_st16(t_state + lane_addr + jb, r);
+        }
+        tmem_wait_st();
+#pragma unroll
+        for (int r = 0; r < D / 128; ++r) {
+            const int j = nj(r);
+            float nv = n0 ? n0[(size_t)bh * D + j] : 0.f;
+            float mc = m_init;
+            for (int gp = 0; gp < g; ++gp) {
+                const float2 st = sstat[(size_t)bh * P + gp];
+                const float mn = fmaxf(st.x + mc, st.y);
+                const float al = expf(st.x + mc - mn), be = expf(st.y - mn);
+                nv = al * nv + be * summ[((size_t)bh * (P - 1) + gp) * ((size_t)D * D + D) + (size_t)D * D + j];
+                mc = mn;
+            }
+            nreg[r] = nv;
+        }
+        // zero the extra key rows 64..71 of both slots, then n'_in (hi, lo) in slot 0
+        for (int e = ct; e < 2 * (D / 64) * 8 * 8; e += 128) {      // (slot, block, row, chunk)
+            const int ch = e & 7, row = 64 + ((e >> 3) & 7), blk = (e >> 6) % (D / 64), slot = e / (64 * (D / 64));
+            *reinterpret_cast<uint4 *>(sK + slot * Lay::kKslot + blk * kKBlock + sw128_offset(row, ch)) =
+                make_uint4(0u, 0u, 0u, 0u);
+        }
+        sync_ops();
+#pragma unroll
+        for (int r = 0; r < D / 128; ++r) {
+            const int j = nj(r);
+            const float hi = __bfloat162float(__float2bfloat16_rn(nreg[r]));
+            uint8_t *blkp = sK + (j / 64) * kKBlock;
+            const int cc = (j % 64) / 8, within = (j % 8) * 2;
+            *reinterpret_cast<__nv_bfloat16 *>(blkp + sw128_offset(64, cc) + within) = __float2bfloat16_rn(hi);
+            *reinterpret_cast<__nv_bfloat16 *>(blkp + sw128_offset(65, cc) + within) = __float2bfloat16_rn(nreg[r] - hi);
+        }
+        if (ct == 0) {       // per-chunk tables
+            float mc = m_init;
+            for (int gp = 0; gp < g; ++gp) {
+                const float2 st = sstat[(size_t)bh * P + gp];
+                mc = fmaxf(st.x + mc, st.y);
+            }
+            // ln Lambda stays in [-60, 0]: a chunk whose own decay of the stabilised
+            // state, m_prev - max_s u_s, is below -60 is taken as -60.  That chunk
+            // holds a term e^60 times heavier than the whole earlier state, so the
+            // earlier state's share after it is below fp32 resolution either way.
+            float lnlam = 0.f;
+            for (int c = 0; c < nch; ++c) {
+                const float2 cs = cstat[(size_t)bh * nchunks + c0 + c];
+                const float mn = cs.x + fmaxf(mc, cs.y);
+                const float lna_true = cs.x + mc - mn;       // <= 0
+                const float lna = fmaxf(lna_true, kLnChunkFloor);
+                tab.mprev[c] = mc;
+                tab.wide[c] = lna_true < kLnChunkFloor ? 1.f : 0.f;
+                if (lnlam + lna < kLnLambdaFloor && c > 0) {
+                    tab.resc[c] = expf(lnlam);               // Cs <- Lambda Cs before chunk c
+                    lnlam = 0.f;
+                } else {
+                    tab.resc[c] = 0.f;
+                }
+                tab.lamret[c] = expf(lnlam);
+                lnlam += lna;
+                tab.lnupd[c] = -lnlam;                       // ln (1 / Lambda) after chunk c
+                mc = mn;
+            }
+        }
+        fence_async_smem();
+        tc_fence_before();
+    }
+    __syncthreads();
+    tc_fence_after();
+
+    const uint32_t idesc_S = idesc_f32acc(kFmtBF16, kFmtBF16, false, false, 64, kKRows);
+    const uint32_t idesc_R = idesc_f32acc(kFmtTF32, kFmtTF32, false, false, 128, 64);
+    const uint32_t idesc_I = idesc_f32acc(kFmtBF16, kFmtBF16, true, false, 128, 64);
+    const uint32_t idesc_U = idesc_f32acc(kFmtBF16, kFmtBF16, true, true, 128, D);
+
+    if (warp == 0) {
+        // ---------------------------------------------------------- TMA producer
+        if (lane == 0) {
+            tma_prefetch_desc(&map_q);
+            tma_prefetch_desc(&map_k);
+            tma_prefetch_desc(&map_v);
+            int issued_q = 0, issued_k[2] = {0, 0}, issued_v = 0;
+            for (int c = 0; c < nch; ++c) {
+                const int t0 = (c0 + c) * kL;
+                if (c >= 1 && !mbar_wait(&bars[B_Q_FREE], (c - 1) & 1, abort_flag, status)) break;
+                mbar_arrive_expect_tx(&bars[B_FULL_Q], kL * D * 2);
+                for (int jb = 0; jb < D / 64; ++jb)
+                    tma_load_3d(sQ + jb * 8192, &map_q, &bars[B_FULL_Q], jb * 64, t0, bh);
+                ++issued_q;
+                const int slot = c & 1;
+                if (c >= 2 && !mbar_wait(&bars[B_K_FREE0 + slot], ((c >> 1) - 1) & 1, abort_flag, status)) break;
+                mbar_arrive_expect_tx(&bars[B_FULL_K0 + slot], kL * D * 2);
+                for (int jb = 0; jb < D / 64; ++jb)
+                    tma_load_3d(sK + slot * Lay::kKslot + jb * kKBlock, &map_k, &bars[B_FULL_K0 + slot],
+                                jb * 64, t0, bh);
+                ++issued_k[slot];
+                if (c >= 1 && !mbar_wait(&bars[B_V_FREE], (c - 1) & 1, abort_flag, status)) break;
+                mbar_arrive_expect_tx(&bars[B_FULL_V], kL * kRows * 2);
+                for (int b = 0; b < 2; ++b)
+                    tma_load_3d(sV + b * 8192, &map_v, &bars[B_FULL_V], i0 + 64 * b, t0, bh);
+                ++issued_v;
+            }
+            // never leave a load in flight into shared memory
+            if (issued_q) mbar_wait(&bars[B_FULL_Q], (issued_q - 1) & 1, nullptr, status);
+            for (int s = 0; s < 2; ++s)
+                if (issued_k[s]) mbar_wait(&bars[B_FULL_K0 + s], (issued_k[s] - 1) & 1, nullptr, status);
+            if (issued_v) mbar_wait(&bars[B_FULL_V], (issued_v - 1) & 1, nullptr, status);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            int nresc = 0;
+            bool ok = true;
+            auto issue_S = [&](int c) {
+                const int slot = c & 1;
+                const uint32_t qa = smem_u32(sQ), ka = smem_u32(sK + slot * Lay::kKslot);
+#pragma unroll 1
+                for (int ks = 0; ks < D / 16; ++ks) {
+                    const uint32_t off_q = (ks >> 2) * 8192 + (ks & 3) * 32;
+                    const uint32_t off_k = (ks >> 2) * kKBlock + (ks & 3) * 32;
+                    mma_bf16_ss(t_S, sdesc_sw128(qa + off_q, 16, 1024), sdesc_sw128(ka + off_k, 16, 1024),
+                                idesc_S, ks > 0);
+                }
+                mma_commit(&bars[B_S_FULL]);
+                mma_commit(&bars[B_Q_FREE]);
+            };
+            ok = mbar_wait(&bars[B_FULL_Q], 0, abort_flag, status) &&
+                 mbar_wait(&bars[B_FULL_K0], 0, abort_flag, status);
+            if (ok) {
+                tc_fence_after();
+                issue_S(0);
+            }
+            for (int c = 0; ok && c < nch; ++c) {
+                const int hb = c & 1;
+                const uint32_t t_H = t_H0 + 64 * hb;
+                if (tab.resc[c] != 0.f) {
+                    if (!mbar_wait(&bars[B_RESC_DONE], nresc & 1, abort_flag, status)) { ok = false; break; }
+                    ++nresc;
+                }
+                if (!mbar_wait(&bars[B_QT_READY], c & 1, abort_flag, status)) { ok = false; break; }
+                if (c >= 2 && !mbar_wait(&bars[B_H_FREE0 + hb], ((c >> 1) - 1) & 1, abort_flag, status)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                TC_TRACE(true, c, 12);
+                {   // retrieval from the state at the chunk start: H^T = Cs Q^T (tf32, Cs in TMEM)
+                    const uint32_t qta = smem_u32(sQt);
+#pragma unroll 1
+                    for (int ks = 0; ks < D / 8; ++ks) {
+                        const uint32_t off = (ks >> 2) * 8192 + (ks & 3) * 32;
+                        mma_tf32_ts(t_H, t_state + ks * 8, sdesc_sw128(qta + off, 16, 1024), idesc_R, ks > 0);
+                    }
+                    mma_commit(&bars[B_QT_FREE]);
+                }
+                auto update = [&]() -> bool {   // state update: Cs += (w^ V)^T K
+                    if (!mbar_wait(&bars[B_VHAT_READY], c & 1, abort_flag, status)) return false;
+                    tc_fence_after();
+                    TC_TRACE(true, c, 15);
+                    const uint32_t va = smem_u32(sV), ka = smem_u32(sK + (c & 1) * Lay::kKslot);
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks)
+                        mma_bf16_ss(t_state, sdesc_sw128(va + ks * 2048, 8192, 1024),
+                                    sdesc_sw128(ka + ks * 2048, kKBlock, 1024), idesc_U, 1);
+                    mma_commit(&bars[B_K_FREE0 + (c & 1)]);
+                    return true;
+                };
+                auto intra = [&]() -> bool {    // H^T += Vs^T (Phi + Plo)^T over the masked scores
+                    if (!mbar_wait(&bars[B_P_READY], c & 1, abort_flag, status)) return false;
+                    tc_fence_after();
+                    TC_TRACE(true, c, 13);
+                    const uint32_t va = smem_u32(sV), pa = smem_u32(sP), pla = smem_u32(sPl);
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks)
+                        mma_bf16_ss(t_H, sdesc_sw128(va + ks * 2048, 8192, 1024),
+                                    sdesc_sw128(pa + ks * 32, 16, 1024), idesc_I, 1);
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks)
+                        mma_bf16_ss(t_H, sdesc_sw128(va + ks * 2048, 8192, 1024),
+                                    sdesc_sw128(pla + ks * 32, 16, 1024), idesc_I, 1);
+                    mma_commit(&bars[B_H_FULL0 + hb]);
+                    mma_commit(&bars[B_P_FREE]);
+                    return true;
+                };
+                if (tab.wide[c] == 0.f) {       // V already holds w^ V
+                    if (!update() || !intra()) { ok = false; break; }
+                } else {                        // V unscaled for the intra term, then w^ V
+                    if (!intra()) { ok = false; break; }
+                    mma_commit(&bars[B_INTRA_DONE]);
+                    if (!update()) { ok = false; break; }
+                }
+                mma_commit(&bars[B_V_FREE]);
+                if (c + 1 < nch) {   // scores of the next chunk
+                    const int slot = (c + 1) & 1;
+                    if (!mbar_wait(&bars[B_FULL_Q], (c + 1) & 1, abort_flag, status) ||
+                        !mbar_wait(&bars[B_FULL_K0 + slot], ((c + 1) >> 1) & 1, abort_flag, status) ||
+                        !mbar_wait(&bars[B_NROW_READY0 + slot], (c >> 1) & 1, abort_flag, status) ||
+                        !mbar_wait(&bars[B_S_FREE], c & 1, abort_flag, status)) { ok = false; break; }
+                    tc_fence_after();
+                    TC_TRACE(true, c, 14);
+                    issue_S(c + 1);
+                }
+            }
+            mma_commit(&bars[B_DONE]);
+            // drain: every MMA issued has completed before TMEM is released
+            mbar_wait(&bars[B_DONE], 0, nullptr, status);
+        }
+    } else if (is_ops) {
+        // --------------------------------------------------------- operand group
+        bool ok = true;
+        int nwide = 0;
+        float pre_b = 0.f, pre_i = 0.f, pre_x = 0.f;         // prefetched gates of the next chunk
+        float2 pre_cs = make_float2(0.f, 0.f);
+        if (nch > 0) {
+            const int t0 = c0 * kL;
+            pre_cs = cstat[(size_t)bh * nchunks + c0];
+            if (ct < kL && t0 + ct < S) {
+                pre_b = bcum[tok0 + t0 + ct];
+                pre_i = i_pre[tok0 + t0 + ct];
+                pre_x = pmx[tok0 + t0 + ct];
+            }
+        }
+        for (int c = 0; ok && c < nch; ++c) {
+            const int t0 = (c0 + c) * kL;
+            const int Lc = min(kL, S - t0);
+            const int pb = c & 1;
+            const float mprev = tab.mprev[c];
+            const float2 cs = pre_cs;                         // (sum of log f, max of u) of this chunk
+            const float mnext = cs.x + fmaxf(mprev, cs.y);
+            const bool wide = tab.wide[c] != 0.f;
+            TC_TRACE(ct == 0, c, 0);
+            // (1) lazy rescale of the TMEM state before this chunk's retrieval
+            if (tab.resc[c] != 0.f) {
+                if (!wait_ops(&bars[B_K_FREE0 + ((c - 1) & 1)], ((c - 1) >> 1) & 1, abort_flag, status)) { ok = false; break; }
+                __syncwarp();
+                tc_fence_after();
+                const float f = tab.resc[c];
+                for (int jb = 0; jb < D; jb += 16) {
+                    uint32_t r[16];
+                    tmem_ld16(t_state + lane_addr + jb, r);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * f);
+                    tmem_st16(t_state + lane_addr + jb, r);
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                sync_ops();
+                if (ct == 0) mbar_arrive(&bars[B_RESC_DONE]);
+            }
+            // (2) per-token gates of this chunk (parity buffer pb):
+            //     m_t = b_t + max(m_prev, chunk prefix max of u)
+            if (c >= 2 && !wait_ops(&bars[B_GATES_FREE0 + pb], ((c >> 1) - 1) & 1, abort_flag, status)) { ok = false; break; }
+            if (ct < kL) {
+                const int t = ct;
+                const bool valid = t < Lc;
+                const float b = valid ? pre_b : 0.f;
+                const float u = valid ? pre_i - pre_b : -INFINITY;
+                const float run = fmaxf(mprev, valid ? pre_x : mprev);
+                const float gt = valid ? expf(mprev - run) : 0.f;     // = e^{b_t + m_prev - m_t}
+                const float wn = valid ? expf(u + cs.x - mnext) * inv_sqrt_d : 0.f;
+                const float wl = valid ? expf(u + cs.x - mnext + tab.lnupd[c]) * inv_sqrt_d : 0.f;
+                fm[64 * pb + t] = b + run;
+                fg[64 * pb + t] = gt;
+                fF[64 * pb + t] = wide ? 1.f : gt * tab.lamret[c];
+                fw[64 * pb + t] = wl;
+                fpw[t] = wn;
+                fu[64 * pb + t] = u;
+                frun[64 * pb + t] = run;
+            }
+            pre_b = pre_i = pre_x = 0.f;
+            if (c + 1 < nch) {
+                pre_cs = cstat[(size_t)bh * nchunks + c0 + c + 1];
+                if (ct < kL && t0 + kL + ct < S) {
+                    pre_b = bcum[tok0 + t0 + kL + ct];
+                    pre_i = i_pre[tok0 + t0 + kL + ct];
+                    pre_x = pmx[tok0 + t0 + kL + ct];
+                }
+            }
+            sync_ops();
+            if (ct == 0) mbar_arrive(&bars[B_GATES_READY0 + pb]);
+            TC_TRACE(ct == 0, c, 1);
+            // (3) Q as fp32 (K-major, tf32 operand of the retrieval); lanes take rows so a
+            // warp's 16-byte stores land on distinct bank groups
+            if (!wait_ops(&bars[B_FULL_Q], c & 1, abort_flag, status)) { ok = false; break; }
+            if (c >= 1 && !wait_ops(&bars[B_QT_FREE], (c - 1) & 1, abort_flag, status)) { ok = false; break; }
+            TC_TRACE(ct == 0, c, 2);
+            if (!wide) {
+#pragma unroll 4
+                for (int e = ct; e < kL * (D / 8); e += 128) {
+                    const int t = e & 63, ch = e >> 6;
+                    const int jb = ch >> 3, cc = ch & 7;
+                    const uint4 src = *reinterpret_cast<const uint4 *>(sQ + jb * 8192 + sw128_offset(t, cc));
+                    const int blk = 2 * jb + (cc >> 2), cd = (cc & 3) * 2;
+                    uint8_t *dst = sQt + blk * 8192;
+                    *reinterpret_cast<float4 *>(dst + sw128_offset(t, cd)) =
+                        make_float4(bf16_lo(src.x), bf16_hi(src.x), bf16_lo(src.y), bf16_hi(src.y));
+                    *reinterpret_cast<float4 *>(dst + sw128_offset(t, cd + 1)) =
+                        make_float4(bf16_lo(src.z), bf16_hi(src.z), bf16_lo(src.w), bf16_hi(src.w));
+                }
+            } else {     // wide chunk: the retrieval operand is g_t q_t
+                for (int e = ct; e < kL * (D / 8); e += 128) {
+                    const int t = e & 63, ch = e >> 6;
+                    const int jb = ch >> 3, cc = ch & 7;
+                    const uint4 src = *reinterpret_cast<const uint4 *>(sQ + jb * 8192 + sw128_offset(t, cc));
+                    const int blk = 2 * jb + (cc >> 2), cd = (cc & 3) * 2;
+                    const float gq = fg[64 * pb + t];
+                    uint8_t *dst = sQt + blk * 8192;
+                    *reinterpret_cast<float4 *>(dst + sw128_offset(t, cd)) =
+                        make_float4(gq * bf16_lo(src.x), gq * bf16_hi(src.x), gq * bf16_lo(src.y), gq * bf16_hi(src.y));
+                    *reinterpret_cast<float4 *>(dst + sw128_offset(t, cd + 1)) =
+                        make_float4(gq * bf16_lo(src.z), gq * bf16_hi(src.z), gq * bf16_lo(src.w), gq * bf16_hi(src.w));
+                }
+            }
+            fence_async_smem();
+            sync_ops();
+            if (ct == 0) {
+                mbar_arrive(&bars[B_QT_READY]);
+                mbar_arrive(&bars[B_Q_FREE]);
+            }
+            TC_TRACE(ct == 0, c, 3);
+            // (4) normaliser chain n'_c = a n'_{c-1} + sum_s w_s k^_s, into the next key slot
+            {
+                const int slot = c & 1;
+                if (!wait_ops(&bars[B_FULL_K0 + slot], (c >> 1) & 1, abort_flag, status)) { ok = false; break; }
+                TC_TRACE(ct == 0, c, 4);
+                const float a = expf(cs.x + mprev - mnext);
+                const uint8_t *kt = sK + slot * Lay::kKslot;
+                if (D == 256) {      // this thread's pair of key columns j = 2 ct, 2 ct + 1
+                    const int j = 2 * ct;
+                    const uint8_t *blkp = kt + (j / 64) * kKBlock;
+                    const int cc = (j % 64) / 8, within = (j % 8) * 2;
+                    float a0 = 0.f, a1 = 0.f;
+#pragma unroll 8
+                    for (int s = 0; s < kL; ++s) {
+                        const uint32_t kv = *reinterpret_cast<const uint32_t *>(blkp + sw128_offset(s, cc) + within);
+                        const float w = fpw[s];
+                        a0 += w * bf16_lo(kv);
+                        a1 += w * bf16_hi(kv);
+                    }
+                    nreg[0] = a * nreg[0] + a0;
+                    nreg[1] = a * nreg[1] + a1;
+                } else {
+                    const int j = ct;
+                    const uint8_t *blkp = kt + (j / 64) * kKBlock;
+                    const int cc = (j % 64) / 8, within = (j % 8) * 2;
+                    float acc = 0.f;
+#pragma unroll 8
+                    for (int s = 0; s < kL; ++s)
+                        acc += fpw[s] * __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(
+                                            blkp + sw128_offset(s, cc) + within));
+                    nreg[0] = a * nreg[0] + acc;
+                }
+                if (c + 1 < nch) {
+                    const int ns = (c + 1) & 1;
+                    if (c >= 1 && !wait_ops(&bars[B_K_FREE0 + ns], ((c - 1) >> 1) & 1, abort_flag, status)) { ok = false; break; }
+                    uint8_t *nt = sK + ns * Lay::kKslot;
+#pragma unroll
+                    for (int r = 0; r < D / 128; ++r) {
+                        const int j = nj(r);
+                        uint8_t *blkp = nt + (j / 64) * kKBlock;
+                        const int cc = (j % 64) / 8, within = (j % 8) * 2;
+                        const float hi = __bfloat162float(__float2bfloat16_rn(nreg[r]));
+                        *reinterpret_cast<__nv_bfloat16 *>(blkp + sw128_offset(64, cc) + within) = __float2bfloat16_rn(hi);
+                        *reinterpret_cast<__nv_bfloat16 *>(blkp + sw128_offset(65, cc) + within) =
+                            __float2bfloat16_rn(nreg[r] - hi);
+                    }
+                    fence_async_smem();
+                    sync_ops();
+                    if (ct == 0) mbar_arrive(&bars[B_NROW_READY0 + ns]);
+                }
+            }
+            TC_TRACE(ct == 0, c, 5);
+            // (5) V scaled in place by w^ (the operand of both the update and the intra term)
+            if (!wait_ops(&bars[B_FULL_V], c & 1, abort_flag, status)) { ok = false; break; }
+            if (wide) {      // the intra-chunk MMA reads V unscaled first
+                if (!wait_ops(&bars[B_INTRA_DONE], nwide & 1, abort_flag, status)) { ok = false; break; }
+                ++nwide;
+            }
+            TC_TRACE(ct == 0, c, 6);
+            {
+                const float *wv = fw + 64 * pb;
+#pragma unroll 4
+                for (int e = ct; e < 2 * kL * 8; e += 128) {       // (block, row s, chunk)
+                    const int blk = e / (kL * 8), s = (e / 8) % kL, cc = e & 7;
+                    uint4 *p = reinterpret_cast<uint4 *>(sV + blk * 8192 + sw128_offset(s, cc));
+                    const uint4 src = *p;
+                    const float w = wv[s];
+                    uint4 dst;
+                    dst.x = pack_bf16x2(bf16_lo(src.x) * w, bf16_hi(src.x) * w);
+                    dst.y = pack_bf16x2(bf16_lo(src.y) * w, bf16_hi(src.y) * w);
+                    dst.z = pack_bf16x2(bf16_lo(src.z) * w, bf16_hi(src.z) * w);
+                    dst.w = pack_bf16x2(bf16_lo(src.w) * w, bf16_hi(src.w) * w);
+                    *p = dst;
+                }
+            }
+            fence_async_smem();
+            sync_ops();
+            if (ct == 0) mbar_arrive(&bars[B_VHAT_READY]);
+            TC_TRACE(ct == 0, c, 7);
+        }
+        // final state (last segment only): Lambda * Cs, n', m
+        if (ok && g == P - 1 && nch > 0) {
+            if (wait_ops(&bars[B_DONE], 0, abort_flag, status)) {
+                __syncwarp();
+                tc_fence_after();
+                const int cl = nch - 1;
+                const float2 cs = cstat[(size_t)bh * nchunks + c0 + cl];
+                const float mn = cs.x + fmaxf(tab.mprev[cl], cs.y);
+                const float lam_last = expf(-tab.lnupd[cl]);
+                if (C_out) {
+                    const int i = 32 * q4 + lane;
+                    for (int jb = 0; jb < D; jb += 16) {
+                        uint32_t r[16];
+                        tmem_ld16(t_state + lane_addr + jb, r);
+                        tmem_wait_ld();
+                        float4 *dst = reinterpret_cast<float4 *>(C_out + ((size_t)bh * D + i0 + i) * D + jb);
+#pragma unroll
+                        for (int e = 0; e < 4; ++e)
+                            dst[e] = make_float4(__uint_as_float(r[4 * e]) * lam_last,
+                                                 __uint_as_float(r[4 * e + 1]) * lam_last,
+                                                 __uint_as_float(r[4 * e + 2]) * lam_last,
+                                                 __uint_as_float(r[4 * e + 3]) * lam_last);
+                    }
+                }
+                if (tile == 0) {
+                    if (n_out) {
+#pragma unroll
+                        for (int r = 0; r < D / 128; ++r) n_out[(size_t)bh * D + nj(r)] = nreg[r];
+                    }
+                    if (m_out && ct == 0) m_out[bh] = mn;
+                }
+            }
+        }
+        tc_fence_before();
+    } else if (is_sco) {
+        // ---------------------------------------------------------- score group
+        // Rows t = 16 q4 + (lane & 15) of S sit in TMEM lanes 0-15 of the warp's
+        // quadrant (M = 64 layout); lanes 16-31 take the same rows' upper 32
+        // columns via shuffles, so every lane masks 32 scores.
+        bool ok = true;
+        const int t = 16 * q4 + (lane & 15);
+        const int hh = lane >> 4;                             // column half of this lane
+        for (int c = 0; ok && c < nch; ++c) {
+            const int t0 = (c0 + c) * kL;
+            const int Lc = min(kL, S - t0);
+            const int pb = c & 1;
+            if (!wait_sco(&bars[B_GATES_READY0 + pb], (c >> 1) & 1, abort_flag, status) ||
+                !wait_sco(&bars[B_S_FULL], c & 1, abort_flag, status) ||
+                (c >= 1 && !wait_sco(&bars[B_P_FREE], (c - 1) & 1, abort_flag, status)) ||
+                (c >= 2 && !wait_sco(&bars[B_FINV_FREE0 + pb], ((c >> 1) - 1) & 1, abort_flag, status))) { ok = false; break; }
+            TC_TRACE(st_ == 0, c, 8);
+            __syncwarp();
+            tc_fence_after();
+            uint32_t sa[32], sb[32], sn[8];
+            tmem_ld16(t_S + lane_addr + 0, *reinterpret_cast<uint32_t(*)[16]>(&sa[0]));
+            tmem_ld16(t_S + lane_addr + 16, *reinterpret_cast<uint32_t(*)[16]>(&sa[16]));
+            tmem_ld16(t_S + lane_addr + 32, *reinterpret_cast<uint32_t(*)[16]>(&sb[0]));
+            tmem_ld16(t_S + lane_addr + 48, *reinterpret_cast<uint32_t(*)[16]>(&sb[16]));
+            tmem_ld8(t_S + lane_addr + 64, sn);
+            tmem_wait_ld();
+            TC_TRACE(st_ == 0, c, 16);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+                const uint32_t up = __shfl_sync(0xffffffffu, sb[e], lane & 15);
+                sa[e] = hh ? up : sa[e];
+            }
+            const bool valid = t < Lc;
+            float rowsum = 0.f;
+            if (tab.wide[c] != 0.f) {
+                // exact weights e^{u_s - (m_t - b_t)} / sqrt(d); exponents <= 0 for s <= t
+                const float rt = frun[64 * pb + t];
+                const float *us = fu + 64 * pb + 32 * hh;
+                for (int cq = 0; cq < 4; ++cq) {
+                    const int cc = 4 * hh + cq;
+                    uint32_t w4[4], l4[4];
+#pragma unroll
+                    for (int p2 = 0; p2 < 4; ++p2) {
+                        float pv[2];
+#pragma unroll
+                        for (int e = 0; e < 2; ++e) {
+                            const int sl = cq * 8 + p2 * 2 + e;
+                            const int s = 32 * hh + sl;
+                            pv[e] = (valid && s <= t) ? expf(us[sl] - rt) * inv_sqrt_d * __uint_as_float(sa[sl]) : 0.f;
+                            rowsum += pv[e];
+                        }
+                        w4[p2] = pack_bf16x2(pv[0], pv[1]);
+                        l4[p2] = pack_bf16x2(pv[0] - bf16_lo(w4[p2]), pv[1] - bf16_hi(w4[p2]));
+                    }
+                    *reinterpret_cast<uint4 *>(sP + sw128_offset(t, cc)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                    *reinterpret_cast<uint4 *>(sPl + sw128_offset(t, cc)) = make_uint4(l4[0], l4[1], l4[2], l4[3]);
+                }
+            } else {
+            const float4 *wv4 = reinterpret_cast<const float4 *>(fw + 64 * pb + 32 * hh);
+#pragma unroll
+            for (int cq = 0; cq < 4; ++cq) {
+                const int cc = 4 * hh + cq;
+                const float4 wa = wv4[2 * cq], wb = wv4[2 * cq + 1];
+                const float wk[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
+                uint32_t w4[4], l4[4];
+#pragma unroll
+                for (int p2 = 0; p2 < 4; ++p2) {
+                    float pv[2];
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const int sl = cq * 8 + p2 * 2 + e;
+                        const int s = 32 * hh + sl;
+                        const float sc = (valid && s <= t) ? __uint_as_float(sa[sl]) : 0.f;
+                        pv[e] = sc;
+                        rowsum += wk[p2 * 2 + e] * sc;
+                    }
+                    w4[p2] = pack_bf16x2(pv[0], pv[1]);
+                    l4[p2] = pack_bf16x2(pv[0] - bf16_lo(w4[p2]), pv[1] - bf16_hi(w4[p2]));
+                }
+                *reinterpret_cast<uint4 *>(sP + sw128_offset(t, cc)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                *reinterpret_cast<uint4 *>(sPl + sw128_offset(t, cc)) = make_uint4(l4[0], l4[1], l4[2], l4[3]);
+            }
+            }
+            TC_TRACE(st_ == 0, c, 17);
+            rowsum += __shfl_xor_sync(0xffffffffu, rowsum, 16);
+            if (hh == 0) {
+                // den = g_t (n'_prev . q_t) + F_t sum_s w^_s S_ts;  h_t = o_t F_t H~_t / max(|den|, e^-m_t)
+                const float nq = __uint_as_float(sn[0]) + __uint_as_float(sn[1]);
+                const float Ft = fF[64 * pb + t];
+                const float den = fg[64 * pb + t] * nq + Ft * rowsum;
+                finv[64 * pb + t] = valid ? Ft / fmaxf(fabsf(den), expf(-fm[64 * pb + t])) : 0.f;
+            }
+            TC_TRACE(st_ == 0, c, 18);
+            fence_async_smem();
+            TC_TRACE(st_ == 0, c, 19);
+            tc_fence_before();
+            sync_sco();
+            if (st_ == 0) {
+                mbar_arrive(&bars[B_P_READY]);
+                mbar_arrive(&bars[B_S_FREE]);
+                mbar_arrive(&bars[B_GATES_FREE0 + pb]);
+                mbar_arrive(&bars[B_FINV_READY0 + pb]);
+            }
+            TC_TRACE(st_ == 0, c, 9);
+        }
+    } else if (is_out) {
+        // --------------------------------------------------------- output group
+        // Thread = value row i of H^T (TMEM lane); h goes through a shared tile and
+        // leaves by TMA store, so the global writes are whole 128-byte rows.
+        bool ok = true;
+        const int i = 32 * q4 + lane;
+        uint8_t *hs = sHs + (i >> 6) * 8192 + (i & 63) * 2;
+        float og[32];                                         // output-gate pre-activations, in flight
+        if (nch > 0) {
+            const int Lc0 = min(kL, S - c0 * kL);
+#pragma unroll
+            for (int kk = 0; kk < 32; ++kk)
+                og[kk] = kk < Lc0 ? ldg_nc_early(o_pre + (tok0 + c0 * kL + kk) * D + i0 + i) : 0.f;
+        }
+        for (int c = 0; ok && c < nch; ++c) {
+            const int hb = c & 1;
+            const int t0 = (c0 + c) * kL;
+            const int Lc = min(kL, S - t0);
+            if (!wait_out(&bars[B_H_FULL0 + hb], (c >> 1) & 1, abort_flag, status) ||
+                !wait_out(&bars[B_FINV_READY0 + hb], (c >> 1) & 1, abort_flag, status)) { ok = false; break; }
+            TC_TRACE(xt == 0, c, 10);
+            if (xt == 0) bulk_wait_read_all();               // the previous tile has left the buffer
+            sync_out();
+            __syncwarp();
+            tc_fence_after();
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {            // tokens [32 half, 32 half + 32)
+                uint32_t r[32];
+                tmem_ld16(t_H0 + 64 * hb + lane_addr + 32 * half, *reinterpret_cast<uint32_t(*)[16]>(&r[0]));
+                tmem_ld16(t_H0 + 64 * hb + lane_addr + 32 * half + 16, *reinterpret_cast<uint32_t(*)[16]>(&r[16]));
+                tmem_wait_ld();
+                TC_TRACE(xt == 0, c, 20 + 2 * half);
+                float ogn[32];                                // the next pass's gates, in flight
+                const int tn0 = half == 0 ? t0 + 32 : t0 + kL;
+                const int ln = half == 0 ? Lc - 32 : (c + 1 < nch ? min(kL, S - t0 - kL) : 0);
+#pragma unroll
+                for (int kk = 0; kk < 32; ++kk)
+                    ogn[kk] = kk < ln ? ldg_nc_early(o_pre + (tok0 + tn0 + kk) * D + i0 + i) : 0.f;
+                const float *inv = finv + 64 * hb + 32 * half;
+#pragma unroll
+                for (int kk = 0; kk < 32; ++kk) {
+                    const float o = __fdividef(1.f, 1.f + __expf(-og[kk]));
+                    *reinterpret_cast<__nv_bfloat16 *>(hs + (32 * half + kk) * 128) =
+                        __float2bfloat16_rn(o * __uint_as_float(r[kk]) * inv[kk]);
+                }
+                TC_TRACE(xt == 0, c, 21 + 2 * half);
+#pragma unroll
+                for (int kk = 0; kk < 32; ++kk) og[kk] = ogn[kk];
+            }
+            fence_async_smem();
+            tc_fence_before();
+            sync_out();
+            if (xt == 0) {
+                tma_store_3d(&map_h, sHs, i0, t0, bh);
+                tma_store_3d(&map_h, sHs + 8192, i0 + 64, t0, bh);
+                bulk_commit();
+                mbar_arrive(&bars[B_H_FREE0 + hb]);
+                mbar_arrive(&bars[B_FINV_FREE0 + hb]);
+            }
+            TC_TRACE(xt == 0, c, 11);
+        }
+        if (xt == 0) bulk_wait_all();                        // h is in global memory before exit
+        tc_fence_before();
+    }
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tbase, 512);
+        tmem_relinquish();
+    }
+}
+
+// ------------------------------------------------------------ segment summaries
+// Per (value tile, segment g < P-1, head): dC = sum_s w_s v_s k^_s^T over the
+// segment, w_s = e^{u_s + E_c - mloc} / sqrt(d) (all exponents <= 0), on the
+// tensor cores with the accumulator in TMEM; dn likewise (tile 0, CUDA cores).
+template <int D>
+struct SumLayout {
+    static constexpr int kKslot = (D / 64) * 8192;        // K bf16 MN-major view: D/64 blocks x 64 rows
+    static constexpr int kSlot = kKslot + 16384;          // + V (2 blocks x 8 KB)
+    static constexpr int kVh = 2 * kSlot;                 // 2 x 16 KB scaled V
+    static constexpr int kF = kVh + 2 * 16384;            // w[2][64]
+    static constexpr int kTab = kF + 2 * 64 * 4;          // E per chunk
+    static constexpr int kBar = kTab + kMaxCps * 4;
+    static constexpr int kMisc = kBar + 8 * 8;
+    static constexpr int kBytes = kMisc + 16 + 1024;
+};
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+segment_summary_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v,
+                          const float *__restrict__ i_pre, const float *__restrict__ bcum,
+                          const float2 *__restrict__ cstat, float2 *__restrict__ sstat, float *__restrict__ summ,
+                          unsigned int *status, int S, int nchunks, int P, int cps) {
+    using Lay = SumLayout<D>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = align1024(smem_raw);
+    float *fw = reinterpret_cast<float *>(smem + Lay::kF);
+    float *tabE = reinterpret_cast<float *>(smem + Lay::kTab);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Lay::kBar);   // full[2], free[2], vh_ready[2], done
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + Lay::kMisc);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + Lay::kMisc + 4);
+    __shared__ float s_mloc, s_etot;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int tile = blockIdx.x, g = blockIdx.y, bh = blockIdx.z;
+    const int i0 = tile * kRows;
+    const int c0 = g * cps;
+    const int nch = min(nchunks, c0 + cps) - c0;
+    const size_t tok0 = (size_t)bh * S;
+    const float inv_sqrt_d = rsqrtf((float)D);
+
+    if (tid == 0) {
+        for (int i = 0; i < 7; ++i) mbar_init(&bars[i], 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+        // segment statistics: E_c = sum_{c' >= c} btot, mloc = max_c (cmax_c + E_c)
+        float E = 0.f, mloc = -INFINITY;
+        for (int c = nch - 1; c >= 0; --c) {
+            const float2 cs = cstat[(size_t)bh * nchunks + c0 + c];
+            E += cs.x;
+            tabE[c] = E;
+            mloc = fmaxf(mloc, cs.y + E);
+        }
+        s_mloc = mloc;
+        s_etot = E;
+        if (tile == 0) sstat[(size_t)bh * P + g] = make_float2(E, mloc);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, 256);
+        tc_fence_before();
+    }
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tacc = *tmem_slot;
+    const float mloc = s_mloc;
+    const uint32_t idesc_U = idesc_f32acc(kFmtBF16, kFmtBF16, true, true, 128, D);
+
+    if (warp == 0) {
+        if (lane == 0) {
+            tma_prefetch_desc(&map_k);
+            tma_prefetch_desc(&map_v);
+            int issued[2] = {0, 0};
+            for (int c = 0; c < nch; ++c) {
+                const int slot = c & 1, t0 = (c0 + c) * kL;
+                if (c >= 2 && !mbar_wait(&bars[2 + slot], ((c >> 1) - 1) & 1, abort_flag, status)) break;
+                uint8_t *base = smem + slot * Lay::kSlot;
+                mbar_arrive_expect_tx(&bars[slot], kL * D * 2 + kL * kRows * 2);
+                for (int jb = 0; jb < D / 64; ++jb) tma_load_3d(base + jb * 8192, &map_k, &bars[slot], jb * 64, t0, bh);
+                for (int b = 0; b < 2; ++b)
+                    tma_load_3d(base + Lay::kKslot + b * 8192, &map_v, &bars[slot], i0 + 64 * b, t0, bh);
+                ++issued[slot];
+            }
+            for (int s = 0; s < 2; ++s)
+                if (issued[s]) mbar_wait(&bars[s], (issued[s] - 1) & 1, nullptr, status);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            for (int c = 0; c < nch; ++c) {
+                const int slot = c & 1;
+                if (!mbar_wait(&bars[4 + slot], (c >> 1) & 1, abort_flag, status)) break;
+                tc_fence_after();
+                const uint32_t vha = smem_u32(smem + Lay::kVh + slot * 16384);
+                const uint32_t ka = smem_u32(smem + slot * Lay::kSlot);
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_bf16_ss(tacc, sdesc_sw128(vha + ks * 2048, 8192, 1024),
+                                sdesc_sw128(ka + ks * 2048, 8192, 1024), idesc_U, (c > 0 || ks > 0) ? 1u : 0u);
+                mma_commit(&bars[2 + slot]);
+            }
+            mma_commit(&bars[6]);
+            mbar_wait(&bars[6], 0, nullptr, status);
+        }
+    } else {
+        const int ct = tid - 64, q4 = warp & 3;
+        float nacc[D / 128];
+#pragma unroll
+        for (int r = 0; r < D / 128; ++r) nacc[r] = 0.f;
+        bool ok = true;
+        for (int c = 0; c < nch; ++c) {
+            const int slot = c & 1, t0 = (c0 + c) * kL, Lc = min(kL, S - t0);
+            if (ct < kL) {
+                const int t = ct;
+                fw[64 * slot + t] = t < Lc
+                    ? expf(i_pre[tok0 + t0 + t] - bcum[tok0 + t0 + t] + tabE[c] - mloc) * inv_sqrt_d : 0.f;
+            }
+            if (!compute_wait(&bars[slot], (c >> 1) & 1, abort_flag, status)) { ok = false; break; }
+            named_sync_compute();
+            const uint8_t *base = smem + slot * Lay::kSlot;
+            const uint8_t *sV = base + Lay::kKslot;
+            uint8_t *sVh = smem + Lay::kVh + slot * 16384;
+            const float *w = fw + 64 * slot;
+            for (int e = ct; e < 2 * kL * 8; e += 128) {
+                const int blk = e / (kL * 8), s = (e / 8) % kL, cc = e & 7;
+                const uint32_t off = blk * 8192 + sw128_offset(s, cc);
+                const uint4 src = *reinterpret_cast<const uint4 *>(sV + off);
+                const float ws = w[s];
+                uint4 dst;
+                dst.x = pack_bf16x2(bf16_lo(src.x) * ws, bf16_hi(src.x) * ws);
+                dst.y = pack_bf16x2(bf16_lo(src.y) * ws, bf16_hi(src.y) * ws);
+                dst.z = pack_bf16x2(bf16_lo(src.z) * ws, bf16_hi(src.z) * ws);
+                dst.w = pack_bf16x2(bf16_lo(src.w) * ws, bf16_hi(src.w) * ws);
+                *reinterpret_cast<uint4 *>(sVh + off) = dst;
+            }
+            if (tile == 0) {
+#pragma unroll
+                for (int r = 0; r < D / 128; ++r) {
+                    const int j = ct + 128 * r;
+                    const uint8_t *blkp = base + (j / 64) * 8192;
+                    const int cc = (j % 64) / 8, within = (j % 8) * 2;
+                    float acc = 0.f;
+                    for (int s = 0; s < kL; ++s)
+                        acc += w[s] * __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(
+                                          blkp + sw128_offset(s, cc) + within));
+                    nacc[r] += acc;
+                }
+            }
+            fence_async_smem();
+            named_sync_compute();
+            if (ct == 0) mbar_arrive(&bars[4 + slot]);
+        }
+        if (ok && compute_wait(&bars[6], 0, abort_flag, status)) {
+            __syncwarp();
+            tc_fence_after();
+            float *out = summ + ((size_t)bh * (P - 1) + g) * ((size_t)D * D + D);
+            const int i = 32 * q4 + lane;
+            const uint32_t lane_addr = ((uint32_t)(32 * q4)) << 16;
+            for (int jb = 0; jb < D; jb += 16) {
+                uint32_t r[16];
+                tmem_ld16(tacc + lane_addr + jb, r);
+                tmem_wait_ld();
+                float4 *dst = reinterpret_cast<float4 *>(out + (size_t)(i0 + i) * D + jb);
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    dst[e] = make_float4(__uint_as_float(r[4 * e]), __uint_as_float(r[4 * e + 1]),
+                                         __uint_as_float(r[4 * e + 2]), __uint_as_float(r[4 * e + 3]));
+            }
+            if (tile == 0) {
+#pragma unroll
+                for (int r = 0; r < D / 128; ++r) out[(size_t)D * D + ct + 128 * r] = nacc[r];
+            }
+        }
+        tc_fence_before();
+    }
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tacc, 256);
+        tmem_relinquish();
+    }
+}
+
+// ------------------------------------------------------------------- host
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *,
+                                  CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static std::once_flag once;
+    static EncodeTiledFn fn = nullptr;
+    std::call_once(once, [] {
+        cudaDriverEntryPointQueryResult q;
+        void *p = nullptr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// [BH, S, D] bf16, box 64 x 64 x 1; loads use the 128-byte swizzle (rows past S
+// read as zeros), the h store map no swizzle (rows past S are not written).
+bool make_map(CUtensorMap *m, const void *base, int BH, int S, int D, bool swizzle = true) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)S, (cuuint64_t)BH};
+    cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)S * D * 2};
+    cuuint32_t box[3] = {64, 64, 1};
+    cuuint32_t es[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D>
+cudaError_t launch_tc_t(const FwdArgs &a, const FwdPlan &p, cudaStream_t st) {
+    CUtensorMap mq, mk, mv, mh;
+    if (!make_map(&mq, a.q, p.BH, p.S, D) || !make_map(&mk, a.k, p.BH, p.S, D) ||
+        !make_map(&mv, a.v, p.BH, p.S, D) || !make_map(&mh, a.h, p.BH, p.S, D, false))
+        return cudaErrorInvalidValue;
+    float *ws = (float *)a.workspace;
+    const float *bcum = ws + p.off_bcum;
+    const float2 *cstat = (const float2 *)(ws + p.off_cstat);
+    float2 *sstat = (float2 *)(ws + p.off_sstat);
+    float *summ = ws + p.off_summ;
+    cudaError_t e;
+    if (p.P > 1) {
+        const int sm = SumLayout<D>::kBytes;
+        e = cudaFuncSetAttribute(segment_summary_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
+        if (e != cudaSuccess) return e;
+        KernelTimer timer("segment_summary_tc", st);
+        segment_summary_tc_kernel<D><<<dim3(D / kRows, p.P - 1, p.BH), kThreads, sm, st>>>(
+            mk, mv, a.i_pre, bcum, cstat, sstat, summ, a.status, p.S, p.nchunks, p.P, p.cps);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    const int sm = OutLayout<D>::kBytes;
+    e = cudaFuncSetAttribute(segment_output_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
+    if (e != cudaSuccess) return e;
+    KernelTimer timer("segment_output_tc", st);
+    segment_output_tc_kernel<D><<<dim3(D / kRows, p.P, p.BH), kOutThreads, sm, st>>>(
+        mq, mk, mv, mh, a.i_pre, a.o_pre, a.C0, a.n0, a.m0, a.C_out, a.n_out, a.m_out,
+        bcum, ws + p.off_pmax, cstat, sstat, summ, a.status, p.S, p.nchunks, p.P, p.cps);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+bool tensor_path_supports(int DH, int L) { return L == kL && (DH == 128 || DH == 256); }
+
+#ifdef XLSTM_TC_TRACE
+extern "C" int xlstm_debug_set_trace(void *buf) {
+    return cudaMemcpyToSymbol(g_tc_trace, &buf, sizeof(buf)) == cudaSuccess ? 0 : 1;
+}
+#endif
+
+int tensor_path_max_chunks_per_segment() { return kMaxCps; }
 
 cudaError_t launch_fwd_tensor(const FwdArgs &a, const FwdPlan &p, cudaStream_t st) {
-    (void)a; (void)p; (void)st;
-    return cudaErrorNotSupported;
+    if (!a.bf16 || !tensor_path_supports(p.DH, p.L) || p.cps > kMaxCps) return cudaErrorInvalidValue;
+    cudaError_t e = launch_gate_prologue(a, p, st);
+    if (e != cudaSuccess) return e;
+    if (p.DH == 128) return launch_tc_t<128>(a, p, st);
+    return launch_tc_t<256>(a, p, st);
 }
 
 }  // namespace xlstm

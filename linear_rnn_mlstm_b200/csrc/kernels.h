@@ -34,6 +34,7 @@ cudaError_t launch_gate_prologue(const FwdArgs &a, const FwdPlan &p, cudaStream_
 cudaError_t launch_fwd_simt(const FwdArgs &a, const FwdPlan &p, cudaStream_t st);
 cudaError_t launch_fwd_tensor(const FwdArgs &a, const FwdPlan &p, cudaStream_t st);
 bool tensor_path_supports(int DH, int L);
+int tensor_path_max_chunks_per_segment();
 cudaError_t launch_state_passthrough(const FwdArgs &a, int BH, int DH, cudaStream_t st);
 cudaError_t launch_step(const StepArgs &a, cudaStream_t st);
 

@@ -30,6 +30,7 @@ struct FwdPlan {
     int ntiles;               // ceil(DH / rows)
     // workspace layout, in floats from the workspace base
     size_t off_bcum;          // [BH, S]        chunk-local inclusive cumsum of log f
+    size_t off_pmax;          // [BH, S]        chunk-local inclusive prefix max of log i - b
     size_t off_cstat;         // [BH, nchunks, 2]  (chunk total of log f, chunk max of log i - b)
     size_t off_sstat;         // [BH, P, 2]     (segment total of log f, segment stabiliser)
     size_t off_summ;          // [BH, P-1, DH*DH + DH]  segment summaries (C part then n part)
