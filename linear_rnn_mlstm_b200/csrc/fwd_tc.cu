@@ -238,45 +238,35 @@ segment_output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
     const uint32_t t_H0 = tbase + 384;             // columns [384, 448) and [448, 512)
 
     if (is_ops) {
-        // Incoming state: the initial state folded with the summaries of segments < g.
+        // Incoming state: the initial state for segment 0, else the state at the end
+        // of segment g - 1, which segment_scan_kernel left in summary slot g - 1.
         const float m_init = m0 ? m0[bh] : 0.f;
         const int i = 32 * q4 + lane;
+        const float *src = g == 0 ? (C0 ? C0 + (size_t)bh * D * D : nullptr)
+                                  : summ + ((size_t)bh * (P - 1) + g - 1) * ((size_t)D * D + D);
+        const float *nsrc = g == 0 ? (n0 ? n0 + (size_t)bh * D : nullptr) : src + (size_t)D * D;
+#pragma unroll 4
         for (int jb = 0; jb < D; jb += 16) {
-            float v[16];
-            const float *c0row = C0 ? C0 + ((size_t)bh * D + i0 + i) * D + jb : nullptr;
-#pragma unroll
-            for (int e = 0; e < 16; ++e) v[e] = c0row ? c0row[e] : 0.f;
-            float mc = m_init;
-            for (int gp = 0; gp < g; ++gp) {
-                const float2 st = sstat[(size_t)bh * P + gp];
-                const float mn = fmaxf(st.x + mc, st.y);
-                const float al = expf(st.x + mc - mn), be = expf(st.y - mn);
-                const float *sm = summ + ((size_t)bh * (P - 1) + gp) * ((size_t)D * D + D) +
-                                  (size_t)(i0 + i) * D + jb;
-#pragma unroll
-                for (int e = 0; e < 16; ++e) v[e] = al * v[e] + be * sm[e];
-                mc = mn;
-            }
             uint32_t r[16];
+            if (src) {
+                const float4 *row = reinterpret_cast<const float4 *>(src + (size_t)(i0 + i) * D + jb);
 #pragma unroll
-            for (int e = 0; e < 16; ++e) r[e] = __float_as_uint(v[e]);
+                for (int e = 0; e < 4; ++e) {
+                    const float4 x = row[e];
+                    r[4 * e] = __float_as_uint(x.x);
+                    r[4 * e + 1] = __float_as_uint(x.y);
+                    r[4 * e + 2] = __float_as_uint(x.z);
+                    r[4 * e + 3] = __float_as_uint(x.w);
+                }
+            } else {
+#pragma unroll
+                for (int e = 0; e < 16; ++e) r[e] = 0u;
+            }
             tmem_st16(t_state + lane_addr + jb, r);
         }
         tmem_wait_st();
 #pragma unroll
-        for (int r = 0; r < D / 128; ++r) {
-            const int j = nj(r);
-            float nv = n0 ? n0[(size_t)bh * D + j] : 0.f;
-            float mc = m_init;
-            for (int gp = 0; gp < g; ++gp) {
-                const float2 st = sstat[(size_t)bh * P + gp];
-                const float mn = fmaxf(st.x + mc, st.y);
-                const float al = expf(st.x + mc - mn), be = expf(st.y - mn);
-                nv = al * nv + be * summ[((size_t)bh * (P - 1) + gp) * ((size_t)D * D + D) + (size_t)D * D + j];
-                mc = mn;
-            }
-            nreg[r] = nv;
-        }
+        for (int r = 0; r < D / 128; ++r) nreg[r] = nsrc ? nsrc[nj(r)] : 0.f;
         // zero the extra key rows 64..71 of both slots, then n'_in (hi, lo) in slot 0
         for (int e = ct; e < 2 * (D / 64) * 8 * 8; e += 128) {      // (slot, block, row, chunk)
             const int ch = e & 7, row = 64 + ((e >> 3) & 7), blk = (e >> 6) % (D / 64), slot = e / (64 * (D / 64));
@@ -837,6 +827,15 @@ segment_output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
 #pragma unroll
                 for (int kk = 0; kk < 32; ++kk)
                     ogn[kk] = kk < ln ? ldg_nc_early(o_pre + (tok0 + tn0 + kk) * D + i0 + i) : 0.f;
+#ifdef XLSTM_TC_TRACE
+                if (g_tc_trace) {                             // time at which this pass's gates have arrived
+                    float acc = 0.f;
+#pragma unroll
+                    for (int kk = 0; kk < 32; ++kk) acc += og[kk];
+                    if (acc == 1.2345e-30f) og[0] += 1.f;
+                    TC_TRACE(xt == 0, c, 24 + half);
+                }
+#endif
                 const float *inv = finv + 64 * hb + 32 * half;
 #pragma unroll
                 for (int kk = 0; kk < 32; ++kk) {
@@ -868,6 +867,46 @@ segment_output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
         tc_fence_after();
         tmem_dealloc(tbase, 512);
         tmem_relinquish();
+    }
+}
+
+// ------------------------------------------------------------ segment scan
+// Turns the segment summaries into incoming states, in place: slot g of the
+// summary buffer becomes the state (C', n') at the end of segment g, i.e. the
+// incoming state of segment g + 1:
+//   X_g = e^{F_g + M_{g-1} - M_g} X_{g-1} + e^{mloc_g - M_g} dX_g,
+//   M_g = max(F_g + M_{g-1}, mloc_g),  X_{-1} = initial state,  M_{-1} = m_0,
+// with (F_g, mloc_g) the segment's total log forget and own stabiliser.  One
+// thread per 4 consecutive floats of a head's (C', n'), all segments in order.
+__global__ void __launch_bounds__(256)
+segment_scan_kernel(const float2 *__restrict__ sstat, float *__restrict__ summ, const float *__restrict__ C0,
+                    const float *__restrict__ n0, const float *__restrict__ m0, int D, int P) {
+    const int bh = blockIdx.y;
+    const size_t per = (size_t)D * D + D;
+    const size_t e4 = ((size_t)blockIdx.x * blockDim.x + threadIdx.x) * 4;
+    if (e4 >= per) return;
+    float x[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        const size_t idx = e4 + e;
+        x[e] = idx < (size_t)D * D ? (C0 ? C0[(size_t)bh * D * D + idx] : 0.f)
+                                   : (n0 ? n0[(size_t)bh * D + idx - (size_t)D * D] : 0.f);
+    }
+    float mc = m0 ? m0[bh] : 0.f;
+    float4 *slot = reinterpret_cast<float4 *>(summ + (size_t)bh * (P - 1) * per + e4);
+    const size_t stride4 = per / 4;
+#pragma unroll 4
+    for (int g = 0; g < P - 1; ++g) {
+        const float2 st = sstat[(size_t)bh * P + g];
+        const float mn = fmaxf(st.x + mc, st.y);
+        const float al = expf(st.x + mc - mn), be = expf(st.y - mn);
+        const float4 d = slot[g * stride4];
+        x[0] = al * x[0] + be * d.x;
+        x[1] = al * x[1] + be * d.y;
+        x[2] = al * x[2] + be * d.z;
+        x[3] = al * x[3] + be * d.w;
+        slot[g * stride4] = make_float4(x[0], x[1], x[2], x[3]);
+        mc = mn;
     }
 }
 
@@ -1100,10 +1139,19 @@ cudaError_t launch_tc_t(const FwdArgs &a, const FwdPlan &p, cudaStream_t st) {
         const int sm = SumLayout<D>::kBytes;
         e = cudaFuncSetAttribute(segment_summary_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
         if (e != cudaSuccess) return e;
-        KernelTimer timer("segment_summary_tc", st);
-        segment_summary_tc_kernel<D><<<dim3(D / kRows, p.P - 1, p.BH), kThreads, sm, st>>>(
-            mk, mv, a.i_pre, bcum, cstat, sstat, summ, a.status, p.S, p.nchunks, p.P, p.cps);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        {
+            KernelTimer timer("segment_summary_tc", st);
+            segment_summary_tc_kernel<D><<<dim3(D / kRows, p.P - 1, p.BH), kThreads, sm, st>>>(
+                mk, mv, a.i_pre, bcum, cstat, sstat, summ, a.status, p.S, p.nchunks, p.P, p.cps);
+            if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        }
+        {
+            KernelTimer timer("segment_scan", st);
+            const size_t per4 = ((size_t)D * D + D) / 4;
+            segment_scan_kernel<<<dim3((unsigned)((per4 + 255) / 256), p.BH), 256, 0, st>>>(
+                sstat, summ, a.C0, a.n0, a.m0, D, p.P);
+            if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        }
     }
     const int sm = OutLayout<D>::kBytes;
     e = cudaFuncSetAttribute(segment_output_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
