@@ -58,7 +58,7 @@ __device__ unsigned long long *g_tc_trace = nullptr;
     do {                                                                                           \
         if (g_tc_trace && (cond)) {                                                                \
             const size_t cta_ = ((size_t)blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x; \
-            g_tc_trace[(cta_ * kMaxCps + (c)) * 32 + (slot)] = globaltimer_ns();                   \
+            g_tc_trace[(cta_ * kMaxCps + (c)) * 32 + (slot)] = clock64();                          \
         }                                                                                          \
     } while (0)
 #else
@@ -165,6 +165,7 @@ template <int D>
 __global__ void __launch_bounds__(kOutThreads, 1)
 segment_output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
                          const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_h,
+                         const __grid_constant__ CUtensorMap map_o,
                          const float *__restrict__ i_pre, const float *__restrict__ o_pre,
                          const float *__restrict__ C0, const float *__restrict__ n0, const float *__restrict__ m0,
                          float *__restrict__ C_out, float *__restrict__ n_out, float *__restrict__ m_out,
@@ -219,7 +220,11 @@ segment_output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
 
     // ------------------------------------------------------------ set-up
     if (tid == 0) {
-        for (int i = 0; i < B_NUM; ++i) mbar_init(&bars[i], i == B_Q_FREE ? 2 : 1);
+        for (int i = 0; i < B_NUM; ++i) {
+            const bool two = i == B_Q_FREE || i == B_H_FREE0 || i == B_H_FREE1 || i == B_FINV_FREE0 ||
+                             i == B_FINV_FREE1;
+            mbar_init(&bars[i], two ? 2 : 1);
+        }
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -283,19 +288,29 @@ segment_output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
             *reinterpret_cast<__nv_bfloat16 *>(blkp + sw128_offset(64, cc) + within) = __float2bfloat16_rn(hi);
             *reinterpret_cast<__nv_bfloat16 *>(blkp + sw128_offset(65, cc) + within) = __float2bfloat16_rn(nreg[r] - hi);
         }
-        if (ct == 0) {       // per-chunk tables
+        // per-chunk tables: the chunk statistics are staged in shared memory by all
+        // operand-group threads (one load each), then one thread scans them
+        for (int c = ct; c < nch; c += 128) {
+            const float2 cs = cstat[(size_t)bh * nchunks + c0 + c];
+            tab.mprev[c] = cs.x;
+            tab.lamret[c] = cs.y;
+        }
+        for (int gp = ct; gp < g; gp += 128) {
+            const float2 st = sstat[(size_t)bh * P + gp];
+            tab.resc[gp] = st.x;
+            tab.lnupd[gp] = st.y;
+        }
+        sync_ops();
+        if (ct == 0) {
             float mc = m_init;
-            for (int gp = 0; gp < g; ++gp) {
-                const float2 st = sstat[(size_t)bh * P + gp];
-                mc = fmaxf(st.x + mc, st.y);
-            }
+            for (int gp = 0; gp < g; ++gp) mc = fmaxf(tab.resc[gp] + mc, tab.lnupd[gp]);
             // ln Lambda stays in [-60, 0]: a chunk whose own decay of the stabilised
             // state, m_prev - max_s u_s, is below -60 is taken as -60.  That chunk
             // holds a term e^60 times heavier than the whole earlier state, so the
             // earlier state's share after it is below fp32 resolution either way.
             float lnlam = 0.f;
             for (int c = 0; c < nch; ++c) {
-                const float2 cs = cstat[(size_t)bh * nchunks + c0 + c];
+                const float2 cs = make_float2(tab.mprev[c], tab.lamret[c]);
                 const float mn = cs.x + fmaxf(mc, cs.y);
                 const float lna_true = cs.x + mc - mn;       // <= 0
                 const float lna = fmaxf(lna_true, kLnChunkFloor);
@@ -324,15 +339,72 @@ segment_output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
     const uint32_t idesc_I = idesc_f32acc(kFmtBF16, kFmtBF16, true, false, 128, 64);
     const uint32_t idesc_U = idesc_f32acc(kFmtBF16, kFmtBF16, true, true, 128, D);
 
+    // One epilogue pass: h for tokens [32 hq, 32 hq + 32) of chunk c, from the H~
+    // accumulator (thread = value row i = TMEM lane), the gates `og` of those
+    // tokens and the per-token factors F_t / (2 den_t), into the shared h tile.
+    // Taken by the output group (hq = 0) and the score group (hq = 1).
+    auto epilogue_pass = [&](int c, int hq, const float (&og)[32]) {
+        const int hb = c & 1;
+        const int i = 32 * q4 + lane;
+        uint8_t *hs = sHs + (i >> 6) * 8192 + (i & 63) * 2 + 32 * hq * 128;
+        uint32_t r[32];
+        tmem_ld16(t_H0 + 64 * hb + lane_addr + 32 * hq, *reinterpret_cast<uint32_t(*)[16]>(&r[0]));
+        tmem_ld16(t_H0 + 64 * hb + lane_addr + 32 * hq + 16, *reinterpret_cast<uint32_t(*)[16]>(&r[16]));
+        tmem_wait_ld();
+        const float *inv = finv + 64 * hb + 32 * hq;          // holds F_t / (2 den_t)
+#pragma unroll
+        for (int kk = 0; kk < 32; ++kk) {
+            // sigma(o) = (1 + tanh(o / 2)) / 2, the 1/2 folded into inv
+            const float hv = __uint_as_float(r[kk]) * inv[kk];
+            *reinterpret_cast<__nv_bfloat16 *>(hs + kk * 128) = __float2bfloat16_rn(fmaf(hv, tanh_approx(0.5f * og[kk]), hv));
+        }
+    };
+    // The gates of tokens [32 hq, 32 hq + 32) of chunk c, for this thread's value row.
+    auto load_gates = [&](int c, int hq, float (&og)[32]) {
+        const int i = 32 * q4 + lane;
+        const int tb = (c0 + c) * kL + 32 * hq;
+        const int n = min(32, S - tb);
+#pragma unroll
+        for (int kk = 0; kk < 32; ++kk)
+            og[kk] = kk < n ? ldg_nc_early(o_pre + (tok0 + tb + kk) * D + i0 + i) : 0.f;
+    };
+    // After a pass: the pass's half of the h tile leaves by TMA store (issued by
+    // the group's leader), and the group's share of H[hb] and finv[hb] is released.
+    auto finish_pass = [&](int c, int hq, bool leader) {
+        if (leader) {
+            const int t0 = (c0 + c) * kL;
+            tma_store_3d(&map_h, sHs + 32 * hq * 128, i0, t0 + 32 * hq, bh);
+            tma_store_3d(&map_h, sHs + 8192 + 32 * hq * 128, i0 + 64, t0 + 32 * hq, bh);
+            bulk_commit();
+            mbar_arrive(&bars[B_H_FREE0 + (c & 1)]);
+            mbar_arrive(&bars[B_FINV_FREE0 + (c & 1)]);
+        }
+    };
+
     if (warp == 0) {
         // ---------------------------------------------------------- TMA producer
         if (lane == 0) {
             tma_prefetch_desc(&map_q);
             tma_prefetch_desc(&map_k);
             tma_prefetch_desc(&map_v);
+            tma_prefetch_desc(&map_o);
+            // The operands of the chunk after next go to L2 ahead of their loads; the
+            // output gates, which the output group reads with plain loads, likewise.
+            auto prefetch = [&](int c) {
+                const int t0 = (c0 + c) * kL;
+                for (int jb = 0; jb < D / 64; ++jb) {
+                    tma_prefetch_l2_3d(&map_q, jb * 64, t0, bh);
+                    tma_prefetch_l2_3d(&map_k, jb * 64, t0, bh);
+                }
+                tma_prefetch_l2_3d(&map_v, i0, t0, bh);
+                tma_prefetch_l2_3d(&map_v, i0 + 64, t0, bh);
+                tma_prefetch_l2_3d(&map_o, i0, t0, bh);
+            };
+            for (int c = 0; c < min(nch, 2); ++c) prefetch(c);
             int issued_q = 0, issued_k[2] = {0, 0}, issued_v = 0;
             for (int c = 0; c < nch; ++c) {
                 const int t0 = (c0 + c) * kL;
+                if (c + 2 < nch) prefetch(c + 2);
                 if (c >= 1 && !mbar_wait(&bars[B_Q_FREE], (c - 1) & 1, abort_flag, status)) break;
                 mbar_arrive_expect_tx(&bars[B_FULL_Q], kL * D * 2);
                 for (int jb = 0; jb < D / 64; ++jb)
@@ -689,9 +761,28 @@ segment_output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
         // Rows t = 16 q4 + (lane & 15) of S sit in TMEM lanes 0-15 of the warp's
         // quadrant (M = 64 layout); lanes 16-31 take the same rows' upper 32
         // columns via shuffles, so every lane masks 32 scores.
+        // After the scores of chunk c it writes h for tokens 32-63 of chunk c - 1.
         bool ok = true;
         const int t = 16 * q4 + (lane & 15);
         const int hh = lane >> 4;                             // column half of this lane
+        float og[32];                                         // gates of the pending epilogue pass
+        if (nch > 0) load_gates(0, 1, og);
+        auto pass1 = [&](int cp) -> bool {                    // epilogue of tokens 32-63 of chunk cp
+            if (!wait_sco(&bars[B_H_FULL0 + (cp & 1)], (cp >> 1) & 1, abort_flag, status)) return false;
+            if (st_ == 0) bulk_wait_read_all();               // this half of the h tile is free again
+            sync_sco();
+            __syncwarp();
+            tc_fence_after();
+            TC_TRACE(st_ == 0, cp, 22);
+            epilogue_pass(cp, 1, og);
+            TC_TRACE(st_ == 0, cp, 23);
+            if (cp + 1 < nch) load_gates(cp + 1, 1, og);
+            fence_async_smem();
+            tc_fence_before();
+            sync_sco();
+            finish_pass(cp, 1, st_ == 0);
+            return true;
+        };
         for (int c = 0; ok && c < nch; ++c) {
             const int t0 = (c0 + c) * kL;
             const int Lc = min(kL, S - t0);
@@ -774,7 +865,7 @@ segment_output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
                 const float nq = __uint_as_float(sn[0]) + __uint_as_float(sn[1]);
                 const float Ft = fF[64 * pb + t];
                 const float den = fg[64 * pb + t] * nq + Ft * rowsum;
-                finv[64 * pb + t] = valid ? Ft / fmaxf(fabsf(den), expf(-fm[64 * pb + t])) : 0.f;
+                finv[64 * pb + t] = valid ? 0.5f * Ft / fmaxf(fabsf(den), expf(-fm[64 * pb + t])) : 0.f;
             }
             TC_TRACE(st_ == 0, c, 18);
             fence_async_smem();
@@ -788,75 +879,35 @@ segment_output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
                 mbar_arrive(&bars[B_FINV_READY0 + pb]);
             }
             TC_TRACE(st_ == 0, c, 9);
+            if (c >= 1 && !pass1(c - 1)) { ok = false; break; }
         }
+        if (ok && nch > 0) ok = pass1(nch - 1);
+        if (st_ == 0) bulk_wait_all();                       // h is in global memory before exit
     } else if (is_out) {
         // --------------------------------------------------------- output group
-        // Thread = value row i of H^T (TMEM lane); h goes through a shared tile and
-        // leaves by TMA store, so the global writes are whole 128-byte rows.
+        // Thread = value row i of H^T (TMEM lane); h for tokens 0-31 of each chunk
+        // goes through the shared h tile and leaves by TMA store, so the global
+        // writes are whole 128-byte rows.  The gates are loaded a chunk ahead.
         bool ok = true;
-        const int i = 32 * q4 + lane;
-        uint8_t *hs = sHs + (i >> 6) * 8192 + (i & 63) * 2;
-        float og[32];                                         // output-gate pre-activations, in flight
-        if (nch > 0) {
-            const int Lc0 = min(kL, S - c0 * kL);
-#pragma unroll
-            for (int kk = 0; kk < 32; ++kk)
-                og[kk] = kk < Lc0 ? ldg_nc_early(o_pre + (tok0 + c0 * kL + kk) * D + i0 + i) : 0.f;
-        }
+        float og[32];
+        if (nch > 0) load_gates(0, 0, og);
         for (int c = 0; ok && c < nch; ++c) {
             const int hb = c & 1;
-            const int t0 = (c0 + c) * kL;
-            const int Lc = min(kL, S - t0);
             if (!wait_out(&bars[B_H_FULL0 + hb], (c >> 1) & 1, abort_flag, status) ||
                 !wait_out(&bars[B_FINV_READY0 + hb], (c >> 1) & 1, abort_flag, status)) { ok = false; break; }
             TC_TRACE(xt == 0, c, 10);
-            if (xt == 0) bulk_wait_read_all();               // the previous tile has left the buffer
+            if (xt == 0) bulk_wait_read_all();               // this half of the h tile is free again
             sync_out();
             __syncwarp();
             tc_fence_after();
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {            // tokens [32 half, 32 half + 32)
-                uint32_t r[32];
-                tmem_ld16(t_H0 + 64 * hb + lane_addr + 32 * half, *reinterpret_cast<uint32_t(*)[16]>(&r[0]));
-                tmem_ld16(t_H0 + 64 * hb + lane_addr + 32 * half + 16, *reinterpret_cast<uint32_t(*)[16]>(&r[16]));
-                tmem_wait_ld();
-                TC_TRACE(xt == 0, c, 20 + 2 * half);
-                float ogn[32];                                // the next pass's gates, in flight
-                const int tn0 = half == 0 ? t0 + 32 : t0 + kL;
-                const int ln = half == 0 ? Lc - 32 : (c + 1 < nch ? min(kL, S - t0 - kL) : 0);
-#pragma unroll
-                for (int kk = 0; kk < 32; ++kk)
-                    ogn[kk] = kk < ln ? ldg_nc_early(o_pre + (tok0 + tn0 + kk) * D + i0 + i) : 0.f;
-#ifdef XLSTM_TC_TRACE
-                if (g_tc_trace) {                             // time at which this pass's gates have arrived
-                    float acc = 0.f;
-#pragma unroll
-                    for (int kk = 0; kk < 32; ++kk) acc += og[kk];
-                    if (acc == 1.2345e-30f) og[0] += 1.f;
-                    TC_TRACE(xt == 0, c, 24 + half);
-                }
-#endif
-                const float *inv = finv + 64 * hb + 32 * half;
-#pragma unroll
-                for (int kk = 0; kk < 32; ++kk) {
-                    const float o = __fdividef(1.f, 1.f + __expf(-og[kk]));
-                    *reinterpret_cast<__nv_bfloat16 *>(hs + (32 * half + kk) * 128) =
-                        __float2bfloat16_rn(o * __uint_as_float(r[kk]) * inv[kk]);
-                }
-                TC_TRACE(xt == 0, c, 21 + 2 * half);
-#pragma unroll
-                for (int kk = 0; kk < 32; ++kk) og[kk] = ogn[kk];
-            }
+            TC_TRACE(xt == 0, c, 20);
+            epilogue_pass(c, 0, og);
+            TC_TRACE(xt == 0, c, 21);
+            if (c + 1 < nch) load_gates(c + 1, 0, og);
             fence_async_smem();
             tc_fence_before();
             sync_out();
-            if (xt == 0) {
-                tma_store_3d(&map_h, sHs, i0, t0, bh);
-                tma_store_3d(&map_h, sHs + 8192, i0 + 64, t0, bh);
-                bulk_commit();
-                mbar_arrive(&bars[B_H_FREE0 + hb]);
-                mbar_arrive(&bars[B_FINV_FREE0 + hb]);
-            }
+            finish_pass(c, 0, xt == 0);
             TC_TRACE(xt == 0, c, 11);
         }
         if (xt == 0) bulk_wait_all();                        // h is in global memory before exit
@@ -911,20 +962,23 @@ segment_scan_kernel(const float2 *__restrict__ sstat, float *__restrict__ summ, 
 }
 
 // ------------------------------------------------------------ segment summaries
-// Per (value tile, segment g < P-1, head): dC = sum_s w_s v_s k^_s^T over the
+// Per (value tile, segment g < P-1, head): dC = sum_s w_s v_s k_s^T over the
 // segment, w_s = e^{u_s + E_c - mloc} / sqrt(d) (all exponents <= 0), on the
-// tensor cores with the accumulator in TMEM; dn likewise (tile 0, CUDA cores).
+// tensor cores with the accumulator in TMEM; dn = sum_s w_s k_s on the CUDA
+// cores, each tile taking 128 of the key columns.  K and V stream through a
+// 4-stage ring; V is scaled by w in place.
 template <int D>
 struct SumLayout {
-    static constexpr int kKslot = (D / 64) * 8192;        // K bf16 MN-major view: D/64 blocks x 64 rows
+    static constexpr int kStages = 4;
+    static constexpr int kKslot = (D / 64) * 8192;        // K bf16: D/64 blocks x 64 rows
     static constexpr int kSlot = kKslot + 16384;          // + V (2 blocks x 8 KB)
-    static constexpr int kVh = 2 * kSlot;                 // 2 x 16 KB scaled V
-    static constexpr int kF = kVh + 2 * 16384;            // w[2][64]
-    static constexpr int kTab = kF + 2 * 64 * 4;          // E per chunk
-    static constexpr int kBar = kTab + kMaxCps * 4;
-    static constexpr int kMisc = kBar + 8 * 8;
+    static constexpr int kF = kStages * kSlot;            // w[64]
+    static constexpr int kTab = kF + 64 * 4;              // E per chunk
+    static constexpr int kBar = kTab + kMaxCps * 4;       // full[4], free[4], ready[4], done
+    static constexpr int kMisc = kBar + 16 * 8;
     static constexpr int kBytes = kMisc + 16 + 1024;
 };
+static_assert(SumLayout<256>::kBytes <= kMaxSmemPerCta, "summary kernel shared memory");
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -933,11 +987,13 @@ segment_summary_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __gri
                           const float2 *__restrict__ cstat, float2 *__restrict__ sstat, float *__restrict__ summ,
                           unsigned int *status, int S, int nchunks, int P, int cps) {
     using Lay = SumLayout<D>;
+    constexpr int NS = Lay::kStages;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = align1024(smem_raw);
     float *fw = reinterpret_cast<float *>(smem + Lay::kF);
     float *tabE = reinterpret_cast<float *>(smem + Lay::kTab);
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Lay::kBar);   // full[2], free[2], vh_ready[2], done
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Lay::kBar);
+    uint64_t *b_full = bars, *b_free = bars + NS, *b_ready = bars + 2 * NS, *b_done = bars + 3 * NS;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + Lay::kMisc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + Lay::kMisc + 4);
     __shared__ float s_mloc, s_etot;
@@ -950,17 +1006,24 @@ segment_summary_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __gri
     const size_t tok0 = (size_t)bh * S;
     const float inv_sqrt_d = rsqrtf((float)D);
 
+    float *tabM = fw;                                  // chunk maxima, staged (fw is free until the loop)
+    for (int c = tid; c < nch; c += blockDim.x) {
+        const float2 cs = cstat[(size_t)bh * nchunks + c0 + c];
+        tabE[c] = cs.x;
+        if (c < 64) tabM[c] = cs.y;
+    }
+    __syncthreads();
     if (tid == 0) {
-        for (int i = 0; i < 7; ++i) mbar_init(&bars[i], 1);
+        for (int i = 0; i < 3 * NS + 1; ++i) mbar_init(&bars[i], 1);
         *abort_flag = 0;
         fence_mbar_init();
         // segment statistics: E_c = sum_{c' >= c} btot, mloc = max_c (cmax_c + E_c)
         float E = 0.f, mloc = -INFINITY;
         for (int c = nch - 1; c >= 0; --c) {
-            const float2 cs = cstat[(size_t)bh * nchunks + c0 + c];
-            E += cs.x;
+            const float cy = c < 64 ? tabM[c] : cstat[(size_t)bh * nchunks + c0 + c].y;
+            E += tabE[c];
             tabE[c] = E;
-            mloc = fmaxf(mloc, cs.y + E);
+            mloc = fmaxf(mloc, cy + E);
         }
         s_mloc = mloc;
         s_etot = E;
@@ -980,86 +1043,90 @@ segment_summary_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __gri
         if (lane == 0) {
             tma_prefetch_desc(&map_k);
             tma_prefetch_desc(&map_v);
-            int issued[2] = {0, 0};
+            int issued[NS] = {};
             for (int c = 0; c < nch; ++c) {
-                const int slot = c & 1, t0 = (c0 + c) * kL;
-                if (c >= 2 && !mbar_wait(&bars[2 + slot], ((c >> 1) - 1) & 1, abort_flag, status)) break;
+                const int slot = c % NS, t0 = (c0 + c) * kL;
+                if (c >= NS && !mbar_wait(&b_free[slot], ((c / NS) - 1) & 1, abort_flag, status)) break;
                 uint8_t *base = smem + slot * Lay::kSlot;
-                mbar_arrive_expect_tx(&bars[slot], kL * D * 2 + kL * kRows * 2);
-                for (int jb = 0; jb < D / 64; ++jb) tma_load_3d(base + jb * 8192, &map_k, &bars[slot], jb * 64, t0, bh);
+                mbar_arrive_expect_tx(&b_full[slot], kL * D * 2 + kL * kRows * 2);
+                for (int jb = 0; jb < D / 64; ++jb)
+                    tma_load_3d(base + jb * 8192, &map_k, &b_full[slot], jb * 64, t0, bh);
                 for (int b = 0; b < 2; ++b)
-                    tma_load_3d(base + Lay::kKslot + b * 8192, &map_v, &bars[slot], i0 + 64 * b, t0, bh);
+                    tma_load_3d(base + Lay::kKslot + b * 8192, &map_v, &b_full[slot], i0 + 64 * b, t0, bh);
                 ++issued[slot];
             }
-            for (int s = 0; s < 2; ++s)
-                if (issued[s]) mbar_wait(&bars[s], (issued[s] - 1) & 1, nullptr, status);
+            // never leave a load in flight into shared memory
+            for (int st = 0; st < NS; ++st)
+                if (issued[st]) mbar_wait(&b_full[st], (issued[st] - 1) & 1, nullptr, status);
         }
     } else if (warp == 1) {
         if (lane == 0) {
             for (int c = 0; c < nch; ++c) {
-                const int slot = c & 1;
-                if (!mbar_wait(&bars[4 + slot], (c >> 1) & 1, abort_flag, status)) break;
+                const int slot = c % NS;
+                if (!mbar_wait(&b_ready[slot], (c / NS) & 1, abort_flag, status)) break;
                 tc_fence_after();
-                const uint32_t vha = smem_u32(smem + Lay::kVh + slot * 16384);
+                const uint32_t va = smem_u32(smem + slot * Lay::kSlot + Lay::kKslot);
                 const uint32_t ka = smem_u32(smem + slot * Lay::kSlot);
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
-                    mma_bf16_ss(tacc, sdesc_sw128(vha + ks * 2048, 8192, 1024),
+                    mma_bf16_ss(tacc, sdesc_sw128(va + ks * 2048, 8192, 1024),
                                 sdesc_sw128(ka + ks * 2048, 8192, 1024), idesc_U, (c > 0 || ks > 0) ? 1u : 0u);
-                mma_commit(&bars[2 + slot]);
+                mma_commit(&b_free[slot]);
             }
-            mma_commit(&bars[6]);
-            mbar_wait(&bars[6], 0, nullptr, status);
+            mma_commit(b_done);
+            mbar_wait(b_done, 0, nullptr, status);
         }
     } else {
         const int ct = tid - 64, q4 = warp & 3;
-        float nacc[D / 128];
-#pragma unroll
-        for (int r = 0; r < D / 128; ++r) nacc[r] = 0.f;
+        const int jn = tile * 128 + ct;                   // this thread's key column of dn
+        float nacc = 0.f;
         bool ok = true;
+        float pre_i = 0.f, pre_b = 0.f;                   // gates of the next chunk, in flight
+        if (nch > 0 && ct < kL && c0 * kL + ct < S) {
+            pre_i = i_pre[tok0 + c0 * kL + ct];
+            pre_b = bcum[tok0 + c0 * kL + ct];
+        }
         for (int c = 0; c < nch; ++c) {
-            const int slot = c & 1, t0 = (c0 + c) * kL, Lc = min(kL, S - t0);
-            if (ct < kL) {
-                const int t = ct;
-                fw[64 * slot + t] = t < Lc
-                    ? expf(i_pre[tok0 + t0 + t] - bcum[tok0 + t0 + t] + tabE[c] - mloc) * inv_sqrt_d : 0.f;
+            const int slot = c % NS, t0 = (c0 + c) * kL, Lc = min(kL, S - t0);
+            if (ct < kL)
+                fw[ct] = ct < Lc ? expf(pre_i - pre_b + tabE[c] - mloc) * inv_sqrt_d : 0.f;
+            pre_i = pre_b = 0.f;
+            if (c + 1 < nch && ct < kL && t0 + kL + ct < S) {
+                pre_i = i_pre[tok0 + t0 + kL + ct];
+                pre_b = bcum[tok0 + t0 + kL + ct];
             }
-            if (!compute_wait(&bars[slot], (c >> 1) & 1, abort_flag, status)) { ok = false; break; }
+            if (!compute_wait(&b_full[slot], (c / NS) & 1, abort_flag, status)) { ok = false; break; }
             named_sync_compute();
-            const uint8_t *base = smem + slot * Lay::kSlot;
-            const uint8_t *sV = base + Lay::kKslot;
-            uint8_t *sVh = smem + Lay::kVh + slot * 16384;
-            const float *w = fw + 64 * slot;
-            for (int e = ct; e < 2 * kL * 8; e += 128) {
+            uint8_t *base = smem + slot * Lay::kSlot;
+            uint8_t *sV = base + Lay::kKslot;
+#pragma unroll 4
+            for (int e = ct; e < 2 * kL * 8; e += 128) {   // V rows scaled in place by w
                 const int blk = e / (kL * 8), s = (e / 8) % kL, cc = e & 7;
-                const uint32_t off = blk * 8192 + sw128_offset(s, cc);
-                const uint4 src = *reinterpret_cast<const uint4 *>(sV + off);
-                const float ws = w[s];
+                uint4 *pv = reinterpret_cast<uint4 *>(sV + blk * 8192 + sw128_offset(s, cc));
+                const uint4 src = *pv;
+                const float ws = fw[s];
                 uint4 dst;
                 dst.x = pack_bf16x2(bf16_lo(src.x) * ws, bf16_hi(src.x) * ws);
                 dst.y = pack_bf16x2(bf16_lo(src.y) * ws, bf16_hi(src.y) * ws);
                 dst.z = pack_bf16x2(bf16_lo(src.z) * ws, bf16_hi(src.z) * ws);
                 dst.w = pack_bf16x2(bf16_lo(src.w) * ws, bf16_hi(src.w) * ws);
-                *reinterpret_cast<uint4 *>(sVh + off) = dst;
+                *pv = dst;
             }
-            if (tile == 0) {
-#pragma unroll
-                for (int r = 0; r < D / 128; ++r) {
-                    const int j = ct + 128 * r;
-                    const uint8_t *blkp = base + (j / 64) * 8192;
-                    const int cc = (j % 64) / 8, within = (j % 8) * 2;
-                    float acc = 0.f;
-                    for (int s = 0; s < kL; ++s)
-                        acc += w[s] * __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(
-                                          blkp + sw128_offset(s, cc) + within));
-                    nacc[r] += acc;
-                }
+            if (jn < D) {
+                const uint8_t *blkp = base + (jn / 64) * 8192;
+                const int cc = (jn % 64) / 8, within = (jn % 8) * 2;
+                float acc = 0.f;
+#pragma unroll 8
+                for (int s = 0; s < kL; ++s)
+                    acc += fw[s] * __bfloat162float(
+                                       *reinterpret_cast<const __nv_bfloat16 *>(blkp + sw128_offset(s, cc) + within));
+                nacc += acc;
             }
             fence_async_smem();
             named_sync_compute();
-            if (ct == 0) mbar_arrive(&bars[4 + slot]);
+            if (ct == 0) mbar_arrive(&b_ready[slot]);
         }
-        if (ok && compute_wait(&bars[6], 0, abort_flag, status)) {
+        if (ok && compute_wait(b_done, 0, abort_flag, status)) {
             __syncwarp();
             tc_fence_after();
             float *out = summ + ((size_t)bh * (P - 1) + g) * ((size_t)D * D + D);
@@ -1075,10 +1142,7 @@ segment_summary_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __gri
                     dst[e] = make_float4(__uint_as_float(r[4 * e]), __uint_as_float(r[4 * e + 1]),
                                          __uint_as_float(r[4 * e + 2]), __uint_as_float(r[4 * e + 3]));
             }
-            if (tile == 0) {
-#pragma unroll
-                for (int r = 0; r < D / 128; ++r) out[(size_t)D * D + ct + 128 * r] = nacc[r];
-            }
+            if (jn < D) out[(size_t)D * D + jn] = nacc;
         }
         tc_fence_before();
     }
@@ -1109,14 +1173,28 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// [BH, S, D] bf16, box 64 x 64 x 1; loads use the 128-byte swizzle (rows past S
-// read as zeros), the h store map no swizzle (rows past S are not written).
-bool make_map(CUtensorMap *m, const void *base, int BH, int S, int D, bool swizzle = true) {
+// [BH, S, D] fp32, box 128 x 64 x 1, no swizzle: L2 prefetches of the output gates.
+bool make_map_f32_rows(CUtensorMap *m, const void *base, int BH, int S, int D) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)S, (cuuint64_t)BH};
+    cuuint64_t strides[2] = {(cuuint64_t)D * 4, (cuuint64_t)S * D * 4};
+    cuuint32_t box[3] = {128, 64, 1};
+    cuuint32_t es[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void *>(base), dims, strides, box, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// [BH, S, D] bf16, box 64 x box_rows x 1.  The q/k/v loads use the 128-byte
+// swizzle (rows past S read as zeros); the h stores use no swizzle and 32-row
+// boxes (rows past S are not written).
+bool make_map(CUtensorMap *m, const void *base, int BH, int S, int D, bool swizzle = true, int box_rows = 64) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)S, (cuuint64_t)BH};
     cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)S * D * 2};
-    cuuint32_t box[3] = {64, 64, 1};
+    cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
     cuuint32_t es[3] = {1, 1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, es,
               CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
@@ -1125,9 +1203,10 @@ bool make_map(CUtensorMap *m, const void *base, int BH, int S, int D, bool swizz
 
 template <int D>
 cudaError_t launch_tc_t(const FwdArgs &a, const FwdPlan &p, cudaStream_t st) {
-    CUtensorMap mq, mk, mv, mh;
+    CUtensorMap mq, mk, mv, mh, mo;
     if (!make_map(&mq, a.q, p.BH, p.S, D) || !make_map(&mk, a.k, p.BH, p.S, D) ||
-        !make_map(&mv, a.v, p.BH, p.S, D) || !make_map(&mh, a.h, p.BH, p.S, D, false))
+        !make_map(&mv, a.v, p.BH, p.S, D) || !make_map(&mh, a.h, p.BH, p.S, D, false, 32) ||
+        !make_map_f32_rows(&mo, a.o_pre, p.BH, p.S, D))
         return cudaErrorInvalidValue;
     float *ws = (float *)a.workspace;
     const float *bcum = ws + p.off_bcum;
@@ -1158,7 +1237,7 @@ cudaError_t launch_tc_t(const FwdArgs &a, const FwdPlan &p, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     KernelTimer timer("segment_output_tc", st);
     segment_output_tc_kernel<D><<<dim3(D / kRows, p.P, p.BH), kOutThreads, sm, st>>>(
-        mq, mk, mv, mh, a.i_pre, a.o_pre, a.C0, a.n0, a.m0, a.C_out, a.n_out, a.m_out,
+        mq, mk, mv, mh, mo, a.i_pre, a.o_pre, a.C0, a.n0, a.m0, a.C_out, a.n_out, a.m_out,
         bcum, ws + p.off_pmax, cstat, sstat, summ, a.status, p.S, p.nchunks, p.P, p.cps);
     return cudaGetLastError();
 }
