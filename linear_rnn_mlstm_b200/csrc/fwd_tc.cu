@@ -43,12 +43,12 @@ constexpr int kL = 64;             // tokens per chunk on this path
 constexpr int kRows = 128;         // value rows per CTA
 constexpr int kKRows = 72;         // key-tile rows: 64 keys, n' hi, n' lo, 6 zero rows
 constexpr int kKBlock = kKRows * 128;   // bytes per 64-column block of the key tile
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;       // segment summaries: TMA warp, MMA warp, 8 compute warps
 constexpr int kMaxCps = 256;       // chunks per segment the tables hold
 constexpr float kLnLambdaFloor = -40.f;  // rescale the TMEM state below this log scale
 constexpr float kLnChunkFloor = -60.f;   // smallest decay of the state's scale over one chunk (see below)
 
-__device__ __forceinline__ void named_sync_compute() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+__device__ __forceinline__ void named_sync_compute() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 
 #ifdef XLSTM_TC_TRACE
 // Timing trace of the pipeline steps (diagnostic builds only): 32 globaltimer
@@ -68,7 +68,7 @@ __device__ unsigned long long *g_tc_trace = nullptr;
 // A bounded wait taken by all 128 compute threads, with a group-uniform result.
 __device__ __forceinline__ bool compute_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
                                              unsigned int *status) {
-    return group_all<1, 128>(mbar_wait(bar, parity, abort_flag, status));
+    return group_wait<1, 256>(bar, parity, threadIdx.x == 64, abort_flag, status);
 }
 
 __device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
@@ -1077,8 +1077,11 @@ segment_summary_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __gri
             mbar_wait(b_done, 0, nullptr, status);
         }
     } else {
+        // 8 compute warps: all scale V; threads 0-127 also accumulate dn, one key
+        // column each; for the readout, the two warps of each TMEM lane quadrant
+        // take one half of the columns each.
         const int ct = tid - 64, q4 = warp & 3;
-        const int jn = tile * 128 + ct;                   // this thread's key column of dn
+        const int jn = ct < 128 ? tile * 128 + ct : D;    // this thread's key column of dn
         float nacc = 0.f;
         bool ok = true;
         float pre_i = 0.f, pre_b = 0.f;                   // gates of the next chunk, in flight
@@ -1100,7 +1103,7 @@ segment_summary_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __gri
             uint8_t *base = smem + slot * Lay::kSlot;
             uint8_t *sV = base + Lay::kKslot;
 #pragma unroll 4
-            for (int e = ct; e < 2 * kL * 8; e += 128) {   // V rows scaled in place by w
+            for (int e = ct; e < 2 * kL * 8; e += 256) {   // V rows scaled in place by w
                 const int blk = e / (kL * 8), s = (e / 8) % kL, cc = e & 7;
                 uint4 *pv = reinterpret_cast<uint4 *>(sV + blk * 8192 + sw128_offset(s, cc));
                 const uint4 src = *pv;
@@ -1132,7 +1135,8 @@ segment_summary_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __gri
             float *out = summ + ((size_t)bh * (P - 1) + g) * ((size_t)D * D + D);
             const int i = 32 * q4 + lane;
             const uint32_t lane_addr = ((uint32_t)(32 * q4)) << 16;
-            for (int jb = 0; jb < D; jb += 16) {
+            const int jhalf = (ct >> 7) * (D / 2);
+            for (int jb = jhalf; jb < jhalf + D / 2; jb += 16) {
                 uint32_t r[16];
                 tmem_ld16(tacc + lane_addr + jb, r);
                 tmem_wait_ld();
