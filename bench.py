@@ -396,7 +396,7 @@ def main():
         line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-                "dtype": "bf16" if (w.dtype == "bf16" and top and top.endswith("_tc")) else "f32",
+                "dtype": "bf16" if (w.dtype == "bf16" and any(k.endswith("_tc") for k in kt)) else "f32",
                 "data": "synthetic (seeded N(0,1)-based draws of the workload shapes)",
                 "config": dict(workload_config(w, args.chunk, world),
                                l2="inputs 406 MB > 126 MB L2; no flush" if w.name == "long"
