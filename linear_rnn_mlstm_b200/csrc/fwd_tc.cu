@@ -964,14 +964,15 @@ segment_scan_kernel(const float2 *__restrict__ sstat, float *__restrict__ summ, 
 // ------------------------------------------------------------ segment summaries
 // Per (value tile, segment g < P-1, head): dC = sum_s w_s v_s k_s^T over the
 // segment, w_s = e^{u_s + E_c - mloc} / sqrt(d) (all exponents <= 0), on the
-// tensor cores with the accumulator in TMEM; dn = sum_s w_s k_s on the CUDA
-// cores, each tile taking 128 of the key columns.  K and V stream through a
-// 4-stage ring; V is scaled by w in place.
+// tensor cores with the accumulator in TMEM; dn = sum_s w_s k_s on the tensor
+// cores too, as rows 0 and 1 (w in bf16 high and low parts) of an M=64 product
+// with the same K tile.  K and V stream through a 4-stage ring; V is scaled by
+// w in place.
 template <int D>
 struct SumLayout {
     static constexpr int kStages = 4;
     static constexpr int kKslot = (D / 64) * 8192;        // K bf16: D/64 blocks x 64 rows
-    static constexpr int kSlot = kKslot + 16384;          // + V (2 blocks x 8 KB)
+    static constexpr int kSlot = kKslot + 16384 + 8192;   // + V (2 blocks x 8 KB) + W (64 x 64 bf16, rows 0-1 used)
     static constexpr int kF = kStages * kSlot;            // w[64]
     static constexpr int kTab = kF + 64 * 4;              // E per chunk
     static constexpr int kBar = kTab + kMaxCps * 4;       // full[4], free[4], ready[4], done
@@ -1030,14 +1031,20 @@ segment_summary_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __gri
         if (tile == 0) sstat[(size_t)bh * P + g] = make_float2(E, mloc);
     }
     if (warp == 1) {
-        tmem_alloc(tmem_slot, 256);
+        tmem_alloc(tmem_slot, 512);
         tc_fence_before();
     }
+    for (int e = tid; e < NS * 512; e += blockDim.x) {     // the W tiles start all zero
+        const int st = e >> 9, off = (e & 511) * 16;
+        *reinterpret_cast<uint4 *>(smem + st * Lay::kSlot + Lay::kKslot + 16384 + off) = make_uint4(0u, 0u, 0u, 0u);
+    }
+    fence_async_smem();
     __syncthreads();
     tc_fence_after();
-    const uint32_t tacc = *tmem_slot;
+    const uint32_t tacc = *tmem_slot;                  // dC in columns [0, D), dn rows in [256, 256 + D)
     const float mloc = s_mloc;
     const uint32_t idesc_U = idesc_f32acc(kFmtBF16, kFmtBF16, true, true, 128, D);
+    const uint32_t idesc_N = idesc_f32acc(kFmtBF16, kFmtBF16, false, true, 64, D);
 
     if (warp == 0) {
         if (lane == 0) {
@@ -1067,22 +1074,25 @@ segment_summary_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __gri
                 tc_fence_after();
                 const uint32_t va = smem_u32(smem + slot * Lay::kSlot + Lay::kKslot);
                 const uint32_t ka = smem_u32(smem + slot * Lay::kSlot);
+                const uint32_t wa = va + 16384;
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
                     mma_bf16_ss(tacc, sdesc_sw128(va + ks * 2048, 8192, 1024),
                                 sdesc_sw128(ka + ks * 2048, 8192, 1024), idesc_U, (c > 0 || ks > 0) ? 1u : 0u);
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_bf16_ss(tacc + 256, sdesc_sw128(wa + ks * 32, 16, 1024),
+                                sdesc_sw128(ka + ks * 2048, 8192, 1024), idesc_N, (c > 0 || ks > 0) ? 1u : 0u);
                 mma_commit(&b_free[slot]);
             }
             mma_commit(b_done);
             mbar_wait(b_done, 0, nullptr, status);
         }
     } else {
-        // 8 compute warps: all scale V; threads 0-127 also accumulate dn, one key
-        // column each; for the readout, the two warps of each TMEM lane quadrant
-        // take one half of the columns each.
+        // 8 compute warps: w and its bf16 parts (threads 0-63), V scaled in place
+        // (all); for the readout, the two warps of each TMEM lane quadrant take
+        // one half of the columns each.
         const int ct = tid - 64, q4 = warp & 3;
-        const int jn = ct < 128 ? tile * 128 + ct : D;    // this thread's key column of dn
-        float nacc = 0.f;
         bool ok = true;
         float pre_i = 0.f, pre_b = 0.f;                   // gates of the next chunk, in flight
         if (nch > 0 && ct < kL && c0 * kL + ct < S) {
@@ -1099,9 +1109,17 @@ segment_summary_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __gri
                 pre_b = bcum[tok0 + t0 + kL + ct];
             }
             if (!compute_wait(&b_full[slot], (c / NS) & 1, abort_flag, status)) { ok = false; break; }
-            named_sync_compute();
             uint8_t *base = smem + slot * Lay::kSlot;
             uint8_t *sV = base + Lay::kKslot;
+            if (ct < kL) {       // rows 0 and 1 of W: w in bf16 high and low parts
+                const float wv = fw[ct];
+                const __nv_bfloat16 whi = __float2bfloat16_rn(wv);
+                uint8_t *sW = sV + 16384;
+                *reinterpret_cast<__nv_bfloat16 *>(sW + sw128_offset(0, ct >> 3) + (ct & 7) * 2) = whi;
+                *reinterpret_cast<__nv_bfloat16 *>(sW + sw128_offset(1, ct >> 3) + (ct & 7) * 2) =
+                    __float2bfloat16_rn(wv - __bfloat162float(whi));
+            }
+            named_sync_compute();
 #pragma unroll 4
             for (int e = ct; e < 2 * kL * 8; e += 256) {   // V rows scaled in place by w
                 const int blk = e / (kL * 8), s = (e / 8) % kL, cc = e & 7;
@@ -1114,16 +1132,6 @@ segment_summary_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __gri
                 dst.z = pack_bf16x2(bf16_lo(src.z) * ws, bf16_hi(src.z) * ws);
                 dst.w = pack_bf16x2(bf16_lo(src.w) * ws, bf16_hi(src.w) * ws);
                 *pv = dst;
-            }
-            if (jn < D) {
-                const uint8_t *blkp = base + (jn / 64) * 8192;
-                const int cc = (jn % 64) / 8, within = (jn % 8) * 2;
-                float acc = 0.f;
-#pragma unroll 8
-                for (int s = 0; s < kL; ++s)
-                    acc += fw[s] * __bfloat162float(
-                                       *reinterpret_cast<const __nv_bfloat16 *>(blkp + sw128_offset(s, cc) + within));
-                nacc += acc;
             }
             fence_async_smem();
             named_sync_compute();
@@ -1146,14 +1154,26 @@ segment_summary_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __gri
                     dst[e] = make_float4(__uint_as_float(r[4 * e]), __uint_as_float(r[4 * e + 1]),
                                          __uint_as_float(r[4 * e + 2]), __uint_as_float(r[4 * e + 3]));
             }
-            if (jn < D) out[(size_t)D * D + jn] = nacc;
+            if (q4 == 0) {      // dn = rows 0 + 1 of the M=64 product (TMEM lanes 0 and 1)
+                for (int jb = jhalf; jb < jhalf + D / 2; jb += 16) {
+                    uint32_t r[16];
+                    tmem_ld16(tacc + 256 + jb, r);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const float v = __uint_as_float(r[e]) + __shfl_down_sync(0xffffffffu, __uint_as_float(r[e]), 1);
+                        if (lane == 0 && (jb + e) / 128 == tile)      // each tile writes its 128 columns
+                            out[(size_t)D * D + jb + e] = v;
+                    }
+                }
+            }
         }
         tc_fence_before();
     }
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tacc, 256);
+        tmem_dealloc(tacc, 512);
         tmem_relinquish();
     }
 }
