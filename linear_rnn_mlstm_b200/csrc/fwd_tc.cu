@@ -97,7 +97,7 @@ struct OutLayout {
     static constexpr int kNF = 16 * 64;
     static constexpr int kTab = kF + kNF * 4;             // per-chunk tables
     static constexpr int kBar = kTab + 5 * kMaxCps * 4;
-    static constexpr int kNumBars = 32;
+    static constexpr int kNumBars = 40;
     static constexpr int kMisc = kBar + kNumBars * 8;     // tmem base, abort flag
     static constexpr int kEnd = kMisc + 16;
     static constexpr int kBytes = kEnd + 1024;            // slack for 1024-byte alignment
@@ -111,7 +111,7 @@ enum {
     B_VHAT_READY, B_QT_READY, B_QT_FREE, B_S_FULL, B_S_FREE, B_P_READY, B_P_FREE,
     B_H_FULL0, B_H_FULL1, B_H_FREE0, B_H_FREE1, B_NROW_READY0, B_NROW_READY1, B_RESC_DONE, B_DONE,
     B_GATES_READY0, B_GATES_READY1, B_GATES_FREE0, B_GATES_FREE1,
-    B_FINV_READY0, B_FINV_READY1, B_FINV_FREE0, B_FINV_FREE1, B_INTRA_DONE, B_NUM
+    B_FINV_READY0, B_FINV_READY1, B_FINV_FREE0, B_FINV_FREE1, B_INTRA_DONE, B_STATE_READY, B_NUM
 };
 static_assert(B_NUM <= OutLayout<128>::kNumBars, "barrier slots");
 // Every barrier is waited by parity, so no producer may complete a barrier twice
@@ -243,33 +243,10 @@ segment_output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
     const uint32_t t_H0 = tbase + 384;             // columns [384, 448) and [448, 512)
 
     if (is_ops) {
-        // Incoming state: the initial state for segment 0, else the state at the end
-        // of segment g - 1, which segment_scan_kernel left in summary slot g - 1.
+        // incoming normaliser (the incoming C' goes to TMEM from the output group)
         const float m_init = m0 ? m0[bh] : 0.f;
-        const int i = 32 * q4 + lane;
-        const float *src = g == 0 ? (C0 ? C0 + (size_t)bh * D * D : nullptr)
-                                  : summ + ((size_t)bh * (P - 1) + g - 1) * ((size_t)D * D + D);
-        const float *nsrc = g == 0 ? (n0 ? n0 + (size_t)bh * D : nullptr) : src + (size_t)D * D;
-#pragma unroll 4
-        for (int jb = 0; jb < D; jb += 16) {
-            uint32_t r[16];
-            if (src) {
-                const float4 *row = reinterpret_cast<const float4 *>(src + (size_t)(i0 + i) * D + jb);
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float4 x = row[e];
-                    r[4 * e] = __float_as_uint(x.x);
-                    r[4 * e + 1] = __float_as_uint(x.y);
-                    r[4 * e + 2] = __float_as_uint(x.z);
-                    r[4 * e + 3] = __float_as_uint(x.w);
-                }
-            } else {
-#pragma unroll
-                for (int e = 0; e < 16; ++e) r[e] = 0u;
-            }
-            tmem_st16(t_state + lane_addr + jb, r);
-        }
-        tmem_wait_st();
+        const float *nsrc = g == 0 ? (n0 ? n0 + (size_t)bh * D : nullptr)
+                                   : summ + ((size_t)bh * (P - 1) + g - 1) * ((size_t)D * D + D) + (size_t)D * D;
 #pragma unroll
         for (int r = 0; r < D / 128; ++r) nreg[r] = nsrc ? nsrc[nj(r)] : 0.f;
         // zero the extra key rows 64..71 of both slots, then n'_in (hi, lo) in slot 0
@@ -461,6 +438,7 @@ segment_output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
                     ++nresc;
                 }
                 if (!mbar_wait(&bars[B_QT_READY], c & 1, abort_flag, status)) { ok = false; break; }
+                if (c == 0 && !mbar_wait(&bars[B_STATE_READY], 0, abort_flag, status)) { ok = false; break; }
                 if (c >= 2 && !mbar_wait(&bars[B_H_FREE0 + hb], ((c >> 1) - 1) & 1, abort_flag, status)) {
                     ok = false;
                     break;
@@ -889,6 +867,36 @@ segment_output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
         // goes through the shared h tile and leaves by TMA store, so the global
         // writes are whole 128-byte rows.  The gates are loaded a chunk ahead.
         bool ok = true;
+        {   // Incoming state into TMEM, while the other groups start on chunk 0: the
+            // initial state for segment 0, else the state at the end of segment g - 1,
+            // which segment_scan_kernel left in summary slot g - 1.
+            const int i = 32 * q4 + lane;
+            const float *src = g == 0 ? (C0 ? C0 + (size_t)bh * D * D : nullptr)
+                                      : summ + ((size_t)bh * (P - 1) + g - 1) * ((size_t)D * D + D);
+#pragma unroll 4
+            for (int jb = 0; jb < D; jb += 16) {
+                uint32_t r[16];
+                if (src) {
+                    const float4 *row = reinterpret_cast<const float4 *>(src + (size_t)(i0 + i) * D + jb);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float4 x = row[e];
+                        r[4 * e] = __float_as_uint(x.x);
+                        r[4 * e + 1] = __float_as_uint(x.y);
+                        r[4 * e + 2] = __float_as_uint(x.z);
+                        r[4 * e + 3] = __float_as_uint(x.w);
+                    }
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) r[e] = 0u;
+                }
+                tmem_st16(t_state + lane_addr + jb, r);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            sync_out();
+            if (xt == 0) mbar_arrive(&bars[B_STATE_READY]);
+        }
         float og[32];
         if (nch > 0) load_gates(0, 0, og);
         for (int c = 0; ok && c < nch; ++c) {
