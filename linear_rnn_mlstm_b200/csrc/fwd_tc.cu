@@ -413,13 +413,18 @@ segment_output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
             bool ok = true;
             auto issue_S = [&](int c) {
                 const int slot = c & 1;
-                const uint32_t qa = smem_u32(sQ), ka = smem_u32(sK + slot * Lay::kKslot);
+                // Descriptors are built once and stepped in place: +32 B (2 units of 16 B)
+                // per K step inside a 128-byte row, one block per four steps.  Shared
+                // addresses are below 256 KB, so the 14-bit address field cannot carry
+                // out.  Four MMAs per loop body keep the issuing thread's code small.
+                uint64_t dq = sdesc_sw128(smem_u32(sQ), 16, 1024);
+                uint64_t dk = sdesc_sw128(smem_u32(sK + slot * Lay::kKslot), 16, 1024);
 #pragma unroll 1
-                for (int ks = 0; ks < D / 16; ++ks) {
-                    const uint32_t off_q = (ks >> 2) * 8192 + (ks & 3) * 32;
-                    const uint32_t off_k = (ks >> 2) * kKBlock + (ks & 3) * 32;
-                    mma_bf16_ss(t_S, sdesc_sw128(qa + off_q, 16, 1024), sdesc_sw128(ka + off_k, 16, 1024),
-                                idesc_S, ks > 0);
+                for (int jb = 0; jb < D / 64; ++jb) {
+#pragma unroll
+                    for (int k4 = 0; k4 < 4; ++k4) mma_bf16_ss(t_S, dq + 2 * k4, dk + 2 * k4, idesc_S, (jb | k4) != 0);
+                    dq += 8192 >> 4;
+                    dk += kKBlock >> 4;
                 }
                 mma_commit(&bars[B_S_FULL]);
                 mma_commit(&bars[B_Q_FREE]);
@@ -446,11 +451,14 @@ segment_output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
                 tc_fence_after();
                 TC_TRACE(true, c, 12);
                 {   // retrieval from the state at the chunk start: H^T = Cs Q^T (tf32, Cs in TMEM)
-                    const uint32_t qta = smem_u32(sQt);
+                    uint64_t dqt = sdesc_sw128(smem_u32(sQt), 16, 1024);
+                    uint32_t ta = t_state;
 #pragma unroll 1
-                    for (int ks = 0; ks < D / 8; ++ks) {
-                        const uint32_t off = (ks >> 2) * 8192 + (ks & 3) * 32;
-                        mma_tf32_ts(t_H, t_state + ks * 8, sdesc_sw128(qta + off, 16, 1024), idesc_R, ks > 0);
+                    for (int blk = 0; blk < D / 32; ++blk) {
+#pragma unroll
+                        for (int k4 = 0; k4 < 4; ++k4) mma_tf32_ts(t_H, ta + 8 * k4, dqt + 2 * k4, idesc_R, (blk | k4) != 0);
+                        dqt += 8192 >> 4;
+                        ta += 32;
                     }
                     mma_commit(&bars[B_QT_FREE]);
                 }
