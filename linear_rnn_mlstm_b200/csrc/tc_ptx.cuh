@@ -48,16 +48,15 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
-// As mbar_try_wait, but the thread may sleep in hardware for up to `hint_ns`
-// nanoseconds (it wakes as soon as the phase completes) instead of spinning.
-__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *bar, uint32_t parity, uint32_t hint_ns) {
+// Non-blocking test of the phase (never suspends the thread).
+__device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+        : "r"(smem_u32(bar)), "r"(parity)
         : "memory");
     return ok != 0;
 }
@@ -78,7 +77,10 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     for (;;) {
-        if (mbar_try_wait_sleep(bar, parity, 200000u)) return true;
+        // poll without suspending (measured a little faster than a suspending wait),
+        // with a short back-off so the poller takes few issue slots
+        if (mbar_test_wait(bar, parity)) return true;
+        __nanosleep(64);
         if (abort_flag && *abort_flag) return false;
         if (globaltimer_ns() - t0 > limit_ns) {
             if (abort_flag) *abort_flag = 1;
