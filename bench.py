@@ -82,15 +82,20 @@ def kernel_algorithmic_bytes(name, w, plan):
 
 
 def source_sha(kernel):
-    files = {"segment_output_simt": "fwd_simt.cu", "segment_summary_simt": "fwd_simt.cu",
-             "gate_prologue": "fwd_simt.cu", "step_rows": "step.cu", "step_state": "step.cu"}
-    fn = files.get(kernel)
-    if fn is None and kernel.endswith("_tc"):
-        fn = "fwd_tc.cu"
-    if fn is None:
+    """sha1 of the source files a kernel is built from (the tensor-core kernels
+    also depend on the tcgen05/TMA wrappers)."""
+    files = {"segment_output_simt": ["fwd_simt.cu"], "segment_summary_simt": ["fwd_simt.cu"],
+             "gate_prologue": ["fwd_simt.cu"], "step_rows": ["step.cu"], "step_state": ["step.cu"]}
+    fns = files.get(kernel)
+    if fns is None and kernel.endswith("_tc"):
+        fns = ["fwd_tc.cu", "tc_ptx.cuh"]
+    if fns is None:
         return None
-    with open(os.path.join(ROOT, "linear_rnn_mlstm_b200", "csrc", fn), "rb") as f:
-        return hashlib.sha1(f.read()).hexdigest()
+    h = hashlib.sha1()
+    for fn in fns:
+        with open(os.path.join(ROOT, "linear_rnn_mlstm_b200", "csrc", fn), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
 
 
 def ncu_traffic(kernel, units):

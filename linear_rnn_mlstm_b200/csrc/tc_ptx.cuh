@@ -74,11 +74,12 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 // before tearing down).  No wait is endless.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
                                           unsigned int *status, uint64_t limit_ns = 2000000000ull) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_test_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     for (;;) {
-        // poll without suspending (measured a little faster than a suspending wait),
-        // with a short back-off so the poller takes few issue slots
+        // poll without suspending: a waiter suspended in try_wait was measured to
+        // resume microseconds after the phase completed; a short back-off keeps
+        // the poller's issue slots few
         if (mbar_test_wait(bar, parity)) return true;
         __nanosleep(64);
         if (abort_flag && *abort_flag) return false;
