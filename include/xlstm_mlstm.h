@@ -59,9 +59,11 @@ typedef enum { XLSTM_F32 = 0, XLSTM_BF16 = 1 } xlstm_dtype;          /* dtype of
 typedef enum { XLSTM_FGATE_SIGMOID = 0, XLSTM_FGATE_EXP = 1 } xlstm_fgate;
 
 /* Kernel family for the forward.  AUTO picks the tensor-core (tcgen05) kernels
- * for bf16 inputs and the fp32 SIMT kernels for fp32 inputs.  SIMT forces the
- * fp32-arithmetic kernels for either dtype (a second, independent path used by
- * the tests). */
+ * for bf16 inputs with DH 128 or 256 and chunk 64, and the fp32 SIMT kernels
+ * for every other case.  SIMT forces the fp32-arithmetic kernels for any
+ * supported arguments (a second, independent path the tests compare against).
+ * TENSOR forces the tensor-core kernels; for arguments they do not take the
+ * call returns XLSTM_ERR_UNSUPPORTED and launches nothing. */
 typedef enum { XLSTM_PATH_AUTO = 0, XLSTM_PATH_SIMT = 1, XLSTM_PATH_TENSOR = 2 } xlstm_path;
 
 typedef struct {
@@ -100,7 +102,7 @@ xlstm_status xlstm_mlstm_fwd_workspace_size_ex(int B, int NH, int S, int DH, int
  *                stabilised units; each may be NULL, meaning zeros.
  *   C_out, n_out, m_out  same shapes, final state; each may be NULL (not written).
  *                They must not overlap C0, n0, m0 or any input (the same
-                pointer passed twice is rejected with XLSTM_ERR_UNSUPPORTED).
+ *              pointer passed twice is rejected with XLSTM_ERR_UNSUPPORTED).
  *   chunk        tokens per chunk of the chunkwise form: 64, 128 or 256 for
  *                bf16; 1..1024 for f32.  S need not be a multiple of chunk.
  *   DH           multiple of 16 in [16, 512].
