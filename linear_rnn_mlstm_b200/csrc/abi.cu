@@ -248,6 +248,8 @@ xlstm_status xlstm_mlstm_step(const void *q, const void *k, const void *v,
     a.BH = B * NH; a.DH = DH;
     a.bf16 = dt == XLSTM_BF16;
     a.fgate_exp = fg == XLSTM_FGATE_EXP;
+    a.status = nullptr;
+    if (cudaGetSymbolAddress((void **)&a.status, g_device_status) != cudaSuccess) return XLSTM_ERR_CUDA;
     return launch_step(a, (cudaStream_t)cuda_stream) == cudaSuccess ? XLSTM_OK : XLSTM_ERR_CUDA;
 }
 

@@ -28,6 +28,7 @@ struct StepArgs {
     int BH, DH;
     int bf16;
     int fgate_exp;
+    unsigned int *status;     // device status word of the current device
 };
 
 cudaError_t launch_gate_prologue(const FwdArgs &a, const FwdPlan &p, cudaStream_t st);

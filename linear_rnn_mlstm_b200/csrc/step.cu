@@ -20,6 +20,7 @@
 #include "common.cuh"
 #include "kernels.h"
 #include "profile.h"
+#include "tc_ptx.cuh"
 
 namespace xlstm {
 
@@ -148,6 +149,152 @@ step_rows_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__re
     }
 }
 
+// The same row update for DH a multiple of 128, with the state streamed through
+// shared memory by bulk copies: each CTA owns 128 consecutive rows of one head
+// and moves them in 8 KB stages (4, 8 or 16 rows) through a ring of kRing
+// stages.  One thread issues the bulk loads (and, after the update, the bulk
+// stores of the same stage); the CTA's 256 threads each update 8 consecutive
+// floats of one row per stage.  Bytes in flight per SM are set by the ring, not
+// by registers.  Every wait is bounded and latches the device status word.
+namespace ts = xlstm::tc;
+constexpr int kStreamRows = 128;           // rows of a head per CTA
+constexpr int kStageBytes = 8192;          // one bulk copy
+constexpr int kRing = 6;                   // stages in flight
+
+template <typename T>
+__global__ void __launch_bounds__(256)
+step_stream_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
+                   const float *__restrict__ i_pre, const float *__restrict__ f_pre,
+                   const float *__restrict__ o_pre, T *__restrict__ h,
+                   float *__restrict__ C, const float *__restrict__ n, const float *__restrict__ m,
+                   int DH, int fgate_exp, unsigned int *status) {
+    extern __shared__ __align__(128) uint8_t st_smem[];
+    float *ring = reinterpret_cast<float *>(st_smem);                           // kRing x 2048 floats
+    uint64_t *full = reinterpret_cast<uint64_t *>(st_smem + kRing * kStageBytes);
+    float *part = reinterpret_cast<float *>(full + kRing);                        // [256] row partial sums
+    __shared__ int abort_flag;
+    __shared__ float s_red[2];
+
+    const int bh = blockIdx.y, tid = threadIdx.x, lane = tid & 31;
+    const int rows_per_stage = kStageBytes / (4 * DH);       // 4, 8 or 16
+    const int tpr = DH / 8;                                   // threads per row: 64, 32 or 16
+    const int nstage = kStreamRows / rows_per_stage;
+    const int row_base = blockIdx.x * kStreamRows;
+    float *Cb = C + ((size_t)bh * DH + row_base) * DH;        // this CTA's 128 rows, contiguous
+    const size_t vec = (size_t)bh * DH;
+    const float inv_sqrt_d = rsqrtf((float)DH);
+
+    if (tid == 0) {
+        for (int s = 0; s < kRing; ++s) ts::mbar_init(&full[s], 1);
+        abort_flag = 0;
+        ts::fence_mbar_init();
+    }
+    __syncthreads();
+    int issued = 0;                           // bulk loads issued (thread 0)
+    auto load_stage = [&](int s) {            // thread 0 only
+        ++issued;
+        float *dst = ring + (s % kRing) * (kStageBytes / 4);
+        ts::mbar_arrive_expect_tx(&full[s % kRing], kStageBytes);
+        asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                     ::"r"(ts::smem_u32(dst)), "l"(Cb + (size_t)s * (kStageBytes / 4)), "r"(kStageBytes),
+                     "r"(ts::smem_u32(&full[s % kRing])) : "memory");
+    };
+    if (tid == 0)
+        for (int s = 0; s < min(kRing - 1, nstage); ++s) load_stage(s);
+
+    float m_new, fp, ip;
+    step_gates(i_pre[bh], f_pre[bh], m[bh], fgate_exp, m_new, fp, ip);
+    // this thread's 8 columns (the same in every stage) and its row inside a stage
+    const int col = 8 * (tid % tpr), rin = tid / tpr;
+    float kh[8], qv[8];
+    float nq = 0.f, kq = 0.f;
+    {
+        float a[4], b[4];
+        Vec4<T>::load(k + vec + col, a); Vec4<T>::load(k + vec + col + 4, b);
+        float c4[4], d4[4];
+        Vec4<T>::load(q + vec + col, c4); Vec4<T>::load(q + vec + col + 4, d4);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            kh[e] = a[e] * inv_sqrt_d; kh[e + 4] = b[e] * inv_sqrt_d;
+            qv[e] = c4[e]; qv[e + 4] = d4[e];
+        }
+        if (rin == 0) {                      // the first row's threads cover every column once
+            float nn[4], nm[4];
+            Vec4<float>::load(n + vec + col, nn); Vec4<float>::load(n + vec + col + 4, nm);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                nq += nn[e] * qv[e] + nm[e] * qv[e + 4];
+                kq += kh[e] * qv[e] + kh[e + 4] * qv[e + 4];
+            }
+        }
+    }
+    nq = warp_sum(nq);
+    kq = warp_sum(kq);
+    if (tid < tpr && lane == 0) { part[tid >> 5] = nq; part[8 + (tid >> 5)] = kq; }
+    __syncthreads();
+    if (tid == 0) {
+        float a = 0.f, b = 0.f;
+        for (int w = 0; w < (tpr + 31) / 32; ++w) { a += part[w]; b += part[8 + w]; }
+        s_red[0] = a; s_red[1] = b;
+    }
+    __syncthreads();
+    const float inv_denom = 1.f / fmaxf(fabsf(fp * s_red[0] + ip * s_red[1]), expf(-m_new));
+    __syncthreads();                          // part[] is reused below
+
+    bool ok = true;
+    for (int s = 0; s < nstage; ++s) {
+        if (tid == 0 && s + kRing - 1 < nstage) {
+            // the slot refilled here held stage s - 1, whose bulk store (the latest
+            // group) must have finished reading it
+            asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+            load_stage(s + kRing - 1);
+        }
+        const bool got = ts::mbar_wait(&full[s % kRing], (s / kRing) & 1, &abort_flag, status);
+        if (!__syncthreads_and(got)) { ok = false; break; }
+        float *st = ring + (s % kRing) * (kStageBytes / 4);
+        const int row = row_base + s * rows_per_stage + rin;          // row of the head
+        const float vr = to_f32(v[vec + row]) * ip;
+        float4 *cp = reinterpret_cast<float4 *>(st + rin * DH + col);
+        float4 x0 = cp[0], x1 = cp[1];
+        x0.x = fp * x0.x + vr * kh[0]; x0.y = fp * x0.y + vr * kh[1];
+        x0.z = fp * x0.z + vr * kh[2]; x0.w = fp * x0.w + vr * kh[3];
+        x1.x = fp * x1.x + vr * kh[4]; x1.y = fp * x1.y + vr * kh[5];
+        x1.z = fp * x1.z + vr * kh[6]; x1.w = fp * x1.w + vr * kh[7];
+        cp[0] = x0; cp[1] = x1;
+        float acc = x0.x * qv[0] + x0.y * qv[1] + x0.z * qv[2] + x0.w * qv[3] +
+                    x1.x * qv[4] + x1.y * qv[5] + x1.z * qv[6] + x1.w * qv[7];
+        // row sums over the row's tpr threads: two warps, one warp, or a half warp
+        if (tpr >= 32) {
+            acc = warp_sum(acc);
+            if (lane == 0) part[tid >> 5] = acc;
+        } else {
+#pragma unroll
+            for (int o = 8; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+            if ((lane & 15) == 0) part[tid >> 4] = acc;
+        }
+        ts::fence_async_smem();               // the updated stage leaves by bulk store
+        __syncthreads();
+        if (tid == 0) {
+            asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;"
+                         ::"l"(Cb + (size_t)s * (kStageBytes / 4)), "r"(ts::smem_u32(st)), "r"(kStageBytes)
+                         : "memory");
+            asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+        }
+        if (tid < rows_per_stage) {           // h for this stage's rows
+            const int r = row_base + s * rows_per_stage + tid;
+            const float dot = tpr == 64 ? part[2 * tid] + part[2 * tid + 1] : part[tid];
+            h[vec + r] = from_f32<T>(sigmoid(o_pre[vec + r]) * dot * inv_denom);
+        }
+        __syncthreads();                      // part[] is rewritten by the next stage
+    }
+    if (tid == 0) {                           // nothing in flight at exit
+        if (!ok)                              // loads issued but maybe not consumed
+            for (int t = max(0, issued - kRing); t < issued; ++t)
+                ts::mbar_wait(&full[t % kRing], (t / kRing) & 1, nullptr, status);
+        asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+    }
+}
+
 // n' <- f' n' + i' khat and m <- m_new, after step_rows_kernel has read them.
 template <typename T>
 __global__ void __launch_bounds__(128)
@@ -176,14 +323,30 @@ static cudaError_t launch_rows(const StepArgs &a, cudaStream_t st) {
 }
 
 template <typename T>
+static cudaError_t launch_stream(const StepArgs &a, cudaStream_t st) {
+    const int sm = kRing * kStageBytes + kRing * 8 + 256 * 4;
+    cudaError_t e = cudaFuncSetAttribute(step_stream_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
+    if (e != cudaSuccess) return e;
+    KernelTimer timer("step_rows", st);
+    step_stream_kernel<T><<<dim3(a.DH / kStreamRows, a.BH), 256, sm, st>>>(
+        (const T *)a.q, (const T *)a.k, (const T *)a.v, a.i_pre, a.f_pre, a.o_pre, (T *)a.h,
+        a.C, a.n, a.m, a.DH, a.fgate_exp, a.status);
+    return cudaGetLastError();
+}
+
+template <typename T>
 static cudaError_t launch_step_t(const StepArgs &a, cudaStream_t st) {
     cudaError_t e;
     const int nv = (a.DH + 127) / 128;
-    switch (nv) {
-        case 1: e = launch_rows<T, 1>(a, st); break;
-        case 2: e = launch_rows<T, 2>(a, st); break;
-        case 3: e = launch_rows<T, 3>(a, st); break;
-        default: e = launch_rows<T, 4>(a, st); break;
+    if (a.DH % kStreamRows == 0) {
+        e = launch_stream<T>(a, st);          // DH 128, 256, 512: bulk-copy stream
+    } else {
+        switch (nv) {
+            case 1: e = launch_rows<T, 1>(a, st); break;
+            case 2: e = launch_rows<T, 2>(a, st); break;
+            case 3: e = launch_rows<T, 3>(a, st); break;
+            default: e = launch_rows<T, 4>(a, st); break;
+        }
     }
     if (e != cudaSuccess) return e;
     KernelTimer timer("step_state", st);
