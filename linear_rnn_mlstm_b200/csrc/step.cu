@@ -11,12 +11,13 @@
 // everything else is O(DH).  Section 2.5 of the paper: constant memory in the
 // sequence length, so a decode step is a pure stream of the state.
 //
-// Two launches per step: step_rows_kernel splits each head's rows over several
-// CTAs (so the grid has many more CTAs than SMs and the tail wave is short)
-// and reads the OLD n' and m to form the shared denominator
+// Two launches per step.  The row update reads the OLD n' and m to form the
+// shared denominator
 //   n'_new . q = f' (n'_old . q) + i' (khat . q);
-// step_state_kernel then overwrites n' and m.  Keeping the two apart avoids
-// any CTA reading n'/m after another CTA wrote them.
+// for DH a multiple of 128 it is step_stream_kernel (the state streamed through
+// shared memory by bulk copies), else step_rows_kernel (rows split over CTAs,
+// staged in registers).  step_state_kernel then overwrites n' and m.  Keeping
+// the two apart avoids any CTA reading n'/m after another CTA wrote them.
 #include "common.cuh"
 #include "kernels.h"
 #include "profile.h"
