@@ -33,6 +33,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 from linear_rnn_mlstm_b200 import binding as xb  # noqa: E402
+from linear_rnn_mlstm_b200 import replicas  # noqa: E402
 from linear_rnn_mlstm_b200 import synthetic as syn  # noqa: E402
 
 METRIC = "mLSTM fwd tokens/s & % bf16 TC peak; decode-step HBM GB/s vs peak"
@@ -189,8 +190,7 @@ def cpu_baseline(w, max_tokens_per_head):
 
 
 def run_reference(args):
-    rank = int(os.environ.get("RANK", "0"))
-    if rank != 0:
+    if not replicas.rank_env().reports:      # under torchrun only rank 0 runs the oracle
         return 0
     import oracle
     w = syn.WORKLOADS[args.config]
@@ -253,9 +253,10 @@ def make_fwd_runner(x, w, chunk, dev, path):
     return run, (h, C, n, m), BH
 
 
-def time_region(fn, steps, dist_on, dev):
-    if dist_on:
-        torch.distributed.barrier()
+def time_region(fn, steps, env, dev):
+    """Device time of `steps` calls, between a barrier and a synchronize on both
+    sides; the max over ranks (every rank gets it)."""
+    replicas.barrier(env)
     torch.cuda.synchronize(dev)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
@@ -264,14 +265,8 @@ def time_region(fn, steps, dist_on, dev):
         fn()
     e1.record()
     torch.cuda.synchronize(dev)
-    if dist_on:
-        torch.distributed.barrier()
-    ms = e0.elapsed_time(e1)
-    if dist_on:
-        t = torch.tensor([ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
-    return ms
+    replicas.barrier(env)
+    return replicas.max_over_ranks(e0.elapsed_time(e1), env, dev)
 
 
 def plan_info(w, chunk, path):
@@ -308,23 +303,18 @@ def main():
     if args.impl == "reference":
         return run_reference(args)
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
-    dist_on = world > 1
+    env = replicas.rank_env()
+    world, rank, local_rank = env.world, env.rank, env.local_rank
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    if dist_on:
-        import datetime
-        torch.distributed.init_process_group("nccl", device_id=dev,
-                                             timeout=datetime.timedelta(seconds=300))
+    replicas.init(env, "nccl", dev, timeout_s=300)
     xb.load()
     peaks, peak_src = load_peaks()
     path = {"auto": xb.PATH_AUTO, "simt": xb.PATH_SIMT, "tensor": xb.PATH_TENSOR}[args.path]
 
     # ------------------------------------------------------------ forward
     w = syn.WORKLOADS[args.config]
-    inp = syn.fwd_inputs(w, seed=w.seed + rank)
+    inp = syn.fwd_inputs(w, seed=replicas.replica_seed(w.seed, rank))
     x = {k: v.to(dev).contiguous() for k, v in inp.items()}
     run, outs, BH = make_fwd_runner(x, w, args.chunk, dev, path)
     sampler = ClockSampler(physical_gpu_index(local_rank)) if rank == 0 else None
@@ -332,11 +322,11 @@ def main():
         run()
     torch.cuda.synchronize(dev)
     xb.xlstm_profile_begin()
-    ms = time_region(run, args.steps, dist_on, dev)
+    ms = time_region(run, args.steps, env, dev)
     _, kt = xb.xlstm_profile_end()
     ms_step = ms / args.steps
     tokens = w.B * w.NH * w.S
-    value = tokens * world / (ms_step * 1e-3)
+    value = replicas.job_throughput(tokens, env, ms_step * 1e-3)
     launches = sum(v[0] for v in kt.values())
     kernels = {k: {"launches": v[0], "avg_us": 1e3 * v[1] / max(v[0], 1),
                    "share": v[1] / max(sum(u[1] for u in kt.values()), 1e-12)}
@@ -378,17 +368,17 @@ def main():
                 hst.copy_(dv, non_blocking=True)
         for _ in range(2):
             e2e_step()
-        ms_e2e = time_region(e2e_step, max(3, min(args.steps, 10)), dist_on, dev) / max(3, min(args.steps, 10))
+        ms_e2e = time_region(e2e_step, max(3, min(args.steps, 10)), env, dev) / max(3, min(args.steps, 10))
         h2d = sum(t.numel() * t.element_size() for t in pin.values())
         d2h = sum(t.numel() * t.element_size() for t in out_host)
-        e2e = {"value": tokens * world / (ms_e2e * 1e-3), "unit": "tokens/s",
+        e2e = {"value": replicas.job_throughput(tokens, env, ms_e2e * 1e-3), "unit": "tokens/s",
                "ms_per_step": ms_e2e, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
     del x, outs, run
 
     # ----------------------------------------------------------------- decode
     decode = None
     if not args.skip_decode:
-        decode = run_decode(args, dev, dist_on, rank, world, peaks, peak_src)
+        decode = run_decode(args, dev, env, peaks, peak_src)
 
     clocks = sampler.stop() if sampler else None
 
@@ -411,27 +401,27 @@ def main():
                 "kernels": kernels, "gpu_launches": launches, "cpu_baseline": cpu, "e2e": e2e,
                 "clocks": clocks, "decode": decode}
         print(json.dumps(line), flush=True)
-    if dist_on:
-        torch.distributed.barrier()
-        torch.distributed.destroy_process_group()
+    replicas.barrier(env)
+    replicas.shutdown(env)
     return 0
 
 
-def run_decode(args, dev, dist_on, rank, world, peaks, peak_src):
+def run_decode(args, dev, env, peaks, peak_src):
+    rank, world = env.rank, env.world
     d = syn.DECODE
     if args.decode_B:
         import dataclasses
         d = dataclasses.replace(d, B=args.decode_B)
     T = args.decode_steps
     BH, DH = d.B * d.NH, d.DH
-    pre = syn.fwd_inputs(d.prefill(), seed=d.seed + rank)
+    pre = syn.fwd_inputs(d.prefill(), seed=replicas.replica_seed(d.seed, rank))
     x = {k: v.to(dev) for k, v in pre.items()}
     _, C, n, m = xb.mlstm_fwd(x["q"], x["k"], x["v"], x["i_pre"], x["f_pre"], x["o_pre"],
                               chunk=d.prefill_chunk, fgate=d.fgate)
     del x
     steps = []
     for t in range(T):
-        s = syn.step_inputs(d, t, seed=d.seed + rank)
+        s = syn.step_inputs(d, t, seed=replicas.replica_seed(d.seed, rank))
         steps.append({k: v.to(dev, non_blocking=False) for k, v in s.items()})
     h = torch.empty((d.B, d.NH, DH), dtype=torch.bfloat16, device=dev)
     stream = torch.cuda.current_stream(dev).cuda_stream
@@ -452,7 +442,7 @@ def run_decode(args, dev, dist_on, rank, world, peaks, peak_src):
     torch.cuda.synchronize(dev)
     cur[0] = 0
     xb.xlstm_profile_begin()
-    ms = time_region(one, T, dist_on, dev)
+    ms = time_region(one, T, env, dev)
     _, kt = xb.xlstm_profile_end()
     ms_step = ms / T
     step_bytes = BH * (8.0 * DH * DH + 8 * DH + 8) + BH * DH * (3 * 2 + 4 + 2) + BH * 8
@@ -463,7 +453,7 @@ def run_decode(args, dev, dist_on, rank, world, peaks, peak_src):
     ach = row_bytes / (rows_us * 1e-6) / 1e9 if rows_us > 0 else None
     return {"metric": "decode-step HBM GB/s", "value": gbs * world, "unit": "GB/s",
             "per_gpu_frac": gbs / peaks["hbm_gbs"], "ms_per_step": ms_step, "steps": T,
-            "tokens_per_s": BH * world / (ms_step * 1e-3),
+            "tokens_per_s": replicas.job_throughput(BH, env, ms_step * 1e-3),
             "algorithmic_bytes_per_step": step_bytes,
             "roofline": {"kernel": "step_rows", "bound": "hbm", "achieved": ach,
                          "peak": peaks["hbm_gbs"], "unit": "GB/s",
