@@ -209,6 +209,19 @@ typedef struct {
 xlstm_status xlstm_profile_begin(void);
 xlstm_status xlstm_profile_end(xlstm_kernel_time *out, int max, int *count);
 
+/*
+ * Self-test of the failure path (the paper has no counterpart).  Enqueues on
+ * `cuda_stream` one single-CTA kernel that waits, with the same bounded wait the
+ * forward and decode kernels use, on a shared-memory barrier that nothing
+ * completes; after about `limit_us` microseconds (1..1000000) the wait gives up
+ * and latches the device status word, and the kernel returns normally.  A
+ * following xlstm_device_status() then reports XLSTM_ERR_TIMEOUT (and clears
+ * the word).  No fault, trap or hang is involved; the context stays usable.
+ * Returns XLSTM_ERR_SHAPE for a limit out of range, XLSTM_ERR_CUDA if the
+ * launch fails.
+ */
+xlstm_status xlstm_selftest_wait_timeout(int limit_us, void *cuda_stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -26,7 +26,7 @@ PATH_AUTO, PATH_SIMT, PATH_TENSOR = 0, 1, 2
 EXPORTED = ("xlstm_abi_version", "xlstm_status_string", "xlstm_mlstm_fwd_workspace_size",
             "xlstm_mlstm_fwd_workspace_size_ex", "xlstm_mlstm_fwd", "xlstm_mlstm_fwd_ex",
             "xlstm_mlstm_step", "xlstm_device_status", "xlstm_profile_begin", "xlstm_profile_end",
-            "xlstm_mlstm_fwd_noalloc")
+            "xlstm_mlstm_fwd_noalloc", "xlstm_selftest_wait_timeout")
 NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
 
 
@@ -77,6 +77,8 @@ def load(path: str = LIB_PATH):
         lib.xlstm_mlstm_step.restype = i
         lib.xlstm_device_status.argtypes = [vp]
         lib.xlstm_device_status.restype = i
+        lib.xlstm_selftest_wait_timeout.argtypes = [i, vp]
+        lib.xlstm_selftest_wait_timeout.restype = i
         lib.xlstm_mlstm_fwd_noalloc.argtypes = [vp] * 3 + [fp] * 3 + [vp] + [fp] * 6 + [i] * 7 + [vp]
         lib.xlstm_mlstm_fwd_noalloc.restype = i
         lib.xlstm_profile_begin.restype = i
@@ -127,6 +129,10 @@ def xlstm_mlstm_step(q, k, v, i_pre, f_pre, o_pre, h, C, n, m, B, NH, DH, dt, fg
 
 def xlstm_device_status(stream) -> int:
     return load().xlstm_device_status(stream)
+
+
+def xlstm_selftest_wait_timeout(limit_us: int, stream) -> int:
+    return load().xlstm_selftest_wait_timeout(limit_us, stream)
 
 
 def xlstm_profile_begin() -> int:

@@ -12,6 +12,12 @@ namespace xlstm {
 
 __device__ unsigned int g_device_status = 0;
 
+// Address of the device status word on the current device (nullptr on failure).
+unsigned int *device_status_ptr() {
+    unsigned int *p = nullptr;
+    return cudaGetSymbolAddress((void **)&p, g_device_status) == cudaSuccess ? p : nullptr;
+}
+
 constexpr int kNumSms = 148;               // B200
 constexpr int kMaxHeads = 65535;           // B * NH rides in a grid dimension
 

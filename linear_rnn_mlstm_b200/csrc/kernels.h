@@ -20,6 +20,9 @@ struct FwdArgs {
     int fgate_exp;
 };
 
+// Address of the device status word on the current device (nullptr on failure).
+unsigned int *device_status_ptr();
+
 struct StepArgs {
     const void *q, *k, *v;
     const float *i_pre, *f_pre, *o_pre;
