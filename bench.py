@@ -5,7 +5,9 @@ bf16 q/k/v, fp32 gates and state) is the timed step; one step is one full
 forward over that batch (gate prologue, segment summaries, chunkwise outputs
 and final state).  The decode step workload (B=256, NH=8, DH=512, fp32 state,
 1024 consecutive tokens after a 512-token prefill) is timed in the same run and
-reported under "decode".  Inputs are seeded synthetic tensors of those shapes.
+reported under "decode", and the block epilogue after the cell (per-head
+GroupNorm, learnable skip, external output gate) on the forward's shape under
+"epilogue".  Inputs are seeded synthetic tensors of those shapes.
 
 Under torchrun (N > 1) every rank runs its own replica of the same workload on
 its own GPU (heads are independent, so the batch shards with no collective);
@@ -86,7 +88,8 @@ def source_sha(kernel):
     """sha1 of the source files a kernel is built from (the tensor-core kernels
     also depend on the tcgen05/TMA wrappers)."""
     files = {"segment_output_simt": ["fwd_simt.cu"], "segment_summary_simt": ["fwd_simt.cu"],
-             "gate_prologue": ["fwd_simt.cu"], "step_rows": ["step.cu"], "step_state": ["step.cu"]}
+             "gate_prologue": ["fwd_simt.cu"], "step_rows": ["step.cu"], "step_state": ["step.cu"],
+             "headnorm_gate": ["headnorm.cu"]}
     fns = files.get(kernel)
     if fns is None and kernel.endswith("_tc"):
         fns = ["fwd_tc.cu", "tc_ptx.cuh"]
@@ -294,6 +297,7 @@ def main():
                     help="batch of the decode workload (0 = its full B of 256); profiling only")
     ap.add_argument("--skip-decode", action="store_true")
     ap.add_argument("--skip-e2e", action="store_true")
+    ap.add_argument("--skip-epilogue", action="store_true")
     ap.add_argument("--skip-cpu", action="store_true")
     ap.add_argument("--ref-tokens", type=int, default=4096,
                     help="tokens per head in each reference (oracle) step")
@@ -375,6 +379,11 @@ def main():
                "ms_per_step": ms_e2e, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
     del x, outs, run
 
+    # -------------------------------------------------- block epilogue (next row)
+    epilogue = None
+    if not args.skip_epilogue:
+        epilogue = run_epilogue(args, w, dev, env, peaks, peak_src)
+
     # ----------------------------------------------------------------- decode
     decode = None
     if not args.skip_decode:
@@ -399,11 +408,51 @@ def main():
                                path=args.path),
                 "roofline": roofline, "tc": tc, "hbm_whole_step": whole,
                 "kernels": kernels, "gpu_launches": launches, "cpu_baseline": cpu, "e2e": e2e,
-                "clocks": clocks, "decode": decode}
+                "clocks": clocks, "decode": decode, "epilogue": epilogue}
         print(json.dumps(line), flush=True)
     replicas.barrier(env)
     replicas.shutdown(env)
     return 0
+
+
+def run_epilogue(args, w, dev, env, peaks, peak_src):
+    """The mLSTM block's epilogue after the cell (per-head GroupNorm, learnable
+    skip, SiLU external output gate) on the forward workload's shape, timed
+    alone: h [B,NH,S,DH] -> y [B,S,NH*DH]."""
+    B, NH, S, DH = w.B, w.NH, w.S, w.DH
+    inp = syn.epilogue_inputs(B, NH, S, DH, w.dtype, seed=replicas.replica_seed(w.seed, env.rank))
+    x = {k: v.to(dev).contiguous() for k, v in inp.items()}
+    y = torch.empty(x["x_skip"].shape, dtype=x["h"].dtype, device=dev)
+    dt = xb.BF16 if w.dtype == "bf16" else xb.F32
+    stream = torch.cuda.current_stream(dev).cuda_stream
+    ptrs = [x[k].data_ptr() for k in ("h", "gamma", "beta", "skip_w", "x_skip", "z")]
+
+    def one():
+        st = xb.xlstm_mlstm_headnorm_gate(*ptrs, y.data_ptr(), B, NH, S, DH, 1e-5, dt,
+                                          xb.OGATE_SILU, stream)
+        if st != xb.OK:
+            raise xb.XlstmError(st, "xlstm_mlstm_headnorm_gate")
+    for _ in range(max(3, args.warmup)):
+        one()
+    torch.cuda.synchronize(dev)
+    steps = max(10, args.steps)
+    xb.xlstm_profile_begin()
+    ms = time_region(one, steps, env, dev)
+    _, kt = xb.xlstm_profile_end()
+    rows = B * S * NH
+    eb = 2 if w.dtype == "bf16" else 4
+    alg = rows * DH * 4 * eb + 3 * 4 * NH * DH         # h, x_skip, z in; y out; 3 parameter rows
+    k = kt.get("headnorm_gate", (0, 0.0))
+    us = 1e3 * k[1] / max(k[0], 1)
+    ach = alg / (us * 1e-6) / 1e9 if us > 0 else None
+    return {"kernel": "headnorm_gate", "us_per_launch": us, "ms_per_call": ms / steps,
+            "launches": k[0],
+            "roofline": {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": (ach / peaks["hbm_gbs"]) if ach else None,
+                         "traffic": ncu_traffic("headnorm_gate", rows), "algorithmic_bytes": alg,
+                         "peak_source": f"{peak_src} (burst copy)"},
+            "config": f"block epilogue: h [{B},{NH},{S},{DH}] {w.dtype} -> y [{B},{S},{NH * DH}], "
+                      f"skip on, SiLU gate, eps 1e-5; {alg / 1e6:.0f} MB per launch (> L2)"}
 
 
 def run_decode(args, dev, env, peaks, peak_src):

@@ -46,7 +46,7 @@ typedef enum {
     XLSTM_OK = 0,
     XLSTM_ERR_NULL = 1,        /* a required pointer is NULL                       */
     XLSTM_ERR_SHAPE = 2,       /* a size is negative, DH unsupported, or too large */
-    XLSTM_ERR_DTYPE = 3,       /* dtype or forget-gate kind out of range           */
+    XLSTM_ERR_DTYPE = 3,       /* dtype or gate kind out of range                  */
     XLSTM_ERR_CHUNK = 4,       /* chunk size not supported for this dtype          */
     XLSTM_ERR_ALIGN = 5,       /* a pointer is not 16-byte aligned                 */
     XLSTM_ERR_CUDA = 6,        /* a CUDA runtime call or kernel launch failed      */
@@ -57,6 +57,8 @@ typedef enum {
 
 typedef enum { XLSTM_F32 = 0, XLSTM_BF16 = 1 } xlstm_dtype;          /* dtype of q, k, v, h */
 typedef enum { XLSTM_FGATE_SIGMOID = 0, XLSTM_FGATE_EXP = 1 } xlstm_fgate;
+/* Activation of the mLSTM block's external output gate (xlstm_mlstm_headnorm_gate). */
+typedef enum { XLSTM_OGATE_SILU = 0, XLSTM_OGATE_SIGMOID = 1 } xlstm_ogate;
 
 /* Kernel family for the forward.  AUTO picks the tensor-core (tcgen05) kernels
  * for bf16 inputs with DH 128 or 256 and chunk 64, and the fp32 SIMT kernels
@@ -183,6 +185,41 @@ xlstm_status xlstm_mlstm_step(const void *q, const void *k, const void *v,
                               void *h, float *C, float *n, float *m,
                               int B, int NH, int DH, xlstm_dtype dt, xlstm_fgate fg,
                               void *cuda_stream);
+
+/*
+ * The mLSTM block's epilogue after the cell ("xLSTM: Extended Long Short-Term
+ * Memory" section 2.4, Figure 10): the cell output is normalised by a GroupNorm
+ * whose groups are the heads (a LayerNorm over each head's DH channels, per
+ * token; GroupNorm as defined by Wu & He: biased variance, eps inside the square
+ * root, per-channel scale and shift), the learnable skip input is added, and the
+ * sum is gated component-wise by the block's external output gate.  One pass;
+ * the output is in the block's layout, ready for the down-projection:
+ *
+ *   y[b, t, c] = ((h[b, hd, t, j] - mean) / sqrt(var + eps) * gamma[c] + beta[c]
+ *                 + skip_w[c] * x_skip[b, t, c]) * act(z[b, t, c]),
+ *   c = hd * DH + j,  mean / var over j of h[b, hd, t, :],
+ *   act(z) = z * sigmoid(z) (XLSTM_OGATE_SILU) or sigmoid(z) (XLSTM_OGATE_SIGMOID).
+ *
+ *   h            [B, NH, S, DH]  dtype dt, the cell output (as xlstm_mlstm_fwd
+ *                writes it; run the cell with o_pre = +inf for the block's form,
+ *                where the output gate is outside the cell)
+ *   gamma, beta  [NH * DH]       float, GroupNorm scale and shift per channel
+ *   skip_w       [NH * DH]       float, learnable skip weight per channel
+ *   x_skip       [B, S, NH * DH] dtype dt, skip input (the cell input after the
+ *                block's causal convolution); skip_w and x_skip are both NULL
+ *                (no skip term) or both given
+ *   z            [B, S, NH * DH] dtype dt, external output-gate pre-activation
+ *   y            [B, S, NH * DH] dtype dt, output; must not be any input buffer
+ *                (the same pointer passed twice is rejected with
+ *                XLSTM_ERR_UNSUPPORTED)
+ *   eps          > 0 and finite (else XLSTM_ERR_UNSUPPORTED)
+ * DH: multiple of 16 in [16, 512].  B, NH or S == 0 is a no-op.  Statistics
+ * and arithmetic are fp32; y is rounded once to dt.
+ */
+xlstm_status xlstm_mlstm_headnorm_gate(const void *h, const float *gamma, const float *beta,
+                                       const float *skip_w, const void *x_skip, const void *z,
+                                       void *y, int B, int NH, int S, int DH, float eps,
+                                       xlstm_dtype dt, xlstm_ogate og, void *cuda_stream);
 
 /*
  * Synchronises `cuda_stream`, then reads and clears the device status word of

@@ -21,12 +21,13 @@ OK, ERR_NULL, ERR_SHAPE, ERR_DTYPE, ERR_CHUNK, ERR_ALIGN, ERR_CUDA, ERR_TIMEOUT,
     ERR_WORKSPACE, ERR_UNSUPPORTED = range(10)
 F32, BF16 = 0, 1
 FGATE_SIGMOID, FGATE_EXP = 0, 1
+OGATE_SILU, OGATE_SIGMOID = 0, 1
 PATH_AUTO, PATH_SIMT, PATH_TENSOR = 0, 1, 2
 
 EXPORTED = ("xlstm_abi_version", "xlstm_status_string", "xlstm_mlstm_fwd_workspace_size",
             "xlstm_mlstm_fwd_workspace_size_ex", "xlstm_mlstm_fwd", "xlstm_mlstm_fwd_ex",
             "xlstm_mlstm_step", "xlstm_device_status", "xlstm_profile_begin", "xlstm_profile_end",
-            "xlstm_mlstm_fwd_noalloc", "xlstm_selftest_wait_timeout")
+            "xlstm_mlstm_fwd_noalloc", "xlstm_selftest_wait_timeout", "xlstm_mlstm_headnorm_gate")
 NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
 
 
@@ -81,6 +82,9 @@ def load(path: str = LIB_PATH):
         lib.xlstm_selftest_wait_timeout.restype = i
         lib.xlstm_mlstm_fwd_noalloc.argtypes = [vp] * 3 + [fp] * 3 + [vp] + [fp] * 6 + [i] * 7 + [vp]
         lib.xlstm_mlstm_fwd_noalloc.restype = i
+        lib.xlstm_mlstm_headnorm_gate.argtypes = [vp] + [fp] * 3 + [vp] * 3 + [i] * 4 + \
+            [ctypes.c_float, i, i, vp]
+        lib.xlstm_mlstm_headnorm_gate.restype = i
         lib.xlstm_profile_begin.restype = i
         lib.xlstm_profile_end.argtypes = [ctypes.POINTER(KernelTime), i, ctypes.POINTER(i)]
         lib.xlstm_profile_end.restype = i
@@ -125,6 +129,12 @@ def xlstm_mlstm_fwd_noalloc(q, k, v, i_pre, f_pre, o_pre, h, C0, n0, m0, C_out, 
 def xlstm_mlstm_step(q, k, v, i_pre, f_pre, o_pre, h, C, n, m, B, NH, DH, dt, fg, stream):
     return load().xlstm_mlstm_step(q, k, v, i_pre, f_pre, o_pre, h, C, n, m, B, NH, DH, dt, fg,
                                    stream)
+
+
+def xlstm_mlstm_headnorm_gate(h, gamma, beta, skip_w, x_skip, z, y, B, NH, S, DH, eps, dt, og,
+                              stream):
+    return load().xlstm_mlstm_headnorm_gate(h, gamma, beta, skip_w, x_skip, z, y, B, NH, S, DH,
+                                            float(eps), dt, og, stream)
 
 
 def xlstm_device_status(stream) -> int:
@@ -246,3 +256,29 @@ def mlstm_step(q, k, v, i_pre, f_pre, o_pre, C, n, m, fgate="sigmoid", h=None):
     if st != OK:
         raise XlstmError(st, "xlstm_mlstm_step")
     return h
+
+
+def mlstm_headnorm_gate(h, gamma, beta, z, skip_w=None, x_skip=None, eps=1e-5, ogate="silu",
+                        y=None):
+    """Block epilogue after the cell: per-head GroupNorm of h [B, NH, S, DH],
+    plus skip_w * x_skip, gated by act(z); x_skip, z and the returned y are
+    [B, S, NH * DH].  Returns y."""
+    torch = _torch()
+    B, NH, S, DH = h.shape
+    dev, dtype, dt = h.device, h.dtype, _dt(h)
+    _check(h, "h", (B, NH, S, DH), dtype, dev)
+    for t, nm in ((gamma, "gamma"), (beta, "beta"), (skip_w, "skip_w")):
+        _check(t, nm, (NH * DH,), torch.float32, dev)
+    _check(x_skip, "x_skip", (B, S, NH * DH), dtype, dev)
+    _check(z, "z", (B, S, NH * DH), dtype, dev)
+    if y is None:
+        y = torch.empty((B, S, NH * DH), dtype=dtype, device=dev)
+    _check(y, "y", (B, S, NH * DH), dtype, dev)
+    if ogate not in ("silu", "sigmoid"):
+        raise ValueError("ogate must be 'silu' or 'sigmoid'")
+    og = OGATE_SILU if ogate == "silu" else OGATE_SIGMOID
+    st = xlstm_mlstm_headnorm_gate(_ptr(h), _ptr(gamma), _ptr(beta), _ptr(skip_w), _ptr(x_skip),
+                                   _ptr(z), _ptr(y), B, NH, S, DH, eps, dt, og, _stream(dev))
+    if st != OK:
+        raise XlstmError(st, "xlstm_mlstm_headnorm_gate")
+    return y

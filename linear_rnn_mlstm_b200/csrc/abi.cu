@@ -144,7 +144,7 @@ const char *xlstm_status_string(xlstm_status s) {
         case XLSTM_OK: return "ok";
         case XLSTM_ERR_NULL: return "a required pointer is NULL";
         case XLSTM_ERR_SHAPE: return "unsupported or inconsistent shape";
-        case XLSTM_ERR_DTYPE: return "unsupported dtype or forget-gate kind";
+        case XLSTM_ERR_DTYPE: return "unsupported dtype or gate kind";
         case XLSTM_ERR_CHUNK: return "unsupported chunk size for this dtype";
         case XLSTM_ERR_ALIGN: return "a pointer is not 16-byte aligned";
         case XLSTM_ERR_CUDA: return "CUDA runtime or launch error";

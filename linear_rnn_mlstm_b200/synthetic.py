@@ -133,3 +133,25 @@ def step_inputs(d: DecodeWorkload, step: int, seed: Optional[int] = None) -> dic
 def custom(name: str, B: int, NH: int, S: int, DH: int, base: Workload = SMALL, **kw) -> Workload:
     """A workload with ``base``'s distributions and the given shape."""
     return replace(base, name=name, B=B, NH=NH, S=S, DH=DH, **kw)
+
+
+def epilogue_inputs(B: int, NH: int, S: int, DH: int, dtype: str = "bf16", seed: int = 0,
+                    skip: bool = True) -> dict:
+    """CPU tensors for the block epilogue after the cell (per-head GroupNorm,
+    learnable skip, external output gate): h [B,NH,S,DH] and x_skip, z
+    [B,S,NH*DH] in ``dtype``; gamma, beta, skip_w [NH*DH] float32.  Scale and
+    shift near their identity initialisation; h with a non-zero mean so that
+    the centring matters.  Drawn in the order h, gamma, beta, skip_w, x_skip, z."""
+    g = _gen(seed)
+    dt = _qkv_dtype(dtype)
+    D = NH * DH
+    h = (torch.randn((B, NH, S, DH), generator=g, dtype=torch.float32) * 1.5 + 0.3).to(dt)
+    gamma = torch.randn(D, generator=g, dtype=torch.float32) * 0.1 + 1.0
+    beta = torch.randn(D, generator=g, dtype=torch.float32) * 0.1
+    skip_w = torch.randn(D, generator=g, dtype=torch.float32) * 0.5
+    x_skip = torch.randn((B, S, D), generator=g, dtype=torch.float32).to(dt)
+    z = torch.randn((B, S, D), generator=g, dtype=torch.float32).to(dt)
+    out = dict(h=h, gamma=gamma, beta=beta, z=z)
+    if skip:
+        out.update(skip_w=skip_w, x_skip=x_skip)
+    return out

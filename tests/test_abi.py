@@ -117,3 +117,40 @@ def _step(**over):
 ])
 def test_step_rejects_bad_arguments_before_device_work(over, expect):
     assert _step(**over) == expect
+
+
+def _headnorm(**over):
+    # distinct aligned fake addresses, so that only the aliasing cases alias
+    a = dict(h=FAKE, gamma=FAKE + 16, beta=FAKE + 32, skip_w=FAKE + 48, x_skip=FAKE + 64,
+             z=FAKE + 80, y=FAKE + 96, B=1, NH=2, S=8, DH=64, eps=1e-5, dt=xb.BF16,
+             og=xb.OGATE_SILU, stream=None)
+    a.update(over)
+    return xb.xlstm_mlstm_headnorm_gate(**a)
+
+
+@pytest.mark.parametrize("over,expect", [
+    (dict(h=None), xb.ERR_NULL),
+    (dict(gamma=None), xb.ERR_NULL),
+    (dict(z=None), xb.ERR_NULL),
+    (dict(y=None), xb.ERR_NULL),
+    (dict(skip_w=None), xb.ERR_NULL),                    # skip weight without the skip input
+    (dict(x_skip=None), xb.ERR_NULL),
+    (dict(z=FAKE + 88), xb.ERR_ALIGN),
+    (dict(beta=FAKE + 36), xb.ERR_ALIGN),
+    (dict(dt=2), xb.ERR_DTYPE),
+    (dict(og=2), xb.ERR_DTYPE),
+    (dict(DH=40), xb.ERR_SHAPE),
+    (dict(DH=528), xb.ERR_SHAPE),
+    (dict(S=-1), xb.ERR_SHAPE),
+    (dict(eps=0.0), xb.ERR_UNSUPPORTED),
+    (dict(eps=-1e-5), xb.ERR_UNSUPPORTED),
+    (dict(eps=float("nan")), xb.ERR_UNSUPPORTED),
+    (dict(eps=float("inf")), xb.ERR_UNSUPPORTED),
+    (dict(y=FAKE), xb.ERR_UNSUPPORTED),                  # y is h
+    (dict(y=FAKE + 80), xb.ERR_UNSUPPORTED),             # y is z
+    (dict(y=FAKE + 64), xb.ERR_UNSUPPORTED),             # y is x_skip
+    (dict(S=0), xb.OK),                                  # no tokens: a no-op
+    (dict(B=0, h=None, y=None), xb.OK),
+])
+def test_headnorm_gate_rejects_bad_arguments_before_device_work(over, expect):
+    assert _headnorm(**over) == expect
