@@ -13,10 +13,12 @@
 // arithmetic, so it is bound by HBM bandwidth.  Each row is one contiguous run
 // of DH elements in every tensor; a group of LPR lanes (a power of two, up to
 // a warp) covers a row with 16-byte vectors, so a warp handles 32 / LPR rows
-// and every access is a full 16-byte load or store.  The row statistics are
-// two butterfly sums over the lane group (mean first, then the centred squares,
-// from values held in registers).  Streaming loads and stores keep the
-// per-row tensors from displacing the per-channel parameters in L2.
+// and every access is a full 16-byte load or store.  A lane group issues the
+// loads of its next rows before it reduces any of them.  The row statistics
+// are two butterfly sums over the lane group (mean first, then the centred
+// squares, from values held in registers).  Streaming loads and stores keep
+// the per-row tensors from displacing the per-channel parameters in L2.  The
+// grid is one resident wave of CTAs; each warp strides over the rows.
 #include <math.h>
 #include <stdint.h>
 
@@ -30,10 +32,10 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kNumSms = 148;           // B200
 
-// Elements per 16-byte vector, and the most vectors one lane holds (DH <= 512).
+// Elements per 16-byte vector.
 template <typename T> struct Vec;
-template <> struct Vec<float> { static constexpr int N = 4; static constexpr int kMax = 4; };
-template <> struct Vec<__nv_bfloat16> { static constexpr int N = 8; static constexpr int kMax = 2; };
+template <> struct Vec<float> { static constexpr int N = 4; };
+template <> struct Vec<__nv_bfloat16> { static constexpr int N = 8; };
 
 template <typename T> __device__ __forceinline__ void unpack(const uint4 &u, float *f);
 template <> __device__ __forceinline__ void unpack<float>(const uint4 &u, float *f) {
@@ -73,96 +75,139 @@ template <int LPR> __device__ __forceinline__ float group_sum(float x) {
     return x;
 }
 
+// The gate's logistic function without branches, from CUDA's fast exponential
+// and division intrinsics: relative error ~1e-6 for |z| < 10 (far below the
+// bf16 output rounding and the fp32 tolerance), exactly 1 at +inf and 0 at
+// -inf.  An accurate expf with an IEEE division on each side of a sign branch
+// made the gate, not HBM, the limit of this kernel.
 __device__ __forceinline__ float external_gate(float z, int silu) {
-    const float s = sigmoid(z);
+    const float s = __fdividef(1.f, 1.f + __expf(-z));
     return silu ? z * s : s;
 }
 
-template <typename T, int LPR>
+// Row r = (b * S + t) * NH + head -> (b, t, head); 32-bit division when the
+// row count allows it (the branch is uniform over the grid).
+__device__ __forceinline__ void split_row(long long r, int S, int NH, bool narrow, long long &b,
+                                          long long &t, int &head) {
+    if (narrow) {
+        const unsigned ur = (unsigned)r, bt = ur / (unsigned)NH, ub = bt / (unsigned)S;
+        head = (int)(ur - bt * (unsigned)NH);
+        b = ub;
+        t = bt - ub * (unsigned)S;
+    } else {
+        const long long bt = r / NH;
+        head = (int)(r - bt * NH);
+        b = bt / S;
+        t = bt - b * S;
+    }
+}
+
+// Rows a lane group takes per pass when each lane holds V 16-byte vectors of a
+// row: two vectors of each of h, z and x_skip in flight per lane.  (Four, with
+// ~120 registers and two CTAs per SM, measured slower than two with ~66
+// registers and three CTAs per SM.)
+__host__ __device__ constexpr int rows_per_pass(int V) { return V >= 2 ? 1 : 2 / V; }
+
+// LPR lanes per row, V 16-byte vectors per lane and row (LPR * V * VN >= DH),
+// R rows per lane group per pass: every load of a pass is issued before the
+// first row's statistics wait on them.
+template <typename T, int LPR, int V>
 __global__ void __launch_bounds__(kThreads)
 headnorm_gate_kernel(const T *__restrict__ h, const float *__restrict__ gamma,
                      const float *__restrict__ beta, const float *__restrict__ skip_w,
                      const T *__restrict__ x_skip, const T *__restrict__ z, T *__restrict__ y,
                      long long rows, int S, int NH, int DH, float eps, int silu) {
     constexpr int VN = Vec<T>::N;
-    constexpr int kMaxV = Vec<T>::kMax;
+    constexpr int R = rows_per_pass(V);
     constexpr int kRowsPerWarp = 32 / LPR;
+    constexpr int kRowsPerPass = kRowsPerWarp * R;
     const int lane = threadIdx.x & 31;
     const int sub = lane % LPR;
     const int slot = lane / LPR;
     const int nvec = DH / VN;
+    const bool narrow = rows < (1LL << 31);
     const long long warp = ((long long)blockIdx.x * kThreads + threadIdx.x) >> 5;
     const long long nwarps = ((long long)gridDim.x * kThreads) >> 5;
 
     // `base` is the same for every lane of the warp, so the shuffles below
     // always run with the whole warp.
-    for (long long base = warp * kRowsPerWarp; base < rows; base += nwarps * kRowsPerWarp) {
-        const long long r = base + slot;          // r = (b * S + t) * NH + head
-        const bool valid = r < rows;
-        const long long bt = valid ? r / NH : 0;
-        const int head = valid ? (int)(r - bt * NH) : 0;
-        const long long b = bt / S, t = bt - b * S;
-        const T *hrow = h + (((size_t)b * NH + head) * S + t) * DH;
-        const size_t yoff = (size_t)(valid ? r : 0) * DH;
-
-        float hv[kMaxV][VN];
-        uint4 zr[kMaxV], xr[kMaxV];
-        float sum = 0.f;
+    for (long long base = warp * kRowsPerPass; base < rows; base += nwarps * kRowsPerPass) {
+        uint4 hr[R][V], zr[R][V], xr[R][V];
+        size_t yoff[R];
+        int head[R];
+        bool valid[R];
 #pragma unroll
-        for (int k = 0; k < kMaxV; ++k) {
-            const int v = sub + k * LPR;
-            zr[k] = make_uint4(0, 0, 0, 0);
-            xr[k] = make_uint4(0, 0, 0, 0);
-            if (valid && v < nvec) {
-                unpack<T>(__ldcs(reinterpret_cast<const uint4 *>(hrow) + v), hv[k]);
-                zr[k] = __ldcs(reinterpret_cast<const uint4 *>(z + yoff) + v);
-                if (x_skip) xr[k] = __ldcs(reinterpret_cast<const uint4 *>(x_skip + yoff) + v);
-            } else {
+        for (int j = 0; j < R; ++j) {
+            const long long r = base + j * kRowsPerWarp + slot;
+            valid[j] = r < rows;
+            long long b = 0, t = 0;
+            head[j] = 0;
+            if (valid[j]) split_row(r, S, NH, narrow, b, t, head[j]);
+            const T *hrow = h + (((size_t)b * NH + head[j]) * S + t) * DH;
+            yoff[j] = (size_t)(valid[j] ? r : 0) * DH;
 #pragma unroll
-                for (int e = 0; e < VN; ++e) hv[k][e] = 0.f;
-            }
-#pragma unroll
-            for (int e = 0; e < VN; ++e) sum += hv[k][e];
-        }
-        // true divisions: a constant row gives exactly its value as the mean
-        const float mean = group_sum<LPR>(sum) / (float)DH;
-        float sq = 0.f;
-#pragma unroll
-        for (int k = 0; k < kMaxV; ++k) {
-            if (valid && sub + k * LPR < nvec) {
-#pragma unroll
-                for (int e = 0; e < VN; ++e) {
-                    const float d = hv[k][e] - mean;
-                    sq += d * d;
+            for (int k = 0; k < V; ++k) {
+                const int v = sub + k * LPR;
+                hr[j][k] = zr[j][k] = xr[j][k] = make_uint4(0, 0, 0, 0);
+                if (valid[j] && v < nvec) {
+                    hr[j][k] = __ldcs(reinterpret_cast<const uint4 *>(hrow) + v);
+                    zr[j][k] = __ldcs(reinterpret_cast<const uint4 *>(z + yoff[j]) + v);
+                    if (x_skip)
+                        xr[j][k] = __ldcs(reinterpret_cast<const uint4 *>(x_skip + yoff[j]) + v);
                 }
             }
         }
-        const float rstd = rsqrtf(group_sum<LPR>(sq) / (float)DH + eps);
-
 #pragma unroll
-        for (int k = 0; k < kMaxV; ++k) {
-            const int v = sub + k * LPR;
-            if (!valid || v >= nvec) continue;
-            const int c0 = head * DH + v * VN;
-            float zf[VN], xf[VN], out[VN];
-            unpack<T>(zr[k], zf);
-            unpack<T>(xr[k], xf);
+        for (int j = 0; j < R; ++j) {
+            // vectors that were not loaded are zero and add nothing to the sum
+            float hv[V][VN];
+            float sum = 0.f;
 #pragma unroll
-            for (int e = 0; e < VN; e += 4) {
-                const float4 g = __ldg(reinterpret_cast<const float4 *>(gamma + c0 + e));
-                const float4 bb = __ldg(reinterpret_cast<const float4 *>(beta + c0 + e));
-                float4 sw = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (x_skip) sw = __ldg(reinterpret_cast<const float4 *>(skip_w + c0 + e));
-                const float gs[4] = {g.x, g.y, g.z, g.w}, bs[4] = {bb.x, bb.y, bb.z, bb.w},
-                            ss[4] = {sw.x, sw.y, sw.z, sw.w};
+            for (int k = 0; k < V; ++k) {
+                unpack<T>(hr[j][k], hv[k]);
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const float xn = (hv[k][e + i] - mean) * rstd;
-                    out[e + i] = (xn * gs[i] + bs[i] + ss[i] * xf[e + i]) *
-                                 external_gate(zf[e + i], silu);
+                for (int e = 0; e < VN; ++e) sum += hv[k][e];
+            }
+            // true divisions: a constant row gives exactly its value as the mean
+            const float mean = group_sum<LPR>(sum) / (float)DH;
+            float sq = 0.f;
+#pragma unroll
+            for (int k = 0; k < V; ++k) {
+                if (sub + k * LPR < nvec) {
+#pragma unroll
+                    for (int e = 0; e < VN; ++e) {
+                        const float d = hv[k][e] - mean;
+                        sq += d * d;
+                    }
                 }
             }
-            __stcs(reinterpret_cast<uint4 *>(y + yoff) + v, pack<T>(out));
+            const float rstd = rsqrtf(group_sum<LPR>(sq) / (float)DH + eps);
+
+#pragma unroll
+            for (int k = 0; k < V; ++k) {
+                const int v = sub + k * LPR;
+                if (!valid[j] || v >= nvec) continue;
+                const int c0 = head[j] * DH + v * VN;
+                float zf[VN], xf[VN], out[VN];
+                unpack<T>(zr[j][k], zf);
+                unpack<T>(xr[j][k], xf);
+#pragma unroll
+                for (int e = 0; e < VN; e += 4) {
+                    const float4 g = __ldg(reinterpret_cast<const float4 *>(gamma + c0 + e));
+                    const float4 bb = __ldg(reinterpret_cast<const float4 *>(beta + c0 + e));
+                    float4 sw = make_float4(0.f, 0.f, 0.f, 0.f);
+                    if (x_skip) sw = __ldg(reinterpret_cast<const float4 *>(skip_w + c0 + e));
+                    const float gs[4] = {g.x, g.y, g.z, g.w}, bs[4] = {bb.x, bb.y, bb.z, bb.w},
+                                ss[4] = {sw.x, sw.y, sw.z, sw.w};
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const float xn = (hv[k][e + i] - mean) * rstd;
+                        out[e + i] = (xn * gs[i] + bs[i] + ss[i] * xf[e + i]) *
+                                     external_gate(zf[e + i], silu);
+                    }
+                }
+                __stcs(reinterpret_cast<uint4 *>(y + yoff[j]) + v, pack<T>(out));
+            }
         }
     }
 }
@@ -175,11 +220,11 @@ int lanes_per_row(int nvec) {
 
 // CTAs of one instantiation resident per SM (registers decide it); the grid is
 // one full wave of them and each warp strides over the rows.
-template <typename T, int LPR> int resident_blocks() {
+template <typename T, int LPR, int V> int resident_blocks() {
     static int n = 0;
     if (n == 0) {
         int b = 0;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, headnorm_gate_kernel<T, LPR>,
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, headnorm_gate_kernel<T, LPR, V>,
                                                           kThreads, 0) != cudaSuccess || b < 1)
             b = 1;
         n = b;
@@ -191,28 +236,31 @@ template <typename T>
 cudaError_t launch_typed(const T *h, const float *gamma, const float *beta, const float *skip_w,
                          const T *x_skip, const T *z, T *y, long long rows, int S, int NH, int DH,
                          float eps, int silu, cudaStream_t st) {
-    const int lpr = lanes_per_row(DH / Vec<T>::N);
-    const long long rows_per_block = (long long)(kThreads / 32) * (32 / lpr);
-    const long long needed = (rows + rows_per_block - 1) / rows_per_block;
+    const int nvec = DH / Vec<T>::N;
+    const int lpr = lanes_per_row(nvec);
+    int vpl = (nvec + lpr - 1) / lpr;                 // vectors per lane: 1, 2, 3 or 4
+    if (vpl == 3) vpl = 4;
     KernelTimer timer("headnorm_gate", st);
-#define XLSTM_HN_CASE(L)                                                                       \
-    case L: {                                                                                  \
-        const long long wave = (long long)kNumSms * resident_blocks<T, L>();                  \
+#define XLSTM_HN_CASE(L, V)                                                                    \
+    if (lpr == L && vpl == V) {                                                                \
+        const long long per_block = (long long)(kThreads / 32) * (32 / L) * rows_per_pass(V);  \
+        const long long needed = (rows + per_block - 1) / per_block;                           \
+        const long long wave = (long long)kNumSms * resident_blocks<T, L, V>();               \
         const dim3 grid((unsigned)(needed < wave ? needed : wave));                            \
-        headnorm_gate_kernel<T, L><<<grid, kThreads, 0, st>>>(h, gamma, beta, skip_w, x_skip, \
-                                                              z, y, rows, S, NH, DH, eps, silu); \
-        break;                                                                                 \
+        headnorm_gate_kernel<T, L, V><<<grid, kThreads, 0, st>>>(h, gamma, beta, skip_w,       \
+                                                                 x_skip, z, y, rows, S, NH, DH, \
+                                                                 eps, silu);                   \
+        return cudaGetLastError();                                                             \
     }
-    switch (lpr) {
-        XLSTM_HN_CASE(2)
-        XLSTM_HN_CASE(4)
-        XLSTM_HN_CASE(8)
-        XLSTM_HN_CASE(16)
-        XLSTM_HN_CASE(32)
-        default: return cudaErrorInvalidValue;
-    }
+    XLSTM_HN_CASE(2, 1)
+    XLSTM_HN_CASE(4, 1)
+    XLSTM_HN_CASE(8, 1)
+    XLSTM_HN_CASE(16, 1)
+    XLSTM_HN_CASE(32, 1)
+    XLSTM_HN_CASE(32, 2)
+    XLSTM_HN_CASE(32, 4)
+    return cudaErrorInvalidValue;
 #undef XLSTM_HN_CASE
-    return cudaGetLastError();
 }
 
 bool misaligned16(const void *p) { return ((uintptr_t)p & 15u) != 0; }
