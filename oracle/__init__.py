@@ -19,6 +19,12 @@ Contents
 ``quadratic_form`` (in ``oracle.quadratic``) the parallel form that section 2.3
                    says the recurrence can be rewritten into, derived by
                    unrolling the recurrence; pure numpy, for tiny inputs.
+``headnorm_gate``  (in ``oracle.headnorm``) the mLSTM block's epilogue after the
+                   cell (section 2.4, Figure 10): per-head GroupNorm, learnable
+                   skip, external output gate; numpy float64.
+``grads``          (in ``oracle.backward``) gradients of a loss through the cell:
+                   the recurrence in plain PyTorch float64 ops, differentiated
+                   by PyTorch's reverse mode.
 """
 from __future__ import annotations
 
