@@ -22,6 +22,9 @@ Contents
 ``headnorm_gate``  (in ``oracle.headnorm``) the mLSTM block's epilogue after the
                    cell (section 2.4, Figure 10): per-head GroupNorm, learnable
                    skip, external output gate; numpy float64.
+``slstm.fwd``      (in ``oracle.slstm``) the sLSTM cell of section 2.2 (scalar
+                   memory, exponential gating, normaliser, stabiliser, memory
+                   mixing within heads) in plain C float64 (``slstm_oracle.c``).
 ``grads``          (in ``oracle.backward``) gradients of a loss through the cell:
                    the recurrence in plain PyTorch float64 ops, differentiated
                    by PyTorch's reverse mode.
@@ -42,21 +45,31 @@ _lock = threading.Lock()
 _lib = None
 
 
-def build(force: bool = False) -> str:
-    """Compile the C oracle into ``oracle/libmlstm_oracle.so`` (gcc, -O2, OpenMP).
+_SLSTM_SRC = os.path.join(_HERE, "slstm_oracle.c")
+_SLSTM_LIB = os.path.join(_HERE, "libslstm_oracle.so")
 
-    No fast-math: the oracle keeps IEEE double semantics and the source order
+
+def _build_one(src: str, lib: str, force: bool) -> str:
+    if (not force and os.path.exists(lib)
+            and os.path.getmtime(lib) >= os.path.getmtime(src)):
+        return lib
+    tmp = lib + f".tmp{os.getpid()}"
+    cmd = ["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11",
+           "-fno-fast-math", "-ffp-contract=off", src, "-o", tmp, "-lm"]
+    subprocess.run(cmd, check=True)
+    os.replace(tmp, lib)
+    return lib
+
+
+def build(force: bool = False) -> str:
+    """Compile the C oracles into ``oracle/libmlstm_oracle.so`` and
+    ``oracle/libslstm_oracle.so`` (gcc, -O2, OpenMP); returns the first.
+
+    No fast-math: the oracles keep IEEE double semantics and the source order
     of every sum.
     """
-    if (not force and os.path.exists(_LIB)
-            and os.path.getmtime(_LIB) >= os.path.getmtime(_SRC)):
-        return _LIB
-    tmp = _LIB + f".tmp{os.getpid()}"
-    cmd = ["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11",
-           "-fno-fast-math", "-ffp-contract=off", _SRC, "-o", tmp, "-lm"]
-    subprocess.run(cmd, check=True)
-    os.replace(tmp, _LIB)
-    return _LIB
+    _build_one(_SLSTM_SRC, _SLSTM_LIB, force)
+    return _build_one(_SRC, _LIB, force)
 
 
 def _bind(lib):
