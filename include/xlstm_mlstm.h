@@ -187,6 +187,40 @@ xlstm_status xlstm_mlstm_step(const void *q, const void *k, const void *v,
                               void *cuda_stream);
 
 /*
+ * Backward of the cell (gradients for training): for the forward with a zero
+ * initial state and the loss L = sum(dh * h) + sum(dC * C'_T) + sum(dn * n'_T),
+ * writes dL/dq, dL/dk, dL/dv, dL/d(itilde), dL/d(ftilde), dL/d(otilde).  The
+ * stabiliser is held fixed, which "xLSTM: Extended Long Short-Term Memory"
+ * section 2.2 (appendix A.2) shows leaves the derivatives unchanged; the
+ * returned state's own stabiliser m_T is differentiated where the final-state
+ * cotangents need it.  fp32 arithmetic on CUDA cores; the chunk-start and
+ * reverse states are materialised in the workspace.
+ *
+ *   q, k, v, dh     [B, NH, S, DH]  dtype dt (dh: cotangent of h)
+ *   i_pre, f_pre    [B, NH, S]      float
+ *   o_pre           [B, NH, S, DH]  float
+ *   dC [B, NH, DH, DH], dn [B, NH, DH]  float, cotangents of the final
+ *                   stabilised state; each may be NULL (zero)
+ *   dq, dk, dv      [B, NH, S, DH]  dtype dt, outputs
+ *   di, df          [B, NH, S]      float, outputs
+ *   d_o             [B, NH, S, DH]  float, output
+ *   chunk           1..64 tokens per chunk (XLSTM_ERR_CHUNK otherwise)
+ *   workspace       at least xlstm_mlstm_bwd_workspace_size() bytes
+ * Outputs must not be any input or each other (the same pointer twice is
+ * rejected with XLSTM_ERR_UNSUPPORTED).  DH: multiple of 16 in [16, 512].
+ * B, NH or S == 0 is a no-op.
+ */
+xlstm_status xlstm_mlstm_bwd_workspace_size(int B, int NH, int S, int DH, int chunk,
+                                            xlstm_dtype dt, size_t *bytes);
+xlstm_status xlstm_mlstm_bwd(const void *q, const void *k, const void *v,
+                             const float *i_pre, const float *f_pre, const float *o_pre,
+                             const void *dh, const float *dC, const float *dn,
+                             void *dq, void *dk, void *dv, float *di, float *df, float *d_o,
+                             int B, int NH, int S, int DH, int chunk,
+                             xlstm_dtype dt, xlstm_fgate fg,
+                             void *workspace, size_t workspace_bytes, void *cuda_stream);
+
+/*
  * The mLSTM block's epilogue after the cell ("xLSTM: Extended Long Short-Term
  * Memory" section 2.4, Figure 10): the cell output is normalised by a GroupNorm
  * whose groups are the heads (a LayerNorm over each head's DH channels, per

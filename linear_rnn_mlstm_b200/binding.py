@@ -27,7 +27,8 @@ PATH_AUTO, PATH_SIMT, PATH_TENSOR = 0, 1, 2
 EXPORTED = ("xlstm_abi_version", "xlstm_status_string", "xlstm_mlstm_fwd_workspace_size",
             "xlstm_mlstm_fwd_workspace_size_ex", "xlstm_mlstm_fwd", "xlstm_mlstm_fwd_ex",
             "xlstm_mlstm_step", "xlstm_device_status", "xlstm_profile_begin", "xlstm_profile_end",
-            "xlstm_mlstm_fwd_noalloc", "xlstm_selftest_wait_timeout", "xlstm_mlstm_headnorm_gate")
+            "xlstm_mlstm_fwd_noalloc", "xlstm_selftest_wait_timeout", "xlstm_mlstm_headnorm_gate",
+            "xlstm_mlstm_bwd_workspace_size", "xlstm_mlstm_bwd")
 NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
 
 
@@ -85,6 +86,11 @@ def load(path: str = LIB_PATH):
         lib.xlstm_mlstm_headnorm_gate.argtypes = [vp] + [fp] * 3 + [vp] * 3 + [i] * 4 + \
             [ctypes.c_float, i, i, vp]
         lib.xlstm_mlstm_headnorm_gate.restype = i
+        lib.xlstm_mlstm_bwd_workspace_size.argtypes = [i] * 6 + [ctypes.POINTER(sz)]
+        lib.xlstm_mlstm_bwd_workspace_size.restype = i
+        lib.xlstm_mlstm_bwd.argtypes = [vp] * 3 + [fp] * 3 + [vp] + [fp] * 2 + [vp] * 3 + \
+            [fp] * 3 + [i] * 7 + [vp, sz, vp]
+        lib.xlstm_mlstm_bwd.restype = i
         lib.xlstm_profile_begin.restype = i
         lib.xlstm_profile_end.argtypes = [ctypes.POINTER(KernelTime), i, ctypes.POINTER(i)]
         lib.xlstm_profile_end.restype = i
@@ -135,6 +141,19 @@ def xlstm_mlstm_headnorm_gate(h, gamma, beta, skip_w, x_skip, z, y, B, NH, S, DH
                               stream):
     return load().xlstm_mlstm_headnorm_gate(h, gamma, beta, skip_w, x_skip, z, y, B, NH, S, DH,
                                             float(eps), dt, og, stream)
+
+
+def xlstm_mlstm_bwd_workspace_size(B, NH, S, DH, chunk, dt):
+    n = ctypes.c_size_t(0)
+    st = load().xlstm_mlstm_bwd_workspace_size(B, NH, S, DH, chunk, dt, ctypes.byref(n))
+    return st, n.value
+
+
+def xlstm_mlstm_bwd(q, k, v, i_pre, f_pre, o_pre, dh, dC, dn, dq, dk, dv, di, df, d_o,
+                    B, NH, S, DH, chunk, dt, fg, workspace, workspace_bytes, stream):
+    return load().xlstm_mlstm_bwd(q, k, v, i_pre, f_pre, o_pre, dh, dC, dn, dq, dk, dv, di, df,
+                                  d_o, B, NH, S, DH, chunk, dt, fg, workspace, workspace_bytes,
+                                  stream)
 
 
 def xlstm_device_status(stream) -> int:
@@ -282,3 +301,34 @@ def mlstm_headnorm_gate(h, gamma, beta, z, skip_w=None, x_skip=None, eps=1e-5, o
     if st != OK:
         raise XlstmError(st, "xlstm_mlstm_headnorm_gate")
     return y
+
+
+def mlstm_bwd(q, k, v, i_pre, f_pre, o_pre, dh, dC=None, dn=None, chunk=64, fgate="sigmoid"):
+    """Gradients of sum(dh h) + sum(dC C'_T) + sum(dn n'_T) through the forward
+    from a zero state.  Returns dict dq, dk, dv (q's dtype), di, df, do (fp32)."""
+    torch = _torch()
+    B, NH, S, DH = q.shape
+    dev, dtype, dt = q.device, q.dtype, _dt(q)
+    for t, nm in ((q, "q"), (k, "k"), (v, "v"), (dh, "dh")):
+        _check(t, nm, (B, NH, S, DH), dtype, dev)
+    _check(i_pre, "i_pre", (B, NH, S), torch.float32, dev)
+    _check(f_pre, "f_pre", (B, NH, S), torch.float32, dev)
+    _check(o_pre, "o_pre", (B, NH, S, DH), torch.float32, dev)
+    _check(dC, "dC", (B, NH, DH, DH), torch.float32, dev)
+    _check(dn, "dn", (B, NH, DH), torch.float32, dev)
+    out = {nm: torch.empty((B, NH, S, DH), dtype=dtype, device=dev) for nm in ("dq", "dk", "dv")}
+    out["di"] = torch.empty((B, NH, S), dtype=torch.float32, device=dev)
+    out["df"] = torch.empty((B, NH, S), dtype=torch.float32, device=dev)
+    out["do"] = torch.empty((B, NH, S, DH), dtype=torch.float32, device=dev)
+    st, nbytes = xlstm_mlstm_bwd_workspace_size(B, NH, S, DH, chunk, dt)
+    if st != OK:
+        raise XlstmError(st, "xlstm_mlstm_bwd_workspace_size")
+    ws = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=dev)
+    fg = FGATE_EXP if fgate == "exp" else FGATE_SIGMOID
+    st = xlstm_mlstm_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(i_pre), _ptr(f_pre), _ptr(o_pre),
+                         _ptr(dh), _ptr(dC), _ptr(dn), _ptr(out["dq"]), _ptr(out["dk"]),
+                         _ptr(out["dv"]), _ptr(out["di"]), _ptr(out["df"]), _ptr(out["do"]),
+                         B, NH, S, DH, chunk, dt, fg, ws.data_ptr(), ws.numel(), _stream(dev))
+    if st != OK:
+        raise XlstmError(st, "xlstm_mlstm_bwd")
+    return out

@@ -154,3 +154,53 @@ def _headnorm(**over):
 ])
 def test_headnorm_gate_rejects_bad_arguments_before_device_work(over, expect):
     assert _headnorm(**over) == expect
+
+
+def _bwd(**over):
+    a = dict(q=FAKE, k=FAKE + 16, v=FAKE + 32, i_pre=FAKE + 48, f_pre=FAKE + 64, o_pre=FAKE + 80,
+             dh=FAKE + 96, dC=None, dn=None, dq=FAKE + 112, dk=FAKE + 128, dv=FAKE + 144,
+             di=FAKE + 160, df=FAKE + 176, d_o=FAKE + 192, B=1, NH=2, S=10, DH=16, chunk=4,
+             dt=xb.F32, fg=xb.FGATE_SIGMOID, workspace=FAKE + 4096, workspace_bytes=1 << 30,
+             stream=None)
+    a.update(over)
+    return xb.xlstm_mlstm_bwd(**a)
+
+
+@pytest.mark.parametrize("over,expect", [
+    (dict(q=None), xb.ERR_NULL),
+    (dict(dh=None), xb.ERR_NULL),
+    (dict(d_o=None), xb.ERR_NULL),
+    (dict(dk=FAKE + 136), xb.ERR_ALIGN),
+    (dict(dC=FAKE + 4), xb.ERR_ALIGN),
+    (dict(dt=5), xb.ERR_DTYPE),
+    (dict(fg=2), xb.ERR_DTYPE),
+    (dict(DH=40), xb.ERR_SHAPE),
+    (dict(S=-3), xb.ERR_SHAPE),
+    (dict(chunk=0), xb.ERR_CHUNK),
+    (dict(chunk=65), xb.ERR_CHUNK),                      # per-thread arrays hold 64 tokens
+    (dict(workspace_bytes=64), xb.ERR_WORKSPACE),
+    (dict(workspace=None), xb.ERR_WORKSPACE),
+    (dict(dq=FAKE), xb.ERR_UNSUPPORTED),                 # an output is an input
+    (dict(dv=FAKE + 112), xb.ERR_UNSUPPORTED),           # two outputs share a buffer
+    (dict(di=FAKE + 4096), xb.ERR_UNSUPPORTED),          # an output is the workspace
+    (dict(S=0), xb.OK),                                  # empty sequence: a no-op
+    (dict(B=0, q=None), xb.OK),
+])
+def test_bwd_rejects_bad_arguments_before_device_work(over, expect):
+    assert _bwd(**over) == expect
+
+
+def test_bwd_workspace_size_matches_its_layout():
+    """Per head: 8 per-token arrays, 3 per-chunk arrays, NC + 1 chunk-start
+    states (C', n'), num' and dnum' per token, NC reverse states (dC, dn); each
+    array padded to 64 floats."""
+    pad = lambda n: (n + 63) // 64 * 64
+    for B, NH, S, DH, L in ((1, 2, 10, 16, 4), (2, 3, 64, 48, 64), (1, 1, 7, 512, 1)):
+        BH, NC = B * NH, (S + L - 1) // L
+        sizes = [BH * S] * 8 + [BH * NC] * 3 + [BH * (NC + 1) * DH * DH, BH * (NC + 1) * DH,
+                                               BH * S * DH, BH * S * DH, BH * NC * DH * DH,
+                                               BH * NC * DH]
+        st, n = xb.xlstm_mlstm_bwd_workspace_size(B, NH, S, DH, L, xb.F32)
+        assert st == xb.OK and n == 4 * sum(pad(x) for x in sizes)
+    assert xb.xlstm_mlstm_bwd_workspace_size(1, 1, 0, 16, 4, xb.F32) == (xb.OK, 0)
+    assert xb.xlstm_mlstm_bwd_workspace_size(1, 1, 8, 16, 65, xb.F32)[0] == xb.ERR_CHUNK

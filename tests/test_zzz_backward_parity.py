@@ -1,0 +1,100 @@
+"""GPU parity of the backward (``xlstm_mlstm_bwd``) against the float64
+gradient oracle (``oracle.backward``: reverse-mode differentiation of the
+plain recurrence).  The same per-thread code is checked on the CPU by
+``test_backward_emulation.py``; here it runs as compiled for sm_100a.
+
+Tolerances, per gradient tensor, max |got - ref| / max(1, max |ref|): fp32
+1e-4, and 5e-4 with wide input gates (plain fp32 evaluation of the definition
+itself reaches 1.7e-4 there); for bf16 q, k, v, dh the fp32 gradients keep
+those bounds and dq, dk, dv add one rounding to bf16, 2^-8 of each element.
+The file is named to be collected after the forward's parity tests.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle.backward as bw
+from linear_rnn_mlstm_b200 import binding as xb
+
+pytestmark = pytest.mark.gpu
+
+NAMES = ("q", "k", "v", "i_pre", "f_pre", "o_pre")
+OUT = {"q": "dq", "k": "dk", "v": "dv", "i_pre": "di", "f_pre": "df", "o_pre": "do"}
+
+
+def _inputs(B, NH, S, DH, fgate, wide, dtype, seed):
+    g = np.random.default_rng(seed)
+    shp = (B, NH, S, DH)
+    f64 = dict(q=g.normal(0, 1, shp), k=g.normal(0, 1, shp), v=g.normal(0, 1, shp),
+               i_pre=g.normal(0, 3 if wide else 1, shp[:3]),
+               f_pre=(g.normal(3, 1, shp[:3]) if fgate == "sigmoid"
+                      else g.normal(-0.05, 1.0 if wide else 0.1, shp[:3])),
+               o_pre=g.normal(0, 1, shp))
+    dh = g.normal(0, 1, shp)
+    dC = g.normal(0, 1, (B, NH, DH, DH))
+    dn = g.normal(0, 1, (B, NH, DH))
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    t = {nm: torch.from_numpy(x).to(tdt if nm in ("q", "k", "v") else torch.float32)
+         for nm, x in f64.items()}
+    t["dh"] = torch.from_numpy(dh).to(tdt)
+    t["dC"] = torch.from_numpy(dC).float()
+    t["dn"] = torch.from_numpy(dn).float()
+    return t
+
+
+def _check(got, ref, dtype, tol):
+    for nm in NAMES:
+        g = got[OUT[nm]].float().cpu().numpy().astype(np.float64)
+        r = ref[nm]
+        assert np.all(np.isfinite(g)), f"d{nm}: non-finite"
+        scale = max(1.0, float(np.max(np.abs(r))))
+        d = np.abs(g - r)
+        if dtype == "bf16" and nm in ("q", "k", "v"):
+            ok = d <= 2.0 ** -8 * np.abs(r) + tol * scale
+            assert np.all(ok), f"d{nm}: worst excess {float(np.max(d - 2.0 ** -8 * np.abs(r))):.3e}"
+        else:
+            assert float(np.max(d)) / scale <= tol, \
+                f"d{nm}: max|d|/max(1,max|ref|) = {float(np.max(d)) / scale:.3e} (tol {tol})"
+
+
+CASES = [
+    # B, NH, S, DH, chunk, fgate, wide, cotangents, dtype
+    (1, 2, 13, 16, 4, "sigmoid", False, False, "f32"),
+    (2, 1, 29, 48, 8, "exp", False, True, "f32"),
+    (1, 2, 21, 32, 8, "exp", True, False, "f32"),
+    (1, 1, 70, 64, 64, "sigmoid", False, True, "f32"),
+    (2, 2, 40, 128, 16, "sigmoid", False, False, "bf16"),
+    (1, 1, 1, 16, 1, "sigmoid", False, True, "f32"),
+]
+
+
+@pytest.mark.parametrize("B,NH,S,DH,chunk,fgate,wide,cot,dtype", CASES,
+                         ids=[f"B{c[0]}NH{c[1]}S{c[2]}DH{c[3]}L{c[4]}-{c[5]}"
+                              f"{'-wide' if c[6] else ''}{'-cot' if c[7] else ''}-{c[8]}"
+                              for c in CASES])
+def test_backward_matches_gradient_oracle(cuda_lib, B, NH, S, DH, chunk, fgate, wide, cot, dtype):
+    t = _inputs(B, NH, S, DH, fgate, wide, dtype, seed=S + DH + chunk)
+    kw = dict(dC=t["dC"], dn=t["dn"]) if cot else {}
+    ref = bw.grads(*(t[nm] for nm in NAMES), t["dh"], fgate,
+                   **({k: v.numpy() for k, v in kw.items()}))[1]
+    d = {k: v.cuda().contiguous() for k, v in t.items()}
+    got = xb.mlstm_bwd(*(d[nm] for nm in NAMES), d["dh"],
+                       dC=d["dC"] if cot else None, dn=d["dn"] if cot else None,
+                       chunk=chunk, fgate=fgate)
+    torch.cuda.synchronize()
+    assert xb.xlstm_device_status(torch.cuda.current_stream().cuda_stream) == xb.OK
+    _check(got, ref, dtype, 5e-4 if wide else 1e-4)
+
+
+def test_backward_chunk_size_invariance(cuda_lib):
+    """The blocking is an implementation detail: chunk sizes 1, 7 and 64 give
+    the same gradients up to fp32 rounding."""
+    t = _inputs(1, 2, 50, 32, "sigmoid", False, "f32", seed=3)
+    d = {k: v.cuda().contiguous() for k, v in t.items()}
+    outs = [xb.mlstm_bwd(*(d[nm] for nm in NAMES), d["dh"], chunk=L) for L in (1, 7, 64)]
+    torch.cuda.synchronize()
+    for nm in OUT.values():
+        a = outs[0][nm].cpu().numpy()
+        for o in outs[1:]:
+            b = o[nm].cpu().numpy()
+            assert np.max(np.abs(a - b)) <= 1e-4 * max(1.0, float(np.max(np.abs(a)))), nm
