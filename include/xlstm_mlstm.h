@@ -221,6 +221,38 @@ xlstm_status xlstm_mlstm_bwd(const void *q, const void *k, const void *v,
                              void *workspace, size_t workspace_bytes, void *cuda_stream);
 
 /*
+ * sLSTM forward ("xLSTM: Extended Long Short-Term Memory" section 2.2): scalar
+ * memory cells with exponential input gating, a sigmoid or exponential forget
+ * gate, a normaliser state, the stabiliser m_t, and memory mixing through
+ * recurrent connections from h_{t-1} to the cell input z and the gates i, f, o
+ * within each head.  Per batch b, head hd, unit j:
+ *
+ *   zt = zx + R_z h_{t-1}, it = ix + R_i h_{t-1}, ft = fx + R_f h_{t-1},
+ *   ot = ox + R_o h_{t-1};  z = tanh(zt), log i = it,
+ *   log f = log sigmoid(ft) | ft, o = sigmoid(ot)
+ *   m_t = max(log f + m_{t-1}, log i)
+ *   c_t = exp(log f + m_{t-1} - m_t) c_{t-1} + exp(log i - m_t) z
+ *   n_t = exp(log f + m_{t-1} - m_t) n_{t-1} + exp(log i - m_t),  h_t = o c_t / n_t
+ *
+ *   zx, ix, fx, ox  [B, NH, S, DH] float, input pre-activations (projection and
+ *                   bias already applied)
+ *   R               [NH, 4, DH, DH] float, recurrent blocks in the order z, i, f,
+ *                   o; R[hd][g][j][l] multiplies h_{t-1}[l] into unit j's gate g
+ *   h               [B, NH, S, DH] float, output
+ *   c0, n0, m0, h0  [B, NH, DH] float, initial state (c, n stabilised); each
+ *                   may be NULL (zeros)
+ *   c_out, n_out, m_out, h_out  [B, NH, DH] float, final state; each nullable
+ * Outputs must not be any input or each other (XLSTM_ERR_UNSUPPORTED).
+ * DH in [1, 512].  S == 0 copies the initial state to the state outputs.
+ * One CTA per (batch, head), fp32; correctness-first (R read from L2 every step).
+ */
+xlstm_status xlstm_slstm_fwd(const float *zx, const float *ix, const float *fx, const float *ox,
+                             const float *R, float *h,
+                             const float *c0, const float *n0, const float *m0, const float *h0,
+                             float *c_out, float *n_out, float *m_out, float *h_out,
+                             int B, int NH, int S, int DH, xlstm_fgate fg, void *cuda_stream);
+
+/*
  * The mLSTM block's epilogue after the cell ("xLSTM: Extended Long Short-Term
  * Memory" section 2.4, Figure 10): the cell output is normalised by a GroupNorm
  * whose groups are the heads (a LayerNorm over each head's DH channels, per

@@ -28,7 +28,7 @@ EXPORTED = ("xlstm_abi_version", "xlstm_status_string", "xlstm_mlstm_fwd_workspa
             "xlstm_mlstm_fwd_workspace_size_ex", "xlstm_mlstm_fwd", "xlstm_mlstm_fwd_ex",
             "xlstm_mlstm_step", "xlstm_device_status", "xlstm_profile_begin", "xlstm_profile_end",
             "xlstm_mlstm_fwd_noalloc", "xlstm_selftest_wait_timeout", "xlstm_mlstm_headnorm_gate",
-            "xlstm_mlstm_bwd_workspace_size", "xlstm_mlstm_bwd")
+            "xlstm_mlstm_bwd_workspace_size", "xlstm_mlstm_bwd", "xlstm_slstm_fwd")
 NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
 
 
@@ -91,6 +91,8 @@ def load(path: str = LIB_PATH):
         lib.xlstm_mlstm_bwd.argtypes = [vp] * 3 + [fp] * 3 + [vp] + [fp] * 2 + [vp] * 3 + \
             [fp] * 3 + [i] * 7 + [vp, sz, vp]
         lib.xlstm_mlstm_bwd.restype = i
+        lib.xlstm_slstm_fwd.argtypes = [fp] * 14 + [i] * 5 + [vp]
+        lib.xlstm_slstm_fwd.restype = i
         lib.xlstm_profile_begin.restype = i
         lib.xlstm_profile_end.argtypes = [ctypes.POINTER(KernelTime), i, ctypes.POINTER(i)]
         lib.xlstm_profile_end.restype = i
@@ -154,6 +156,12 @@ def xlstm_mlstm_bwd(q, k, v, i_pre, f_pre, o_pre, dh, dC, dn, dq, dk, dv, di, df
     return load().xlstm_mlstm_bwd(q, k, v, i_pre, f_pre, o_pre, dh, dC, dn, dq, dk, dv, di, df,
                                   d_o, B, NH, S, DH, chunk, dt, fg, workspace, workspace_bytes,
                                   stream)
+
+
+def xlstm_slstm_fwd(zx, ix, fx, ox, R, h, c0, n0, m0, h0, c_out, n_out, m_out, h_out,
+                    B, NH, S, DH, fg, stream):
+    return load().xlstm_slstm_fwd(zx, ix, fx, ox, R, h, c0, n0, m0, h0, c_out, n_out, m_out,
+                                  h_out, B, NH, S, DH, fg, stream)
 
 
 def xlstm_device_status(stream) -> int:
@@ -332,3 +340,25 @@ def mlstm_bwd(q, k, v, i_pre, f_pre, o_pre, dh, dC=None, dn=None, chunk=64, fgat
     if st != OK:
         raise XlstmError(st, "xlstm_mlstm_bwd")
     return out
+
+
+def slstm_fwd(zx, ix, fx, ox, R, fgate="sigmoid", c0=None, n0=None, m0=None, h0=None):
+    """sLSTM forward on fp32 CUDA tensors zx, ix, fx, ox [B, NH, S, DH] and
+    R [NH, 4, DH, DH].  Returns (h, c, n, m, h_last)."""
+    torch = _torch()
+    B, NH, S, DH = zx.shape
+    dev = zx.device
+    for t, nm in ((zx, "zx"), (ix, "ix"), (fx, "fx"), (ox, "ox")):
+        _check(t, nm, (B, NH, S, DH), torch.float32, dev)
+    _check(R, "R", (NH, 4, DH, DH), torch.float32, dev)
+    for t, nm in ((c0, "c0"), (n0, "n0"), (m0, "m0"), (h0, "h0")):
+        _check(t, nm, (B, NH, DH), torch.float32, dev)
+    h = torch.empty((B, NH, S, DH), dtype=torch.float32, device=dev)
+    st_out = [torch.empty((B, NH, DH), dtype=torch.float32, device=dev) for _ in range(4)]
+    fg = FGATE_EXP if fgate == "exp" else FGATE_SIGMOID
+    st = xlstm_slstm_fwd(_ptr(zx), _ptr(ix), _ptr(fx), _ptr(ox), _ptr(R), _ptr(h), _ptr(c0),
+                         _ptr(n0), _ptr(m0), _ptr(h0), *(_ptr(t) for t in st_out),
+                         B, NH, S, DH, fg, _stream(dev))
+    if st != OK:
+        raise XlstmError(st, "xlstm_slstm_fwd")
+    return (h, *st_out)

@@ -204,3 +204,30 @@ def test_bwd_workspace_size_matches_its_layout():
         assert st == xb.OK and n == 4 * sum(pad(x) for x in sizes)
     assert xb.xlstm_mlstm_bwd_workspace_size(1, 1, 0, 16, 4, xb.F32) == (xb.OK, 0)
     assert xb.xlstm_mlstm_bwd_workspace_size(1, 1, 8, 16, 65, xb.F32)[0] == xb.ERR_CHUNK
+
+
+def _slstm(**over):
+    a = dict(zx=FAKE, ix=FAKE + 16, fx=FAKE + 32, ox=FAKE + 48, R=FAKE + 64, h=FAKE + 80,
+             c0=None, n0=None, m0=None, h0=None, c_out=FAKE + 96, n_out=None, m_out=None,
+             h_out=None, B=1, NH=2, S=5, DH=16, fg=xb.FGATE_SIGMOID, stream=None)
+    a.update(over)
+    return xb.xlstm_slstm_fwd(**a)
+
+
+@pytest.mark.parametrize("over,expect", [
+    (dict(zx=None), xb.ERR_NULL),
+    (dict(R=None), xb.ERR_NULL),
+    (dict(h=None), xb.ERR_NULL),
+    (dict(ox=FAKE + 52), xb.ERR_ALIGN),
+    (dict(h0=FAKE + 8), xb.ERR_ALIGN),
+    (dict(fg=3), xb.ERR_DTYPE),
+    (dict(DH=0), xb.ERR_SHAPE),
+    (dict(DH=513), xb.ERR_SHAPE),
+    (dict(S=-1), xb.ERR_SHAPE),
+    (dict(h=FAKE), xb.ERR_UNSUPPORTED),                  # output is an input
+    (dict(n_out=FAKE + 96), xb.ERR_UNSUPPORTED),         # two outputs share a buffer
+    (dict(B=0, zx=None), xb.OK),
+    (dict(S=0, zx=None, h=None, c_out=None), xb.OK),     # nothing to do
+])
+def test_slstm_rejects_bad_arguments_before_device_work(over, expect):
+    assert _slstm(**over) == expect
