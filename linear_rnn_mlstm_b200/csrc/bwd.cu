@@ -101,6 +101,7 @@ xlstm_status check_bwd_shape(int B, int NH, int S, int DH, int chunk, xlstm_dtyp
     if (B < 0 || NH < 0 || S < 0) return XLSTM_ERR_SHAPE;
     if (DH < 16 || DH > 512 || DH % 16 != 0) return XLSTM_ERR_SHAPE;
     if ((long long)B * NH * S * DH > (1LL << 40)) return XLSTM_ERR_SHAPE;
+    if ((long long)B * NH > 0x7fffffffLL) return XLSTM_ERR_SHAPE;     // heads index an int
     if (chunk < 1 || chunk > bwd::kMaxChunk) return XLSTM_ERR_CHUNK;
     return XLSTM_OK;
 }

@@ -176,6 +176,7 @@ def _bwd(**over):
     (dict(fg=2), xb.ERR_DTYPE),
     (dict(DH=40), xb.ERR_SHAPE),
     (dict(S=-3), xb.ERR_SHAPE),
+    (dict(B=70000, NH=70000, S=0), xb.ERR_SHAPE),        # more heads than an int indexes
     (dict(chunk=0), xb.ERR_CHUNK),
     (dict(chunk=65), xb.ERR_CHUNK),                      # per-thread arrays hold 64 tokens
     (dict(workspace_bytes=64), xb.ERR_WORKSPACE),
