@@ -219,7 +219,8 @@ int lanes_per_row(int nvec) {
 }
 
 // CTAs of one instantiation resident per SM (registers decide it); the grid is
-// one full wave of them and each warp strides over the rows.
+// one full wave of them and each warp strides over the rows.  Cached after the
+// first query; host threads that race on the cache all store the same value.
 template <typename T, int LPR, int V> int resident_blocks() {
     static int n = 0;
     if (n == 0) {
