@@ -49,9 +49,21 @@ def _sigmoid(x):
                     np.exp(-np.abs(x)) / (1.0 + np.exp(-np.abs(x))))
 
 
-def head_backward(q, k, v, itl, ftl, otl, dh, L, fgate="sigmoid", dC=None, dn=None):
+def _matmul(a, b):
+    return a @ b
+
+
+# The backward's matrix products, by name; ``ops`` may replace any of them
+# (e.g. with operands rounded to a tensor-core type) to study precision.
+PRODUCTS = ("dP", "G_khat", "G_q", "WS_dnum", "Cprev", "dCb_terms", "dCb_update")
+
+
+def head_backward(q, k, v, itl, ftl, otl, dh, L, fgate="sigmoid", dC=None, dn=None, ops=None):
     """One head: q, k, v, otl, dh [S, DH]; itl, ftl [S]; dC [DH, DH], dn [DH]
-    or None.  Returns dict of gradients dq, dk, dv, di, df, do."""
+    or None.  Returns dict of gradients dq, dk, dv, di, df, do.  ``ops`` maps
+    names in PRODUCTS to replacements for ``a @ b`` in the backward pass."""
+    mm = {nm: _matmul for nm in PRODUCTS}
+    mm.update(ops or {})
     S, DH = q.shape
     khat = k / math.sqrt(DH)
     log_f = _log_sigmoid(ftl) if fgate == "sigmoid" else ftl.copy()
@@ -106,16 +118,16 @@ def head_backward(q, k, v, itl, ftl, otl, dh, L, fgate="sigmoid", dC=None, dn=No
     for sv in reversed(saved):
         a, e = sv["a"], sv["e"]
         W, Sc, g, wk = sv["W"], sv["Sc"], sv["g"], sv["wk"]
-        dv[a:e] += wk[:, None] * (khat[a:e] @ dCb.T)
-        dkh[a:e] += wk[:, None] * (v[a:e] @ dCb + dnb[None, :])
-        dP = dnum[a:e] @ v[a:e].T + dnq[a:e][:, None]
+        dv[a:e] += wk[:, None] * mm["dCb_terms"](khat[a:e], dCb.T)
+        dkh[a:e] += wk[:, None] * (mm["dCb_terms"](v[a:e], dCb) + dnb[None, :])
+        dP = mm["dP"](dnum[a:e], v[a:e].T) + dnq[a:e][:, None]
         G = W * dP
-        dq[a:e] += G @ khat[a:e] + g[:, None] * (dnum[a:e] @ sv["C_prev"] + dnq[a:e][:, None]
-                                                 * sv["n_prev"][None, :])
-        dkh[a:e] += G.T @ q[a:e]
-        dv[a:e] += (W * Sc).T @ dnum[a:e]
+        dq[a:e] += mm["G_khat"](G, khat[a:e]) + g[:, None] * (
+            mm["Cprev"](dnum[a:e], sv["C_prev"]) + dnq[a:e][:, None] * sv["n_prev"][None, :])
+        dkh[a:e] += mm["G_q"](G.T, q[a:e])
+        dv[a:e] += mm["WS_dnum"]((W * Sc).T, dnum[a:e])
         decay = np.exp(sv["B"] + sv["m_prev"] - sv["m_end"])
-        dCb = decay * dCb + (dnum[a:e] * g[:, None]).T @ q[a:e]
+        dCb = decay * dCb + mm["dCb_update"]((dnum[a:e] * g[:, None]).T, q[a:e])
         dnb = decay * dnb + (g * dnq[a:e]) @ q[a:e]
     di = (khat * dkh).sum(1)
     dF = A - di
@@ -133,7 +145,7 @@ def head_backward(q, k, v, itl, ftl, otl, dh, L, fgate="sigmoid", dC=None, dn=No
     return dict(q=dq, k=dkh / math.sqrt(DH), v=dv, i_pre=di, f_pre=df, o_pre=d_o)
 
 
-def backward(q, k, v, i_pre, f_pre, o_pre, dh, L, fgate="sigmoid", dC=None, dn=None):
+def backward(q, k, v, i_pre, f_pre, o_pre, dh, L, fgate="sigmoid", dC=None, dn=None, ops=None):
     """All heads of [B, NH, S, DH] inputs; returns {name: gradient}."""
     B, NH, S, DH = q.shape
     out = {nm: np.zeros(np.shape(x)) for nm, x in
@@ -143,7 +155,7 @@ def backward(q, k, v, i_pre, f_pre, o_pre, dh, L, fgate="sigmoid", dC=None, dn=N
             g = head_backward(q[bi, hi], k[bi, hi], v[bi, hi], i_pre[bi, hi], f_pre[bi, hi],
                               o_pre[bi, hi], dh[bi, hi], L, fgate,
                               None if dC is None else dC[bi, hi],
-                              None if dn is None else dn[bi, hi])
+                              None if dn is None else dn[bi, hi], ops)
             for nm in out:
                 out[nm][bi, hi] = g[nm]
     return out
