@@ -80,16 +80,19 @@ def forward(q, k, v, i_pre, f_pre, o_pre, fgate="sigmoid", raw=False):
 def grads(q, k, v, i_pre, f_pre, o_pre, dh, fgate="sigmoid", dC=None, dn=None, raw=False):
     """dL/d(input) for L = sum(dh h) + sum(dC C_T) + sum(dn n_T).  Returns
     (L, {name: float64 numpy array}) with names ``GRAD_NAMES``."""
-    xs = {nm: _t(x).requires_grad_(True) for nm, x in
-          zip(GRAD_NAMES, (q, k, v, i_pre, f_pre, o_pre))}
-    h, C, n = forward(*(xs[nm] for nm in GRAD_NAMES), fgate=fgate, raw=raw)
-    loss = (h * _t(dh)).sum()
-    if dC is not None:
-        loss = loss + (C * _t(dC)).sum()
-    if dn is not None:
-        loss = loss + (n * _t(dn)).sum()
-    if loss.requires_grad:
-        loss.backward()
+    # the caller may be inside torch.no_grad() (e.g. an autograd backward):
+    # the derivative is taken here regardless
+    with torch.enable_grad():
+        xs = {nm: _t(x).requires_grad_(True) for nm, x in
+              zip(GRAD_NAMES, (q, k, v, i_pre, f_pre, o_pre))}
+        h, C, n = forward(*(xs[nm] for nm in GRAD_NAMES), fgate=fgate, raw=raw)
+        loss = (h * _t(dh)).sum()
+        if dC is not None:
+            loss = loss + (C * _t(dC)).sum()
+        if dn is not None:
+            loss = loss + (n * _t(dn)).sum()
+        if loss.requires_grad:
+            loss.backward()
     # an input the loss does not reach (e.g. every input of an empty sequence)
     # has a zero gradient
     return float(loss.detach()), {nm: (xs[nm].grad.numpy().copy() if xs[nm].grad is not None

@@ -178,3 +178,12 @@ def test_planted_mistake_fails_a_pin(name):
         except AssertionError:
             failed.append(pin.__name__)
     assert failed, f"mutant {name} passed every pin"
+
+
+def test_gradients_are_taken_under_no_grad_too():
+    d, dh, _, _ = _inputs(seed=9)
+    _, g0 = bw.grads(*(d[nm] for nm in bw.GRAD_NAMES), dh)
+    with torch.no_grad():
+        _, g1 = bw.grads(*(d[nm] for nm in bw.GRAD_NAMES), dh)
+    for nm in bw.GRAD_NAMES:
+        assert np.any(g1[nm]) and np.array_equal(g0[nm], g1[nm])

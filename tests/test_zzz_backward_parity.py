@@ -98,3 +98,18 @@ def test_backward_chunk_size_invariance(cuda_lib):
         for o in outs[1:]:
             b = o[nm].cpu().numpy()
             assert np.max(np.abs(a - b)) <= 1e-4 * max(1.0, float(np.max(np.abs(a)))), nm
+
+
+def test_differentiable_op_matches_gradient_oracle(cuda_lib):
+    """The torch.autograd op (forward and backward entry points joined) on the
+    GPU: gradients of a loss on h and on the final state."""
+    from linear_rnn_mlstm_b200.autograd import mlstm_cell
+    t = _inputs(1, 2, 45, 64, "sigmoid", False, "f32", seed=11)
+    x = {nm: t[nm].cuda().requires_grad_(True) for nm in NAMES}
+    h, C, n, m = mlstm_cell(*(x[nm] for nm in NAMES), chunk=64)
+    ((h * t["dh"].cuda()).sum() + (C * t["dC"].cuda()).sum() + (n * t["dn"].cuda()).sum()).backward()
+    torch.cuda.synchronize()
+    ref = bw.grads(*(t[nm] for nm in NAMES), t["dh"], "sigmoid", dC=t["dC"].numpy(),
+                   dn=t["dn"].numpy())[1]
+    got = {OUT[nm]: x[nm].grad for nm in NAMES}
+    _check(got, ref, "f32", 1e-4)
