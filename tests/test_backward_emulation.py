@@ -116,6 +116,29 @@ def test_backward_kernel_bodies_match_gradient_oracle(emulator, B, NH, S, DH, L,
     _compare(got, ref, 5e-4 if wide else 1e-4)
 
 
+def test_backward_kernel_bodies_floor_dominated(emulator):
+    """Input gates so small (itilde ~ N(-4, 1)) that the normaliser's floor is
+    active on every token of this draw: dnq' = 0 throughout, the floor passes
+    no gradient, and only the numerator's terms carry one."""
+    d, dh, dC, dn = _inputs(1, 2, 30, 16, "sigmoid", False, seed=5)
+    g = np.random.default_rng(6)
+    d["i_pre"] = g.normal(-4, 1, d["i_pre"].shape).astype(np.float32)
+    ref = bw.grads(*(d[nm] for nm in NAMES), dh, "sigmoid", dC=dC, dn=dn)[1]
+    got = _run(emulator, d, dh, 8, "sigmoid", dC=dC, dn=dn)
+    _compare(got, ref, 1e-4)
+
+
+def test_backward_kernel_bodies_growing_forget(emulator):
+    """Exponential forget gate above 1 (ftilde ~ N(0.3, 0.2)): the state grows
+    along the sequence and the stabiliser carries the scale."""
+    d, dh, _, _ = _inputs(1, 1, 48, 16, "exp", False, seed=8)
+    g = np.random.default_rng(9)
+    d["f_pre"] = g.normal(0.3, 0.2, d["f_pre"].shape).astype(np.float32)
+    ref = bw.grads(*(d[nm] for nm in NAMES), dh, "exp")[1]
+    got = _run(emulator, d, dh, 16, "exp")
+    _compare(got, ref, 5e-4)
+
+
 def test_backward_kernel_bodies_empty_sequence(emulator):
     d, dh, _, _ = _inputs(1, 2, 0, 16, "sigmoid", False, seed=1)
     got = _run(emulator, d, dh, 8, "sigmoid")

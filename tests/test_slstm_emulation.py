@@ -97,3 +97,13 @@ CASES = [(1, 2, 17, 16, "sigmoid", False), (2, 3, 9, 8, "exp", False),
 def test_slstm_unit_code_matches_oracle(emulator, B, NH, S, DH, fgate, state):
     x = inputs(B, NH, S, DH, fgate, seed=S + DH, state=state)
     compare(run(emulator, x, fgate), oracle_run(x, fgate))
+
+
+def test_slstm_unit_code_growing_forget_and_wide_input_gates(emulator):
+    """Exponential forget above 1 and input gates ~ N(0, 3): the raw state would
+    grow without bound; the stabilised one does not, and h stays a mean."""
+    x = inputs(1, 2, 64, 16, "exp", seed=12)
+    g = np.random.default_rng(13)
+    x["fx"] = g.normal(0.3, 0.2, x["fx"].shape).astype(np.float32)
+    x["ix"] = g.normal(0.0, 3.0, x["ix"].shape).astype(np.float32)
+    compare(run(emulator, x, "exp"), oracle_run(x, "exp"))
