@@ -183,6 +183,7 @@ xlstm_status xlstm_mlstm_fwd_ex(const void *q, const void *k, const void *v,
                                 xlstm_dtype dt, xlstm_fgate fg,
                                 void *workspace, size_t workspace_bytes,
                                 const xlstm_fwd_options *opts, void *cuda_stream) {
+    CallRange range("xlstm_mlstm_fwd");
     xlstm_status st = check_fwd_shape(B, NH, S, DH, chunk, dt);
     if (st != XLSTM_OK) return st;
     if (fg != XLSTM_FGATE_SIGMOID && fg != XLSTM_FGATE_EXP) return XLSTM_ERR_DTYPE;
@@ -239,6 +240,7 @@ xlstm_status xlstm_mlstm_step(const void *q, const void *k, const void *v,
                               void *h, float *C, float *n, float *m,
                               int B, int NH, int DH, xlstm_dtype dt, xlstm_fgate fg,
                               void *cuda_stream) {
+    CallRange range("xlstm_mlstm_step");
     if (dt != XLSTM_F32 && dt != XLSTM_BF16) return XLSTM_ERR_DTYPE;
     if (fg != XLSTM_FGATE_SIGMOID && fg != XLSTM_FGATE_EXP) return XLSTM_ERR_DTYPE;
     if (B < 0 || NH < 0 || DH < 16 || DH > 512 || DH % 16 != 0) return XLSTM_ERR_SHAPE;

@@ -167,6 +167,7 @@ extern "C" xlstm_status xlstm_mlstm_bwd(const void *q, const void *k, const void
                                         int DH, int chunk, xlstm_dtype dt, xlstm_fgate fg,
                                         void *workspace, size_t workspace_bytes,
                                         void *cuda_stream) {
+    CallRange range("xlstm_mlstm_bwd");
     xlstm_status st = check_bwd_shape(B, NH, S, DH, chunk, dt);
     if (st != XLSTM_OK) return st;
     if (fg != XLSTM_FGATE_SIGMOID && fg != XLSTM_FGATE_EXP) return XLSTM_ERR_DTYPE;

@@ -276,6 +276,7 @@ extern "C" xlstm_status xlstm_mlstm_headnorm_gate(const void *h, const float *ga
                                                   xlstm_dtype dt, xlstm_ogate og,
                                                   void *cuda_stream) {
     using namespace xlstm;
+    CallRange range("xlstm_mlstm_headnorm_gate");
     if (dt != XLSTM_F32 && dt != XLSTM_BF16) return XLSTM_ERR_DTYPE;
     if (og != XLSTM_OGATE_SILU && og != XLSTM_OGATE_SIGMOID) return XLSTM_ERR_DTYPE;
     if (B < 0 || NH < 0 || S < 0) return XLSTM_ERR_SHAPE;

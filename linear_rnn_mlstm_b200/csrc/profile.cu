@@ -4,10 +4,15 @@
 #include <string>
 #include <vector>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "../../include/xlstm_mlstm.h"
 #include "profile.h"
 
 namespace xlstm {
+
+CallRange::CallRange(const char *name) { nvtxRangePushA(name); }
+CallRange::~CallRange() { nvtxRangePop(); }
 
 namespace {
 struct Record {

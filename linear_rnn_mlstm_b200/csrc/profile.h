@@ -21,4 +21,15 @@ class KernelTimer {
     cudaEvent_t start_ = nullptr;
 };
 
+// Marks one C-ABI call as a named range on the host timeline (NVTX), so a
+// profiler's timeline shows which library call issued which kernels.  Without
+// a profiler attached the NVTX calls do nothing.
+class CallRange {
+  public:
+    explicit CallRange(const char *name);
+    ~CallRange();
+    CallRange(const CallRange &) = delete;
+    CallRange &operator=(const CallRange &) = delete;
+};
+
 }  // namespace xlstm

@@ -44,6 +44,7 @@ extern "C" xlstm_status xlstm_slstm_fwd(const float *zx, const float *ix, const 
                                         const float *h0, float *c_out, float *n_out,
                                         float *m_out, float *h_out, int B, int NH, int S,
                                         int DH, xlstm_fgate fg, void *cuda_stream) {
+    CallRange range("xlstm_slstm_fwd");
     if (fg != XLSTM_FGATE_SIGMOID && fg != XLSTM_FGATE_EXP) return XLSTM_ERR_DTYPE;
     if (B < 0 || NH < 0 || S < 0 || DH < 1 || DH > 512) return XLSTM_ERR_SHAPE;
     if ((long long)B * NH * S * DH > (1LL << 40) || (long long)B * NH > 0x7fffffffLL)
