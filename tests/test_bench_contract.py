@@ -41,3 +41,21 @@ def test_reference_arm_prints_one_complete_line():
 def test_fewer_than_three_warmup_steps_are_refused():
     r = _bench("--impl", "reference", "--steps", "1", "--warmup", "2")
     assert r.returncode != 0 and "warmup" in r.stderr
+
+
+def test_roofline_arithmetic_matches_the_stated_figures():
+    """Algorithmic bytes and useful flops of the long-context forward, as
+    stated for the roofline: 3080 B per token (bf16 q/k/v/h, fp32 otilde per
+    element, two fp32 gates) plus the final fp32 state, 405.8 MB per forward;
+    B*NH*S*(4 DH^2 + 2 (L+1) DH) useful flops, 3.87e10 at L = 64."""
+    sys.path.insert(0, ROOT)
+    import bench
+    from linear_rnn_mlstm_b200 import synthetic as syn
+    w = syn.LONG
+    assert bench.fwd_token_bytes(w.DH, 2) == 3080
+    per_step = w.B * w.NH * w.S * bench.fwd_token_bytes(w.DH, 2) + bench.state_bytes(w.B * w.NH, w.DH)
+    assert abs(per_step / 1e6 - 405.8) < 0.05
+    assert bench.kernel_algorithmic_bytes("segment_output_tc", w, {"P": 9}) == per_step
+    assert bench.kernel_algorithmic_bytes("gate_prologue", w, {"P": 9}) == w.B * w.NH * w.S * 12
+    flops = bench.fwd_flops(w.B * w.NH, w.S, w.DH, 64)
+    assert abs(flops / 1e10 - 3.87) < 0.005
