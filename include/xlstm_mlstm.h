@@ -85,7 +85,9 @@ const char *xlstm_status_string(xlstm_status status);
  * to *bytes; may be 0).  The workspace holds per-chunk gate prefix sums and,
  * when a head's sequence is split into segments that run in parallel, one
  * summary state per segment (the two-level chunk-state scan).  Same validation
- * as xlstm_mlstm_fwd.  Pure host function; touches no device.
+ * as xlstm_mlstm_fwd.  Launches nothing; it reads the current device's SM
+ * count (the segment plan fills one wave of SMs), and without a usable device
+ * plans for 148 SMs.  Ask with the device current that the forward will run on.
  */
 xlstm_status xlstm_mlstm_fwd_workspace_size(int B, int NH, int S, int DH, int chunk,
                                             xlstm_dtype dt, size_t *bytes);
@@ -124,6 +126,17 @@ xlstm_status xlstm_mlstm_fwd(const void *q, const void *k, const void *v,
                              xlstm_dtype dt, xlstm_fgate fg,
                              void *workspace, size_t workspace_bytes, void *cuda_stream);
 
+/*
+ * Which kernel family xlstm_mlstm_fwd_ex would run for these arguments
+ * (written to *path: XLSTM_PATH_SIMT or XLSTM_PATH_TENSOR), resolving
+ * XLSTM_PATH_AUTO; same validation and error codes as the forward for DH,
+ * chunk, dt and the options.  The paper has no counterpart: this lets a caller
+ * (and the tests) know whether the fp32 CUDA-core kernels or the tcgen05
+ * tensor-core kernels will compute the result.  Pure host function.
+ */
+xlstm_status xlstm_mlstm_fwd_path(int DH, int chunk, xlstm_dtype dt, const xlstm_fwd_options *opts,
+                                  int *path);
+
 /* As xlstm_mlstm_fwd, with explicit options (NULL = defaults). */
 xlstm_status xlstm_mlstm_fwd_ex(const void *q, const void *k, const void *v,
                                 const float *i_pre, const float *f_pre, const float *o_pre,
@@ -149,9 +162,11 @@ xlstm_status xlstm_mlstm_fwd_ex(const void *q, const void *k, const void *v,
  * holds until the process exits.
  *  - Calls whose xlstm_mlstm_fwd_workspace_size() exceeds that size return
  *    XLSTM_ERR_WORKSPACE and launch nothing.  Nothing is allocated, ever.
- *  - The first call on a device looks up the array's device address
- *    (cudaGetSymbolAddress) with that device current; make that first call
- *    before any stream capture.
+ *  - Every call looks up the array's device address (cudaGetSymbolAddress)
+ *    on the current device; the first call on a device also loads the
+ *    library's device code there, so make that first call before any stream
+ *    capture.  Nothing is cached between calls, so the entry point stays valid
+ *    after a cudaDeviceReset.
  *  - All calls share the one array: two calls whose kernels overlap on the GPU
  *    (different streams, or different host threads) race on it and give wrong
  *    results.  Serialise them, e.g. by issuing them on one stream.  The array
@@ -179,6 +194,9 @@ xlstm_status xlstm_mlstm_fwd_noalloc(const void *q, const void *k, const void *v
  *                read and overwritten with the state after this token.  This
  *                is exactly the state xlstm_mlstm_fwd returns.
  * DH: multiple of 16 in [16, 512].  B == 0 or NH == 0 is a no-op.
+ * If a bounded wait inside the step runs out (xlstm_device_status() then
+ * reports XLSTM_ERR_TIMEOUT), h and the state are undefined: synchronise and
+ * restore the state before the next step.
  */
 xlstm_status xlstm_mlstm_step(const void *q, const void *k, const void *v,
                               const float *i_pre, const float *f_pre, const float *o_pre,
@@ -291,6 +309,14 @@ xlstm_status xlstm_mlstm_headnorm_gate(const void *h, const float *gamma, const 
  * Synchronises `cuda_stream`, then reads and clears the device status word of
  * the current device.  Returns XLSTM_OK, XLSTM_ERR_TIMEOUT if a kernel gave up
  * a bounded wait since the last call, or XLSTM_ERR_CUDA.
+ *
+ * The status word is one per device and per process, shared by every stream
+ * and host thread, and this call clears it: a timeout latched by a kernel on
+ * another stream is reported (and consumed) by whichever caller reads the
+ * word first, and only work on `cuda_stream` is waited for.  Callers that use
+ * several streams should read it after synchronising all of them.  After a
+ * timeout the outputs of the call whose kernel gave up (h, the state) are
+ * undefined; synchronise and re-run that call before relying on them.
  */
 xlstm_status xlstm_device_status(void *cuda_stream);
 

@@ -28,7 +28,8 @@ EXPORTED = ("xlstm_abi_version", "xlstm_status_string", "xlstm_mlstm_fwd_workspa
             "xlstm_mlstm_fwd_workspace_size_ex", "xlstm_mlstm_fwd", "xlstm_mlstm_fwd_ex",
             "xlstm_mlstm_step", "xlstm_device_status", "xlstm_profile_begin", "xlstm_profile_end",
             "xlstm_mlstm_fwd_noalloc", "xlstm_selftest_wait_timeout", "xlstm_mlstm_headnorm_gate",
-            "xlstm_mlstm_bwd_workspace_size", "xlstm_mlstm_bwd", "xlstm_slstm_fwd")
+            "xlstm_mlstm_bwd_workspace_size", "xlstm_mlstm_bwd", "xlstm_slstm_fwd",
+            "xlstm_mlstm_fwd_path")
 NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
 
 
@@ -70,6 +71,8 @@ def load(path: str = LIB_PATH):
         lib.xlstm_mlstm_fwd_workspace_size_ex.argtypes = [i] * 6 + [ctypes.POINTER(FwdOptions),
                                                                    ctypes.POINTER(sz)]
         lib.xlstm_mlstm_fwd_workspace_size_ex.restype = i
+        lib.xlstm_mlstm_fwd_path.argtypes = [i] * 3 + [ctypes.POINTER(FwdOptions), ctypes.POINTER(i)]
+        lib.xlstm_mlstm_fwd_path.restype = i
         fwd_args = [vp] * 3 + [fp] * 3 + [vp] + [fp] * 6 + [i] * 7 + [vp, sz]
         lib.xlstm_mlstm_fwd.argtypes = fwd_args + [vp]
         lib.xlstm_mlstm_fwd.restype = i
@@ -115,6 +118,14 @@ def xlstm_mlstm_fwd_workspace_size(B, NH, S, DH, chunk, dt, path=PATH_AUTO, segm
     st = load().xlstm_mlstm_fwd_workspace_size_ex(B, NH, S, DH, chunk, dt, ctypes.byref(opts),
                                                    ctypes.byref(n))
     return st, n.value
+
+
+def xlstm_mlstm_fwd_path(DH, chunk, dt, path=PATH_AUTO, segments=0):
+    """(status, kernel family) the forward would run: PATH_SIMT or PATH_TENSOR."""
+    out = ctypes.c_int(0)
+    opts = FwdOptions(path, segments)
+    st = load().xlstm_mlstm_fwd_path(DH, chunk, dt, ctypes.byref(opts), ctypes.byref(out))
+    return st, out.value
 
 
 def xlstm_mlstm_fwd(q, k, v, i_pre, f_pre, o_pre, h, C0, n0, m0, C_out, n_out, m_out,

@@ -18,8 +18,20 @@ unsigned int *device_status_ptr() {
     return cudaGetSymbolAddress((void **)&p, g_device_status) == cudaSuccess ? p : nullptr;
 }
 
-constexpr int kNumSms = 148;               // B200
 constexpr int kMaxHeads = 65535;           // B * NH rides in a grid dimension
+
+// SM count of the current device, which the forward's segment plan fills one
+// wave of.  Without a usable device (a host-only process asking for a
+// workspace size) the plan is made for a full B200 (148 SMs).
+int num_sms_current_device() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+        cudaGetLastError();   // a failed query must not leak into a later launch check
+        return 148;
+    }
+    return n;
+}
 
 static size_t align64(size_t x) { return (x + 63) & ~size_t(63); }
 
@@ -90,7 +102,7 @@ __global__ void state_passthrough_kernel(const float *C0, const float *n0, const
 cudaError_t launch_state_passthrough(const FwdArgs &a, int BH, int DH, cudaStream_t st) {
     if (!a.C_out && !a.n_out && !a.m_out) return cudaSuccess;
     KernelTimer timer("state_passthrough", st);
-    state_passthrough_kernel<<<4 * kNumSms, 256, 0, st>>>(a.C0, a.n0, a.m0, a.C_out, a.n_out,
+    state_passthrough_kernel<<<4 * num_sms_current_device(), 256, 0, st>>>(a.C0, a.n0, a.m0, a.C_out, a.n_out,
                                                           a.m_out, BH, DH);
     return cudaGetLastError();
 }
@@ -164,9 +176,21 @@ xlstm_status xlstm_mlstm_fwd_workspace_size_ex(int B, int NH, int S, int DH, int
     const int path = resolve_path(dt, DH, chunk, opts, &st);
     if (st != XLSTM_OK) return st;
     FwdPlan p;
-    if (!make_fwd_plan(B, NH, S, DH, chunk, path, opts ? opts->segments : 0, kNumSms, &p))
+    if (!make_fwd_plan(B, NH, S, DH, chunk, path, opts ? opts->segments : 0, num_sms_current_device(), &p))
         return XLSTM_ERR_SHAPE;
     *bytes = p.bytes();
+    return XLSTM_OK;
+}
+
+xlstm_status xlstm_mlstm_fwd_path(int DH, int chunk, xlstm_dtype dt, const xlstm_fwd_options *opts,
+                                  int *path) {
+    if (!path) return XLSTM_ERR_NULL;
+    xlstm_status st = check_fwd_shape(1, 1, 1, DH, chunk, dt);
+    if (st != XLSTM_OK) return st;
+    if (opts && opts->segments < 0) return XLSTM_ERR_UNSUPPORTED;
+    const int p = resolve_path(dt, DH, chunk, opts, &st);
+    if (st != XLSTM_OK) return st;
+    *path = p;
     return XLSTM_OK;
 }
 
@@ -199,7 +223,7 @@ xlstm_status xlstm_mlstm_fwd_ex(const void *q, const void *k, const void *v,
     if ((C_out && C_out == C0) || (n_out && n_out == n0) || (m_out && m_out == m0))
         return XLSTM_ERR_UNSUPPORTED;
     FwdPlan plan;
-    if (!make_fwd_plan(B, NH, S, DH, chunk, path, opts ? opts->segments : 0, kNumSms, &plan))
+    if (!make_fwd_plan(B, NH, S, DH, chunk, path, opts ? opts->segments : 0, num_sms_current_device(), &plan))
         return XLSTM_ERR_SHAPE;
     if (plan.bytes() > 0 && (!workspace || workspace_bytes < plan.bytes())) return XLSTM_ERR_WORKSPACE;
 

@@ -11,10 +11,10 @@
 // The scratch is one file-scope device array of a fixed size.  Every GPU that
 // loads this library holds it until the process exits.  Host code cannot use
 // the array's name as a device address (in host code it names a host-side
-// stand-in), so the device address is fetched with cudaGetSymbolAddress once
-// per device, with that device current, on the first call made on it.
-#include <mutex>
-
+// stand-in), so every call fetches the device address with
+// cudaGetSymbolAddress, with the call's device current.  The address is not
+// cached: after a cudaDeviceReset, or under another context, the module is
+// loaded afresh and an address kept from before would be stale.
 #include "../../include/xlstm_mlstm.h"
 #include <cuda_runtime.h>
 
@@ -22,23 +22,11 @@ namespace {
 
 static __device__ __align__(256) unsigned char g_fwd_noalloc_scratch[XLSTM_NOALLOC_SCRATCH_BYTES];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_mu;
-void *g_scratch_ptr[kMaxDevices] = {};
-
-// Device address of the scratch array on the current device (set-up on first use).
+// Device address of the scratch array on the current device.
 xlstm_status scratch_for_current_device(void **out) {
-    int dev = -1;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return XLSTM_ERR_CUDA;
-    if (dev >= kMaxDevices) return XLSTM_ERR_UNSUPPORTED;
-    std::lock_guard<std::mutex> lk(g_mu);
-    if (!g_scratch_ptr[dev]) {
-        void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_fwd_noalloc_scratch) != cudaSuccess || !p)
-            return XLSTM_ERR_CUDA;
-        g_scratch_ptr[dev] = p;
-    }
-    *out = g_scratch_ptr[dev];
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_fwd_noalloc_scratch) != cudaSuccess || !p) return XLSTM_ERR_CUDA;
+    *out = p;
     return XLSTM_OK;
 }
 

@@ -30,7 +30,6 @@ namespace xlstm {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kNumSms = 148;           // B200
 
 // Elements per 16-byte vector.
 template <typename T> struct Vec;
@@ -241,12 +240,13 @@ cudaError_t launch_typed(const T *h, const float *gamma, const float *beta, cons
     const int lpr = lanes_per_row(nvec);
     int vpl = (nvec + lpr - 1) / lpr;                 // vectors per lane: 1, 2, 3 or 4
     if (vpl == 3) vpl = 4;
+    const int num_sms = num_sms_current_device();
     KernelTimer timer("headnorm_gate", st);
 #define XLSTM_HN_CASE(L, V)                                                                    \
     if (lpr == L && vpl == V) {                                                                \
         const long long per_block = (long long)(kThreads / 32) * (32 / L) * rows_per_pass(V);  \
         const long long needed = (rows + per_block - 1) / per_block;                           \
-        const long long wave = (long long)kNumSms * resident_blocks<T, L, V>();               \
+        const long long wave = (long long)num_sms * resident_blocks<T, L, V>();               \
         const dim3 grid((unsigned)(needed < wave ? needed : wave));                            \
         headnorm_gate_kernel<T, L, V><<<grid, kThreads, 0, st>>>(h, gamma, beta, skip_w,       \
                                                                  x_skip, z, y, rows, S, NH, DH, \

@@ -23,6 +23,9 @@ struct FwdArgs {
 // Address of the device status word on the current device (nullptr on failure).
 unsigned int *device_status_ptr();
 
+// SM count of the current device (148 when it cannot be queried).
+int num_sms_current_device();
+
 struct StepArgs {
     const void *q, *k, *v;
     const float *i_pre, *f_pre, *o_pre;

@@ -289,9 +289,17 @@ step_stream_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__
         __syncthreads();                      // part[] is rewritten by the next stage
     }
     if (tid == 0) {                           // nothing in flight at exit
-        if (!ok)                              // loads issued but maybe not consumed
-            for (int t = max(0, issued - kRing); t < issued; ++t)
-                ts::mbar_wait(&full[t % kRing], (t / kRing) & 1, nullptr, status);
+        if (!ok) {
+            // Loads issued but maybe not consumed.  One deadline (200 ms) covers
+            // the whole drain rather than a full wait per stage; the status word
+            // is already latched, and the call's outputs are undefined.
+            const uint64_t deadline = ts::globaltimer_ns() + 200000000ull;
+            for (int t = max(0, issued - kRing); t < issued; ++t) {
+                const uint64_t now = ts::globaltimer_ns();
+                const uint64_t left = now < deadline ? deadline - now : 0ull;
+                ts::mbar_wait(&full[t % kRing], (t / kRing) & 1, nullptr, status, left);
+            }
+        }
         asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
     }
 }

@@ -7,17 +7,22 @@ import torch
 import oracle
 from linear_rnn_mlstm_b200 import binding as xb
 
-# Tolerances on h: (max error, relative L2 over the whole tensor).  The max
-# error is normwise: max |got - ref| in units of max(1, max |ref|), i.e. an
-# absolute bound for outputs of unit scale and relative to the largest output
-# above that.  A literal absolute bound is unattainable for a bf16 output: |h|
-# reaches several hundred on these workloads, where one bf16 ulp is far larger
-# than 2e-2 (rounding the exact oracle output to bf16 alone exceeds it).  A
-# per-element relative bound is unattainable for any path with bf16 or tf32
-# tensor-core operands: where the terms of C'q cancel, their rounding error
-# (~1e-3 of the terms) is large relative to the small result.  The fp32 paths
-# also meet the stricter per-element bound (max |d| / max(1, |ref|) element by
-# element), which assert_close checks for them.
+# Tolerances on h: (max error, relative L2 over the whole tensor).
+#
+# bf16 inputs: the max error is taken token by token and is normwise within a
+# token: for every token t, max_j |dh_tj| / max(1, max_j |h_ref,tj|) <= 2e-2,
+# i.e. absolute for tokens whose output is of unit scale and relative to that
+# token's own largest output above it; relative L2 <= 1e-2 over the tensor.
+# A literal absolute bound is unattainable for a bf16 output: |h| reaches
+# several hundred on these workloads, where one bf16 ulp alone exceeds 2e-2.
+# A per-element relative bound is unattainable for tensor-core operands in
+# bf16: inside one token, an element where the terms of C'q cancel carries the
+# rounding error of the large terms.  Paths whose arithmetic is fp32 (the SIMT
+# kernels, on bf16 inputs too) are also held element by element:
+# max |dh| / max(1, |h_ref|) <= 2e-2 on every element.
+#
+# fp32 inputs: every element within 1e-5 (absolute for outputs of unit scale,
+# relative above), and relative L2 <= 1e-5.
 #
 # "f32_wide": fp32 inputs with wide input gates (itilde ~ N(0, 3)) and the
 # exponential forget gate.  There the stabiliser m reaches |m| ~ 10, so each
@@ -30,29 +35,47 @@ STATE_M_ABS = 1e-4         # final m
 
 
 def errors(got, ref):
-    """(max |got - ref| / max(1, max |ref|), ||got - ref||_2 / ||ref||_2,
-    max over elements of |got - ref| / max(1, |ref|))."""
+    """(max over tokens of max_j |d_tj| / max(1, max_j |ref_tj|),
+    ||got - ref||_2 / ||ref||_2, max over elements of |d| / max(1, |ref|)).
+    The last axis is the one a token's output spans (DH)."""
     got = np.asarray(got, dtype=np.float64)
     ref = np.asarray(ref, dtype=np.float64)
     diff = got - ref
     if diff.size == 0:
         return 0.0, 0.0, 0.0
-    max_norm = float(np.max(np.abs(diff))) / max(1.0, float(np.max(np.abs(ref))))
+    if ref.ndim == 0:
+        ref, diff = ref.reshape(1), diff.reshape(1)
+    tok_err = np.max(np.abs(diff), axis=-1) / np.maximum(1.0, np.max(np.abs(ref), axis=-1))
+    max_tok = float(np.max(tok_err))
     max_elem = float(np.max(np.abs(diff) / np.maximum(1.0, np.abs(ref))))
     denom = float(np.linalg.norm(ref))
     rel = float(np.linalg.norm(diff)) / denom if denom > 0 else float(np.linalg.norm(diff))
-    return max_norm, rel, max_elem
+    return max_tok, rel, max_elem
 
 
-def assert_close(got, ref, dtype, what="h"):
+def fp32_arith(DH, chunk, dtype, path=xb.PATH_AUTO):
+    """True if the forward for these arguments runs on the fp32 SIMT kernels."""
+    dt = xb.BF16 if dtype == "bf16" else xb.F32
+    st, fam = xb.xlstm_mlstm_fwd_path(DH, chunk, dt, path)
+    assert st == xb.OK, xb.status_string(st)
+    return fam == xb.PATH_SIMT
+
+
+def assert_close(got, ref, dtype, what="h", elementwise=None):
+    """`elementwise` (default: True for fp32 inputs) also holds every element
+    to the max-error bound; pass True for bf16 inputs on an fp32-arithmetic
+    path."""
     tol_abs, tol_rel = TOL[dtype]
-    max_norm, rel, max_elem = errors(got, ref)
-    ok = max_norm <= tol_abs and rel <= tol_rel
-    if dtype != "bf16":
+    max_tok, rel, max_elem = errors(got, ref)
+    if elementwise is None:
+        elementwise = dtype != "bf16"
+    ok = max_tok <= tol_abs and rel <= tol_rel
+    if elementwise:
         ok = ok and max_elem <= tol_abs
-    assert ok, (f"{what}: max|d|/max(1,max|ref|)={max_norm:.3e} (tol {tol_abs}), relL2={rel:.3e} "
-                f"(tol {tol_rel}), per-element max|d|/max(1,|ref|)={max_elem:.3e}")
-    return max_norm, rel
+    assert ok, (f"{what}: max over tokens of max|d|/max(1,max|ref|)={max_tok:.3e} (tol {tol_abs}), "
+                f"relL2={rel:.3e} (tol {tol_rel}), per-element max|d|/max(1,|ref|)={max_elem:.3e}"
+                f"{' (checked)' if elementwise else ''}")
+    return max_tok, rel
 
 
 def to_cuda(inp):

@@ -14,7 +14,7 @@ import oracle
 from linear_rnn_mlstm_b200 import binding as xb
 from linear_rnn_mlstm_b200 import synthetic as syn
 
-from parity import STATE_M_ABS, TOL, assert_close, errors, to_cuda
+from parity import STATE_M_ABS, TOL, assert_close, errors, fp32_arith, to_cuda
 
 pytestmark = pytest.mark.gpu
 
@@ -69,7 +69,8 @@ def test_prefill_then_steps_bf16():
                                      inp["o_pre"], Cr, nr, mr, d.fgate)
         hrs.append(hr)
     torch.cuda.synchronize()
-    assert_close(np.stack(hs), np.stack(hrs), "bf16")
+    # the steps are fp32 arithmetic; so is the prefill when it runs on the SIMT kernels
+    assert_close(np.stack(hs), np.stack(hrs), "bf16", elementwise=fp32_arith(d.DH, 64, "bf16"))
     assert errors(Cg.cpu().numpy(), Cr)[1] <= 1e-2
     assert np.max(np.abs(mg.cpu().numpy() - mr)) <= STATE_M_ABS
     assert xb.xlstm_device_status(_stream()) == xb.OK
@@ -110,7 +111,8 @@ def test_decode_workload_full_size_sampled_heads():
                                      Cr, nr, mr, d.fgate)
         hrs.append(hr[0])
     torch.cuda.synchronize()
-    assert_close(np.stack(hs), np.stack(hrs), "bf16")
+    assert_close(np.stack(hs), np.stack(hrs), "bf16",
+                 elementwise=fp32_arith(d.DH, d.prefill_chunk, "bf16"))
     assert errors(pick(Cg).cpu().numpy(), Cr[0])[1] <= 1e-2
     assert np.max(np.abs(pick(mg).cpu().numpy() - mr[0])) <= STATE_M_ABS
     assert xb.xlstm_device_status(_stream()) == xb.OK
