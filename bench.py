@@ -89,7 +89,7 @@ def source_sha(kernel):
     also depend on the tcgen05/TMA wrappers)."""
     files = {"segment_output_simt": ["fwd_simt.cu"], "segment_summary_simt": ["fwd_simt.cu"],
              "gate_prologue": ["fwd_simt.cu"], "step_rows": ["step.cu"], "step_state": ["step.cu"],
-             "headnorm_gate": ["headnorm.cu"]}
+             "headnorm_gate": ["headnorm.cu"], "segment_output_rs": ["fwd_rs.cu", "tc_ptx.cuh"]}
     fns = files.get(kernel)
     if fns is None and kernel.endswith("_tc"):
         fns = ["fwd_tc.cu", "tc_ptx.cuh"]
@@ -291,7 +291,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--config", default="long", choices=sorted(syn.WORKLOADS))
     ap.add_argument("--chunk", type=int, default=64)
-    ap.add_argument("--path", default="auto", choices=["auto", "simt", "tensor"])
+    ap.add_argument("--path", default="auto", choices=["auto", "simt", "tensor", "tensor_tmem"])
     ap.add_argument("--decode-steps", type=int, default=1024)
     ap.add_argument("--decode-B", type=int, default=0,
                     help="batch of the decode workload (0 = its full B of 256); profiling only")
@@ -314,7 +314,8 @@ def main():
     replicas.init(env, "nccl", dev, timeout_s=300)
     xb.load()
     peaks, peak_src = load_peaks()
-    path = {"auto": xb.PATH_AUTO, "simt": xb.PATH_SIMT, "tensor": xb.PATH_TENSOR}[args.path]
+    path = {"auto": xb.PATH_AUTO, "simt": xb.PATH_SIMT, "tensor": xb.PATH_TENSOR,
+            "tensor_tmem": xb.PATH_TENSOR_TMEM}[args.path]
 
     # ------------------------------------------------------------ forward
     w = syn.WORKLOADS[args.config]

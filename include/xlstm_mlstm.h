@@ -61,12 +61,17 @@ typedef enum { XLSTM_FGATE_SIGMOID = 0, XLSTM_FGATE_EXP = 1 } xlstm_fgate;
 typedef enum { XLSTM_OGATE_SILU = 0, XLSTM_OGATE_SIGMOID = 1 } xlstm_ogate;
 
 /* Kernel family for the forward.  AUTO picks the tensor-core (tcgen05) kernels
- * for bf16 inputs with DH 128 or 256 and chunk 64, and the fp32 SIMT kernels
- * for every other case.  SIMT forces the fp32-arithmetic kernels for any
- * supported arguments (a second, independent path the tests compare against).
- * TENSOR forces the tensor-core kernels; for arguments they do not take the
- * call returns XLSTM_ERR_UNSUPPORTED and launches nothing. */
-typedef enum { XLSTM_PATH_AUTO = 0, XLSTM_PATH_SIMT = 1, XLSTM_PATH_TENSOR = 2 } xlstm_path;
+ * for bf16 inputs where they apply (chunk 64 and DH 64, 128 or 256), and the
+ * fp32 SIMT kernels for every other case.  SIMT forces the fp32-arithmetic
+ * kernels for any supported arguments (a second, independent path the tests
+ * compare against).  TENSOR forces the tensor-core kernels; for arguments they
+ * do not take the call returns XLSTM_ERR_UNSUPPORTED and launches nothing.
+ * TENSOR_TMEM forces the older tensor-core output kernel that keeps the state
+ * in tensor memory and retrieves with tf32 operands (DH 128 or 256, chunk 64;
+ * about 11 significant bits in the retrieval), kept for comparison. */
+typedef enum {
+    XLSTM_PATH_AUTO = 0, XLSTM_PATH_SIMT = 1, XLSTM_PATH_TENSOR = 2, XLSTM_PATH_TENSOR_TMEM = 3
+} xlstm_path;
 
 typedef struct {
     int path;       /* xlstm_path                                                       */

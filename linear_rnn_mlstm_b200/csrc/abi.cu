@@ -42,7 +42,8 @@ bool make_fwd_plan(int B, int NH, int S, int DH, int L, int path, int forced_seg
     p->BH = B * NH;
     p->path = path;
     p->nchunks = S > 0 ? (S + L - 1) / L : 0;
-    if (path == XLSTM_PATH_TENSOR) {
+    const bool tensor = path == XLSTM_PATH_TENSOR || path == XLSTM_PATH_TENSOR_TMEM;
+    if (tensor) {
         p->rows = DH < 128 ? DH : 128;
     } else {
         p->rows = DH < 32 ? DH : 32;
@@ -57,7 +58,7 @@ bool make_fwd_plan(int B, int NH, int S, int DH, int L, int path, int forced_seg
     const long per_set = (long)p->BH * p->ntiles;
     if (forced_segments > 0) {
         P = forced_segments;
-    } else if (path == XLSTM_PATH_TENSOR) {
+    } else if (tensor) {
         // one CTA per SM (shared memory and TMEM are sized for that): fill one wave
         P = (int)(num_sms / per_set);
     } else {
@@ -65,7 +66,7 @@ bool make_fwd_plan(int B, int NH, int S, int DH, int L, int path, int forced_seg
         P = (int)((target + per_set - 1) / per_set);
     }
     if (P < 1) P = 1;
-    if (path == XLSTM_PATH_TENSOR) {
+    if (tensor) {
         // the per-CTA chunk tables hold a bounded number of chunks
         const int cap = tensor_path_max_chunks_per_segment();
         const int need = (p->nchunks + cap - 1) / cap;
@@ -127,23 +128,29 @@ static xlstm_status check_fwd_shape(int B, int NH, int S, int DH, int chunk, xls
     return XLSTM_OK;
 }
 
+static bool any_tensor_path(int DH, int chunk) {
+    return rs_path_supports(DH, chunk) || tensor_path_supports(DH, chunk);
+}
+
 static int resolve_path(xlstm_dtype dt, int DH, int chunk, const xlstm_fwd_options *opts,
                         xlstm_status *st) {
     *st = XLSTM_OK;
     const int want = opts ? opts->path : XLSTM_PATH_AUTO;
     if (want == XLSTM_PATH_SIMT) return XLSTM_PATH_SIMT;
-    if (want == XLSTM_PATH_TENSOR) {
-        if (dt != XLSTM_BF16 || !tensor_path_supports(DH, chunk)) {
+    if (want == XLSTM_PATH_TENSOR || want == XLSTM_PATH_TENSOR_TMEM) {
+        const bool ok = dt == XLSTM_BF16 && (want == XLSTM_PATH_TENSOR ? any_tensor_path(DH, chunk)
+                                                                       : tensor_path_supports(DH, chunk));
+        if (!ok) {
             *st = XLSTM_ERR_UNSUPPORTED;
             return 0;
         }
-        return XLSTM_PATH_TENSOR;
+        return want;
     }
     if (want != XLSTM_PATH_AUTO) {
         *st = XLSTM_ERR_UNSUPPORTED;
         return 0;
     }
-    if (dt == XLSTM_BF16 && tensor_path_supports(DH, chunk)) return XLSTM_PATH_TENSOR;
+    if (dt == XLSTM_BF16 && any_tensor_path(DH, chunk)) return XLSTM_PATH_TENSOR;
     return XLSTM_PATH_SIMT;
 }
 
@@ -239,7 +246,9 @@ xlstm_status xlstm_mlstm_fwd_ex(const void *q, const void *k, const void *v,
     cudaError_t e;
     if (S == 0) {
         e = launch_state_passthrough(a, plan.BH, DH, stream);
-    } else if (path == XLSTM_PATH_TENSOR) {
+    } else if (path == XLSTM_PATH_TENSOR && rs_path_supports(DH, chunk)) {
+        e = launch_fwd_rs(a, plan, stream);
+    } else if (path == XLSTM_PATH_TENSOR || path == XLSTM_PATH_TENSOR_TMEM) {
         e = launch_fwd_tensor(a, plan, stream);
     } else {
         e = launch_fwd_simt(a, plan, stream);

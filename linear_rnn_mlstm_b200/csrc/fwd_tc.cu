@@ -1005,6 +1005,9 @@ segment_summary_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __gri
                           unsigned int *status, int S, int nchunks, int P, int cps) {
     using Lay = SumLayout<D>;
     constexpr int NS = Lay::kStages;
+    // value rows of this CTA: 128, or all DH when DH < 128 (the MMAs keep M = 128;
+    // the second 64-row block of V stays zero, so rows >= DH of dC are zero)
+    constexpr int kVBlocks = D < 128 ? 1 : 2;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = align1024(smem_raw);
     float *fw = reinterpret_cast<float *>(smem + Lay::kF);
@@ -1053,6 +1056,8 @@ segment_summary_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __gri
     for (int e = tid; e < NS * 512; e += blockDim.x) {     // the W tiles start all zero
         const int st = e >> 9, off = (e & 511) * 16;
         *reinterpret_cast<uint4 *>(smem + st * Lay::kSlot + Lay::kKslot + 16384 + off) = make_uint4(0u, 0u, 0u, 0u);
+        if (kVBlocks == 1)                                  // and so does an unloaded V block
+            *reinterpret_cast<uint4 *>(smem + st * Lay::kSlot + Lay::kKslot + 8192 + off) = make_uint4(0u, 0u, 0u, 0u);
     }
     fence_async_smem();
     __syncthreads();
@@ -1071,10 +1076,10 @@ segment_summary_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __gri
                 const int slot = c % NS, t0 = (c0 + c) * kL;
                 if (c >= NS && !mbar_wait(&b_free[slot], ((c / NS) - 1) & 1, abort_flag, status)) break;
                 uint8_t *base = smem + slot * Lay::kSlot;
-                mbar_arrive_expect_tx(&b_full[slot], kL * D * 2 + kL * kRows * 2);
+                mbar_arrive_expect_tx(&b_full[slot], kL * D * 2 + kL * kVBlocks * 64 * 2);
                 for (int jb = 0; jb < D / 64; ++jb)
                     tma_load_3d(base + jb * 8192, &map_k, &b_full[slot], jb * 64, t0, bh);
-                for (int b = 0; b < 2; ++b)
+                for (int b = 0; b < kVBlocks; ++b)
                     tma_load_3d(base + Lay::kKslot + b * 8192, &map_v, &b_full[slot], i0 + 64 * b, t0, bh);
                 ++issued[slot];
             }
@@ -1137,7 +1142,7 @@ segment_summary_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __gri
             }
             named_sync_compute();
 #pragma unroll 4
-            for (int e = ct; e < 2 * kL * 8; e += 256) {   // V rows scaled in place by w
+            for (int e = ct; e < kVBlocks * kL * 8; e += 256) {   // V rows scaled in place by w
                 const int blk = e / (kL * 8), s = (e / 8) % kL, cc = e & 7;
                 uint4 *pv = reinterpret_cast<uint4 *>(sV + blk * 8192 + sw128_offset(s, cc));
                 const uint4 src = *pv;
@@ -1164,6 +1169,7 @@ segment_summary_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __gri
                 uint32_t r[16];
                 tmem_ld16(tacc + lane_addr + jb, r);
                 tmem_wait_ld();
+                if (i0 + i >= D) continue;                  // padding rows (DH < 128)
                 float4 *dst = reinterpret_cast<float4 *>(out + (size_t)(i0 + i) * D + jb);
 #pragma unroll
                 for (int e = 0; e < 4; ++e)
@@ -1195,12 +1201,65 @@ segment_summary_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __gri
 }
 
 // ------------------------------------------------------------------- host
+template <int D>
+cudaError_t launch_summaries_t(const FwdArgs &a, const FwdPlan &p, cudaStream_t st) {
+    if (p.P <= 1) return cudaSuccess;
+    CUtensorMap mk, mv;
+    if (!make_map_bf16(&mk, a.k, p.BH, p.S, D) || !make_map_bf16(&mv, a.v, p.BH, p.S, D))
+        return cudaErrorInvalidValue;
+    float *ws = (float *)a.workspace;
+    const float *bcum = ws + p.off_bcum;
+    const float2 *cstat = (const float2 *)(ws + p.off_cstat);
+    float2 *sstat = (float2 *)(ws + p.off_sstat);
+    float *summ = ws + p.off_summ;
+    const int sm = SumLayout<D>::kBytes;
+    cudaError_t e = cudaFuncSetAttribute(segment_summary_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
+    if (e != cudaSuccess) return e;
+    {
+        KernelTimer timer("segment_summary_tc", st);
+        segment_summary_tc_kernel<D><<<dim3((D + kRows - 1) / kRows, p.P - 1, p.BH), kThreads, sm, st>>>(
+            mk, mv, a.i_pre, bcum, cstat, sstat, summ, a.status, p.S, p.nchunks, p.P, p.cps);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    KernelTimer timer("segment_scan", st);
+    const size_t per4 = ((size_t)D * D + D) / 4;
+    segment_scan_kernel<<<dim3((unsigned)((per4 + 255) / 256), p.BH), 256, 0, st>>>(
+        sstat, summ, a.C0, a.n0, a.m0, D, p.P);
+    return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_tc_t(const FwdArgs &a, const FwdPlan &p, cudaStream_t st) {
+    CUtensorMap mq, mk, mv, mh, mo;
+    if (!make_map_bf16(&mq, a.q, p.BH, p.S, D) || !make_map_bf16(&mk, a.k, p.BH, p.S, D) ||
+        !make_map_bf16(&mv, a.v, p.BH, p.S, D) || !make_map_bf16(&mh, a.h, p.BH, p.S, D, false, 32) ||
+        !make_map_f32_rows(&mo, a.o_pre, p.BH, p.S, D))
+        return cudaErrorInvalidValue;
+    float *ws = (float *)a.workspace;
+    const float *bcum = ws + p.off_bcum;
+    const float2 *cstat = (const float2 *)(ws + p.off_cstat);
+    float2 *sstat = (float2 *)(ws + p.off_sstat);
+    float *summ = ws + p.off_summ;
+    cudaError_t e = launch_summaries_t<D>(a, p, st);
+    if (e != cudaSuccess) return e;
+    const int sm = OutLayout<D>::kBytes;
+    e = cudaFuncSetAttribute(segment_output_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
+    if (e != cudaSuccess) return e;
+    KernelTimer timer("segment_output_tc", st);
+    segment_output_tc_kernel<D><<<dim3(D / kRows, p.P, p.BH), kOutThreads, sm, st>>>(
+        mq, mk, mv, mh, mo, a.i_pre, a.o_pre, a.C0, a.n0, a.m0, a.C_out, a.n_out, a.m_out,
+        bcum, ws + p.off_pmax, cstat, sstat, summ, a.status, p.S, p.nchunks, p.P, p.cps);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *,
                                   CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
                                   CUtensorMapFloatOOBfill);
 
-EncodeTiledFn encode_fn() {
+static EncodeTiledFn encode_fn() {
     static std::once_flag once;
     static EncodeTiledFn fn = nullptr;
     std::call_once(once, [] {
@@ -1213,23 +1272,19 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// [BH, S, D] fp32, box 128 x 64 x 1, no swizzle: L2 prefetches of the output gates.
-bool make_map_f32_rows(CUtensorMap *m, const void *base, int BH, int S, int D) {
+bool make_map_f32_rows(CUtensorMap *m, const void *base, int BH, int S, int D, int box_cols, int box_rows) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)S, (cuuint64_t)BH};
     cuuint64_t strides[2] = {(cuuint64_t)D * 4, (cuuint64_t)S * D * 4};
-    cuuint32_t box[3] = {128, 64, 1};
+    cuuint32_t box[3] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows, 1};
     cuuint32_t es[3] = {1, 1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void *>(base), dims, strides, box, es,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// [BH, S, D] bf16, box 64 x box_rows x 1.  The q/k/v loads use the 128-byte
-// swizzle (rows past S read as zeros); the h stores use no swizzle and 32-row
-// boxes (rows past S are not written).
-bool make_map(CUtensorMap *m, const void *base, int BH, int S, int D, bool swizzle = true, int box_rows = 64) {
+bool make_map_bf16(CUtensorMap *m, const void *base, int BH, int S, int D, bool swizzle, int box_rows) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)S, (cuuint64_t)BH};
@@ -1241,48 +1296,14 @@ bool make_map(CUtensorMap *m, const void *base, int BH, int S, int D, bool swizz
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int D>
-cudaError_t launch_tc_t(const FwdArgs &a, const FwdPlan &p, cudaStream_t st) {
-    CUtensorMap mq, mk, mv, mh, mo;
-    if (!make_map(&mq, a.q, p.BH, p.S, D) || !make_map(&mk, a.k, p.BH, p.S, D) ||
-        !make_map(&mv, a.v, p.BH, p.S, D) || !make_map(&mh, a.h, p.BH, p.S, D, false, 32) ||
-        !make_map_f32_rows(&mo, a.o_pre, p.BH, p.S, D))
-        return cudaErrorInvalidValue;
-    float *ws = (float *)a.workspace;
-    const float *bcum = ws + p.off_bcum;
-    const float2 *cstat = (const float2 *)(ws + p.off_cstat);
-    float2 *sstat = (float2 *)(ws + p.off_sstat);
-    float *summ = ws + p.off_summ;
-    cudaError_t e;
-    if (p.P > 1) {
-        const int sm = SumLayout<D>::kBytes;
-        e = cudaFuncSetAttribute(segment_summary_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
-        if (e != cudaSuccess) return e;
-        {
-            KernelTimer timer("segment_summary_tc", st);
-            segment_summary_tc_kernel<D><<<dim3(D / kRows, p.P - 1, p.BH), kThreads, sm, st>>>(
-                mk, mv, a.i_pre, bcum, cstat, sstat, summ, a.status, p.S, p.nchunks, p.P, p.cps);
-            if ((e = cudaGetLastError()) != cudaSuccess) return e;
-        }
-        {
-            KernelTimer timer("segment_scan", st);
-            const size_t per4 = ((size_t)D * D + D) / 4;
-            segment_scan_kernel<<<dim3((unsigned)((per4 + 255) / 256), p.BH), 256, 0, st>>>(
-                sstat, summ, a.C0, a.n0, a.m0, D, p.P);
-            if ((e = cudaGetLastError()) != cudaSuccess) return e;
-        }
+cudaError_t launch_segment_summaries(const FwdArgs &a, const FwdPlan &p, cudaStream_t st) {
+    switch (p.DH) {
+        case 64: return launch_summaries_t<64>(a, p, st);
+        case 128: return launch_summaries_t<128>(a, p, st);
+        case 256: return launch_summaries_t<256>(a, p, st);
     }
-    const int sm = OutLayout<D>::kBytes;
-    e = cudaFuncSetAttribute(segment_output_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
-    if (e != cudaSuccess) return e;
-    KernelTimer timer("segment_output_tc", st);
-    segment_output_tc_kernel<D><<<dim3(D / kRows, p.P, p.BH), kOutThreads, sm, st>>>(
-        mq, mk, mv, mh, mo, a.i_pre, a.o_pre, a.C0, a.n0, a.m0, a.C_out, a.n_out, a.m_out,
-        bcum, ws + p.off_pmax, cstat, sstat, summ, a.status, p.S, p.nchunks, p.P, p.cps);
-    return cudaGetLastError();
+    return cudaErrorInvalidValue;
 }
-
-}  // namespace
 
 bool tensor_path_supports(int DH, int L) { return L == kL && (DH == 128 || DH == 256); }
 

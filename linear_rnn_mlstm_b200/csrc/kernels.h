@@ -1,6 +1,7 @@
 // Internal launch interface between the C ABI (abi.cu) and the kernel files.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 
@@ -38,12 +39,26 @@ struct StepArgs {
 };
 
 cudaError_t launch_gate_prologue(const FwdArgs &a, const FwdPlan &p, cudaStream_t st);
+// Segment summaries + segment scan of the two-level chunk-state scan, on the
+// tensor cores (bf16, DH 64, 128 or 256); nothing when the plan has one segment.
+cudaError_t launch_segment_summaries(const FwdArgs &a, const FwdPlan &p, cudaStream_t st);
 cudaError_t launch_fwd_simt(const FwdArgs &a, const FwdPlan &p, cudaStream_t st);
 cudaError_t launch_fwd_tensor(const FwdArgs &a, const FwdPlan &p, cudaStream_t st);
 bool tensor_path_supports(int DH, int L);
+// Register-state tensor-core forward (fwd_rs.cu): bf16, chunk 64, DH 64 / 128 / 256.
+bool rs_path_supports(int DH, int L);
+cudaError_t launch_fwd_rs(const FwdArgs &a, const FwdPlan &p, cudaStream_t st);
 int tensor_path_max_chunks_per_segment();
 cudaError_t launch_state_passthrough(const FwdArgs &a, int BH, int DH, cudaStream_t st);
 cudaError_t launch_step(const StepArgs &a, cudaStream_t st);
+
+// TMA descriptors over a [BH, S, D] tensor: bf16 with 64-column boxes of
+// `box_rows` rows (128-byte swizzle or none), or fp32 with box_cols x box_rows
+// boxes and no swizzle.  False if the driver refuses the encoding.
+bool make_map_bf16(CUtensorMap *m, const void *base, int BH, int S, int D, bool swizzle = true,
+                   int box_rows = 64);
+bool make_map_f32_rows(CUtensorMap *m, const void *base, int BH, int S, int D, int box_cols = 128,
+                       int box_rows = 64);
 
 size_t simt_summary_smem(int DH, int rows);
 size_t simt_output_smem(int DH, int rows, int L);

@@ -1,6 +1,8 @@
-"""The tensor-core forward (bf16, chunk 64, DH 128 or 256) against the float64
-oracle, forced through the tensor path, on the cases its design has to get
-right beyond the plain workloads:
+"""The tensor-core forwards (bf16, chunk 64) against the float64 oracle, forced
+through the tensor path, on the cases their design has to get right beyond the
+plain workloads.  Two kernel families: the register-state kernel (DH 64, 128,
+256; XLSTM_PATH_TENSOR) and the tensor-memory-state kernel (DH 128, 256;
+XLSTM_PATH_TENSOR_TMEM).  Cases:
 
 - several value-row tiles and several segments per head, ragged tails;
 - the exponential forget gate;
@@ -24,12 +26,19 @@ from parity import STATE_M_ABS, STATE_REL_L2, assert_close, errors, gpu_fwd, ora
 pytestmark = pytest.mark.gpu
 
 
-def _check(inp, fgate, seg, C0=None, n0=None, m0=None):
+FAMILIES = [xb.PATH_TENSOR, xb.PATH_TENSOR_TMEM]
+
+
+def _check(inp, fgate, seg, C0=None, n0=None, m0=None, families=FAMILIES):
     hr, Cr, nr, mr = oracle_fwd(inp, fgate, C0, n0, m0)
-    h, C, n, m = gpu_fwd(inp, 64, fgate, xb.PATH_TENSOR, seg, C0, n0, m0)
-    assert_close(h, hr, "bf16")
-    assert errors(C, Cr)[1] <= STATE_REL_L2 and errors(n, nr)[1] <= STATE_REL_L2
-    assert np.max(np.abs(m - mr)) <= STATE_M_ABS
+    DH = inp["q"].shape[-1]
+    for fam in families:
+        if fam == xb.PATH_TENSOR_TMEM and DH not in (128, 256):
+            continue
+        h, C, n, m = gpu_fwd(inp, 64, fgate, fam, seg, C0, n0, m0)
+        assert_close(h, hr, "bf16", what=f"h (family {fam})")
+        assert errors(C, Cr)[1] <= STATE_REL_L2 and errors(n, nr)[1] <= STATE_REL_L2
+        assert np.max(np.abs(m - mr)) <= STATE_M_ABS
 
 
 CASES = [
@@ -43,6 +52,9 @@ CASES = [
     (1, 1, 1, 128, "sigmoid", 0),
     (1, 1, 63, 256, "exp", 0),
     (2, 1, 640, 256, "sigmoid", 10),
+    (1, 1, 64, 64, "sigmoid", 0),
+    (2, 3, 777, 64, "sigmoid", 4),
+    (1, 2, 300, 64, "exp", 0),
 ]
 
 
@@ -54,7 +66,7 @@ def test_tensor_path_vs_oracle(case):
     _check(syn.fwd_inputs(w), fgate, seg)
 
 
-@pytest.mark.parametrize("DH", [128, 256])
+@pytest.mark.parametrize("DH", [64, 128, 256])
 def test_tensor_path_rescaled_state(DH):
     # log sigmoid(1 +- 0.5) ~ -0.3 per token: the state's scale falls below
     # e^-40 every few chunks and is reset in TMEM
@@ -93,11 +105,13 @@ def test_tensor_path_initial_state():
         _check(inp, "sigmoid", seg, C0, n0, m0)
 
 
-@pytest.mark.parametrize("dtype,DH,chunk", [("f32", 128, 64), ("bf16", 64, 64), ("bf16", 128, 128)])
-def test_tensor_path_refuses_unsupported(dtype, DH, chunk):
+@pytest.mark.parametrize("dtype,DH,chunk,fam", [("f32", 128, 64, xb.PATH_TENSOR), ("bf16", 48, 64, xb.PATH_TENSOR),
+                                                ("bf16", 64, 64, xb.PATH_TENSOR_TMEM),
+                                                ("bf16", 128, 128, xb.PATH_TENSOR_TMEM)])
+def test_tensor_path_refuses_unsupported(dtype, DH, chunk, fam):
     w = syn.custom("tc_unsup", 1, 1, 128, DH, syn.SMALL, dtype=dtype, seed=1)
     d = to_cuda(syn.fwd_inputs(w))
     with pytest.raises(xb.XlstmError) as err:
         xb.mlstm_fwd(d["q"], d["k"], d["v"], d["i_pre"], d["f_pre"], d["o_pre"], chunk=chunk,
-                     path=xb.PATH_TENSOR)
+                     path=fam)
     assert err.value.status == xb.ERR_UNSUPPORTED
