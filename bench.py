@@ -291,7 +291,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--config", default="long", choices=sorted(syn.WORKLOADS))
     ap.add_argument("--chunk", type=int, default=64)
-    ap.add_argument("--path", default="auto", choices=["auto", "simt", "tensor", "tensor_tmem"])
+    ap.add_argument("--path", default="auto", choices=["auto", "simt", "tensor", "tensor_tmem", "tensor_rs"])
     ap.add_argument("--decode-steps", type=int, default=1024)
     ap.add_argument("--decode-B", type=int, default=0,
                     help="batch of the decode workload (0 = its full B of 256); profiling only")
@@ -299,6 +299,8 @@ def main():
     ap.add_argument("--skip-e2e", action="store_true")
     ap.add_argument("--skip-epilogue", action="store_true")
     ap.add_argument("--skip-cpu", action="store_true")
+    ap.add_argument("--skip-sweep", action="store_true",
+                    help="skip the per-config / per-chunk entries (small, block, long at 128 and 256)")
     ap.add_argument("--ref-tokens", type=int, default=4096,
                     help="tokens per head in each reference (oracle) step")
     args = ap.parse_args()
@@ -315,7 +317,7 @@ def main():
     xb.load()
     peaks, peak_src = load_peaks()
     path = {"auto": xb.PATH_AUTO, "simt": xb.PATH_SIMT, "tensor": xb.PATH_TENSOR,
-            "tensor_tmem": xb.PATH_TENSOR_TMEM}[args.path]
+            "tensor_tmem": xb.PATH_TENSOR_TMEM, "tensor_rs": xb.PATH_TENSOR_RS}[args.path]
 
     # ------------------------------------------------------------ forward
     w = syn.WORKLOADS[args.config]
@@ -360,24 +362,7 @@ def main():
     # ------------------------------------------------------------- end to end
     e2e = None
     if not args.skip_e2e:
-        pin = {k: v.pin_memory() for k, v in inp.items()}
-        h, C, n, m = outs
-        out_host = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in (h, C, n, m)]
-        dev_in = x
-
-        def e2e_step():
-            for k in dev_in:
-                dev_in[k].copy_(pin[k], non_blocking=True)
-            run()
-            for hst, dv in zip(out_host, (h, C, n, m)):
-                hst.copy_(dv, non_blocking=True)
-        for _ in range(2):
-            e2e_step()
-        ms_e2e = time_region(e2e_step, max(3, min(args.steps, 10)), env, dev) / max(3, min(args.steps, 10))
-        h2d = sum(t.numel() * t.element_size() for t in pin.values())
-        d2h = sum(t.numel() * t.element_size() for t in out_host)
-        e2e = {"value": replicas.job_throughput(tokens, env, ms_e2e * 1e-3), "unit": "tokens/s",
-               "ms_per_step": ms_e2e, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+        e2e = run_e2e(args, w, inp, x, outs, run, dev, env, path)
     del x, outs, run
 
     # -------------------------------------------------- block epilogue (next row)
@@ -390,6 +375,11 @@ def main():
     if not args.skip_decode:
         decode = run_decode(args, dev, env, peaks, peak_src)
 
+    # ------------------------------------------- every config and chunk size
+    sweep = None
+    if not args.skip_sweep:
+        sweep = run_sweep(args, dev, env, peaks, peak_src, with_cpu=(rank == 0 and world == 1 and not args.skip_cpu))
+
     clocks = sampler.stop() if sampler else None
 
     # ------------------------------------------------------------ CPU baseline
@@ -401,7 +391,7 @@ def main():
         line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-                "dtype": "bf16" if (w.dtype == "bf16" and any(k.endswith("_tc") for k in kt)) else "f32",
+                "dtype": "bf16" if (w.dtype == "bf16" and any(k.endswith(("_tc", "_rs")) for k in kt)) else "f32",
                 "data": "synthetic (seeded N(0,1)-based draws of the workload shapes)",
                 "config": dict(workload_config(w, args.chunk, world),
                                l2="inputs 406 MB > 126 MB L2; no flush" if w.name == "long"
@@ -409,11 +399,155 @@ def main():
                                path=args.path),
                 "roofline": roofline, "tc": tc, "hbm_whole_step": whole,
                 "kernels": kernels, "gpu_launches": launches, "cpu_baseline": cpu, "e2e": e2e,
-                "clocks": clocks, "decode": decode, "epilogue": epilogue}
+                "clocks": clocks, "decode": decode, "epilogue": epilogue, "sweep": sweep}
         print(json.dumps(line), flush=True)
     replicas.barrier(env)
     replicas.shutdown(env)
     return 0
+
+
+SWEEP = (("small", 64), ("block", 64), ("block", 128), ("long", 128), ("long", 256))
+SWEEP_CPU_TOKENS = {"small": 1024, "block": 256, "long": 1024}
+
+
+def path_name(w, chunk):
+    st, fam = xb.xlstm_mlstm_fwd_path(w.DH, chunk, xb.BF16 if w.dtype == "bf16" else xb.F32)
+    return {xb.PATH_TENSOR: "tensor (tcgen05)", xb.PATH_SIMT: "simt (fp32 CUDA cores)"}.get(fam, str(fam))
+
+
+def run_sweep(args, dev, env, peaks, peak_src, with_cpu):
+    """The other forward configurations and chunk sizes, each timed on its own
+    (AUTO path, which kernel family ran is named): per step, the L2 is flushed
+    by writing a 256 MB buffer outside the timed events, then one forward is
+    timed with CUDA events; the median over the steps is reported.  Each entry
+    carries tokens/s, useful TFLOP/s, the whole-step HBM fraction, the dominant
+    kernel's roofline and the float64 oracle on a bounded sample beside it."""
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    out = []
+    for name, chunk in SWEEP:
+        w = syn.WORKLOADS[name]
+        inp = syn.fwd_inputs(w, seed=replicas.replica_seed(w.seed, env.rank))
+        x = {k: v.to(dev).contiguous() for k, v in inp.items()}
+        run, outs, BH = make_fwd_runner(x, w, chunk, dev, xb.PATH_AUTO)
+        for _ in range(3):
+            run()
+        torch.cuda.synchronize(dev)
+        steps = max(5, min(args.steps, 10))
+        times = []
+        xb.xlstm_profile_begin()
+        for _ in range(steps):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            run()
+            e1.record()
+            torch.cuda.synchronize(dev)
+            times.append(e0.elapsed_time(e1))
+        _, kt = xb.xlstm_profile_end()
+        ms = replicas.max_over_ranks(statistics.median(times), env, dev)
+        tokens = w.B * w.NH * w.S
+        eb = 2 if w.dtype == "bf16" else 4
+        step_bytes = tokens * fwd_token_bytes(w.DH, eb) + state_bytes(BH, w.DH)
+        flops = fwd_flops(BH, w.S, w.DH, chunk)
+        kernels = {k: {"launches": v[0], "avg_us": 1e3 * v[1] / max(v[0], 1)} for k, v in kt.items()}
+        top = max(kt.items(), key=lambda kv: kv[1][1])[0] if kt else None
+        roof = None
+        if top:
+            alg = kernel_algorithmic_bytes(top, w, plan_info(w, chunk, xb.PATH_AUTO))
+            if alg:
+                ach = alg / (kernels[top]["avg_us"] * 1e-6) / 1e9
+                roof = {"kernel": top, "bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"],
+                        "unit": "GB/s", "frac": ach / peaks["hbm_gbs"], "algorithmic_bytes": alg,
+                        "note": "kernel average over the flushed steps"}
+        entry = {"workload": workload_config(w, chunk, env.world)["workload"], "chunk": chunk,
+                 "path": path_name(w, chunk), "ms_per_step": ms,
+                 "tokens_per_s": replicas.job_throughput(tokens, env, ms * 1e-3),
+                 "useful_tflops": flops / (ms * 1e-3) / 1e12,
+                 "tc_frac": flops / (ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
+                 "hbm_frac_whole_step": step_bytes / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                 "algorithmic_bytes_per_step": step_bytes, "useful_flops_per_step": flops,
+                 "l2": "256 MB flush before every timed step", "roofline": roof, "kernels": kernels,
+                 "peak_source": f"{peak_src} (burst copy / burst cuBLAS bf16)"}
+        if with_cpu:
+            entry["cpu_baseline"] = cpu_baseline(w, SWEEP_CPU_TOKENS[name])
+        out.append(entry)
+        del x, outs, run
+    del flush
+    return out
+
+
+def run_e2e(args, w, inp, x, outs, run, dev, env, path):
+    """End to end through the C ABI with host buffers: every step copies that
+    step's inputs from pinned host memory to the device, runs the forward and
+    copies h and the final state back.  Steps are pipelined over two device
+    buffer sets and three streams (upload, compute, download), so the upload
+    of step k+1 and the download of step k-1 overlap the forward of step k
+    (PCIe is full duplex); every copy of every timed step is inside the timed
+    region, which ends when the last download has landed."""
+    pin = {k: v.pin_memory() for k, v in inp.items()}
+    x2 = {k: torch.empty_like(v) for k, v in x.items()}
+    run2, outs2, _ = make_fwd_runner(x2, w, args.chunk, dev, path)
+    bufs = [(x, outs, run), (x2, outs2, run2)]
+    hosts = [[torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outs] for _ in range(2)]
+    comp = torch.cuda.current_stream(dev)
+    up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_comp = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
+    for e in ev_comp + ev_out:
+        e.record(comp)
+    state = {"k": 0}
+
+    def step():
+        k = state["k"]
+        state["k"] += 1
+        b = k % 2
+        xin, yout, fn = bufs[b]
+        with torch.cuda.stream(up):
+            up.wait_event(ev_comp[b])                 # the forward that last read these inputs
+            for name in xin:
+                xin[name].copy_(pin[name], non_blocking=True)
+            ev_in[b].record(up)
+        comp.wait_event(ev_in[b])
+        comp.wait_event(ev_out[b])                    # the download that last read these outputs
+        fn()
+        ev_comp[b].record(comp)
+        with torch.cuda.stream(down):
+            down.wait_event(ev_comp[b])
+            for hst, dv in zip(hosts[b], yout):
+                hst.copy_(dv, non_blocking=True)
+            ev_out[b].record(down)
+
+    def drain():
+        comp.wait_event(ev_out[0])
+        comp.wait_event(ev_out[1])
+
+    for _ in range(2):
+        step()
+    drain()
+    torch.cuda.synchronize(dev)
+    steps = max(3, min(args.steps, 10))
+
+    def timed():
+        step()
+    replicas.barrier(env)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(comp)
+    for _ in range(steps):
+        timed()
+    drain()
+    e1.record(comp)
+    torch.cuda.synchronize(dev)
+    replicas.barrier(env)
+    ms_e2e = replicas.max_over_ranks(e0.elapsed_time(e1), env, dev) / steps
+    tokens = w.B * w.NH * w.S
+    h2d = sum(t.numel() * t.element_size() for t in pin.values())
+    d2h = sum(t.numel() * t.element_size() for t in hosts[0])
+    del x2, outs2, run2
+    return {"value": replicas.job_throughput(tokens, env, ms_e2e * 1e-3), "unit": "tokens/s",
+            "ms_per_step": ms_e2e, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "pipelined": "upload, forward, download on three streams over two buffer sets"}
 
 
 def run_epilogue(args, w, dev, env, peaks, peak_src):

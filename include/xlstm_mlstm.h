@@ -66,11 +66,15 @@ typedef enum { XLSTM_OGATE_SILU = 0, XLSTM_OGATE_SIGMOID = 1 } xlstm_ogate;
  * kernels for any supported arguments (a second, independent path the tests
  * compare against).  TENSOR forces the tensor-core kernels; for arguments they
  * do not take the call returns XLSTM_ERR_UNSUPPORTED and launches nothing.
- * TENSOR_TMEM forces the older tensor-core output kernel that keeps the state
- * in tensor memory and retrieves with tf32 operands (DH 128 or 256, chunk 64;
- * about 11 significant bits in the retrieval), kept for comparison. */
+ * Two tensor-core output kernels exist: one keeps the state in tensor memory
+ * and retrieves with tf32 operands (TENSOR_TMEM: DH 128 or 256, chunk 64;
+ * about 11 significant bits in the retrieval), the other keeps the state in
+ * fp32 registers and retrieves with two bf16 parts (TENSOR_RS: DH 64, 128 or
+ * 256, chunk 64; 15 to 16 bits).  TENSOR takes TENSOR_TMEM where it applies
+ * (it is the faster at DH 128 / 256) and TENSOR_RS elsewhere. */
 typedef enum {
-    XLSTM_PATH_AUTO = 0, XLSTM_PATH_SIMT = 1, XLSTM_PATH_TENSOR = 2, XLSTM_PATH_TENSOR_TMEM = 3
+    XLSTM_PATH_AUTO = 0, XLSTM_PATH_SIMT = 1, XLSTM_PATH_TENSOR = 2, XLSTM_PATH_TENSOR_TMEM = 3,
+    XLSTM_PATH_TENSOR_RS = 4
 } xlstm_path;
 
 typedef struct {

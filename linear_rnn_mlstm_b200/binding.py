@@ -22,7 +22,7 @@ OK, ERR_NULL, ERR_SHAPE, ERR_DTYPE, ERR_CHUNK, ERR_ALIGN, ERR_CUDA, ERR_TIMEOUT,
 F32, BF16 = 0, 1
 FGATE_SIGMOID, FGATE_EXP = 0, 1
 OGATE_SILU, OGATE_SIGMOID = 0, 1
-PATH_AUTO, PATH_SIMT, PATH_TENSOR, PATH_TENSOR_TMEM = 0, 1, 2, 3
+PATH_AUTO, PATH_SIMT, PATH_TENSOR, PATH_TENSOR_TMEM, PATH_TENSOR_RS = 0, 1, 2, 3, 4
 
 EXPORTED = ("xlstm_abi_version", "xlstm_status_string", "xlstm_mlstm_fwd_workspace_size",
             "xlstm_mlstm_fwd_workspace_size_ex", "xlstm_mlstm_fwd", "xlstm_mlstm_fwd_ex",

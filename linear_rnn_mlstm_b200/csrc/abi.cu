@@ -42,7 +42,7 @@ bool make_fwd_plan(int B, int NH, int S, int DH, int L, int path, int forced_seg
     p->BH = B * NH;
     p->path = path;
     p->nchunks = S > 0 ? (S + L - 1) / L : 0;
-    const bool tensor = path == XLSTM_PATH_TENSOR || path == XLSTM_PATH_TENSOR_TMEM;
+    const bool tensor = path == XLSTM_PATH_TENSOR || path == XLSTM_PATH_TENSOR_TMEM || path == XLSTM_PATH_TENSOR_RS;
     if (tensor) {
         p->rows = DH < 128 ? DH : 128;
     } else {
@@ -55,7 +55,8 @@ bool make_fwd_plan(int B, int NH, int S, int DH, int L, int path, int forced_seg
         return true;
     }
     int P;
-    const long per_set = (long)p->BH * p->ntiles;
+    // DH 512 on the tensor path splits each value tile's keys over two CTAs
+    const long per_set = (long)p->BH * p->ntiles * (tensor && DH > 256 ? 2 : 1);
     if (forced_segments > 0) {
         P = forced_segments;
     } else if (tensor) {
@@ -83,6 +84,11 @@ bool make_fwd_plan(int B, int NH, int S, int DH, int L, int path, int forced_seg
     p->off_cstat = off; off = align64(off + (size_t)p->BH * p->nchunks * 2);
     p->off_sstat = off; off = align64(off + (size_t)p->BH * p->P * 2);
     p->off_summ = off;  off = align64(off + (size_t)p->BH * (p->P - 1) * ((size_t)DH * DH + DH));
+    if (tensor && DH > 256) {
+        p->off_part = off;  off = align64(off + 2 * (size_t)p->BH * S * DH);
+        p->off_dpart = off; off = align64(off + 2 * (size_t)p->BH * S);
+        p->off_tok = off;   off = align64(off + 2 * (size_t)p->BH * S);
+    }
     p->total_floats = off;
     return true;
 }
@@ -137,9 +143,10 @@ static int resolve_path(xlstm_dtype dt, int DH, int chunk, const xlstm_fwd_optio
     *st = XLSTM_OK;
     const int want = opts ? opts->path : XLSTM_PATH_AUTO;
     if (want == XLSTM_PATH_SIMT) return XLSTM_PATH_SIMT;
-    if (want == XLSTM_PATH_TENSOR || want == XLSTM_PATH_TENSOR_TMEM) {
-        const bool ok = dt == XLSTM_BF16 && (want == XLSTM_PATH_TENSOR ? any_tensor_path(DH, chunk)
-                                                                       : tensor_path_supports(DH, chunk));
+    if (want == XLSTM_PATH_TENSOR || want == XLSTM_PATH_TENSOR_TMEM || want == XLSTM_PATH_TENSOR_RS) {
+        const bool ok = dt == XLSTM_BF16 && (want == XLSTM_PATH_TENSOR      ? any_tensor_path(DH, chunk)
+                                             : want == XLSTM_PATH_TENSOR_RS ? rs_path_supports(DH, chunk)
+                                                                            : tensor_path_supports(DH, chunk));
         if (!ok) {
             *st = XLSTM_ERR_UNSUPPORTED;
             return 0;
@@ -246,9 +253,13 @@ xlstm_status xlstm_mlstm_fwd_ex(const void *q, const void *k, const void *v,
     cudaError_t e;
     if (S == 0) {
         e = launch_state_passthrough(a, plan.BH, DH, stream);
-    } else if (path == XLSTM_PATH_TENSOR && rs_path_supports(DH, chunk)) {
+    } else if (path == XLSTM_PATH_TENSOR_RS ||
+               (path == XLSTM_PATH_TENSOR && !tensor_path_supports(DH, chunk))) {
+        // the register-state kernels: where the tensor-memory-state kernel does not
+        // apply (DH 64), or when asked for
         e = launch_fwd_rs(a, plan, stream);
     } else if (path == XLSTM_PATH_TENSOR || path == XLSTM_PATH_TENSOR_TMEM) {
+        // measured faster at DH 128 / 256 with chunk 64 (the long workload)
         e = launch_fwd_tensor(a, plan, stream);
     } else {
         e = launch_fwd_simt(a, plan, stream);

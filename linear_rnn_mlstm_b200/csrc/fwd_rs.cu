@@ -11,32 +11,35 @@
 // C' = Chi + Clo (15 to 16 significant bits), the A operand of the retrieval.
 // Per chunk c with queries Q, keys K, values V (bf16, staged by TMA):
 //
-//   S    = Q K^T                                    M=64,  N=64, K=DH
+//   S    = Q [K; n'hi; n'mid; n'lo]^T               M=64,  N=72, K=DH
 //   H^T  = (Chi + Clo) Q^T                          M=128, N=64, K=DH (A in TMEM)
 //   H^T += (w V)^T P^T,  P = rho * S masked s <= t  M=128, N=64, K=64
 //   U    = (w V)^T K                                M=128, N=DH, K=64
-//   C'  <- a C' + beta U                            (fp32, in the state warps)
+//   C'  <- a C' + U                                 (fp32, in the state warps)
 //
 // with u_s = itilde_s - b_s (b = within-chunk cumulative log f), Mc = max_s
-// u_s, m_prev the stabiliser before the chunk and
-//   w_s = e^{u_s - Mc} / sqrt(d),  rho = e^{Mc - m_prev},
-//   a = e^{m_prev - max(m_prev, Mc)},  beta = e^{Mc - max(m_prev, Mc)},
-//   g_t = e^{m_prev - max(m_prev, pmax_t)},  m_t = b_t + max(m_prev, pmax_t).
-// Then the exact intra-chunk weight e^{b_t - b_s + itilde_s - m_t} / sqrt(d)
+// u_s, m_prev the stabiliser before the chunk, M = max(m_prev, Mc) and
+//   w_s = e^{u_s - M} / sqrt(d),  rho = e^{M - m_prev},  a = e^{m_prev - M},
+//   g_t = e^{m_prev - max(m_prev, pmax_t)},  m_t = b_t + max(m_prev, pmax_t),
+// so the state after the chunk is exactly a C' + U (all exponents <= 0), and
+// the exact intra-chunk weight e^{b_t - b_s + itilde_s - m_t} / sqrt(d)
 // equals g_t rho w_s, so
 //   h_t = o_t * g_t H_t / max(|g_t (n'.q_t + rho sum_s w_s S_ts)|, e^{-m_t}),
-// where n'.q_t is formed in fp32 from the normaliser kept in shared memory.
+// where n'.q_t rides in the scores product: the normaliser n', as three bf16
+// parts (hi + mid + lo, about 24 significant bits), fills key rows 64-66 of
+// the key tile, so S has 72 columns.
 // A chunk is "wide" when Mc > m_prev + 40 (rho would leave the fp32 range):
 // then P carries exact per-row weights against V as loaded (rows whose own
 // stabiliser moved by more than e^40 have the old state's share below fp32
 // resolution; their retrieval term is dropped by zeroing those query rows),
 // and V is scaled by w only after the intra-chunk product has read it.
 //
-// Warp roles (16 warps): 0 TMA (q, k, v), 1 MMA issue and TMEM owner, 2 gates,
-// 3 TMA (output gates); 4-11 state (C' rows, the fold, the bf16 parts, w V,
-// the normaliser chain, and h from H); 12-15 scores (masked weighted scores,
-// n'.q and the denominators).  Every wait is bounded (tc_ptx.cuh): on a
-// timeout the kernel raises the device status word and unwinds.
+// Warp roles (16 warps): 0 TMA (q, k, v), 1 MMA issue and TMEM owner, 2 gates
+// and the normaliser chain n', 3 TMA (output gates); 4-11 state (C' rows, the
+// fold, the bf16 parts, w V, and h from H, stored straight to global memory);
+// 12-15 scores (masked weighted scores and the denominators).  Every wait is
+// bounded (tc_ptx.cuh): on a timeout the kernel raises the device status word
+// and unwinds.
 #include "common.cuh"
 #include "kernels.h"
 #include "profile.h"
@@ -54,37 +57,39 @@ constexpr float kWideGap = 40.f;   // ln of the largest factor rho may take
 
 template <int D>
 struct RsCfg {
-    static constexpr int KC = D;                       // key columns of the state in this CTA
+    static constexpr int KC = D > 256 ? 256 : D;       // key columns of the state in this CTA
+    static constexpr int KS = D / KC;                  // key splits (DH 512: two CTAs per value tile)
     static constexpr int RV = D < 128 ? D : 128;       // value rows (MMAs keep M = 128)
     static constexpr int VB = RV / 64;                 // 64-column blocks of the value tile
     static constexpr int KPT = KC / 2;                 // keys per state thread (two warps per lane quadrant)
-    static constexpr bool kSharedRU = 2 * KC + 64 + 128 > 512;
+    static constexpr bool kSharedRU = 2 * KC + 72 + 128 > 512;
     static constexpr uint32_t R0 = 0;                  // bf16 parts: hi [0, KC/2), lo [KC/2, KC)
     static constexpr uint32_t U0 = kSharedRU ? 0 : KC; // fp32 chunk update
     static constexpr uint32_t S0 = kSharedRU ? KC : 2 * KC;
-    static constexpr uint32_t H0 = S0 + 64;            // two 64-column buffers
+    static constexpr uint32_t H0 = S0 + 72;            // two 64-column buffers
     static_assert(H0 + 128 <= 512, "tensor memory");
+    static_assert(!kSharedRU || KC + 72 + 128 <= 512, "tensor memory");
     // shared memory (bytes; 1024-aligned operand tiles first)
-    static constexpr int kQbytes = (D / 64) * 8192;    // [64 tokens][D] bf16, 64-key blocks, 128 B swizzle
+    static constexpr int kQbytes = (KC / 64) * 8192;   // [64 tokens][KC] bf16, 64-key blocks, 128 B swizzle
+    static constexpr int kKBlock = 72 * 128;           // key block: 64 key rows + n' hi/mid/lo + 5 zero rows
+    static constexpr int kKbytes = (KC / 64) * kKBlock;
     static constexpr int kVbytes = 16384;              // [64 tokens][128 values] bf16, two blocks
-    static constexpr int kObytes = 64 * RV * 4;        // [64 tokens][RV] fp32 output-gate pre-activations
+    static constexpr int kObytes = KS == 1 ? 64 * RV * 4 : 0;   // [64 tokens][RV] fp32 output-gate pre-activations
     static constexpr int kQ = 0;
     static constexpr int kK = kQ + 2 * kQbytes;
-    static constexpr int kV = kK + 2 * kQbytes;
+    static constexpr int kV = kK + 2 * kKbytes;
     static constexpr int kO = kV + 2 * kVbytes;
     static constexpr int kP = kO + kObytes;            // [64][64] bf16 masked scores, 128 B swizzle
-    static constexpr int kHs = kP + 8192;              // h tile: VB blocks of [64 tokens][64 values] bf16
     static constexpr int kGB = 3;                      // gate buffers (ring)
-    static constexpr int kG = kHs + 16384;             // per-token gate arrays [kGB][kNG][64]
+    static constexpr int kG = kP + 8192;               // per-token gate arrays [kGB][kNG][64]
     static constexpr int kNG = 8;
     static constexpr int kGs = kG + kGB * kNG * 64 * 4;  // per-chunk gate scalars [kGB][8]
-    static constexpr int kNp = kGs + kGB * 8 * 4;      // normaliser n' [2][D] fp32
-    static constexpr int kBar = kNp + 2 * D * 4;
+    static constexpr int kBar = kGs + kGB * 8 * 4;
     static constexpr int kNumBars = 48;
     static constexpr int kMisc = kBar + kNumBars * 8;
     static constexpr int kBytes = kMisc + 64 + 1024;   // + slack for 1024-byte alignment
 };
-static_assert(RsCfg<256>::kBytes <= 232448, "shared memory");
+static_assert(RsCfg<256>::kBytes <= 232448 && RsCfg<512>::kBytes <= 232448, "shared memory");
 
 // per-token gate arrays
 enum { G_W = 0, G_G, G_FL, G_U, G_REF, G_OF, G_INV, G_LATE };
@@ -94,7 +99,7 @@ enum { GS_RHO = 0, GS_A, GS_BETA, GS_WIDE, GS_LC };
 enum {
     B_QF0 = 0, B_QF1, B_QE0, B_QE1, B_KF0, B_KF1, B_KE0, B_KE1, B_VF0, B_VF1, B_VE0, B_VE1,
     B_OF, B_OE, B_SF, B_SE, B_PR, B_PE, B_HF0, B_HF1, B_HE0, B_HE1, B_RR, B_RD, B_UF,
-    B_VH0, B_VH1, B_ID, B_GR0, B_GR1, B_GR2, B_GE0, B_GE1, B_GE2, B_NR0, B_NR1, B_NE0, B_NE1, B_DONE, B_NUM
+    B_VH0, B_VH1, B_ID, B_GR0, B_GR1, B_GR2, B_GE0, B_GE1, B_GE2, B_NR0, B_NR1, B_DONE, B_NUM
 };
 static_assert(B_NUM <= RsCfg<64>::kNumBars, "barrier slots");
 
@@ -113,6 +118,17 @@ constexpr int kRsTraceChunks = 64;
 #else
 #define RS_TRACE(cond, c, slot) do { } while (0)
 #endif
+
+// Waits of this kernel: hardware-suspending by default (a spinning poller
+// costs the co-scheduled warps issue slots); XLSTM_RS_SPIN_WAITS selects the
+// spinning variant for comparison.
+__device__ __forceinline__ bool rs_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag, unsigned int *status) {
+#ifdef XLSTM_RS_SPIN_WAITS
+    return mbar_wait(bar, parity, abort_flag, status);
+#else
+    return mbar_wait_sleep(bar, parity, abort_flag, status);
+#endif
+}
 
 __device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
     return p + ((1024u - (smem_u32(p) & 1023u)) & 1023u);
@@ -153,16 +169,17 @@ __device__ __forceinline__ void write_parts(const float (&Cs)[KPT], uint32_t t_r
 template <int D>
 __global__ void __launch_bounds__(kRsThreads, 1)
 segment_output_rs_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
-                         const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_h,
-                         const __grid_constant__ CUtensorMap map_o,
-                         const float *__restrict__ i_pre,
+                         const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_o,
+                         __nv_bfloat16 *__restrict__ h_out, const float *__restrict__ i_pre,
                          const float *__restrict__ C0, const float *__restrict__ n0, const float *__restrict__ m0,
                          float *__restrict__ C_out, float *__restrict__ n_out, float *__restrict__ m_out,
                          const float *__restrict__ bcum, const float *__restrict__ pmx,
                          const float2 *__restrict__ cstat, const float2 *__restrict__ sstat,
-                         const float *__restrict__ summ, unsigned int *status, int S, int nchunks, int P, int cps) {
+                         const float *__restrict__ summ, float *__restrict__ part, float *__restrict__ dpart,
+                         float2 *__restrict__ tokrec, unsigned int *status, int S, int nchunks, int P, int cps) {
     using Cfg = RsCfg<D>;
-    constexpr int KC = Cfg::KC, RV = Cfg::RV, VB = Cfg::VB, KPT = Cfg::KPT, GB = Cfg::kGB;
+    constexpr int KC = Cfg::KC, KS = Cfg::KS, RV = Cfg::RV, VB = Cfg::VB, KPT = Cfg::KPT, GB = Cfg::kGB;
+    constexpr int KB = Cfg::kKBlock;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = align1024(smem_raw);
     uint8_t *sQ = smem + Cfg::kQ;
@@ -170,18 +187,16 @@ segment_output_rs_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
     uint8_t *sV = smem + Cfg::kV;
     float *sO = reinterpret_cast<float *>(smem + Cfg::kO);
     uint8_t *sP = smem + Cfg::kP;
-    uint8_t *sHs = smem + Cfg::kHs;
     float *gA = reinterpret_cast<float *>(smem + Cfg::kG);      // [GB][kNG][64]
     float *gS = reinterpret_cast<float *>(smem + Cfg::kGs);     // [GB][8]
-    float *sNp = reinterpret_cast<float *>(smem + Cfg::kNp);    // [2][D]
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cfg::kBar);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + Cfg::kMisc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + Cfg::kMisc + 4);
     auto garr = [&](int gb, int which) { return gA + (gb * Cfg::kNG + which) * 64; };
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int tile = blockIdx.x, g = blockIdx.y, bh = blockIdx.z;
-    const int i0 = tile * RV;
+    const int tile = blockIdx.x / KS, kh = blockIdx.x % KS, g = blockIdx.y, bh = blockIdx.z;
+    const int i0 = tile * RV, k0 = kh * KC;        // value rows and key columns of this CTA
     const int c0 = g * cps;
     const int nch = max(0, min(nchunks, c0 + cps) - c0);
     const size_t tok0 = (size_t)bh * S;
@@ -191,8 +206,7 @@ segment_output_rs_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
 
     if (tid == 0) {
         for (int i = 0; i < B_NUM; ++i) {
-            const bool two = i == B_QE0 || i == B_QE1 || i == B_KE0 || i == B_KE1 || i == B_GE0 || i == B_GE1 ||
-                             i == B_GE2;
+            const bool two = i == B_KE0 || i == B_KE1 || i == B_GE0 || i == B_GE1 || i == B_GE2;
             mbar_init(&bars[i], two ? 2 : 1);
         }
         *abort_flag = 0;
@@ -203,20 +217,26 @@ segment_output_rs_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
         tmem_relinquish();
         tc_fence_before();
     }
-    if (VB == 1) {     // the unloaded second value block of both V slots stays zero
+    // rows 64-71 of every key block start at zero (TMA writes rows 0-63 only;
+    // the normaliser parts go to rows 64-66), and so does an unloaded value block
+    for (int e = tid; e < 2 * (KC / 64) * 64; e += kRsThreads) {     // (slot, block, row 64-71, chunk)
+        const int ch = e & 7, row = 64 + ((e >> 3) & 7), blk = (e >> 6) % (KC / 64), sl = e / (64 * (KC / 64));
+        *reinterpret_cast<uint4 *>(sK + sl * Cfg::kKbytes + blk * KB + sw128_offset(row, ch)) = make_uint4(0u, 0u, 0u, 0u);
+    }
+    if (VB == 1) {
         for (int e = tid; e < 2 * 512; e += kRsThreads)
             *reinterpret_cast<uint4 *>(sV + (e >> 9) * Cfg::kVbytes + 8192 + (e & 511) * 16) = make_uint4(0u, 0u, 0u, 0u);
-        fence_async_smem();
     }
+    fence_async_smem();
     __syncthreads();
     tc_fence_after();
     const uint32_t tbase = *tmem_slot;
     const uint32_t tR = tbase + Cfg::R0, tU = tbase + Cfg::U0, tS = tbase + Cfg::S0, tH = tbase + Cfg::H0;
 
-    // Register budget per warpgroup (D = 256: the state warps hold 128 floats of
+    // Register budget per warpgroup (KC = 256: the state warps hold 128 floats of
     // C' per thread): 128 x 48 + 256 x 176 + 128 x 104 = 64512 <= 512 x 128.
     if (warp < 4) {
-        if (D == 256) regs_dec<48>();
+        if (KC == 256) regs_dec<48>();
         if (warp == 0) {
             // -------------------------------------------------------- TMA: q, k, v
             if (lane == 0 && nch > 0) {
@@ -228,23 +248,23 @@ segment_output_rs_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
                     const int t0 = (c0 + c) * kL, sl = c & 1;
                     const uint32_t par = ((c >> 1) - 1) & 1;
                     if (c + 2 < nch) {
-                        for (int jb = 0; jb < D / 64; ++jb) {
-                            tma_prefetch_l2_3d(&map_q, jb * 64, t0 + 2 * kL, bh);
-                            tma_prefetch_l2_3d(&map_k, jb * 64, t0 + 2 * kL, bh);
+                        for (int jb = 0; jb < KC / 64; ++jb) {
+                            tma_prefetch_l2_3d(&map_q, k0 + jb * 64, t0 + 2 * kL, bh);
+                            tma_prefetch_l2_3d(&map_k, k0 + jb * 64, t0 + 2 * kL, bh);
                         }
                         for (int b = 0; b < VB; ++b) tma_prefetch_l2_3d(&map_v, i0 + 64 * b, t0 + 2 * kL, bh);
                     }
-                    if (c >= 2 && !mbar_wait(&bars[B_QE0 + sl], par, abort_flag, status)) break;
-                    mbar_arrive_expect_tx(&bars[B_QF0 + sl], kL * D * 2);
-                    for (int jb = 0; jb < D / 64; ++jb)
-                        tma_load_3d(sQ + sl * Cfg::kQbytes + jb * 8192, &map_q, &bars[B_QF0 + sl], jb * 64, t0, bh);
+                    if (c >= 2 && !rs_wait(&bars[B_QE0 + sl], par, abort_flag, status)) break;
+                    mbar_arrive_expect_tx(&bars[B_QF0 + sl], kL * KC * 2);
+                    for (int jb = 0; jb < KC / 64; ++jb)
+                        tma_load_3d(sQ + sl * Cfg::kQbytes + jb * 8192, &map_q, &bars[B_QF0 + sl], k0 + jb * 64, t0, bh);
                     ++issued[0][sl];
-                    if (c >= 2 && !mbar_wait(&bars[B_KE0 + sl], par, abort_flag, status)) break;
-                    mbar_arrive_expect_tx(&bars[B_KF0 + sl], kL * D * 2);
-                    for (int jb = 0; jb < D / 64; ++jb)
-                        tma_load_3d(sK + sl * Cfg::kQbytes + jb * 8192, &map_k, &bars[B_KF0 + sl], jb * 64, t0, bh);
+                    if (c >= 2 && !rs_wait(&bars[B_KE0 + sl], par, abort_flag, status)) break;
+                    mbar_arrive_expect_tx(&bars[B_KF0 + sl], kL * KC * 2);
+                    for (int jb = 0; jb < KC / 64; ++jb)
+                        tma_load_3d(sK + sl * Cfg::kKbytes + jb * KB, &map_k, &bars[B_KF0 + sl], k0 + jb * 64, t0, bh);
                     ++issued[1][sl];
-                    if (c >= 2 && !mbar_wait(&bars[B_VE0 + sl], par, abort_flag, status)) break;
+                    if (c >= 2 && !rs_wait(&bars[B_VE0 + sl], par, abort_flag, status)) break;
                     mbar_arrive_expect_tx(&bars[B_VF0 + sl], kL * VB * 64 * 2);
                     for (int b = 0; b < VB; ++b)
                         tma_load_3d(sV + sl * Cfg::kVbytes + b * 8192, &map_v, &bars[B_VF0 + sl], i0 + 64 * b, t0, bh);
@@ -259,13 +279,13 @@ segment_output_rs_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
             }
         } else if (warp == 3) {
             // -------------------------------------------------- TMA: output gates
-            if (lane == 0 && nch > 0) {
+            if (KS == 1 && lane == 0 && nch > 0) {
                 tma_prefetch_desc(&map_o);
                 int issued = 0;
                 for (int c = 0; c < nch; ++c) {
                     const int t0 = (c0 + c) * kL;
                     if (c + 1 < nch) tma_prefetch_l2_3d(&map_o, i0, t0 + kL, bh);
-                    if (c >= 1 && !mbar_wait(&bars[B_OE], (c - 1) & 1, abort_flag, status)) break;
+                    if (c >= 1 && !rs_wait(&bars[B_OE], (c - 1) & 1, abort_flag, status)) break;
                     mbar_arrive_expect_tx(&bars[B_OF], kL * RV * 4);
                     tma_load_3d(sO, &map_o, &bars[B_OF], i0, t0, bh);
                     ++issued;
@@ -273,9 +293,10 @@ segment_output_rs_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
                 if (issued) mbar_wait(&bars[B_OF], (issued - 1) & 1, nullptr, status);
             }
         } else if (warp == 2) {
-            // ---------------------------------------------------------- gates
-            // Stabiliser entering this segment: the initial m, folded through the
-            // statistics (total log f, own stabiliser) of the segments before it.
+            // ------------------------------------------- gates and normaliser chain
+            // Gates run two chunks ahead of the normaliser.  Stabiliser entering
+            // this segment: the initial m, folded through the statistics (total
+            // log f, own stabiliser) of the segments before it.
             float mc = m0 ? m0[bh] : 0.f;
             for (int gp = 0; gp < g; ++gp) {
                 const float2 st = sstat[(size_t)bh * P + gp];
@@ -293,11 +314,9 @@ segment_output_rs_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
                     pi_[h2] = ok ? i_pre[tok0 + t] : 0.f;
                 }
             };
-            if (nch > 0) fetch(0);
-            bool ok = true;
-            for (int c = 0; c < nch; ++c) {
+            auto gates = [&](int c) -> bool {
                 const int gb = c % GB, t0 = (c0 + c) * kL, Lc = min(kL, S - t0);
-                if (c >= GB && !mbar_wait(&bars[B_GE0 + gb], ((c / GB) - 1) & 1, abort_flag, status)) { ok = false; break; }
+                if (c >= GB && !rs_wait(&bars[B_GE0 + gb], ((c / GB) - 1) & 1, abort_flag, status)) return false;
                 const float2 cs = cstat[(size_t)bh * nchunks + c0 + c];   // (sum of log f, max of u)
                 const float Mc = cs.y;
                 const bool wide = Mc > mc + kWideGap;
@@ -313,7 +332,7 @@ segment_output_rs_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
                     const float run = fmaxf(mc, pm);
                     const bool late = wide && pm > mc + kWideGap;
                     const float gt = valid ? expf(mc - run) : 0.f;
-                    garr(gb, G_W)[t] = valid ? expf(u - Mc) * inv_sqrt_d : 0.f;
+                    garr(gb, G_W)[t] = valid ? expf(u - big) * inv_sqrt_d : 0.f;
                     garr(gb, G_G)[t] = gt;
                     garr(gb, G_FL)[t] = valid ? expf(-(b_[h2] + run)) : 1.f;
                     garr(gb, G_U)[t] = valid ? u : -INFINITY;
@@ -323,7 +342,7 @@ segment_output_rs_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
                 }
                 if (lane == 0) {
                     float *gs = gS + gb * 8;
-                    gs[GS_RHO] = wide ? 0.f : expf(Mc - mc);
+                    gs[GS_RHO] = wide ? 0.f : expf(big - mc);
                     gs[GS_A] = expf(mc - big);
                     gs[GS_BETA] = expf(Mc - big);
                     gs[GS_WIDE] = wide ? 1.f : 0.f;
@@ -333,29 +352,122 @@ segment_output_rs_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
                 __syncwarp();
                 RS_TRACE(lane == 0, c, 24);
                 if (lane == 0) mbar_arrive(&bars[B_GR0 + gb]);
+                return true;
+            };
+            // normaliser n': lane holds keys [KPL lane, KPL lane + KPL)
+            constexpr int KPL = KC / 32;
+            float nr[KPL];
+            const float *nsrc = g == 0 ? (n0 ? n0 + (size_t)bh * D : nullptr)
+                                       : summ + ((size_t)bh * (P - 1) + g - 1) * ((size_t)D * D + D) + (size_t)D * D;
+#pragma unroll
+            for (int e = 0; e < KPL; ++e) nr[e] = nsrc ? nsrc[k0 + KPL * lane + e] : 0.f;
+            const int kblk = (KPL * lane) / 64;                     // key block of this lane's keys
+            const int kbyte = (KPL * lane * 2) % 128;               // byte offset within a 128-byte row
+            // n' as bf16 hi / mid / lo parts into rows 64-66 of key slot sl
+            auto write_nparts = [&](int sl) {
+                uint8_t *blk = sK + sl * Cfg::kKbytes + kblk * KB;
+                uint32_t ph[KPL / 2], pmid[KPL / 2], plo[KPL / 2];
+#pragma unroll
+                for (int e = 0; e < KPL / 2; ++e) {
+                    const float x0 = nr[2 * e], x1 = nr[2 * e + 1];
+                    const uint32_t h2 = cvt_bf16x2(x0, x1);
+                    const float r0 = x0 - bf_lo(h2), r1 = x1 - bf_hi(h2);
+                    const uint32_t m2 = cvt_bf16x2(r0, r1);
+                    ph[e] = h2;
+                    pmid[e] = m2;
+                    plo[e] = cvt_bf16x2(r0 - bf_lo(m2), r1 - bf_hi(m2));
+                }
+#pragma unroll
+                for (int e = 0; e < KPL / 2; ++e) {
+                    const int byte = kbyte + 4 * e;
+                    const int cc = byte >> 4, within = byte & 15;
+                    *reinterpret_cast<uint32_t *>(blk + sw128_offset(64, cc) + within) = ph[e];
+                    *reinterpret_cast<uint32_t *>(blk + sw128_offset(65, cc) + within) = pmid[e];
+                    *reinterpret_cast<uint32_t *>(blk + sw128_offset(66, cc) + within) = plo[e];
+                }
+                fence_async_smem();
+                __syncwarp();
+            };
+            bool ok = true;
+            if (nch > 0) {
+                fetch(0);
+                ok = gates(0) && (nch < 2 || gates(1));
+                if (ok) {
+                    write_nparts(0);
+                    if (lane == 0) mbar_arrive(&bars[B_NR0]);
+                }
             }
-            if (ok && g == P - 1 && tile == 0 && lane == 0 && m_out && nch > 0 && !*abort_flag) m_out[bh] = mc;
+            for (int c = 0; ok && c < nch; ++c) {
+                const int sl = c & 1, gb = c % GB;
+                // n'(c+1) = a n'(c) + sum_s w_s k_s over this chunk's keys, fp32
+                if (!rs_wait(&bars[B_KF0 + sl], (c >> 1) & 1, abort_flag, status)) { ok = false; break; }
+                const float *w = garr(gb, G_W);
+                const float a = gS[gb * 8 + GS_A];
+                const uint8_t *kt = sK + sl * Cfg::kKbytes + kblk * KB;
+                float acc[KPL];
+#pragma unroll
+                for (int e = 0; e < KPL; ++e) acc[e] = 0.f;
+#pragma unroll 4
+                for (int s = 0; s < kL; ++s) {
+                    const float ws = w[s];
+                    const uint8_t *rp = kt + sw128_offset(s, kbyte >> 4) + (kbyte & 15);
+                    if (KPL == 8) {
+                        const uint4 kv = *reinterpret_cast<const uint4 *>(rp);
+                        acc[0] += ws * bf_lo(kv.x); acc[1] += ws * bf_hi(kv.x);
+                        acc[2] += ws * bf_lo(kv.y); acc[3] += ws * bf_hi(kv.y);
+                        acc[4] += ws * bf_lo(kv.z); acc[5] += ws * bf_hi(kv.z);
+                        acc[6 % KPL] += ws * bf_lo(kv.w); acc[7 % KPL] += ws * bf_hi(kv.w);
+                    } else if (KPL == 4) {
+                        const uint2 kv = *reinterpret_cast<const uint2 *>(rp);
+                        acc[0] += ws * bf_lo(kv.x); acc[1] += ws * bf_hi(kv.x);
+                        acc[2 % KPL] += ws * bf_lo(kv.y); acc[3 % KPL] += ws * bf_hi(kv.y);
+                    } else {
+                        const uint32_t kv = *reinterpret_cast<const uint32_t *>(rp);
+                        acc[0] += ws * bf_lo(kv); acc[1 % KPL] += ws * bf_hi(kv);
+                    }
+                }
+#pragma unroll
+                for (int e = 0; e < KPL; ++e) nr[e] = fmaf(a, nr[e], acc[e]);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars[B_KE0 + sl]);
+                if (c + 1 < nch) {
+                    // scores(c - 1) read this slot's normaliser rows; the update of chunk
+                    // c - 1 completing implies they are done
+                    if (c >= 1 && !rs_wait(&bars[B_UF], (c - 1) & 1, abort_flag, status)) { ok = false; break; }
+                    write_nparts((c + 1) & 1);
+                    if (lane == 0) mbar_arrive(&bars[B_NR0 + ((c + 1) & 1)]);
+                }
+                if (c + 2 < nch && !gates(c + 2)) { ok = false; break; }
+            }
+            if (ok && g == P - 1 && tile == 0 && nch > 0 && !*abort_flag) {
+                if (lane == 0 && kh == 0 && m_out) m_out[bh] = mc;
+                if (n_out) {
+#pragma unroll
+                    for (int e = 0; e < KPL; ++e) n_out[(size_t)bh * D + k0 + KPL * lane + e] = nr[e];
+                }
+            }
         } else {
             // ------------------------------------------------------- MMA issue
             if (lane == 0 && nch > 0) {
-                const uint32_t idesc_S = idesc_f32acc(kFmtBF16, kFmtBF16, false, false, 64, 64);
+                const uint32_t idesc_S = idesc_f32acc(kFmtBF16, kFmtBF16, false, false, 64, 72);
                 const uint32_t idesc_R = idesc_f32acc(kFmtBF16, kFmtBF16, false, false, 128, 64);
                 const uint32_t idesc_I = idesc_f32acc(kFmtBF16, kFmtBF16, true, false, 128, 64);
                 const uint32_t idesc_U = idesc_f32acc(kFmtBF16, kFmtBF16, true, true, 128, KC);
                 auto issue_scores = [&](int c) {
                     const int sl = c & 1;
                     uint64_t dq = sdesc_sw128(smem_u32(sQ + sl * Cfg::kQbytes), 16, 1024);
-                    uint64_t dk = sdesc_sw128(smem_u32(sK + sl * Cfg::kQbytes), 16, 1024);
+                    uint64_t dk = sdesc_sw128(smem_u32(sK + sl * Cfg::kKbytes), 16, 1024);
 #pragma unroll 1
-                    for (int jb = 0; jb < D / 64; ++jb) {
+                    for (int jb = 0; jb < KC / 64; ++jb) {
 #pragma unroll
                         for (int k4 = 0; k4 < 4; ++k4) mma_bf16_ss(tS, dq + 2 * k4, dk + 2 * k4, idesc_S, (jb | k4) != 0);
                         dq += 8192 >> 4;
-                        dk += 8192 >> 4;
+                        dk += KB >> 4;
                     }
                     mma_commit(&bars[B_SF]);
                 };
-                bool ok = mbar_wait(&bars[B_QF0], 0, abort_flag, status) && mbar_wait(&bars[B_KF0], 0, abort_flag, status);
+                bool ok = rs_wait(&bars[B_QF0], 0, abort_flag, status) && rs_wait(&bars[B_KF0], 0, abort_flag, status) &&
+                          rs_wait(&bars[B_NR0], 0, abort_flag, status);
                 if (ok) {
                     tc_fence_after();
                     issue_scores(0);
@@ -365,15 +477,15 @@ segment_output_rs_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
                     const uint32_t par = (c >> 1) & 1;
                     const uint32_t tHb = tH + 64 * hb;
                     RS_TRACE(true, c, 0);
-                    if (!mbar_wait(&bars[B_RR], c & 1, abort_flag, status) ||
-                        !mbar_wait(&bars[B_GR0 + gb], (c / GB) & 1, abort_flag, status) ||
-                        (c >= 2 && !mbar_wait(&bars[B_HE0 + hb], ((c >> 1) - 1) & 1, abort_flag, status))) { ok = false; break; }
+                    if (!rs_wait(&bars[B_RR], c & 1, abort_flag, status) ||
+                        !rs_wait(&bars[B_GR0 + gb], (c / GB) & 1, abort_flag, status) ||
+                        (c >= 2 && !rs_wait(&bars[B_HE0 + hb], ((c >> 1) - 1) & 1, abort_flag, status))) { ok = false; break; }
                     tc_fence_after();
                     const bool wide = gS[gb * 8 + GS_WIDE] != 0.f;
                     {   // retrieval: H^T = (Chi + Clo) Q^T, the parts of C' from TMEM
                         uint64_t dq = sdesc_sw128(smem_u32(sQ + sl * Cfg::kQbytes), 16, 1024);
 #pragma unroll 1
-                        for (int jb = 0; jb < D / 64; ++jb) {
+                        for (int jb = 0; jb < KC / 64; ++jb) {
 #pragma unroll
                             for (int k4 = 0; k4 < 4; ++k4) {
                                 const uint32_t col = (uint32_t)(jb * 32 + 8 * k4);
@@ -387,9 +499,9 @@ segment_output_rs_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
                     }
                     RS_TRACE(true, c, 1);
                     // intra-chunk term: H^T += (w V)^T P^T (wide chunks: V as loaded)
-                    if ((!wide && !mbar_wait(&bars[B_VH0 + sl], par, abort_flag, status)) ||
-                        !mbar_wait(&bars[B_VF0 + sl], par, abort_flag, status) ||
-                        !mbar_wait(&bars[B_PR], c & 1, abort_flag, status)) { ok = false; break; }
+                    if ((!wide && !rs_wait(&bars[B_VH0 + sl], par, abort_flag, status)) ||
+                        !rs_wait(&bars[B_VF0 + sl], par, abort_flag, status) ||
+                        !rs_wait(&bars[B_PR], c & 1, abort_flag, status)) { ok = false; break; }
                     tc_fence_after();
                     {
                         const uint32_t va = smem_u32(sV + sl * Cfg::kVbytes), pa = smem_u32(sP);
@@ -406,22 +518,23 @@ segment_output_rs_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
                     if (c + 1 < nch) {
                         const int ns = (c + 1) & 1;
                         const uint32_t npar = ((c + 1) >> 1) & 1;
-                        if (!mbar_wait(&bars[B_QF0 + ns], npar, abort_flag, status) ||
-                            !mbar_wait(&bars[B_KF0 + ns], npar, abort_flag, status) ||
-                            !mbar_wait(&bars[B_SE], c & 1, abort_flag, status)) { ok = false; break; }
+                        if (!rs_wait(&bars[B_QF0 + ns], npar, abort_flag, status) ||
+                            !rs_wait(&bars[B_KF0 + ns], npar, abort_flag, status) ||
+                            !rs_wait(&bars[B_NR0 + ns], npar, abort_flag, status) ||
+                            !rs_wait(&bars[B_SE], c & 1, abort_flag, status)) { ok = false; break; }
                         tc_fence_after();
                         issue_scores(c + 1);
                         RS_TRACE(true, c, 3);
                     }
                     // update of the state: U = (w V)^T K, after the retrieval has read the parts
-                    if ((Cfg::kSharedRU && !mbar_wait(&bars[B_RD], c & 1, abort_flag, status)) ||
-                        (wide && !mbar_wait(&bars[B_VH0 + sl], par, abort_flag, status))) { ok = false; break; }
+                    if ((Cfg::kSharedRU && !rs_wait(&bars[B_RD], c & 1, abort_flag, status)) ||
+                        (wide && !rs_wait(&bars[B_VH0 + sl], par, abort_flag, status))) { ok = false; break; }
                     tc_fence_after();
                     {
-                        const uint32_t va = smem_u32(sV + sl * Cfg::kVbytes), ka = smem_u32(sK + sl * Cfg::kQbytes);
+                        const uint32_t va = smem_u32(sV + sl * Cfg::kVbytes), ka = smem_u32(sK + sl * Cfg::kKbytes);
 #pragma unroll
                         for (int ks = 0; ks < 4; ++ks)
-                            mma_bf16_ss(tU, sdesc_sw128(va + ks * 2048, 8192, 1024), sdesc_sw128(ka + ks * 2048, 8192, 1024),
+                            mma_bf16_ss(tU, sdesc_sw128(va + ks * 2048, 8192, 1024), sdesc_sw128(ka + ks * 2048, KB, 1024),
                                         idesc_U, ks > 0 ? 1u : 0u);
                         mma_commit(&bars[B_UF]);
                         mma_commit(&bars[B_VE0 + sl]);
@@ -434,21 +547,18 @@ segment_output_rs_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
             }
         }
     } else if (warp < 12) {
-        if (D == 256) regs_inc<176>();
+        if (KC == 256) regs_inc<176>();
         // ------------------------------------------------------------ state group
         const int sw = warp - 4;                 // 0..7
         const int half = sw >> 2;                // key half (fold) and token half (outputs) of this thread
         const int i = 32 * q4 + lane;            // value row within the tile
         const bool has_row = i < RV;
         const int kbase = half * KPT;            // first key column of this thread
-        const int j = sw * 32 + lane;            // normaliser entry of this thread (j < D)
-        const bool has_j = j < D;
         const bool leader = sw == 0 && lane == 0;
         float Cs[KPT];
-        float nreg = 0.f;
         bool ok = true;
         auto swait = [&](uint64_t *bar, uint32_t parity) -> bool {
-            const bool r = leader ? mbar_wait(bar, parity, abort_flag, status) : true;
+            const bool r = leader ? rs_wait(bar, parity, abort_flag, status) : true;
             return group_all<1, 256>(r);
         };
         // V of chunk c scaled in place by w (the operand of the intra and update products)
@@ -476,48 +586,50 @@ segment_output_rs_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
         auto zero_late_rows = [&](int c, int gb) {
             const float *lt = garr(gb, G_LATE);
             uint8_t *qt = sQ + (c & 1) * Cfg::kQbytes;
-            for (int e = sw * 32 + lane; e < (D / 64) * kL * 8; e += 256) {
+            for (int e = sw * 32 + lane; e < (KC / 64) * kL * 8; e += 256) {
                 const int blk = e / (kL * 8), t = (e / 8) % kL, ch = e & 7;
                 if (lt[t] != 0.f)
                     *reinterpret_cast<uint4 *>(qt + blk * 8192 + sw128_offset(t, ch)) = make_uint4(0u, 0u, 0u, 0u);
             }
             fence_async_smem();
         };
-        // h of chunk c from H (this thread: value row i, tokens 32 half ... + 31),
-        // then the tile leaves by TMA store
+        // h of chunk c from H: this thread takes value row i, tokens 32 half ... + 31,
+        // and stores straight to global memory (a warp writes 64 contiguous bytes per token)
         auto out_pass = [&](int c, int gb) -> bool {
             const int hb = c & 1;
-            if (!swait(&bars[B_HF0 + hb], (c >> 1) & 1) || !swait(&bars[B_OF], c & 1)) return false;
+            if (!swait(&bars[B_HF0 + hb], (c >> 1) & 1) || (KS == 1 && !swait(&bars[B_OF], c & 1))) return false;
             RS_TRACE(leader, c, 20);
-            if (leader) bulk_wait_read_all();       // the previous h tile has left shared memory
-            sync_state();
             tc_fence_after();
             const float *inv = garr(gb, G_INV);
-            uint8_t *hs = sHs + (i >> 6) * 8192 + (i & 63) * 2;
+            const int t0 = (c0 + c) * kL;
+            __nv_bfloat16 *hrow = h_out + (tok0 + t0) * D + i0 + i;
+            float *prow = part + (((size_t)kh * gridDim.z + bh) * S + t0) * D + i0 + i;
 #pragma unroll 1
             for (int pc = 0; pc < 2; ++pc) {
                 const int tb = 32 * half + 16 * pc;
                 uint32_t r[16];
                 tmem_ld16(tH + 64 * hb + lane_addr + tb, r);
                 tmem_wait_ld();
-                if (has_row) {
+                if (KS > 1) {          // this CTA's share of the numerator, combined later
+                    const int lim = min(16, S - t0 - tb);
+#pragma unroll
+                    for (int kk = 0; kk < 16; ++kk)
+                        if (lim >= 16 || kk < lim) prow[(size_t)(tb + kk) * D] = __uint_as_float(r[kk]);
+                } else if (has_row) {
+                    const int lim = min(16, S - t0 - tb);            // tokens of this piece inside the sequence
 #pragma unroll
                     for (int kk = 0; kk < 16; ++kk) {
                         const int tt = tb + kk;
                         const float hv = __uint_as_float(r[kk]) * inv[tt];
                         const float o = sO[tt * RV + i];
-                        *reinterpret_cast<__nv_bfloat16 *>(hs + tt * 128) =
-                            __float2bfloat16_rn(fmaf(hv, tanh_approx(0.5f * o), hv));
+                        const __nv_bfloat16 hb16 = __float2bfloat16_rn(fmaf(hv, tanh_approx(0.5f * o), hv));
+                        if (lim >= 16 || kk < lim) hrow[(size_t)tt * D] = hb16;
                     }
                 }
             }
-            fence_async_smem();
             tc_fence_before();
             sync_state();
             if (leader) {
-                const int t0 = (c0 + c) * kL;
-                for (int b = 0; b < VB; ++b) tma_store_3d(&map_h, sHs + b * 8192, i0 + 64 * b, t0, bh);
-                bulk_commit();
                 mbar_arrive(&bars[B_HE0 + hb]);
                 mbar_arrive(&bars[B_OE]);
             }
@@ -530,7 +642,7 @@ segment_output_rs_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
             const float *src = g == 0 ? (C0 ? C0 + (size_t)bh * D * D : nullptr)
                                       : summ + ((size_t)bh * (P - 1) + g - 1) * ((size_t)D * D + D);
             if (src && has_row) {
-                const float4 *row = reinterpret_cast<const float4 *>(src + (size_t)(i0 + i) * D + kbase);
+                const float4 *row = reinterpret_cast<const float4 *>(src + (size_t)(i0 + i) * D + k0 + kbase);
 #pragma unroll
                 for (int e = 0; e < KPT / 4; ++e) {
                     const float4 x = row[e];
@@ -540,10 +652,6 @@ segment_output_rs_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
 #pragma unroll
                 for (int e = 0; e < KPT; ++e) Cs[e] = 0.f;
             }
-            const float *nsrc = g == 0 ? (n0 ? n0 + (size_t)bh * D : nullptr)
-                                       : summ + ((size_t)bh * (P - 1) + g - 1) * ((size_t)D * D + D) + (size_t)D * D;
-            nreg = (nsrc && has_j) ? nsrc[j] : 0.f;
-            if (has_j) sNp[j] = nreg;
         }
         if (nch > 0) {
             ok = swait(&bars[B_GR0], 0);
@@ -556,10 +664,7 @@ segment_output_rs_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
                 write_parts<KPT, KC>(Cs, tR + lane_addr, kbase);
                 tc_fence_before();
                 sync_state();
-                if (leader) {
-                    mbar_arrive(&bars[B_NR0]);
-                    mbar_arrive(&bars[B_RR]);
-                }
+                if (leader) mbar_arrive(&bars[B_RR]);
                 if (!wide0) {
                     ok = swait(&bars[B_VF0], 0);
                     if (ok) scale_v(0, 0);
@@ -568,9 +673,8 @@ segment_output_rs_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
         }
         int nwide = 0;
         for (int c = 0; ok && c < nch; ++c) {
-            const int sl = c & 1, gb = c % GB;
-            const uint32_t par = (c >> 1) & 1;
-            const float a = gS[gb * 8 + GS_A], beta = gS[gb * 8 + GS_BETA];
+            const int gb = c % GB;
+            const float a = gS[gb * 8 + GS_A];
             const bool wide = gS[gb * 8 + GS_WIDE] != 0.f;
             // (1) wide chunk: scale V after the intra-chunk product has read it
             if (wide) {
@@ -578,31 +682,8 @@ segment_output_rs_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
                 ++nwide;
                 scale_v(c, gb);
             }
-            // (2) normaliser chain n'(c+1) = a n'(c) + beta sum_s w_s k_s, in fp32
+            // (2) fold the chunk's update into the fp32 state, then the next chunk's parts
             RS_TRACE(leader, c, 8);
-            if (!swait(&bars[B_KF0 + sl], par)) { ok = false; break; }
-            {
-                const float *w = garr(gb, G_W);
-                const uint8_t *kt = sK + sl * Cfg::kQbytes + (j / 64) * 8192;
-                const int cc = (j % 64) / 8, within = (j % 8) * 2;
-                float acc = 0.f;
-                if (has_j) {
-#pragma unroll 8
-                    for (int s = 0; s < kL; ++s)
-                        acc += w[s] * __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(kt + sw128_offset(s, cc) + within));
-                }
-                nreg = a * nreg + beta * acc;
-            }
-            sync_state();
-            if (leader) mbar_arrive(&bars[B_KE0 + sl]);
-            if (c + 1 < nch) {
-                const int nb = (c + 1) & 1;
-                if (c + 1 >= 2 && !swait(&bars[B_NE0 + nb], (((c + 1) >> 1) - 1) & 1)) { ok = false; break; }
-                if (has_j) sNp[nb * D + j] = nreg;
-                sync_state();
-                if (leader) mbar_arrive(&bars[B_NR0 + nb]);
-            }
-            // (3) fold the chunk's update into the fp32 state, then the next chunk's parts
             if (!swait(&bars[B_UF], c & 1)) { ok = false; break; }
             RS_TRACE(leader, c, 10);
             tc_fence_after();
@@ -612,7 +693,7 @@ segment_output_rs_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
                 tmem_ld16(tU + lane_addr + kbase + 16 * pc, r);
                 tmem_wait_ld();
 #pragma unroll
-                for (int e = 0; e < 16; ++e) Cs[16 * pc + e] = fmaf(a, Cs[16 * pc + e], beta * __uint_as_float(r[e]));
+                for (int e = 0; e < 16; ++e) Cs[16 * pc + e] = fmaf(a, Cs[16 * pc + e], __uint_as_float(r[e]));
             }
             tc_fence_before();
             sync_state();                         // every read of U precedes the parts' writes
@@ -635,25 +716,21 @@ segment_output_rs_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
                     RS_TRACE(leader, c, 13);
                 }
             }
-            // (4) h of this chunk
+            // (3) h of this chunk
             if (!out_pass(c, gb)) { ok = false; break; }
             sync_state();
             if (leader) mbar_arrive(&bars[B_GE0 + gb]);
         }
         // final state (last segment only)
-        if (ok && g == P - 1 && nch > 0 && !*abort_flag) {
-            if (C_out && has_row) {
-                float4 *dst = reinterpret_cast<float4 *>(C_out + ((size_t)bh * D + i0 + i) * D + kbase);
+        if (ok && g == P - 1 && nch > 0 && !*abort_flag && C_out && has_row) {
+            float4 *dst = reinterpret_cast<float4 *>(C_out + ((size_t)bh * D + i0 + i) * D + k0 + kbase);
 #pragma unroll
-                for (int e = 0; e < KPT / 4; ++e)
-                    dst[e] = make_float4(Cs[4 * e], Cs[4 * e + 1], Cs[4 * e + 2], Cs[4 * e + 3]);
-            }
-            if (n_out && tile == 0 && has_j) n_out[(size_t)bh * D + j] = nreg;
+            for (int e = 0; e < KPT / 4; ++e)
+                dst[e] = make_float4(Cs[4 * e], Cs[4 * e + 1], Cs[4 * e + 2], Cs[4 * e + 3]);
         }
-        if (leader) bulk_wait_all();             // h is in global memory before exit
         tc_fence_before();
     } else {
-        if (D == 256) regs_dec<104>();
+        if (KC == 256) regs_dec<104>();
         // ------------------------------------------------------------ scores
         const int xt = tid - 384;                    // 0..127
         const bool xleader = xt == 0;
@@ -661,22 +738,21 @@ segment_output_rs_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
         const int hh = lane >> 4;                    // column half of this lane
         bool ok = true;
         auto xwait = [&](uint64_t *bar, uint32_t parity) -> bool {
-            const bool r = xleader ? mbar_wait(bar, parity, abort_flag, status) : true;
+            const bool r = xleader ? rs_wait(bar, parity, abort_flag, status) : true;
             return group_all<2, 128>(r);
         };
         for (int c = 0; ok && c < nch; ++c) {
-            const int sl = c & 1, gb = c % GB;
-            const uint32_t par = (c >> 1) & 1;
+            const int gb = c % GB;
             if (!xwait(&bars[B_SF], c & 1) || !xwait(&bars[B_GR0 + gb], (c / GB) & 1) ||
-                !xwait(&bars[B_NR0 + sl], par) || !xwait(&bars[B_QF0 + sl], par) ||
                 (c >= 1 && !xwait(&bars[B_PE], (c - 1) & 1))) { ok = false; break; }
             RS_TRACE(xleader, c, 16);
             tc_fence_after();
-            uint32_t sa[32], sb[32];
+            uint32_t sa[32], sb[32], sn[8];
             tmem_ld16(tS + lane_addr + 0, *reinterpret_cast<uint32_t(*)[16]>(&sa[0]));
             tmem_ld16(tS + lane_addr + 16, *reinterpret_cast<uint32_t(*)[16]>(&sa[16]));
             tmem_ld16(tS + lane_addr + 32, *reinterpret_cast<uint32_t(*)[16]>(&sb[0]));
             tmem_ld16(tS + lane_addr + 48, *reinterpret_cast<uint32_t(*)[16]>(&sb[16]));
+            tmem_ld8(tS + lane_addr + 64, sn);
             tmem_wait_ld();
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
@@ -689,20 +765,8 @@ segment_output_rs_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
             const bool valid = t < Lc;
             const float ref_t = garr(gb, G_REF)[t];
             const bool late = garr(gb, G_LATE)[t] != 0.f;
-            // n'.q_t over this lane's half of the keys, fp32 (late rows: not needed)
-            float nq = 0.f;
-            if (!late) {
-                const uint8_t *qrow = sQ + sl * Cfg::kQbytes;
-                const float *np = sNp + sl * D;
-#pragma unroll 2
-                for (int ch = hh * (D / 16); ch < (hh + 1) * (D / 16); ++ch) {   // 16-byte chunks of 8 keys
-                    const uint4 qv = *reinterpret_cast<const uint4 *>(qrow + (ch >> 3) * 8192 + sw128_offset(t, ch & 7));
-                    const float4 na = *reinterpret_cast<const float4 *>(np + 8 * ch);
-                    const float4 nb = *reinterpret_cast<const float4 *>(np + 8 * ch + 4);
-                    nq += bf_lo(qv.x) * na.x + bf_hi(qv.x) * na.y + bf_lo(qv.y) * na.z + bf_hi(qv.y) * na.w +
-                          bf_lo(qv.z) * nb.x + bf_hi(qv.z) * nb.y + bf_lo(qv.w) * nb.z + bf_hi(qv.w) * nb.w;
-                }
-            }
+            // n'.q_t from the normaliser columns (hi + mid + lo parts)
+            const float nq = __uint_as_float(sn[0]) + __uint_as_float(sn[1]) + __uint_as_float(sn[2]);
             // masked, weighted scores as bf16 (the B operand of the intra product) and their row sum
             const float rho = gs[GS_RHO];
             const float *w = garr(gb, G_W) + 32 * hh;
@@ -733,15 +797,19 @@ segment_output_rs_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
                 *reinterpret_cast<uint4 *>(sP + sw128_offset(t, 4 * hh + cq)) = make_uint4(p4[0], p4[1], p4[2], p4[3]);
             }
             rowsum += __shfl_xor_sync(0xffffffffu, rowsum, 16);
-            nq += __shfl_xor_sync(0xffffffffu, nq, 16);
             if (hh == 0) {
                 const float gt = garr(gb, G_G)[t];
                 float den;
                 if (!wide) den = gt * (nq + rho * rowsum);
                 else if (!late) den = gt * (nq + rowsum);
-                else den = rowsum;
+                else den = rowsum;            // the old state's share is below fp32 resolution
                 // 0.5: sigma(o) = (1 + tanh(o / 2)) / 2
                 garr(gb, G_INV)[t] = valid ? 0.5f * garr(gb, G_OF)[t] / fmaxf(fabsf(den), garr(gb, G_FL)[t]) : 0.f;
+                if (KS > 1 && tile == 0 && valid) {   // this CTA's share of the denominator, and the row factors
+                    const size_t tk = tok0 + (size_t)(c0 + c) * kL + t;
+                    dpart[(size_t)kh * gridDim.z * S + tk] = den;
+                    if (kh == 0) tokrec[tk] = make_float2(garr(gb, G_OF)[t], garr(gb, G_FL)[t]);
+                }
             }
             fence_async_smem();
             tc_fence_before();
@@ -749,8 +817,6 @@ segment_output_rs_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
             if (xleader) {
                 mbar_arrive(&bars[B_PR]);
                 mbar_arrive(&bars[B_SE]);
-                mbar_arrive(&bars[B_QE0 + sl]);
-                mbar_arrive(&bars[B_NE0 + sl]);
                 mbar_arrive(&bars[B_GE0 + gb]);
             }
             RS_TRACE(xleader, c, 17);
@@ -764,13 +830,37 @@ segment_output_rs_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
     }
 }
 
+// DH 512: the two key halves' numerators and denominators are summed and the
+// output formed, h = sigma(o) * f_t (N_0 + N_1) / max(|d_0 + d_1|, e^{-m_t});
+// f_t is the row factor (g_t, or 1 in a wide chunk's rows whose retrieval was
+// dropped).  An HBM stream: four value columns of one token per thread.
+__global__ void __launch_bounds__(256)
+combine_keysplit_kernel(const float *__restrict__ part, const float *__restrict__ dpart,
+                        const float2 *__restrict__ tokrec, const float *__restrict__ o_pre,
+                        __nv_bfloat16 *__restrict__ h, size_t tokens, int D) {
+    const size_t n4 = tokens * (size_t)(D / 4);
+    const size_t stride = (size_t)gridDim.x * blockDim.x;
+    for (size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x; e < n4; e += stride) {
+        const size_t tk = e / (D / 4);
+        const float4 a = reinterpret_cast<const float4 *>(part)[e];
+        const float4 b = reinterpret_cast<const float4 *>(part + tokens * D)[e];
+        const float4 o = reinterpret_cast<const float4 *>(o_pre)[e];
+        const float2 tr = tokrec[tk];
+        const float f = tr.x / fmaxf(fabsf(dpart[tk] + dpart[tokens + tk]), tr.y);
+        const float x0 = (a.x + b.x) * f, x1 = (a.y + b.y) * f, x2 = (a.z + b.z) * f, x3 = (a.w + b.w) * f;
+        uint2 out;
+        out.x = cvt_bf16x2(x0 * sigmoid(o.x), x1 * sigmoid(o.y));
+        out.y = cvt_bf16x2(x2 * sigmoid(o.z), x3 * sigmoid(o.w));
+        reinterpret_cast<uint2 *>(h)[e] = out;
+    }
+}
+
 template <int D>
 cudaError_t launch_rs_t(const FwdArgs &a, const FwdPlan &p, cudaStream_t st) {
     using Cfg = RsCfg<D>;
-    CUtensorMap mq, mk, mv, mh, mo;
+    CUtensorMap mq, mk, mv, mo;
     if (!make_map_bf16(&mq, a.q, p.BH, p.S, D) || !make_map_bf16(&mk, a.k, p.BH, p.S, D) ||
-        !make_map_bf16(&mv, a.v, p.BH, p.S, D) || !make_map_bf16(&mh, a.h, p.BH, p.S, D, false, 64) ||
-        !make_map_f32_rows(&mo, a.o_pre, p.BH, p.S, D, Cfg::RV, 64))
+        !make_map_bf16(&mv, a.v, p.BH, p.S, D) || !make_map_f32_rows(&mo, a.o_pre, p.BH, p.S, D, Cfg::RV, 64))
         return cudaErrorInvalidValue;
     cudaError_t e = launch_segment_summaries(a, p, st);
     if (e != cudaSuccess) return e;
@@ -779,12 +869,27 @@ cudaError_t launch_rs_t(const FwdArgs &a, const FwdPlan &p, cudaStream_t st) {
     const int sm = Cfg::kBytes > 118784 ? Cfg::kBytes : 118784;
     e = cudaFuncSetAttribute(segment_output_rs_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
     if (e != cudaSuccess) return e;
-    KernelTimer timer("segment_output_rs", st);
-    segment_output_rs_kernel<D><<<dim3(D / Cfg::RV, p.P, p.BH), kRsThreads, sm, st>>>(
-        mq, mk, mv, mh, mo, a.i_pre, a.C0, a.n0, a.m0, a.C_out, a.n_out, a.m_out, ws + p.off_bcum,
-        ws + p.off_pmax, (const float2 *)(ws + p.off_cstat), (const float2 *)(ws + p.off_sstat),
-        ws + p.off_summ, a.status, p.S, p.nchunks, p.P, p.cps);
-    return cudaGetLastError();
+    float *part = Cfg::KS > 1 ? ws + p.off_part : nullptr;
+    float *dpart = Cfg::KS > 1 ? ws + p.off_dpart : nullptr;
+    float2 *tokrec = Cfg::KS > 1 ? (float2 *)(ws + p.off_tok) : nullptr;
+    {
+        KernelTimer timer("segment_output_rs", st);
+        segment_output_rs_kernel<D><<<dim3((D / Cfg::RV) * Cfg::KS, p.P, p.BH), kRsThreads, sm, st>>>(
+            mq, mk, mv, mo, (__nv_bfloat16 *)a.h, a.i_pre, a.C0, a.n0, a.m0, a.C_out, a.n_out, a.m_out,
+            ws + p.off_bcum, ws + p.off_pmax, (const float2 *)(ws + p.off_cstat), (const float2 *)(ws + p.off_sstat),
+            ws + p.off_summ, part, dpart, tokrec, a.status, p.S, p.nchunks, p.P, p.cps);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    if (Cfg::KS > 1) {
+        KernelTimer timer("combine_keysplit", st);
+        const size_t n4 = (size_t)p.BH * p.S * (D / 4);
+        const unsigned blocks = (unsigned)((n4 + 255) / 256 < (size_t)8 * num_sms_current_device()
+                                               ? (n4 + 255) / 256 : (size_t)8 * num_sms_current_device());
+        combine_keysplit_kernel<<<blocks, 256, 0, st>>>(part, dpart, tokrec, a.o_pre, (__nv_bfloat16 *)a.h,
+                                                        (size_t)p.BH * p.S, D);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    return cudaSuccess;
 }
 
 }  // namespace
@@ -795,7 +900,7 @@ extern "C" int xlstm_debug_set_rs_trace(void *buf) {
 }
 #endif
 
-bool rs_path_supports(int DH, int L) { return L == kL && (DH == 64 || DH == 128 || DH == 256); }
+bool rs_path_supports(int DH, int L) { return L == kL && (DH == 64 || DH == 128 || DH == 256 || DH == 512); }
 
 cudaError_t launch_fwd_rs(const FwdArgs &a, const FwdPlan &p, cudaStream_t st) {
     if (!a.bf16 || !rs_path_supports(p.DH, p.L)) return cudaErrorInvalidValue;
@@ -805,6 +910,7 @@ cudaError_t launch_fwd_rs(const FwdArgs &a, const FwdPlan &p, cudaStream_t st) {
         case 64: return launch_rs_t<64>(a, p, st);
         case 128: return launch_rs_t<128>(a, p, st);
         case 256: return launch_rs_t<256>(a, p, st);
+        case 512: return launch_rs_t<512>(a, p, st);
     }
     return cudaErrorInvalidValue;
 }

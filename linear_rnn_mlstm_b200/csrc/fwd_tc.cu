@@ -984,10 +984,15 @@ segment_scan_kernel(const float2 *__restrict__ sstat, float *__restrict__ summ, 
 // cores too, as rows 0 and 1 (w in bf16 high and low parts) of an M=64 product
 // with the same K tile.  K and V stream through a 4-stage ring; V is scaled by
 // w in place.
+// DH 512 splits the key columns over two CTAs (KC = 256 each); their summaries
+// are independent column blocks of the same dC, so nothing is exchanged.
 template <int D>
 struct SumLayout {
+    static constexpr int KC = D > 256 ? 256 : D;          // key columns per CTA
+    static constexpr int KS = D / KC;                     // key splits
+    static constexpr int NT = (D + 127) / 128;            // value-row tiles
     static constexpr int kStages = 4;
-    static constexpr int kKslot = (D / 64) * 8192;        // K bf16: D/64 blocks x 64 rows
+    static constexpr int kKslot = (KC / 64) * 8192;       // K bf16: KC/64 blocks x 64 rows
     static constexpr int kSlot = kKslot + 16384 + 8192;   // + V (2 blocks x 8 KB) + W (64 x 64 bf16, rows 0-1 used)
     static constexpr int kF = kStages * kSlot;            // w[64]
     static constexpr int kTab = kF + 64 * 4;              // E per chunk
@@ -995,7 +1000,7 @@ struct SumLayout {
     static constexpr int kMisc = kBar + 16 * 8;
     static constexpr int kBytes = kMisc + 16 + 1024;
 };
-static_assert(SumLayout<256>::kBytes <= kMaxSmemPerCta, "summary kernel shared memory");
+static_assert(SumLayout<512>::kBytes <= kMaxSmemPerCta, "summary kernel shared memory");
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -1019,8 +1024,9 @@ segment_summary_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __gri
     __shared__ float s_mloc, s_etot;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int tile = blockIdx.x, g = blockIdx.y, bh = blockIdx.z;
-    const int i0 = tile * kRows;
+    constexpr int KC = Lay::KC, KS = Lay::KS, NT = Lay::NT;
+    const int tile = blockIdx.x / KS, kh = blockIdx.x % KS, g = blockIdx.y, bh = blockIdx.z;
+    const int i0 = tile * kRows, k0 = kh * KC;
     const int c0 = g * cps;
     const int nch = min(nchunks, c0 + cps) - c0;
     const size_t tok0 = (size_t)bh * S;
@@ -1047,7 +1053,7 @@ segment_summary_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __gri
         }
         s_mloc = mloc;
         s_etot = E;
-        if (tile == 0) sstat[(size_t)bh * P + g] = make_float2(E, mloc);
+        if (blockIdx.x == 0) sstat[(size_t)bh * P + g] = make_float2(E, mloc);
     }
     if (warp == 1) {
         tmem_alloc(tmem_slot, 512);
@@ -1062,10 +1068,10 @@ segment_summary_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __gri
     fence_async_smem();
     __syncthreads();
     tc_fence_after();
-    const uint32_t tacc = *tmem_slot;                  // dC in columns [0, D), dn rows in [256, 256 + D)
+    const uint32_t tacc = *tmem_slot;                  // dC in columns [0, KC), dn rows in [256, 256 + KC)
     const float mloc = s_mloc;
-    const uint32_t idesc_U = idesc_f32acc(kFmtBF16, kFmtBF16, true, true, 128, D);
-    const uint32_t idesc_N = idesc_f32acc(kFmtBF16, kFmtBF16, false, true, 64, D);
+    const uint32_t idesc_U = idesc_f32acc(kFmtBF16, kFmtBF16, true, true, 128, KC);
+    const uint32_t idesc_N = idesc_f32acc(kFmtBF16, kFmtBF16, false, true, 64, KC);
 
     if (warp == 0) {
         if (lane == 0) {
@@ -1076,9 +1082,9 @@ segment_summary_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __gri
                 const int slot = c % NS, t0 = (c0 + c) * kL;
                 if (c >= NS && !mbar_wait(&b_free[slot], ((c / NS) - 1) & 1, abort_flag, status)) break;
                 uint8_t *base = smem + slot * Lay::kSlot;
-                mbar_arrive_expect_tx(&b_full[slot], kL * D * 2 + kL * kVBlocks * 64 * 2);
-                for (int jb = 0; jb < D / 64; ++jb)
-                    tma_load_3d(base + jb * 8192, &map_k, &b_full[slot], jb * 64, t0, bh);
+                mbar_arrive_expect_tx(&b_full[slot], kL * KC * 2 + kL * kVBlocks * 64 * 2);
+                for (int jb = 0; jb < KC / 64; ++jb)
+                    tma_load_3d(base + jb * 8192, &map_k, &b_full[slot], k0 + jb * 64, t0, bh);
                 for (int b = 0; b < kVBlocks; ++b)
                     tma_load_3d(base + Lay::kKslot + b * 8192, &map_v, &b_full[slot], i0 + 64 * b, t0, bh);
                 ++issued[slot];
@@ -1164,28 +1170,28 @@ segment_summary_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __gri
             float *out = summ + ((size_t)bh * (P - 1) + g) * ((size_t)D * D + D);
             const int i = 32 * q4 + lane;
             const uint32_t lane_addr = ((uint32_t)(32 * q4)) << 16;
-            const int jhalf = (ct >> 7) * (D / 2);
-            for (int jb = jhalf; jb < jhalf + D / 2; jb += 16) {
+            const int jhalf = (ct >> 7) * (KC / 2);
+            for (int jb = jhalf; jb < jhalf + KC / 2; jb += 16) {
                 uint32_t r[16];
                 tmem_ld16(tacc + lane_addr + jb, r);
                 tmem_wait_ld();
                 if (i0 + i >= D) continue;                  // padding rows (DH < 128)
-                float4 *dst = reinterpret_cast<float4 *>(out + (size_t)(i0 + i) * D + jb);
+                float4 *dst = reinterpret_cast<float4 *>(out + (size_t)(i0 + i) * D + k0 + jb);
 #pragma unroll
                 for (int e = 0; e < 4; ++e)
                     dst[e] = make_float4(__uint_as_float(r[4 * e]), __uint_as_float(r[4 * e + 1]),
                                          __uint_as_float(r[4 * e + 2]), __uint_as_float(r[4 * e + 3]));
             }
             if (q4 == 0) {      // dn = rows 0 + 1 of the M=64 product (TMEM lanes 0 and 1)
-                for (int jb = jhalf; jb < jhalf + D / 2; jb += 16) {
+                for (int jb = jhalf; jb < jhalf + KC / 2; jb += 16) {
                     uint32_t r[16];
                     tmem_ld16(tacc + 256 + jb, r);
                     tmem_wait_ld();
 #pragma unroll
                     for (int e = 0; e < 16; ++e) {
                         const float v = __uint_as_float(r[e]) + __shfl_down_sync(0xffffffffu, __uint_as_float(r[e]), 1);
-                        if (lane == 0 && (jb + e) / 128 == tile)      // each tile writes its 128 columns
-                            out[(size_t)D * D + jb + e] = v;
+                        if (lane == 0 && (jb + e) / (KC / NT) == tile)   // the value tiles share out the columns
+                            out[(size_t)D * D + k0 + jb + e] = v;
                     }
                 }
             }
@@ -1217,7 +1223,7 @@ cudaError_t launch_summaries_t(const FwdArgs &a, const FwdPlan &p, cudaStream_t 
     if (e != cudaSuccess) return e;
     {
         KernelTimer timer("segment_summary_tc", st);
-        segment_summary_tc_kernel<D><<<dim3((D + kRows - 1) / kRows, p.P - 1, p.BH), kThreads, sm, st>>>(
+        segment_summary_tc_kernel<D><<<dim3(SumLayout<D>::NT * SumLayout<D>::KS, p.P - 1, p.BH), kThreads, sm, st>>>(
             mk, mv, a.i_pre, bcum, cstat, sstat, summ, a.status, p.S, p.nchunks, p.P, p.cps);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
@@ -1301,6 +1307,7 @@ cudaError_t launch_segment_summaries(const FwdArgs &a, const FwdPlan &p, cudaStr
         case 64: return launch_summaries_t<64>(a, p, st);
         case 128: return launch_summaries_t<128>(a, p, st);
         case 256: return launch_summaries_t<256>(a, p, st);
+        case 512: return launch_summaries_t<512>(a, p, st);
     }
     return cudaErrorInvalidValue;
 }

@@ -34,6 +34,10 @@ struct FwdPlan {
     size_t off_cstat;         // [BH, nchunks, 2]  (chunk total of log f, chunk max of log i - b)
     size_t off_sstat;         // [BH, P, 2]     (segment total of log f, segment stabiliser)
     size_t off_summ;          // [BH, P-1, DH*DH + DH]  segment summaries (C part then n part)
+    // DH 512 on the tensor path (key columns split over two CTAs):
+    size_t off_part;          // [2, BH, S, DH]  each key half's numerator
+    size_t off_dpart;         // [2, BH, S]      each key half's denominator
+    size_t off_tok;           // [BH, S, 2]      row factor and floor per token
     size_t total_floats;
     size_t bytes() const { return total_floats * sizeof(float); }
 };

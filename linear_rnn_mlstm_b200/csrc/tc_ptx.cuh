@@ -80,6 +80,39 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
     }
 }
 
+// Potentially suspending test of the phase: the thread may sleep in hardware
+// until the phase completes or about `hint_ns` nanoseconds pass.
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity, uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+
+// As mbar_wait, but the waiting thread sleeps in hardware between checks
+// (mbarrier.try_wait with a suspend hint) instead of spinning, so a waiter
+// takes almost no issue slots from the warps sharing its scheduler.  Same
+// bound, abort and status semantics.
+__device__ __forceinline__ bool mbar_wait_sleep(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                                unsigned int *status, uint64_t limit_ns = 2000000000ull) {
+    if (mbar_test_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (;;) {
+        if (mbar_try_wait(bar, parity, 100000u)) return true;
+        if (abort_flag && *abort_flag) return false;
+        if (globaltimer_ns() - t0 > limit_ns) {
+            if (abort_flag) *abort_flag = 1;
+            if (status) atomicOr(status, 1u);
+            return false;
+        }
+    }
+}
+
 // A bounded wait on behalf of the `N` threads that use named barrier `ID`:
 // only `leader` polls the mbarrier (the others block in the named barrier and
 // issue nothing), then all of them receive the same verdict.

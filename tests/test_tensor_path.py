@@ -1,8 +1,8 @@
 """The tensor-core forwards (bf16, chunk 64) against the float64 oracle, forced
 through the tensor path, on the cases their design has to get right beyond the
 plain workloads.  Two kernel families: the register-state kernel (DH 64, 128,
-256; XLSTM_PATH_TENSOR) and the tensor-memory-state kernel (DH 128, 256;
-XLSTM_PATH_TENSOR_TMEM).  Cases:
+256; XLSTM_PATH_TENSOR_RS) and the tensor-memory-state kernel (DH 128, 256;
+XLSTM_PATH_TENSOR_TMEM); XLSTM_PATH_TENSOR picks between them.  Cases:
 
 - several value-row tiles and several segments per head, ragged tails;
 - the exponential forget gate;
@@ -26,7 +26,7 @@ from parity import STATE_M_ABS, STATE_REL_L2, assert_close, errors, gpu_fwd, ora
 pytestmark = pytest.mark.gpu
 
 
-FAMILIES = [xb.PATH_TENSOR, xb.PATH_TENSOR_TMEM]
+FAMILIES = [xb.PATH_TENSOR_RS, xb.PATH_TENSOR_TMEM]
 
 
 def _check(inp, fgate, seg, C0=None, n0=None, m0=None, families=FAMILIES):
@@ -53,6 +53,8 @@ CASES = [
     (1, 1, 63, 256, "exp", 0),
     (2, 1, 640, 256, "sigmoid", 10),
     (1, 1, 64, 64, "sigmoid", 0),
+    (1, 2, 300, 512, "exp", 0),
+    (2, 1, 517, 512, "sigmoid", 3),
     (2, 3, 777, 64, "sigmoid", 4),
     (1, 2, 300, 64, "exp", 0),
 ]
@@ -66,7 +68,7 @@ def test_tensor_path_vs_oracle(case):
     _check(syn.fwd_inputs(w), fgate, seg)
 
 
-@pytest.mark.parametrize("DH", [64, 128, 256])
+@pytest.mark.parametrize("DH", [64, 128, 256, 512])
 def test_tensor_path_rescaled_state(DH):
     # log sigmoid(1 +- 0.5) ~ -0.3 per token: the state's scale falls below
     # e^-40 every few chunks and is reset in TMEM
@@ -76,10 +78,11 @@ def test_tensor_path_rescaled_state(DH):
 
 
 @pytest.mark.parametrize("seg", [0, 3])
-def test_tensor_path_wide_chunks(seg):
+@pytest.mark.parametrize("DH", [256, 512])
+def test_tensor_path_wide_chunks(seg, DH):
     # log sigmoid(-4 +- 1) ~ -4 per token and itilde ~ N(0, 3): within one chunk
     # the input terms span e^250
-    w = syn.custom("tc_wide", 1, 2, 1000, 256, syn.SMALL, dtype="bf16", seed=11,
+    w = syn.custom("tc_wide", 1, 2, 1000, DH, syn.SMALL, dtype="bf16", seed=11,
                    f_mu=-4.0, f_sd=1.0, i_sd=3.0)
     _check(syn.fwd_inputs(w), "sigmoid", seg)
 
@@ -106,6 +109,7 @@ def test_tensor_path_initial_state():
 
 
 @pytest.mark.parametrize("dtype,DH,chunk,fam", [("f32", 128, 64, xb.PATH_TENSOR), ("bf16", 48, 64, xb.PATH_TENSOR),
+                                                ("bf16", 512, 128, xb.PATH_TENSOR),
                                                 ("bf16", 64, 64, xb.PATH_TENSOR_TMEM),
                                                 ("bf16", 128, 128, xb.PATH_TENSOR_TMEM)])
 def test_tensor_path_refuses_unsupported(dtype, DH, chunk, fam):
