@@ -79,9 +79,13 @@ struct RsCfg {
     static constexpr int kK = kQ + 2 * kQbytes;
     static constexpr int kV = kK + 2 * kKbytes;
     static constexpr int kO = kV + 2 * kVbytes;
-    static constexpr int kP = kO + kObytes;            // [64][64] bf16 masked scores, 128 B swizzle
+    // [64][64] bf16 masked scores, 128 B swizzle; with split keys also a low part
+    // (each CTA's partial scores are rounded on their own, so where the halves
+    // cancel one bf16 rounding would be amplified)
+    static constexpr int kPparts = KS > 1 ? 2 : 1;
+    static constexpr int kP = kO + kObytes;
     static constexpr int kGB = 3;                      // gate buffers (ring)
-    static constexpr int kG = kP + 8192;               // per-token gate arrays [kGB][kNG][64]
+    static constexpr int kG = kP + kPparts * 8192;     // per-token gate arrays [kGB][kNG][64]
     static constexpr int kNG = 8;
     static constexpr int kGs = kG + kGB * kNG * 64 * 4;  // per-chunk gate scalars [kGB][8]
     static constexpr int kBar = kGs + kGB * 8 * 4;
@@ -506,9 +510,11 @@ segment_output_rs_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
                     {
                         const uint32_t va = smem_u32(sV + sl * Cfg::kVbytes), pa = smem_u32(sP);
 #pragma unroll
-                        for (int ks = 0; ks < 4; ++ks)
-                            mma_bf16_ss(tHb, sdesc_sw128(va + ks * 2048, 8192, 1024), sdesc_sw128(pa + ks * 32, 16, 1024),
-                                        idesc_I, 1u);
+                        for (int pp = 0; pp < Cfg::kPparts; ++pp)
+#pragma unroll
+                            for (int ks = 0; ks < 4; ++ks)
+                                mma_bf16_ss(tHb, sdesc_sw128(va + ks * 2048, 8192, 1024),
+                                            sdesc_sw128(pa + pp * 8192 + ks * 32, 16, 1024), idesc_I, 1u);
                         mma_commit(&bars[B_PE]);
                         mma_commit(&bars[B_HF0 + hb]);
                         if (wide) mma_commit(&bars[B_ID]);
@@ -774,7 +780,7 @@ segment_output_rs_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
             float rowsum = 0.f;
 #pragma unroll
             for (int cq = 0; cq < 4; ++cq) {
-                uint32_t p4[4];
+                uint32_t p4[4], l4[4];
 #pragma unroll
                 for (int p2 = 0; p2 < 4; ++p2) {
                     float pv[2];
@@ -793,8 +799,11 @@ segment_output_rs_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
                         }
                     }
                     p4[p2] = cvt_bf16x2(pv[0], pv[1]);
+                    if (KS > 1) l4[p2] = cvt_bf16x2(pv[0] - bf_lo(p4[p2]), pv[1] - bf_hi(p4[p2]));
                 }
                 *reinterpret_cast<uint4 *>(sP + sw128_offset(t, 4 * hh + cq)) = make_uint4(p4[0], p4[1], p4[2], p4[3]);
+                if (KS > 1)
+                    *reinterpret_cast<uint4 *>(sP + 8192 + sw128_offset(t, 4 * hh + cq)) = make_uint4(l4[0], l4[1], l4[2], l4[3]);
             }
             rowsum += __shfl_xor_sync(0xffffffffu, rowsum, 16);
             if (hh == 0) {
