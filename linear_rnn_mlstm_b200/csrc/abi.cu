@@ -56,7 +56,8 @@ bool make_fwd_plan(int B, int NH, int S, int DH, int L, int path, int forced_seg
     }
     int P;
     // DH 512 on the tensor path splits each value tile's keys over two CTAs
-    const long per_set = (long)p->BH * p->ntiles * (tensor && DH > 256 ? 2 : 1);
+    const int ksplit = tensor ? rs_key_splits(DH, L) : 1;
+    const long per_set = (long)p->BH * p->ntiles * ksplit;
     if (forced_segments > 0) {
         P = forced_segments;
     } else if (tensor) {
@@ -84,7 +85,7 @@ bool make_fwd_plan(int B, int NH, int S, int DH, int L, int path, int forced_seg
     p->off_cstat = off; off = align64(off + (size_t)p->BH * p->nchunks * 2);
     p->off_sstat = off; off = align64(off + (size_t)p->BH * p->P * 2);
     p->off_summ = off;  off = align64(off + (size_t)p->BH * (p->P - 1) * ((size_t)DH * DH + DH));
-    if (tensor && DH > 256) {
+    if (ksplit > 1) {
         p->off_part = off;  off = align64(off + 2 * (size_t)p->BH * S * DH);
         p->off_dpart = off; off = align64(off + 2 * (size_t)p->BH * S);
         p->off_tok = off;   off = align64(off + 2 * (size_t)p->BH * S);

@@ -3,36 +3,50 @@
 // 2.3: retrieval by matrix multiplication, covariance update of the matrix
 // memory; section 2.2: exponential gating with the stabiliser m).
 //
-// One CTA owns RV = min(DH, 128) value rows of one head over one segment of
-// the sequence (the segments combine through the two-level scan of
-// fwd_tc.cu).  Chunk L = 64.  The CTA's rows of the stabilised state C' stay
-// in fp32 registers of eight "state" warps for the whole segment; before each
-// chunk those warps write the state into tensor memory as two bf16 parts,
-// C' = Chi + Clo (15 to 16 significant bits), the A operand of the retrieval.
-// Per chunk c with queries Q, keys K, values V (bf16, staged by TMA):
+// One CTA owns RV = min(DH, 128) value rows and KC key columns of one head's
+// state over one segment of the sequence (the segments combine through the
+// two-level scan of fwd_tc.cu).  The CTA's part of the stabilised state C'
+// stays in fp32 registers of eight "state" warps for the whole segment; at
+// each chunk boundary those warps fold the chunk's update into it and write
+// it into tensor memory as two bf16 parts, C' = Chi + Clo (15 to 16
+// significant bits), the A operand of the retrieval.
 //
-//   S    = Q [K; n'hi; n'mid; n'lo]^T               M=64,  N=72, K=DH
-//   H^T  = (Chi + Clo) Q^T                          M=128, N=64, K=DH (A in TMEM)
-//   H^T += (w V)^T P^T,  P = rho * S masked s <= t  M=128, N=64, K=64
-//   U    = (w V)^T K                                M=128, N=DH, K=64
-//   C'  <- a C' + U                                 (fp32, in the state warps)
+// A chunk of L = 64 NSUB tokens is processed as NSUB sub-blocks of 64 tokens.
+// The state is carried across chunks only; inside a chunk the outputs are the
+// causal quadratic form over all L tokens, taken tile by tile.  Per chunk,
+// with Q_j, K_i, V_i the bf16 tiles of sub-blocks j, i (staged by TMA):
+//
+//   S_ji  = Q_j [K_i; n'hi; n'mid; n'lo]^T        M=64,  N=72, K=KC  (i <= j)
+//   H_j^T = sum_{i<=j} (w V_i)^T P_ji^T            M=128, N=64, K=64
+//           P_ji = rho * S_ji (masked s <= t when i = j)
+//   H_j^T += (Chi + Clo) Q_j^T                     M=128, N=64, K=KC (A in TMEM)
+//   U     = sum_i (w V_i)^T K_i                    M=128, N=KC, K=64
+//   C'   <- a C' + U                               (fp32, in the state warps)
 //
 // with u_s = itilde_s - b_s (b = within-chunk cumulative log f), Mc = max_s
-// u_s, m_prev the stabiliser before the chunk, M = max(m_prev, Mc) and
+// u_s over the chunk, m_prev the stabiliser before the chunk, M = max(m_prev,
+// Mc) and
 //   w_s = e^{u_s - M} / sqrt(d),  rho = e^{M - m_prev},  a = e^{m_prev - M},
 //   g_t = e^{m_prev - max(m_prev, pmax_t)},  m_t = b_t + max(m_prev, pmax_t),
-// so the state after the chunk is exactly a C' + U (all exponents <= 0), and
-// the exact intra-chunk weight e^{b_t - b_s + itilde_s - m_t} / sqrt(d)
-// equals g_t rho w_s, so
-//   h_t = o_t * g_t H_t / max(|g_t (n'.q_t + rho sum_s w_s S_ts)|, e^{-m_t}),
-// where n'.q_t rides in the scores product: the normaliser n', as three bf16
-// parts (hi + mid + lo, about 24 significant bits), fills key rows 64-66 of
-// the key tile, so S has 72 columns.
+// so the state after the chunk is exactly a C' + U (all exponents <= 0), the
+// exact intra-chunk weight e^{b_t - b_s + itilde_s - m_t} / sqrt(d) equals
+// g_t rho w_s, and
+//   h_t = o_t * g_t H_t / max(|g_t (n'.q_t + rho sum_s w_s S_ts)|, e^{-m_t}).
+// n'.q_t rides in the scores product: the normaliser n' (of the chunk start),
+// as three bf16 parts (about 24 significant bits), fills key rows 64-66 of
+// every key tile, so S has 72 columns.
 // A chunk is "wide" when Mc > m_prev + 40 (rho would leave the fp32 range):
 // then P carries exact per-row weights against V as loaded (rows whose own
 // stabiliser moved by more than e^40 have the old state's share below fp32
-// resolution; their retrieval term is dropped by zeroing those query rows),
-// and V is scaled by w only after the intra-chunk product has read it.
+// resolution; their retrieval term is dropped by zeroing those query rows
+// after the scores have read them), and V is scaled by w only after the
+// intra-chunk products have read it.
+//
+// DH 512 (and DH 256 at chunk 256) split the key columns over KS = 2 CTAs:
+// the cell is linear in the scores and the state until the final division, so
+// each CTA writes its share of the numerator and the denominator (its scores
+// carried as bf16 hi + lo parts, since the halves' partial scores can cancel)
+// and combine_keysplit_kernel forms h.
 //
 // Warp roles (16 warps): 0 TMA (q, k, v), 1 MMA issue and TMEM owner, 2 gates
 // and the normaliser chain n', 3 TMA (output gates); 4-11 state (C' rows, the
@@ -51,24 +65,25 @@ using namespace tc;
 
 namespace {
 
-constexpr int kL = 64;
 constexpr int kRsThreads = 512;
 constexpr float kWideGap = 40.f;   // ln of the largest factor rho may take
 
-template <int D>
+template <int D, int NSUB>
 struct RsCfg {
-    static constexpr int KC = D > 256 ? 256 : D;       // key columns of the state in this CTA
-    static constexpr int KS = D / KC;                  // key splits (DH 512: two CTAs per value tile)
+    static constexpr int L = 64 * NSUB;                // chunk (tokens)
+    static constexpr int KC = (NSUB == 4 && D >= 256) ? 128 : (D > 256 ? 256 : D);   // key columns per CTA
+    static constexpr int KS = D / KC;                  // key splits (CTAs per value tile)
     static constexpr int RV = D < 128 ? D : 128;       // value rows (MMAs keep M = 128)
     static constexpr int VB = RV / 64;                 // 64-column blocks of the value tile
     static constexpr int KPT = KC / 2;                 // keys per state thread (two warps per lane quadrant)
+    static constexpr int NKV = NSUB >= 2 ? NSUB : 2;   // key / value slots (one chunk, or a ring of two)
+    static constexpr int TPC = NSUB * (NSUB + 1) / 2;  // score tiles per chunk
     static constexpr bool kSharedRU = 2 * KC + 72 + 128 > 512;
     static constexpr uint32_t R0 = 0;                  // bf16 parts: hi [0, KC/2), lo [KC/2, KC)
     static constexpr uint32_t U0 = kSharedRU ? 0 : KC; // fp32 chunk update
     static constexpr uint32_t S0 = kSharedRU ? KC : 2 * KC;
     static constexpr uint32_t H0 = S0 + 72;            // two 64-column buffers
     static_assert(H0 + 128 <= 512, "tensor memory");
-    static_assert(!kSharedRU || KC + 72 + 128 <= 512, "tensor memory");
     // shared memory (bytes; 1024-aligned operand tiles first)
     static constexpr int kQbytes = (KC / 64) * 8192;   // [64 tokens][KC] bf16, 64-key blocks, 128 B swizzle
     static constexpr int kKBlock = 72 * 128;           // key block: 64 key rows + n' hi/mid/lo + 5 zero rows
@@ -77,35 +92,36 @@ struct RsCfg {
     static constexpr int kObytes = KS == 1 ? 64 * RV * 4 : 0;   // [64 tokens][RV] fp32 output-gate pre-activations
     static constexpr int kQ = 0;
     static constexpr int kK = kQ + 2 * kQbytes;
-    static constexpr int kV = kK + 2 * kKbytes;
-    static constexpr int kO = kV + 2 * kVbytes;
+    static constexpr int kV = kK + NKV * kKbytes;
+    static constexpr int kO = kV + NKV * kVbytes;
     // [64][64] bf16 masked scores, 128 B swizzle; with split keys also a low part
     // (each CTA's partial scores are rounded on their own, so where the halves
     // cancel one bf16 rounding would be amplified)
     static constexpr int kPparts = KS > 1 ? 2 : 1;
     static constexpr int kP = kO + kObytes;
-    static constexpr int kGB = 3;                      // gate buffers (ring)
-    static constexpr int kG = kP + kPparts * 8192;     // per-token gate arrays [kGB][kNG][64]
+    static constexpr int kGB = NSUB >= 4 ? 2 : 3;      // gate buffers (ring)
     static constexpr int kNG = 8;
-    static constexpr int kGs = kG + kGB * kNG * 64 * 4;  // per-chunk gate scalars [kGB][8]
+    static constexpr int kG = kP + kPparts * 8192;     // per-token gate arrays [kGB][kNG][L]
+    static constexpr int kGs = kG + kGB * kNG * L * 4; // per-chunk gate scalars [kGB][8]
     static constexpr int kBar = kGs + kGB * 8 * 4;
-    static constexpr int kNumBars = 48;
+    static constexpr int kNumBars = 56;
     static constexpr int kMisc = kBar + kNumBars * 8;
     static constexpr int kBytes = kMisc + 64 + 1024;   // + slack for 1024-byte alignment
+    static_assert(kBytes <= 232448, "shared memory");
 };
-static_assert(RsCfg<256>::kBytes <= 232448 && RsCfg<512>::kBytes <= 232448, "shared memory");
 
 // per-token gate arrays
 enum { G_W = 0, G_G, G_FL, G_U, G_REF, G_OF, G_INV, G_LATE };
 // per-chunk scalars
-enum { GS_RHO = 0, GS_A, GS_BETA, GS_WIDE, GS_LC };
+enum { GS_RHO = 0, GS_A, GS_WIDE, GS_LC };
 
+// barriers; the K / V ones have one slot per key/value buffer (up to 4)
 enum {
-    B_QF0 = 0, B_QF1, B_QE0, B_QE1, B_KF0, B_KF1, B_KE0, B_KE1, B_VF0, B_VF1, B_VE0, B_VE1,
-    B_OF, B_OE, B_SF, B_SE, B_PR, B_PE, B_HF0, B_HF1, B_HE0, B_HE1, B_RR, B_RD, B_UF,
-    B_VH0, B_VH1, B_ID, B_GR0, B_GR1, B_GR2, B_GE0, B_GE1, B_GE2, B_NR0, B_NR1, B_DONE, B_NUM
+    B_QF = 0, B_QE = 2, B_KF = 4, B_KE = 8, B_VF = 12, B_VE = 16, B_VH = 20,
+    B_OF = 24, B_OE, B_SF, B_SE, B_PR, B_PE, B_HF, B_HE = B_HF + 2, B_RR = B_HE + 2, B_RD, B_UF, B_ID,
+    B_SQ, B_QZ, B_GR, B_GE = B_GR + 3, B_NR = B_GE + 3, B_INV, B_DONE = B_INV + 2, B_NUM
 };
-static_assert(B_NUM <= RsCfg<64>::kNumBars, "barrier slots");
+static_assert(B_NUM <= 56, "barrier slots");
 
 #ifdef XLSTM_RS_TRACE
 // Timing trace of the pipeline steps (diagnostic builds only): 32 clock64()
@@ -140,7 +156,7 @@ __device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
 __device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
-// named barriers: 1 = state group (256 threads), 2 = score/output group (128)
+// named barriers: 1 = state group (256 threads), 2 = score group (128)
 __device__ __forceinline__ void sync_state() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 __device__ __forceinline__ void sync_so() { asm volatile("bar.sync 2, 128;" ::: "memory"); }
 
@@ -170,7 +186,15 @@ __device__ __forceinline__ void write_parts(const float (&Cs)[KPT], uint32_t t_r
     tmem_wait_st();
 }
 
-template <int D>
+// Score tile t of a chunk (0 <= t < NSUB (NSUB + 1) / 2) in issue order
+// (0,0), (1,0), (1,1), (2,0), ...: query sub-block j, key sub-block i <= j.
+__device__ __forceinline__ void tile_ji(int t, int &j, int &i) {
+    j = 0;
+    while ((j + 1) * (j + 2) / 2 <= t) ++j;
+    i = t - j * (j + 1) / 2;
+}
+
+template <int D, int NSUB>
 __global__ void __launch_bounds__(kRsThreads, 1)
 segment_output_rs_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
                          const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_o,
@@ -181,9 +205,9 @@ segment_output_rs_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
                          const float2 *__restrict__ cstat, const float2 *__restrict__ sstat,
                          const float *__restrict__ summ, float *__restrict__ part, float *__restrict__ dpart,
                          float2 *__restrict__ tokrec, unsigned int *status, int S, int nchunks, int P, int cps) {
-    using Cfg = RsCfg<D>;
-    constexpr int KC = Cfg::KC, KS = Cfg::KS, RV = Cfg::RV, VB = Cfg::VB, KPT = Cfg::KPT, GB = Cfg::kGB;
-    constexpr int KB = Cfg::kKBlock;
+    using Cfg = RsCfg<D, NSUB>;
+    constexpr int L = Cfg::L, KC = Cfg::KC, KS = Cfg::KS, RV = Cfg::RV, VB = Cfg::VB, KPT = Cfg::KPT;
+    constexpr int GB = Cfg::kGB, KB = Cfg::kKBlock, NKV = Cfg::NKV, TPC = Cfg::TPC;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = align1024(smem_raw);
     uint8_t *sQ = smem + Cfg::kQ;
@@ -191,18 +215,20 @@ segment_output_rs_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
     uint8_t *sV = smem + Cfg::kV;
     float *sO = reinterpret_cast<float *>(smem + Cfg::kO);
     uint8_t *sP = smem + Cfg::kP;
-    float *gA = reinterpret_cast<float *>(smem + Cfg::kG);      // [GB][kNG][64]
+    float *gA = reinterpret_cast<float *>(smem + Cfg::kG);      // [GB][kNG][L]
     float *gS = reinterpret_cast<float *>(smem + Cfg::kGs);     // [GB][8]
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cfg::kBar);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + Cfg::kMisc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + Cfg::kMisc + 4);
-    auto garr = [&](int gb, int which) { return gA + (gb * Cfg::kNG + which) * 64; };
+    auto garr = [&](int gb, int which) { return gA + (gb * Cfg::kNG + which) * L; };
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int tile = blockIdx.x / KS, kh = blockIdx.x % KS, g = blockIdx.y, bh = blockIdx.z;
     const int i0 = tile * RV, k0 = kh * KC;        // value rows and key columns of this CTA
-    const int c0 = g * cps;
+    const int c0 = g * cps;                        // first chunk of this segment
     const int nch = max(0, min(nchunks, c0 + cps) - c0);
+    const int nsb = nch * NSUB;                    // sub-blocks of this segment
+    const int tseg = c0 * L;                       // first token of this segment
     const size_t tok0 = (size_t)bh * S;
     const float inv_sqrt_d = rsqrtf((float)D);
     const int q4 = warp & 3;
@@ -210,7 +236,7 @@ segment_output_rs_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
 
     if (tid == 0) {
         for (int i = 0; i < B_NUM; ++i) {
-            const bool two = i == B_KE0 || i == B_KE1 || i == B_GE0 || i == B_GE1 || i == B_GE2;
+            const bool two = (i >= B_KE && i < B_KE + 4) || (i >= B_GE && i < B_GE + 3);
             mbar_init(&bars[i], two ? 2 : 1);
         }
         *abort_flag = 0;
@@ -223,12 +249,12 @@ segment_output_rs_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
     }
     // rows 64-71 of every key block start at zero (TMA writes rows 0-63 only;
     // the normaliser parts go to rows 64-66), and so does an unloaded value block
-    for (int e = tid; e < 2 * (KC / 64) * 64; e += kRsThreads) {     // (slot, block, row 64-71, chunk)
+    for (int e = tid; e < NKV * (KC / 64) * 64; e += kRsThreads) {     // (slot, block, row 64-71, chunk)
         const int ch = e & 7, row = 64 + ((e >> 3) & 7), blk = (e >> 6) % (KC / 64), sl = e / (64 * (KC / 64));
         *reinterpret_cast<uint4 *>(sK + sl * Cfg::kKbytes + blk * KB + sw128_offset(row, ch)) = make_uint4(0u, 0u, 0u, 0u);
     }
     if (VB == 1) {
-        for (int e = tid; e < 2 * 512; e += kRsThreads)
+        for (int e = tid; e < NKV * 512; e += kRsThreads)
             *reinterpret_cast<uint4 *>(sV + (e >> 9) * Cfg::kVbytes + 8192 + (e & 511) * 16) = make_uint4(0u, 0u, 0u, 0u);
     }
     fence_async_smem();
@@ -238,59 +264,58 @@ segment_output_rs_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
     const uint32_t tR = tbase + Cfg::R0, tU = tbase + Cfg::U0, tS = tbase + Cfg::S0, tH = tbase + Cfg::H0;
 
     // Register budget per warpgroup (KC = 256: the state warps hold 128 floats of
-    // C' per thread): 128 x 48 + 256 x 176 + 128 x 104 = 64512 <= 512 x 128.
+    // C' per thread): 128 x 64 + 256 x 168 + 128 x 104 = 64512 <= 512 x 128.
     if (warp < 4) {
-        if (KC == 256) regs_dec<48>();
+        if (KC == 256) regs_dec<64>();
         if (warp == 0) {
-            // -------------------------------------------------------- TMA: q, k, v
+            // ------------------------------------------------ TMA: q, k, v per sub-block
             if (lane == 0 && nch > 0) {
                 tma_prefetch_desc(&map_q);
                 tma_prefetch_desc(&map_k);
                 tma_prefetch_desc(&map_v);
-                int issued[3][2] = {};
-                for (int c = 0; c < nch; ++c) {
-                    const int t0 = (c0 + c) * kL, sl = c & 1;
-                    const uint32_t par = ((c >> 1) - 1) & 1;
-                    if (c + 2 < nch) {
+                int issued[3][4] = {};
+                for (int b = 0; b < nsb; ++b) {
+                    const int t0 = tseg + 64 * b, qs = b & 1, ks = b % NKV;
+                    if (b + 2 < nsb) {
                         for (int jb = 0; jb < KC / 64; ++jb) {
-                            tma_prefetch_l2_3d(&map_q, k0 + jb * 64, t0 + 2 * kL, bh);
-                            tma_prefetch_l2_3d(&map_k, k0 + jb * 64, t0 + 2 * kL, bh);
+                            tma_prefetch_l2_3d(&map_q, k0 + jb * 64, t0 + 128, bh);
+                            tma_prefetch_l2_3d(&map_k, k0 + jb * 64, t0 + 128, bh);
                         }
-                        for (int b = 0; b < VB; ++b) tma_prefetch_l2_3d(&map_v, i0 + 64 * b, t0 + 2 * kL, bh);
+                        for (int vb = 0; vb < VB; ++vb) tma_prefetch_l2_3d(&map_v, i0 + 64 * vb, t0 + 128, bh);
                     }
-                    if (c >= 2 && !rs_wait(&bars[B_QE0 + sl], par, abort_flag, status)) break;
-                    mbar_arrive_expect_tx(&bars[B_QF0 + sl], kL * KC * 2);
+                    if (b >= 2 && !rs_wait(&bars[B_QE + qs], ((b >> 1) - 1) & 1, abort_flag, status)) break;
+                    mbar_arrive_expect_tx(&bars[B_QF + qs], 64 * KC * 2);
                     for (int jb = 0; jb < KC / 64; ++jb)
-                        tma_load_3d(sQ + sl * Cfg::kQbytes + jb * 8192, &map_q, &bars[B_QF0 + sl], k0 + jb * 64, t0, bh);
-                    ++issued[0][sl];
-                    if (c >= 2 && !rs_wait(&bars[B_KE0 + sl], par, abort_flag, status)) break;
-                    mbar_arrive_expect_tx(&bars[B_KF0 + sl], kL * KC * 2);
+                        tma_load_3d(sQ + qs * Cfg::kQbytes + jb * 8192, &map_q, &bars[B_QF + qs], k0 + jb * 64, t0, bh);
+                    ++issued[0][qs];
+                    if (b >= NKV && !rs_wait(&bars[B_KE + ks], ((b / NKV) - 1) & 1, abort_flag, status)) break;
+                    mbar_arrive_expect_tx(&bars[B_KF + ks], 64 * KC * 2);
                     for (int jb = 0; jb < KC / 64; ++jb)
-                        tma_load_3d(sK + sl * Cfg::kKbytes + jb * KB, &map_k, &bars[B_KF0 + sl], k0 + jb * 64, t0, bh);
-                    ++issued[1][sl];
-                    if (c >= 2 && !rs_wait(&bars[B_VE0 + sl], par, abort_flag, status)) break;
-                    mbar_arrive_expect_tx(&bars[B_VF0 + sl], kL * VB * 64 * 2);
-                    for (int b = 0; b < VB; ++b)
-                        tma_load_3d(sV + sl * Cfg::kVbytes + b * 8192, &map_v, &bars[B_VF0 + sl], i0 + 64 * b, t0, bh);
-                    ++issued[2][sl];
+                        tma_load_3d(sK + ks * Cfg::kKbytes + jb * KB, &map_k, &bars[B_KF + ks], k0 + jb * 64, t0, bh);
+                    ++issued[1][ks];
+                    if (b >= NKV && !rs_wait(&bars[B_VE + ks], ((b / NKV) - 1) & 1, abort_flag, status)) break;
+                    mbar_arrive_expect_tx(&bars[B_VF + ks], 64 * VB * 64 * 2);
+                    for (int vb = 0; vb < VB; ++vb)
+                        tma_load_3d(sV + ks * Cfg::kVbytes + vb * 8192, &map_v, &bars[B_VF + ks], i0 + 64 * vb, t0, bh);
+                    ++issued[2][ks];
                 }
                 // never leave a load in flight into shared memory
-                for (int sl = 0; sl < 2; ++sl) {
-                    if (issued[0][sl]) mbar_wait(&bars[B_QF0 + sl], (issued[0][sl] - 1) & 1, nullptr, status);
-                    if (issued[1][sl]) mbar_wait(&bars[B_KF0 + sl], (issued[1][sl] - 1) & 1, nullptr, status);
-                    if (issued[2][sl]) mbar_wait(&bars[B_VF0 + sl], (issued[2][sl] - 1) & 1, nullptr, status);
+                for (int s = 0; s < 4; ++s) {
+                    if (s < 2 && issued[0][s]) mbar_wait(&bars[B_QF + s], (issued[0][s] - 1) & 1, nullptr, status);
+                    if (s < NKV && issued[1][s]) mbar_wait(&bars[B_KF + s], (issued[1][s] - 1) & 1, nullptr, status);
+                    if (s < NKV && issued[2][s]) mbar_wait(&bars[B_VF + s], (issued[2][s] - 1) & 1, nullptr, status);
                 }
             }
         } else if (warp == 3) {
-            // -------------------------------------------------- TMA: output gates
+            // ------------------------------------------ TMA: output gates per sub-block
             if (KS == 1 && lane == 0 && nch > 0) {
                 tma_prefetch_desc(&map_o);
                 int issued = 0;
-                for (int c = 0; c < nch; ++c) {
-                    const int t0 = (c0 + c) * kL;
-                    if (c + 1 < nch) tma_prefetch_l2_3d(&map_o, i0, t0 + kL, bh);
-                    if (c >= 1 && !rs_wait(&bars[B_OE], (c - 1) & 1, abort_flag, status)) break;
-                    mbar_arrive_expect_tx(&bars[B_OF], kL * RV * 4);
+                for (int b = 0; b < nsb; ++b) {
+                    const int t0 = tseg + 64 * b;
+                    if (b + 1 < nsb) tma_prefetch_l2_3d(&map_o, i0, t0 + 64, bh);
+                    if (b >= 1 && !rs_wait(&bars[B_OE], (b - 1) & 1, abort_flag, status)) break;
+                    mbar_arrive_expect_tx(&bars[B_OF], 64 * RV * 4);
                     tma_load_3d(sO, &map_o, &bars[B_OF], i0, t0, bh);
                     ++issued;
                 }
@@ -306,11 +331,12 @@ segment_output_rs_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
                 const float2 st = sstat[(size_t)bh * P + gp];
                 mc = fmaxf(st.x + mc, st.y);
             }
-            float pb_[2] = {0.f, 0.f}, px_[2] = {0.f, 0.f}, pi_[2] = {0.f, 0.f};
+            constexpr int TPL = L / 32;                      // tokens per lane
+            float pb_[TPL], px_[TPL], pi_[TPL];
             auto fetch = [&](int c) {
-                const int t0 = (c0 + c) * kL;
+                const int t0 = tseg + c * L;
 #pragma unroll
-                for (int h2 = 0; h2 < 2; ++h2) {
+                for (int h2 = 0; h2 < TPL; ++h2) {
                     const int t = t0 + lane + 32 * h2;
                     const bool ok = t < S;
                     pb_[h2] = ok ? bcum[tok0 + t] : 0.f;
@@ -319,16 +345,18 @@ segment_output_rs_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
                 }
             };
             auto gates = [&](int c) -> bool {
-                const int gb = c % GB, t0 = (c0 + c) * kL, Lc = min(kL, S - t0);
-                if (c >= GB && !rs_wait(&bars[B_GE0 + gb], ((c / GB) - 1) & 1, abort_flag, status)) return false;
+                const int gb = c % GB, t0 = tseg + c * L, Lc = min(L, S - t0);
+                if (c >= GB && !rs_wait(&bars[B_GE + gb], ((c / GB) - 1) & 1, abort_flag, status)) return false;
                 const float2 cs = cstat[(size_t)bh * nchunks + c0 + c];   // (sum of log f, max of u)
                 const float Mc = cs.y;
                 const bool wide = Mc > mc + kWideGap;
                 const float big = fmaxf(mc, Mc);
-                const float b_[2] = {pb_[0], pb_[1]}, x_[2] = {px_[0], px_[1]}, ii_[2] = {pi_[0], pi_[1]};
+                float b_[TPL], x_[TPL], ii_[TPL];
+#pragma unroll
+                for (int h2 = 0; h2 < TPL; ++h2) { b_[h2] = pb_[h2]; x_[h2] = px_[h2]; ii_[h2] = pi_[h2]; }
                 if (c + 1 < nch) fetch(c + 1);
 #pragma unroll
-                for (int h2 = 0; h2 < 2; ++h2) {
+                for (int h2 = 0; h2 < TPL; ++h2) {
                     const int t = lane + 32 * h2;
                     const bool valid = t < Lc;
                     const float u = ii_[h2] - b_[h2];
@@ -348,17 +376,16 @@ segment_output_rs_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
                     float *gs = gS + gb * 8;
                     gs[GS_RHO] = wide ? 0.f : expf(big - mc);
                     gs[GS_A] = expf(mc - big);
-                    gs[GS_BETA] = expf(Mc - big);
                     gs[GS_WIDE] = wide ? 1.f : 0.f;
                     gs[GS_LC] = (float)Lc;
                 }
                 mc = cs.x + big;
                 __syncwarp();
                 RS_TRACE(lane == 0, c, 24);
-                if (lane == 0) mbar_arrive(&bars[B_GR0 + gb]);
+                if (lane == 0) mbar_arrive(&bars[B_GR + gb]);
                 return true;
             };
-            // normaliser n': lane holds keys [KPL lane, KPL lane + KPL)
+            // normaliser n': lane holds keys [KPL lane, KPL lane + KPL) of this CTA's columns
             constexpr int KPL = KC / 32;
             float nr[KPL];
             const float *nsrc = g == 0 ? (n0 ? n0 + (size_t)bh * D : nullptr)
@@ -389,57 +416,63 @@ segment_output_rs_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
                     *reinterpret_cast<uint32_t *>(blk + sw128_offset(65, cc) + within) = pmid[e];
                     *reinterpret_cast<uint32_t *>(blk + sw128_offset(66, cc) + within) = plo[e];
                 }
+            };
+            // the parts of chunk c go to the key slots of its sub-blocks
+            auto publish_n = [&](int c) {
+                for (int j = 0; j < NSUB; ++j) write_nparts((c * NSUB + j) % NKV);
                 fence_async_smem();
                 __syncwarp();
+                if (lane == 0) mbar_arrive(&bars[B_NR]);
             };
             bool ok = true;
             if (nch > 0) {
                 fetch(0);
                 ok = gates(0) && (nch < 2 || gates(1));
-                if (ok) {
-                    write_nparts(0);
-                    if (lane == 0) mbar_arrive(&bars[B_NR0]);
-                }
+                if (ok) publish_n(0);
             }
             for (int c = 0; ok && c < nch; ++c) {
-                const int sl = c & 1, gb = c % GB;
+                const int gb = c % GB;
                 // n'(c+1) = a n'(c) + sum_s w_s k_s over this chunk's keys, fp32
-                if (!rs_wait(&bars[B_KF0 + sl], (c >> 1) & 1, abort_flag, status)) { ok = false; break; }
                 const float *w = garr(gb, G_W);
                 const float a = gS[gb * 8 + GS_A];
-                const uint8_t *kt = sK + sl * Cfg::kKbytes + kblk * KB;
                 float acc[KPL];
 #pragma unroll
                 for (int e = 0; e < KPL; ++e) acc[e] = 0.f;
+                for (int j = 0; j < NSUB && ok; ++j) {
+                    const int b = c * NSUB + j, ks = b % NKV;
+                    if (!rs_wait(&bars[B_KF + ks], (b / NKV) & 1, abort_flag, status)) { ok = false; break; }
+                    const uint8_t *kt = sK + ks * Cfg::kKbytes + kblk * KB;
 #pragma unroll 4
-                for (int s = 0; s < kL; ++s) {
-                    const float ws = w[s];
-                    const uint8_t *rp = kt + sw128_offset(s, kbyte >> 4) + (kbyte & 15);
-                    if (KPL == 8) {
-                        const uint4 kv = *reinterpret_cast<const uint4 *>(rp);
-                        acc[0] += ws * bf_lo(kv.x); acc[1] += ws * bf_hi(kv.x);
-                        acc[2] += ws * bf_lo(kv.y); acc[3] += ws * bf_hi(kv.y);
-                        acc[4] += ws * bf_lo(kv.z); acc[5] += ws * bf_hi(kv.z);
-                        acc[6 % KPL] += ws * bf_lo(kv.w); acc[7 % KPL] += ws * bf_hi(kv.w);
-                    } else if (KPL == 4) {
-                        const uint2 kv = *reinterpret_cast<const uint2 *>(rp);
-                        acc[0] += ws * bf_lo(kv.x); acc[1] += ws * bf_hi(kv.x);
-                        acc[2 % KPL] += ws * bf_lo(kv.y); acc[3 % KPL] += ws * bf_hi(kv.y);
-                    } else {
-                        const uint32_t kv = *reinterpret_cast<const uint32_t *>(rp);
-                        acc[0] += ws * bf_lo(kv); acc[1 % KPL] += ws * bf_hi(kv);
+                    for (int s = 0; s < 64; ++s) {
+                        const float ws = w[64 * j + s];
+                        const uint8_t *rp = kt + sw128_offset(s, kbyte >> 4) + (kbyte & 15);
+                        if (KPL == 8) {
+                            const uint4 kv = *reinterpret_cast<const uint4 *>(rp);
+                            acc[0] += ws * bf_lo(kv.x); acc[1] += ws * bf_hi(kv.x);
+                            acc[2] += ws * bf_lo(kv.y); acc[3] += ws * bf_hi(kv.y);
+                            acc[4 % KPL] += ws * bf_lo(kv.z); acc[5 % KPL] += ws * bf_hi(kv.z);
+                            acc[6 % KPL] += ws * bf_lo(kv.w); acc[7 % KPL] += ws * bf_hi(kv.w);
+                        } else if (KPL == 4) {
+                            const uint2 kv = *reinterpret_cast<const uint2 *>(rp);
+                            acc[0] += ws * bf_lo(kv.x); acc[1] += ws * bf_hi(kv.x);
+                            acc[2 % KPL] += ws * bf_lo(kv.y); acc[3 % KPL] += ws * bf_hi(kv.y);
+                        } else {
+                            const uint32_t kv = *reinterpret_cast<const uint32_t *>(rp);
+                            acc[0] += ws * bf_lo(kv); acc[1 % KPL] += ws * bf_hi(kv);
+                        }
                     }
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&bars[B_KE + ks]);
                 }
+                if (!ok) break;
 #pragma unroll
                 for (int e = 0; e < KPL; ++e) nr[e] = fmaf(a, nr[e], acc[e]);
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&bars[B_KE0 + sl]);
                 if (c + 1 < nch) {
-                    // scores(c - 1) read this slot's normaliser rows; the update of chunk
-                    // c - 1 completing implies they are done
-                    if (c >= 1 && !rs_wait(&bars[B_UF], (c - 1) & 1, abort_flag, status)) { ok = false; break; }
-                    write_nparts((c + 1) & 1);
-                    if (lane == 0) mbar_arrive(&bars[B_NR0 + ((c + 1) & 1)]);
+                    // the slots chunk c+1 uses were last read by the scores of chunk
+                    // c + 1 - NKV / NSUB; that chunk's update completing implies they are done
+                    const int cp = c + 1 - NKV / NSUB;
+                    if (cp >= 0 && !rs_wait(&bars[B_UF], cp & 1, abort_flag, status)) { ok = false; break; }
+                    publish_n(c + 1);
                 }
                 if (c + 2 < nch && !gates(c + 2)) { ok = false; break; }
             }
@@ -457,10 +490,23 @@ segment_output_rs_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
                 const uint32_t idesc_R = idesc_f32acc(kFmtBF16, kFmtBF16, false, false, 128, 64);
                 const uint32_t idesc_I = idesc_f32acc(kFmtBF16, kFmtBF16, true, false, 128, 64);
                 const uint32_t idesc_U = idesc_f32acc(kFmtBF16, kFmtBF16, true, true, 128, KC);
-                auto issue_scores = [&](int c) {
-                    const int sl = c & 1;
-                    uint64_t dq = sdesc_sw128(smem_u32(sQ + sl * Cfg::kQbytes), 16, 1024);
-                    uint64_t dk = sdesc_sw128(smem_u32(sK + sl * Cfg::kKbytes), 16, 1024);
+                bool ok = true;
+                int nw = 0;                  // wide sub-blocks seen
+                // scores of global tile gt (chunk gt / TPC): wait for its operands and a free S
+                auto issue_scores = [&](int gt_) -> bool {
+                    const int c = gt_ / TPC;
+                    int j, i;
+                    tile_ji(gt_ % TPC, j, i);
+                    const int bq = c * NSUB + j, bk = c * NSUB + i;
+                    const int qs = bq & 1, ks = bk % NKV;
+                    if (!rs_wait(&bars[B_QF + qs], (bq >> 1) & 1, abort_flag, status) ||
+                        !rs_wait(&bars[B_KF + ks], (bk / NKV) & 1, abort_flag, status) ||
+                        !rs_wait(&bars[B_NR], c & 1, abort_flag, status) ||
+                        (gt_ >= 1 && !rs_wait(&bars[B_SE], (gt_ - 1) & 1, abort_flag, status)))
+                        return false;
+                    tc_fence_after();
+                    uint64_t dq = sdesc_sw128(smem_u32(sQ + qs * Cfg::kQbytes), 16, 1024);
+                    uint64_t dk = sdesc_sw128(smem_u32(sK + ks * Cfg::kKbytes), 16, 1024);
 #pragma unroll 1
                     for (int jb = 0; jb < KC / 64; ++jb) {
 #pragma unroll
@@ -469,83 +515,101 @@ segment_output_rs_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
                         dk += KB >> 4;
                     }
                     mma_commit(&bars[B_SF]);
+                    return true;
                 };
-                bool ok = rs_wait(&bars[B_QF0], 0, abort_flag, status) && rs_wait(&bars[B_KF0], 0, abort_flag, status) &&
-                          rs_wait(&bars[B_NR0], 0, abort_flag, status);
-                if (ok) {
-                    tc_fence_after();
-                    issue_scores(0);
-                }
+                const int ntiles = nch * TPC;
+                int issued_s = 0;            // score tiles issued so far (global order)
+                ok = issue_scores(0);
+                if (ok) issued_s = 1;
                 for (int c = 0; ok && c < nch; ++c) {
-                    const int sl = c & 1, hb = c & 1, gb = c % GB;
-                    const uint32_t par = (c >> 1) & 1;
-                    const uint32_t tHb = tH + 64 * hb;
-                    RS_TRACE(true, c, 0);
-                    if (!rs_wait(&bars[B_RR], c & 1, abort_flag, status) ||
-                        !rs_wait(&bars[B_GR0 + gb], (c / GB) & 1, abort_flag, status) ||
-                        (c >= 2 && !rs_wait(&bars[B_HE0 + hb], ((c >> 1) - 1) & 1, abort_flag, status))) { ok = false; break; }
-                    tc_fence_after();
+                    const int gb = c % GB;
+                    if (!rs_wait(&bars[B_GR + gb], (c / GB) & 1, abort_flag, status)) { ok = false; break; }
                     const bool wide = gS[gb * 8 + GS_WIDE] != 0.f;
-                    {   // retrieval: H^T = (Chi + Clo) Q^T, the parts of C' from TMEM
-                        uint64_t dq = sdesc_sw128(smem_u32(sQ + sl * Cfg::kQbytes), 16, 1024);
-#pragma unroll 1
-                        for (int jb = 0; jb < KC / 64; ++jb) {
-#pragma unroll
-                            for (int k4 = 0; k4 < 4; ++k4) {
-                                const uint32_t col = (uint32_t)(jb * 32 + 8 * k4);
-                                mma_bf16_ts(tHb, tR + col, dq + 2 * k4, idesc_R, (jb | k4) != 0);
-                                mma_bf16_ts(tHb, tR + KC / 2 + col, dq + 2 * k4, idesc_R, 1u);
-                            }
-                            dq += 8192 >> 4;
+                    for (int tt = 0; ok && tt < TPC; ++tt) {
+                        const int gt_ = c * TPC + tt;
+                        int j, i;
+                        tile_ji(tt, j, i);
+                        const int bq = c * NSUB + j, bk = c * NSUB + i;
+                        const int hb = bq & 1, ks = bk % NKV;
+                        const uint32_t tHb = tH + 64 * hb;
+                        RS_TRACE(tt == 0, c, 0);
+                        // the next score tile into S as soon as this one has been read
+                        // (across chunks only when the key slots allow it)
+                        if (gt_ + 1 < ntiles && issued_s == gt_ + 1 && (NKV > NSUB || tt + 1 < TPC)) {
+                            if (!issue_scores(gt_ + 1)) { ok = false; break; }
+                            issued_s = gt_ + 2;
                         }
-                        if (Cfg::kSharedRU) mma_commit(&bars[B_RD]);
-                        mma_commit(&bars[B_QE0 + sl]);
-                    }
-                    RS_TRACE(true, c, 1);
-                    // intra-chunk term: H^T += (w V)^T P^T (wide chunks: V as loaded)
-                    if ((!wide && !rs_wait(&bars[B_VH0 + sl], par, abort_flag, status)) ||
-                        !rs_wait(&bars[B_VF0 + sl], par, abort_flag, status) ||
-                        !rs_wait(&bars[B_PR], c & 1, abort_flag, status)) { ok = false; break; }
-                    tc_fence_after();
-                    {
-                        const uint32_t va = smem_u32(sV + sl * Cfg::kVbytes), pa = smem_u32(sP);
-#pragma unroll
-                        for (int pp = 0; pp < Cfg::kPparts; ++pp)
-#pragma unroll
-                            for (int ks = 0; ks < 4; ++ks)
-                                mma_bf16_ss(tHb, sdesc_sw128(va + ks * 2048, 8192, 1024),
-                                            sdesc_sw128(pa + pp * 8192 + ks * 32, 16, 1024), idesc_I, 1u);
-                        mma_commit(&bars[B_PE]);
-                        mma_commit(&bars[B_HF0 + hb]);
-                        if (wide) mma_commit(&bars[B_ID]);
-                    }
-                    RS_TRACE(true, c, 2);
-                    // scores of the next chunk
-                    if (c + 1 < nch) {
-                        const int ns = (c + 1) & 1;
-                        const uint32_t npar = ((c + 1) >> 1) & 1;
-                        if (!rs_wait(&bars[B_QF0 + ns], npar, abort_flag, status) ||
-                            !rs_wait(&bars[B_KF0 + ns], npar, abort_flag, status) ||
-                            !rs_wait(&bars[B_NR0 + ns], npar, abort_flag, status) ||
-                            !rs_wait(&bars[B_SE], c & 1, abort_flag, status)) { ok = false; break; }
+                        if (i == 0 && bq >= 2 && !rs_wait(&bars[B_HE + hb], ((bq >> 1) - 1) & 1, abort_flag, status)) { ok = false; break; }
+                        if ((!wide && !rs_wait(&bars[B_VH + ks], (bk / NKV) & 1, abort_flag, status)) ||
+                            !rs_wait(&bars[B_VF + ks], (bk / NKV) & 1, abort_flag, status) ||
+                            !rs_wait(&bars[B_PR], gt_ & 1, abort_flag, status)) { ok = false; break; }
                         tc_fence_after();
-                        issue_scores(c + 1);
-                        RS_TRACE(true, c, 3);
-                    }
-                    // update of the state: U = (w V)^T K, after the retrieval has read the parts
-                    if ((Cfg::kSharedRU && !rs_wait(&bars[B_RD], c & 1, abort_flag, status)) ||
-                        (wide && !rs_wait(&bars[B_VH0 + sl], par, abort_flag, status))) { ok = false; break; }
-                    tc_fence_after();
-                    {
-                        const uint32_t va = smem_u32(sV + sl * Cfg::kVbytes), ka = smem_u32(sK + sl * Cfg::kKbytes);
+                        {   // intra-chunk term: H_j^T (+)= (w V_i)^T P_ji^T (wide chunks: V as loaded)
+                            const uint32_t va = smem_u32(sV + ks * Cfg::kVbytes), pa = smem_u32(sP);
 #pragma unroll
-                        for (int ks = 0; ks < 4; ++ks)
-                            mma_bf16_ss(tU, sdesc_sw128(va + ks * 2048, 8192, 1024), sdesc_sw128(ka + ks * 2048, KB, 1024),
-                                        idesc_U, ks > 0 ? 1u : 0u);
-                        mma_commit(&bars[B_UF]);
-                        mma_commit(&bars[B_VE0 + sl]);
-                        mma_commit(&bars[B_KE0 + sl]);
-                        RS_TRACE(true, c, 4);
+                            for (int pp = 0; pp < Cfg::kPparts; ++pp)
+#pragma unroll
+                                for (int k4 = 0; k4 < 4; ++k4)
+                                    mma_bf16_ss(tHb, sdesc_sw128(va + k4 * 2048, 8192, 1024),
+                                                sdesc_sw128(pa + pp * 8192 + k4 * 32, 16, 1024), idesc_I,
+                                                (i | pp | k4) != 0);
+                            mma_commit(&bars[B_PE]);
+                        }
+                        RS_TRACE(tt == 0, c, 2);
+                        if (i == j) {
+                            // the sub-block's scores are all issued: a wide chunk zeroes the
+                            // query rows whose retrieval term is dropped before the retrieval
+                            if (wide) {
+                                mma_commit(&bars[B_SQ]);
+                                if (!rs_wait(&bars[B_QZ], nw & 1, abort_flag, status)) { ok = false; break; }
+                                ++nw;
+                            }
+                            if (j == 0 && !rs_wait(&bars[B_RR], c & 1, abort_flag, status)) { ok = false; break; }
+                            tc_fence_after();
+                            // retrieval: H_j^T += (Chi + Clo) Q_j^T, the parts of C' from TMEM
+                            uint64_t dq = sdesc_sw128(smem_u32(sQ + (bq & 1) * Cfg::kQbytes), 16, 1024);
+#pragma unroll 1
+                            for (int jb = 0; jb < KC / 64; ++jb) {
+#pragma unroll
+                                for (int k4 = 0; k4 < 4; ++k4) {
+                                    const uint32_t col = (uint32_t)(jb * 32 + 8 * k4);
+                                    mma_bf16_ts(tHb, tR + col, dq + 2 * k4, idesc_R, 1u);
+                                    mma_bf16_ts(tHb, tR + KC / 2 + col, dq + 2 * k4, idesc_R, 1u);
+                                }
+                                dq += 8192 >> 4;
+                            }
+                            mma_commit(&bars[B_HF + hb]);
+                            mma_commit(&bars[B_QE + (bq & 1)]);
+                            if (Cfg::kSharedRU && j == NSUB - 1) mma_commit(&bars[B_RD]);
+                            RS_TRACE(j == 0, c, 1);
+                        }
+                    }
+                    if (!ok) break;
+                    // the chunk's update: U = sum_i (w V_i)^T K_i, after every retrieval has read the parts
+                    if (wide) mma_commit(&bars[B_ID]);
+                    if (Cfg::kSharedRU && !rs_wait(&bars[B_RD], c & 1, abort_flag, status)) { ok = false; break; }
+                    for (int i = 0; ok && i < NSUB; ++i) {
+                        const int bk = c * NSUB + i, ks = bk % NKV;
+                        if (wide && !rs_wait(&bars[B_VH + ks], (bk / NKV) & 1, abort_flag, status)) { ok = false; break; }
+                        tc_fence_after();
+                        const uint32_t va = smem_u32(sV + ks * Cfg::kVbytes), ka = smem_u32(sK + ks * Cfg::kKbytes);
+#pragma unroll
+                        for (int k4 = 0; k4 < 4; ++k4)
+                            mma_bf16_ss(tU, sdesc_sw128(va + k4 * 2048, 8192, 1024), sdesc_sw128(ka + k4 * 2048, KB, 1024),
+                                        idesc_U, (i | k4) != 0);
+                    }
+                    if (!ok) break;
+                    mma_commit(&bars[B_UF]);
+                    for (int i = 0; i < NSUB; ++i) {
+                        const int ks = (c * NSUB + i) % NKV;
+                        mma_commit(&bars[B_VE + ks]);
+                        mma_commit(&bars[B_KE + ks]);
+                    }
+                    RS_TRACE(true, c, 4);
+                    // the first score tile of the next chunk, when it could not go early
+                    if (c + 1 < nch && issued_s == (c + 1) * TPC) {
+                        if (!issue_scores((c + 1) * TPC)) { ok = false; break; }
+                        issued_s = (c + 1) * TPC + 1;
                     }
                 }
                 mma_commit(&bars[B_DONE]);
@@ -553,13 +617,13 @@ segment_output_rs_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
             }
         }
     } else if (warp < 12) {
-        if (KC == 256) regs_inc<176>();
+        if (KC == 256) regs_inc<168>();
         // ------------------------------------------------------------ state group
         const int sw = warp - 4;                 // 0..7
         const int half = sw >> 2;                // key half (fold) and token half (outputs) of this thread
         const int i = 32 * q4 + lane;            // value row within the tile
         const bool has_row = i < RV;
-        const int kbase = half * KPT;            // first key column of this thread
+        const int kbase = half * KPT;            // first key column of this thread (within the CTA's KC)
         const bool leader = sw == 0 && lane == 0;
         float Cs[KPT];
         bool ok = true;
@@ -567,13 +631,13 @@ segment_output_rs_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
             const bool r = leader ? rs_wait(bar, parity, abort_flag, status) : true;
             return group_all<1, 256>(r);
         };
-        // V of chunk c scaled in place by w (the operand of the intra and update products)
-        auto scale_v = [&](int c, int gb) {
-            const int sl = c & 1;
-            const float *w = garr(gb, G_W);
-            uint8_t *vb = sV + sl * Cfg::kVbytes;
-            for (int e = sw * 32 + lane; e < VB * kL * 8; e += 256) {       // (block, row s, 16 B chunk)
-                const int blk = e / (kL * 8), s = (e / 8) % kL, cc = e & 7;
+        // V of sub-block b scaled in place by w (the operand of the intra and update products)
+        auto scale_v = [&](int b, int gb) {
+            const int ks = b % NKV;
+            const float *w = garr(gb, G_W) + 64 * (b % NSUB);
+            uint8_t *vb = sV + ks * Cfg::kVbytes;
+            for (int e = sw * 32 + lane; e < VB * 64 * 8; e += 256) {       // (block, row s, 16 B chunk)
+                const int blk = e / (64 * 8), s = (e / 8) % 64, cc = e & 7;
                 uint4 *pv = reinterpret_cast<uint4 *>(vb + blk * 8192 + sw128_offset(s, cc));
                 const uint4 src = *pv;
                 const float ws = w[s];
@@ -586,28 +650,20 @@ segment_output_rs_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
             }
             fence_async_smem();
             sync_state();
-            if (leader) mbar_arrive(&bars[B_VH0 + sl]);
+            if (leader) mbar_arrive(&bars[B_VH + ks]);
         };
-        // wide chunk c: zero the query rows whose retrieval term is dropped
-        auto zero_late_rows = [&](int c, int gb) {
-            const float *lt = garr(gb, G_LATE);
-            uint8_t *qt = sQ + (c & 1) * Cfg::kQbytes;
-            for (int e = sw * 32 + lane; e < (KC / 64) * kL * 8; e += 256) {
-                const int blk = e / (kL * 8), t = (e / 8) % kL, ch = e & 7;
-                if (lt[t] != 0.f)
-                    *reinterpret_cast<uint4 *>(qt + blk * 8192 + sw128_offset(t, ch)) = make_uint4(0u, 0u, 0u, 0u);
-            }
-            fence_async_smem();
-        };
-        // h of chunk c from H: this thread takes value row i, tokens 32 half ... + 31,
-        // and stores straight to global memory (a warp writes 64 contiguous bytes per token)
-        auto out_pass = [&](int c, int gb) -> bool {
-            const int hb = c & 1;
-            if (!swait(&bars[B_HF0 + hb], (c >> 1) & 1) || (KS == 1 && !swait(&bars[B_OF], c & 1))) return false;
-            RS_TRACE(leader, c, 20);
+        // h of sub-block b from H: this thread takes value row i, tokens 32 half ... + 31
+        // of the sub-block, and stores straight to global memory (a warp writes 64
+        // contiguous bytes per token); with split keys, this CTA's numerator share
+        auto out_pass = [&](int b, int gb) -> bool {
+            const int hb = b & 1;
+            if (!swait(&bars[B_HF + hb], (b >> 1) & 1) || !swait(&bars[B_INV + hb], (b >> 1) & 1) ||
+                (KS == 1 && !swait(&bars[B_OF], b & 1)))
+                return false;
+            RS_TRACE(leader, b / NSUB, 20);
             tc_fence_after();
-            const float *inv = garr(gb, G_INV);
-            const int t0 = (c0 + c) * kL;
+            const float *inv = garr(gb, G_INV) + 64 * (b % NSUB);
+            const int t0 = tseg + 64 * b;
             __nv_bfloat16 *hrow = h_out + (tok0 + t0) * D + i0 + i;
             float *prow = part + (((size_t)kh * gridDim.z + bh) * S + t0) * D + i0 + i;
 #pragma unroll 1
@@ -616,13 +672,14 @@ segment_output_rs_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
                 uint32_t r[16];
                 tmem_ld16(tH + 64 * hb + lane_addr + tb, r);
                 tmem_wait_ld();
-                if (KS > 1) {          // this CTA's share of the numerator, combined later
-                    const int lim = min(16, S - t0 - tb);
+                const int lim = min(16, S - t0 - tb);            // tokens of this piece inside the sequence
+                if (KS > 1) {
+                    if (has_row) {
 #pragma unroll
-                    for (int kk = 0; kk < 16; ++kk)
-                        if (lim >= 16 || kk < lim) prow[(size_t)(tb + kk) * D] = __uint_as_float(r[kk]);
+                        for (int kk = 0; kk < 16; ++kk)
+                            if (lim >= 16 || kk < lim) prow[(size_t)(tb + kk) * D] = __uint_as_float(r[kk]);
+                    }
                 } else if (has_row) {
-                    const int lim = min(16, S - t0 - tb);            // tokens of this piece inside the sequence
 #pragma unroll
                     for (int kk = 0; kk < 16; ++kk) {
                         const int tt = tb + kk;
@@ -636,11 +693,22 @@ segment_output_rs_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
             tc_fence_before();
             sync_state();
             if (leader) {
-                mbar_arrive(&bars[B_HE0 + hb]);
+                mbar_arrive(&bars[B_HE + hb]);
                 mbar_arrive(&bars[B_OE]);
             }
-            RS_TRACE(leader, c, 21);
+            RS_TRACE(leader, b / NSUB, 21);
             return true;
+        };
+        // wide chunk: zero the query rows of sub-block b whose retrieval term is dropped
+        auto zero_late_rows = [&](int b, int gb) {
+            const float *lt = garr(gb, G_LATE) + 64 * (b % NSUB);
+            uint8_t *qt = sQ + (b & 1) * Cfg::kQbytes;
+            for (int e = sw * 32 + lane; e < (KC / 64) * 64 * 8; e += 256) {
+                const int blk = e / (64 * 8), t = (e / 8) % 64, ch = e & 7;
+                if (lt[t] != 0.f)
+                    *reinterpret_cast<uint4 *>(qt + blk * 8192 + sw128_offset(t, ch)) = make_uint4(0u, 0u, 0u, 0u);
+            }
+            fence_async_smem();
         };
         // incoming state: the initial state for segment 0, else the state at the
         // end of segment g - 1, which segment_scan_kernel left in summary slot g - 1
@@ -660,35 +728,45 @@ segment_output_rs_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
             }
         }
         if (nch > 0) {
-            ok = swait(&bars[B_GR0], 0);
-            const bool wide0 = ok && gS[GS_WIDE] != 0.f;
-            if (wide0) {      // the scores of chunk 0 read Q before its late rows are zeroed
-                ok = swait(&bars[B_SF], 0) && swait(&bars[B_QF0], 0);
-                if (ok) zero_late_rows(0, 0);
-            }
-            if (ok) {
-                write_parts<KPT, KC>(Cs, tR + lane_addr, kbase);
-                tc_fence_before();
-                sync_state();
-                if (leader) mbar_arrive(&bars[B_RR]);
-                if (!wide0) {
-                    ok = swait(&bars[B_VF0], 0);
-                    if (ok) scale_v(0, 0);
-                }
-            }
+            write_parts<KPT, KC>(Cs, tR + lane_addr, kbase);
+            tc_fence_before();
+            sync_state();
+            if (leader) mbar_arrive(&bars[B_RR]);
+            ok = swait(&bars[B_GR], 0);
         }
-        int nwide = 0;
+        int nw = 0, nwc = 0;
         for (int c = 0; ok && c < nch; ++c) {
             const int gb = c % GB;
             const float a = gS[gb * 8 + GS_A];
             const bool wide = gS[gb * 8 + GS_WIDE] != 0.f;
-            // (1) wide chunk: scale V after the intra-chunk product has read it
-            if (wide) {
-                if (!swait(&bars[B_ID], nwide & 1)) { ok = false; break; }
-                ++nwide;
-                scale_v(c, gb);
+            // (1) w V for the chunk's sub-blocks as they land (wide chunks: after the intra products)
+            if (!wide) {
+                for (int j = 0; ok && j < NSUB; ++j) {
+                    const int b = c * NSUB + j;
+                    if (!swait(&bars[B_VF + b % NKV], (b / NKV) & 1)) { ok = false; break; }
+                    scale_v(b, gb);
+                }
+                if (!ok) break;
             }
-            // (2) fold the chunk's update into the fp32 state, then the next chunk's parts
+            // (2) per sub-block: the wide-chunk query rows, then h
+            for (int j = 0; ok && j < NSUB; ++j) {
+                const int b = c * NSUB + j;
+                if (wide) {
+                    if (!swait(&bars[B_SQ], nw & 1)) { ok = false; break; }
+                    ++nw;
+                    zero_late_rows(b, gb);
+                    sync_state();
+                    if (leader) mbar_arrive(&bars[B_QZ]);
+                }
+                if (!out_pass(b, gb)) { ok = false; break; }
+            }
+            if (!ok) break;
+            if (wide) {
+                if (!swait(&bars[B_ID], nwc & 1)) { ok = false; break; }
+                ++nwc;
+                for (int j = 0; j < NSUB; ++j) scale_v(c * NSUB + j, gb);
+            }
+            // (3) fold the chunk's update into the fp32 state, then the next chunk's parts
             RS_TRACE(leader, c, 8);
             if (!swait(&bars[B_UF], c & 1)) { ok = false; break; }
             RS_TRACE(leader, c, 10);
@@ -706,26 +784,14 @@ segment_output_rs_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
             tc_fence_after();
             RS_TRACE(leader, c, 11);
             if (c + 1 < nch) {
-                const int ngb = (c + 1) % GB;
-                if (!swait(&bars[B_GR0 + ngb], ((c + 1) / GB) & 1)) { ok = false; break; }
-                const bool nwide_c = gS[ngb * 8 + GS_WIDE] != 0.f;
-                if (nwide_c) zero_late_rows(c + 1, ngb);
+                if (!swait(&bars[B_GR + (c + 1) % GB], ((c + 1) / GB) & 1)) { ok = false; break; }
                 write_parts<KPT, KC>(Cs, tR + lane_addr, kbase);
                 tc_fence_before();
                 sync_state();
                 if (leader) mbar_arrive(&bars[B_RR]);
                 RS_TRACE(leader, c, 12);
-                // w V for the next chunk (wide chunks wait for their intra product)
-                if (!nwide_c) {
-                    if (!swait(&bars[B_VF0 + ((c + 1) & 1)], ((c + 1) >> 1) & 1)) { ok = false; break; }
-                    scale_v(c + 1, ngb);
-                    RS_TRACE(leader, c, 13);
-                }
             }
-            // (3) h of this chunk
-            if (!out_pass(c, gb)) { ok = false; break; }
-            sync_state();
-            if (leader) mbar_arrive(&bars[B_GE0 + gb]);
+            if (leader) mbar_arrive(&bars[B_GE + gb]);
         }
         // final state (last segment only)
         if (ok && g == P - 1 && nch > 0 && !*abort_flag && C_out && has_row) {
@@ -740,95 +806,109 @@ segment_output_rs_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
         // ------------------------------------------------------------ scores
         const int xt = tid - 384;                    // 0..127
         const bool xleader = xt == 0;
-        const int t = 16 * q4 + (lane & 15);         // score row (M = 64 layout: lanes 0-15 of the quadrant)
+        const int tr = 16 * q4 + (lane & 15);        // score row in the sub-block (M = 64 layout: lanes 0-15)
         const int hh = lane >> 4;                    // column half of this lane
         bool ok = true;
         auto xwait = [&](uint64_t *bar, uint32_t parity) -> bool {
             const bool r = xleader ? rs_wait(bar, parity, abort_flag, status) : true;
             return group_all<2, 128>(r);
         };
+        float rowsum = 0.f;
         for (int c = 0; ok && c < nch; ++c) {
             const int gb = c % GB;
-            if (!xwait(&bars[B_SF], c & 1) || !xwait(&bars[B_GR0 + gb], (c / GB) & 1) ||
-                (c >= 1 && !xwait(&bars[B_PE], (c - 1) & 1))) { ok = false; break; }
-            RS_TRACE(xleader, c, 16);
-            tc_fence_after();
-            uint32_t sa[32], sb[32], sn[8];
-            tmem_ld16(tS + lane_addr + 0, *reinterpret_cast<uint32_t(*)[16]>(&sa[0]));
-            tmem_ld16(tS + lane_addr + 16, *reinterpret_cast<uint32_t(*)[16]>(&sa[16]));
-            tmem_ld16(tS + lane_addr + 32, *reinterpret_cast<uint32_t(*)[16]>(&sb[0]));
-            tmem_ld16(tS + lane_addr + 48, *reinterpret_cast<uint32_t(*)[16]>(&sb[16]));
-            tmem_ld8(tS + lane_addr + 64, sn);
-            tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 32; ++e) {
-                const uint32_t up = __shfl_sync(0xffffffffu, sb[e], lane & 15);
-                sa[e] = hh ? up : sa[e];
-            }
+            if (!xwait(&bars[B_GR + gb], (c / GB) & 1)) { ok = false; break; }
             const float *gs = gS + gb * 8;
             const bool wide = gs[GS_WIDE] != 0.f;
             const int Lc = (int)gs[GS_LC];
-            const bool valid = t < Lc;
-            const float ref_t = garr(gb, G_REF)[t];
-            const bool late = garr(gb, G_LATE)[t] != 0.f;
-            // n'.q_t from the normaliser columns (hi + mid + lo parts)
-            const float nq = __uint_as_float(sn[0]) + __uint_as_float(sn[1]) + __uint_as_float(sn[2]);
-            // masked, weighted scores as bf16 (the B operand of the intra product) and their row sum
             const float rho = gs[GS_RHO];
-            const float *w = garr(gb, G_W) + 32 * hh;
-            const float *us = garr(gb, G_U) + 32 * hh;
-            float rowsum = 0.f;
+            for (int tt = 0; tt < TPC; ++tt) {
+                const int gt_ = c * TPC + tt;
+                int j, i;
+                tile_ji(tt, j, i);
+                if (!xwait(&bars[B_SF], gt_ & 1) || (gt_ >= 1 && !xwait(&bars[B_PE], (gt_ - 1) & 1))) { ok = false; break; }
+                RS_TRACE(xleader && tt == 0, c, 16);
+                tc_fence_after();
+                uint32_t sa[32], sb[32], sn[8];
+                tmem_ld16(tS + lane_addr + 0, *reinterpret_cast<uint32_t(*)[16]>(&sa[0]));
+                tmem_ld16(tS + lane_addr + 16, *reinterpret_cast<uint32_t(*)[16]>(&sa[16]));
+                tmem_ld16(tS + lane_addr + 32, *reinterpret_cast<uint32_t(*)[16]>(&sb[0]));
+                tmem_ld16(tS + lane_addr + 48, *reinterpret_cast<uint32_t(*)[16]>(&sb[16]));
+                tmem_ld8(tS + lane_addr + 64, sn);
+                tmem_wait_ld();
+                tc_fence_before();
+                sync_so();
+                if (xleader) mbar_arrive(&bars[B_SE]);           // S may be overwritten by the next tile
 #pragma unroll
-            for (int cq = 0; cq < 4; ++cq) {
-                uint32_t p4[4], l4[4];
+                for (int e = 0; e < 32; ++e) {
+                    const uint32_t up = __shfl_sync(0xffffffffu, sb[e], lane & 15);
+                    sa[e] = hh ? up : sa[e];
+                }
+                const int t = 64 * j + tr;                   // token of this row within the chunk
+                const bool valid = t < Lc;
+                const float ref_t = garr(gb, G_REF)[t];
+                const bool late = garr(gb, G_LATE)[t] != 0.f;
+                // masked, weighted scores as bf16 (the B operand of the intra product) and their row sum
+                const float *w = garr(gb, G_W) + 64 * i + 32 * hh;
+                const float *us = garr(gb, G_U) + 64 * i + 32 * hh;
+                if (i == 0) rowsum = 0.f;
 #pragma unroll
-                for (int p2 = 0; p2 < 4; ++p2) {
-                    float pv[2];
+                for (int cq = 0; cq < 4; ++cq) {
+                    uint32_t p4[4], l4[4];
 #pragma unroll
-                    for (int e = 0; e < 2; ++e) {
-                        const int sl2 = cq * 8 + p2 * 2 + e;
-                        const int s = 32 * hh + sl2;
-                        const bool keep = valid && s <= t;
-                        const float sc = keep ? __uint_as_float(sa[sl2]) : 0.f;
-                        if (!wide) {
-                            pv[e] = rho * sc;
-                            rowsum += w[sl2] * sc;
-                        } else {     // exp(u_s - ref_t) <= e^40 only where s <= t
-                            pv[e] = keep ? sc * (expf(us[sl2] - ref_t) * inv_sqrt_d) : 0.f;
-                            rowsum += pv[e];
+                    for (int p2 = 0; p2 < 4; ++p2) {
+                        float pv[2];
+#pragma unroll
+                        for (int e = 0; e < 2; ++e) {
+                            const int sl2 = cq * 8 + p2 * 2 + e;
+                            const int s = 64 * i + 32 * hh + sl2;     // key token within the chunk
+                            const bool keep = valid && s <= t;
+                            const float sc = keep ? __uint_as_float(sa[sl2]) : 0.f;
+                            if (!wide) {
+                                pv[e] = rho * sc;
+                                rowsum += w[sl2] * sc;
+                            } else {     // exp(u_s - ref_t) <= e^40 only where s <= t
+                                pv[e] = keep ? sc * (expf(us[sl2] - ref_t) * inv_sqrt_d) : 0.f;
+                                rowsum += pv[e];
+                            }
+                        }
+                        p4[p2] = cvt_bf16x2(pv[0], pv[1]);
+                        if (KS > 1) l4[p2] = cvt_bf16x2(pv[0] - bf_lo(p4[p2]), pv[1] - bf_hi(p4[p2]));
+                    }
+                    *reinterpret_cast<uint4 *>(sP + sw128_offset(tr, 4 * hh + cq)) = make_uint4(p4[0], p4[1], p4[2], p4[3]);
+                    if (KS > 1)
+                        *reinterpret_cast<uint4 *>(sP + 8192 + sw128_offset(tr, 4 * hh + cq)) =
+                            make_uint4(l4[0], l4[1], l4[2], l4[3]);
+                }
+                if (i == j) {       // the sub-block's last tile: denominators of its rows
+                    const float rs = rowsum + __shfl_xor_sync(0xffffffffu, rowsum, 16);
+                    if (hh == 0) {
+                        // n'.q_t from the normaliser columns (hi + mid + lo parts)
+                        const float nq = __uint_as_float(sn[0]) + __uint_as_float(sn[1]) + __uint_as_float(sn[2]);
+                        const float gt = garr(gb, G_G)[t];
+                        float den;
+                        if (!wide) den = gt * (nq + rho * rs);
+                        else if (!late) den = gt * (nq + rs);
+                        else den = rs;            // the old state's share is below fp32 resolution
+                        // 0.5: sigma(o) = (1 + tanh(o / 2)) / 2
+                        garr(gb, G_INV)[t] = valid ? 0.5f * garr(gb, G_OF)[t] / fmaxf(fabsf(den), garr(gb, G_FL)[t]) : 0.f;
+                        if (KS > 1 && tile == 0 && valid) {   // this CTA's share of the denominator, and the row factors
+                            const size_t tk = tok0 + (size_t)tseg + (size_t)c * L + t;
+                            dpart[(size_t)kh * gridDim.z * S + tk] = den;
+                            if (kh == 0) tokrec[tk] = make_float2(garr(gb, G_OF)[t], garr(gb, G_FL)[t]);
                         }
                     }
-                    p4[p2] = cvt_bf16x2(pv[0], pv[1]);
-                    if (KS > 1) l4[p2] = cvt_bf16x2(pv[0] - bf_lo(p4[p2]), pv[1] - bf_hi(p4[p2]));
                 }
-                *reinterpret_cast<uint4 *>(sP + sw128_offset(t, 4 * hh + cq)) = make_uint4(p4[0], p4[1], p4[2], p4[3]);
-                if (KS > 1)
-                    *reinterpret_cast<uint4 *>(sP + 8192 + sw128_offset(t, 4 * hh + cq)) = make_uint4(l4[0], l4[1], l4[2], l4[3]);
-            }
-            rowsum += __shfl_xor_sync(0xffffffffu, rowsum, 16);
-            if (hh == 0) {
-                const float gt = garr(gb, G_G)[t];
-                float den;
-                if (!wide) den = gt * (nq + rho * rowsum);
-                else if (!late) den = gt * (nq + rowsum);
-                else den = rowsum;            // the old state's share is below fp32 resolution
-                // 0.5: sigma(o) = (1 + tanh(o / 2)) / 2
-                garr(gb, G_INV)[t] = valid ? 0.5f * garr(gb, G_OF)[t] / fmaxf(fabsf(den), garr(gb, G_FL)[t]) : 0.f;
-                if (KS > 1 && tile == 0 && valid) {   // this CTA's share of the denominator, and the row factors
-                    const size_t tk = tok0 + (size_t)(c0 + c) * kL + t;
-                    dpart[(size_t)kh * gridDim.z * S + tk] = den;
-                    if (kh == 0) tokrec[tk] = make_float2(garr(gb, G_OF)[t], garr(gb, G_FL)[t]);
+                fence_async_smem();
+                sync_so();
+                if (xleader) {
+                    mbar_arrive(&bars[B_PR]);
+                    if (i == j) mbar_arrive(&bars[B_INV + ((c * NSUB + j) & 1)]);   // the sub-block's 1 / denominators
                 }
+                RS_TRACE(xleader && tt == 0, c, 17);
             }
-            fence_async_smem();
-            tc_fence_before();
-            sync_so();
-            if (xleader) {
-                mbar_arrive(&bars[B_PR]);
-                mbar_arrive(&bars[B_SE]);
-                mbar_arrive(&bars[B_GE0 + gb]);
-            }
-            RS_TRACE(xleader, c, 17);
+            if (!ok) break;
+            sync_so();                                       // G_INV written before the chunk's gates are released
+            if (xleader) mbar_arrive(&bars[B_GE + gb]);
         }
         tc_fence_before();
     }
@@ -839,10 +919,11 @@ segment_output_rs_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
     }
 }
 
-// DH 512: the two key halves' numerators and denominators are summed and the
-// output formed, h = sigma(o) * f_t (N_0 + N_1) / max(|d_0 + d_1|, e^{-m_t});
-// f_t is the row factor (g_t, or 1 in a wide chunk's rows whose retrieval was
-// dropped).  An HBM stream: four value columns of one token per thread.
+// Split key columns (DH 512, and DH 256 at chunk 256): the two halves'
+// numerators and denominators are summed and the output formed,
+// h = sigma(o) * f_t (N_0 + N_1) / max(|d_0 + d_1|, e^{-m_t}); f_t is the row
+// factor (g_t, or 1 in a wide chunk's rows whose retrieval was dropped).  An
+// HBM stream: four value columns of one token per thread.
 __global__ void __launch_bounds__(256)
 combine_keysplit_kernel(const float *__restrict__ part, const float *__restrict__ dpart,
                         const float2 *__restrict__ tokrec, const float *__restrict__ o_pre,
@@ -864,9 +945,9 @@ combine_keysplit_kernel(const float *__restrict__ part, const float *__restrict_
     }
 }
 
-template <int D>
+template <int D, int NSUB>
 cudaError_t launch_rs_t(const FwdArgs &a, const FwdPlan &p, cudaStream_t st) {
-    using Cfg = RsCfg<D>;
+    using Cfg = RsCfg<D, NSUB>;
     CUtensorMap mq, mk, mv, mo;
     if (!make_map_bf16(&mq, a.q, p.BH, p.S, D) || !make_map_bf16(&mk, a.k, p.BH, p.S, D) ||
         !make_map_bf16(&mv, a.v, p.BH, p.S, D) || !make_map_f32_rows(&mo, a.o_pre, p.BH, p.S, D, Cfg::RV, 64))
@@ -876,14 +957,14 @@ cudaError_t launch_rs_t(const FwdArgs &a, const FwdPlan &p, cudaStream_t st) {
     float *ws = (float *)a.workspace;
     // at least 116 KB so that one CTA runs per SM: each allocates all 512 TMEM columns
     const int sm = Cfg::kBytes > 118784 ? Cfg::kBytes : 118784;
-    e = cudaFuncSetAttribute(segment_output_rs_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
+    e = cudaFuncSetAttribute(segment_output_rs_kernel<D, NSUB>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
     if (e != cudaSuccess) return e;
     float *part = Cfg::KS > 1 ? ws + p.off_part : nullptr;
     float *dpart = Cfg::KS > 1 ? ws + p.off_dpart : nullptr;
     float2 *tokrec = Cfg::KS > 1 ? (float2 *)(ws + p.off_tok) : nullptr;
     {
         KernelTimer timer("segment_output_rs", st);
-        segment_output_rs_kernel<D><<<dim3((D / Cfg::RV) * Cfg::KS, p.P, p.BH), kRsThreads, sm, st>>>(
+        segment_output_rs_kernel<D, NSUB><<<dim3((D / Cfg::RV) * Cfg::KS, p.P, p.BH), kRsThreads, sm, st>>>(
             mq, mk, mv, mo, (__nv_bfloat16 *)a.h, a.i_pre, a.C0, a.n0, a.m0, a.C_out, a.n_out, a.m_out,
             ws + p.off_bcum, ws + p.off_pmax, (const float2 *)(ws + p.off_cstat), (const float2 *)(ws + p.off_sstat),
             ws + p.off_summ, part, dpart, tokrec, a.status, p.S, p.nchunks, p.P, p.cps);
@@ -901,6 +982,17 @@ cudaError_t launch_rs_t(const FwdArgs &a, const FwdPlan &p, cudaStream_t st) {
     return cudaSuccess;
 }
 
+template <int NSUB>
+cudaError_t launch_rs_nsub(const FwdArgs &a, const FwdPlan &p, cudaStream_t st) {
+    switch (p.DH) {
+        case 64: return launch_rs_t<64, NSUB>(a, p, st);
+        case 128: return launch_rs_t<128, NSUB>(a, p, st);
+        case 256: return launch_rs_t<256, NSUB>(a, p, st);
+        case 512: return launch_rs_t<512, NSUB < 4 ? NSUB : 2>(a, p, st);   // DH 512 takes chunks 64 and 128
+    }
+    return cudaErrorInvalidValue;
+}
+
 }  // namespace
 
 #ifdef XLSTM_RS_TRACE
@@ -909,17 +1001,22 @@ extern "C" int xlstm_debug_set_rs_trace(void *buf) {
 }
 #endif
 
-bool rs_path_supports(int DH, int L) { return L == kL && (DH == 64 || DH == 128 || DH == 256 || DH == 512); }
+bool rs_path_supports(int DH, int L) {
+    if (DH != 64 && DH != 128 && DH != 256 && DH != 512) return false;
+    if (L == 64 || L == 128) return true;
+    return L == 256 && DH <= 256;
+}
+
+int rs_key_splits(int DH, int L) { return DH > 256 || (DH == 256 && L == 256) ? 2 : 1; }
 
 cudaError_t launch_fwd_rs(const FwdArgs &a, const FwdPlan &p, cudaStream_t st) {
     if (!a.bf16 || !rs_path_supports(p.DH, p.L)) return cudaErrorInvalidValue;
     cudaError_t e = launch_gate_prologue(a, p, st);
     if (e != cudaSuccess) return e;
-    switch (p.DH) {
-        case 64: return launch_rs_t<64>(a, p, st);
-        case 128: return launch_rs_t<128>(a, p, st);
-        case 256: return launch_rs_t<256>(a, p, st);
-        case 512: return launch_rs_t<512>(a, p, st);
+    switch (p.L) {
+        case 64: return launch_rs_nsub<1>(a, p, st);
+        case 128: return launch_rs_nsub<2>(a, p, st);
+        case 256: return launch_rs_nsub<4>(a, p, st);
     }
     return cudaErrorInvalidValue;
 }

@@ -1007,7 +1007,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 segment_summary_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v,
                           const float *__restrict__ i_pre, const float *__restrict__ bcum,
                           const float2 *__restrict__ cstat, float2 *__restrict__ sstat, float *__restrict__ summ,
-                          unsigned int *status, int S, int nchunks, int P, int cps) {
+                          unsigned int *status, int S, int nchunks, int P, int cps, int L) {
     using Lay = SumLayout<D>;
     constexpr int NS = Lay::kStages;
     // value rows of this CTA: 128, or all DH when DH < 128 (the MMAs keep M = 128;
@@ -1029,6 +1029,10 @@ segment_summary_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __gri
     const int i0 = tile * kRows, k0 = kh * KC;
     const int c0 = g * cps;
     const int nch = min(nchunks, c0 + cps) - c0;
+    // 64-token tiles of the segment; tile tl lies in chunk tl / nsub (chunks of L tokens)
+    const int nsub = L / kL;
+    const int tseg = c0 * L;
+    const int ntl = (min(S, (c0 + nch) * L) - tseg + kL - 1) / kL;
     const size_t tok0 = (size_t)bh * S;
     const float inv_sqrt_d = rsqrtf((float)D);
 
@@ -1078,8 +1082,8 @@ segment_summary_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __gri
             tma_prefetch_desc(&map_k);
             tma_prefetch_desc(&map_v);
             int issued[NS] = {};
-            for (int c = 0; c < nch; ++c) {
-                const int slot = c % NS, t0 = (c0 + c) * kL;
+            for (int c = 0; c < ntl; ++c) {
+                const int slot = c % NS, t0 = tseg + c * kL;
                 if (c >= NS && !mbar_wait(&b_free[slot], ((c / NS) - 1) & 1, abort_flag, status)) break;
                 uint8_t *base = smem + slot * Lay::kSlot;
                 mbar_arrive_expect_tx(&b_full[slot], kL * KC * 2 + kL * kVBlocks * 64 * 2);
@@ -1095,7 +1099,7 @@ segment_summary_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __gri
         }
     } else if (warp == 1) {
         if (lane == 0) {
-            for (int c = 0; c < nch; ++c) {
+            for (int c = 0; c < ntl; ++c) {
                 const int slot = c % NS;
                 if (!mbar_wait(&b_ready[slot], (c / NS) & 1, abort_flag, status)) break;
                 tc_fence_after();
@@ -1122,16 +1126,16 @@ segment_summary_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __gri
         const int ct = tid - 64, q4 = warp & 3;
         bool ok = true;
         float pre_i = 0.f, pre_b = 0.f;                   // gates of the next chunk, in flight
-        if (nch > 0 && ct < kL && c0 * kL + ct < S) {
-            pre_i = i_pre[tok0 + c0 * kL + ct];
-            pre_b = bcum[tok0 + c0 * kL + ct];
+        if (ntl > 0 && ct < kL && tseg + ct < S) {
+            pre_i = i_pre[tok0 + tseg + ct];
+            pre_b = bcum[tok0 + tseg + ct];
         }
-        for (int c = 0; c < nch; ++c) {
-            const int slot = c % NS, t0 = (c0 + c) * kL, Lc = min(kL, S - t0);
+        for (int c = 0; c < ntl; ++c) {
+            const int slot = c % NS, t0 = tseg + c * kL, Lc = min(kL, S - t0);
             if (ct < kL)
-                fw[ct] = ct < Lc ? expf(pre_i - pre_b + tabE[c] - mloc) * inv_sqrt_d : 0.f;
+                fw[ct] = ct < Lc ? expf(pre_i - pre_b + tabE[c / nsub] - mloc) * inv_sqrt_d : 0.f;
             pre_i = pre_b = 0.f;
-            if (c + 1 < nch && ct < kL && t0 + kL + ct < S) {
+            if (c + 1 < ntl && ct < kL && t0 + kL + ct < S) {
                 pre_i = i_pre[tok0 + t0 + kL + ct];
                 pre_b = bcum[tok0 + t0 + kL + ct];
             }
@@ -1224,7 +1228,7 @@ cudaError_t launch_summaries_t(const FwdArgs &a, const FwdPlan &p, cudaStream_t 
     {
         KernelTimer timer("segment_summary_tc", st);
         segment_summary_tc_kernel<D><<<dim3(SumLayout<D>::NT * SumLayout<D>::KS, p.P - 1, p.BH), kThreads, sm, st>>>(
-            mk, mv, a.i_pre, bcum, cstat, sstat, summ, a.status, p.S, p.nchunks, p.P, p.cps);
+            mk, mv, a.i_pre, bcum, cstat, sstat, summ, a.status, p.S, p.nchunks, p.P, p.cps, p.L);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     KernelTimer timer("segment_scan", st);

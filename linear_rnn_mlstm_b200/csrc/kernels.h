@@ -45,8 +45,11 @@ cudaError_t launch_segment_summaries(const FwdArgs &a, const FwdPlan &p, cudaStr
 cudaError_t launch_fwd_simt(const FwdArgs &a, const FwdPlan &p, cudaStream_t st);
 cudaError_t launch_fwd_tensor(const FwdArgs &a, const FwdPlan &p, cudaStream_t st);
 bool tensor_path_supports(int DH, int L);
-// Register-state tensor-core forward (fwd_rs.cu): bf16, chunk 64, DH 64 / 128 / 256.
+// Register-state tensor-core forward (fwd_rs.cu): bf16, DH 64 / 128 / 256 / 512,
+// chunk 64 / 128 / 256 (DH 512: 64 / 128); rs_key_splits = CTAs sharing one
+// value tile's key columns (their partial outputs are combined afterwards).
 bool rs_path_supports(int DH, int L);
+int rs_key_splits(int DH, int L);
 cudaError_t launch_fwd_rs(const FwdArgs &a, const FwdPlan &p, cudaStream_t st);
 int tensor_path_max_chunks_per_segment();
 cudaError_t launch_state_passthrough(const FwdArgs &a, int BH, int DH, cudaStream_t st);

@@ -29,13 +29,13 @@ pytestmark = pytest.mark.gpu
 FAMILIES = [xb.PATH_TENSOR_RS, xb.PATH_TENSOR_TMEM]
 
 
-def _check(inp, fgate, seg, C0=None, n0=None, m0=None, families=FAMILIES):
+def _check(inp, fgate, seg, C0=None, n0=None, m0=None, families=FAMILIES, chunk=64):
     hr, Cr, nr, mr = oracle_fwd(inp, fgate, C0, n0, m0)
     DH = inp["q"].shape[-1]
     for fam in families:
-        if fam == xb.PATH_TENSOR_TMEM and DH not in (128, 256):
+        if fam == xb.PATH_TENSOR_TMEM and (DH not in (128, 256) or chunk != 64):
             continue
-        h, C, n, m = gpu_fwd(inp, 64, fgate, fam, seg, C0, n0, m0)
+        h, C, n, m = gpu_fwd(inp, chunk, fgate, fam, seg, C0, n0, m0)
         assert_close(h, hr, "bf16", what=f"h (family {fam})")
         assert errors(C, Cr)[1] <= STATE_REL_L2 and errors(n, nr)[1] <= STATE_REL_L2
         assert np.max(np.abs(m - mr)) <= STATE_M_ABS
@@ -109,7 +109,7 @@ def test_tensor_path_initial_state():
 
 
 @pytest.mark.parametrize("dtype,DH,chunk,fam", [("f32", 128, 64, xb.PATH_TENSOR), ("bf16", 48, 64, xb.PATH_TENSOR),
-                                                ("bf16", 512, 128, xb.PATH_TENSOR),
+                                                ("bf16", 512, 256, xb.PATH_TENSOR),
                                                 ("bf16", 64, 64, xb.PATH_TENSOR_TMEM),
                                                 ("bf16", 128, 128, xb.PATH_TENSOR_TMEM)])
 def test_tensor_path_refuses_unsupported(dtype, DH, chunk, fam):
@@ -119,3 +119,44 @@ def test_tensor_path_refuses_unsupported(dtype, DH, chunk, fam):
         xb.mlstm_fwd(d["q"], d["k"], d["v"], d["i_pre"], d["f_pre"], d["o_pre"], chunk=chunk,
                      path=fam)
     assert err.value.status == xb.ERR_UNSUPPORTED
+
+
+# Chunks of 128 and 256 tokens: the state is carried across chunks only and the
+# intra-chunk quadratic form spans the whole chunk (sub-block tiles below the
+# diagonal, masked tiles on it); DH 256 at chunk 256 and DH 512 split the key
+# columns over two CTAs.
+CHUNK_CASES = [
+    # (B, NH, S, DH, fgate, segments, chunk)
+    (1, 2, 300, 64, "sigmoid", 0, 128),
+    (2, 2, 700, 64, "exp", 3, 256),
+    (1, 2, 517, 128, "sigmoid", 1, 128),
+    (1, 2, 1000, 128, "exp", 3, 256),
+    (2, 1, 640, 256, "sigmoid", 0, 128),
+    (1, 2, 777, 256, "sigmoid", 2, 256),
+    (1, 1, 129, 256, "exp", 0, 256),
+    (1, 2, 300, 512, "exp", 0, 128),
+    (2, 1, 517, 512, "sigmoid", 3, 128),
+]
+
+
+@pytest.mark.parametrize("case", CHUNK_CASES, ids=lambda c: "x".join(map(str, c)))
+def test_tensor_path_long_chunks(case):
+    B, NH, S, DH, fgate, seg, chunk = case
+    base = syn.BLOCK if fgate == "exp" else syn.SMALL
+    w = syn.custom("tc_chunk", B, NH, S, DH, base, dtype="bf16", seed=S + DH + chunk)
+    _check(syn.fwd_inputs(w), fgate, seg, chunk=chunk)
+
+
+@pytest.mark.parametrize("DH,chunk", [(128, 256), (256, 128), (512, 128)])
+def test_tensor_path_long_chunks_wide_and_state(DH, chunk):
+    # wide chunks (input terms spanning e^250 inside one chunk) and a given
+    # initial state, at the longer chunk sizes
+    w = syn.custom("tc_chunk_wide", 1, 2, 900, DH, syn.SMALL, dtype="bf16", seed=11 + chunk,
+                   f_mu=-4.0, f_sd=1.0, i_sd=3.0)
+    _check(syn.fwd_inputs(w), "sigmoid", 0, chunk=chunk)
+    w = syn.custom("tc_chunk_init", 2, 2, 300, DH, syn.SMALL, dtype="bf16", seed=3 + chunk)
+    g = torch.Generator().manual_seed(17)
+    C0 = torch.randn(2, 2, DH, DH, generator=g) * 0.1
+    n0 = torch.randn(2, 2, DH, generator=g) * 0.1
+    m0 = torch.randn(2, 2, generator=g)
+    _check(syn.fwd_inputs(w), "sigmoid", 2, C0, n0, m0, chunk=chunk)
