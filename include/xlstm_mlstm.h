@@ -61,17 +61,21 @@ typedef enum { XLSTM_FGATE_SIGMOID = 0, XLSTM_FGATE_EXP = 1 } xlstm_fgate;
 typedef enum { XLSTM_OGATE_SILU = 0, XLSTM_OGATE_SIGMOID = 1 } xlstm_ogate;
 
 /* Kernel family for the forward.  AUTO picks the tensor-core (tcgen05) kernels
- * for bf16 inputs where they apply (chunk 64 and DH 64, 128 or 256), and the
- * fp32 SIMT kernels for every other case.  SIMT forces the fp32-arithmetic
- * kernels for any supported arguments (a second, independent path the tests
- * compare against).  TENSOR forces the tensor-core kernels; for arguments they
- * do not take the call returns XLSTM_ERR_UNSUPPORTED and launches nothing.
- * Two tensor-core output kernels exist: one keeps the state in tensor memory
- * and retrieves with tf32 operands (TENSOR_TMEM: DH 128 or 256, chunk 64;
- * about 11 significant bits in the retrieval), the other keeps the state in
- * fp32 registers and retrieves with two bf16 parts (TENSOR_RS: DH 64, 128 or
- * 256, chunk 64; 15 to 16 bits).  TENSOR takes TENSOR_TMEM where it applies
- * (it is the faster at DH 128 / 256) and TENSOR_RS elsewhere. */
+ * for bf16 inputs where they apply (chunk 64 or 128 with DH 64, 128, 256 or
+ * 512; chunk 256 with DH 64, 128 or 256), and the fp32 SIMT kernels for every
+ * other case.  SIMT forces the fp32-arithmetic kernels for any supported
+ * arguments (a second, independent path the tests compare against).  TENSOR
+ * forces the tensor-core kernels; for arguments they do not take the call
+ * returns XLSTM_ERR_UNSUPPORTED and launches nothing.  Two tensor-core output
+ * kernels exist: one keeps the state in tensor memory and retrieves with tf32
+ * operands (TENSOR_TMEM: DH 128 or 256, chunk 64; about 11 significant bits
+ * in the retrieval), the other keeps the state in fp32 registers and
+ * retrieves with two bf16 parts (TENSOR_RS: every tensor-core case above; 15
+ * to 16 bits).  TENSOR_RS splits the key columns of the state over two CTAs
+ * at DH 512, and at DH 256 with chunk 256, and a combining kernel adds the two
+ * partial numerators and denominators.  TENSOR takes TENSOR_TMEM where it
+ * applies (it is the faster at DH 128 / 256, chunk 64) and TENSOR_RS
+ * elsewhere. */
 typedef enum {
     XLSTM_PATH_AUTO = 0, XLSTM_PATH_SIMT = 1, XLSTM_PATH_TENSOR = 2, XLSTM_PATH_TENSOR_TMEM = 3,
     XLSTM_PATH_TENSOR_RS = 4
@@ -137,8 +141,8 @@ xlstm_status xlstm_mlstm_fwd(const void *q, const void *k, const void *v,
 
 /*
  * Which kernel family xlstm_mlstm_fwd_ex would run for these arguments
- * (written to *path: XLSTM_PATH_SIMT or XLSTM_PATH_TENSOR), resolving
- * XLSTM_PATH_AUTO; same validation and error codes as the forward for DH,
+ * (written to *path: XLSTM_PATH_SIMT or XLSTM_PATH_TENSOR after resolving
+ * XLSTM_PATH_AUTO; a forced family is returned as given when it applies); same validation and error codes as the forward for DH,
  * chunk, dt and the options.  The paper has no counterpart: this lets a caller
  * (and the tests) know whether the fp32 CUDA-core kernels or the tcgen05
  * tensor-core kernels will compute the result.  Pure host function.
