@@ -61,8 +61,16 @@ __device__ unsigned long long *g_tc_trace = nullptr;
             g_tc_trace[(cta_ * kMaxCps + (c)) * 32 + (slot)] = clock64();                          \
         }                                                                                          \
     } while (0)
+#define TC_TRACE_NS(cond, slot)                                                                    \
+    do {                                                                                           \
+        if (g_tc_trace && (cond)) {                                                                \
+            const size_t cta_ = ((size_t)blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x; \
+            g_tc_trace[cta_ * kMaxCps * 32 + (slot)] = globaltimer_ns();                           \
+        }                                                                                          \
+    } while (0)
 #else
 #define TC_TRACE(cond, c, slot) do { } while (0)
+#define TC_TRACE_NS(cond, slot) do { } while (0)
 #endif
 
 // A bounded wait taken by all 128 compute threads, with a group-uniform result.
@@ -92,14 +100,14 @@ struct OutLayout {
     static constexpr int kQt = kV + 16384;                // Q as fp32 (tf32 operand), K-major: D/32 blocks x 8 KB
     static constexpr int kP = kQt + D * 256;              // masked scores, high bf16 part, K-major: 64 x 128 B
     static constexpr int kPl = kP + 8192;                 // masked scores, low bf16 part
-    static constexpr int kHs = kPl + 8192;                // h tile for the TMA store: 2 blocks x 64 rows x 128 B
-    static constexpr int kF = kHs + 16384;                // float arrays (see kernel)
+    static constexpr int kO = kPl + 8192;                 // o-gate tile: 32 tokens x 128 value rows fp32 (TMA)
+    static constexpr int kF = kO + 16384;                 // float arrays (see kernel)
     static constexpr int kNF = 16 * 64;
     static constexpr int kTab = kF + kNF * 4;             // per-chunk tables
     static constexpr int kBar = kTab + 5 * kMaxCps * 4;
     static constexpr int kNumBars = 40;
-    static constexpr int kMisc = kBar + kNumBars * 8;     // tmem base, abort flag
-    static constexpr int kEnd = kMisc + 16;
+    static constexpr int kMisc = kBar + kNumBars * 8;     // tmem base, abort flag, o-tile counters
+    static constexpr int kEnd = kMisc + 32;
     static constexpr int kBytes = kEnd + 1024;            // slack for 1024-byte alignment
 };
 
@@ -111,7 +119,8 @@ enum {
     B_VHAT_READY, B_QT_READY, B_QT_FREE, B_S_FULL, B_S_FREE, B_P_READY, B_P_FREE,
     B_H_FULL0, B_H_FULL1, B_H_FREE0, B_H_FREE1, B_NROW_READY0, B_NROW_READY1, B_RESC_DONE, B_DONE,
     B_GATES_READY0, B_GATES_READY1, B_GATES_FREE0, B_GATES_FREE1,
-    B_FINV_READY0, B_FINV_READY1, B_FINV_FREE0, B_FINV_FREE1, B_INTRA_DONE, B_STATE_READY, B_NUM
+    B_FINV_READY0, B_FINV_READY1, B_FINV_FREE0, B_FINV_FREE1, B_INTRA_DONE, B_STATE_READY,
+    B_O_FULL0, B_O_FULL1, B_NUM
 };
 static_assert(B_NUM <= OutLayout<128>::kNumBars, "barrier slots");
 // Every barrier is waited by parity, so no producer may complete a barrier twice
@@ -133,12 +142,6 @@ static_assert(B_NUM <= OutLayout<128>::kNumBars, "barrier slots");
 struct ChunkTab {
     float *mprev, *lamret, *resc, *lnupd, *wide;
 };
-
-__device__ __forceinline__ float ldg_nc_early(const float *p) {
-    float v;
-    asm volatile("ld.global.nc.f32 %0, [%1];" : "=f"(v) : "l"(p));   // volatile: issued where written
-    return v;
-}
 
 // Warp roles: 0 TMA, 1 MMA (and TMEM owner), 2-5 operand group (gates, Q as
 // fp32, normaliser chain, w^ V, rescale, final state), 6-9 score group (masked
@@ -164,8 +167,8 @@ __device__ __forceinline__ bool wait_out(uint64_t *bar, uint32_t parity, volatil
 template <int D>
 __global__ void __launch_bounds__(kOutThreads, 1)
 segment_output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
-                         const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_h,
-                         const __grid_constant__ CUtensorMap map_o,
+                         const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_o,
+                         __nv_bfloat16 *__restrict__ h_out,
                          const float *__restrict__ i_pre, const float *__restrict__ o_pre,
                          const float *__restrict__ C0, const float *__restrict__ n0, const float *__restrict__ m0,
                          float *__restrict__ C_out, float *__restrict__ n_out, float *__restrict__ m_out,
@@ -182,7 +185,7 @@ segment_output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
     uint8_t *sQt = smem + Lay::kQt;
     uint8_t *sP = smem + Lay::kP;
     uint8_t *sPl = smem + Lay::kPl;
-    uint8_t *sHs = smem + Lay::kHs;
+    const float *sO = reinterpret_cast<const float *>(smem + Lay::kO);
     // per-token arrays, [2][64] by chunk parity, written by the operand group
     float *fm = reinterpret_cast<float *>(smem + Lay::kF);   // m_t
     float *fg = fm + 128;                                    // g_t = e^{b_t + m_prev - m_t}
@@ -201,6 +204,9 @@ segment_output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Lay::kBar);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + Lay::kMisc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + Lay::kMisc + 4);
+    // o-gate tiles issued into / taken from the shared tile, per pass (hq = 0, 1)
+    int *o_issued = reinterpret_cast<int *>(smem + Lay::kMisc + 8);
+    int *o_taken = reinterpret_cast<int *>(smem + Lay::kMisc + 16);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int tile = blockIdx.x, g = blockIdx.y, bh = blockIdx.z;
@@ -219,6 +225,7 @@ segment_output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
     const int xt = tid - 320;                                // output-group thread 0..127
 
     // ------------------------------------------------------------ set-up
+    TC_TRACE_NS(tid == 0, 30);
     if (tid == 0) {
         for (int i = 0; i < B_NUM; ++i) {
             const bool two = i == B_Q_FREE || i == B_H_FREE0 || i == B_H_FREE1 || i == B_FINV_FREE0 ||
@@ -226,6 +233,7 @@ segment_output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
             mbar_init(&bars[i], two ? 2 : 1);
         }
         *abort_flag = 0;
+        o_issued[0] = o_issued[1] = o_taken[0] = o_taken[1] = 0;
         fence_mbar_init();
     }
     if (warp == 1) {
@@ -316,14 +324,34 @@ segment_output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
     const uint32_t idesc_I = idesc_f32acc(kFmtBF16, kFmtBF16, true, false, 128, 64);
     const uint32_t idesc_U = idesc_f32acc(kFmtBF16, kFmtBF16, true, true, 128, D);
 
+    // The o gates of one epilogue pass reach shared memory by TMA, one tile of
+    // 32 tokens x 128 value rows at a time: the output group takes tokens 0-31 of
+    // each chunk (hq = 0), the score group tokens 32-63 (hq = 1).  Whichever group
+    // has just read the tile issues the load of the next one, so the epilogue
+    // threads never hold a global load across a barrier or an arrival.
+    auto issue_o = [&](int c, int hq) {
+        uint64_t *bar = &bars[B_O_FULL0 + hq];
+        mbar_arrive_expect_tx(bar, 32 * kRows * 4);
+        tma_load_3d(const_cast<float *>(sO), &map_o, bar, i0, (c0 + c) * kL + 32 * hq, bh);
+        ++o_issued[hq];
+    };
+    // This thread's 32 gates of the tile in shared memory (thread = value row i;
+    // a warp reads 32 consecutive floats per token).
+    auto read_gates = [&](float (&og)[32]) {
+        const int i = 32 * q4 + lane;
+#pragma unroll
+        for (int kk = 0; kk < 32; ++kk) og[kk] = sO[kk * kRows + i];
+    };
     // One epilogue pass: h for tokens [32 hq, 32 hq + 32) of chunk c, from the H~
     // accumulator (thread = value row i = TMEM lane), the gates `og` of those
-    // tokens and the per-token factors F_t / (2 den_t), into the shared h tile.
-    // Taken by the output group (hq = 0) and the score group (hq = 1).
+    // tokens and the per-token factors F_t / (2 den_t); each h element is stored
+    // straight to global memory (a warp writes 64 contiguous bytes per token).
     auto epilogue_pass = [&](int c, int hq, const float (&og)[32]) {
         const int hb = c & 1;
         const int i = 32 * q4 + lane;
-        uint8_t *hs = sHs + (i >> 6) * 8192 + (i & 63) * 2 + 32 * hq * 128;
+        const int tb = (c0 + c) * kL + 32 * hq;
+        const int n = min(32, S - tb);
+        __nv_bfloat16 *hrow = h_out + (tok0 + tb) * D + i0 + i;
         uint32_t r[32];
         tmem_ld16(t_H0 + 64 * hb + lane_addr + 32 * hq, *reinterpret_cast<uint32_t(*)[16]>(&r[0]));
         tmem_ld16(t_H0 + 64 * hb + lane_addr + 32 * hq + 16, *reinterpret_cast<uint32_t(*)[16]>(&r[16]));
@@ -333,26 +361,12 @@ segment_output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
         for (int kk = 0; kk < 32; ++kk) {
             // sigma(o) = (1 + tanh(o / 2)) / 2, the 1/2 folded into inv
             const float hv = __uint_as_float(r[kk]) * inv[kk];
-            *reinterpret_cast<__nv_bfloat16 *>(hs + kk * 128) = __float2bfloat16_rn(fmaf(hv, tanh_approx(0.5f * og[kk]), hv));
+            if (kk < n) hrow[(size_t)kk * D] = __float2bfloat16_rn(fmaf(hv, tanh_approx(0.5f * og[kk]), hv));
         }
     };
-    // The gates of tokens [32 hq, 32 hq + 32) of chunk c, for this thread's value row.
-    auto load_gates = [&](int c, int hq, float (&og)[32]) {
-        const int i = 32 * q4 + lane;
-        const int tb = (c0 + c) * kL + 32 * hq;
-        const int n = min(32, S - tb);
-#pragma unroll
-        for (int kk = 0; kk < 32; ++kk)
-            og[kk] = kk < n ? ldg_nc_early(o_pre + (tok0 + tb + kk) * D + i0 + i) : 0.f;
-    };
-    // After a pass: the pass's half of the h tile leaves by TMA store (issued by
-    // the group's leader), and the group's share of H[hb] and finv[hb] is released.
-    auto finish_pass = [&](int c, int hq, bool leader) {
+    // After a pass the group's share of H[hb] and finv[hb] is released.
+    auto finish_pass = [&](int c, bool leader) {
         if (leader) {
-            const int t0 = (c0 + c) * kL;
-            tma_store_3d(&map_h, sHs + 32 * hq * 128, i0, t0 + 32 * hq, bh);
-            tma_store_3d(&map_h, sHs + 8192 + 32 * hq * 128, i0 + 64, t0 + 32 * hq, bh);
-            bulk_commit();
             mbar_arrive(&bars[B_H_FREE0 + (c & 1)]);
             mbar_arrive(&bars[B_FINV_FREE0 + (c & 1)]);
         }
@@ -376,6 +390,7 @@ segment_output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
                 tma_prefetch_l2_3d(&map_v, i0, t0, bh);
                 tma_prefetch_l2_3d(&map_v, i0 + 64, t0, bh);
                 tma_prefetch_l2_3d(&map_o, i0, t0, bh);
+                tma_prefetch_l2_3d(&map_o, i0, t0 + 32, bh);
             };
             for (int c = 0; c < min(nch, 2); ++c) prefetch(c);
             int issued_q = 0, issued_k[2] = {0, 0}, issued_v = 0;
@@ -442,7 +457,9 @@ segment_output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
                     if (!mbar_wait(&bars[B_RESC_DONE], nresc & 1, abort_flag, status)) { ok = false; break; }
                     ++nresc;
                 }
+                TC_TRACE(true, c, 25);
                 if (!mbar_wait(&bars[B_QT_READY], c & 1, abort_flag, status)) { ok = false; break; }
+                TC_TRACE(true, c, 26);
                 if (c == 0 && !mbar_wait(&bars[B_STATE_READY], 0, abort_flag, status)) { ok = false; break; }
                 if (c >= 2 && !mbar_wait(&bars[B_H_FREE0 + hb], ((c >> 1) - 1) & 1, abort_flag, status)) {
                     ok = false;
@@ -462,6 +479,7 @@ segment_output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
                     }
                     mma_commit(&bars[B_QT_FREE]);
                 }
+                TC_TRACE(true, c, 27);
                 auto update = [&]() -> bool {   // state update: Cs += (w^ V)^T K
                     if (!mbar_wait(&bars[B_VHAT_READY], c & 1, abort_flag, status)) return false;
                     tc_fence_after();
@@ -508,6 +526,7 @@ segment_output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
                     tc_fence_after();
                     TC_TRACE(true, c, 14);
                     issue_S(c + 1);
+                    TC_TRACE(true, c, 24);
                 }
             }
             mma_commit(&bars[B_DONE]);
@@ -751,22 +770,25 @@ segment_output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
         bool ok = true;
         const int t = 16 * q4 + (lane & 15);
         const int hh = lane >> 4;                             // column half of this lane
-        float og[32];                                         // gates of the pending epilogue pass
-        if (nch > 0) load_gates(0, 1, og);
         auto pass1 = [&](int cp) -> bool {                    // epilogue of tokens 32-63 of chunk cp
-            if (!wait_sco(&bars[B_H_FULL0 + (cp & 1)], (cp >> 1) & 1, abort_flag, status)) return false;
-            if (st_ == 0) bulk_wait_read_all();               // this half of the h tile is free again
-            sync_sco();
+            if (!wait_sco(&bars[B_H_FULL0 + (cp & 1)], (cp >> 1) & 1, abort_flag, status) ||
+                !wait_sco(&bars[B_O_FULL1], cp & 1, abort_flag, status)) return false;
+            float og[32];
+            read_gates(og);
+            sync_sco();                                       // every thread has its gates: the tile is free
+            if (st_ == 0) {
+                ++o_taken[1];
+                if (cp + 1 < nch) issue_o(cp + 1, 0);         // tokens 0-31 of the next chunk
+            }
             __syncwarp();
             tc_fence_after();
             TC_TRACE(st_ == 0, cp, 22);
             epilogue_pass(cp, 1, og);
             TC_TRACE(st_ == 0, cp, 23);
-            if (cp + 1 < nch) load_gates(cp + 1, 1, og);
-            fence_async_smem();
             tc_fence_before();
             sync_sco();
-            finish_pass(cp, 1, st_ == 0);
+            finish_pass(cp, st_ == 0);
+            TC_TRACE(st_ == 0, cp, 28);
             return true;
         };
         for (int c = 0; ok && c < nch; ++c) {
@@ -868,13 +890,13 @@ segment_output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
             if (c >= 1 && !pass1(c - 1)) { ok = false; break; }
         }
         if (ok && nch > 0) ok = pass1(nch - 1);
-        if (st_ == 0) bulk_wait_all();                       // h is in global memory before exit
     } else if (is_out) {
         // --------------------------------------------------------- output group
         // Thread = value row i of H^T (TMEM lane); h for tokens 0-31 of each chunk
         // goes through the shared h tile and leaves by TMA store, so the global
         // writes are whole 128-byte rows.  The gates are loaded a chunk ahead.
         bool ok = true;
+        if (xt == 0 && nch > 0) issue_o(0, 0);             // gates of tokens 0-31 of chunk 0
         {   // Incoming state into TMEM, while the other groups start on chunk 0: the
             // initial state for segment 0, else the state at the end of segment g - 1,
             // which segment_scan_kernel left in summary slot g - 1.
@@ -905,31 +927,40 @@ segment_output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
             sync_out();
             if (xt == 0) mbar_arrive(&bars[B_STATE_READY]);
         }
-        float og[32];
-        if (nch > 0) load_gates(0, 0, og);
         for (int c = 0; ok && c < nch; ++c) {
             const int hb = c & 1;
             if (!wait_out(&bars[B_H_FULL0 + hb], (c >> 1) & 1, abort_flag, status) ||
-                !wait_out(&bars[B_FINV_READY0 + hb], (c >> 1) & 1, abort_flag, status)) { ok = false; break; }
+                !wait_out(&bars[B_FINV_READY0 + hb], (c >> 1) & 1, abort_flag, status) ||
+                !wait_out(&bars[B_O_FULL0], c & 1, abort_flag, status)) { ok = false; break; }
             TC_TRACE(xt == 0, c, 10);
-            if (xt == 0) bulk_wait_read_all();               // this half of the h tile is free again
-            sync_out();
+            float og[32];
+            read_gates(og);
+            sync_out();                                      // every thread has its gates: the tile is free
+            if (xt == 0) {
+                ++o_taken[0];
+                issue_o(c, 1);                               // tokens 32-63 of this chunk
+            }
             __syncwarp();
             tc_fence_after();
             TC_TRACE(xt == 0, c, 20);
             epilogue_pass(c, 0, og);
             TC_TRACE(xt == 0, c, 21);
-            if (c + 1 < nch) load_gates(c + 1, 0, og);
-            fence_async_smem();
             tc_fence_before();
             sync_out();
-            finish_pass(c, 0, xt == 0);
+            finish_pass(c, xt == 0);
             TC_TRACE(xt == 0, c, 11);
         }
-        if (xt == 0) bulk_wait_all();                        // h is in global memory before exit
         tc_fence_before();
     }
     __syncthreads();
+    TC_TRACE_NS(tid == 0, 31);
+    // never leave an o-gate load in flight into shared memory (a group that gave
+    // up a wait may not have taken the last tile issued for it)
+    if (tid == 0) {
+        for (int hq = 0; hq < 2; ++hq)
+            if (o_issued[hq] > o_taken[hq])
+                mbar_wait(&bars[B_O_FULL0 + hq], (o_issued[hq] - 1) & 1, nullptr, status, 200000000ull);
+    }
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tbase, 512);
@@ -1240,10 +1271,9 @@ cudaError_t launch_summaries_t(const FwdArgs &a, const FwdPlan &p, cudaStream_t 
 
 template <int D>
 cudaError_t launch_tc_t(const FwdArgs &a, const FwdPlan &p, cudaStream_t st) {
-    CUtensorMap mq, mk, mv, mh, mo;
+    CUtensorMap mq, mk, mv, mo;
     if (!make_map_bf16(&mq, a.q, p.BH, p.S, D) || !make_map_bf16(&mk, a.k, p.BH, p.S, D) ||
-        !make_map_bf16(&mv, a.v, p.BH, p.S, D) || !make_map_bf16(&mh, a.h, p.BH, p.S, D, false, 32) ||
-        !make_map_f32_rows(&mo, a.o_pre, p.BH, p.S, D))
+        !make_map_bf16(&mv, a.v, p.BH, p.S, D) || !make_map_f32_rows(&mo, a.o_pre, p.BH, p.S, D, kRows, 32))
         return cudaErrorInvalidValue;
     float *ws = (float *)a.workspace;
     const float *bcum = ws + p.off_bcum;
@@ -1257,7 +1287,7 @@ cudaError_t launch_tc_t(const FwdArgs &a, const FwdPlan &p, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     KernelTimer timer("segment_output_tc", st);
     segment_output_tc_kernel<D><<<dim3(D / kRows, p.P, p.BH), kOutThreads, sm, st>>>(
-        mq, mk, mv, mh, mo, a.i_pre, a.o_pre, a.C0, a.n0, a.m0, a.C_out, a.n_out, a.m_out,
+        mq, mk, mv, mo, (__nv_bfloat16 *)a.h, a.i_pre, a.o_pre, a.C0, a.n0, a.m0, a.C_out, a.n_out, a.m_out,
         bcum, ws + p.off_pmax, cstat, sstat, summ, a.status, p.S, p.nchunks, p.P, p.cps);
     return cudaGetLastError();
 }
