@@ -328,8 +328,11 @@ def main():
     for _ in range(args.warmup):
         run()
     torch.cuda.synchronize(dev)
-    xb.xlstm_profile_begin()
+    # the step time is taken without per-kernel events (they would stand between
+    # the chained launches); a second pass of the same steps gives the breakdown
     ms = time_region(run, args.steps, env, dev)
+    xb.xlstm_profile_begin()
+    time_region(run, args.steps, env, dev)
     _, kt = xb.xlstm_profile_end()
     ms_step = ms / args.steps
     tokens = w.B * w.NH * w.S
@@ -434,15 +437,18 @@ def run_sweep(args, dev, env, peaks, peak_src, with_cpu):
         torch.cuda.synchronize(dev)
         steps = max(5, min(args.steps, 10))
         times = []
-        xb.xlstm_profile_begin()
-        for _ in range(steps):
-            flush.zero_()
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record()
-            run()
-            e1.record()
-            torch.cuda.synchronize(dev)
-            times.append(e0.elapsed_time(e1))
+        for profiled in (False, True):      # step times without per-kernel events, then the breakdown
+            if profiled:
+                xb.xlstm_profile_begin()
+            for _ in range(steps):
+                flush.zero_()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record()
+                run()
+                e1.record()
+                torch.cuda.synchronize(dev)
+                if not profiled:
+                    times.append(e0.elapsed_time(e1))
         _, kt = xb.xlstm_profile_end()
         ms = replicas.max_over_ranks(statistics.median(times), env, dev)
         tokens = w.B * w.NH * w.S

@@ -50,6 +50,19 @@ __device__ __forceinline__ float warp_max(float x) {
     return x;
 }
 
+// ------------------------------------------------ programmatic dependent launch
+// The forward's kernels after the first are launched with the programmatic
+// stream-serialisation attribute, so each may be scheduled while its
+// predecessor on the stream drains.  pdl_wait() returns once the predecessor
+// grid has completed and its writes are visible; every thread calls it before
+// touching memory the predecessor writes (or reads).  pdl_launch_dependents()
+// lets the next kernel be scheduled before this one ends.  Both are no-ops for
+// a kernel launched without the attribute.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // Bits of the device status word (see xlstm_device_status); kernels that can
 // give up a bounded wait get its address as an argument.
 constexpr unsigned int kStatusTimeout = 1u;

@@ -234,6 +234,7 @@ segment_output_rs_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
     const int q4 = warp & 3;
     const uint32_t lane_addr = ((uint32_t)(32 * q4)) << 16;
 
+    pdl_launch_dependents();
     if (tid == 0) {
         for (int i = 0; i < B_NUM; ++i) {
             const bool two = (i >= B_KE && i < B_KE + 4) || (i >= B_GE && i < B_GE + 3);
@@ -260,6 +261,7 @@ segment_output_rs_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
     fence_async_smem();
     __syncthreads();
     tc_fence_after();
+    pdl_wait();                                    // the segment scan's states and the gate statistics
     const uint32_t tbase = *tmem_slot;
     const uint32_t tR = tbase + Cfg::R0, tU = tbase + Cfg::U0, tS = tbase + Cfg::S0, tH = tbase + Cfg::H0;
 
@@ -928,6 +930,7 @@ __global__ void __launch_bounds__(256)
 combine_keysplit_kernel(const float *__restrict__ part, const float *__restrict__ dpart,
                         const float2 *__restrict__ tokrec, const float *__restrict__ o_pre,
                         __nv_bfloat16 *__restrict__ h, size_t tokens, int D) {
+    pdl_wait();                                    // the output kernel's partial sums
     const size_t n4 = tokens * (size_t)(D / 4);
     const size_t stride = (size_t)gridDim.x * blockDim.x;
     for (size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x; e < n4; e += stride) {
@@ -964,20 +967,23 @@ cudaError_t launch_rs_t(const FwdArgs &a, const FwdPlan &p, cudaStream_t st) {
     float2 *tokrec = Cfg::KS > 1 ? (float2 *)(ws + p.off_tok) : nullptr;
     {
         KernelTimer timer("segment_output_rs", st);
-        segment_output_rs_kernel<D, NSUB><<<dim3((D / Cfg::RV) * Cfg::KS, p.P, p.BH), kRsThreads, sm, st>>>(
-            mq, mk, mv, mo, (__nv_bfloat16 *)a.h, a.i_pre, a.C0, a.n0, a.m0, a.C_out, a.n_out, a.m_out,
-            ws + p.off_bcum, ws + p.off_pmax, (const float2 *)(ws + p.off_cstat), (const float2 *)(ws + p.off_sstat),
-            ws + p.off_summ, part, dpart, tokrec, a.status, p.S, p.nchunks, p.P, p.cps);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        e = launch_chained(segment_output_rs_kernel<D, NSUB>, dim3((D / Cfg::RV) * Cfg::KS, p.P, p.BH),
+                           dim3(kRsThreads), sm, st, mq, mk, mv, mo, (__nv_bfloat16 *)a.h, a.i_pre, a.C0, a.n0,
+                           a.m0, a.C_out, a.n_out, a.m_out, (const float *)(ws + p.off_bcum),
+                           (const float *)(ws + p.off_pmax), (const float2 *)(ws + p.off_cstat),
+                           (const float2 *)(ws + p.off_sstat), (const float *)(ws + p.off_summ), part, dpart,
+                           tokrec, a.status, p.S, p.nchunks, p.P, p.cps);
+        if (e != cudaSuccess) return e;
     }
     if (Cfg::KS > 1) {
         KernelTimer timer("combine_keysplit", st);
         const size_t n4 = (size_t)p.BH * p.S * (D / 4);
         const unsigned blocks = (unsigned)((n4 + 255) / 256 < (size_t)8 * num_sms_current_device()
                                                ? (n4 + 255) / 256 : (size_t)8 * num_sms_current_device());
-        combine_keysplit_kernel<<<blocks, 256, 0, st>>>(part, dpart, tokrec, a.o_pre, (__nv_bfloat16 *)a.h,
-                                                        (size_t)p.BH * p.S, D);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        e = launch_chained(combine_keysplit_kernel, dim3(blocks), dim3(256), 0, st, (const float *)part,
+                           (const float *)dpart, (const float2 *)tokrec, a.o_pre, (__nv_bfloat16 *)a.h,
+                           (size_t)p.BH * p.S, D);
+        if (e != cudaSuccess) return e;
     }
     return cudaSuccess;
 }

@@ -31,6 +31,7 @@ __global__ void __launch_bounds__(256)
 gate_prologue_kernel(const float *__restrict__ i_pre, const float *__restrict__ f_pre,
                      float *__restrict__ bcum, float *__restrict__ pmx, float2 *__restrict__ cstat,
                      int BH, int S, int L, int nchunks, int fgate_exp) {
+    pdl_launch_dependents();      // the next kernel may be scheduled; it waits for this one
     const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
     if (warp >= BH * nchunks) return;

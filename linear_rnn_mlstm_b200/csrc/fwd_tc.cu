@@ -226,6 +226,7 @@ segment_output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
 
     // ------------------------------------------------------------ set-up
     TC_TRACE_NS(tid == 0, 30);
+    pdl_launch_dependents();
     if (tid == 0) {
         for (int i = 0; i < B_NUM; ++i) {
             const bool two = i == B_Q_FREE || i == B_H_FREE0 || i == B_H_FREE1 || i == B_FINV_FREE0 ||
@@ -245,6 +246,7 @@ segment_output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
     auto nj = [&](int r) { return D == 256 ? 2 * (tid - 64) + r : (tid - 64); };
     __syncthreads();
     tc_fence_after();
+    pdl_wait();                                    // the segment scan's states and the gate statistics
     const uint32_t tbase = *tmem_slot;
     const uint32_t t_state = tbase;                // columns [0, D)
     const uint32_t t_S = tbase + 256;              // columns [256, 328)
@@ -402,6 +404,7 @@ segment_output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
                 for (int jb = 0; jb < D / 64; ++jb)
                     tma_load_3d(sQ + jb * 8192, &map_q, &bars[B_FULL_Q], jb * 64, t0, bh);
                 ++issued_q;
+                TC_TRACE(true, c, 29);
                 const int slot = c & 1;
                 if (c >= 2 && !mbar_wait(&bars[B_K_FREE0 + slot], ((c >> 1) - 1) & 1, abort_flag, status)) break;
                 mbar_arrive_expect_tx(&bars[B_FULL_K0 + slot], kL * D * 2);
@@ -519,9 +522,11 @@ segment_output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
                 mma_commit(&bars[B_V_FREE]);
                 if (c + 1 < nch) {   // scores of the next chunk
                     const int slot = (c + 1) & 1;
-                    if (!mbar_wait(&bars[B_FULL_Q], (c + 1) & 1, abort_flag, status) ||
-                        !mbar_wait(&bars[B_FULL_K0 + slot], ((c + 1) >> 1) & 1, abort_flag, status) ||
-                        !mbar_wait(&bars[B_NROW_READY0 + slot], (c >> 1) & 1, abort_flag, status) ||
+                    if (!mbar_wait(&bars[B_FULL_Q], (c + 1) & 1, abort_flag, status)) { ok = false; break; }
+                    TC_TRACE(true, c + 1, 30);
+                    if (!mbar_wait(&bars[B_FULL_K0 + slot], ((c + 1) >> 1) & 1, abort_flag, status)) { ok = false; break; }
+                    TC_TRACE(true, c + 1, 31);
+                    if (!mbar_wait(&bars[B_NROW_READY0 + slot], (c >> 1) & 1, abort_flag, status) ||
                         !mbar_wait(&bars[B_S_FREE], c & 1, abort_flag, status)) { ok = false; break; }
                     tc_fence_after();
                     TC_TRACE(true, c, 14);
@@ -979,6 +984,8 @@ segment_output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
 __global__ void __launch_bounds__(256)
 segment_scan_kernel(const float2 *__restrict__ sstat, float *__restrict__ summ, const float *__restrict__ C0,
                     const float *__restrict__ n0, const float *__restrict__ m0, int D, int P) {
+    pdl_launch_dependents();
+    pdl_wait();
     const int bh = blockIdx.y;
     const size_t per = (size_t)D * D + D;
     const size_t e4 = ((size_t)blockIdx.x * blockDim.x + threadIdx.x) * 4;
@@ -1067,6 +1074,8 @@ segment_summary_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __gri
     const size_t tok0 = (size_t)bh * S;
     const float inv_sqrt_d = rsqrtf((float)D);
 
+    pdl_launch_dependents();
+    pdl_wait();
     float *tabM = fw;                                  // chunk maxima, staged (fw is free until the loop)
     for (int c = tid; c < nch; c += blockDim.x) {
         const float2 cs = cstat[(size_t)bh * nchunks + c0 + c];
@@ -1258,15 +1267,15 @@ cudaError_t launch_summaries_t(const FwdArgs &a, const FwdPlan &p, cudaStream_t 
     if (e != cudaSuccess) return e;
     {
         KernelTimer timer("segment_summary_tc", st);
-        segment_summary_tc_kernel<D><<<dim3(SumLayout<D>::NT * SumLayout<D>::KS, p.P - 1, p.BH), kThreads, sm, st>>>(
-            mk, mv, a.i_pre, bcum, cstat, sstat, summ, a.status, p.S, p.nchunks, p.P, p.cps, p.L);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        e = launch_chained(segment_summary_tc_kernel<D>, dim3(SumLayout<D>::NT * SumLayout<D>::KS, p.P - 1, p.BH),
+                           dim3(kThreads), sm, st, mk, mv, a.i_pre, bcum, cstat, sstat, summ, a.status, p.S,
+                           p.nchunks, p.P, p.cps, p.L);
+        if (e != cudaSuccess) return e;
     }
     KernelTimer timer("segment_scan", st);
     const size_t per4 = ((size_t)D * D + D) / 4;
-    segment_scan_kernel<<<dim3((unsigned)((per4 + 255) / 256), p.BH), 256, 0, st>>>(
-        sstat, summ, a.C0, a.n0, a.m0, D, p.P);
-    return cudaGetLastError();
+    return launch_chained(segment_scan_kernel, dim3((unsigned)((per4 + 255) / 256), p.BH), dim3(256), 0, st,
+                          (const float2 *)sstat, summ, a.C0, a.n0, a.m0, D, p.P);
 }
 
 template <int D>
@@ -1286,10 +1295,10 @@ cudaError_t launch_tc_t(const FwdArgs &a, const FwdPlan &p, cudaStream_t st) {
     e = cudaFuncSetAttribute(segment_output_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
     if (e != cudaSuccess) return e;
     KernelTimer timer("segment_output_tc", st);
-    segment_output_tc_kernel<D><<<dim3(D / kRows, p.P, p.BH), kOutThreads, sm, st>>>(
-        mq, mk, mv, mo, (__nv_bfloat16 *)a.h, a.i_pre, a.o_pre, a.C0, a.n0, a.m0, a.C_out, a.n_out, a.m_out,
-        bcum, ws + p.off_pmax, cstat, sstat, summ, a.status, p.S, p.nchunks, p.P, p.cps);
-    return cudaGetLastError();
+    return launch_chained(segment_output_tc_kernel<D>, dim3(D / kRows, p.P, p.BH), dim3(kOutThreads), sm, st,
+                          mq, mk, mv, mo, (__nv_bfloat16 *)a.h, a.i_pre, a.o_pre, a.C0, a.n0, a.m0, a.C_out,
+                          a.n_out, a.m_out, bcum, (const float *)(ws + p.off_pmax), cstat,
+                          (const float2 *)sstat, (const float *)summ, a.status, p.S, p.nchunks, p.P, p.cps);
 }
 
 }  // namespace

@@ -38,6 +38,25 @@ struct StepArgs {
     unsigned int *status;     // device status word of the current device
 };
 
+// Launches `kern` with the programmatic stream-serialisation attribute: it may
+// be scheduled while the previous kernel on `st` finishes, and waits for it in
+// pdl_wait() (common.cuh).  Used for the forward's kernels after the first.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_chained(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                           Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
 cudaError_t launch_gate_prologue(const FwdArgs &a, const FwdPlan &p, cudaStream_t st);
 // Segment summaries + segment scan of the two-level chunk-state scan, on the
 // tensor cores (bf16, DH 64, 128 or 256); nothing when the plan has one segment.
