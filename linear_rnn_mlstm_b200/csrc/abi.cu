@@ -42,6 +42,7 @@ bool make_fwd_plan(int B, int NH, int S, int DH, int L, int path, int forced_seg
     p->BH = B * NH;
     p->path = path;
     p->nchunks = S > 0 ? (S + L - 1) / L : 0;
+    p->Spad = (S + 63) / 64 * 64;
     const bool tensor = path == XLSTM_PATH_TENSOR || path == XLSTM_PATH_TENSOR_TMEM || path == XLSTM_PATH_TENSOR_RS;
     if (tensor) {
         p->rows = DH < 128 ? DH : 128;
@@ -82,6 +83,9 @@ bool make_fwd_plan(int B, int NH, int S, int DH, int L, int path, int forced_seg
     size_t off = 0;
     p->off_bcum = off;  off = align64(off + (size_t)p->BH * S);
     p->off_pmax = off;  off = align64(off + (size_t)p->BH * S);
+    p->off_upad = off;  off = align64(off + (size_t)p->BH * p->Spad);
+    p->off_bpad = off;  off = align64(off + (size_t)p->BH * p->Spad);
+    p->off_xpad = off;  off = align64(off + (size_t)p->BH * p->Spad);
     p->off_cstat = off; off = align64(off + (size_t)p->BH * p->nchunks * 2);
     p->off_sstat = off; off = align64(off + (size_t)p->BH * p->P * 2);
     p->off_summ = off;  off = align64(off + (size_t)p->BH * (p->P - 1) * ((size_t)DH * DH + DH));

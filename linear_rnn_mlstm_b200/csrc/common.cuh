@@ -55,9 +55,11 @@ __device__ __forceinline__ float warp_max(float x) {
 // stream-serialisation attribute, so each may be scheduled while its
 // predecessor on the stream drains.  pdl_wait() returns once the predecessor
 // grid has completed and its writes are visible; every thread calls it before
-// touching memory the predecessor writes (or reads).  pdl_launch_dependents()
-// lets the next kernel be scheduled before this one ends.  Both are no-ops for
-// a kernel launched without the attribute.
+// touching memory the predecessor writes (or reads).  pdl_launch_dependents(),
+// issued near the end of a kernel, lets the next kernel be scheduled while this
+// one drains (issued at the start instead, the waiting CTAs of the next kernel
+// were measured to slow the forward down).  Both are no-ops for a kernel
+// launched without the attribute.
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_launch_dependents() {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");

@@ -234,7 +234,6 @@ segment_output_rs_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
     const int q4 = warp & 3;
     const uint32_t lane_addr = ((uint32_t)(32 * q4)) << 16;
 
-    pdl_launch_dependents();
     if (tid == 0) {
         for (int i = 0; i < B_NUM; ++i) {
             const bool two = (i >= B_KE && i < B_KE + 4) || (i >= B_GE && i < B_GE + 3);
@@ -914,6 +913,7 @@ segment_output_rs_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
         }
         tc_fence_before();
     }
+    pdl_launch_dependents();      // the combining kernel may be scheduled; it waits for this one
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();

@@ -26,12 +26,14 @@ namespace xlstm {
 // ------------------------------------------------------------------ phase 0
 // One warp per (head, chunk): lf, the chunk-local inclusive prefix sum b, the
 // chunk-local inclusive prefix maximum of u = li - b, the chunk total and the
-// chunk maximum of u.
+// chunk maximum of u; u, b and the prefix maximum also go to copies whose rows
+// are padded to 64 tokens, so that 64-token tiles of them can be fetched by
+// bulk copies.
 __global__ void __launch_bounds__(256)
 gate_prologue_kernel(const float *__restrict__ i_pre, const float *__restrict__ f_pre,
                      float *__restrict__ bcum, float *__restrict__ pmx, float2 *__restrict__ cstat,
-                     int BH, int S, int L, int nchunks, int fgate_exp) {
-    pdl_launch_dependents();      // the next kernel may be scheduled; it waits for this one
+                     float *__restrict__ upad, float *__restrict__ bpad, float *__restrict__ xpad,
+                     int BH, int S, int Spad, int L, int nchunks, int fgate_exp) {
     const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
     if (warp >= BH * nchunks) return;
@@ -50,7 +52,8 @@ gate_prologue_kernel(const float *__restrict__ i_pre, const float *__restrict__ 
             if (lane >= o) lf += y;
         }
         const float b = carry + lf;
-        float u = ok ? i_pre[base + tt] - b : -INFINITY;
+        const float u_raw = ok ? i_pre[base + tt] - b : 0.f;
+        float u = ok ? u_raw : -INFINITY;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {          // inclusive prefix max of u
             const float y = __shfl_up_sync(0xffffffffu, u, o);
@@ -60,11 +63,15 @@ gate_prologue_kernel(const float *__restrict__ i_pre, const float *__restrict__ 
         if (ok) {
             bcum[base + tt] = b;
             pmx[base + tt] = u;
+            upad[(size_t)bh * Spad + tt] = u_raw;
+            bpad[(size_t)bh * Spad + tt] = b;
+            xpad[(size_t)bh * Spad + tt] = u;
         }
         carry = __shfl_sync(0xffffffffu, b, 31);
         umax = __shfl_sync(0xffffffffu, u, 31);
     }
     if (lane == 0) cstat[(size_t)bh * nchunks + c] = make_float2(carry, umax);
+    pdl_launch_dependents();      // the next kernel may be scheduled; it waits for this one
 }
 
 // ------------------------------------------------------------------ phase 1
@@ -393,8 +400,9 @@ cudaError_t launch_gate_prologue(const FwdArgs &a, const FwdPlan &p, cudaStream_
     const int blocks = (warps + 7) / 8;
     KernelTimer timer("gate_prologue", st);
     gate_prologue_kernel<<<blocks, 256, 0, st>>>(a.i_pre, a.f_pre, ws + p.off_bcum, ws + p.off_pmax,
-                                                 (float2 *)(ws + p.off_cstat), p.BH, p.S, p.L,
-                                                 p.nchunks, a.fgate_exp);
+                                                 (float2 *)(ws + p.off_cstat), ws + p.off_upad,
+                                                 ws + p.off_bpad, ws + p.off_xpad, p.BH, p.S,
+                                                 p.Spad, p.L, p.nchunks, a.fgate_exp);
     return cudaGetLastError();
 }
 

@@ -41,8 +41,11 @@ namespace {
 
 constexpr int kL = 64;             // tokens per chunk on this path
 constexpr int kRows = 128;         // value rows per CTA
-constexpr int kKRows = 72;         // key-tile rows: 64 keys, n' hi, n' lo, 6 zero rows
+constexpr int kKRows = 72;         // key-tile rows: 64 keys, n' hi, n' lo, 6 spare rows
 constexpr int kKBlock = kKRows * 128;   // bytes per 64-column block of the key tile
+// Key rows 66-71 of the first block only feed score columns 66-71, which nothing
+// reads: a chunk's per-token u, b and prefix maxima ride there (3 x 256 bytes).
+constexpr int kGateRow = 66;
 constexpr int kThreads = 320;       // segment summaries: TMA warp, MMA warp, 8 compute warps
 constexpr int kMaxCps = 256;       // chunks per segment the tables hold
 constexpr float kLnLambdaFloor = -40.f;  // rescale the TMEM state below this log scale
@@ -172,10 +175,10 @@ segment_output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
                          const float *__restrict__ i_pre, const float *__restrict__ o_pre,
                          const float *__restrict__ C0, const float *__restrict__ n0, const float *__restrict__ m0,
                          float *__restrict__ C_out, float *__restrict__ n_out, float *__restrict__ m_out,
-                         const float *__restrict__ bcum, const float *__restrict__ pmx,
-                         const float2 *__restrict__ cstat,
+                         const float *__restrict__ upad, const float *__restrict__ bpad,
+                         const float *__restrict__ xpad, const float2 *__restrict__ cstat,
                          const float2 *__restrict__ sstat, const float *__restrict__ summ,
-                         unsigned int *status, int S, int nchunks, int P, int cps) {
+                         unsigned int *status, int S, int Spad, int nchunks, int P, int cps) {
     using Lay = OutLayout<D>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = align1024(smem_raw);
@@ -226,7 +229,6 @@ segment_output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
 
     // ------------------------------------------------------------ set-up
     TC_TRACE_NS(tid == 0, 30);
-    pdl_launch_dependents();
     if (tid == 0) {
         for (int i = 0; i < B_NUM; ++i) {
             const bool two = i == B_Q_FREE || i == B_H_FREE0 || i == B_H_FREE1 || i == B_FINV_FREE0 ||
@@ -407,10 +409,17 @@ segment_output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
                 TC_TRACE(true, c, 29);
                 const int slot = c & 1;
                 if (c >= 2 && !mbar_wait(&bars[B_K_FREE0 + slot], ((c >> 1) - 1) & 1, abort_flag, status)) break;
-                mbar_arrive_expect_tx(&bars[B_FULL_K0 + slot], kL * D * 2);
+                mbar_arrive_expect_tx(&bars[B_FULL_K0 + slot], kL * D * 2 + 3 * kL * 4);
                 for (int jb = 0; jb < D / 64; ++jb)
                     tma_load_3d(sK + slot * Lay::kKslot + jb * kKBlock, &map_k, &bars[B_FULL_K0 + slot],
                                 jb * 64, t0, bh);
+                {   // the chunk's u, b and prefix maxima, into the slot's spare rows
+                    uint8_t *gdst = sK + slot * Lay::kKslot + kGateRow * 128;
+                    const size_t gsrc = (size_t)bh * Spad + t0;
+                    bulk_load(gdst, upad + gsrc, kL * 4, &bars[B_FULL_K0 + slot]);
+                    bulk_load(gdst + 256, bpad + gsrc, kL * 4, &bars[B_FULL_K0 + slot]);
+                    bulk_load(gdst + 512, xpad + gsrc, kL * 4, &bars[B_FULL_K0 + slot]);
+                }
                 ++issued_k[slot];
                 if (c >= 1 && !mbar_wait(&bars[B_V_FREE], (c - 1) & 1, abort_flag, status)) break;
                 mbar_arrive_expect_tx(&bars[B_FULL_V], kL * kRows * 2);
@@ -542,24 +551,11 @@ segment_output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
         // --------------------------------------------------------- operand group
         bool ok = true;
         int nwide = 0;
-        float pre_b = 0.f, pre_i = 0.f, pre_x = 0.f;         // prefetched gates of the next chunk
-        float2 pre_cs = make_float2(0.f, 0.f);
-        if (nch > 0) {
-            const int t0 = c0 * kL;
-            pre_cs = cstat[(size_t)bh * nchunks + c0];
-            if (ct < kL && t0 + ct < S) {
-                pre_b = bcum[tok0 + t0 + ct];
-                pre_i = i_pre[tok0 + t0 + ct];
-                pre_x = pmx[tok0 + t0 + ct];
-            }
-        }
         for (int c = 0; ok && c < nch; ++c) {
             const int t0 = (c0 + c) * kL;
             const int Lc = min(kL, S - t0);
             const int pb = c & 1;
             const float mprev = tab.mprev[c];
-            const float2 cs = pre_cs;                         // (sum of log f, max of u) of this chunk
-            const float mnext = cs.x + fmaxf(mprev, cs.y);
             const bool wide = tab.wide[c] != 0.f;
             TC_TRACE(ct == 0, c, 0);
             // (1) lazy rescale of the TMEM state before this chunk's retrieval
@@ -583,13 +579,20 @@ segment_output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
             }
             // (2) per-token gates of this chunk (parity buffer pb):
             //     m_t = b_t + max(m_prev, chunk prefix max of u)
-            if (c >= 2 && !wait_ops(&bars[B_GATES_FREE0 + pb], ((c >> 1) - 1) & 1, abort_flag, status)) { ok = false; break; }
+            // u, b and the prefix maximum of u arrived with the chunk's keys, in the
+            // key slot's spare rows; the chunk totals are their values at the last token
+            if (!wait_ops(&bars[B_FULL_K0 + (c & 1)], (c >> 1) & 1, abort_flag, status) ||
+                (c >= 2 && !wait_ops(&bars[B_GATES_FREE0 + pb], ((c >> 1) - 1) & 1, abort_flag, status))) { ok = false; break; }
+            const float *g_u = reinterpret_cast<const float *>(sK + (c & 1) * Lay::kKslot + kGateRow * 128);
+            const float *g_b = g_u + 64, *g_x = g_u + 128;
+            const float2 cs = make_float2(g_b[Lc - 1], g_x[Lc - 1]);   // (sum of log f, max of u) of this chunk
+            const float mnext = cs.x + fmaxf(mprev, cs.y);
             if (ct < kL) {
                 const int t = ct;
                 const bool valid = t < Lc;
-                const float b = valid ? pre_b : 0.f;
-                const float u = valid ? pre_i - pre_b : -INFINITY;
-                const float run = fmaxf(mprev, valid ? pre_x : mprev);
+                const float b = valid ? g_b[t] : 0.f;
+                const float u = valid ? g_u[t] : -INFINITY;
+                const float run = fmaxf(mprev, valid ? g_x[t] : mprev);
                 const float gt = valid ? expf(mprev - run) : 0.f;     // = e^{b_t + m_prev - m_t}
                 const float wn = valid ? expf(u + cs.x - mnext) * inv_sqrt_d : 0.f;
                 const float wl = valid ? expf(u + cs.x - mnext + tab.lnupd[c]) * inv_sqrt_d : 0.f;
@@ -600,15 +603,6 @@ segment_output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
                 fpw[t] = wn;
                 fu[64 * pb + t] = u;
                 frun[64 * pb + t] = run;
-            }
-            pre_b = pre_i = pre_x = 0.f;
-            if (c + 1 < nch) {
-                pre_cs = cstat[(size_t)bh * nchunks + c0 + c + 1];
-                if (ct < kL && t0 + kL + ct < S) {
-                    pre_b = bcum[tok0 + t0 + kL + ct];
-                    pre_i = i_pre[tok0 + t0 + kL + ct];
-                    pre_x = pmx[tok0 + t0 + kL + ct];
-                }
             }
             sync_ops();
             if (ct == 0) mbar_arrive(&bars[B_GATES_READY0 + pb]);
@@ -984,7 +978,6 @@ segment_output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid
 __global__ void __launch_bounds__(256)
 segment_scan_kernel(const float2 *__restrict__ sstat, float *__restrict__ summ, const float *__restrict__ C0,
                     const float *__restrict__ n0, const float *__restrict__ m0, int D, int P) {
-    pdl_launch_dependents();
     pdl_wait();
     const int bh = blockIdx.y;
     const size_t per = (size_t)D * D + D;
@@ -1013,6 +1006,7 @@ segment_scan_kernel(const float2 *__restrict__ sstat, float *__restrict__ summ, 
         slot[g * stride4] = make_float4(x[0], x[1], x[2], x[3]);
         mc = mn;
     }
+    pdl_launch_dependents();
 }
 
 // ------------------------------------------------------------ segment summaries
@@ -1021,7 +1015,10 @@ segment_scan_kernel(const float2 *__restrict__ sstat, float *__restrict__ summ, 
 // tensor cores with the accumulator in TMEM; dn = sum_s w_s k_s on the tensor
 // cores too, as rows 0 and 1 (w in bf16 high and low parts) of an M=64 product
 // with the same K tile.  K and V stream through a 4-stage ring; V is scaled by
-// w in place.
+// w in place.  The tile's u = log i - b travels with it: a bulk copy puts the
+// 64 floats into rows 2-3 of the stage's W tile, rows whose products (rows 2-3
+// of the dn accumulator) are never read, so the compute warps hold no global
+// load across their barriers.
 // DH 512 splits the key columns over two CTAs (KC = 256 each); their summaries
 // are independent column blocks of the same dC, so nothing is exchanged.
 template <int D>
@@ -1043,9 +1040,9 @@ static_assert(SumLayout<512>::kBytes <= kMaxSmemPerCta, "summary kernel shared m
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
 segment_summary_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v,
-                          const float *__restrict__ i_pre, const float *__restrict__ bcum,
-                          const float2 *__restrict__ cstat, float2 *__restrict__ sstat, float *__restrict__ summ,
-                          unsigned int *status, int S, int nchunks, int P, int cps, int L) {
+                          const float *__restrict__ upad, const float2 *__restrict__ cstat,
+                          float2 *__restrict__ sstat, float *__restrict__ summ,
+                          unsigned int *status, int S, int Spad, int nchunks, int P, int cps, int L) {
     using Lay = SumLayout<D>;
     constexpr int NS = Lay::kStages;
     // value rows of this CTA: 128, or all DH when DH < 128 (the MMAs keep M = 128;
@@ -1071,10 +1068,8 @@ segment_summary_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __gri
     const int nsub = L / kL;
     const int tseg = c0 * L;
     const int ntl = (min(S, (c0 + nch) * L) - tseg + kL - 1) / kL;
-    const size_t tok0 = (size_t)bh * S;
     const float inv_sqrt_d = rsqrtf((float)D);
 
-    pdl_launch_dependents();
     pdl_wait();
     float *tabM = fw;                                  // chunk maxima, staged (fw is free until the loop)
     for (int c = tid; c < nch; c += blockDim.x) {
@@ -1126,11 +1121,12 @@ segment_summary_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __gri
                 const int slot = c % NS, t0 = tseg + c * kL;
                 if (c >= NS && !mbar_wait(&b_free[slot], ((c / NS) - 1) & 1, abort_flag, status)) break;
                 uint8_t *base = smem + slot * Lay::kSlot;
-                mbar_arrive_expect_tx(&b_full[slot], kL * KC * 2 + kL * kVBlocks * 64 * 2);
+                mbar_arrive_expect_tx(&b_full[slot], kL * KC * 2 + kL * kVBlocks * 64 * 2 + kL * 4);
                 for (int jb = 0; jb < KC / 64; ++jb)
                     tma_load_3d(base + jb * 8192, &map_k, &b_full[slot], k0 + jb * 64, t0, bh);
                 for (int b = 0; b < kVBlocks; ++b)
                     tma_load_3d(base + Lay::kKslot + b * 8192, &map_v, &b_full[slot], i0 + 64 * b, t0, bh);
+                bulk_load(base + Lay::kKslot + 16384 + 256, upad + (size_t)bh * Spad + t0, kL * 4, &b_full[slot]);
                 ++issued[slot];
             }
             // never leave a load in flight into shared memory
@@ -1165,25 +1161,15 @@ segment_summary_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __gri
         // one half of the columns each.
         const int ct = tid - 64, q4 = warp & 3;
         bool ok = true;
-        float pre_i = 0.f, pre_b = 0.f;                   // gates of the next chunk, in flight
-        if (ntl > 0 && ct < kL && tseg + ct < S) {
-            pre_i = i_pre[tok0 + tseg + ct];
-            pre_b = bcum[tok0 + tseg + ct];
-        }
         for (int c = 0; c < ntl; ++c) {
             const int slot = c % NS, t0 = tseg + c * kL, Lc = min(kL, S - t0);
-            if (ct < kL)
-                fw[ct] = ct < Lc ? expf(pre_i - pre_b + tabE[c / nsub] - mloc) * inv_sqrt_d : 0.f;
-            pre_i = pre_b = 0.f;
-            if (c + 1 < ntl && ct < kL && t0 + kL + ct < S) {
-                pre_i = i_pre[tok0 + t0 + kL + ct];
-                pre_b = bcum[tok0 + t0 + kL + ct];
-            }
             if (!compute_wait(&b_full[slot], (c / NS) & 1, abort_flag, status)) { ok = false; break; }
             uint8_t *base = smem + slot * Lay::kSlot;
             uint8_t *sV = base + Lay::kKslot;
             if (ct < kL) {       // rows 0 and 1 of W: w in bf16 high and low parts
-                const float wv = fw[ct];
+                const float u = reinterpret_cast<const float *>(sV + 16384 + 256)[ct];
+                const float wv = ct < Lc ? expf(u + tabE[c / nsub] - mloc) * inv_sqrt_d : 0.f;
+                fw[ct] = wv;
                 const __nv_bfloat16 whi = __float2bfloat16_rn(wv);
                 uint8_t *sW = sV + 16384;
                 *reinterpret_cast<__nv_bfloat16 *>(sW + sw128_offset(0, ct >> 3) + (ct & 7) * 2) = whi;
@@ -1242,6 +1228,7 @@ segment_summary_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __gri
         }
         tc_fence_before();
     }
+    pdl_launch_dependents();      // the next kernel may be scheduled; it waits for this one
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
@@ -1258,7 +1245,6 @@ cudaError_t launch_summaries_t(const FwdArgs &a, const FwdPlan &p, cudaStream_t 
     if (!make_map_bf16(&mk, a.k, p.BH, p.S, D) || !make_map_bf16(&mv, a.v, p.BH, p.S, D))
         return cudaErrorInvalidValue;
     float *ws = (float *)a.workspace;
-    const float *bcum = ws + p.off_bcum;
     const float2 *cstat = (const float2 *)(ws + p.off_cstat);
     float2 *sstat = (float2 *)(ws + p.off_sstat);
     float *summ = ws + p.off_summ;
@@ -1268,8 +1254,8 @@ cudaError_t launch_summaries_t(const FwdArgs &a, const FwdPlan &p, cudaStream_t 
     {
         KernelTimer timer("segment_summary_tc", st);
         e = launch_chained(segment_summary_tc_kernel<D>, dim3(SumLayout<D>::NT * SumLayout<D>::KS, p.P - 1, p.BH),
-                           dim3(kThreads), sm, st, mk, mv, a.i_pre, bcum, cstat, sstat, summ, a.status, p.S,
-                           p.nchunks, p.P, p.cps, p.L);
+                           dim3(kThreads), sm, st, mk, mv, (const float *)(ws + p.off_upad), cstat, sstat, summ,
+                           a.status, p.S, p.Spad, p.nchunks, p.P, p.cps, p.L);
         if (e != cudaSuccess) return e;
     }
     KernelTimer timer("segment_scan", st);
@@ -1285,7 +1271,6 @@ cudaError_t launch_tc_t(const FwdArgs &a, const FwdPlan &p, cudaStream_t st) {
         !make_map_bf16(&mv, a.v, p.BH, p.S, D) || !make_map_f32_rows(&mo, a.o_pre, p.BH, p.S, D, kRows, 32))
         return cudaErrorInvalidValue;
     float *ws = (float *)a.workspace;
-    const float *bcum = ws + p.off_bcum;
     const float2 *cstat = (const float2 *)(ws + p.off_cstat);
     float2 *sstat = (float2 *)(ws + p.off_sstat);
     float *summ = ws + p.off_summ;
@@ -1297,8 +1282,9 @@ cudaError_t launch_tc_t(const FwdArgs &a, const FwdPlan &p, cudaStream_t st) {
     KernelTimer timer("segment_output_tc", st);
     return launch_chained(segment_output_tc_kernel<D>, dim3(D / kRows, p.P, p.BH), dim3(kOutThreads), sm, st,
                           mq, mk, mv, mo, (__nv_bfloat16 *)a.h, a.i_pre, a.o_pre, a.C0, a.n0, a.m0, a.C_out,
-                          a.n_out, a.m_out, bcum, (const float *)(ws + p.off_pmax), cstat,
-                          (const float2 *)sstat, (const float *)summ, a.status, p.S, p.nchunks, p.P, p.cps);
+                          a.n_out, a.m_out, (const float *)(ws + p.off_upad), (const float *)(ws + p.off_bpad),
+                          (const float *)(ws + p.off_xpad), cstat, (const float2 *)sstat, (const float *)summ,
+                          a.status, p.S, p.Spad, p.nchunks, p.P, p.cps);
 }
 
 }  // namespace

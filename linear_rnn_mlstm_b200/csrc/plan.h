@@ -28,9 +28,15 @@ struct FwdPlan {
     int path;                 // 1 = SIMT, 2 = tensor core
     int rows;                 // value rows per output CTA
     int ntiles;               // ceil(DH / rows)
+    int Spad;                 // S rounded up to 64 tokens (row stride of off_upad)
     // workspace layout, in floats from the workspace base
     size_t off_bcum;          // [BH, S]        chunk-local inclusive cumsum of log f
     size_t off_pmax;          // [BH, S]        chunk-local inclusive prefix max of log i - b
+    // the same per-token gate values with rows padded to Spad (256-byte aligned
+    // 64-token tiles, fetched by bulk copies):
+    size_t off_upad;          // [BH, Spad]     log i - b
+    size_t off_bpad;          // [BH, Spad]     b
+    size_t off_xpad;          // [BH, Spad]     chunk-local prefix max of log i - b
     size_t off_cstat;         // [BH, nchunks, 2]  (chunk total of log f, chunk max of log i - b)
     size_t off_sstat;         // [BH, P, 2]     (segment total of log f, segment stabiliser)
     size_t off_summ;          // [BH, P-1, DH*DH + DH]  segment summaries (C part then n part)
