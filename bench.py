@@ -89,7 +89,8 @@ def source_sha(kernel):
     also depend on the tcgen05/TMA wrappers)."""
     files = {"segment_output_simt": ["fwd_simt.cu"], "segment_summary_simt": ["fwd_simt.cu"],
              "gate_prologue": ["fwd_simt.cu"], "step_rows": ["step.cu"], "step_state": ["step.cu"],
-             "headnorm_gate": ["headnorm.cu"], "segment_output_rs": ["fwd_rs.cu", "tc_ptx.cuh"]}
+             "headnorm_gate": ["headnorm.cu"], "segment_output_rs": ["fwd_rs.cu", "tc_ptx.cuh"],
+             "combine_keysplit": ["fwd_rs.cu"]}
     fns = files.get(kernel)
     if fns is None and kernel.endswith("_tc"):
         fns = ["fwd_tc.cu", "tc_ptx.cuh"]

@@ -71,9 +71,18 @@ __device__ unsigned long long *g_tc_trace = nullptr;
             g_tc_trace[cta_ * kMaxCps * 32 + (slot)] = globaltimer_ns();                           \
         }                                                                                          \
     } while (0)
+// the segment-summary kernel's records, after the output kernel's (CTA index + 1024)
+#define TC_TRACE_SUM(cond, c, slot)                                                                \
+    do {                                                                                           \
+        if (g_tc_trace && (cond) && (c) < kMaxCps) {                                               \
+            const size_t cta_ = ((size_t)blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x + 1024; \
+            g_tc_trace[(cta_ * kMaxCps + (c)) * 32 + (slot)] = clock64();                          \
+        }                                                                                          \
+    } while (0)
 #else
 #define TC_TRACE(cond, c, slot) do { } while (0)
 #define TC_TRACE_NS(cond, slot) do { } while (0)
+#define TC_TRACE_SUM(cond, c, slot) do { } while (0)
 #endif
 
 // A bounded wait taken by all 128 compute threads, with a group-uniform result.
@@ -1120,6 +1129,7 @@ segment_summary_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __gri
             for (int c = 0; c < ntl; ++c) {
                 const int slot = c % NS, t0 = tseg + c * kL;
                 if (c >= NS && !mbar_wait(&b_free[slot], ((c / NS) - 1) & 1, abort_flag, status)) break;
+                TC_TRACE_SUM(true, c, 0);
                 uint8_t *base = smem + slot * Lay::kSlot;
                 mbar_arrive_expect_tx(&b_full[slot], kL * KC * 2 + kL * kVBlocks * 64 * 2 + kL * 4);
                 for (int jb = 0; jb < KC / 64; ++jb)
@@ -1138,6 +1148,7 @@ segment_summary_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __gri
             for (int c = 0; c < ntl; ++c) {
                 const int slot = c % NS;
                 if (!mbar_wait(&b_ready[slot], (c / NS) & 1, abort_flag, status)) break;
+                TC_TRACE_SUM(true, c, 1);
                 tc_fence_after();
                 const uint32_t va = smem_u32(smem + slot * Lay::kSlot + Lay::kKslot);
                 const uint32_t ka = smem_u32(smem + slot * Lay::kSlot);
@@ -1164,6 +1175,7 @@ segment_summary_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __gri
         for (int c = 0; c < ntl; ++c) {
             const int slot = c % NS, t0 = tseg + c * kL, Lc = min(kL, S - t0);
             if (!compute_wait(&b_full[slot], (c / NS) & 1, abort_flag, status)) { ok = false; break; }
+            TC_TRACE_SUM(ct == 0, c, 2);
             uint8_t *base = smem + slot * Lay::kSlot;
             uint8_t *sV = base + Lay::kKslot;
             if (ct < kL) {       // rows 0 and 1 of W: w in bf16 high and low parts
@@ -1193,6 +1205,7 @@ segment_summary_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __gri
             fence_async_smem();
             named_sync_compute();
             if (ct == 0) mbar_arrive(&b_ready[slot]);
+            TC_TRACE_SUM(ct == 0, c, 3);
         }
         if (ok && compute_wait(b_done, 0, abort_flag, status)) {
             __syncwarp();
