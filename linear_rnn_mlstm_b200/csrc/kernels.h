@@ -79,6 +79,11 @@ cudaError_t launch_step(const StepArgs &a, cudaStream_t st);
 // boxes and no swizzle.  False if the driver refuses the encoding.
 bool make_map_bf16(CUtensorMap *m, const void *base, int BH, int S, int D, bool swizzle = true,
                    int box_rows = 64);
+// A 3-D tensor map without swizzle: dims innermost first, strides in bytes of
+// dimensions 1 and 2 (multiples of 16), box sizes (box[0] * elem_bytes a
+// multiple of 16, each at most 256).  elem_bytes 2 (bf16) or 4 (fp32).
+bool make_tensor_map_3d(CUtensorMap *m, const void *base, int elem_bytes, const unsigned long long dims[3],
+                        const unsigned long long strides_bytes[2], const unsigned box[3]);
 bool make_map_f32_rows(CUtensorMap *m, const void *base, int BH, int S, int D, int box_cols = 128,
                        int box_rows = 64);
 

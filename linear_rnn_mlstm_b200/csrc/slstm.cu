@@ -4,7 +4,9 @@
 // order; h_{t-1} lives in one of two shared arrays while h_t is written to the
 // other, one barrier per step.  The recurrent matrices are read from global
 // memory (each head's 4 DH x DH block stays in L2).  This is the
-// correctness-first form; the per-unit step is in slstm_body.cuh.
+// correctness-first form, kept for the head sizes the cluster kernel
+// (slstm_cluster.cu: DH 64, 128, 256) does not take; the per-unit step is in
+// slstm_body.cuh.
 #include <math.h>
 #include <stdint.h>
 
@@ -34,6 +36,11 @@ __global__ void __launch_bounds__(512) slstm_fwd_kernel(SlstmPtrs p) {
 bool misaligned16(const void *ptr) { return ((uintptr_t)ptr & 15u) != 0; }
 
 }  // namespace
+
+// The cluster kernel for DH 64, 128 and 256 (slstm_cluster.cu).
+bool slstm_cluster_supports(int DH);
+cudaError_t launch_slstm_cluster(const slstm::SlstmPtrs &p, cudaStream_t st);
+
 }  // namespace xlstm
 
 using namespace xlstm;
@@ -73,6 +80,10 @@ extern "C" xlstm_status xlstm_slstm_fwd(const float *zx, const float *ix, const 
     p.BH = (int)BH; p.NH = NH; p.S = S; p.DH = DH;
     p.fgate_exp = fg == XLSTM_FGATE_EXP;
     cudaStream_t st = (cudaStream_t)cuda_stream;
+    if (slstm_cluster_supports(DH)) {
+        KernelTimer timer("slstm_cluster", st);
+        return launch_slstm_cluster(p, st) == cudaSuccess ? XLSTM_OK : XLSTM_ERR_CUDA;
+    }
     KernelTimer timer("slstm_fwd", st);
     slstm_fwd_kernel<<<(unsigned)BH, DH, 2 * DH * sizeof(float), st>>>(p);
     return cudaGetLastError() == cudaSuccess ? XLSTM_OK : XLSTM_ERR_CUDA;
