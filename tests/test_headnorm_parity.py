@@ -70,6 +70,22 @@ def test_epilogue_matches_oracle(cuda_lib, dtype, DH, ogate, skip):
     _check(_gpu(inp, ogate), _ref(inp, ogate), dtype)
 
 
+# Longer sequences at the wide-row widths (a whole warp per row, one to four
+# vectors per lane): row counts that leave every warp of the last pass partly
+# empty, with and without the skip input, and fp32 DH 64.
+STREAM_CASES = [("bf16", 128, 70, "silu", True), ("bf16", 256, 37, "sigmoid", True),
+                ("bf16", 512, 19, "silu", False), ("f32", 64, 70, "sigmoid", True),
+                ("f32", 256, 21, "silu", False), ("f32", 512, 10, "sigmoid", True)]
+
+
+@pytest.mark.parametrize("dtype,DH,S,ogate,skip", STREAM_CASES,
+                         ids=[f"{c[0]}-DH{c[1]}-S{c[2]}-{c[3]}-{'skip' if c[4] else 'noskip'}"
+                              for c in STREAM_CASES])
+def test_epilogue_longer_sequences(cuda_lib, dtype, DH, S, ogate, skip):
+    inp = syn.epilogue_inputs(2, 3, S, DH, dtype, seed=DH + S, skip=skip)
+    _check(_gpu(inp, ogate), _ref(inp, ogate), dtype)
+
+
 def test_epilogue_many_rows_grid_stride(cuda_lib):
     """More rows than one resident wave of CTAs: every warp strides."""
     inp = syn.epilogue_inputs(2, 4, 3001, 128, "bf16", seed=5)
