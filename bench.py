@@ -300,6 +300,7 @@ def main():
     ap.add_argument("--skip-e2e", action="store_true")
     ap.add_argument("--skip-epilogue", action="store_true")
     ap.add_argument("--skip-cpu", action="store_true")
+    ap.add_argument("--skip-slstm", action="store_true")
     ap.add_argument("--skip-sweep", action="store_true",
                     help="skip the per-config / per-chunk entries (small, block, long at 128 and 256)")
     ap.add_argument("--ref-tokens", type=int, default=4096,
@@ -374,6 +375,11 @@ def main():
     if not args.skip_epilogue:
         epilogue = run_epilogue(args, w, dev, env, peaks, peak_src)
 
+    # ------------------------------------------------------ sLSTM (next row)
+    slstm = None
+    if not args.skip_slstm:
+        slstm = run_slstm(args, dev, env, with_cpu=(rank == 0 and world == 1 and not args.skip_cpu))
+
     # ----------------------------------------------------------------- decode
     decode = None
     if not args.skip_decode:
@@ -403,7 +409,7 @@ def main():
                                path=args.path),
                 "roofline": roofline, "tc": tc, "hbm_whole_step": whole,
                 "kernels": kernels, "gpu_launches": launches, "cpu_baseline": cpu, "e2e": e2e,
-                "clocks": clocks, "decode": decode, "epilogue": epilogue, "sweep": sweep}
+                "clocks": clocks, "decode": decode, "epilogue": epilogue, "slstm": slstm, "sweep": sweep}
         print(json.dumps(line), flush=True)
     replicas.barrier(env)
     replicas.shutdown(env)
@@ -595,6 +601,44 @@ def run_epilogue(args, w, dev, env, peaks, peak_src):
                          "peak_source": f"{peak_src} (burst copy)"},
             "config": f"block epilogue: h [{B},{NH},{S},{DH}] {w.dtype} -> y [{B},{S},{NH * DH}], "
                       f"skip on, SiLU gate, eps 1e-5; {alg / 1e6:.0f} MB per launch (> L2)"}
+
+
+def run_slstm(args, dev, env, with_cpu):
+    """The sLSTM forward on its timing workload (B4 NH4 S2048 DH256, fp32): one
+    call walks the sequence; tokens/s and microseconds per recurrent step, with
+    the float64 sLSTM oracle on a bounded sample beside it."""
+    c = syn.SLSTM
+    B, NH, S, DH = c["B"], c["NH"], c["S"], c["DH"]
+    inp = syn.slstm_inputs(B, NH, S, DH, seed=replicas.replica_seed(11, env.rank))
+    x = {k: v.to(dev).contiguous() for k, v in inp.items()}
+    run = lambda: xb.slstm_fwd(x["zx"], x["ix"], x["fx"], x["ox"], x["R"], "sigmoid")
+    for _ in range(max(3, args.warmup)):
+        run()
+    torch.cuda.synchronize(dev)
+    steps = max(3, min(args.steps, 10))
+    ms = time_region(run, steps, env, dev) / steps
+    xb.xlstm_profile_begin()
+    run()
+    torch.cuda.synchronize(dev)
+    _, kt = xb.xlstm_profile_end()
+    tokens = B * NH * S
+    out = {"metric": "sLSTM fwd tokens/s", "value": replicas.job_throughput(tokens, env, ms * 1e-3),
+           "unit": "tokens/s", "ms_per_call": ms, "us_per_step": 1e3 * ms / S,
+           "kernels": {k: {"launches": v[0], "avg_us": 1e3 * v[1] / max(v[0], 1)} for k, v in kt.items()},
+           "config": f"sLSTM fwd: B={B} NH={NH} S={S} DH={DH} fp32, sigmoid forget gate, zero initial state; "
+                     f"{B * NH} heads walk their sequences concurrently"}
+    if with_cpu:
+        import oracle.slstm as so
+        Ss = 128
+        sub = {k: (v[:, :, :Ss] if k != "R" else v).numpy() for k, v in inp.items()}
+        t0 = time.perf_counter()
+        so.fwd(sub["zx"], sub["ix"], sub["fx"], sub["ox"], sub["R"], "sigmoid")
+        dt = time.perf_counter() - t0
+        import oracle
+        out["cpu_baseline"] = {"value": B * NH * Ss / dt, "unit": "tokens/s",
+                               "cores": min(oracle.max_threads(), B * NH), "kind": "oracle",
+                               "sample": f"{B * NH} heads x first {Ss} steps ({B * NH * Ss} tokens, {dt:.2f} s wall)"}
+    return out
 
 
 def run_decode(args, dev, env, peaks, peak_src):

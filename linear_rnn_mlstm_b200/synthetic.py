@@ -155,3 +155,18 @@ def epilogue_inputs(B: int, NH: int, S: int, DH: int, dtype: str = "bf16", seed:
     if skip:
         out.update(skip_w=skip_w, x_skip=x_skip)
     return out
+
+
+# sLSTM timing workload: the 1.3B block width (1024) split over four heads.
+SLSTM = dict(B=4, NH=4, S=2048, DH=256)
+
+
+def slstm_inputs(B: int, NH: int, S: int, DH: int, seed: int = 0) -> dict:
+    """CPU float32 tensors for the sLSTM forward: gate pre-activations zx, ix,
+    fx, ox [B,NH,S,DH] ~ N(0, 0.5^2) and recurrent blocks R [NH,4,DH,DH] ~
+    N(0, 1/DH) per element.  Drawn in the order zx, ix, fx, ox, R."""
+    g = _gen(seed)
+    shp = (B, NH, S, DH)
+    out = {k: torch.randn(shp, generator=g, dtype=torch.float32) * 0.5 for k in ("zx", "ix", "fx", "ox")}
+    out["R"] = torch.randn((NH, 4, DH, DH), generator=g, dtype=torch.float32) / DH ** 0.5
+    return out
