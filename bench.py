@@ -301,6 +301,7 @@ def main():
     ap.add_argument("--skip-epilogue", action="store_true")
     ap.add_argument("--skip-cpu", action="store_true")
     ap.add_argument("--skip-slstm", action="store_true")
+    ap.add_argument("--skip-backward", action="store_true")
     ap.add_argument("--skip-sweep", action="store_true",
                     help="skip the per-config / per-chunk entries (small, block, long at 128 and 256)")
     ap.add_argument("--ref-tokens", type=int, default=4096,
@@ -380,6 +381,11 @@ def main():
     if not args.skip_slstm:
         slstm = run_slstm(args, dev, env, with_cpu=(rank == 0 and world == 1 and not args.skip_cpu))
 
+    # --------------------------------------------------- backward (next row)
+    backward = None
+    if not args.skip_backward:
+        backward = run_backward(args, dev, env, peaks, peak_src)
+
     # ----------------------------------------------------------------- decode
     decode = None
     if not args.skip_decode:
@@ -409,7 +415,8 @@ def main():
                                path=args.path),
                 "roofline": roofline, "tc": tc, "hbm_whole_step": whole,
                 "kernels": kernels, "gpu_launches": launches, "cpu_baseline": cpu, "e2e": e2e,
-                "clocks": clocks, "decode": decode, "epilogue": epilogue, "slstm": slstm, "sweep": sweep}
+                "clocks": clocks, "decode": decode, "epilogue": epilogue, "slstm": slstm, "backward": backward,
+                "sweep": sweep}
         print(json.dumps(line), flush=True)
     replicas.barrier(env)
     replicas.shutdown(env)
@@ -629,7 +636,7 @@ def run_slstm(args, dev, env, with_cpu):
                      f"{B * NH} heads walk their sequences concurrently"}
     if with_cpu:
         import oracle.slstm as so
-        Ss = 128
+        Ss = S                                       # the whole workload: ~0.3 s of float64
         sub = {k: (v[:, :, :Ss] if k != "R" else v).numpy() for k, v in inp.items()}
         t0 = time.perf_counter()
         so.fwd(sub["zx"], sub["ix"], sub["fx"], sub["ox"], sub["R"], "sigmoid")
@@ -638,6 +645,43 @@ def run_slstm(args, dev, env, with_cpu):
         out["cpu_baseline"] = {"value": B * NH * Ss / dt, "unit": "tokens/s",
                                "cores": min(oracle.max_threads(), B * NH), "kind": "oracle",
                                "sample": f"{B * NH} heads x first {Ss} steps ({B * NH * Ss} tokens, {dt:.2f} s wall)"}
+    return out
+
+
+def run_backward(args, dev, env, peaks, peak_src):
+    """The backward (fp32 kernels) on the small workload and on the long one,
+    chunk 64, gradients of sum(dh h) with dh ~ N(0, 1) in bf16: time per call
+    and HBM fraction at the algorithmic 22 DH + 16 bytes per token (bf16 q, k,
+    v, dh in and dq, dk, dv out; fp32 o in and do out; the gates and their
+    gradients)."""
+    out = []
+    for name in ("small", "long"):
+        w = syn.WORKLOADS[name]
+        inp = syn.fwd_inputs(w, seed=replicas.replica_seed(w.seed, env.rank))
+        x = {k: v.to(dev).contiguous() for k, v in inp.items()}
+        g = torch.Generator().manual_seed(5)
+        dh = torch.randn(inp["q"].shape, generator=g).to(inp["q"].dtype).to(dev)
+        run = lambda: xb.mlstm_bwd(x["q"], x["k"], x["v"], x["i_pre"], x["f_pre"], x["o_pre"], dh,
+                                   chunk=64, fgate=w.fgate)
+        run()
+        torch.cuda.synchronize(dev)
+        steps = 3
+        ms = time_region(run, steps, env, dev) / steps
+        xb.xlstm_profile_begin()
+        run()
+        torch.cuda.synchronize(dev)
+        _, kt = xb.xlstm_profile_end()
+        tokens = w.B * w.NH * w.S
+        alg = tokens * (22 * w.DH + 16)
+        ach = alg / (ms * 1e-3) / 1e9
+        out.append({"workload": f"{name}: B={w.B} NH={w.NH} S={w.S} DH={w.DH} {w.dtype}, chunk 64",
+                    "ms_per_call": ms, "tokens_per_s": replicas.job_throughput(tokens, env, ms * 1e-3),
+                    "roofline": {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                 "frac": ach / peaks["hbm_gbs"], "algorithmic_bytes": alg,
+                                 "peak_source": f"{peak_src} (burst copy)"},
+                    "kernels": {k: {"launches": v[0], "avg_us": 1e3 * v[1] / max(v[0], 1)}
+                                for k, v in kt.items()}})
+        del x, dh
     return out
 
 

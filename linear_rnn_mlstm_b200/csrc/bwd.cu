@@ -5,8 +5,10 @@
 // bwd_body.cuh (the algorithm is described there):
 //   K1 bwd_gates       one thread per head     log f, chunk-local cumsum, m_t
 //   K2 bwd_states      one thread per state row  chunk-start states C'_c, n'_c
+//                      (DH a multiple of 32: one CTA per 32 rows, bwd_rows_kernel)
 //   K3 bwd_token_fwd   one thread per token    num', nq', den', dotilde, dnum', dnq'
 //   K4 bwd_reverse     one thread per state row  reverse state at each chunk end
+//                      (DH a multiple of 32: one CTA per 32 rows, bwd_rows_kernel)
 //   K5 bwd_token_grad  one thread per token    dq, dk, dv, ditilde
 //   K6 bwd_forget      one thread per head     dftilde (reverse cumulative sum)
 // The chunk-start and reverse states are materialised in the workspace
@@ -60,6 +62,132 @@ template <typename T>
 __global__ void __launch_bounds__(kThreads) bwd_token_grad_kernel(BwdPtrs p) {
     const long long i = thread_index();
     if (i < (long long)p.BH * p.S) bwd::token_grad<T>(p, (int)(i / p.S), (int)(i % p.S));
+}
+
+// K2 and K4 for DH a multiple of 32 (up to 512), one CTA per (32 state rows,
+// head) instead of one thread per row: lanes take the key columns (DH / 32
+// each), a warp four rows, so the rows stay in registers across chunks; per
+// chunk the key tile (K2) or query tile (K4) and the 32 rows' coefficients are
+// staged in shared memory once and shared by all 32 rows.  Same arithmetic,
+// in the same order per element, as states_row / reverse_row.
+constexpr int kRowBlock = 32;
+constexpr int kRowThreads = 256;      // 8 warps x 4 rows
+
+template <typename T>
+size_t rows_smem_bytes(int L, int DH) { return (size_t)L * DH * sizeof(T) + (size_t)L * (kRowBlock + 1) * 4; }
+
+template <typename T, int NCL, bool REVERSE>
+__global__ void __launch_bounds__(kRowThreads) bwd_rows_kernel(BwdPtrs p) {
+    constexpr int DH = 32 * NCL;
+    extern __shared__ __align__(16) uint8_t rows_smem[];
+    const int L = p.L, S = p.S, NC = p.NC;
+    T *tile = reinterpret_cast<T *>(rows_smem);                           // [L][DH]
+    float *coef = reinterpret_cast<float *>(rows_smem + (size_t)L * DH * sizeof(T));   // [L][32]
+    float *wt = coef + (size_t)L * kRowBlock;                             // [L] per-token weight
+    const int bh = blockIdx.y, r0 = blockIdx.x * kRowBlock;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const size_t DD = (size_t)DH * DH;
+    const float inv_sqrt = 1.f / sqrtf((float)DH);
+    const T *src = (const T *)(REVERSE ? p.q : p.k);
+    const T *v = (const T *)p.v;
+    // this warp's rows r0 + 4 warp + i (row DH is the normaliser; rows past it unused)
+    float st[4][NCL];
+    auto slot_ptr = [&](int r, int slot) -> float * {
+        if (r == DH) return (REVERSE ? p.dnb + (size_t)bh * NC * DH : p.nst + (size_t)bh * (NC + 1) * DH) +
+                            (size_t)slot * DH;
+        return (REVERSE ? p.dCb + (size_t)bh * NC * DD : p.Cst + (size_t)bh * (NC + 1) * DD) +
+               (size_t)slot * DD + (size_t)r * DH;
+    };
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int r = r0 + 4 * warp + i;
+#pragma unroll
+        for (int j = 0; j < NCL; ++j) {
+            const int col = lane + 32 * j;
+            float x = 0.f;
+            if (REVERSE && r < DH && p.dC) x = p.dC[(size_t)bh * DD + (size_t)r * DH + col];
+            if (REVERSE && r == DH && p.dn) x = p.dn[(size_t)bh * DH + col];
+            st[i][j] = x;
+            if (r <= DH) slot_ptr(r, REVERSE ? NC - 1 : 0)[col] = x;
+        }
+    }
+    const int c_first = REVERSE ? NC - 1 : 0, c_end = REVERSE ? 0 : NC, dir = REVERSE ? -1 : 1;
+    for (int c = c_first; c != c_end; c += dir) {
+        const size_t hc = (size_t)bh * NC + c;
+        const int a = c * L, n = bwd::imin(S, a + L) - a;
+        __syncthreads();                       // the previous chunk's tile and coefficients are read
+        for (int e = threadIdx.x; e < n * DH / 8; e += kRowThreads) {
+            const int s = e / (DH / 8), part = e % (DH / 8);
+            const size_t g = ((size_t)bh * S + a + s) * DH + part * 8;
+            if (sizeof(T) == 2) {
+                reinterpret_cast<uint4 *>(tile)[(size_t)s * DH / 8 + part] = *reinterpret_cast<const uint4 *>(src + g);
+            } else {
+                reinterpret_cast<uint4 *>(tile)[(size_t)s * DH / 4 + 2 * part] = *reinterpret_cast<const uint4 *>(src + g);
+                reinterpret_cast<uint4 *>(tile)[(size_t)s * DH / 4 + 2 * part + 1] =
+                    *reinterpret_cast<const uint4 *>(src + g + 4);
+            }
+        }
+        const float mend = p.mend[hc], mprev = p.mprev[hc];
+        for (int s = threadIdx.x; s < n; s += kRowThreads) {
+            const size_t ts = (size_t)bh * S + a + s;
+            wt[s] = REVERSE ? expf(p.b[ts] + mprev - p.mt[ts]) : expf(p.Bsum[hc] - p.b[ts] + p.ip[ts] - mend) * inv_sqrt;
+        }
+        __syncthreads();
+        for (int e = threadIdx.x; e < n * kRowBlock; e += kRowThreads) {
+            const int s = e / kRowBlock, rr = e % kRowBlock, r = r0 + rr;
+            const size_t ts = (size_t)bh * S + a + s;
+            float x = 0.f;
+            if (r < DH) x = REVERSE ? p.dnum[ts * DH + r] : bwd::ld(v, ts * DH + r);
+            else if (r == DH) x = REVERSE ? p.dnq[ts] : 1.f;
+            coef[s * kRowBlock + rr] = wt[s] * x;
+        }
+        __syncthreads();
+        const float decay = expf(p.Bsum[hc] + mprev - mend);
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < NCL; ++j) st[i][j] *= decay;
+        for (int s = 0; s < n; ++s) {
+            float kv[NCL];
+#pragma unroll
+            for (int j = 0; j < NCL; ++j) kv[j] = bwd::ld(tile, (size_t)s * DH + lane + 32 * j);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float cf = coef[s * kRowBlock + 4 * warp + i];
+#pragma unroll
+                for (int j = 0; j < NCL; ++j) st[i][j] += cf * kv[j];
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int r = r0 + 4 * warp + i;
+            if (r > DH) continue;
+            float *dst = slot_ptr(r, REVERSE ? c - 1 : c + 1);
+#pragma unroll
+            for (int j = 0; j < NCL; ++j) dst[lane + 32 * j] = st[i][j];
+        }
+    }
+}
+
+template <typename T, bool REVERSE>
+bool launch_rows(const BwdPtrs &p, cudaStream_t st) {
+    const int ncl = p.DH / 32;
+    if (p.DH % 32 != 0 || (ncl != 1 && ncl != 2 && ncl != 4 && ncl != 8 && ncl != 16)) return false;
+    const size_t sm = rows_smem_bytes<T>(p.L, p.DH);
+    const dim3 grid((unsigned)((p.DH + 1 + kRowBlock - 1) / kRowBlock), (unsigned)p.BH);
+#define XLSTM_BWD_ROWS(N)                                                                         \
+    if (ncl == N) {                                                                                \
+        cudaFuncSetAttribute(bwd_rows_kernel<T, N, REVERSE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm); \
+        bwd_rows_kernel<T, N, REVERSE><<<grid, kRowThreads, sm, st>>>(p);                          \
+        return true;                                                                               \
+    }
+    XLSTM_BWD_ROWS(1)
+    XLSTM_BWD_ROWS(2)
+    XLSTM_BWD_ROWS(4)
+    XLSTM_BWD_ROWS(8)
+    XLSTM_BWD_ROWS(16)
+#undef XLSTM_BWD_ROWS
+    return false;
 }
 
 __global__ void __launch_bounds__(kThreads) bwd_forget_kernel(BwdPtrs p) {
@@ -118,7 +246,7 @@ cudaError_t launch_bwd(const BwdPtrs &p, cudaStream_t st) {
     }
     {
         KernelTimer timer("bwd_states", st);
-        bwd_states_kernel<T><<<blocks_for(rows), kThreads, 0, st>>>(p);
+        if (!launch_rows<T, false>(p, st)) bwd_states_kernel<T><<<blocks_for(rows), kThreads, 0, st>>>(p);
     }
     {
         KernelTimer timer("bwd_token_fwd", st);
@@ -126,7 +254,7 @@ cudaError_t launch_bwd(const BwdPtrs &p, cudaStream_t st) {
     }
     {
         KernelTimer timer("bwd_reverse", st);
-        bwd_reverse_kernel<T><<<blocks_for(rows), kThreads, 0, st>>>(p);
+        if (!launch_rows<T, true>(p, st)) bwd_reverse_kernel<T><<<blocks_for(rows), kThreads, 0, st>>>(p);
     }
     {
         KernelTimer timer("bwd_token_grad", st);

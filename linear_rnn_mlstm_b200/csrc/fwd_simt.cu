@@ -41,10 +41,18 @@ gate_prologue_kernel(const float *__restrict__ i_pre, const float *__restrict__ 
     const int t0 = c * L, t1 = min(S, t0 + L);
     const size_t base = (size_t)bh * S;
     float carry = 0.f, umax = -INFINITY;
+    // the next 32 tokens' gates are loaded while this group is scanned
+    float nf = t0 + lane < t1 ? f_pre[base + t0 + lane] : 0.f;
+    float ni = t0 + lane < t1 ? i_pre[base + t0 + lane] : 0.f;
     for (int t = t0; t < t1; t += 32) {
         const int tt = t + lane;
         const bool ok = tt < t1;
-        float lf = ok ? log_forget(f_pre[base + tt], fgate_exp) : 0.f;
+        const float fcur = nf, icur = ni;
+        if (t + 32 < t1) {
+            nf = tt + 32 < t1 ? f_pre[base + tt + 32] : 0.f;
+            ni = tt + 32 < t1 ? i_pre[base + tt + 32] : 0.f;
+        }
+        float lf = ok ? log_forget(fcur, fgate_exp) : 0.f;
         // inclusive warp scan
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
@@ -52,7 +60,7 @@ gate_prologue_kernel(const float *__restrict__ i_pre, const float *__restrict__ 
             if (lane >= o) lf += y;
         }
         const float b = carry + lf;
-        const float u_raw = ok ? i_pre[base + tt] - b : 0.f;
+        const float u_raw = ok ? icur - b : 0.f;
         float u = ok ? u_raw : -INFINITY;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {          // inclusive prefix max of u
