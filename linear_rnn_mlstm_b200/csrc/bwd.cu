@@ -3,14 +3,16 @@
 // Short-Term Memory" section 2.3; the stabiliser held fixed as section 2.2
 // allows).  Six launches, each a thin wrapper around a per-thread body in
 // bwd_body.cuh (the algorithm is described there):
-//   K1 bwd_gates       one thread per head     log f, chunk-local cumsum, m_t
+//   K1 bwd_gates       one warp per head       log f, chunk-local cumsum, m_t
 //   K2 bwd_states      one thread per state row  chunk-start states C'_c, n'_c
 //                      (DH a multiple of 32: one CTA per 32 rows, bwd_rows_kernel)
 //   K3 bwd_token_fwd   one thread per token    num', nq', den', dotilde, dnum', dnq'
+//                      (DH a multiple of 32: one warp per token)
 //   K4 bwd_reverse     one thread per state row  reverse state at each chunk end
 //                      (DH a multiple of 32: one CTA per 32 rows, bwd_rows_kernel)
 //   K5 bwd_token_grad  one thread per token    dq, dk, dv, ditilde
-//   K6 bwd_forget      one thread per head     dftilde (reverse cumulative sum)
+//                      (DH a multiple of 32: one warp per token)
+//   K6 bwd_forget      one warp per head       dftilde (reverse cumulative sum)
 // The chunk-start and reverse states are materialised in the workspace
 // (2 (NC + 1) DH^2 floats per head); this is the correctness-first form of the
 // backward, not a tuned one.
@@ -31,11 +33,6 @@ constexpr int kThreads = 128;
 
 __device__ __forceinline__ long long thread_index() {
     return (long long)blockIdx.x * blockDim.x + threadIdx.x;
-}
-
-__global__ void __launch_bounds__(kThreads) bwd_gates_kernel(BwdPtrs p) {
-    const long long i = thread_index();
-    if (i < p.BH) bwd::gates_head(p, (int)i);
 }
 
 template <typename T>
@@ -190,9 +187,363 @@ bool launch_rows(const BwdPtrs &p, cudaStream_t st) {
     return false;
 }
 
-__global__ void __launch_bounds__(kThreads) bwd_forget_kernel(BwdPtrs p) {
-    const long long i = thread_index();
-    if (i < p.BH) bwd::forget_head(p, (int)i);
+// K3 and K5 for DH a multiple of 32 (up to 512), one warp per token instead of
+// one thread: each lane takes the columns lane + 32 i, the dot products over
+// DH are warp sums, and the products with the chunk's DH x DH states are read
+// row by row in coalesced 128-byte pieces (row-indexed vectors come in as
+// uniform loads).  The same quantities as token_fwd / token_grad; only the
+// summation order inside each dot product differs.
+constexpr int kTokWarps = 8;
+
+__device__ __forceinline__ float wsum(float x) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+    return x;
+}
+
+template <typename T, int NCL>
+__global__ void __launch_bounds__(32 * kTokWarps) bwd_token_fwd_warp_kernel(BwdPtrs p) {
+    constexpr int DH = 32 * NCL;
+    __shared__ float s_ws[kTokWarps][bwd::kMaxChunk];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const long long gt = (long long)blockIdx.x * kTokWarps + warp;
+    if (gt >= (long long)p.BH * p.S) return;
+    const int bh = (int)(gt / p.S), t = (int)(gt % p.S);
+    const int S = p.S, L = p.L, NC = p.NC;
+    const size_t DD = (size_t)DH * DH;
+    const float inv_sqrt = 1.f / sqrtf((float)DH);
+    const T *q = (const T *)p.q, *k = (const T *)p.k, *v = (const T *)p.v, *dh = (const T *)p.dh;
+    const size_t ts = (size_t)bh * S + t;
+    const int c = t / L, a = c * L;
+    const size_t hc = (size_t)bh * NC + c;
+    const float m_t = p.mt[ts], b_t = p.b[ts];
+    const float g = expf(b_t + p.mprev[hc] - m_t);
+    const float *Cc = p.Cst + ((size_t)bh * (NC + 1) + c) * DD;
+    const float *nc = p.nst + ((size_t)bh * (NC + 1) + c) * DH;
+    float qv[NCL];
+#pragma unroll
+    for (int i = 0; i < NCL; ++i) qv[i] = bwd::ld(q, ts * DH + lane + 32 * i);
+    float *ws = s_ws[warp];
+    float nq = 0.f;
+    for (int s = a; s <= t; ++s) {
+        const size_t ss = (size_t)bh * S + s;
+        float dot = 0.f;
+#pragma unroll
+        for (int i = 0; i < NCL; ++i) dot += qv[i] * bwd::ld(k, ss * DH + lane + 32 * i);
+        dot = wsum(dot);
+        const float w = expf(b_t - p.b[ss] + p.ip[ss] - m_t) * dot * inv_sqrt;
+        if (lane == 0) ws[s - a] = w;
+        nq += w;
+    }
+    __syncwarp();
+    float ni = 0.f;
+#pragma unroll
+    for (int i = 0; i < NCL; ++i) ni += nc[lane + 32 * i] * qv[i];
+    nq += g * wsum(ni);
+    // num'[r]: lane r % 32 keeps row r = lane + 32 i
+    float num[NCL];
+#pragma unroll
+    for (int i = 0; i < NCL; ++i) num[i] = 0.f;
+#pragma unroll
+    for (int rb = 0; rb < NCL; ++rb) {
+        for (int rl = 0; rl < 32; ++rl) {
+            const int r = 32 * rb + rl;
+            float part = 0.f;
+#pragma unroll
+            for (int i = 0; i < NCL; ++i) part += Cc[(size_t)r * DH + lane + 32 * i] * qv[i];
+            part = wsum(part);
+            if (rl == lane) num[rb] = part;
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < NCL; ++i) {
+        const int r = lane + 32 * i;
+        float acc = num[i] * g;
+        for (int s = a; s <= t; ++s) acc += ws[s - a] * bwd::ld(v, ((size_t)bh * S + s) * DH + r);
+        num[i] = acc;
+        p.num[ts * DH + r] = acc;
+    }
+    const float floor_ = expf(-m_t);
+    const float den = fmaxf(fabsf(nq), floor_);
+    float sdot = 0.f, A = 0.f;
+#pragma unroll
+    for (int i = 0; i < NCL; ++i) {
+        const int r = lane + 32 * i;
+        const float o = bwd::sigmoid_hd(p.op[ts * DH + r]);
+        const float hv = num[i] / den;
+        const float dhr = bwd::ld(dh, ts * DH + r);
+        const float dht = dhr * o;
+        p.dO[ts * DH + r] = dhr * hv * o * (1.f - o);
+        const float dn_r = dht / den;
+        p.dnum[ts * DH + r] = dn_r;
+        sdot += dht * hv;
+        A += dn_r * num[i];
+    }
+    sdot = wsum(sdot);
+    A = wsum(A);
+    if (lane == 0) {
+        const float dnq = fabsf(nq) > floor_ ? -sdot / den * (nq > 0.f ? 1.f : -1.f) : 0.f;
+        p.dnq[ts] = dnq;
+        p.nq[ts] = nq;
+        p.den[ts] = den;
+        p.A[ts] = A + dnq * nq;
+    }
+}
+
+template <typename T, int NCL>
+__global__ void __launch_bounds__(32 * kTokWarps) bwd_token_grad_warp_kernel(BwdPtrs p) {
+    constexpr int DH = 32 * NCL;
+    __shared__ float s_w[kTokWarps][3][bwd::kMaxChunk];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const long long gs = (long long)blockIdx.x * kTokWarps + warp;
+    if (gs >= (long long)p.BH * p.S) return;
+    const int bh = (int)(gs / p.S), s = (int)(gs % p.S);
+    const int S = p.S, L = p.L, NC = p.NC;
+    const size_t DD = (size_t)DH * DH;
+    const float inv_sqrt = 1.f / sqrtf((float)DH);
+    const T *q = (const T *)p.q, *k = (const T *)p.k, *v = (const T *)p.v;
+    T *dq = (T *)p.dq, *dk = (T *)p.dk, *dv = (T *)p.dv;
+    const size_t ss = (size_t)bh * S + s;
+    const int c = s / L, a = c * L, e = bwd::imin(S, a + L);
+    const size_t hc = (size_t)bh * NC + c;
+    const float m_s = p.mt[ss], b_s = p.b[ss], i_s = p.ip[ss];
+    const float *dnum_s = p.dnum + ss * DH;
+    float *wdp_a = s_w[warp][0], *wdp_b = s_w[warp][1], *wsc_b = s_w[warp][2];
+    float dns[NCL], vs[NCL], ks[NCL];
+#pragma unroll
+    for (int i = 0; i < NCL; ++i) {
+        const int j = lane + 32 * i;
+        dns[i] = dnum_s[j];
+        vs[i] = bwd::ld(v, ss * DH + j);
+        ks[i] = bwd::ld(k, ss * DH + j);
+    }
+    const float dnq_s = p.dnq[ss];
+    for (int u = a; u <= s; ++u) {
+        const size_t us = (size_t)bh * S + u;
+        float dot = 0.f;
+#pragma unroll
+        for (int i = 0; i < NCL; ++i) dot += dns[i] * bwd::ld(v, us * DH + lane + 32 * i);
+        dot = wsum(dot);
+        if (lane == 0) wdp_a[u - a] = expf(b_s - p.b[us] + p.ip[us] - m_s) * (dot + dnq_s);
+    }
+    for (int t = s; t < e; ++t) {
+        const size_t tt = (size_t)bh * S + t;
+        float dot = 0.f, sc = 0.f;
+#pragma unroll
+        for (int i = 0; i < NCL; ++i) {
+            const int j = lane + 32 * i;
+            dot += p.dnum[tt * DH + j] * vs[i];
+            sc += bwd::ld(q, tt * DH + j) * ks[i];
+        }
+        dot = wsum(dot);
+        sc = wsum(sc);
+        if (lane == 0) {
+            const float w = expf(p.b[tt] - b_s + i_s - p.mt[tt]);
+            wdp_b[t - s] = w * (dot + p.dnq[tt]);
+            wsc_b[t - s] = w * sc * inv_sqrt;
+        }
+    }
+    __syncwarp();
+    const float g = expf(b_s + p.mprev[hc] - m_s);
+    const float wk = expf(p.Bsum[hc] - b_s + i_s - p.mend[hc]);
+    const float *Cc = p.Cst + ((size_t)bh * (NC + 1) + c) * DD;
+    const float *ncs = p.nst + ((size_t)bh * (NC + 1) + c) * DH;
+    const float *dCc = p.dCb + ((size_t)bh * NC + c) * DD;
+    const float *dnc = p.dnb + ((size_t)bh * NC + c) * DH;
+    // dq and dk: lanes own the key columns j; the states are read row by row
+    float aq[NCL], ak[NCL], inter[NCL], rv[NCL];
+#pragma unroll
+    for (int i = 0; i < NCL; ++i) aq[i] = ak[i] = inter[i] = rv[i] = 0.f;
+    for (int u = a; u <= s; ++u) {
+        const float w = wdp_a[u - a];
+#pragma unroll
+        for (int i = 0; i < NCL; ++i) aq[i] += w * bwd::ld(k, ((size_t)bh * S + u) * DH + lane + 32 * i);
+    }
+    for (int t = s; t < e; ++t) {
+        const float w = wdp_b[t - s];
+#pragma unroll
+        for (int i = 0; i < NCL; ++i) ak[i] += w * bwd::ld(q, ((size_t)bh * S + t) * DH + lane + 32 * i);
+    }
+    for (int r = 0; r < DH; ++r) {
+        const float dr = dnum_s[r], vr = bwd::ld(v, ss * DH + r);
+#pragma unroll
+        for (int i = 0; i < NCL; ++i) {
+            inter[i] += Cc[(size_t)r * DH + lane + 32 * i] * dr;
+            rv[i] += dCc[(size_t)r * DH + lane + 32 * i] * vr;
+        }
+    }
+    float di = 0.f;
+#pragma unroll
+    for (int i = 0; i < NCL; ++i) {
+        const int j = lane + 32 * i;
+        const float dqj = aq[i] * inv_sqrt + g * (inter[i] + dnq_s * ncs[j]);
+        bwd::st(dq, ss * DH + j, dqj);
+        const float dkh = ak[i] + wk * (rv[i] + dnc[j]);
+        di += dkh * ks[i] * inv_sqrt;
+        bwd::st(dk, ss * DH + j, dkh * inv_sqrt);
+    }
+    di = wsum(di);
+    // dv: lanes own the value rows r = lane + 32 i; dC k_s by one warp sum per row
+    float av[NCL];
+#pragma unroll
+    for (int i = 0; i < NCL; ++i) av[i] = 0.f;
+    for (int t = s; t < e; ++t) {
+        const float w = wsc_b[t - s];
+#pragma unroll
+        for (int i = 0; i < NCL; ++i) av[i] += w * p.dnum[((size_t)bh * S + t) * DH + lane + 32 * i];
+    }
+#pragma unroll
+    for (int rb = 0; rb < NCL; ++rb) {
+        for (int rl = 0; rl < 32; ++rl) {
+            const int r = 32 * rb + rl;
+            float part = 0.f;
+#pragma unroll
+            for (int i = 0; i < NCL; ++i) part += dCc[(size_t)r * DH + lane + 32 * i] * ks[i];
+            part = wsum(part);
+            if (rl == lane) av[rb] += wk * part * inv_sqrt;
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < NCL; ++i) bwd::st(dv, ss * DH + lane + 32 * i, av[i]);
+    if (lane == 0) {
+        p.di[ss] = di;
+        p.dF[ss] = p.A[ss] - di;
+    }
+}
+
+template <typename T, bool GRAD>
+bool launch_token_warp(const BwdPtrs &p, cudaStream_t st) {
+    const int ncl = p.DH / 32;
+    if (p.DH % 32 != 0 || (ncl != 1 && ncl != 2 && ncl != 4 && ncl != 8 && ncl != 16)) return false;
+    const long long tokens = (long long)p.BH * p.S;
+    const unsigned blocks = (unsigned)((tokens + kTokWarps - 1) / kTokWarps);
+#define XLSTM_BWD_TOK(N)                                                                          \
+    if (ncl == N) {                                                                                \
+        if (GRAD) bwd_token_grad_warp_kernel<T, N><<<blocks, 32 * kTokWarps, 0, st>>>(p);          \
+        else bwd_token_fwd_warp_kernel<T, N><<<blocks, 32 * kTokWarps, 0, st>>>(p);                \
+        return true;                                                                               \
+    }
+    XLSTM_BWD_TOK(1)
+    XLSTM_BWD_TOK(2)
+    XLSTM_BWD_TOK(4)
+    XLSTM_BWD_TOK(8)
+    XLSTM_BWD_TOK(16)
+#undef XLSTM_BWD_TOK
+    return false;
+}
+
+// K1 and K6 with one warp per head instead of one thread: 32 tokens at a time
+// with warp scans.  K1's stabiliser uses the unrolled form of the recurrence,
+// m_t = b_t + max(m_prev, max_{s <= t in the chunk} (itilde_s - b_s)) with b
+// chunk-local (equal to the sequential max-plus recurrence up to rounding; the
+// backward only needs one consistent m with all exponents <= 0).
+__global__ void __launch_bounds__(128) bwd_gates_warp_kernel(BwdPtrs p) {
+    const long long w = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (w >= p.BH) return;
+    const int bh = (int)w, S = p.S, L = p.L;
+    const size_t base = (size_t)bh * S, cbase = (size_t)bh * p.NC;
+    float m = 0.f;
+    for (int c = 0; c < p.NC; ++c) {
+        const int a = c * L, e = bwd::imin(S, a + L);
+        float carry = 0.f, umax = -INFINITY, mlast = m;
+        if (lane == 0) p.mprev[cbase + c] = m;
+        for (int t0 = a; t0 < e; t0 += 32) {
+            const int t = t0 + lane;
+            const bool ok = t < e;
+            const float fpre = ok ? p.fp[base + t] : 0.f;
+            const float lf = ok ? (p.fgate_exp ? fpre : bwd::log_sigmoid_hd(fpre)) : 0.f;
+            float b = lf;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const float y = __shfl_up_sync(0xffffffffu, b, o);
+                if (lane >= o) b += y;
+            }
+            b += carry;
+            float u = ok ? p.ip[base + t] - b : -INFINITY;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const float y = __shfl_up_sync(0xffffffffu, u, o);
+                if (lane >= o) u = fmaxf(u, y);
+            }
+            u = fmaxf(u, umax);
+            const float mt = b + fmaxf(m, u);
+            if (ok) {
+                p.logf[base + t] = lf;
+                p.b[base + t] = b;
+                p.mt[base + t] = mt;
+            }
+            const int last = bwd::imin(31, e - 1 - t0);
+            carry = __shfl_sync(0xffffffffu, b, last);
+            umax = __shfl_sync(0xffffffffu, u, last);
+            mlast = __shfl_sync(0xffffffffu, mt, last);
+        }
+        if (lane == 0) {
+            p.mend[cbase + c] = mlast;
+            p.Bsum[cbase + c] = carry;
+        }
+        m = mlast;
+    }
+}
+
+__global__ void __launch_bounds__(128) bwd_forget_warp_kernel(BwdPtrs p) {
+    const long long w = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (w >= p.BH) return;
+    const int bh = (int)w, S = p.S, DH = p.DH, NC = p.NC;
+    const size_t base = (size_t)bh * S, DD = (size_t)DH * DH;
+    if (p.dC || p.dn) {
+        float a_final = 0.f;
+        const float *CT = p.Cst + ((size_t)bh * (NC + 1) + NC) * DD;
+        const float *nT = p.nst + ((size_t)bh * (NC + 1) + NC) * DH;
+        if (p.dC)
+            for (size_t i = lane; i < DD; i += 32) a_final += p.dC[(size_t)bh * DD + i] * CT[i];
+        if (p.dn)
+            for (int j = lane; j < DH; j += 32) a_final += p.dn[(size_t)bh * DH + j] * nT[j];
+        a_final = wsum(a_final);
+        // the first t with the largest itilde_t - F_t, if that is > 0 (m_T's maximising key)
+        float F0 = 0.f, best = 0.f;
+        int sstar = -1;
+        for (int t0 = 0; t0 < S; t0 += 32) {
+            const int t = t0 + lane;
+            float F = t < S ? p.logf[base + t] : 0.f;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const float y = __shfl_up_sync(0xffffffffu, F, o);
+                if (lane >= o) F += y;
+            }
+            F += F0;
+            float cand = t < S ? p.ip[base + t] - F : -INFINITY;
+            int ct = t;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {             // max, earliest token on ties
+                const float oc = __shfl_xor_sync(0xffffffffu, cand, o);
+                const int ot = __shfl_xor_sync(0xffffffffu, ct, o);
+                if (oc > cand || (oc == cand && ot < ct)) { cand = oc; ct = ot; }
+            }
+            if (cand > best) { best = cand; sstar = ct; }
+            F0 = __shfl_sync(0xffffffffu, F, 31);
+        }
+        if (lane == 0 && sstar >= 0) {
+            p.di[base + sstar] -= a_final;
+            p.dF[base + sstar] += a_final;
+        }
+        __syncwarp();
+    }
+    float acc = 0.f;                                     // reverse cumulative sum of dF
+    const int ng = (S + 31) / 32;
+    for (int gi = ng - 1; gi >= 0; --gi) {
+        const int t = gi * 32 + lane;
+        float x = t < S ? p.dF[base + t] : 0.f;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const float y = __shfl_down_sync(0xffffffffu, x, o);
+            if (lane + o < 32) x += y;
+        }
+        x += acc;
+        if (t < S) p.df[base + t] = p.fgate_exp ? x : x * bwd::sigmoid_hd(-p.fp[base + t]);
+        acc = __shfl_sync(0xffffffffu, x, 0);
+    }
 }
 
 size_t align64(size_t x) { return (x + 63) & ~size_t(63); }
@@ -242,7 +593,7 @@ cudaError_t launch_bwd(const BwdPtrs &p, cudaStream_t st) {
                     tokens = (long long)p.BH * p.S;
     {
         KernelTimer timer("bwd_gates", st);
-        bwd_gates_kernel<<<blocks_for(heads), kThreads, 0, st>>>(p);
+        bwd_gates_warp_kernel<<<(unsigned)((heads * 32 + 127) / 128), 128, 0, st>>>(p);
     }
     {
         KernelTimer timer("bwd_states", st);
@@ -250,7 +601,7 @@ cudaError_t launch_bwd(const BwdPtrs &p, cudaStream_t st) {
     }
     {
         KernelTimer timer("bwd_token_fwd", st);
-        bwd_token_fwd_kernel<T><<<blocks_for(tokens), kThreads, 0, st>>>(p);
+        if (!launch_token_warp<T, false>(p, st)) bwd_token_fwd_kernel<T><<<blocks_for(tokens), kThreads, 0, st>>>(p);
     }
     {
         KernelTimer timer("bwd_reverse", st);
@@ -258,11 +609,11 @@ cudaError_t launch_bwd(const BwdPtrs &p, cudaStream_t st) {
     }
     {
         KernelTimer timer("bwd_token_grad", st);
-        bwd_token_grad_kernel<T><<<blocks_for(tokens), kThreads, 0, st>>>(p);
+        if (!launch_token_warp<T, true>(p, st)) bwd_token_grad_kernel<T><<<blocks_for(tokens), kThreads, 0, st>>>(p);
     }
     {
         KernelTimer timer("bwd_forget", st);
-        bwd_forget_kernel<<<blocks_for(heads), kThreads, 0, st>>>(p);
+        bwd_forget_warp_kernel<<<(unsigned)((heads * 32 + 127) / 128), 128, 0, st>>>(p);
     }
     return cudaGetLastError();
 }
