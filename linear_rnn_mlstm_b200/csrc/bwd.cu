@@ -73,22 +73,77 @@ constexpr int kRowBlock = 32;
 constexpr int kRowThreads = 256;      // 8 warps x 4 rows
 
 template <typename T>
-size_t rows_smem_bytes(int L, int DH) { return (size_t)L * DH * sizeof(T) + (size_t)L * (kRowBlock + 1) * 4; }
+__host__ __device__ size_t rows_stage_bytes(int L, int DH) {     // a multiple of 128 bytes
+    return ((size_t)L * DH * sizeof(T) + (size_t)L * kRowBlock * 4 + (size_t)3 * L * 4 + 127) & ~(size_t)127;
+}
+template <typename T>
+size_t rows_smem_bytes(int L, int DH) { return 2 * rows_stage_bytes<T>(L, DH) + (size_t)L * kRowBlock * 4; }
 
+__device__ __forceinline__ uint32_t tc_smem_u32(const void *ptr) {
+    return (uint32_t)__cvta_generic_to_shared(ptr);
+}
+__device__ __forceinline__ void cp_async16(void *dst, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(tc_smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async4(void *dst, const void *src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(tc_smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N> __device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// Stages (two, by chunk parity) hold a chunk's key (K2) or query (K4) tile, the
+// 32 rows' raw coefficients (v or dnum' entries) and the per-token scalars;
+// the next chunk's stage is filled by cp.async while this one is used, so the
+// walk over chunks waits on no global-memory round trip.
 template <typename T, int NCL, bool REVERSE>
 __global__ void __launch_bounds__(kRowThreads) bwd_rows_kernel(BwdPtrs p) {
     constexpr int DH = 32 * NCL;
     extern __shared__ __align__(16) uint8_t rows_smem[];
     const int L = p.L, S = p.S, NC = p.NC;
-    T *tile = reinterpret_cast<T *>(rows_smem);                           // [L][DH]
-    float *coef = reinterpret_cast<float *>(rows_smem + (size_t)L * DH * sizeof(T));   // [L][32]
-    float *wt = coef + (size_t)L * kRowBlock;                             // [L] per-token weight
+    const size_t stage_bytes = rows_stage_bytes<T>(L, DH);
+    float *coef = reinterpret_cast<float *>(rows_smem + 2 * stage_bytes);     // [L][32]
     const int bh = blockIdx.y, r0 = blockIdx.x * kRowBlock;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const size_t DD = (size_t)DH * DH;
     const float inv_sqrt = 1.f / sqrtf((float)DH);
     const T *src = (const T *)(REVERSE ? p.q : p.k);
     const T *v = (const T *)p.v;
+    auto stage = [&](int buf, T *&tile, float *&raw, float *&sc) {
+        uint8_t *base = rows_smem + buf * stage_bytes;
+        tile = reinterpret_cast<T *>(base);
+        raw = reinterpret_cast<float *>(base + (size_t)L * DH * sizeof(T));
+        sc = raw + (size_t)L * kRowBlock;                                   // [3][L]
+    };
+    // the copies of chunk c into stage buf
+    auto issue = [&](int c, int buf) {
+        T *tile; float *raw, *sc;
+        stage(buf, tile, raw, sc);
+        const int a = c * L, n = bwd::imin(S, a + L) - a;
+        const size_t row0 = (size_t)bh * S + a;
+        constexpr int EPV = 16 / (int)sizeof(T);                            // elements per 16 bytes
+        for (int e = threadIdx.x; e < n * DH / EPV; e += kRowThreads)
+            cp_async16(tile + (size_t)e * EPV, src + row0 * DH + (size_t)e * EPV);
+        for (int e = threadIdx.x; e < n * kRowBlock; e += kRowThreads) {
+            const int s = e / kRowBlock, rr = e % kRowBlock, r = r0 + rr;
+            const size_t ts = row0 + s;
+            if (r < DH) {
+                if (REVERSE) cp_async4(raw + e, p.dnum + ts * DH + r);
+                else if (sizeof(T) == 4) cp_async4(raw + e, v + ts * DH + r);
+                else    // bf16: the 4-byte word holding element r (picked apart below)
+                    cp_async4(raw + e, reinterpret_cast<const uint8_t *>(v) + ((ts * DH + r) & ~(size_t)1) * 2);
+            } else {
+                if (REVERSE && r == DH) cp_async4(raw + e, p.dnq + ts);
+                else raw[e] = r == DH ? 1.f : 0.f;
+            }
+        }
+        for (int s = threadIdx.x; s < n; s += kRowThreads) {
+            cp_async4(sc + s, p.b + row0 + s);
+            if (REVERSE) cp_async4(sc + L + s, p.mt + row0 + s);
+            else cp_async4(sc + L + s, p.ip + row0 + s);
+        }
+    };
     // this warp's rows r0 + 4 warp + i (row DH is the normaliser; rows past it unused)
     float st[4][NCL];
     auto slot_ptr = [&](int r, int slot) -> float * {
@@ -110,38 +165,45 @@ __global__ void __launch_bounds__(kRowThreads) bwd_rows_kernel(BwdPtrs p) {
             if (r <= DH) slot_ptr(r, REVERSE ? NC - 1 : 0)[col] = x;
         }
     }
-    const int c_first = REVERSE ? NC - 1 : 0, c_end = REVERSE ? 0 : NC, dir = REVERSE ? -1 : 1;
-    for (int c = c_first; c != c_end; c += dir) {
-        const size_t hc = (size_t)bh * NC + c;
+    // chunks walked: 0 .. NC-1 forward; NC-1 .. 1 in reverse (slot c-1 from chunk c)
+    const int nsteps = REVERSE ? NC - 1 : NC;
+    auto chunk_of = [&](int k) { return REVERSE ? NC - 1 - k : k; };
+    if (nsteps > 0) issue(chunk_of(0), 0);
+    cp_async_commit();
+    // the chunk scalars are loaded one chunk ahead too (a barrier would wait for them)
+    float nBs = 0.f, nmprev = 0.f, nmend = 0.f;
+    if (nsteps > 0) {
+        const size_t h0 = (size_t)bh * NC + chunk_of(0);
+        nBs = p.Bsum[h0]; nmprev = p.mprev[h0]; nmend = p.mend[h0];
+    }
+    for (int k = 0; k < nsteps; ++k) {
+        const int c = chunk_of(k), buf = k & 1;
+        const float Bs = nBs, mprev = nmprev, mend = nmend;
+        __syncthreads();                       // everyone is done with stage buf ^ 1 and the coefficients
+        if (k + 1 < nsteps) issue(chunk_of(k + 1), buf ^ 1);
+        cp_async_commit();
+        cp_async_wait<1>();                    // this chunk's copies (the newest group may still fly)
+        __syncthreads();
+        T *tile; float *raw, *sc;
+        stage(buf, tile, raw, sc);
         const int a = c * L, n = bwd::imin(S, a + L) - a;
-        __syncthreads();                       // the previous chunk's tile and coefficients are read
-        for (int e = threadIdx.x; e < n * DH / 8; e += kRowThreads) {
-            const int s = e / (DH / 8), part = e % (DH / 8);
-            const size_t g = ((size_t)bh * S + a + s) * DH + part * 8;
-            if (sizeof(T) == 2) {
-                reinterpret_cast<uint4 *>(tile)[(size_t)s * DH / 8 + part] = *reinterpret_cast<const uint4 *>(src + g);
-            } else {
-                reinterpret_cast<uint4 *>(tile)[(size_t)s * DH / 4 + 2 * part] = *reinterpret_cast<const uint4 *>(src + g);
-                reinterpret_cast<uint4 *>(tile)[(size_t)s * DH / 4 + 2 * part + 1] =
-                    *reinterpret_cast<const uint4 *>(src + g + 4);
-            }
-        }
-        const float mend = p.mend[hc], mprev = p.mprev[hc];
-        for (int s = threadIdx.x; s < n; s += kRowThreads) {
-            const size_t ts = (size_t)bh * S + a + s;
-            wt[s] = REVERSE ? expf(p.b[ts] + mprev - p.mt[ts]) : expf(p.Bsum[hc] - p.b[ts] + p.ip[ts] - mend) * inv_sqrt;
-        }
-        __syncthreads();
         for (int e = threadIdx.x; e < n * kRowBlock; e += kRowThreads) {
-            const int s = e / kRowBlock, rr = e % kRowBlock, r = r0 + rr;
-            const size_t ts = (size_t)bh * S + a + s;
-            float x = 0.f;
-            if (r < DH) x = REVERSE ? p.dnum[ts * DH + r] : bwd::ld(v, ts * DH + r);
-            else if (r == DH) x = REVERSE ? p.dnq[ts] : 1.f;
-            coef[s * kRowBlock + rr] = wt[s] * x;
+            const int s = e / kRowBlock, r = r0 + e % kRowBlock;
+            const float w = REVERSE ? expf(sc[s] + mprev - sc[L + s])
+                                    : expf(Bs - sc[s] + sc[L + s] - mend) * inv_sqrt;
+            float x = raw[e];
+            if (!REVERSE && sizeof(T) == 2 && r < DH) {
+                const uint32_t word = __float_as_uint(x);
+                x = __uint_as_float((r & 1) ? (word & 0xffff0000u) : (word << 16));
+            }
+            coef[e] = w * x;
         }
         __syncthreads();
-        const float decay = expf(p.Bsum[hc] + mprev - mend);
+        if (k + 1 < nsteps) {                  // in flight during this chunk's products
+            const size_t hn = (size_t)bh * NC + chunk_of(k + 1);
+            nBs = p.Bsum[hn]; nmprev = p.mprev[hn]; nmend = p.mend[hn];
+        }
+        const float decay = expf(Bs + mprev - mend);
 #pragma unroll
         for (int i = 0; i < 4; ++i)
 #pragma unroll
@@ -166,6 +228,7 @@ __global__ void __launch_bounds__(kRowThreads) bwd_rows_kernel(BwdPtrs p) {
             for (int j = 0; j < NCL; ++j) dst[lane + 32 * j] = st[i][j];
         }
     }
+    cp_async_wait<0>();
 }
 
 template <typename T, bool REVERSE>
@@ -173,6 +236,7 @@ bool launch_rows(const BwdPtrs &p, cudaStream_t st) {
     const int ncl = p.DH / 32;
     if (p.DH % 32 != 0 || (ncl != 1 && ncl != 2 && ncl != 4 && ncl != 8 && ncl != 16)) return false;
     const size_t sm = rows_smem_bytes<T>(p.L, p.DH);
+    if (sm > 232448) return false;        // two stages do not fit (fp32 at DH 512): per-thread kernel
     const dim3 grid((unsigned)((p.DH + 1 + kRowBlock - 1) / kRowBlock), (unsigned)p.BH);
 #define XLSTM_BWD_ROWS(N)                                                                         \
     if (ncl == N) {                                                                                \

@@ -1,4 +1,4 @@
-// sLSTM forward on a cluster of CTAs per (batch, head), for DH 64, 128 or 256
+// sLSTM forward on a cluster of CTAs per (batch, head), for DH 64, 128, 256 or 512
 // ("xLSTM: Extended Long Short-Term Memory" section 2.2: scalar memory cells
 // with exponential gating and memory mixing through recurrent connections
 // within a head; the per-unit step is the one written out in slstm_body.cuh).
@@ -47,6 +47,16 @@ __device__ __forceinline__ void st_cluster(float *local, uint32_t rank, float v)
     asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(remote), "f"(v) : "memory");
 }
 
+// Columns per lane held in registers; at DH 512 (a 16-CTA cluster) the other
+// eight per lane live in shared memory (128 KB per CTA), laid out so that a
+// lane reads only its own words: [warp][row][column - 8][lane].
+template <int DH> struct ClSplit {
+    static constexpr int NC = DH / 32;                  // columns per lane
+    static constexpr int NREG = NC < 8 ? NC : 8;
+    static constexpr int NSM = NC - NREG;
+    static constexpr size_t kSmem = (size_t)(kClThreads / 32) * 16 * NSM * 32 * 4;
+};
+
 template <int DH>
 __global__ void __launch_bounds__(kClThreads, 1)
 slstm_cluster_kernel(const __grid_constant__ CUtensorMap map_z, const __grid_constant__ CUtensorMap map_i,
@@ -54,6 +64,8 @@ slstm_cluster_kernel(const __grid_constant__ CUtensorMap map_z, const __grid_con
                      slstm::SlstmPtrs p, unsigned int *status) {
     constexpr int CS = DH / 32;                  // CTAs per cluster
     constexpr int NC = DH / 32;                  // columns per lane
+    constexpr int NREG = ClSplit<DH>::NREG, NSM = ClSplit<DH>::NSM;
+    extern __shared__ __align__(16) float rsm[];   // [8 warps][16 rows][NSM][32 lanes]
     __shared__ __align__(128) float pre[kClStages][4][kClSteps][32];   // gate pre-activations
     __shared__ __align__(16) float hbuf[2][DH];                       // h_{t-1} / h_t of the whole head
     __shared__ __align__(8) uint64_t full[kClStages];
@@ -68,7 +80,8 @@ slstm_cluster_kernel(const __grid_constant__ CUtensorMap map_z, const __grid_con
     const int nblk = (S + kClSteps - 1) / kClSteps;
 
     // the warp's 16 rows (row r = 4 u + g: unit 4 warp + u, gate g in z, i, f, o)
-    float Rr[16][NC];
+    float Rr[16][NREG];
+    float *Rs = rsm + (size_t)warp * 16 * NSM * 32;
     {
         const size_t DD = (size_t)DH * DH;
 #pragma unroll
@@ -76,7 +89,9 @@ slstm_cluster_kernel(const __grid_constant__ CUtensorMap map_z, const __grid_con
             const int jr = (int)rank * 32 + 4 * warp + (r >> 2);
             const float *row = p.R + ((size_t)head * 4 + (r & 3)) * DD + (size_t)jr * DH;
 #pragma unroll
-            for (int k = 0; k < NC; ++k) Rr[r][k] = __ldg(row + lane + 32 * k);
+            for (int k = 0; k < NREG; ++k) Rr[r][k] = __ldg(row + lane + 32 * k);
+#pragma unroll
+            for (int k = 0; k < NSM; ++k) Rs[(r * NSM + k) * 32 + lane] = __ldg(row + lane + 32 * (NREG + k));
         }
     }
     float c = 0.f, n = 0.f, m = 0.f;
@@ -130,7 +145,9 @@ slstm_cluster_kernel(const __grid_constant__ CUtensorMap map_z, const __grid_con
         for (int r = 0; r < 16; ++r) {
             float a = 0.f;
 #pragma unroll
-            for (int k = 0; k < NC; ++k) a = fmaf(Rr[r][k], hc[k], a);
+            for (int k = 0; k < NREG; ++k) a = fmaf(Rr[r][k], hc[k], a);
+#pragma unroll
+            for (int k = 0; k < NSM; ++k) a = fmaf(Rs[(r * NSM + k) * 32 + lane], hc[NREG + k], a);
             v[r] = a;
         }
         // halving butterfly: after it lanes 2r and 2r + 1 hold row r's total
@@ -198,10 +215,18 @@ cudaError_t launch_cluster_t(const slstm::SlstmPtrs &p, cudaStream_t st) {
                     !make_tensor_map_3d(&mf, p.fx, 4, dims, strides, box) ||
                     !make_tensor_map_3d(&mo, p.ox, 4, dims, strides, box)))
         return cudaErrorInvalidValue;
+    const int sm = (int)ClSplit<DH>::kSmem;
+    cudaError_t e;
+    if (sm > 0 && (e = cudaFuncSetAttribute(slstm_cluster_kernel<DH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            sm)) != cudaSuccess)
+        return e;
+    if (DH / 32 > 8 && (e = cudaFuncSetAttribute(slstm_cluster_kernel<DH>,
+                                                 cudaFuncAttributeNonPortableClusterSizeAllowed, 1)) != cudaSuccess)
+        return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)p.BH * (DH / 32));
     cfg.blockDim = dim3(kClThreads);
-    cfg.dynamicSmemBytes = 0;
+    cfg.dynamicSmemBytes = (size_t)sm;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -215,13 +240,43 @@ cudaError_t launch_cluster_t(const slstm::SlstmPtrs &p, cudaStream_t st) {
 
 }  // namespace
 
-bool slstm_cluster_supports(int DH) { return DH == 64 || DH == 128 || DH == 256; }
+// DH 512 needs a 16-CTA cluster (beyond the portable 8): taken only where the
+// device can place one with this kernel's resources.
+bool slstm_cluster_supports(int DH) {
+    if (DH == 64 || DH == 128 || DH == 256) return true;
+    if (DH != 512) return false;
+    static int ok = -1;
+    if (ok < 0) {
+        int n = 0;
+        const int sm = (int)ClSplit<512>::kSmem;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(16);
+        cfg.blockDim = dim3(kClThreads);
+        cfg.dynamicSmemBytes = (size_t)sm;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 16;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        ok = cudaFuncSetAttribute(slstm_cluster_kernel<512>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm) ==
+                     cudaSuccess &&
+                 cudaFuncSetAttribute(slstm_cluster_kernel<512>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
+                     cudaSuccess &&
+                 cudaOccupancyMaxActiveClusters(&n, slstm_cluster_kernel<512>, &cfg) == cudaSuccess && n >= 1
+             ? 1 : 0;
+        cudaGetLastError();   // a refused query must not leak into a later launch check
+    }
+    return ok == 1;
+}
 
 cudaError_t launch_slstm_cluster(const slstm::SlstmPtrs &p, cudaStream_t st) {
     switch (p.DH) {
         case 64: return launch_cluster_t<64>(p, st);
         case 128: return launch_cluster_t<128>(p, st);
         case 256: return launch_cluster_t<256>(p, st);
+        case 512: return launch_cluster_t<512>(p, st);
     }
     return cudaErrorInvalidValue;
 }

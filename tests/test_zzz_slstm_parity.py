@@ -12,14 +12,15 @@ from test_slstm_emulation import compare, inputs, oracle_run
 
 pytestmark = pytest.mark.gpu
 
-# DH 64, 128 and 256 run on the cluster kernel (DH / 32 CTAs per head, the
-# recurrent blocks in registers, 16-step input stages: S below one stage, across
-# several and with a ragged last one); the other head sizes on the per-unit kernel.
+# DH 64, 128, 256 and 512 run on the cluster kernel (DH / 32 CTAs per head, the
+# recurrent blocks in registers, at DH 512 half of them in shared memory; 16-step
+# input stages: S below one stage, across several and with a ragged last one);
+# the other head sizes on the per-unit kernel.
 CASES = [(1, 2, 17, 16, "sigmoid", False), (2, 3, 9, 8, "exp", False),
          (1, 2, 33, 48, "sigmoid", True), (2, 4, 256, 64, "sigmoid", False),
          (1, 2, 40, 512, "exp", True), (1, 1, 1, 4, "exp", True),
          (1, 2, 100, 128, "exp", True), (2, 2, 70, 256, "sigmoid", True),
-         (1, 1, 5, 256, "exp", False), (3, 1, 33, 64, "exp", True)]
+         (1, 1, 5, 256, "exp", False), (3, 1, 33, 64, "exp", True), (2, 1, 37, 512, "sigmoid", False)]
 
 
 @pytest.mark.parametrize("B,NH,S,DH,fgate,state", CASES,
