@@ -61,13 +61,16 @@ template <int DH>
 __global__ void __launch_bounds__(kClThreads, 1)
 slstm_cluster_kernel(const __grid_constant__ CUtensorMap map_z, const __grid_constant__ CUtensorMap map_i,
                      const __grid_constant__ CUtensorMap map_f, const __grid_constant__ CUtensorMap map_o,
-                     slstm::SlstmPtrs p, unsigned int *status) {
+                     const __grid_constant__ CUtensorMap map_h, slstm::SlstmPtrs p, unsigned int *status) {
     constexpr int CS = DH / 32;                  // CTAs per cluster
     constexpr int NC = DH / 32;                  // columns per lane
     constexpr int NREG = ClSplit<DH>::NREG, NSM = ClSplit<DH>::NSM;
     extern __shared__ __align__(16) float rsm[];   // [8 warps][16 rows][NSM][32 lanes]
     __shared__ __align__(128) float pre[kClStages][4][kClSteps][32];   // gate pre-activations
     __shared__ __align__(16) float hbuf[2][DH];                       // h_{t-1} / h_t of the whole head
+    // this CTA's h of a 16-step block, sent out by one TMA store per block (a
+    // per-step global store would sit inside every step's release)
+    __shared__ __align__(128) float hst[2][kClSteps][32];
     __shared__ __align__(8) uint64_t full[kClStages];
     __shared__ int abort_flag;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -129,6 +132,10 @@ slstm_cluster_kernel(const __grid_constant__ CUtensorMap map_z, const __grid_con
             // the stage refilled here held block blk - 1, which every thread
             // finished before the cluster barrier that ended step t - 1
             if (threadIdx.x == 0 && issued < nblk && issued == blk + kClStages - 1) load_block(issued++);
+            if (blk >= 2) {                      // block blk - 2's h store has read hst[blk & 1]
+                if (threadIdx.x == 0) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+                __syncthreads();
+            }
             bool got = true;
             if (lane == 0) got = tc::mbar_wait(&full[s], (blk / kClStages) & 1, &abort_flag, status);
             got = __shfl_sync(0xffffffffu, got, 0);
@@ -182,12 +189,17 @@ slstm_cluster_kernel(const __grid_constant__ CUtensorMap map_z, const __grid_con
             c = fg * c + ig * zz;
             n = fg * n + ig;
             const float h = o * c / n;
-            p.h[((size_t)bh * S + t) * DH + j] = h;
+            hst[blk & 1][tin][ul] = h;
             float *dst = &hbuf[(t + 1) & 1][j];
 #pragma unroll
             for (int r2 = 0; r2 < CS; ++r2) st_cluster(dst, (uint32_t)r2, h);
         }
+        if (tin == kClSteps - 1 || t == S - 1) tc::fence_async_smem();   // hst visible to the TMA store
         cluster_sync_all();                      // h_t complete in every CTA
+        if (threadIdx.x == 0 && (tin == kClSteps - 1 || t == S - 1)) {
+            tc::tma_store_3d(&map_h, &hst[blk & 1][0][0], (int)rank * 32, blk * kClSteps, bh);
+            tc::bulk_commit();
+        }
     }
     if (!ok && lane == 0 && warp == 0) atomicOr(status, kStatusTimeout);
     if (unit_lane) {
@@ -197,6 +209,7 @@ slstm_cluster_kernel(const __grid_constant__ CUtensorMap map_z, const __grid_con
         if (p.m_out) p.m_out[s0] = m;
         if (p.h_out) p.h_out[s0] = hbuf[S & 1][j];
     }
+    if (threadIdx.x == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");   // h written
     if (threadIdx.x == 0) {                      // never leave a load in flight into shared memory
         for (int b = max(0, issued - kClStages); b < issued; ++b)
             tc::mbar_wait(&full[b % kClStages], (b / kClStages) & 1, nullptr, status, 200000000ull);
@@ -210,7 +223,9 @@ cudaError_t launch_cluster_t(const slstm::SlstmPtrs &p, cudaStream_t st) {
     const unsigned long long dims[3] = {(unsigned long long)DH, (unsigned long long)p.S, (unsigned long long)p.BH};
     const unsigned long long strides[2] = {(unsigned long long)DH * 4, (unsigned long long)p.S * DH * 4};
     const unsigned box[3] = {32u, (unsigned)kClSteps, 1u};
-    if (p.S > 0 && (!make_tensor_map_3d(&mz, p.zx, 4, dims, strides, box) ||
+    CUtensorMap mh;
+    if (p.S > 0 && (!make_tensor_map_3d(&mh, p.h, 4, dims, strides, box) ||
+                    !make_tensor_map_3d(&mz, p.zx, 4, dims, strides, box) ||
                     !make_tensor_map_3d(&mi, p.ix, 4, dims, strides, box) ||
                     !make_tensor_map_3d(&mf, p.fx, 4, dims, strides, box) ||
                     !make_tensor_map_3d(&mo, p.ox, 4, dims, strides, box)))
@@ -235,7 +250,7 @@ cudaError_t launch_cluster_t(const slstm::SlstmPtrs &p, cudaStream_t st) {
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, slstm_cluster_kernel<DH>, mz, mi, mf, mo, p, device_status_ptr());
+    return cudaLaunchKernelEx(&cfg, slstm_cluster_kernel<DH>, mz, mi, mf, mo, mh, p, device_status_ptr());
 }
 
 }  // namespace
