@@ -302,6 +302,7 @@ def main():
     ap.add_argument("--skip-cpu", action="store_true")
     ap.add_argument("--skip-slstm", action="store_true")
     ap.add_argument("--skip-backward", action="store_true")
+    ap.add_argument("--skip-seqpar", action="store_true")
     ap.add_argument("--skip-sweep", action="store_true",
                     help="skip the per-config / per-chunk entries (small, block, long at 128 and 256)")
     ap.add_argument("--ref-tokens", type=int, default=4096,
@@ -386,6 +387,11 @@ def main():
     if not args.skip_backward:
         backward = run_backward(args, dev, env, peaks, peak_src)
 
+    # ------------------------------------- sequence parallelism (next row)
+    seqpar_entry = None
+    if not args.skip_seqpar:
+        seqpar_entry = run_seqpar(args, dev, env)
+
     # ----------------------------------------------------------------- decode
     decode = None
     if not args.skip_decode:
@@ -416,6 +422,7 @@ def main():
                 "roofline": roofline, "tc": tc, "hbm_whole_step": whole,
                 "kernels": kernels, "gpu_launches": launches, "cpu_baseline": cpu, "e2e": e2e,
                 "clocks": clocks, "decode": decode, "epilogue": epilogue, "slstm": slstm, "backward": backward,
+                "sequence_parallel": seqpar_entry,
                 "sweep": sweep}
         print(json.dumps(line), flush=True)
     replicas.barrier(env)
@@ -682,6 +689,66 @@ def run_backward(args, dev, env, peaks, peak_src):
                     "kernels": {k: {"launches": v[0], "avg_us": 1e3 * v[1] / max(v[0], 1)}
                                 for k, v in kt.items()}})
         del x, dh
+    return out
+
+
+def run_seqpar(args, dev, env):
+    """Sequence parallelism on the long workload (B1 NH8 S16384 DH256 bf16, chunk
+    64): the one sequence cut into as many slices as there are ranks, each rank
+    summarising its slice, one all-gather of the summaries, a fold, and the
+    slice's forward (seqpar.sequence_parallel_fwd); time = max over ranks,
+    tokens/s over the whole sequence (strong scaling).  Beside it, measured on
+    this GPU, what each rank of an eight-way split runs: the summary of a
+    2048-token slice, the fold of seven summaries, and the slice's forward from
+    a folded state."""
+    from linear_rnn_mlstm_b200 import seqpar
+    w = syn.LONG
+    chunk = 64
+    world, rank = env.world, env.rank
+    inp = syn.fwd_inputs(w, seed=w.seed)             # every rank draws the same sequence
+    a, b = rank * w.S // world, (rank + 1) * w.S // world
+    x = {k: v[:, :, a:b].to(dev).contiguous() for k, v in inp.items()}
+    args_fwd = [x[k] for k in ("q", "k", "v", "i_pre", "f_pre", "o_pre")]
+    run = lambda: seqpar.sequence_parallel_fwd(*args_fwd, chunk=chunk, fgate=w.fgate)
+    for _ in range(max(3, args.warmup)):
+        run()
+    torch.cuda.synchronize(dev)
+    steps = max(3, min(args.steps, 10))
+    ms = time_region(run, steps, env, dev) / steps
+    tokens = w.B * w.NH * w.S
+    out = {"metric": "mLSTM fwd tokens/s, one sequence split over the ranks",
+           "value": tokens / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms, "n_ranks": world,
+           "scaling": "strong", "tokens_per_rank": w.B * w.NH * (b - a),
+           "config": f"long: B={w.B} NH={w.NH} S={w.S} DH={w.DH} bf16, chunk {chunk}, "
+                     f"S split into {world} slice(s)"}
+    del x, args_fwd
+    # one rank's share of an eight-way split, timed alone on this GPU
+    R = 8
+    Ss = w.S // R
+    sl = {k: v[:, :, :Ss].to(dev).contiguous() for k, v in inp.items()}
+    nf = xb.seg_state_floats(w.B, w.NH, w.DH)
+    parts = torch.zeros((R, nf), dtype=torch.float32, device=dev)
+    for r in range(R):
+        xb.mlstm_seg_state(sl["k"], sl["v"], sl["i_pre"], sl["f_pre"], chunk=chunk, fgate=w.fgate,
+                           packed=parts[r])
+    C, n, m = xb.mlstm_state_combine(parts, R - 1, w.B, w.NH, w.DH)
+    pieces = {
+        "seg_state": lambda: xb.mlstm_seg_state(sl["k"], sl["v"], sl["i_pre"], sl["f_pre"], chunk=chunk,
+                                                fgate=w.fgate, packed=parts[0]),
+        "state_combine_7": lambda: xb.mlstm_state_combine(parts, R - 1, w.B, w.NH, w.DH, out=(C, n, m)),
+        "fwd_from_state": lambda: xb.mlstm_fwd(*(sl[k] for k in ("q", "k", "v", "i_pre", "f_pre", "o_pre")),
+                                               chunk=chunk, fgate=w.fgate, C0=C, n0=n, m0=m),
+    }
+    share = {}
+    for name, fn in pieces.items():
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize(dev)
+        share[name + "_ms"] = time_region(fn, 10, env, dev) / 10
+    share["summary_bytes_per_rank"] = nf * 4
+    out["eight_way_rank_share"] = dict(share, slice_tokens=w.B * w.NH * Ss,
+                                       note="per-rank device time of an 8-GPU split (exchange of "
+                                            f"{R} x {nf * 4 / 1e6:.1f} MB not included)")
     return out
 
 

@@ -218,6 +218,61 @@ xlstm_status xlstm_mlstm_step(const void *q, const void *k, const void *v,
                               void *cuda_stream);
 
 /*
+ * Sequence parallelism: a sequence cut into consecutive slices, one per GPU
+ * (or per call), each slice's forward started from the state the slices before
+ * it leave.  Unrolling the recurrence of section 2.3 over a slice j that
+ * starts from the zero state summarises it as (C'_j, n'_j) under the slice's
+ * own stabiliser mloc_j = max_s(log i_s + F_j - F_{j,s}), plus F_j, the slice's
+ * total log forget (F_{j,s}: its prefix up to token s).  Slices then join
+ * exactly as tokens do:
+ *   M = max(F_j + M_prev, mloc_j),
+ *   (C', n') = e^{F_j + M_prev - M} (C', n')_prev + e^{mloc_j - M} (C'_j, n'_j).
+ * The state a rank starts from is therefore the fold of the summaries of the
+ * slices before it (an all-gather of summaries, then a local fold: no
+ * sequential hand-off between GPUs), and its forward (xlstm_mlstm_fwd with that
+ * state as C0/n0/m0) reproduces the single-sequence result.
+ *
+ * A summary is one "packed" float buffer of xlstm_mlstm_seg_state_floats()
+ * floats: C' [B, NH, DH, DH], then n' [B, NH, DH], then mloc [B, NH], then
+ * F [B, NH], then zero to three floats of padding (the size is a multiple of 4
+ * floats, so packed summaries laid end to end stay 16-byte aligned).  An empty
+ * slice (S == 0) is summarised as zero state, mloc = -inf, F = 0, which the
+ * fold treats as the identity.
+ */
+xlstm_status xlstm_mlstm_seg_state_floats(int B, int NH, int DH, size_t *floats);
+
+/*
+ * Summary of one slice (see above): k, v [B, NH, S, DH] dtype dt, i_pre, f_pre
+ * [B, NH, S] float, packed: output of xlstm_mlstm_seg_state_floats() floats.
+ * Runs the forward's gate pass and segment summaries (tensor-core kernels for
+ * bf16 where the forward has them, fp32 SIMT kernels otherwise) and a fold of
+ * the segments; no h is formed and q, o are not read.  chunk, dtype and shape
+ * rules and error codes as xlstm_mlstm_fwd; workspace of at least
+ * xlstm_mlstm_seg_state_workspace_size() bytes (overwritten).  B or NH == 0 is
+ * a no-op.
+ */
+xlstm_status xlstm_mlstm_seg_state_workspace_size(int B, int NH, int S, int DH, int chunk,
+                                                  xlstm_dtype dt, size_t *bytes);
+xlstm_status xlstm_mlstm_seg_state(const void *k, const void *v, const float *i_pre, const float *f_pre,
+                                   float *packed, int B, int NH, int S, int DH, int chunk,
+                                   xlstm_dtype dt, xlstm_fgate fg, void *workspace,
+                                   size_t workspace_bytes, void *cuda_stream);
+
+/*
+ * Folds `count` packed summaries (laid end to end at `parts`, each
+ * xlstm_mlstm_seg_state_floats() floats; count == 0 allowed, parts may then be
+ * NULL) into the state that the token-by-token recurrence reaches after those
+ * slices when it starts from (C0, n0, m0) ([B, NH, DH, DH], [B, NH, DH],
+ * [B, NH] float; each NULL = zeros, m0 NULL = 0, the forward's convention).
+ * Writes C_out [B, NH, DH, DH], n_out [B, NH, DH], m_out [B, NH] (all
+ * required); they must not be C0, n0 or m0 (XLSTM_ERR_UNSUPPORTED) nor overlap
+ * parts.  DH: multiple of 16 in [16, 512].
+ */
+xlstm_status xlstm_mlstm_state_combine(const float *parts, int count, const float *C0, const float *n0,
+                                       const float *m0, float *C_out, float *n_out, float *m_out,
+                                       int B, int NH, int DH, void *cuda_stream);
+
+/*
  * Backward of the cell (gradients for training): for the forward with a zero
  * initial state and the loss L = sum(dh * h) + sum(dC * C'_T) + sum(dn * n'_T),
  * writes dL/dq, dL/dk, dL/dv, dL/d(itilde), dL/d(ftilde), dL/d(otilde).  The

@@ -29,7 +29,9 @@ EXPORTED = ("xlstm_abi_version", "xlstm_status_string", "xlstm_mlstm_fwd_workspa
             "xlstm_mlstm_step", "xlstm_device_status", "xlstm_profile_begin", "xlstm_profile_end",
             "xlstm_mlstm_fwd_noalloc", "xlstm_selftest_wait_timeout", "xlstm_mlstm_headnorm_gate",
             "xlstm_mlstm_bwd_workspace_size", "xlstm_mlstm_bwd", "xlstm_slstm_fwd",
-            "xlstm_mlstm_fwd_path")
+            "xlstm_mlstm_fwd_path", "xlstm_mlstm_seg_state_floats",
+            "xlstm_mlstm_seg_state_workspace_size", "xlstm_mlstm_seg_state",
+            "xlstm_mlstm_state_combine")
 NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
 
 
@@ -96,6 +98,14 @@ def load(path: str = LIB_PATH):
         lib.xlstm_mlstm_bwd.restype = i
         lib.xlstm_slstm_fwd.argtypes = [fp] * 14 + [i] * 5 + [vp]
         lib.xlstm_slstm_fwd.restype = i
+        lib.xlstm_mlstm_seg_state_floats.argtypes = [i] * 3 + [ctypes.POINTER(sz)]
+        lib.xlstm_mlstm_seg_state_floats.restype = i
+        lib.xlstm_mlstm_seg_state_workspace_size.argtypes = [i] * 6 + [ctypes.POINTER(sz)]
+        lib.xlstm_mlstm_seg_state_workspace_size.restype = i
+        lib.xlstm_mlstm_seg_state.argtypes = [vp] * 2 + [fp] * 3 + [i] * 7 + [vp, sz, vp]
+        lib.xlstm_mlstm_seg_state.restype = i
+        lib.xlstm_mlstm_state_combine.argtypes = [fp, i] + [fp] * 6 + [i] * 3 + [vp]
+        lib.xlstm_mlstm_state_combine.restype = i
         lib.xlstm_profile_begin.restype = i
         lib.xlstm_profile_end.argtypes = [ctypes.POINTER(KernelTime), i, ctypes.POINTER(i)]
         lib.xlstm_profile_end.restype = i
@@ -173,6 +183,29 @@ def xlstm_slstm_fwd(zx, ix, fx, ox, R, h, c0, n0, m0, h0, c_out, n_out, m_out, h
                     B, NH, S, DH, fg, stream):
     return load().xlstm_slstm_fwd(zx, ix, fx, ox, R, h, c0, n0, m0, h0, c_out, n_out, m_out,
                                   h_out, B, NH, S, DH, fg, stream)
+
+
+def xlstm_mlstm_seg_state_floats(B, NH, DH):
+    n = ctypes.c_size_t(0)
+    st = load().xlstm_mlstm_seg_state_floats(B, NH, DH, ctypes.byref(n))
+    return st, n.value
+
+
+def xlstm_mlstm_seg_state_workspace_size(B, NH, S, DH, chunk, dt):
+    n = ctypes.c_size_t(0)
+    st = load().xlstm_mlstm_seg_state_workspace_size(B, NH, S, DH, chunk, dt, ctypes.byref(n))
+    return st, n.value
+
+
+def xlstm_mlstm_seg_state(k, v, i_pre, f_pre, packed, B, NH, S, DH, chunk, dt, fg, workspace,
+                          workspace_bytes, stream):
+    return load().xlstm_mlstm_seg_state(k, v, i_pre, f_pre, packed, B, NH, S, DH, chunk, dt, fg,
+                                        workspace, workspace_bytes, stream)
+
+
+def xlstm_mlstm_state_combine(parts, count, C0, n0, m0, C_out, n_out, m_out, B, NH, DH, stream):
+    return load().xlstm_mlstm_state_combine(parts, count, C0, n0, m0, C_out, n_out, m_out, B, NH,
+                                            DH, stream)
 
 
 def xlstm_device_status(stream) -> int:
@@ -271,6 +304,74 @@ def mlstm_fwd(q, k, v, i_pre, f_pre, o_pre, chunk=64, fgate="sigmoid", C0=None, 
     if st != OK:
         raise XlstmError(st, "xlstm_mlstm_fwd")
     return h, C, n, m
+
+
+def seg_state_floats(B, NH, DH) -> int:
+    st, n = xlstm_mlstm_seg_state_floats(B, NH, DH)
+    if st != OK:
+        raise XlstmError(st, "xlstm_mlstm_seg_state_floats")
+    return n
+
+
+def unpack_seg_state(packed, B, NH, DH):
+    """Views (C', n', mloc, F) of one packed slice summary (layout of the C header)."""
+    BH = B * NH
+    o1 = BH * DH * DH
+    o2 = o1 + BH * DH
+    return (packed[:o1].view(B, NH, DH, DH), packed[o1:o2].view(B, NH, DH),
+            packed[o2:o2 + BH].view(B, NH), packed[o2 + BH:o2 + 2 * BH].view(B, NH))
+
+
+def mlstm_seg_state(k, v, i_pre, f_pre, chunk=64, fgate="sigmoid", packed=None, workspace=None):
+    """Summary of one slice of a sequence (zero start): a flat float32 tensor of
+    ``seg_state_floats`` floats, see ``unpack_seg_state``."""
+    torch = _torch()
+    B, NH, S, DH = k.shape
+    dev, dtype, dt = k.device, k.dtype, _dt(k)
+    _check(k, "k", (B, NH, S, DH), dtype, dev)
+    _check(v, "v", (B, NH, S, DH), dtype, dev)
+    _check(i_pre, "i_pre", (B, NH, S), torch.float32, dev)
+    _check(f_pre, "f_pre", (B, NH, S), torch.float32, dev)
+    nf = seg_state_floats(B, NH, DH)
+    if packed is None:
+        packed = torch.empty(nf, dtype=torch.float32, device=dev)
+    _check(packed, "packed", (nf,), torch.float32, dev)
+    st, nbytes = xlstm_mlstm_seg_state_workspace_size(B, NH, S, DH, chunk, dt)
+    if st != OK:
+        raise XlstmError(st, "xlstm_mlstm_seg_state_workspace_size")
+    if workspace is None or workspace.numel() < nbytes:
+        workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=dev)
+    fg = FGATE_EXP if fgate == "exp" else FGATE_SIGMOID
+    st = xlstm_mlstm_seg_state(_ptr(k), _ptr(v), _ptr(i_pre), _ptr(f_pre), _ptr(packed), B, NH, S,
+                               DH, chunk, dt, fg, workspace.data_ptr(), workspace.numel(),
+                               _stream(dev))
+    if st != OK:
+        raise XlstmError(st, "xlstm_mlstm_seg_state")
+    return packed
+
+
+def mlstm_state_combine(parts, count, B, NH, DH, C0=None, n0=None, m0=None, out=None):
+    """Fold the first ``count`` packed summaries of ``parts`` ([>= count, floats])
+    onto (C0, n0, m0).  Returns (C', n', m)."""
+    torch = _torch()
+    dev = parts.device
+    nf = seg_state_floats(B, NH, DH)
+    if parts.dim() != 2 or parts.shape[1] != nf or parts.shape[0] < count:
+        raise ValueError(f"parts must be [>= {count}, {nf}], got {tuple(parts.shape)}")
+    _check(parts, "parts", tuple(parts.shape), torch.float32, dev)
+    _check(C0, "C0", (B, NH, DH, DH), torch.float32, dev)
+    _check(n0, "n0", (B, NH, DH), torch.float32, dev)
+    _check(m0, "m0", (B, NH), torch.float32, dev)
+    if out is None:
+        out = (torch.empty((B, NH, DH, DH), dtype=torch.float32, device=dev),
+               torch.empty((B, NH, DH), dtype=torch.float32, device=dev),
+               torch.empty((B, NH), dtype=torch.float32, device=dev))
+    C, n, m = out
+    st = xlstm_mlstm_state_combine(_ptr(parts), count, _ptr(C0), _ptr(n0), _ptr(m0), _ptr(C),
+                                   _ptr(n), _ptr(m), B, NH, DH, _stream(dev))
+    if st != OK:
+        raise XlstmError(st, "xlstm_mlstm_state_combine")
+    return C, n, m
 
 
 def mlstm_step(q, k, v, i_pre, f_pre, o_pre, C, n, m, fgate="sigmoid", h=None):

@@ -79,7 +79,15 @@ bool make_fwd_plan(int B, int NH, int S, int DH, int L, int path, int forced_seg
     if (P > kMaxHeads) P = kMaxHeads;
     p->cps = (p->nchunks + P - 1) / P;
     p->P = (p->nchunks + p->cps - 1) / p->cps;
+    layout_fwd_workspace(p);
+    return true;
+}
 
+void layout_fwd_workspace(FwdPlan *p) {
+    const int S = p->S, DH = p->DH;
+    const bool tensor = p->path == XLSTM_PATH_TENSOR || p->path == XLSTM_PATH_TENSOR_TMEM ||
+                        p->path == XLSTM_PATH_TENSOR_RS;
+    const int ksplit = tensor ? rs_key_splits(DH, p->L) : 1;
     size_t off = 0;
     p->off_bcum = off;  off = align64(off + (size_t)p->BH * S);
     p->off_pmax = off;  off = align64(off + (size_t)p->BH * S);
@@ -95,7 +103,6 @@ bool make_fwd_plan(int B, int NH, int S, int DH, int L, int path, int forced_seg
         p->off_tok = off;   off = align64(off + 2 * (size_t)p->BH * S);
     }
     p->total_floats = off;
-    return true;
 }
 
 // Copies (or zero-fills) the initial state into the final-state outputs: the
@@ -282,6 +289,163 @@ xlstm_status xlstm_mlstm_fwd(const void *q, const void *k, const void *v,
     return xlstm_mlstm_fwd_ex(q, k, v, i_pre, f_pre, o_pre, h, C0, n0, m0, C_out, n_out, m_out,
                               B, NH, S, DH, chunk, dt, fg, workspace, workspace_bytes, nullptr,
                               cuda_stream);
+}
+
+// ---------------------------------------------------------- sequence parallelism
+static size_t seg_state_floats(long long BH, int DH) {
+    const size_t n = (size_t)BH * ((size_t)DH * DH + DH + 2);
+    return (n + 3) & ~size_t(3);
+}
+
+static xlstm_status check_state_shape(int B, int NH, int DH) {
+    if (B < 0 || NH < 0) return XLSTM_ERR_SHAPE;
+    if (DH < 16 || DH > 512 || DH % 16 != 0) return XLSTM_ERR_SHAPE;
+    if ((long long)B * NH > kMaxHeads) return XLSTM_ERR_SHAPE;
+    return XLSTM_OK;
+}
+
+// The segment-state pass reuses the forward's segmentation and summary kernels
+// with every segment summarised (the forward leaves the last one to its output
+// kernel), then folds the summaries; a BH-float buffer after the forward's
+// layout holds the fold's starting stabiliser for the in-place scan.
+static xlstm_status make_seg_state_plan(int B, int NH, int S, int DH, int chunk, xlstm_dtype dt,
+                                        FwdPlan *p, size_t *off_mstart, size_t *total_floats) {
+    xlstm_status st;
+    const int path = resolve_path(dt, DH, chunk, nullptr, &st);
+    if (st != XLSTM_OK) return st;
+    if (!make_fwd_plan(B, NH, S, DH, chunk, path, 0, num_sms_current_device(), p)) return XLSTM_ERR_SHAPE;
+    if (p->P == 0) {
+        *off_mstart = 0;
+        *total_floats = 0;
+        return XLSTM_OK;
+    }
+    p->P += 1;
+    layout_fwd_workspace(p);
+    *off_mstart = p->total_floats;
+    *total_floats = align64(p->total_floats + (size_t)p->BH);
+    return XLSTM_OK;
+}
+
+xlstm_status xlstm_mlstm_seg_state_floats(int B, int NH, int DH, size_t *floats) {
+    if (!floats) return XLSTM_ERR_NULL;
+    xlstm_status st = check_state_shape(B, NH, DH);
+    if (st != XLSTM_OK) return st;
+    *floats = seg_state_floats((long long)B * NH, DH);
+    return XLSTM_OK;
+}
+
+xlstm_status xlstm_mlstm_seg_state_workspace_size(int B, int NH, int S, int DH, int chunk,
+                                                  xlstm_dtype dt, size_t *bytes) {
+    if (!bytes) return XLSTM_ERR_NULL;
+    xlstm_status st = check_fwd_shape(B, NH, S, DH, chunk, dt);
+    if (st != XLSTM_OK) return st;
+    FwdPlan p;
+    size_t off_m, total;
+    st = make_seg_state_plan(B, NH, S, DH, chunk, dt, &p, &off_m, &total);
+    if (st != XLSTM_OK) return st;
+    *bytes = total * sizeof(float);
+    return XLSTM_OK;
+}
+
+xlstm_status xlstm_mlstm_seg_state(const void *k, const void *v, const float *i_pre, const float *f_pre,
+                                   float *packed, int B, int NH, int S, int DH, int chunk,
+                                   xlstm_dtype dt, xlstm_fgate fg, void *workspace,
+                                   size_t workspace_bytes, void *cuda_stream) {
+    CallRange range("xlstm_mlstm_seg_state");
+    xlstm_status st = check_fwd_shape(B, NH, S, DH, chunk, dt);
+    if (st != XLSTM_OK) return st;
+    if (fg != XLSTM_FGATE_SIGMOID && fg != XLSTM_FGATE_EXP) return XLSTM_ERR_DTYPE;
+    const int BH = B * NH;
+    if (BH == 0) return XLSTM_OK;
+    if (!packed) return XLSTM_ERR_NULL;
+    if (S > 0 && (!k || !v || !i_pre || !f_pre)) return XLSTM_ERR_NULL;
+    const void *ptrs[] = {k, v, i_pre, f_pre, packed, workspace};
+    for (const void *p : ptrs)
+        if (misaligned(p)) return XLSTM_ERR_ALIGN;
+    FwdPlan plan;
+    size_t off_m, total;
+    st = make_seg_state_plan(B, NH, S, DH, chunk, dt, &plan, &off_m, &total);
+    if (st != XLSTM_OK) return st;
+    if (total > 0 && (!workspace || workspace_bytes < total * sizeof(float))) return XLSTM_ERR_WORKSPACE;
+    cudaStream_t stream = (cudaStream_t)cuda_stream;
+    float *Cp = packed, *np = packed + (size_t)BH * DH * DH, *mp = np + (size_t)BH * DH, *Fp = mp + BH;
+    FoldSource src = {};
+    if (S == 0) {
+        // an empty run: zero state, stabiliser -inf, no forgetting
+        return launch_state_fold(src, 0, 0, nullptr, nullptr, nullptr, 1, Cp, np, mp, Fp, BH, DH, stream) ==
+                       cudaSuccess ? XLSTM_OK : XLSTM_ERR_CUDA;
+    }
+    FwdArgs a = {};
+    a.k = k; a.v = v; a.i_pre = i_pre; a.f_pre = f_pre;
+    a.workspace = workspace;
+    if (cudaGetSymbolAddress((void **)&a.status, g_device_status) != cudaSuccess) return XLSTM_ERR_CUDA;
+    a.bf16 = dt == XLSTM_BF16;
+    a.fgate_exp = fg == XLSTM_FGATE_EXP;
+    float *ws = (float *)workspace;
+    const bool tensor = plan.path != XLSTM_PATH_SIMT;
+    cudaError_t e = cudaSuccess;
+    if (tensor && plan.Spad > S) {
+        // the tensor-core summaries fetch 64-token tiles of log i - b; past the
+        // end of the run every byte 0xFE (-1.7e38) makes the token's weight 0
+        e = cudaMemset2DAsync(ws + plan.off_upad + S, (size_t)plan.Spad * sizeof(float), 0xFE,
+                              (size_t)(plan.Spad - S) * sizeof(float), BH, stream);
+        if (e != cudaSuccess) return XLSTM_ERR_CUDA;
+    }
+    if ((e = launch_gate_prologue(a, plan, stream)) != cudaSuccess) return XLSTM_ERR_CUDA;
+    if (tensor) {
+        // summaries + the in-place segment scan, started from stabiliser -1.7e38
+        // (bytes 0xFE): the same fold as from -inf for any finite statistics
+        float *mstart = ws + off_m;
+        if (cudaMemsetAsync(mstart, 0xFE, (size_t)BH * sizeof(float), stream) != cudaSuccess)
+            return XLSTM_ERR_CUDA;
+        a.m0 = mstart;
+        e = launch_segment_summaries(a, plan, stream);
+    } else {
+        e = launch_segment_summaries_simt(a, plan, stream);
+    }
+    if (e != cudaSuccess) return XLSTM_ERR_CUDA;
+    const size_t per = (size_t)DH * DH + DH;
+    float *summ = ws + plan.off_summ;
+    const float *sst = ws + plan.off_sstat;
+    src.C = summ;
+    src.n = summ + (size_t)DH * DH;
+    src.F = sst;
+    src.m = sst + 1;
+    src.cg = src.ng = per;
+    src.cbh = src.nbh = (size_t)(plan.P - 1) * per;
+    src.sg = 2;
+    src.sbh = 2 * (size_t)plan.P;
+    e = launch_state_fold(src, plan.P - 1, tensor ? 1 : 0, nullptr, nullptr, nullptr, 1, Cp, np, mp, Fp, BH, DH,
+                          stream);
+    return e == cudaSuccess ? XLSTM_OK : XLSTM_ERR_CUDA;
+}
+
+xlstm_status xlstm_mlstm_state_combine(const float *parts, int count, const float *C0, const float *n0,
+                                       const float *m0, float *C_out, float *n_out, float *m_out,
+                                       int B, int NH, int DH, void *cuda_stream) {
+    CallRange range("xlstm_mlstm_state_combine");
+    xlstm_status st = check_state_shape(B, NH, DH);
+    if (st != XLSTM_OK) return st;
+    if (count < 0) return XLSTM_ERR_SHAPE;
+    const int BH = B * NH;
+    if (BH == 0) return XLSTM_OK;
+    if (!C_out || !n_out || !m_out || (count > 0 && !parts)) return XLSTM_ERR_NULL;
+    const void *ptrs[] = {parts, C0, n0, m0, C_out, n_out, m_out};
+    for (const void *p : ptrs)
+        if (misaligned(p)) return XLSTM_ERR_ALIGN;
+    if ((C0 && C_out == C0) || (n0 && n_out == n0) || (m0 && m_out == m0)) return XLSTM_ERR_UNSUPPORTED;
+    const size_t packed = seg_state_floats(BH, DH);
+    FoldSource src = {};
+    src.C = parts;
+    src.n = parts ? parts + (size_t)BH * DH * DH : nullptr;
+    src.m = parts ? src.n + (size_t)BH * DH : nullptr;
+    src.F = parts ? src.m + BH : nullptr;
+    src.cg = src.ng = src.sg = packed;
+    src.cbh = (size_t)DH * DH;
+    src.nbh = DH;
+    src.sbh = 1;
+    return launch_state_fold(src, count, 0, C0, n0, m0, 0, C_out, n_out, m_out, nullptr, BH, DH,
+                             (cudaStream_t)cuda_stream) == cudaSuccess ? XLSTM_OK : XLSTM_ERR_CUDA;
 }
 
 xlstm_status xlstm_mlstm_step(const void *q, const void *k, const void *v,

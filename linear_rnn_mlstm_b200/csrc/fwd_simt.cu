@@ -447,6 +447,26 @@ static cudaError_t launch_simt_t(const FwdArgs &a, const FwdPlan &p, cudaStream_
     return cudaGetLastError();
 }
 
+template <typename T>
+static cudaError_t launch_summaries_simt_t(const FwdArgs &a, const FwdPlan &p, cudaStream_t st) {
+    float *ws = (float *)a.workspace;
+    const size_t sm1 = simt_summary_smem(p.DH, p.rows);
+    cudaError_t e = cudaFuncSetAttribute(segment_summary_simt_kernel<T>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm1);
+    if (e != cudaSuccess) return e;
+    KernelTimer timer("segment_summary_simt", st);
+    segment_summary_simt_kernel<T><<<dim3(p.ntiles, p.P - 1, p.BH), 256, sm1, st>>>(
+        (const T *)a.k, (const T *)a.v, a.i_pre, ws + p.off_bcum, (const float2 *)(ws + p.off_cstat),
+        (float2 *)(ws + p.off_sstat), ws + p.off_summ, p.S, p.DH, p.L, p.nchunks, p.P, p.cps, p.rows);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_segment_summaries_simt(const FwdArgs &a, const FwdPlan &p, cudaStream_t st) {
+    if (p.P <= 1) return cudaSuccess;
+    if (a.bf16) return launch_summaries_simt_t<__nv_bfloat16>(a, p, st);
+    return launch_summaries_simt_t<float>(a, p, st);
+}
+
 cudaError_t launch_fwd_simt(const FwdArgs &a, const FwdPlan &p, cudaStream_t st) {
     cudaError_t e = launch_gate_prologue(a, p, st);
     if (e != cudaSuccess) return e;

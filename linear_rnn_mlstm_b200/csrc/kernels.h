@@ -57,10 +57,29 @@ cudaError_t launch_chained(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t
     return cudaLaunchKernelEx(&cfg, kern, args...);
 }
 
+// Where the fold of seqpar.cu finds run g of head bh: its (C' | n') summary at
+// C + g*cg + bh*cbh (DH*DH floats) and n + g*ng + bh*nbh (DH floats), and its
+// total log forget and own stabiliser at F / m + g*sg + bh*sbh.  Every C/n
+// offset is a multiple of 4 floats and the bases are 16-byte aligned.
+struct FoldSource {
+    const float *C, *n, *F, *m;
+    size_t cg, cbh, ng, nbh, sg, sbh;
+};
+// Folds `count` runs into (C_out, n_out, m_out) from (C0, n0, m0) (NULL: zeros,
+// and m = 0, or -inf when start_neg_inf); F_out (nullable) gets the summed log
+// forget.  scanned != 0: the runs were already folded in place by the segment
+// scan from the same start, so only the last one is read.
+cudaError_t launch_state_fold(const FoldSource &src, int count, int scanned, const float *C0, const float *n0,
+                              const float *m0, int start_neg_inf, float *C_out, float *n_out, float *m_out,
+                              float *F_out, int BH, int D, cudaStream_t st);
+
 cudaError_t launch_gate_prologue(const FwdArgs &a, const FwdPlan &p, cudaStream_t st);
 // Segment summaries + segment scan of the two-level chunk-state scan, on the
 // tensor cores (bf16, DH 64, 128 or 256); nothing when the plan has one segment.
 cudaError_t launch_segment_summaries(const FwdArgs &a, const FwdPlan &p, cudaStream_t st);
+// Segment summaries only (no scan), fp32 arithmetic, any DH and chunk: the raw
+// per-segment (dC, dn) and (total log forget, stabiliser) of segments 0..P-2.
+cudaError_t launch_segment_summaries_simt(const FwdArgs &a, const FwdPlan &p, cudaStream_t st);
 cudaError_t launch_fwd_simt(const FwdArgs &a, const FwdPlan &p, cudaStream_t st);
 cudaError_t launch_fwd_tensor(const FwdArgs &a, const FwdPlan &p, cudaStream_t st);
 bool tensor_path_supports(int DH, int L);

@@ -51,5 +51,8 @@ struct FwdPlan {
 // Fills `p`; returns false if the configuration cannot be planned.
 bool make_fwd_plan(int B, int NH, int S, int DH, int L, int path, int forced_segments,
                    int num_sms, FwdPlan *p);
+// Recomputes the workspace offsets of `p` from its sizes and P (make_fwd_plan
+// calls it; a caller that changes P afterwards calls it again).
+void layout_fwd_workspace(FwdPlan *p);
 
 }  // namespace xlstm

@@ -232,3 +232,61 @@ def _slstm(**over):
 ])
 def test_slstm_rejects_bad_arguments_before_device_work(over, expect):
     assert _slstm(**over) == expect
+
+
+def _seg_state(**over):
+    a = dict(k=FAKE, v=FAKE, i_pre=FAKE, f_pre=FAKE, packed=FAKE, B=1, NH=2, S=200, DH=64, chunk=64,
+             dt=xb.BF16, fg=xb.FGATE_SIGMOID, workspace=FAKE, workspace_bytes=0, stream=None)
+    a.update(over)
+    return xb.xlstm_mlstm_seg_state(**a)
+
+
+@pytest.mark.parametrize("over,expect", [
+    (dict(k=None), xb.ERR_NULL),
+    (dict(packed=None), xb.ERR_NULL),
+    (dict(f_pre=FAKE + 4), xb.ERR_ALIGN),
+    (dict(packed=FAKE + 8), xb.ERR_ALIGN),
+    (dict(fg=3), xb.ERR_DTYPE),
+    (dict(dt=xb.BF16, chunk=32), xb.ERR_CHUNK),
+    (dict(DH=24), xb.ERR_SHAPE),
+    (dict(S=-1), xb.ERR_SHAPE),
+    (dict(workspace_bytes=64), xb.ERR_WORKSPACE),
+    (dict(B=0), xb.OK),
+])
+def test_seg_state_rejects_bad_arguments_before_device_work(over, expect):
+    assert _seg_state(**over) == expect
+
+
+def _combine(**over):
+    a = dict(parts=FAKE, count=2, C0=None, n0=None, m0=None, C_out=FAKE, n_out=FAKE, m_out=FAKE,
+             B=1, NH=2, DH=64, stream=None)
+    a.update(over)
+    return xb.xlstm_mlstm_state_combine(**a)
+
+
+@pytest.mark.parametrize("over,expect", [
+    (dict(parts=None), xb.ERR_NULL),
+    (dict(C_out=None), xb.ERR_NULL),
+    (dict(m_out=None), xb.ERR_NULL),
+    (dict(count=-1), xb.ERR_SHAPE),
+    (dict(DH=520), xb.ERR_SHAPE),
+    (dict(n0=FAKE + 4), xb.ERR_ALIGN),
+    (dict(C0=FAKE, C_out=FAKE), xb.ERR_UNSUPPORTED),       # in place is refused
+    (dict(m0=FAKE + 64, m_out=FAKE + 64), xb.ERR_UNSUPPORTED),
+    (dict(NH=0), xb.OK),
+])
+def test_state_combine_rejects_bad_arguments_before_device_work(over, expect):
+    assert _combine(**over) == expect
+
+
+def test_seg_state_sizes():
+    # packed summary: C' [BH,DH,DH] + n' [BH,DH] + mloc, F [BH], padded to 4 floats
+    assert xb.xlstm_mlstm_seg_state_floats(1, 8, 256) == (xb.OK, 8 * (256 * 256 + 256 + 2))
+    assert xb.xlstm_mlstm_seg_state_floats(1, 1, 16) == (xb.OK, 276)      # 274 -> 276
+    assert xb.xlstm_mlstm_seg_state_floats(1, 1, 20)[0] == xb.ERR_SHAPE
+    # every segment summarised: at least the forward's workspace, plus one slot
+    for dt, DH, L in ((xb.BF16, 256, 64), (xb.BF16, 64, 128), (xb.F32, 32, 16)):
+        st, ws = xb.xlstm_mlstm_seg_state_workspace_size(1, 8, 4096, DH, L, dt)
+        st2, wf = xb.xlstm_mlstm_fwd_workspace_size(1, 8, 4096, DH, L, dt)
+        assert st == st2 == xb.OK and ws >= wf + 8 * (DH * DH + DH) * 4
+    assert xb.xlstm_mlstm_seg_state_workspace_size(1, 8, 0, 64, 64, xb.BF16) == (xb.OK, 0)
