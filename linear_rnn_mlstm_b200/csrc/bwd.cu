@@ -25,6 +25,7 @@
 #include "common.cuh"
 #include "kernels.h"
 #include "profile.h"
+#include "bwd_tc.cuh"
 
 namespace xlstm {
 namespace {
@@ -97,7 +98,11 @@ template <int N> __device__ __forceinline__ void cp_async_wait() {
 // 32 rows' raw coefficients (v or dnum' entries) and the per-token scalars;
 // the next chunk's stage is filled by cp.async while this one is used, so the
 // walk over chunks waits on no global-memory round trip.
-template <typename T, int NCL, bool REVERSE>
+//
+// SPLIT: the DH x DH slots are stored as bf16 high and low planes in the
+// tensor-core kernels' tile order (bwdtc::plane_offset) instead of fp32 rows;
+// the normaliser row stays fp32.
+template <typename T, int NCL, bool REVERSE, bool SPLIT>
 __global__ void __launch_bounds__(kRowThreads) bwd_rows_kernel(BwdPtrs p) {
     constexpr int DH = 32 * NCL;
     extern __shared__ __align__(16) uint8_t rows_smem[];
@@ -152,6 +157,25 @@ __global__ void __launch_bounds__(kRowThreads) bwd_rows_kernel(BwdPtrs p) {
         return (REVERSE ? p.dCb + (size_t)bh * NC * DD : p.Cst + (size_t)bh * (NC + 1) * DD) +
                (size_t)slot * DD + (size_t)r * DH;
     };
+    // row r's values (lane + 32 j) into `slot`
+    auto store_row = [&](int r, int slot, const float (&x)[NCL]) {
+        if (SPLIT && r < DH) {
+            uint8_t *pl = reinterpret_cast<uint8_t *>(
+                (REVERSE ? p.dCb + (size_t)bh * NC * DD : p.Cst + (size_t)bh * (NC + 1) * DD) + (size_t)slot * DD);
+#pragma unroll
+            for (int j = 0; j < NCL; ++j) {
+                const uint32_t off = bwdtc::plane_offset(r, lane + 32 * j, DH);
+                const __nv_bfloat16 hi = __float2bfloat16_rn(x[j]);
+                *reinterpret_cast<__nv_bfloat16 *>(pl + off) = hi;
+                *reinterpret_cast<__nv_bfloat16 *>(pl + DD * 2 + off) =
+                    __float2bfloat16_rn(x[j] - __bfloat162float(hi));
+            }
+        } else {
+            float *dst = slot_ptr(r, slot);
+#pragma unroll
+            for (int j = 0; j < NCL; ++j) dst[lane + 32 * j] = x[j];
+        }
+    };
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         const int r = r0 + 4 * warp + i;
@@ -162,8 +186,8 @@ __global__ void __launch_bounds__(kRowThreads) bwd_rows_kernel(BwdPtrs p) {
             if (REVERSE && r < DH && p.dC) x = p.dC[(size_t)bh * DD + (size_t)r * DH + col];
             if (REVERSE && r == DH && p.dn) x = p.dn[(size_t)bh * DH + col];
             st[i][j] = x;
-            if (r <= DH) slot_ptr(r, REVERSE ? NC - 1 : 0)[col] = x;
         }
+        if (r <= DH) store_row(r, REVERSE ? NC - 1 : 0, st[i]);
     }
     // chunks walked: 0 .. NC-1 forward; NC-1 .. 1 in reverse (slot c-1 from chunk c)
     const int nsteps = REVERSE ? NC - 1 : NC;
@@ -223,9 +247,7 @@ __global__ void __launch_bounds__(kRowThreads) bwd_rows_kernel(BwdPtrs p) {
         for (int i = 0; i < 4; ++i) {
             const int r = r0 + 4 * warp + i;
             if (r > DH) continue;
-            float *dst = slot_ptr(r, REVERSE ? c - 1 : c + 1);
-#pragma unroll
-            for (int j = 0; j < NCL; ++j) dst[lane + 32 * j] = st[i][j];
+            store_row(r, REVERSE ? c - 1 : c + 1, st[i]);
         }
     }
     cp_async_wait<0>();
@@ -238,10 +260,24 @@ bool launch_rows(const BwdPtrs &p, cudaStream_t st) {
     const size_t sm = rows_smem_bytes<T>(p.L, p.DH);
     if (sm > 232448) return false;        // two stages do not fit (fp32 at DH 512): per-thread kernel
     const dim3 grid((unsigned)((p.DH + 1 + kRowBlock - 1) / kRowBlock), (unsigned)p.BH);
+    if (p.tc) {                           // bf16, DH 128 / 256: slots as bf16 planes
+        if constexpr (sizeof(T) == 2) {
+#define XLSTM_BWD_ROWS_SPLIT(N)                                                                   \
+            if (ncl == N) {                                                                        \
+                cudaFuncSetAttribute(bwd_rows_kernel<T, N, REVERSE, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm); \
+                bwd_rows_kernel<T, N, REVERSE, true><<<grid, kRowThreads, sm, st>>>(p);            \
+                return true;                                                                       \
+            }
+            XLSTM_BWD_ROWS_SPLIT(4)
+            XLSTM_BWD_ROWS_SPLIT(8)
+#undef XLSTM_BWD_ROWS_SPLIT
+        }
+        return false;
+    }
 #define XLSTM_BWD_ROWS(N)                                                                         \
     if (ncl == N) {                                                                                \
-        cudaFuncSetAttribute(bwd_rows_kernel<T, N, REVERSE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm); \
-        bwd_rows_kernel<T, N, REVERSE><<<grid, kRowThreads, sm, st>>>(p);                          \
+        cudaFuncSetAttribute(bwd_rows_kernel<T, N, REVERSE, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm); \
+        bwd_rows_kernel<T, N, REVERSE, false><<<grid, kRowThreads, sm, st>>>(p);                   \
         return true;                                                                               \
     }
     XLSTM_BWD_ROWS(1)
@@ -494,7 +530,9 @@ size_t chunk_grad_smem_bytes() {
     return (size_t)3 * L * DH * 2 + (size_t)L * DH * 4 + (size_t)2 * L * L * 4 + (size_t)8 * L * 4;
 }
 
-template <int NCL>
+// TC: the products with the chunk's states come from the tensor-core kernels
+// (dq: p.num, dk: p.dki, dv: p.dvi, unscaled) instead of the state rows.
+template <int NCL, bool TC>
 __global__ void __launch_bounds__(32 * kChWarps, 1) bwd_token_grad_chunk_kernel(BwdPtrs p) {
     constexpr int DH = 32 * NCL, LM = bwd::kMaxChunk;
     using T = __nv_bfloat16;
@@ -571,15 +609,25 @@ __global__ void __launch_bounds__(32 * kChWarps, 1) bwd_token_grad_chunk_kernel(
             for (int i = 0; i < NCL; ++i) acc[x][i] += w * __bfloat162float(sk[u * DH + lane + 32 * i]);
         }
     }
-    for (int r = 0; r < DH; ++r) {                  // C' rows, once per CTA
-        float cr[NCL];
-#pragma unroll
-        for (int i = 0; i < NCL; ++i) cr[i] = Cc[(size_t)r * DH + lane + 32 * i];
+    if constexpr (TC) {
 #pragma unroll
         for (int x = 0; x < kChTok; ++x) {
-            const float dn_r = sdn[(warp * kChTok + x) * DH + r];
+            const int s = warp * kChTok + x;
+            if (s >= n) continue;
 #pragma unroll
-            for (int i = 0; i < NCL; ++i) inter[x][i] += cr[i] * dn_r;
+            for (int i = 0; i < NCL; ++i) inter[x][i] = p.num[(row0 + s) * DH + lane + 32 * i];
+        }
+    } else {
+        for (int r = 0; r < DH; ++r) {              // C' rows, once per CTA
+            float cr[NCL];
+#pragma unroll
+            for (int i = 0; i < NCL; ++i) cr[i] = Cc[(size_t)r * DH + lane + 32 * i];
+#pragma unroll
+            for (int x = 0; x < kChTok; ++x) {
+                const float dn_r = sdn[(warp * kChTok + x) * DH + r];
+#pragma unroll
+                for (int i = 0; i < NCL; ++i) inter[x][i] += cr[i] * dn_r;
+            }
         }
     }
 #pragma unroll
@@ -606,15 +654,25 @@ __global__ void __launch_bounds__(32 * kChWarps, 1) bwd_token_grad_chunk_kernel(
             for (int i = 0; i < NCL; ++i) acc[x][i] += w * __bfloat162float(sq[t * DH + lane + 32 * i]);
         }
     }
-    for (int r = 0; r < DH; ++r) {                  // dC~ rows, once per CTA
-        float dr[NCL];
-#pragma unroll
-        for (int i = 0; i < NCL; ++i) dr[i] = dCc[(size_t)r * DH + lane + 32 * i];
+    if constexpr (TC) {
 #pragma unroll
         for (int x = 0; x < kChTok; ++x) {
-            const float v_r = __bfloat162float(sv[(warp * kChTok + x) * DH + r]);
+            const int s = warp * kChTok + x;
+            if (s >= n) continue;
 #pragma unroll
-            for (int i = 0; i < NCL; ++i) inter[x][i] += dr[i] * v_r;
+            for (int i = 0; i < NCL; ++i) inter[x][i] = p.dki[(row0 + s) * DH + lane + 32 * i];
+        }
+    } else {
+        for (int r = 0; r < DH; ++r) {              // dC~ rows, once per CTA
+            float dr[NCL];
+#pragma unroll
+            for (int i = 0; i < NCL; ++i) dr[i] = dCc[(size_t)r * DH + lane + 32 * i];
+#pragma unroll
+            for (int x = 0; x < kChTok; ++x) {
+                const float v_r = __bfloat162float(sv[(warp * kChTok + x) * DH + r]);
+#pragma unroll
+                for (int i = 0; i < NCL; ++i) inter[x][i] += dr[i] * v_r;
+            }
         }
     }
     float di_tok[kChTok], wk_tok[kChTok];
@@ -647,21 +705,32 @@ __global__ void __launch_bounds__(32 * kChWarps, 1) bwd_token_grad_chunk_kernel(
             for (int i = 0; i < NCL; ++i) acc[x][i] += w * sdn[t * DH + lane + 32 * i];
         }
     }
+    if constexpr (TC) {
 #pragma unroll
-    for (int rb = 0; rb < NCL; ++rb) {
-        for (int rl = 0; rl < 32; ++rl) {
-            const int r = 32 * rb + rl;
-            float dr[NCL];
+        for (int x = 0; x < kChTok; ++x) {
+            const int s = warp * kChTok + x;
+            if (s >= n) continue;
 #pragma unroll
-            for (int i = 0; i < NCL; ++i) dr[i] = dCc[(size_t)r * DH + lane + 32 * i];
+            for (int i = 0; i < NCL; ++i)
+                acc[x][i] += wk_tok[x] * inv_sqrt * p.dvi[(row0 + s) * DH + lane + 32 * i];
+        }
+    } else {
 #pragma unroll
-            for (int x = 0; x < kChTok; ++x) {
-                float part = 0.f;
+        for (int rb = 0; rb < NCL; ++rb) {
+            for (int rl = 0; rl < 32; ++rl) {
+                const int r = 32 * rb + rl;
+                float dr[NCL];
 #pragma unroll
-                for (int i = 0; i < NCL; ++i)
-                    part += dr[i] * __bfloat162float(sk[(warp * kChTok + x) * DH + lane + 32 * i]);
-                part = wsum(part);
-                if (rl == lane) acc[x][rb] += wk_tok[x] * inv_sqrt * part;
+                for (int i = 0; i < NCL; ++i) dr[i] = dCc[(size_t)r * DH + lane + 32 * i];
+#pragma unroll
+                for (int x = 0; x < kChTok; ++x) {
+                    float part = 0.f;
+#pragma unroll
+                    for (int i = 0; i < NCL; ++i)
+                        part += dr[i] * __bfloat162float(sk[(warp * kChTok + x) * DH + lane + 32 * i]);
+                    part = wsum(part);
+                    if (rl == lane) acc[x][rb] += wk_tok[x] * inv_sqrt * part;
+                }
             }
         }
     }
@@ -689,7 +758,9 @@ size_t chunk_fwd_smem_bytes() {
     return (size_t)3 * L * DH * 2 + (size_t)L * L * 4 + (size_t)4 * L * 4;
 }
 
-template <int NCL>
+// TC: C' q_t comes from the tensor-core kernel (p.num, unscaled) instead of the
+// state rows, and dnum' is also written as bf16 high and low planes (p.dnhl).
+template <int NCL, bool TC>
 __global__ void __launch_bounds__(32 * kChWarps, 1) bwd_token_fwd_chunk_kernel(BwdPtrs p) {
     constexpr int DH = 32 * NCL, LM = bwd::kMaxChunk;
     using T = __nv_bfloat16;
@@ -739,21 +810,31 @@ __global__ void __launch_bounds__(32 * kChWarps, 1) bwd_token_fwd_chunk_kernel(B
     for (int x = 0; x < kChTok; ++x)
 #pragma unroll
         for (int i = 0; i < NCL; ++i) num[x][i] = 0.f;
+    if constexpr (TC) {
 #pragma unroll
-    for (int rb = 0; rb < NCL; ++rb) {
-        for (int rl = 0; rl < 32; ++rl) {
-            const int r = 32 * rb + rl;
-            float cr[NCL];
+        for (int x = 0; x < kChTok; ++x) {
+            const int t = warp * kChTok + x;
+            if (t >= n) continue;
 #pragma unroll
-            for (int i = 0; i < NCL; ++i) cr[i] = Cc[(size_t)r * DH + lane + 32 * i];
+            for (int i = 0; i < NCL; ++i) num[x][i] = p.num[(row0 + t) * DH + lane + 32 * i];
+        }
+    } else {
 #pragma unroll
-            for (int x = 0; x < kChTok; ++x) {
-                float part = 0.f;
+        for (int rb = 0; rb < NCL; ++rb) {
+            for (int rl = 0; rl < 32; ++rl) {
+                const int r = 32 * rb + rl;
+                float cr[NCL];
 #pragma unroll
-                for (int i = 0; i < NCL; ++i)
-                    part += cr[i] * __bfloat162float(sq[(warp * kChTok + x) * DH + lane + 32 * i]);
-                part = wsum(part);
-                if (rl == lane) num[x][rb] = part;
+                for (int i = 0; i < NCL; ++i) cr[i] = Cc[(size_t)r * DH + lane + 32 * i];
+#pragma unroll
+                for (int x = 0; x < kChTok; ++x) {
+                    float part = 0.f;
+#pragma unroll
+                    for (int i = 0; i < NCL; ++i)
+                        part += cr[i] * __bfloat162float(sq[(warp * kChTok + x) * DH + lane + 32 * i]);
+                    part = wsum(part);
+                    if (rl == lane) num[x][rb] = part;
+                }
             }
         }
     }
@@ -789,6 +870,12 @@ __global__ void __launch_bounds__(32 * kChWarps, 1) bwd_token_fwd_chunk_kernel(B
             p.dO[ts * DH + r] = dhr * hv * o * (1.f - o);
             const float dn_r = dht / den;
             p.dnum[ts * DH + r] = dn_r;
+            if constexpr (TC) {
+                __nv_bfloat16 *hl = reinterpret_cast<__nv_bfloat16 *>(p.dnhl);
+                const __nv_bfloat16 hi = __float2bfloat16_rn(dn_r);
+                hl[ts * DH + r] = hi;
+                hl[(size_t)p.BH * p.S * DH + ts * DH + r] = __float2bfloat16_rn(dn_r - __bfloat162float(hi));
+            }
             sdot += dht * hv;
             A += dn_r * num[x][i];
         }
@@ -812,8 +899,13 @@ bool launch_token_fwd_chunk(const BwdPtrs &p, cudaStream_t st) {
 #define XLSTM_BWD_CF(N)                                                                           \
     if (p.DH == 32 * N) {                                                                          \
         const size_t sm = chunk_fwd_smem_bytes<N>();                                               \
-        cudaFuncSetAttribute(bwd_token_fwd_chunk_kernel<N>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm); \
-        bwd_token_fwd_chunk_kernel<N><<<grid, 32 * kChWarps, sm, st>>>(p);                         \
+        if (p.tc) {                                                                                \
+            cudaFuncSetAttribute(bwd_token_fwd_chunk_kernel<N, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm); \
+            bwd_token_fwd_chunk_kernel<N, true><<<grid, 32 * kChWarps, sm, st>>>(p);               \
+        } else {                                                                                   \
+            cudaFuncSetAttribute(bwd_token_fwd_chunk_kernel<N, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm); \
+            bwd_token_fwd_chunk_kernel<N, false><<<grid, 32 * kChWarps, sm, st>>>(p);              \
+        }                                                                                          \
         return true;                                                                               \
     }
     XLSTM_BWD_CF(4)
@@ -829,8 +921,13 @@ bool launch_token_grad_chunk(const BwdPtrs &p, cudaStream_t st) {
 #define XLSTM_BWD_CH(N)                                                                           \
     if (p.DH == 32 * N) {                                                                          \
         const size_t sm = chunk_grad_smem_bytes<N>();                                              \
-        cudaFuncSetAttribute(bwd_token_grad_chunk_kernel<N>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm); \
-        bwd_token_grad_chunk_kernel<N><<<grid, 32 * kChWarps, sm, st>>>(p);                        \
+        if (p.tc) {                                                                                \
+            cudaFuncSetAttribute(bwd_token_grad_chunk_kernel<N, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm); \
+            bwd_token_grad_chunk_kernel<N, true><<<grid, 32 * kChWarps, sm, st>>>(p);              \
+        } else {                                                                                   \
+            cudaFuncSetAttribute(bwd_token_grad_chunk_kernel<N, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm); \
+            bwd_token_grad_chunk_kernel<N, false><<<grid, 32 * kChWarps, sm, st>>>(p);             \
+        }                                                                                          \
         return true;                                                                               \
     }
     XLSTM_BWD_CH(4)
@@ -924,8 +1021,17 @@ __global__ void __launch_bounds__(128) bwd_forget_warp_kernel(BwdPtrs p) {
         float a_final = 0.f;
         const float *CT = p.Cst + ((size_t)bh * (NC + 1) + NC) * DD;
         const float *nT = p.nst + ((size_t)bh * (NC + 1) + NC) * DH;
-        if (p.dC)
+        if (p.dC && p.tc) {                    // C'_T as bf16 high + low planes
+            const uint8_t *pl = reinterpret_cast<const uint8_t *>(CT);
+            for (size_t i = lane; i < DD; i += 32) {
+                const uint32_t off = bwdtc::plane_offset((int)(i / DH), (int)(i % DH), DH);
+                const float x = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(pl + off)) +
+                                __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(pl + DD * 2 + off));
+                a_final += p.dC[(size_t)bh * DD + i] * x;
+            }
+        } else if (p.dC) {
             for (size_t i = lane; i < DD; i += 32) a_final += p.dC[(size_t)bh * DD + i] * CT[i];
+        }
         if (p.dn)
             for (int j = lane; j < DH; j += 32) a_final += p.dn[(size_t)bh * DH + j] * nT[j];
         a_final = wsum(a_final);
@@ -978,28 +1084,37 @@ size_t align64(size_t x) { return (x + 63) & ~size_t(63); }
 
 // Workspace layout in floats, each array 256-byte aligned; when `p` is given
 // its workspace pointers are set from `base`.  Returns the number of floats.
-size_t bwd_layout(long long BH, long long S, long long DH, long long NC, float *base,
+size_t bwd_layout(long long BH, long long S, long long DH, long long NC, bool tc, float *base,
                   BwdPtrs *p) {
     const size_t ng = (size_t)(BH * S), nc = (size_t)(BH * NC), DD = (size_t)(DH * DH);
+    const size_t xt = tc ? ng * DH : 0;
     const size_t sizes[] = {ng, ng, ng, ng, ng, ng, ng, ng,                 // per token
                             nc, nc, nc,                                     // per chunk
                             (size_t)BH * (NC + 1) * DD, (size_t)BH * (NC + 1) * DH,
                             ng * DH, ng * DH,                               // num', dnum'
-                            (size_t)BH * NC * DD, (size_t)BH * NC * DH};
+                            (size_t)BH * NC * DD, (size_t)BH * NC * DH,
+                            xt, xt, xt};                                    // dnum' planes, dk / dv products
     BwdPtrs unused;
     BwdPtrs *t = p ? p : &unused;
+    float *dnhl = nullptr;
     float **dst[] = {&t->logf, &t->b, &t->mt, &t->den, &t->nq, &t->A, &t->dF, &t->dnq,
                      &t->mprev, &t->mend, &t->Bsum, &t->Cst, &t->nst, &t->num, &t->dnum,
-                     &t->dCb, &t->dnb};
+                     &t->dCb, &t->dnb, &dnhl, &t->dki, &t->dvi};
     static_assert(sizeof(sizes) / sizeof(sizes[0]) == sizeof(dst) / sizeof(dst[0]),
                   "one size per workspace array");
     size_t off = 0;
     for (size_t i = 0; i < sizeof(sizes) / sizeof(sizes[0]); ++i) {
-        *dst[i] = base ? base + off : nullptr;
+        *dst[i] = base && sizes[i] ? base + off : nullptr;
         off = align64(off + sizes[i]);
     }
+    t->dnhl = dnhl;
+    t->tc = tc ? 1 : 0;
     return off;
 }
+
+// The backward's products with the chunk states run on the tensor cores for
+// bf16 inputs with DH 128 or 256 (the per-chunk token kernels' shapes).
+bool bwd_uses_tc(xlstm_dtype dt, int DH) { return dt == XLSTM_BF16 && (DH == 128 || DH == 256); }
 
 bool misaligned16(const void *p) { return ((uintptr_t)p & 15u) != 0; }
 
@@ -1015,6 +1130,45 @@ xlstm_status check_bwd_shape(int B, int NH, int S, int DH, int chunk, xlstm_dtyp
 
 unsigned blocks_for(long long n) { return (unsigned)((n + kThreads - 1) / kThreads); }
 
+// One of the four state products (bwd_tc.cuh) for every chunk: `states` holds
+// the planes of C' (NC + 1 slots per head) or dC~ (NC slots), `b` (and `b2`,
+// the low plane, when B_SPLIT) the token rows, `out` [BH, S, D] fp32.
+template <int D, bool A_T, bool B_SPLIT>
+cudaError_t launch_state_mma_t(const BwdPtrs &p, const float *states, int slots_per_head, const void *b,
+                               const void *b2, float *out, cudaStream_t st) {
+    CUtensorMap m1, m2;
+    if (!make_map_bf16(&m1, b, p.BH, p.S, D, true, 64)) return cudaErrorInvalidValue;
+    if (!make_map_bf16(&m2, B_SPLIT ? b2 : b, p.BH, p.S, D, true, 64)) return cudaErrorInvalidValue;
+    const size_t slot_bytes = (size_t)D * D * sizeof(float);
+    const int sm = bwdtc::MmaLay<D, B_SPLIT>::kBytes;
+    cudaError_t e = cudaFuncSetAttribute(bwdtc::state_mma_kernel<D, A_T, B_SPLIT>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
+    if (e != cudaSuccess) return e;
+    bwdtc::state_mma_kernel<D, A_T, B_SPLIT><<<dim3((unsigned)((long long)p.NC * p.BH), D / 128),
+                                               bwdtc::kMmaThreads, sm, st>>>(
+        m1, m2, reinterpret_cast<const uint8_t *>(states), (size_t)slots_per_head * slot_bytes, slot_bytes, out,
+        p.S, p.L, p.NC, device_status_ptr());
+    return cudaGetLastError();
+}
+
+// which: 0 C' q (-> num), 1 C'^T dnum' (-> num), 2 dC~^T v (-> dki), 3 dC~ k (-> dvi)
+template <int D>
+cudaError_t launch_state_mma(const BwdPtrs &p, int which, cudaStream_t st) {
+    const __nv_bfloat16 *dn_hi = reinterpret_cast<const __nv_bfloat16 *>(p.dnhl);
+    switch (which) {
+        case 0: return launch_state_mma_t<D, false, false>(p, p.Cst, p.NC + 1, p.q, nullptr, p.num, st);
+        case 1: return launch_state_mma_t<D, true, true>(p, p.Cst, p.NC + 1, dn_hi,
+                                                         dn_hi + (size_t)p.BH * p.S * D, p.num, st);
+        case 2: return launch_state_mma_t<D, true, false>(p, p.dCb, p.NC, p.v, nullptr, p.dki, st);
+        default: return launch_state_mma_t<D, false, false>(p, p.dCb, p.NC, p.k, nullptr, p.dvi, st);
+    }
+}
+
+cudaError_t launch_state_products(const BwdPtrs &p, int which, cudaStream_t st) {
+    KernelTimer timer("bwd_state_mma", st);
+    return p.DH == 128 ? launch_state_mma<128>(p, which, st) : launch_state_mma<256>(p, which, st);
+}
+
 template <typename T>
 cudaError_t launch_bwd(const BwdPtrs &p, cudaStream_t st) {
     const long long heads = p.BH, rows = (long long)p.BH * (p.DH + 1),
@@ -1025,8 +1179,13 @@ cudaError_t launch_bwd(const BwdPtrs &p, cudaStream_t st) {
     }
     {
         KernelTimer timer("bwd_states", st);
-        if (!launch_rows<T, false>(p, st)) bwd_states_kernel<T><<<blocks_for(rows), kThreads, 0, st>>>(p);
+        if (!launch_rows<T, false>(p, st)) {
+            if (p.tc) return cudaErrorInvalidValue;     // the planes' writer must run
+            bwd_states_kernel<T><<<blocks_for(rows), kThreads, 0, st>>>(p);
+        }
     }
+    cudaError_t e;
+    if (p.tc && (e = launch_state_products(p, 0, st)) != cudaSuccess) return e;
     {
         KernelTimer timer("bwd_token_fwd", st);
         if (!launch_token_fwd_chunk<T>(p, st) && !launch_token_warp<T, false>(p, st))
@@ -1034,8 +1193,14 @@ cudaError_t launch_bwd(const BwdPtrs &p, cudaStream_t st) {
     }
     {
         KernelTimer timer("bwd_reverse", st);
-        if (!launch_rows<T, true>(p, st)) bwd_reverse_kernel<T><<<blocks_for(rows), kThreads, 0, st>>>(p);
+        if (!launch_rows<T, true>(p, st)) {
+            if (p.tc) return cudaErrorInvalidValue;
+            bwd_reverse_kernel<T><<<blocks_for(rows), kThreads, 0, st>>>(p);
+        }
     }
+    if (p.tc)
+        for (int which = 1; which <= 3; ++which)
+            if ((e = launch_state_products(p, which, st)) != cudaSuccess) return e;
     {
         KernelTimer timer("bwd_token_grad", st);
         if (!launch_token_grad_chunk<T>(p, st) && !launch_token_warp<T, true>(p, st))
@@ -1064,7 +1229,7 @@ extern "C" xlstm_status xlstm_mlstm_bwd_workspace_size(int B, int NH, int S, int
         return XLSTM_OK;
     }
     const long long NC = (S + chunk - 1) / chunk;
-    *bytes = bwd_layout(BH, S, DH, NC, nullptr, nullptr) * sizeof(float);
+    *bytes = bwd_layout(BH, S, DH, NC, bwd_uses_tc(dt, DH), nullptr, nullptr) * sizeof(float);
     return XLSTM_OK;
 }
 
@@ -1102,7 +1267,8 @@ extern "C" xlstm_status xlstm_mlstm_bwd(const void *q, const void *k, const void
         for (int b = a + 1; b < 6; ++b)
             if (outputs[a] == outputs[b]) return XLSTM_ERR_UNSUPPORTED;
     const long long NC = (S + chunk - 1) / chunk;
-    const size_t need = bwd_layout(BH, S, DH, NC, nullptr, nullptr) * sizeof(float);
+    const bool tc = bwd_uses_tc(dt, DH);
+    const size_t need = bwd_layout(BH, S, DH, NC, tc, nullptr, nullptr) * sizeof(float);
     if (!workspace || workspace_bytes < need) return XLSTM_ERR_WORKSPACE;
 
     bwd::BwdPtrs p;
@@ -1110,7 +1276,7 @@ extern "C" xlstm_status xlstm_mlstm_bwd(const void *q, const void *k, const void
     p.ip = i_pre; p.fp = f_pre; p.op = o_pre; p.dh = dh;
     p.dC = dC; p.dn = dn;
     p.dq = dq; p.dk = dk; p.dv = dv; p.di = di; p.df = df; p.dO = d_o;
-    bwd_layout(BH, S, DH, NC, (float *)workspace, &p);
+    bwd_layout(BH, S, DH, NC, tc, (float *)workspace, &p);
     p.BH = (int)BH; p.S = S; p.DH = DH; p.L = chunk; p.NC = (int)NC;
     p.fgate_exp = fg == XLSTM_FGATE_EXP;
     cudaStream_t stream = (cudaStream_t)cuda_stream;

@@ -85,6 +85,13 @@ struct BwdPtrs {
     float *dCb;                       // [BH, NC, DH, DH] reverse state at the end of chunk c
     float *dnb;                       // [BH, NC, DH]
     int BH, S, DH, L, NC, fgate_exp;
+    // Tensor-core products with the states (bf16, DH 128 / 256): tc != 0 stores
+    // every C' and dC~ slot as two bf16 planes (high part, then low part, each
+    // DH*DH, in the 128-byte-swizzled tile order the MMAs read) instead of
+    // fp32, and the per-token kernels take the state products from:
+    void *dnhl;                       // [2][BH, S, DH] bf16: dnum' high, then low part
+    float *dki, *dvi;                 // [BH, S, DH]: v_s^T dC~ and dC~ k_s per token
+    int tc;
 };
 
 // K1, one head: log f, chunk-local cumulative log forget, the stabiliser per

@@ -65,6 +65,7 @@ int main(int argc, char **argv) {
     p.Cst = Cst.data(); p.nst = nst.data(); p.num = num.data(); p.dnum = dnum.data();
     p.dCb = dCb.data(); p.dnb = dnb.data();
     p.BH = BH; p.S = S; p.DH = DH; p.L = L; p.NC = NC; p.fgate_exp = hdr[5];
+    p.dnhl = nullptr; p.dki = nullptr; p.dvi = nullptr; p.tc = 0;
 
     if (S > 0) {
         for (int h = 0; h < BH; ++h) xlstm::bwd::gates_head(p, h);

@@ -19,10 +19,11 @@ STACK_LIMIT = 1024             # default per-thread stack, bytes
 # kernels on the forward / decode hot path: no spills allowed
 HOT = ("segment_output_tc_kernel", "segment_summary_tc_kernel", "segment_scan_kernel",
        "gate_prologue_kernel", "step_stream_kernel", "step_rows_kernel", "step_state_kernel",
-       "headnorm_gate_kernel", "combine_keysplit_kernel", "slstm_cluster_kernel")
+       "headnorm_gate_kernel", "combine_keysplit_kernel", "slstm_cluster_kernel", "state_mma_kernel",
+       "state_fold_kernel")
 # threads per CTA the launchers use for the tensor-core and streamed kernels
 LAUNCH_THREADS = {"segment_output_tc_kernel": 448, "segment_summary_tc_kernel": 320,
-                  "slstm_cluster_kernel": 256}
+                  "slstm_cluster_kernel": 256, "state_mma_kernel": 128}
 
 
 def _ptxas_report(src):
