@@ -98,11 +98,7 @@ template <int N> __device__ __forceinline__ void cp_async_wait() {
 // 32 rows' raw coefficients (v or dnum' entries) and the per-token scalars;
 // the next chunk's stage is filled by cp.async while this one is used, so the
 // walk over chunks waits on no global-memory round trip.
-//
-// SPLIT: the DH x DH slots are stored as bf16 high and low planes in the
-// tensor-core kernels' tile order (bwdtc::plane_offset) instead of fp32 rows;
-// the normaliser row stays fp32.
-template <typename T, int NCL, bool REVERSE, bool SPLIT>
+template <typename T, int NCL, bool REVERSE>
 __global__ void __launch_bounds__(kRowThreads) bwd_rows_kernel(BwdPtrs p) {
     constexpr int DH = 32 * NCL;
     extern __shared__ __align__(16) uint8_t rows_smem[];
@@ -159,22 +155,9 @@ __global__ void __launch_bounds__(kRowThreads) bwd_rows_kernel(BwdPtrs p) {
     };
     // row r's values (lane + 32 j) into `slot`
     auto store_row = [&](int r, int slot, const float (&x)[NCL]) {
-        if (SPLIT && r < DH) {
-            uint8_t *pl = reinterpret_cast<uint8_t *>(
-                (REVERSE ? p.dCb + (size_t)bh * NC * DD : p.Cst + (size_t)bh * (NC + 1) * DD) + (size_t)slot * DD);
+        float *dst = slot_ptr(r, slot);
 #pragma unroll
-            for (int j = 0; j < NCL; ++j) {
-                const uint32_t off = bwdtc::plane_offset(r, lane + 32 * j, DH);
-                const __nv_bfloat16 hi = __float2bfloat16_rn(x[j]);
-                *reinterpret_cast<__nv_bfloat16 *>(pl + off) = hi;
-                *reinterpret_cast<__nv_bfloat16 *>(pl + DD * 2 + off) =
-                    __float2bfloat16_rn(x[j] - __bfloat162float(hi));
-            }
-        } else {
-            float *dst = slot_ptr(r, slot);
-#pragma unroll
-            for (int j = 0; j < NCL; ++j) dst[lane + 32 * j] = x[j];
-        }
+        for (int j = 0; j < NCL; ++j) dst[lane + 32 * j] = x[j];
     };
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -260,24 +243,10 @@ bool launch_rows(const BwdPtrs &p, cudaStream_t st) {
     const size_t sm = rows_smem_bytes<T>(p.L, p.DH);
     if (sm > 232448) return false;        // two stages do not fit (fp32 at DH 512): per-thread kernel
     const dim3 grid((unsigned)((p.DH + 1 + kRowBlock - 1) / kRowBlock), (unsigned)p.BH);
-    if (p.tc) {                           // bf16, DH 128 / 256: slots as bf16 planes
-        if constexpr (sizeof(T) == 2) {
-#define XLSTM_BWD_ROWS_SPLIT(N)                                                                   \
-            if (ncl == N) {                                                                        \
-                cudaFuncSetAttribute(bwd_rows_kernel<T, N, REVERSE, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm); \
-                bwd_rows_kernel<T, N, REVERSE, true><<<grid, kRowThreads, sm, st>>>(p);            \
-                return true;                                                                       \
-            }
-            XLSTM_BWD_ROWS_SPLIT(4)
-            XLSTM_BWD_ROWS_SPLIT(8)
-#undef XLSTM_BWD_ROWS_SPLIT
-        }
-        return false;
-    }
 #define XLSTM_BWD_ROWS(N)                                                                         \
     if (ncl == N) {                                                                                \
-        cudaFuncSetAttribute(bwd_rows_kernel<T, N, REVERSE, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm); \
-        bwd_rows_kernel<T, N, REVERSE, false><<<grid, kRowThreads, sm, st>>>(p);                   \
+        cudaFuncSetAttribute(bwd_rows_kernel<T, N, REVERSE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm); \
+        bwd_rows_kernel<T, N, REVERSE><<<grid, kRowThreads, sm, st>>>(p);                          \
         return true;                                                                               \
     }
     XLSTM_BWD_ROWS(1)
@@ -962,121 +931,188 @@ bool launch_token_warp(const BwdPtrs &p, cudaStream_t st) {
 // m_t = b_t + max(m_prev, max_{s <= t in the chunk} (itilde_s - b_s)) with b
 // chunk-local (equal to the sequential max-plus recurrence up to rounding; the
 // backward only needs one consistent m with all exponents <= 0).
-__global__ void __launch_bounds__(128) bwd_gates_warp_kernel(BwdPtrs p) {
-    const long long w = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    const int lane = threadIdx.x & 31;
-    if (w >= p.BH) return;
-    const int bh = (int)w, S = p.S, L = p.L;
-    const size_t base = (size_t)bh * S, cbase = (size_t)bh * p.NC;
-    float m = 0.f;
-    for (int c = 0; c < p.NC; ++c) {
-        const int a = c * L, e = bwd::imin(S, a + L);
-        float carry = 0.f, umax = -INFINITY, mlast = m;
-        if (lane == 0) p.mprev[cbase + c] = m;
-        for (int t0 = a; t0 < e; t0 += 32) {
-            const int t = t0 + lane;
-            const bool ok = t < e;
-            const float fpre = ok ? p.fp[base + t] : 0.f;
-            const float lf = ok ? (p.fgate_exp ? fpre : bwd::log_sigmoid_hd(fpre)) : 0.f;
-            float b = lf;
+// K1 and K6 with one CTA per head: the per-chunk work (scans over a chunk's
+// tokens, one warp per chunk) runs in parallel, and only the short chain over
+// chunks (the stabiliser carried from chunk to chunk; the suffix sums of the
+// chunks' d log f totals) is walked by one thread, from shared memory.
+constexpr int kSeqThreads = 1024;
+constexpr int kSeqTile = 2048;                 // chunks per pass through shared memory
+
+// K1: (a) per chunk, log f, the chunk-local cumulative log forget b and the
+// chunk-local prefix maximum of itilde - b (held in mt for now), the chunk's
+// total (Bsum) and maximum; (b) the chunk-to-chunk stabiliser
+// m_end = Bsum + max(m_prev, chunk maximum), m_0 = 0; (c) per token
+// m_t = b_t + max(m_prev, prefix maximum).  Same operations per value as the
+// token-by-token unrolled form b_t + max(m_prev, max_{s<=t}(itilde_s - b_s)).
+__global__ void __launch_bounds__(kSeqThreads) bwd_gates_seq_kernel(BwdPtrs p) {
+    __shared__ float s_u[kSeqTile], s_B[kSeqTile], s_m[kSeqTile];
+    __shared__ float s_carry;
+    const int bh = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int S = p.S, L = p.L, NC = p.NC;
+    const size_t base = (size_t)bh * S, cbase = (size_t)bh * NC;
+    for (int c0 = 0; c0 < NC; c0 += kSeqTile) {
+        const int nt = bwd::imin(kSeqTile, NC - c0);
+        for (int cc = warp; cc < nt; cc += kSeqThreads / 32) {
+            const int a = (c0 + cc) * L, e = bwd::imin(S, a + L);
+            float carry = 0.f, umax = -INFINITY;
+            for (int t0 = a; t0 < e; t0 += 32) {
+                const int t = t0 + lane;
+                const bool ok = t < e;
+                const float fpre = ok ? p.fp[base + t] : 0.f;
+                const float lf = ok ? (p.fgate_exp ? fpre : bwd::log_sigmoid_hd(fpre)) : 0.f;
+                float b = lf;
 #pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const float y = __shfl_up_sync(0xffffffffu, b, o);
-                if (lane >= o) b += y;
-            }
-            b += carry;
-            float u = ok ? p.ip[base + t] - b : -INFINITY;
+                for (int o = 1; o < 32; o <<= 1) {
+                    const float y = __shfl_up_sync(0xffffffffu, b, o);
+                    if (lane >= o) b += y;
+                }
+                b += carry;
+                float u = ok ? p.ip[base + t] - b : -INFINITY;
 #pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const float y = __shfl_up_sync(0xffffffffu, u, o);
-                if (lane >= o) u = fmaxf(u, y);
+                for (int o = 1; o < 32; o <<= 1) {
+                    const float y = __shfl_up_sync(0xffffffffu, u, o);
+                    if (lane >= o) u = fmaxf(u, y);
+                }
+                u = fmaxf(u, umax);
+                if (ok) {
+                    p.logf[base + t] = lf;
+                    p.b[base + t] = b;
+                    p.mt[base + t] = u;
+                }
+                const int last = bwd::imin(31, e - 1 - t0);
+                carry = __shfl_sync(0xffffffffu, b, last);
+                umax = __shfl_sync(0xffffffffu, u, last);
             }
-            u = fmaxf(u, umax);
-            const float mt = b + fmaxf(m, u);
-            if (ok) {
-                p.logf[base + t] = lf;
-                p.b[base + t] = b;
-                p.mt[base + t] = mt;
+            if (lane == 0) {
+                s_B[cc] = carry;
+                s_u[cc] = umax;
             }
-            const int last = bwd::imin(31, e - 1 - t0);
-            carry = __shfl_sync(0xffffffffu, b, last);
-            umax = __shfl_sync(0xffffffffu, u, last);
-            mlast = __shfl_sync(0xffffffffu, mt, last);
         }
-        if (lane == 0) {
-            p.mend[cbase + c] = mlast;
-            p.Bsum[cbase + c] = carry;
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            float m = c0 == 0 ? 0.f : s_carry;
+            for (int cc = 0; cc < nt; ++cc) {
+                s_m[cc] = m;
+                p.mprev[cbase + c0 + cc] = m;
+                p.Bsum[cbase + c0 + cc] = s_B[cc];
+                m = s_B[cc] + fmaxf(m, s_u[cc]);
+                p.mend[cbase + c0 + cc] = m;
+            }
+            s_carry = m;
         }
-        m = mlast;
+        __syncthreads();
+        for (int cc = warp; cc < nt; cc += kSeqThreads / 32) {
+            const int a = (c0 + cc) * L, e = bwd::imin(S, a + L);
+            const float m = s_m[cc];
+            for (int t = a + lane; t < e; t += 32) p.mt[base + t] = p.b[base + t] + fmaxf(m, p.mt[base + t]);
+        }
+        __syncthreads();
     }
 }
 
-__global__ void __launch_bounds__(128) bwd_forget_warp_kernel(BwdPtrs p) {
+// K6, first part (only with final-state cotangents), one warp per head: the
+// returned state's stabiliser m_T = F_T + max(0, max_s(itilde_s - F_s)); its
+// explicit dependence moves A_final = sum dC' o C'_T + sum dn' o n'_T from
+// itilde to F at the maximising key s*.
+__global__ void __launch_bounds__(128) bwd_final_state_kernel(BwdPtrs p) {
     const long long w = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
     if (w >= p.BH) return;
     const int bh = (int)w, S = p.S, DH = p.DH, NC = p.NC;
     const size_t base = (size_t)bh * S, DD = (size_t)DH * DH;
-    if (p.dC || p.dn) {
-        float a_final = 0.f;
-        const float *CT = p.Cst + ((size_t)bh * (NC + 1) + NC) * DD;
-        const float *nT = p.nst + ((size_t)bh * (NC + 1) + NC) * DH;
-        if (p.dC && p.tc) {                    // C'_T as bf16 high + low planes
-            const uint8_t *pl = reinterpret_cast<const uint8_t *>(CT);
-            for (size_t i = lane; i < DD; i += 32) {
-                const uint32_t off = bwdtc::plane_offset((int)(i / DH), (int)(i % DH), DH);
-                const float x = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(pl + off)) +
-                                __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(pl + DD * 2 + off));
-                a_final += p.dC[(size_t)bh * DD + i] * x;
-            }
-        } else if (p.dC) {
-            for (size_t i = lane; i < DD; i += 32) a_final += p.dC[(size_t)bh * DD + i] * CT[i];
+    float a_final = 0.f;
+    const float *CT = p.Cst + ((size_t)bh * (NC + 1) + NC) * DD;
+    const float *nT = p.nst + ((size_t)bh * (NC + 1) + NC) * DH;
+    if (p.dC && p.tc) {                    // C'_T as bf16 high + low planes
+        const uint8_t *pl = reinterpret_cast<const uint8_t *>(CT);
+        for (size_t i = lane; i < DD; i += 32) {
+            const uint32_t off = bwdtc::plane_offset((int)(i / DH), (int)(i % DH), DH);
+            const float x = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(pl + off)) +
+                            __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(pl + DD * 2 + off));
+            a_final += p.dC[(size_t)bh * DD + i] * x;
         }
-        if (p.dn)
-            for (int j = lane; j < DH; j += 32) a_final += p.dn[(size_t)bh * DH + j] * nT[j];
-        a_final = wsum(a_final);
-        // the first t with the largest itilde_t - F_t, if that is > 0 (m_T's maximising key)
-        float F0 = 0.f, best = 0.f;
-        int sstar = -1;
-        for (int t0 = 0; t0 < S; t0 += 32) {
-            const int t = t0 + lane;
-            float F = t < S ? p.logf[base + t] : 0.f;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const float y = __shfl_up_sync(0xffffffffu, F, o);
-                if (lane >= o) F += y;
-            }
-            F += F0;
-            float cand = t < S ? p.ip[base + t] - F : -INFINITY;
-            int ct = t;
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {             // max, earliest token on ties
-                const float oc = __shfl_xor_sync(0xffffffffu, cand, o);
-                const int ot = __shfl_xor_sync(0xffffffffu, ct, o);
-                if (oc > cand || (oc == cand && ot < ct)) { cand = oc; ct = ot; }
-            }
-            if (cand > best) { best = cand; sstar = ct; }
-            F0 = __shfl_sync(0xffffffffu, F, 31);
-        }
-        if (lane == 0 && sstar >= 0) {
-            p.di[base + sstar] -= a_final;
-            p.dF[base + sstar] += a_final;
-        }
-        __syncwarp();
+    } else if (p.dC) {
+        for (size_t i = lane; i < DD; i += 32) a_final += p.dC[(size_t)bh * DD + i] * CT[i];
     }
-    float acc = 0.f;                                     // reverse cumulative sum of dF
-    const int ng = (S + 31) / 32;
-    for (int gi = ng - 1; gi >= 0; --gi) {
-        const int t = gi * 32 + lane;
-        float x = t < S ? p.dF[base + t] : 0.f;
+    if (p.dn)
+        for (int j = lane; j < DH; j += 32) a_final += p.dn[(size_t)bh * DH + j] * nT[j];
+    a_final = wsum(a_final);
+    // the first t with the largest itilde_t - F_t, if that is > 0 (m_T's maximising key)
+    float F0 = 0.f, best = 0.f;
+    int sstar = -1;
+    for (int t0 = 0; t0 < S; t0 += 32) {
+        const int t = t0 + lane;
+        float F = t < S ? p.logf[base + t] : 0.f;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
-            const float y = __shfl_down_sync(0xffffffffu, x, o);
-            if (lane + o < 32) x += y;
+            const float y = __shfl_up_sync(0xffffffffu, F, o);
+            if (lane >= o) F += y;
         }
-        x += acc;
-        if (t < S) p.df[base + t] = p.fgate_exp ? x : x * bwd::sigmoid_hd(-p.fp[base + t]);
-        acc = __shfl_sync(0xffffffffu, x, 0);
+        F += F0;
+        float cand = t < S ? p.ip[base + t] - F : -INFINITY;
+        int ct = t;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {             // max, earliest token on ties
+            const float oc = __shfl_xor_sync(0xffffffffu, cand, o);
+            const int ot = __shfl_xor_sync(0xffffffffu, ct, o);
+            if (oc > cand || (oc == cand && ot < ct)) { cand = oc; ct = ot; }
+        }
+        if (cand > best) { best = cand; sstar = ct; }
+        F0 = __shfl_sync(0xffffffffu, F, 31);
+    }
+    if (lane == 0 && sstar >= 0) {
+        p.di[base + sstar] -= a_final;
+        p.dF[base + sstar] += a_final;
+    }
+}
+
+// K6, second part: d log f_j = sum_{t >= j} dF_t.  (a) each chunk's total,
+// (b) the suffix sums of the totals (one thread, last chunk first), (c) each
+// chunk's own reverse cumulative sum started from its suffix; then the forget
+// activation's derivative.
+__global__ void __launch_bounds__(kSeqThreads) bwd_forget_seq_kernel(BwdPtrs p) {
+    __shared__ float s_sum[kSeqTile];
+    __shared__ float s_carry;
+    const int bh = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int S = p.S, L = p.L, NC = p.NC;
+    const size_t base = (size_t)bh * S;
+    for (int c1 = NC; c1 > 0; c1 -= kSeqTile) {
+        const int c0 = c1 > kSeqTile ? c1 - kSeqTile : 0, nt = c1 - c0;
+        for (int cc = warp; cc < nt; cc += kSeqThreads / 32) {
+            const int a = (c0 + cc) * L, e = bwd::imin(S, a + L);
+            float x = 0.f;
+            for (int t = a + lane; t < e; t += 32) x += p.dF[base + t];
+            x = wsum(x);
+            if (lane == 0) s_sum[cc] = x;
+        }
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            float acc = c1 == NC ? 0.f : s_carry;
+            for (int cc = nt - 1; cc >= 0; --cc) {
+                const float x = s_sum[cc];
+                s_sum[cc] = acc;                 // total of the chunks after cc
+                acc += x;
+            }
+            s_carry = acc;
+        }
+        __syncthreads();
+        for (int cc = warp; cc < nt; cc += kSeqThreads / 32) {
+            const int a = (c0 + cc) * L, e = bwd::imin(S, a + L);
+            float acc = s_sum[cc];
+            for (int g0 = a + ((e - a - 1) / 32) * 32; g0 >= a; g0 -= 32) {
+                const int t = g0 + lane;
+                float x = t < e ? p.dF[base + t] : 0.f;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const float y = __shfl_down_sync(0xffffffffu, x, o);
+                    if (lane + o < 32) x += y;
+                }
+                x += acc;
+                if (t < e) p.df[base + t] = p.fgate_exp ? x : x * bwd::sigmoid_hd(-p.fp[base + t]);
+                acc = __shfl_sync(0xffffffffu, x, 0);
+            }
+        }
+        __syncthreads();
     }
 }
 
@@ -1164,6 +1200,40 @@ cudaError_t launch_state_mma(const BwdPtrs &p, int which, cudaStream_t st) {
     }
 }
 
+// The state recurrences on the tensor cores (bwd_tc.cuh): every chunk's
+// increment at once, then the scan over chunks.
+template <int D, bool REVERSE>
+cudaError_t launch_state_recurrence_t(const BwdPtrs &p, cudaStream_t st) {
+    const int c_first = REVERSE ? 1 : 0, nce = REVERSE ? p.NC - 1 : p.NC;
+    if (nce > 0) {
+        CUtensorMap ma, ma2, mb;
+        const __nv_bfloat16 *dn_hi = reinterpret_cast<const __nv_bfloat16 *>(p.dnhl);
+        const void *a1 = REVERSE ? (const void *)dn_hi : p.v;
+        const void *a2 = REVERSE ? (const void *)(dn_hi + (size_t)p.BH * p.S * D) : p.v;
+        if (!make_map_bf16(&ma, a1, p.BH, p.S, D, true, 64) || !make_map_bf16(&ma2, a2, p.BH, p.S, D, true, 64) ||
+            !make_map_bf16(&mb, REVERSE ? p.q : p.k, p.BH, p.S, D, true, 64))
+            return cudaErrorInvalidValue;
+        const int sm = bwdtc::DeltaLay<D, REVERSE>::kBytes;
+        cudaError_t e = cudaFuncSetAttribute(bwdtc::delta_mma_kernel<D, REVERSE>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
+        if (e != cudaSuccess) return e;
+        KernelTimer timer(REVERSE ? "bwd_reverse_mma" : "bwd_states_mma", st);
+        bwdtc::delta_mma_kernel<D, REVERSE><<<dim3((unsigned)((long long)nce * p.BH), D / 128), bwdtc::kMmaThreads,
+                                              sm, st>>>(ma, ma2, mb, p, c_first, nce, device_status_ptr());
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    KernelTimer timer(REVERSE ? "bwd_reverse_scan" : "bwd_states_scan", st);
+    const size_t threads = (size_t)D * D / 2 + D / 2;
+    bwdtc::state_scan_kernel<D, REVERSE><<<dim3((unsigned)((threads + 255) / 256), (unsigned)p.BH), 256, 0, st>>>(p);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_state_recurrence(const BwdPtrs &p, bool reverse, cudaStream_t st) {
+    if (p.DH == 128)
+        return reverse ? launch_state_recurrence_t<128, true>(p, st) : launch_state_recurrence_t<128, false>(p, st);
+    return reverse ? launch_state_recurrence_t<256, true>(p, st) : launch_state_recurrence_t<256, false>(p, st);
+}
+
 cudaError_t launch_state_products(const BwdPtrs &p, int which, cudaStream_t st) {
     KernelTimer timer("bwd_state_mma", st);
     return p.DH == 128 ? launch_state_mma<128>(p, which, st) : launch_state_mma<256>(p, which, st);
@@ -1175,32 +1245,29 @@ cudaError_t launch_bwd(const BwdPtrs &p, cudaStream_t st) {
                     tokens = (long long)p.BH * p.S;
     {
         KernelTimer timer("bwd_gates", st);
-        bwd_gates_warp_kernel<<<(unsigned)((heads * 32 + 127) / 128), 128, 0, st>>>(p);
-    }
-    {
-        KernelTimer timer("bwd_states", st);
-        if (!launch_rows<T, false>(p, st)) {
-            if (p.tc) return cudaErrorInvalidValue;     // the planes' writer must run
-            bwd_states_kernel<T><<<blocks_for(rows), kThreads, 0, st>>>(p);
-        }
+        bwd_gates_seq_kernel<<<(unsigned)heads, kSeqThreads, 0, st>>>(p);
     }
     cudaError_t e;
-    if (p.tc && (e = launch_state_products(p, 0, st)) != cudaSuccess) return e;
+    if (p.tc) {
+        if ((e = launch_state_recurrence(p, false, st)) != cudaSuccess) return e;
+        if ((e = launch_state_products(p, 0, st)) != cudaSuccess) return e;
+    } else {
+        KernelTimer timer("bwd_states", st);
+        if (!launch_rows<T, false>(p, st)) bwd_states_kernel<T><<<blocks_for(rows), kThreads, 0, st>>>(p);
+    }
     {
         KernelTimer timer("bwd_token_fwd", st);
         if (!launch_token_fwd_chunk<T>(p, st) && !launch_token_warp<T, false>(p, st))
             bwd_token_fwd_kernel<T><<<blocks_for(tokens), kThreads, 0, st>>>(p);
     }
-    {
-        KernelTimer timer("bwd_reverse", st);
-        if (!launch_rows<T, true>(p, st)) {
-            if (p.tc) return cudaErrorInvalidValue;
-            bwd_reverse_kernel<T><<<blocks_for(rows), kThreads, 0, st>>>(p);
-        }
-    }
-    if (p.tc)
+    if (p.tc) {
+        if ((e = launch_state_recurrence(p, true, st)) != cudaSuccess) return e;
         for (int which = 1; which <= 3; ++which)
             if ((e = launch_state_products(p, which, st)) != cudaSuccess) return e;
+    } else {
+        KernelTimer timer("bwd_reverse", st);
+        if (!launch_rows<T, true>(p, st)) bwd_reverse_kernel<T><<<blocks_for(rows), kThreads, 0, st>>>(p);
+    }
     {
         KernelTimer timer("bwd_token_grad", st);
         if (!launch_token_grad_chunk<T>(p, st) && !launch_token_warp<T, true>(p, st))
@@ -1208,7 +1275,8 @@ cudaError_t launch_bwd(const BwdPtrs &p, cudaStream_t st) {
     }
     {
         KernelTimer timer("bwd_forget", st);
-        bwd_forget_warp_kernel<<<(unsigned)((heads * 32 + 127) / 128), 128, 0, st>>>(p);
+        if (p.dC || p.dn) bwd_final_state_kernel<<<(unsigned)((heads * 32 + 127) / 128), 128, 0, st>>>(p);
+        bwd_forget_seq_kernel<<<(unsigned)heads, kSeqThreads, 0, st>>>(p);
     }
     return cudaGetLastError();
 }

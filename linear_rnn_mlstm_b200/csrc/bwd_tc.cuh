@@ -81,6 +81,7 @@ state_mma_kernel(const __grid_constant__ CUtensorMap map_b, const __grid_constan
         *abort_flag = 0;
         fence_mbar_init();
     }
+    __syncwarp();
     if (warp == 0) tmem_alloc(tslot, 64);
     tc_fence_before();
     __syncthreads();
@@ -135,6 +136,7 @@ state_mma_kernel(const __grid_constant__ CUtensorMap map_b, const __grid_constan
     __syncwarp();
     int ok = 0;
     if (lane == 0) ok = mbar_wait(&bar[1], 0, abort_flag, status) ? 1 : 0;
+    __syncwarp();
     const bool done = __shfl_sync(0xffffffffu, ok, 0) != 0;
     if (done) {
         tc_fence_after();
@@ -156,6 +158,301 @@ state_mma_kernel(const __grid_constant__ CUtensorMap map_b, const __grid_constan
     if (warp == 0) {
         tc_fence_after();
         tmem_dealloc(tacc, 64);
+    }
+}
+
+// ------------------------------------------------------------ state increments
+// The chunk recurrences of the states, C'_{c+1} = decay_c C'_c + dC_c (forward)
+// and dC~_{c-1} = decay_c dC~_c + ddC_c (reverse), split into a parallel part
+// and a scan.  The increments, for every chunk at once on the tensor cores:
+//   dC_c[r][j]  = sum_{s in c} w_s v_s[r] k_s[j],  w_s = e^{B_c - b_s + itilde_s - m_end,c} / sqrt(d)
+//   ddC_c[r][j] = sum_{t in c} g_t dnum'_t[r] q_t[j],  g_t = e^{b_t + m_prev,c - m_t}
+// as one M = 128 (rows r), N = DH (columns j), K = 64 (tokens) product per
+// (chunk, row tile, head): A = (w v)^T, MN-major, formed in shared memory from
+// the TMA-loaded v (or dnum' high + low) tile scaled per token and split into
+// bf16 high and low parts; B = k (or q) as loaded, MN-major.  The fp32
+// accumulator leaves tensor memory as bf16 high / low planes staged in shared
+// memory in the state planes' tile order and stored by two bulk copies into
+// the slot the scan turns into the state (forward: slot c + 1; reverse: slot
+// c - 1).  The normaliser's increment (w_s k_s, or g_t dnq'_t q_t, summed)
+// is formed on the CUDA cores from the same B tile.
+template <int D, bool REVERSE>
+struct DeltaLay {
+    static constexpr int kRaw = 0;                                   // v: 2 boxes; dnum': 2 planes x 2 boxes
+    static constexpr int kRawBytes = REVERSE ? 32768 : 16384;
+    static constexpr int kA = kRaw + kRawBytes;                      // A high, then low: 2 x 16 KB
+    static constexpr int kB = kA + 32768;                            // D / 64 boxes of 64 tokens
+    static constexpr int kIn = kB + D / 64 * 8192;
+    static constexpr int kOut = 2 * (D / 64) * 16384;                // staged planes (over the inputs)
+    static constexpr int kRegion = kIn > kOut ? kIn : kOut;
+    static constexpr int kW = kRegion;                               // w[64], wn[64]
+    static constexpr int kBar = kW + 512;
+    static constexpr int kBytes = kBar + 64 + 1024;
+};
+
+__device__ __forceinline__ void bulk_store(void *gdst, const void *ssrc, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst),
+                 "r"(tc::smem_u32(ssrc)), "r"(bytes)
+                 : "memory");
+}
+
+// grid (chunks x heads, D / 128); chunk c = c_first + blockIdx.x % nce.
+template <int D, bool REVERSE>
+__global__ void __launch_bounds__(kMmaThreads, 1)
+delta_mma_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_a2,
+                 const __grid_constant__ CUtensorMap map_b, bwd::BwdPtrs p, int c_first, int nce,
+                 unsigned int *status) {
+    using Lay = DeltaLay<D, REVERSE>;
+    using namespace tc;
+    extern __shared__ uint8_t delta_smem_raw[];
+    uint8_t *smem = align1k(delta_smem_raw);
+    float *sw = reinterpret_cast<float *>(smem + Lay::kW), *swn = sw + 64;
+    uint64_t *bar = reinterpret_cast<uint64_t *>(smem + Lay::kBar);
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(smem + Lay::kBar + 16);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + Lay::kBar + 20);
+    const int c = c_first + (int)(blockIdx.x % (unsigned)nce), bh = (int)(blockIdx.x / (unsigned)nce);
+    const int mt = blockIdx.y, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int S = p.S, L = p.L, NC = p.NC;
+    const int a0 = c * L, n = min(S, a0 + L) - a0;
+    const size_t DD = (size_t)D * D, hc = (size_t)bh * NC + c, row0 = (size_t)bh * S + a0;
+
+    if (tid == 0) {
+        mbar_init(&bar[0], 1);
+        mbar_init(&bar[1], 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+        mbar_arrive_expect_tx(&bar[0], (uint32_t)(Lay::kRawBytes + D / 64 * 8192));
+        for (int h = 0; h < 2; ++h) {
+            tma_load_3d(smem + Lay::kRaw + h * 8192, &map_a, &bar[0], 128 * mt + 64 * h, a0, bh);
+            if (REVERSE) tma_load_3d(smem + Lay::kRaw + 16384 + h * 8192, &map_a2, &bar[0], 128 * mt + 64 * h, a0, bh);
+        }
+        for (int a = 0; a < D / 64; ++a) tma_load_3d(smem + Lay::kB + a * 8192, &map_b, &bar[0], 64 * a, a0, bh);
+    }
+    __syncwarp();
+    if (warp == 0) tmem_alloc(tslot, D);
+    if (tid < 64) {                                  // per-token weights; 0 past the chunk
+        float w = 0.f, wn = 0.f;
+        if (tid < n) {
+            const size_t ts = row0 + tid;
+            if (REVERSE) {
+                w = expf(p.b[ts] + p.mprev[hc] - p.mt[ts]);
+                wn = w * p.dnq[ts];
+            } else {
+                w = expf(p.Bsum[hc] - p.b[ts] + p.ip[ts] - p.mend[hc]) * rsqrtf((float)D);
+                wn = w;
+            }
+        }
+        sw[tid] = w;
+        swn[tid] = wn;
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tacc = *tslot;
+    int ok = 0;
+    if (lane == 0) ok = mbar_wait(&bar[0], 0, abort_flag, status) ? 1 : 0;
+    __syncwarp();                                    // orders the loaded tiles for the whole warp
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    if (ok) {
+        // A = (w v)^T: every 16-byte piece of the raw tile is scaled by its row's
+        // (token's) weight and split, in place of the same piece in both planes
+        for (int e = tid; e < 16384 / 16; e += kMmaThreads) {
+            const int s = (e * 16 % 8192) / 128;
+            const float w = sw[s];
+            uint4 raw = reinterpret_cast<const uint4 *>(smem + Lay::kRaw)[e];
+            float x[8];
+            const __nv_bfloat16 *rb = reinterpret_cast<const __nv_bfloat16 *>(&raw);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) x[i] = __bfloat162float(rb[i]);
+            if (REVERSE) {
+                const uint4 low = reinterpret_cast<const uint4 *>(smem + Lay::kRaw + 16384)[e];
+                const __nv_bfloat16 *lb = reinterpret_cast<const __nv_bfloat16 *>(&low);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) x[i] += __bfloat162float(lb[i]);
+            }
+            uint32_t hi[4], lo[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float x0 = w * x[2 * i], x1 = w * x[2 * i + 1];
+                hi[i] = cvt_bf16x2(x0, x1);
+                const __nv_bfloat162 h2 = *reinterpret_cast<const __nv_bfloat162 *>(&hi[i]);
+                lo[i] = cvt_bf16x2(x0 - __low2float(h2), x1 - __high2float(h2));
+            }
+            reinterpret_cast<uint4 *>(smem + Lay::kA)[e] = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+            reinterpret_cast<uint4 *>(smem + Lay::kA + 16384)[e] = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        }
+        fence_async_smem();
+    }
+    __syncthreads();
+    if (ok && tid == 0) {
+        tc_fence_after();
+        const uint32_t idesc = idesc_f32acc(kFmtBF16, kFmtBF16, true, true, 128, D);
+        const uint32_t sa = smem_u32(smem + Lay::kA), sb = smem_u32(smem + Lay::kB);
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+            const uint64_t bdesc = sdesc_sw128(sb + ks * 2048, 8192, 1024);
+            mma_bf16_ss(tacc, sdesc_sw128(sa + ks * 2048, 8192, 1024), bdesc, idesc, ks > 0 ? 1u : 0u);
+            mma_bf16_ss(tacc, sdesc_sw128(sa + 16384 + ks * 2048, 8192, 1024), bdesc, idesc, 1u);
+        }
+        mma_commit(&bar[1]);
+    }
+    if (ok && mt == 0) {                             // the normaliser's increment
+        float *dn = REVERSE ? p.dnb + ((size_t)bh * NC + c - 1) * D : p.nst + ((size_t)bh * (NC + 1) + c + 1) * D;
+        for (int j = tid; j < D; j += kMmaThreads) {
+            const uint8_t *box = smem + Lay::kB + (j >> 6) * 8192;
+            float acc = 0.f;
+            for (int s = 0; s < n; ++s) {
+                const uint32_t off = (uint32_t)s * 128u + ((uint32_t)(((j & 63) >> 3) ^ (s & 7)) << 4) +
+                                     ((uint32_t)(j & 7) << 1);
+                acc += swn[s] * __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(box + off));
+            }
+            dn[j] = acc;
+        }
+    }
+    __syncthreads();                                 // the B tile is read: the inputs may be overwritten
+    int done = 0;
+    if (ok && lane == 0) done = mbar_wait(&bar[1], 0, abort_flag, status) ? 1 : 0;
+    __syncwarp();
+    done = __shfl_sync(0xffffffffu, done, 0);
+    if (done) {
+        tc_fence_after();
+        const int rr = 32 * warp + lane;             // this thread's row of the tile
+#pragma unroll 1
+        for (int q = 0; q < D / 16; ++q) {
+            uint32_t v[16];
+            tmem_ld16(tacc + ((uint32_t)(32 * warp) << 16) + 16 * q, v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                uint32_t hi[4], lo[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float x0 = __uint_as_float(v[8 * half + 2 * i]), x1 = __uint_as_float(v[8 * half + 2 * i + 1]);
+                    hi[i] = cvt_bf16x2(x0, x1);
+                    const __nv_bfloat162 h2 = *reinterpret_cast<const __nv_bfloat162 *>(&hi[i]);
+                    lo[i] = cvt_bf16x2(x0 - __low2float(h2), x1 - __high2float(h2));
+                }
+                const int j0 = 16 * q + 8 * half;
+                const uint32_t off = (uint32_t)(j0 >> 6) * 16384u + (uint32_t)rr * 128u +
+                                     ((uint32_t)(((j0 & 63) >> 3) ^ (rr & 7)) << 4);
+                *reinterpret_cast<uint4 *>(smem + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+                *reinterpret_cast<uint4 *>(smem + (D / 64) * 16384 + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+            }
+        }
+        fence_async_smem();
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (tid == 0 && done) {
+        uint8_t *slot = reinterpret_cast<uint8_t *>(REVERSE ? p.dCb + ((size_t)bh * NC + c - 1) * DD
+                                                            : p.Cst + ((size_t)bh * (NC + 1) + c + 1) * DD);
+        const uint32_t bytes = (uint32_t)(D / 64) * 16384u;
+        for (int pl = 0; pl < 2; ++pl)
+            bulk_store(slot + (size_t)pl * DD * 2 + (size_t)mt * bytes, smem + pl * bytes, bytes);
+        bulk_commit();
+        bulk_wait_all();
+    }
+    if (tid == 0 && !ok) mbar_wait(&bar[0], 0, nullptr, nullptr);    // no copy left in flight
+    __syncwarp();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tacc, D);
+    }
+}
+
+// The scans: one thread per pair of state elements (one 32-bit word of each
+// bf16 plane; the planes' tile order is the same in every slot, so the
+// recurrence is elementwise on words) or per pair of normaliser elements,
+// walking the chunks with the running values in fp32 registers.  Forward:
+// slot 0 = 0, slot c + 1 = decay_c slot c + increment (read from slot c + 1).
+// Reverse: slot NC - 1 = the final-state cotangent (or 0), slot c - 1 =
+// decay_c slot c + increment (read from slot c - 1).
+template <int D, bool REVERSE>
+__global__ void __launch_bounds__(256) state_scan_kernel(bwd::BwdPtrs p) {
+    const int bh = blockIdx.y, NC = p.NC;
+    const size_t DD = (size_t)D * D;
+    const size_t wi = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const size_t nwords = DD / 2;
+    if (wi >= nwords + D / 2) return;
+    const size_t hbase = (size_t)bh * NC;
+    float x0 = 0.f, x1 = 0.f;
+    if (wi < nwords) {
+        uint8_t *st = reinterpret_cast<uint8_t *>(REVERSE ? p.dCb + hbase * DD : p.Cst + (size_t)bh * (NC + 1) * DD);
+        const size_t slot_bytes = DD * 4;
+        auto put = [&](int slot) {
+            uint32_t *w = reinterpret_cast<uint32_t *>(st + (size_t)slot * slot_bytes) + wi;
+            const uint32_t hi = tc::cvt_bf16x2(x0, x1);
+            const __nv_bfloat162 h2 = *reinterpret_cast<const __nv_bfloat162 *>(&hi);
+            w[0] = hi;
+            w[DD / 2] = tc::cvt_bf16x2(x0 - __low2float(h2), x1 - __high2float(h2));
+        };
+        auto get = [&](int slot, float &d0, float &d1) {
+            const uint32_t *w = reinterpret_cast<const uint32_t *>(st + (size_t)slot * slot_bytes) + wi;
+            const uint32_t hw = w[0], lw = w[DD / 2];
+            const __nv_bfloat162 h2 = *reinterpret_cast<const __nv_bfloat162 *>(&hw);
+            const __nv_bfloat162 l2 = *reinterpret_cast<const __nv_bfloat162 *>(&lw);
+            d0 = __low2float(h2) + __low2float(l2);
+            d1 = __high2float(h2) + __high2float(l2);
+        };
+        if (REVERSE) {
+            if (p.dC) {                                  // (r, j), (r, j + 1) of this word
+                const uint32_t o = (uint32_t)wi * 4u, blk = o >> 14, rem = o & 16383u;
+                const uint32_t rr = rem >> 7, pc = (rem & 127u) >> 4, e = (rem & 15u) >> 1;
+                const int j = (int)((blk % (D / 64)) * 64 + ((pc ^ (rr & 7u)) << 3) + e);
+                const int r = (int)((blk / (D / 64)) * 128 + rr);
+                x0 = p.dC[(size_t)bh * DD + (size_t)r * D + j];
+                x1 = p.dC[(size_t)bh * DD + (size_t)r * D + j + 1];
+            }
+            put(NC - 1);
+            for (int c = NC - 1; c >= 1; --c) {
+                const float decay = expf(p.Bsum[hbase + c] + p.mprev[hbase + c] - p.mend[hbase + c]);
+                float d0, d1;
+                get(c - 1, d0, d1);
+                x0 = x0 * decay + d0;
+                x1 = x1 * decay + d1;
+                put(c - 1);
+            }
+        } else {
+            put(0);
+            for (int c = 0; c < NC; ++c) {
+                const float decay = expf(p.Bsum[hbase + c] + p.mprev[hbase + c] - p.mend[hbase + c]);
+                float d0, d1;
+                get(c + 1, d0, d1);
+                x0 = x0 * decay + d0;
+                x1 = x1 * decay + d1;
+                put(c + 1);
+            }
+        }
+    } else {
+        const int j = 2 * (int)(wi - nwords);
+        float *nv = REVERSE ? p.dnb + hbase * D : p.nst + (size_t)bh * (NC + 1) * D;
+        if (REVERSE) {
+            if (p.dn) {
+                x0 = p.dn[(size_t)bh * D + j];
+                x1 = p.dn[(size_t)bh * D + j + 1];
+            }
+            nv[(size_t)(NC - 1) * D + j] = x0;
+            nv[(size_t)(NC - 1) * D + j + 1] = x1;
+            for (int c = NC - 1; c >= 1; --c) {
+                const float decay = expf(p.Bsum[hbase + c] + p.mprev[hbase + c] - p.mend[hbase + c]);
+                float *d = nv + (size_t)(c - 1) * D + j;
+                x0 = x0 * decay + d[0];
+                x1 = x1 * decay + d[1];
+                d[0] = x0;
+                d[1] = x1;
+            }
+        } else {
+            nv[j] = 0.f;
+            nv[j + 1] = 0.f;
+            for (int c = 0; c < NC; ++c) {
+                const float decay = expf(p.Bsum[hbase + c] + p.mprev[hbase + c] - p.mend[hbase + c]);
+                float *d = nv + (size_t)(c + 1) * D + j;
+                x0 = x0 * decay + d[0];
+                x1 = x1 * decay + d[1];
+                d[0] = x0;
+                d[1] = x1;
+            }
+        }
     }
 }
 
