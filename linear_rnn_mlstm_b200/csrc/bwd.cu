@@ -1234,6 +1234,20 @@ cudaError_t launch_state_recurrence(const BwdPtrs &p, bool reverse, cudaStream_t
     return reverse ? launch_state_recurrence_t<256, true>(p, st) : launch_state_recurrence_t<256, false>(p, st);
 }
 
+template <int D>
+cudaError_t launch_token_fwd_tc_t(const BwdPtrs &p, cudaStream_t st) {
+    CUtensorMap mq, mk, mv;
+    if (!make_map_bf16(&mq, p.q, p.BH, p.S, D, true, 64) || !make_map_bf16(&mk, p.k, p.BH, p.S, D, true, 64) ||
+        !make_map_bf16(&mv, p.v, p.BH, p.S, D, true, 64))
+        return cudaErrorInvalidValue;
+    const int sm = bwdtc::TokLay<D>::kBytes;
+    cudaError_t e = cudaFuncSetAttribute(bwdtc::token_fwd_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
+    if (e != cudaSuccess) return e;
+    bwdtc::token_fwd_tc_kernel<D><<<(unsigned)((long long)p.NC * p.BH), bwdtc::kTokThreads, sm, st>>>(
+        mq, mk, mv, p, device_status_ptr());
+    return cudaGetLastError();
+}
+
 cudaError_t launch_state_products(const BwdPtrs &p, int which, cudaStream_t st) {
     KernelTimer timer("bwd_state_mma", st);
     return p.DH == 128 ? launch_state_mma<128>(p, which, st) : launch_state_mma<256>(p, which, st);
@@ -1255,7 +1269,11 @@ cudaError_t launch_bwd(const BwdPtrs &p, cudaStream_t st) {
         KernelTimer timer("bwd_states", st);
         if (!launch_rows<T, false>(p, st)) bwd_states_kernel<T><<<blocks_for(rows), kThreads, 0, st>>>(p);
     }
-    {
+    if (p.tc) {
+        KernelTimer timer("bwd_token_fwd_tc", st);
+        e = p.DH == 128 ? launch_token_fwd_tc_t<128>(p, st) : launch_token_fwd_tc_t<256>(p, st);
+        if (e != cudaSuccess) return e;
+    } else {
         KernelTimer timer("bwd_token_fwd", st);
         if (!launch_token_fwd_chunk<T>(p, st) && !launch_token_warp<T, false>(p, st))
             bwd_token_fwd_kernel<T><<<blocks_for(tokens), kThreads, 0, st>>>(p);

@@ -456,5 +456,262 @@ __global__ void __launch_bounds__(256) state_scan_kernel(bwd::BwdPtrs p) {
     }
 }
 
+// ------------------------------------------------------------ per-token pass
+// K3 on the tensor cores, one CTA per (chunk, head): the forward quantities of
+// every token of the chunk and the first gradients.
+//   S   = Q K^T                       M = 64 tokens t, N = 64 keys s, K = DH
+//   W_ts = e^{b_t - b_s + itilde_s - m_t} S_ts / sqrt(d)  (s <= t), rowsum_t = sum_s W_ts
+//   num_intra^T = V^T W^T              M = 128 value rows per tile, N = 64 tokens, K = 64
+// (W as bf16 high + low parts), then per (value row i, token t), with
+// C'_c q_t from the state product kernel (p.num):
+//   num' = g_t C'q + num_intra,  nq' = g_t n'_c.q_t + rowsum_t,  den' = max(|nq'|, e^{-m_t}),
+//   h~ = num'/den', dh~ = dh o, d o~ = dh h~ o (1 - o), dnum' = dh~ / den',
+//   dnq' = -(dh~ . h~)/den' sign(nq') where |nq'| > e^{-m_t}, A = dnum'.num' + dnq' nq'.
+// 16 warps: in the epilogue warp w owns TMEM lane quadrant w % 4 (32 value
+// rows of each 128-row tile, coalesced per token) and tokens 16 (w / 4) to
+// 16 (w / 4) + 15; the per-token sums over the value rows go through warp
+// shuffles and shared memory.
+constexpr int kTokThreads = 512;
+
+template <int D>
+struct TokLay {
+    static constexpr int kTile = D / 64 * 8192;          // 64 token rows x D, bf16, 128-byte swizzle
+    static constexpr int kQ = 0, kK = kTile, kV = 2 * kTile;
+    static constexpr int kWhi = 3 * kTile, kWlo = kWhi + 8192;
+    static constexpr int kF = kWlo + 8192;                // floats: b ip mt g den nq nqi rs [64 each], red [2][4][64], n' [D]
+    static constexpr int kFloats = 8 * 64 + 2 * 8 * 64 + D;
+    static constexpr int kBar = kF + kFloats * 4;
+    static constexpr int kBytes = kBar + 64 + 1024;
+    static constexpr int kCols = D == 256 ? 256 : 128;    // TMEM: S in 0-63, num_intra^T tiles from 64
+};
+
+template <int D>
+__global__ void __launch_bounds__(kTokThreads, 1)
+token_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
+                    const __grid_constant__ CUtensorMap map_v, bwd::BwdPtrs p, unsigned int *status) {
+    using Lay = TokLay<D>;
+    using namespace tc;
+    extern __shared__ uint8_t tok_smem_raw[];
+    uint8_t *smem = align1k(tok_smem_raw);
+    float *fb = reinterpret_cast<float *>(smem + Lay::kF);
+    float *sb = fb, *sip = fb + 64, *smt = fb + 128, *sg = fb + 192, *sden = fb + 256, *snq = fb + 320,
+          *srs = fb + 448, *red = fb + 512, *snp = fb + 512 + 1024;
+    uint64_t *bar = reinterpret_cast<uint64_t *>(smem + Lay::kBar);
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(smem + Lay::kBar + 32);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + Lay::kBar + 36);
+    const int NC = p.NC, S = p.S, L = p.L;
+    const int c = (int)(blockIdx.x % (unsigned)NC), bh = (int)(blockIdx.x / (unsigned)NC);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int a0 = c * L, n = min(S, a0 + L) - a0;
+    const size_t row0 = (size_t)bh * S + a0, hc = (size_t)bh * NC + c;
+    const float inv_sqrt = rsqrtf((float)D);
+
+    if (tid == 0) {
+        for (int i = 0; i < 3; ++i) mbar_init(&bar[i], 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+        mbar_arrive_expect_tx(&bar[0], 3 * Lay::kTile);
+        for (int a = 0; a < D / 64; ++a) {
+            tma_load_3d(smem + Lay::kQ + a * 8192, &map_q, &bar[0], 64 * a, a0, bh);
+            tma_load_3d(smem + Lay::kK + a * 8192, &map_k, &bar[0], 64 * a, a0, bh);
+            tma_load_3d(smem + Lay::kV + a * 8192, &map_v, &bar[0], 64 * a, a0, bh);
+        }
+    }
+    __syncwarp();
+    if (warp == 0) tmem_alloc(tslot, Lay::kCols);
+    if (tid < 64) {
+        const int t = tid;
+        float b = 0.f, ip = -INFINITY, mt = 0.f, g = 0.f;
+        if (t < n) {
+            b = p.b[row0 + t];
+            ip = p.ip[row0 + t];
+            mt = p.mt[row0 + t];
+            g = expf(b + p.mprev[hc] - mt);
+        }
+        sb[t] = b; sip[t] = ip; smt[t] = mt; sg[t] = g;
+    }
+    for (int j = tid; j < D; j += kTokThreads) snp[j] = p.nst[((size_t)bh * (NC + 1) + c) * D + j];
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tacc = *tslot;
+    const int quad = warp & 3;
+    const uint32_t lane_addr = ((uint32_t)(32 * quad)) << 16;
+    int ok = 0;
+    if (lane == 0) ok = mbar_wait(&bar[0], 0, abort_flag, status) ? 1 : 0;
+    __syncwarp();
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    if (ok && tid == 0) {
+        tc_fence_after();
+        const uint32_t idesc = idesc_f32acc(kFmtBF16, kFmtBF16, false, false, 64, 64);
+        const uint32_t sq = smem_u32(smem + Lay::kQ), sk = smem_u32(smem + Lay::kK);
+#pragma unroll 1
+        for (int ks = 0; ks < D / 16; ++ks) {
+            const uint32_t off = (uint32_t)((ks >> 2) * 8192 + (ks & 3) * 32);
+            mma_bf16_ss(tacc, sdesc_sw128(sq + off, 16, 1024), sdesc_sw128(sk + off, 16, 1024), idesc,
+                        ks > 0 ? 1u : 0u);
+        }
+        mma_commit(&bar[1]);
+    }
+    if (ok) {                                         // n'_c . q_t, eight threads per token
+        const int t = tid >> 3, h = tid & 7;
+        float acc = 0.f;
+        for (int pc = h * (D / 64); pc < (h + 1) * (D / 64); ++pc) {      // 16-byte pieces of the row
+            const int j0 = pc * 8;
+            const uint4 raw = *reinterpret_cast<const uint4 *>(
+                smem + Lay::kQ + (j0 >> 6) * 8192 + t * 128 + ((((j0 & 63) >> 3) ^ (t & 7)) << 4));
+            const __nv_bfloat16 *qb = reinterpret_cast<const __nv_bfloat16 *>(&raw);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc += snp[j0 + e] * __bfloat162float(qb[e]);
+        }
+        acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+        acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+        acc += __shfl_xor_sync(0xffffffffu, acc, 4);
+        if (h == 0) red[t] = acc;
+    }
+    // ---- scores -> W (bf16 high / low tiles), row sums
+    int done1 = 0;
+    if (ok && lane == 0) done1 = mbar_wait(&bar[1], 0, abort_flag, status) ? 1 : 0;
+    __syncwarp();
+    done1 = __shfl_sync(0xffffffffu, done1, 0);
+    if (done1 && warp < 4) {
+        tc_fence_after();
+        uint32_t sa[64];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) tmem_ld16(tacc + lane_addr + 16 * q, *reinterpret_cast<uint32_t(*)[16]>(&sa[16 * q]));
+        tmem_wait_ld();
+        // M = 64 layout: row t = 16 warp + (lane & 15) in TMEM lanes 0-15 of the
+        // warp's quadrant; lanes 16-31 take that row's columns 32-63
+        const int t = 16 * warp + (lane & 15), hh = lane >> 4;
+        float sv[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+            const uint32_t up = __shfl_sync(0xffffffffu, sa[32 + e], lane & 15);
+            sv[e] = __uint_as_float(hh ? up : sa[e]);
+        }
+        float rs = 0.f;
+        const float bt = sb[t], mtt = smt[t];
+        uint32_t hi[16], lo[16];
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+            float w2[2];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int s_ = 32 * hh + e + u;
+                w2[u] = (t < n && s_ <= t) ? expf(bt - sb[s_] + sip[s_] - mtt) * sv[e + u] * inv_sqrt : 0.f;
+                rs += w2[u];
+            }
+            hi[e / 2] = cvt_bf16x2(w2[0], w2[1]);
+            const __nv_bfloat162 h2 = *reinterpret_cast<const __nv_bfloat162 *>(&hi[e / 2]);
+            lo[e / 2] = cvt_bf16x2(w2[0] - __low2float(h2), w2[1] - __high2float(h2));
+        }
+        rs += __shfl_xor_sync(0xffffffffu, rs, 16);
+        if (hh == 0) srs[t] = rs;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {                 // pieces 4 hh + q of row t
+            const uint32_t off = (uint32_t)t * 128u + ((uint32_t)((4 * hh + q) ^ (t & 7)) << 4);
+            *reinterpret_cast<uint4 *>(smem + Lay::kWhi + off) = make_uint4(hi[4 * q], hi[4 * q + 1], hi[4 * q + 2], hi[4 * q + 3]);
+            *reinterpret_cast<uint4 *>(smem + Lay::kWlo + off) = make_uint4(lo[4 * q], lo[4 * q + 1], lo[4 * q + 2], lo[4 * q + 3]);
+        }
+        fence_async_smem();
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (done1 && tid == 0) {
+        tc_fence_after();
+        const uint32_t idesc = idesc_f32acc(kFmtBF16, kFmtBF16, true, false, 128, 64);
+        const uint32_t svv = smem_u32(smem + Lay::kV), wh = smem_u32(smem + Lay::kWhi), wl = smem_u32(smem + Lay::kWlo);
+#pragma unroll
+        for (int mt = 0; mt < D / 128; ++mt)
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks) {
+                const uint64_t ad = sdesc_sw128(svv + 2 * mt * 8192 + ks * 2048, 8192, 1024);
+                mma_bf16_ss(tacc + 64 + 64 * mt, ad, sdesc_sw128(wh + ks * 32, 16, 1024), idesc, ks > 0 ? 1u : 0u);
+                mma_bf16_ss(tacc + 64 + 64 * mt, ad, sdesc_sw128(wl + ks * 32, 16, 1024), idesc, 1u);
+            }
+        mma_commit(&bar[2]);
+    }
+    if (done1 && tid < 64) {                          // normaliser and floor per token
+        const int t = tid;
+        const float nq = sg[t] * red[t] + srs[t];
+        snq[t] = nq;
+        sden[t] = t < n ? fmaxf(fabsf(nq), expf(-smt[t])) : 1.f;
+    }
+    __syncthreads();
+    int done2 = 0;
+    if (done1 && lane == 0) done2 = mbar_wait(&bar[2], 0, abort_flag, status) ? 1 : 0;
+    __syncwarp();
+    done2 = __shfl_sync(0xffffffffu, done2, 0);
+    if (done2) {
+        tc_fence_after();
+        __nv_bfloat16 *hl = reinterpret_cast<__nv_bfloat16 *>(p.dnhl);
+        const size_t plane = (size_t)p.BH * S * D;
+        {
+            const int tg = warp >> 2;
+            uint32_t v[D / 128][16];
+#pragma unroll
+            for (int mt = 0; mt < D / 128; ++mt) tmem_ld16(tacc + lane_addr + 64 + 64 * mt + 16 * tg, v[mt]);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+                const int t = 16 * tg + e;
+                if (t >= n) continue;
+                const float g = sg[t], den = sden[t];
+                const size_t rowoff = (row0 + t) * D;
+                float sdot = 0.f, A = 0.f;
+#pragma unroll
+                for (int mt = 0; mt < D / 128; ++mt) {
+                    const int i = 128 * mt + 32 * quad + lane;
+                    const float num = g * p.num[rowoff + i] + __uint_as_float(v[mt][e]);
+                    const float ht = num / den;
+                    const float o = bwd::sigmoid_hd(p.op[rowoff + i]);
+                    const float dhr = __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(p.dh)[rowoff + i]);
+                    const float dht = dhr * o;
+                    p.dO[rowoff + i] = dhr * ht * o * (1.f - o);
+                    const float dn = dht / den;
+                    p.dnum[rowoff + i] = dn;
+                    const __nv_bfloat16 h16 = __float2bfloat16_rn(dn);
+                    hl[rowoff + i] = h16;
+                    hl[plane + rowoff + i] = __float2bfloat16_rn(dn - __bfloat162float(h16));
+                    sdot += dht * ht;
+                    A += dn * num;
+                }
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) {
+                    sdot += __shfl_xor_sync(0xffffffffu, sdot, o);
+                    A += __shfl_xor_sync(0xffffffffu, A, o);
+                }
+                if (lane == 0) {
+                    red[quad * 64 + t] = sdot;
+                    red[256 + quad * 64 + t] = A;
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (done2 && tid < n) {
+        const int t = tid;
+        float sdot = 0.f, A = 0.f;
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+            sdot += red[w * 64 + t];
+            A += red[256 + w * 64 + t];
+        }
+        const float nq = snq[t], den = sden[t];
+        const float dnq = fabsf(nq) > expf(-smt[t]) ? -sdot / den * (nq > 0.f ? 1.f : -1.f) : 0.f;
+        p.dnq[row0 + t] = dnq;
+        p.nq[row0 + t] = nq;
+        p.den[row0 + t] = den;
+        p.A[row0 + t] = A + dnq * nq;
+    }
+    if (tid == 0 && !ok) mbar_wait(&bar[0], 0, nullptr, nullptr);     // no copy left in flight
+    __syncwarp();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tacc, Lay::kCols);
+    }
+}
+
 }  // namespace bwdtc
 }  // namespace xlstm
