@@ -482,429 +482,6 @@ __global__ void __launch_bounds__(32 * kTokWarps) bwd_token_grad_warp_kernel(Bwd
     }
 }
 
-// K5 for bf16 inputs with DH 128 or 256: one CTA per (chunk,
-// head), 16 warps, 4 tokens per warp.  The chunk's q, k, v tiles and dnum' sit
-// in shared memory; the intra-chunk weights are formed once per chunk as two
-// lower-triangular 64 x 64 matrices (M1_ts = W_ts (dnum'_t . v_s + dnq'_t),
-// M2_ts = W_ts (q_t . khat_s)), and the chunk's states C'_c and dC~_c are read
-// once per CTA, row by row, instead of once per token: the products with the
-// DH x DH states are where the per-token kernel spent its time (768 KB of L2
-// reads per token).
-constexpr int kChWarps = 16;
-constexpr int kChTok = bwd::kMaxChunk / kChWarps;       // tokens per warp
-
-template <int NCL>
-size_t chunk_grad_smem_bytes() {
-    constexpr int DH = 32 * NCL, L = bwd::kMaxChunk;
-    return (size_t)3 * L * DH * 2 + (size_t)L * DH * 4 + (size_t)2 * L * L * 4 + (size_t)8 * L * 4;
-}
-
-// TC: the products with the chunk's states come from the tensor-core kernels
-// (dq: p.num, dk: p.dki, dv: p.dvi, unscaled) instead of the state rows.
-template <int NCL, bool TC>
-__global__ void __launch_bounds__(32 * kChWarps, 1) bwd_token_grad_chunk_kernel(BwdPtrs p) {
-    constexpr int DH = 32 * NCL, LM = bwd::kMaxChunk;
-    using T = __nv_bfloat16;
-    extern __shared__ __align__(16) uint8_t ch_smem[];
-    T *sq = reinterpret_cast<T *>(ch_smem);                      // [LM][DH]
-    T *sk = sq + LM * DH;
-    T *sv = sk + LM * DH;
-    float *sdn = reinterpret_cast<float *>(sv + LM * DH);        // dnum' [LM][DH]
-    float *M1 = sdn + LM * DH;                                   // [t][s], s <= t
-    float *M2 = M1 + LM * LM;
-    float *sb = M2 + LM * LM, *sip = sb + LM, *smt = sip + LM, *sdnq = smt + LM, *sA = sdnq + LM;
-    const int c = blockIdx.x, bh = blockIdx.y;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int S = p.S, L = p.L, NC = p.NC;
-    const int a = c * L, n = bwd::imin(S, a + L) - a;
-    const size_t DD = (size_t)DH * DH;
-    const float inv_sqrt = 1.f / sqrtf((float)DH);
-    const size_t row0 = (size_t)bh * S + a;
-    const size_t hc = (size_t)bh * NC + c;
-    // ---- tiles and per-token scalars
-    for (int e = threadIdx.x; e < n * DH / 8; e += 32 * kChWarps) {
-        const size_t g = row0 * DH + (size_t)e * 8;
-        reinterpret_cast<uint4 *>(sq)[e] = *reinterpret_cast<const uint4 *>((const T *)p.q + g);
-        reinterpret_cast<uint4 *>(sk)[e] = *reinterpret_cast<const uint4 *>((const T *)p.k + g);
-        reinterpret_cast<uint4 *>(sv)[e] = *reinterpret_cast<const uint4 *>((const T *)p.v + g);
-    }
-    for (int e = threadIdx.x; e < n * DH / 4; e += 32 * kChWarps)
-        reinterpret_cast<float4 *>(sdn)[e] = reinterpret_cast<const float4 *>(p.dnum + row0 * DH)[e];
-    for (int s = threadIdx.x; s < n; s += 32 * kChWarps) {
-        sb[s] = p.b[row0 + s];
-        sip[s] = p.ip[row0 + s];
-        smt[s] = p.mt[row0 + s];
-        sdnq[s] = p.dnq[row0 + s];
-        sA[s] = p.A[row0 + s];
-    }
-    __syncthreads();
-    // ---- intra weights: pairs (t, s), s <= t, one warp per pair
-    for (int pr = warp; pr < n * n; pr += kChWarps) {
-        const int t = pr / n, s = pr % n;
-        if (s > t) continue;
-        float d1 = 0.f, d2 = 0.f;
-#pragma unroll
-        for (int i = 0; i < NCL; ++i) {
-            const int j = lane + 32 * i;
-            d1 += sdn[t * DH + j] * __bfloat162float(sv[s * DH + j]);
-            d2 += __bfloat162float(sq[t * DH + j]) * __bfloat162float(sk[s * DH + j]);
-        }
-        d1 = wsum(d1);
-        d2 = wsum(d2);
-        if (lane == 0) {
-            const float w = expf(sb[t] - sb[s] + sip[s] - smt[t]);
-            M1[t * LM + s] = w * (d1 + sdnq[t]);
-            M2[t * LM + s] = w * d2 * inv_sqrt;
-        }
-    }
-    __syncthreads();
-    // ---- per token: intra parts, then the products with the chunk's states
-    const float mprev = p.mprev[hc], Bs = p.Bsum[hc], mend = p.mend[hc];
-    const float *Cc = p.Cst + ((size_t)bh * (NC + 1) + c) * DD;
-    const float *ncs = p.nst + ((size_t)bh * (NC + 1) + c) * DH;
-    const float *dCc = p.dCb + hc * DD;
-    const float *dnc = p.dnb + hc * DH;
-    float acc[kChTok][NCL], inter[kChTok][NCL];
-    // phase 1, dq_s = (1/sqrt d) sum_{u<=s} M1_su k_u + g_s (C'^T dnum'_s + dnq'_s n')
-#pragma unroll
-    for (int x = 0; x < kChTok; ++x) {
-        const int s = warp * kChTok + x;
-#pragma unroll
-        for (int i = 0; i < NCL; ++i) acc[x][i] = inter[x][i] = 0.f;
-        if (s >= n) continue;
-        for (int u = 0; u <= s; ++u) {
-            const float w = M1[s * LM + u];
-#pragma unroll
-            for (int i = 0; i < NCL; ++i) acc[x][i] += w * __bfloat162float(sk[u * DH + lane + 32 * i]);
-        }
-    }
-    if constexpr (TC) {
-#pragma unroll
-        for (int x = 0; x < kChTok; ++x) {
-            const int s = warp * kChTok + x;
-            if (s >= n) continue;
-#pragma unroll
-            for (int i = 0; i < NCL; ++i) inter[x][i] = p.num[(row0 + s) * DH + lane + 32 * i];
-        }
-    } else {
-        for (int r = 0; r < DH; ++r) {              // C' rows, once per CTA
-            float cr[NCL];
-#pragma unroll
-            for (int i = 0; i < NCL; ++i) cr[i] = Cc[(size_t)r * DH + lane + 32 * i];
-#pragma unroll
-            for (int x = 0; x < kChTok; ++x) {
-                const float dn_r = sdn[(warp * kChTok + x) * DH + r];
-#pragma unroll
-                for (int i = 0; i < NCL; ++i) inter[x][i] += cr[i] * dn_r;
-            }
-        }
-    }
-#pragma unroll
-    for (int x = 0; x < kChTok; ++x) {
-        const int s = warp * kChTok + x;
-        if (s >= n) continue;
-        const float g = expf(sb[s] + mprev - smt[s]);
-#pragma unroll
-        for (int i = 0; i < NCL; ++i) {
-            const int j = lane + 32 * i;
-            bwd::st((T *)p.dq, (row0 + s) * DH + j, acc[x][i] * inv_sqrt + g * (inter[x][i] + sdnq[s] * ncs[j]));
-        }
-    }
-    // phase 2, dk_s = (1/sqrt d)(sum_{t>=s} M1_ts q_t + wk_s (dC~^T v_s + dn~)); di_s = khat_s . dkhat_s
-#pragma unroll
-    for (int x = 0; x < kChTok; ++x) {
-        const int s = warp * kChTok + x;
-#pragma unroll
-        for (int i = 0; i < NCL; ++i) acc[x][i] = inter[x][i] = 0.f;
-        if (s >= n) continue;
-        for (int t = s; t < n; ++t) {
-            const float w = M1[t * LM + s];
-#pragma unroll
-            for (int i = 0; i < NCL; ++i) acc[x][i] += w * __bfloat162float(sq[t * DH + lane + 32 * i]);
-        }
-    }
-    if constexpr (TC) {
-#pragma unroll
-        for (int x = 0; x < kChTok; ++x) {
-            const int s = warp * kChTok + x;
-            if (s >= n) continue;
-#pragma unroll
-            for (int i = 0; i < NCL; ++i) inter[x][i] = p.dki[(row0 + s) * DH + lane + 32 * i];
-        }
-    } else {
-        for (int r = 0; r < DH; ++r) {              // dC~ rows, once per CTA
-            float dr[NCL];
-#pragma unroll
-            for (int i = 0; i < NCL; ++i) dr[i] = dCc[(size_t)r * DH + lane + 32 * i];
-#pragma unroll
-            for (int x = 0; x < kChTok; ++x) {
-                const float v_r = __bfloat162float(sv[(warp * kChTok + x) * DH + r]);
-#pragma unroll
-                for (int i = 0; i < NCL; ++i) inter[x][i] += dr[i] * v_r;
-            }
-        }
-    }
-    float di_tok[kChTok], wk_tok[kChTok];
-#pragma unroll
-    for (int x = 0; x < kChTok; ++x) {
-        const int s = warp * kChTok + x;
-        di_tok[x] = 0.f;
-        wk_tok[x] = s < n ? expf(Bs - sb[s] + sip[s] - mend) : 0.f;
-        if (s >= n) continue;
-        float di = 0.f;
-#pragma unroll
-        for (int i = 0; i < NCL; ++i) {
-            const int j = lane + 32 * i;
-            const float dkh = acc[x][i] + wk_tok[x] * (inter[x][i] + dnc[j]);
-            di += dkh * __bfloat162float(sk[s * DH + j]) * inv_sqrt;
-            bwd::st((T *)p.dk, (row0 + s) * DH + j, dkh * inv_sqrt);
-        }
-        di_tok[x] = wsum(di);
-    }
-    // phase 3, dv_s = sum_{t>=s} M2_ts dnum'_t + wk_s / sqrt d dC~ k_s: lanes own rows r
-#pragma unroll
-    for (int x = 0; x < kChTok; ++x) {
-        const int s = warp * kChTok + x;
-#pragma unroll
-        for (int i = 0; i < NCL; ++i) acc[x][i] = 0.f;
-        if (s >= n) continue;
-        for (int t = s; t < n; ++t) {
-            const float w = M2[t * LM + s];
-#pragma unroll
-            for (int i = 0; i < NCL; ++i) acc[x][i] += w * sdn[t * DH + lane + 32 * i];
-        }
-    }
-    if constexpr (TC) {
-#pragma unroll
-        for (int x = 0; x < kChTok; ++x) {
-            const int s = warp * kChTok + x;
-            if (s >= n) continue;
-#pragma unroll
-            for (int i = 0; i < NCL; ++i)
-                acc[x][i] += wk_tok[x] * inv_sqrt * p.dvi[(row0 + s) * DH + lane + 32 * i];
-        }
-    } else {
-#pragma unroll
-        for (int rb = 0; rb < NCL; ++rb) {
-            for (int rl = 0; rl < 32; ++rl) {
-                const int r = 32 * rb + rl;
-                float dr[NCL];
-#pragma unroll
-                for (int i = 0; i < NCL; ++i) dr[i] = dCc[(size_t)r * DH + lane + 32 * i];
-#pragma unroll
-                for (int x = 0; x < kChTok; ++x) {
-                    float part = 0.f;
-#pragma unroll
-                    for (int i = 0; i < NCL; ++i)
-                        part += dr[i] * __bfloat162float(sk[(warp * kChTok + x) * DH + lane + 32 * i]);
-                    part = wsum(part);
-                    if (rl == lane) acc[x][rb] += wk_tok[x] * inv_sqrt * part;
-                }
-            }
-        }
-    }
-#pragma unroll
-    for (int x = 0; x < kChTok; ++x) {
-        const int s = warp * kChTok + x;
-        if (s >= n) continue;
-        const size_t ss = row0 + s;
-#pragma unroll
-        for (int i = 0; i < NCL; ++i) bwd::st((T *)p.dv, ss * DH + lane + 32 * i, acc[x][i]);
-        if (lane == 0) {
-            p.di[ss] = di_tok[x];
-            p.dF[ss] = sA[s] - di_tok[x];
-        }
-    }
-}
-
-// K3 for bf16 inputs with DH 128 or 256: one CTA per (chunk,
-// head), 16 warps, 4 tokens per warp; the chunk's q, k, v in shared memory,
-// the intra weights W_ts (q_t . khat_s) formed once per chunk, and C'_c read
-// once per CTA, row by row.
-template <int NCL>
-size_t chunk_fwd_smem_bytes() {
-    constexpr int DH = 32 * NCL, L = bwd::kMaxChunk;
-    return (size_t)3 * L * DH * 2 + (size_t)L * L * 4 + (size_t)4 * L * 4;
-}
-
-// TC: C' q_t comes from the tensor-core kernel (p.num, unscaled) instead of the
-// state rows, and dnum' is also written as bf16 high and low planes (p.dnhl).
-template <int NCL, bool TC>
-__global__ void __launch_bounds__(32 * kChWarps, 1) bwd_token_fwd_chunk_kernel(BwdPtrs p) {
-    constexpr int DH = 32 * NCL, LM = bwd::kMaxChunk;
-    using T = __nv_bfloat16;
-    extern __shared__ __align__(16) uint8_t ch_smem[];
-    T *sq = reinterpret_cast<T *>(ch_smem);
-    T *sk = sq + LM * DH;
-    T *sv = sk + LM * DH;
-    float *W2 = reinterpret_cast<float *>(sv + LM * DH);         // [t][s], s <= t
-    float *sb = W2 + LM * LM, *sip = sb + LM, *smt = sip + LM;
-    const int c = blockIdx.x, bh = blockIdx.y;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int S = p.S, L = p.L, NC = p.NC;
-    const int a = c * L, n = bwd::imin(S, a + L) - a;
-    const size_t DD = (size_t)DH * DH;
-    const float inv_sqrt = 1.f / sqrtf((float)DH);
-    const size_t row0 = (size_t)bh * S + a;
-    const size_t hc = (size_t)bh * NC + c;
-    for (int e = threadIdx.x; e < n * DH / 8; e += 32 * kChWarps) {
-        const size_t g = row0 * DH + (size_t)e * 8;
-        reinterpret_cast<uint4 *>(sq)[e] = *reinterpret_cast<const uint4 *>((const T *)p.q + g);
-        reinterpret_cast<uint4 *>(sk)[e] = *reinterpret_cast<const uint4 *>((const T *)p.k + g);
-        reinterpret_cast<uint4 *>(sv)[e] = *reinterpret_cast<const uint4 *>((const T *)p.v + g);
-    }
-    for (int s = threadIdx.x; s < n; s += 32 * kChWarps) {
-        sb[s] = p.b[row0 + s];
-        sip[s] = p.ip[row0 + s];
-        smt[s] = p.mt[row0 + s];
-    }
-    __syncthreads();
-    for (int pr = warp; pr < n * n; pr += kChWarps) {
-        const int t = pr / n, s = pr % n;
-        if (s > t) continue;
-        float d = 0.f;
-#pragma unroll
-        for (int i = 0; i < NCL; ++i)
-            d += __bfloat162float(sq[t * DH + lane + 32 * i]) * __bfloat162float(sk[s * DH + lane + 32 * i]);
-        d = wsum(d);
-        if (lane == 0) W2[t * LM + s] = expf(sb[t] - sb[s] + sip[s] - smt[t]) * d * inv_sqrt;
-    }
-    __syncthreads();
-    const float mprev = p.mprev[hc];
-    const float *Cc = p.Cst + ((size_t)bh * (NC + 1) + c) * DD;
-    const float *nc = p.nst + ((size_t)bh * (NC + 1) + c) * DH;
-    // num'_t[r] = g_t (C' q_t)[r] + sum_{s<=t} W_ts v_s[r]: lanes own rows r
-    float num[kChTok][NCL];
-#pragma unroll
-    for (int x = 0; x < kChTok; ++x)
-#pragma unroll
-        for (int i = 0; i < NCL; ++i) num[x][i] = 0.f;
-    if constexpr (TC) {
-#pragma unroll
-        for (int x = 0; x < kChTok; ++x) {
-            const int t = warp * kChTok + x;
-            if (t >= n) continue;
-#pragma unroll
-            for (int i = 0; i < NCL; ++i) num[x][i] = p.num[(row0 + t) * DH + lane + 32 * i];
-        }
-    } else {
-#pragma unroll
-        for (int rb = 0; rb < NCL; ++rb) {
-            for (int rl = 0; rl < 32; ++rl) {
-                const int r = 32 * rb + rl;
-                float cr[NCL];
-#pragma unroll
-                for (int i = 0; i < NCL; ++i) cr[i] = Cc[(size_t)r * DH + lane + 32 * i];
-#pragma unroll
-                for (int x = 0; x < kChTok; ++x) {
-                    float part = 0.f;
-#pragma unroll
-                    for (int i = 0; i < NCL; ++i)
-                        part += cr[i] * __bfloat162float(sq[(warp * kChTok + x) * DH + lane + 32 * i]);
-                    part = wsum(part);
-                    if (rl == lane) num[x][rb] = part;
-                }
-            }
-        }
-    }
-#pragma unroll
-    for (int x = 0; x < kChTok; ++x) {
-        const int t = warp * kChTok + x;
-        if (t >= n) continue;
-        const size_t ts = row0 + t;
-        const float g = expf(sb[t] + mprev - smt[t]);
-        float nq = 0.f, ni = 0.f;
-        for (int s = 0; s <= t; ++s) nq += W2[t * LM + s];
-#pragma unroll
-        for (int i = 0; i < NCL; ++i) ni += nc[lane + 32 * i] * __bfloat162float(sq[t * DH + lane + 32 * i]);
-        nq += g * wsum(ni);
-#pragma unroll
-        for (int i = 0; i < NCL; ++i) {
-            const int r = lane + 32 * i;
-            float acc = num[x][i] * g;
-            for (int s = 0; s <= t; ++s) acc += W2[t * LM + s] * __bfloat162float(sv[s * DH + r]);
-            num[x][i] = acc;
-            p.num[ts * DH + r] = acc;
-        }
-        const float floor_ = expf(-smt[t]);
-        const float den = fmaxf(fabsf(nq), floor_);
-        float sdot = 0.f, A = 0.f;
-#pragma unroll
-        for (int i = 0; i < NCL; ++i) {
-            const int r = lane + 32 * i;
-            const float o = bwd::sigmoid_hd(p.op[ts * DH + r]);
-            const float hv = num[x][i] / den;
-            const float dhr = bwd::ld((const T *)p.dh, ts * DH + r);
-            const float dht = dhr * o;
-            p.dO[ts * DH + r] = dhr * hv * o * (1.f - o);
-            const float dn_r = dht / den;
-            p.dnum[ts * DH + r] = dn_r;
-            if constexpr (TC) {
-                __nv_bfloat16 *hl = reinterpret_cast<__nv_bfloat16 *>(p.dnhl);
-                const __nv_bfloat16 hi = __float2bfloat16_rn(dn_r);
-                hl[ts * DH + r] = hi;
-                hl[(size_t)p.BH * p.S * DH + ts * DH + r] = __float2bfloat16_rn(dn_r - __bfloat162float(hi));
-            }
-            sdot += dht * hv;
-            A += dn_r * num[x][i];
-        }
-        sdot = wsum(sdot);
-        A = wsum(A);
-        if (lane == 0) {
-            const float dnq = fabsf(nq) > floor_ ? -sdot / den * (nq > 0.f ? 1.f : -1.f) : 0.f;
-            p.dnq[ts] = dnq;
-            p.nq[ts] = nq;
-            p.den[ts] = den;
-            p.A[ts] = A + dnq * nq;
-        }
-    }
-}
-
-template <typename T>
-bool launch_token_fwd_chunk(const BwdPtrs &p, cudaStream_t st) {
-    // DH 128 / 256 (below that one warp per token measured faster)
-    if (sizeof(T) != 2 || (p.DH != 128 && p.DH != 256)) return false;
-    const dim3 grid((unsigned)p.NC, (unsigned)p.BH);
-#define XLSTM_BWD_CF(N)                                                                           \
-    if (p.DH == 32 * N) {                                                                          \
-        const size_t sm = chunk_fwd_smem_bytes<N>();                                               \
-        if (p.tc) {                                                                                \
-            cudaFuncSetAttribute(bwd_token_fwd_chunk_kernel<N, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm); \
-            bwd_token_fwd_chunk_kernel<N, true><<<grid, 32 * kChWarps, sm, st>>>(p);               \
-        } else {                                                                                   \
-            cudaFuncSetAttribute(bwd_token_fwd_chunk_kernel<N, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm); \
-            bwd_token_fwd_chunk_kernel<N, false><<<grid, 32 * kChWarps, sm, st>>>(p);              \
-        }                                                                                          \
-        return true;                                                                               \
-    }
-    XLSTM_BWD_CF(4)
-    XLSTM_BWD_CF(8)
-#undef XLSTM_BWD_CF
-    return false;
-}
-
-template <typename T>
-bool launch_token_grad_chunk(const BwdPtrs &p, cudaStream_t st) {
-    if (sizeof(T) != 2 || (p.DH != 128 && p.DH != 256)) return false;
-    const dim3 grid((unsigned)p.NC, (unsigned)p.BH);
-#define XLSTM_BWD_CH(N)                                                                           \
-    if (p.DH == 32 * N) {                                                                          \
-        const size_t sm = chunk_grad_smem_bytes<N>();                                              \
-        if (p.tc) {                                                                                \
-            cudaFuncSetAttribute(bwd_token_grad_chunk_kernel<N, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm); \
-            bwd_token_grad_chunk_kernel<N, true><<<grid, 32 * kChWarps, sm, st>>>(p);              \
-        } else {                                                                                   \
-            cudaFuncSetAttribute(bwd_token_grad_chunk_kernel<N, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm); \
-            bwd_token_grad_chunk_kernel<N, false><<<grid, 32 * kChWarps, sm, st>>>(p);             \
-        }                                                                                          \
-        return true;                                                                               \
-    }
-    XLSTM_BWD_CH(4)
-    XLSTM_BWD_CH(8)
-#undef XLSTM_BWD_CH
-    return false;
-}
-
 template <typename T, bool GRAD>
 bool launch_token_warp(const BwdPtrs &p, cudaStream_t st) {
     const int ncl = p.DH / 32;
@@ -1248,6 +825,22 @@ cudaError_t launch_token_fwd_tc_t(const BwdPtrs &p, cudaStream_t st) {
     return cudaGetLastError();
 }
 
+template <int D>
+cudaError_t launch_token_grad_tc_t(const BwdPtrs &p, cudaStream_t st) {
+    CUtensorMap mq, mk, mv, mdh, mdl;
+    const __nv_bfloat16 *dn_hi = reinterpret_cast<const __nv_bfloat16 *>(p.dnhl);
+    if (!make_map_bf16(&mq, p.q, p.BH, p.S, D, true, 64) || !make_map_bf16(&mk, p.k, p.BH, p.S, D, true, 64) ||
+        !make_map_bf16(&mv, p.v, p.BH, p.S, D, true, 64) || !make_map_bf16(&mdh, dn_hi, p.BH, p.S, D, true, 64) ||
+        !make_map_bf16(&mdl, dn_hi + (size_t)p.BH * p.S * D, p.BH, p.S, D, true, 64))
+        return cudaErrorInvalidValue;
+    const int sm = bwdtc::GradLay<D>::kBytes;
+    cudaError_t e = cudaFuncSetAttribute(bwdtc::token_grad_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
+    if (e != cudaSuccess) return e;
+    bwdtc::token_grad_tc_kernel<D><<<(unsigned)((long long)p.NC * p.BH), bwdtc::kTokThreads, sm, st>>>(
+        mq, mk, mv, mdh, mdl, p, device_status_ptr());
+    return cudaGetLastError();
+}
+
 cudaError_t launch_state_products(const BwdPtrs &p, int which, cudaStream_t st) {
     KernelTimer timer("bwd_state_mma", st);
     return p.DH == 128 ? launch_state_mma<128>(p, which, st) : launch_state_mma<256>(p, which, st);
@@ -1275,7 +868,7 @@ cudaError_t launch_bwd(const BwdPtrs &p, cudaStream_t st) {
         if (e != cudaSuccess) return e;
     } else {
         KernelTimer timer("bwd_token_fwd", st);
-        if (!launch_token_fwd_chunk<T>(p, st) && !launch_token_warp<T, false>(p, st))
+        if (!launch_token_warp<T, false>(p, st))
             bwd_token_fwd_kernel<T><<<blocks_for(tokens), kThreads, 0, st>>>(p);
     }
     if (p.tc) {
@@ -1286,9 +879,13 @@ cudaError_t launch_bwd(const BwdPtrs &p, cudaStream_t st) {
         KernelTimer timer("bwd_reverse", st);
         if (!launch_rows<T, true>(p, st)) bwd_reverse_kernel<T><<<blocks_for(rows), kThreads, 0, st>>>(p);
     }
-    {
+    if (p.tc) {
+        KernelTimer timer("bwd_token_grad_tc", st);
+        e = p.DH == 128 ? launch_token_grad_tc_t<128>(p, st) : launch_token_grad_tc_t<256>(p, st);
+        if (e != cudaSuccess) return e;
+    } else {
         KernelTimer timer("bwd_token_grad", st);
-        if (!launch_token_grad_chunk<T>(p, st) && !launch_token_warp<T, true>(p, st))
+        if (!launch_token_warp<T, true>(p, st))
             bwd_token_grad_kernel<T><<<blocks_for(tokens), kThreads, 0, st>>>(p);
     }
     {

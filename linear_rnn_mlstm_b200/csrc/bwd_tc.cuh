@@ -713,5 +713,267 @@ token_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_cons
     }
 }
 
+// ------------------------------------------------------------ gradient pass
+// K5 on the tensor cores, one CTA per (chunk, head), 16 warps:
+//   S = Q K^T, dP0 = dnum' V^T                      M = 64 tokens, N = 64 keys, K = DH
+//   W~_ts = e^{b_t - b_s + itilde_s - m_t} (s <= t), M2 = W~ S / sqrt(d), M1 = W~ (dP0 + dnq'_t)
+//   dq^T = K^T M1^T,  dk^T = Q^T M1,  dv^T = dnum'^T M2    M = 128 rows per tile, N = 64, K = 64
+// (M1, M2 as bf16 high + low tiles, dnum' from its high / low planes); then,
+// with the state products of the tensor-core kernels (p.num: C'^T dnum',
+// p.dki: dC~^T v, p.dvi: dC~ k):
+//   dq_t = dq^T_t / sqrt(d) + g_t (C'^T dnum'_t + dnq'_t n'_c)
+//   dkhat_s = dk^T_s + wk_s (dC~^T v_s + dn~_c),  dk = dkhat / sqrt(d),  ditilde_s = khat_s . dkhat_s
+//   dv_s = dv^T_s + wk_s / sqrt(d) dC~ k_s,   d log f term dF_s = A_s - ditilde_s.
+template <int D>
+struct GradLay {
+    static constexpr int kTile = D / 64 * 8192;
+    static constexpr int kQ = 0, kK = kTile, kV = 2 * kTile, kDh = 3 * kTile, kDl = 4 * kTile;
+    static constexpr int kM1h = 5 * kTile, kM1l = kM1h + 8192, kM2h = kM1l + 8192, kM2l = kM2h + 8192;
+    static constexpr int kF = kM2l + 8192;        // floats: b ip mt dnq A g wk [64 each], red [4][64], n', dn~ [D]
+    static constexpr int kFloats = 7 * 64 + 4 * 64 + 2 * D;
+    static constexpr int kBar = kF + kFloats * 4;
+    static constexpr int kBytes = kBar + 64 + 1024;
+    static constexpr int cS = 0, cP = 64, cDq = 128, cDk = 128 + 64 * (D / 128), cDv = 128 + 128 * (D / 128);
+};
+
+template <int D>
+__global__ void __launch_bounds__(kTokThreads, 1)
+token_grad_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
+                     const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_dh,
+                     const __grid_constant__ CUtensorMap map_dl, bwd::BwdPtrs p, unsigned int *status) {
+    using Lay = GradLay<D>;
+    using namespace tc;
+    extern __shared__ uint8_t grad_smem_raw[];
+    uint8_t *smem = align1k(grad_smem_raw);
+    float *fb = reinterpret_cast<float *>(smem + Lay::kF);
+    float *sb = fb, *sip = fb + 64, *smt = fb + 128, *sdnq = fb + 192, *sA = fb + 256, *sg = fb + 320,
+          *swk = fb + 384, *red = fb + 448, *snp = fb + 704, *sdnb = snp + D;
+    uint64_t *bar = reinterpret_cast<uint64_t *>(smem + Lay::kBar);
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(smem + Lay::kBar + 32);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + Lay::kBar + 36);
+    const int NC = p.NC, S = p.S, L = p.L;
+    const int c = (int)(blockIdx.x % (unsigned)NC), bh = (int)(blockIdx.x / (unsigned)NC);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, quad = warp & 3;
+    const int a0 = c * L, n = min(S, a0 + L) - a0;
+    const size_t row0 = (size_t)bh * S + a0, hc = (size_t)bh * NC + c;
+    const float inv_sqrt = rsqrtf((float)D);
+
+    if (tid == 0) {
+        for (int i = 0; i < 3; ++i) mbar_init(&bar[i], 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+        mbar_arrive_expect_tx(&bar[0], 5 * Lay::kTile);
+        for (int a = 0; a < D / 64; ++a) {
+            tma_load_3d(smem + Lay::kQ + a * 8192, &map_q, &bar[0], 64 * a, a0, bh);
+            tma_load_3d(smem + Lay::kK + a * 8192, &map_k, &bar[0], 64 * a, a0, bh);
+            tma_load_3d(smem + Lay::kV + a * 8192, &map_v, &bar[0], 64 * a, a0, bh);
+            tma_load_3d(smem + Lay::kDh + a * 8192, &map_dh, &bar[0], 64 * a, a0, bh);
+            tma_load_3d(smem + Lay::kDl + a * 8192, &map_dl, &bar[0], 64 * a, a0, bh);
+        }
+    }
+    __syncwarp();
+    if (warp == 0) tmem_alloc(tslot, 512);
+    if (tid < 64) {
+        const int t = tid;
+        float b = 0.f, ip = -INFINITY, mt = 0.f, dnq = 0.f, A = 0.f, g = 0.f, wk = 0.f;
+        if (t < n) {
+            b = p.b[row0 + t];
+            ip = p.ip[row0 + t];
+            mt = p.mt[row0 + t];
+            dnq = p.dnq[row0 + t];
+            A = p.A[row0 + t];
+            g = expf(b + p.mprev[hc] - mt);
+            wk = expf(p.Bsum[hc] - b + ip - p.mend[hc]);
+        }
+        sb[t] = b; sip[t] = ip; smt[t] = mt; sdnq[t] = dnq; sA[t] = A; sg[t] = g; swk[t] = wk;
+    }
+    for (int j = tid; j < D; j += kTokThreads) {
+        snp[j] = p.nst[((size_t)bh * (NC + 1) + c) * D + j];
+        sdnb[j] = p.dnb[hc * D + j];
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tacc = *tslot;
+    const uint32_t lane_addr = ((uint32_t)(32 * quad)) << 16;
+    int ok = 0;
+    if (lane == 0) ok = mbar_wait(&bar[0], 0, abort_flag, status) ? 1 : 0;
+    __syncwarp();
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    if (ok && tid == 0) {
+        tc_fence_after();
+        const uint32_t idesc = idesc_f32acc(kFmtBF16, kFmtBF16, false, false, 64, 64);
+        const uint32_t sq = smem_u32(smem + Lay::kQ), sk = smem_u32(smem + Lay::kK), sv = smem_u32(smem + Lay::kV),
+                       sdh = smem_u32(smem + Lay::kDh), sdl = smem_u32(smem + Lay::kDl);
+#pragma unroll 1
+        for (int ks = 0; ks < D / 16; ++ks) {
+            const uint32_t off = (uint32_t)((ks >> 2) * 8192 + (ks & 3) * 32);
+            const uint32_t acc = ks > 0 ? 1u : 0u;
+            mma_bf16_ss(tacc + Lay::cS, sdesc_sw128(sq + off, 16, 1024), sdesc_sw128(sk + off, 16, 1024), idesc, acc);
+            const uint64_t bv = sdesc_sw128(sv + off, 16, 1024);
+            mma_bf16_ss(tacc + Lay::cP, sdesc_sw128(sdh + off, 16, 1024), bv, idesc, acc);
+            mma_bf16_ss(tacc + Lay::cP, sdesc_sw128(sdl + off, 16, 1024), bv, idesc, 1u);
+        }
+        mma_commit(&bar[1]);
+    }
+    // ---- M1, M2 tiles (warps 0-3: M = 64 layout, row t = 16 quad + (lane & 15))
+    int done1 = 0;
+    if (ok && lane == 0) done1 = mbar_wait(&bar[1], 0, abort_flag, status) ? 1 : 0;
+    __syncwarp();
+    done1 = __shfl_sync(0xffffffffu, done1, 0);
+    if (done1 && warp < 4) {
+        tc_fence_after();
+        const int t = 16 * warp + (lane & 15), hh = lane >> 4;
+        const float bt = sb[t], mtt = smt[t], dnqt = sdnq[t];
+#pragma unroll 1
+        for (int ph = 0; ph < 2; ++ph) {              // 0: S -> M2; 1: dP0 -> M1
+            const uint32_t base = tacc + (ph ? Lay::cP : Lay::cS) + lane_addr;
+            const int ho = ph ? Lay::kM1h : Lay::kM2h, lo_ = ph ? Lay::kM1l : Lay::kM2l;
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {    // columns 32 hh + 16 half + [0, 16)
+                uint32_t ra[16], rb[16];
+                tmem_ld16(base + 16 * half, ra);
+                tmem_ld16(base + 32 + 16 * half, rb);
+                tmem_wait_ld();
+                uint32_t hi[8], lo[8];
+#pragma unroll
+                for (int e = 0; e < 16; e += 2) {
+                    float x[2];
+#pragma unroll
+                    for (int u = 0; u < 2; ++u) {
+                        const uint32_t up = __shfl_sync(0xffffffffu, rb[e + u], lane & 15);
+                        const float val = __uint_as_float(hh ? up : ra[e + u]);
+                        const int s_ = 32 * hh + 16 * half + e + u;
+                        const float w = (t < n && s_ <= t) ? expf(bt - sb[s_] + sip[s_] - mtt) : 0.f;
+                        x[u] = ph ? w * (val + dnqt) : w * val * inv_sqrt;
+                    }
+                    hi[e / 2] = cvt_bf16x2(x[0], x[1]);
+                    const __nv_bfloat162 h2 = *reinterpret_cast<const __nv_bfloat162 *>(&hi[e / 2]);
+                    lo[e / 2] = cvt_bf16x2(x[0] - __low2float(h2), x[1] - __high2float(h2));
+                }
+#pragma unroll
+                for (int q = 0; q < 2; ++q) {
+                    const int piece = 4 * hh + 2 * half + q;
+                    const uint32_t off = (uint32_t)t * 128u + ((uint32_t)(piece ^ (t & 7)) << 4);
+                    *reinterpret_cast<uint4 *>(smem + ho + off) = make_uint4(hi[4 * q], hi[4 * q + 1], hi[4 * q + 2], hi[4 * q + 3]);
+                    *reinterpret_cast<uint4 *>(smem + lo_ + off) = make_uint4(lo[4 * q], lo[4 * q + 1], lo[4 * q + 2], lo[4 * q + 3]);
+                }
+            }
+        }
+        fence_async_smem();
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (done1 && tid == 0) {
+        tc_fence_after();
+        const uint32_t i_kt = idesc_f32acc(kFmtBF16, kFmtBF16, true, false, 128, 64);   // A^T, B K-major
+        const uint32_t i_tt = idesc_f32acc(kFmtBF16, kFmtBF16, true, true, 128, 64);    // A^T, B^T
+        const uint32_t sq = smem_u32(smem + Lay::kQ), sk = smem_u32(smem + Lay::kK), sdh = smem_u32(smem + Lay::kDh),
+                       sdl = smem_u32(smem + Lay::kDl), m1h = smem_u32(smem + Lay::kM1h), m1l = smem_u32(smem + Lay::kM1l),
+                       m2h = smem_u32(smem + Lay::kM2h), m2l = smem_u32(smem + Lay::kM2l);
+#pragma unroll
+        for (int mt = 0; mt < D / 128; ++mt)
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks) {
+                const uint32_t ta = 2 * mt * 8192 + ks * 2048;          // 16 token rows of a 128-row tile's two boxes
+                const uint32_t acc = ks > 0 ? 1u : 0u;
+                // dq^T = K^T M1^T: B = M1 rows t, K = s (K-major)
+                const uint64_t ak = sdesc_sw128(sk + ta, 8192, 1024);
+                mma_bf16_ss(tacc + Lay::cDq + 64 * mt, ak, sdesc_sw128(m1h + ks * 32, 16, 1024), i_kt, acc);
+                mma_bf16_ss(tacc + Lay::cDq + 64 * mt, ak, sdesc_sw128(m1l + ks * 32, 16, 1024), i_kt, 1u);
+                // dk^T = Q^T M1: B = M1 read as (N = s contiguous, K = t rows)
+                const uint64_t aq = sdesc_sw128(sq + ta, 8192, 1024);
+                mma_bf16_ss(tacc + Lay::cDk + 64 * mt, aq, sdesc_sw128(m1h + ks * 2048, 8192, 1024), i_tt, acc);
+                mma_bf16_ss(tacc + Lay::cDk + 64 * mt, aq, sdesc_sw128(m1l + ks * 2048, 8192, 1024), i_tt, 1u);
+                // dv^T = dnum'^T M2
+                const uint64_t adh = sdesc_sw128(sdh + ta, 8192, 1024), adl = sdesc_sw128(sdl + ta, 8192, 1024);
+                const uint64_t bm2h = sdesc_sw128(m2h + ks * 2048, 8192, 1024);
+                mma_bf16_ss(tacc + Lay::cDv + 64 * mt, adh, bm2h, i_tt, acc);
+                mma_bf16_ss(tacc + Lay::cDv + 64 * mt, adl, bm2h, i_tt, 1u);
+                mma_bf16_ss(tacc + Lay::cDv + 64 * mt, adh, sdesc_sw128(m2l + ks * 2048, 8192, 1024), i_tt, 1u);
+            }
+        mma_commit(&bar[2]);
+    }
+    int done2 = 0;
+    if (done1 && lane == 0) done2 = mbar_wait(&bar[2], 0, abort_flag, status) ? 1 : 0;
+    __syncwarp();
+    done2 = __shfl_sync(0xffffffffu, done2, 0);
+    if (done2) {
+        tc_fence_after();
+        const int tg = warp >> 2;
+        uint32_t v[D / 128][16];
+        __nv_bfloat16 *dq = reinterpret_cast<__nv_bfloat16 *>(p.dq), *dk = reinterpret_cast<__nv_bfloat16 *>(p.dk),
+                      *dv = reinterpret_cast<__nv_bfloat16 *>(p.dv);
+        // dq
+#pragma unroll
+        for (int mt = 0; mt < D / 128; ++mt) tmem_ld16(tacc + Lay::cDq + 64 * mt + lane_addr + 16 * tg, v[mt]);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+            const int t = 16 * tg + e;
+            if (t >= n) continue;
+            const size_t ro = (row0 + t) * D;
+#pragma unroll
+            for (int mt = 0; mt < D / 128; ++mt) {
+                const int j = 128 * mt + 32 * quad + lane;
+                dq[ro + j] = __float2bfloat16_rn(__uint_as_float(v[mt][e]) * inv_sqrt +
+                                                 sg[t] * (p.num[ro + j] + sdnq[t] * snp[j]));
+            }
+        }
+        // dk, ditilde
+#pragma unroll
+        for (int mt = 0; mt < D / 128; ++mt) tmem_ld16(tacc + Lay::cDk + 64 * mt + lane_addr + 16 * tg, v[mt]);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+            const int s_ = 16 * tg + e;
+            if (s_ >= n) continue;
+            const size_t ro = (row0 + s_) * D;
+            float di = 0.f;
+#pragma unroll
+            for (int mt = 0; mt < D / 128; ++mt) {
+                const int j = 128 * mt + 32 * quad + lane;
+                const float dkh = __uint_as_float(v[mt][e]) + swk[s_] * (p.dki[ro + j] + sdnb[j]);
+                const float kv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(
+                    smem + Lay::kK + (j >> 6) * 8192 + s_ * 128 + ((((j & 63) >> 3) ^ (s_ & 7)) << 4) + ((j & 7) << 1)));
+                di += dkh * kv * inv_sqrt;
+                dk[ro + j] = __float2bfloat16_rn(dkh * inv_sqrt);
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) di += __shfl_xor_sync(0xffffffffu, di, o);
+            if (lane == 0) red[quad * 64 + s_] = di;
+        }
+        // dv
+#pragma unroll
+        for (int mt = 0; mt < D / 128; ++mt) tmem_ld16(tacc + Lay::cDv + 64 * mt + lane_addr + 16 * tg, v[mt]);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+            const int s_ = 16 * tg + e;
+            if (s_ >= n) continue;
+            const size_t ro = (row0 + s_) * D;
+#pragma unroll
+            for (int mt = 0; mt < D / 128; ++mt) {
+                const int i = 128 * mt + 32 * quad + lane;
+                dv[ro + i] = __float2bfloat16_rn(__uint_as_float(v[mt][e]) + swk[s_] * inv_sqrt * p.dvi[ro + i]);
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (done2 && tid < n) {
+        const int s_ = tid;
+        const float di = red[s_] + red[64 + s_] + red[128 + s_] + red[192 + s_];
+        p.di[row0 + s_] = di;
+        p.dF[row0 + s_] = sA[s_] - di;
+    }
+    if (tid == 0 && !ok) mbar_wait(&bar[0], 0, nullptr, nullptr);     // no copy left in flight
+    __syncwarp();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tacc, 512);
+    }
+}
+
 }  // namespace bwdtc
 }  // namespace xlstm
