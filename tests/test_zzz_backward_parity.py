@@ -64,6 +64,10 @@ CASES = [
     (1, 2, 21, 32, 8, "exp", True, False, "f32"),
     (1, 1, 70, 64, 64, "sigmoid", False, True, "f32"),
     (2, 2, 40, 128, 16, "sigmoid", False, False, "bf16"),
+    # the tensor-core path (bf16, DH 128 / 256) with final-state cotangents,
+    # ragged chunks and wide gates
+    (1, 2, 70, 128, 32, "exp", True, True, "bf16"),
+    (1, 1, 100, 256, 64, "sigmoid", False, True, "bf16"),
     (1, 1, 1, 16, 1, "sigmoid", False, True, "f32"),
 ]
 
