@@ -652,39 +652,64 @@ token_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_cons
 #pragma unroll
             for (int mt = 0; mt < D / 128; ++mt) tmem_ld16(tacc + lane_addr + 64 + 64 * mt + 16 * tg, v[mt]);
             tmem_wait_ld();
+            // eight tokens at a time: every load of the batch is issued before
+            // the first store (the stores could alias them otherwise)
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-                const int t = 16 * tg + e;
-                if (t >= n) continue;
-                const float g = sg[t], den = sden[t];
-                const size_t rowoff = (row0 + t) * D;
-                float sdot = 0.f, A = 0.f;
+            for (int e0 = 0; e0 < 16; e0 += 8) {
+                float xn[8][D / 128], xo[8][D / 128], xd[8][D / 128];
 #pragma unroll
-                for (int mt = 0; mt < D / 128; ++mt) {
-                    const int i = 128 * mt + 32 * quad + lane;
-                    const float num = g * p.num[rowoff + i] + __uint_as_float(v[mt][e]);
-                    const float ht = num / den;
-                    const float o = bwd::sigmoid_hd(p.op[rowoff + i]);
-                    const float dhr = __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(p.dh)[rowoff + i]);
-                    const float dht = dhr * o;
-                    p.dO[rowoff + i] = dhr * ht * o * (1.f - o);
-                    const float dn = dht / den;
-                    p.dnum[rowoff + i] = dn;
-                    const __nv_bfloat16 h16 = __float2bfloat16_rn(dn);
-                    hl[rowoff + i] = h16;
-                    hl[plane + rowoff + i] = __float2bfloat16_rn(dn - __bfloat162float(h16));
-                    sdot += dht * ht;
-                    A += dn * num;
+                for (int e = 0; e < 8; ++e) {
+                    const int t = 16 * tg + e0 + e;
+                    const size_t rowoff = (row0 + (t < n ? t : 0)) * D;
+#pragma unroll
+                    for (int mt = 0; mt < D / 128; ++mt) {
+                        const int i = 128 * mt + 32 * quad + lane;
+                        xn[e][mt] = t < n ? p.num[rowoff + i] : 0.f;
+                        xo[e][mt] = t < n ? p.op[rowoff + i] : 0.f;
+                        xd[e][mt] = t < n ? __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(p.dh)[rowoff + i]) : 0.f;
+                    }
+                }
+                float sd[8], aa[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const int t = 16 * tg + e0 + e;
+                    sd[e] = 0.f;
+                    aa[e] = 0.f;
+                    if (t >= n) continue;
+                    const float g = sg[t], den = sden[t];
+                    const size_t rowoff = (row0 + t) * D;
+#pragma unroll
+                    for (int mt = 0; mt < D / 128; ++mt) {
+                        const int i = 128 * mt + 32 * quad + lane;
+                        const float num = g * xn[e][mt] + __uint_as_float(v[mt][e0 + e]);
+                        const float ht = num / den;
+                        const float o = bwd::sigmoid_hd(xo[e][mt]);
+                        const float dhr = xd[e][mt];
+                        const float dht = dhr * o;
+                        p.dO[rowoff + i] = dhr * ht * o * (1.f - o);
+                        const float dn = dht / den;
+                        p.dnum[rowoff + i] = dn;
+                        const __nv_bfloat16 h16 = __float2bfloat16_rn(dn);
+                        hl[rowoff + i] = h16;
+                        hl[plane + rowoff + i] = __float2bfloat16_rn(dn - __bfloat162float(h16));
+                        sd[e] += dht * ht;
+                        aa[e] += dn * num;
+                    }
                 }
 #pragma unroll
-                for (int o = 16; o > 0; o >>= 1) {
-                    sdot += __shfl_xor_sync(0xffffffffu, sdot, o);
-                    A += __shfl_xor_sync(0xffffffffu, A, o);
-                }
-                if (lane == 0) {
-                    red[quad * 64 + t] = sdot;
-                    red[256 + quad * 64 + t] = A;
-                }
+                for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        sd[e] += __shfl_xor_sync(0xffffffffu, sd[e], o);
+                        aa[e] += __shfl_xor_sync(0xffffffffu, aa[e], o);
+                    }
+                if (lane == 0)
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const int t = 16 * tg + e0 + e;
+                        red[quad * 64 + t] = sd[e];
+                        red[256 + quad * 64 + t] = aa[e];
+                    }
             }
         }
     }
@@ -904,7 +929,20 @@ token_grad_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_con
         uint32_t v[D / 128][16];
         __nv_bfloat16 *dq = reinterpret_cast<__nv_bfloat16 *>(p.dq), *dk = reinterpret_cast<__nv_bfloat16 *>(p.dk),
                       *dv = reinterpret_cast<__nv_bfloat16 *>(p.dv);
+        // the state products of the 16 tokens are loaded before the first store
+        // (the stores could alias them otherwise)
+        float x[16][D / 128];
+        auto preload = [&](const float *src) {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+                const int t = 16 * tg + e;
+#pragma unroll
+                for (int mt = 0; mt < D / 128; ++mt)
+                    x[e][mt] = t < n ? src[(row0 + t) * D + 128 * mt + 32 * quad + lane] : 0.f;
+            }
+        };
         // dq
+        preload(p.num);
 #pragma unroll
         for (int mt = 0; mt < D / 128; ++mt) tmem_ld16(tacc + Lay::cDq + 64 * mt + lane_addr + 16 * tg, v[mt]);
         tmem_wait_ld();
@@ -917,10 +955,11 @@ token_grad_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_con
             for (int mt = 0; mt < D / 128; ++mt) {
                 const int j = 128 * mt + 32 * quad + lane;
                 dq[ro + j] = __float2bfloat16_rn(__uint_as_float(v[mt][e]) * inv_sqrt +
-                                                 sg[t] * (p.num[ro + j] + sdnq[t] * snp[j]));
+                                                 sg[t] * (x[e][mt] + sdnq[t] * snp[j]));
             }
         }
         // dk, ditilde
+        preload(p.dki);
 #pragma unroll
         for (int mt = 0; mt < D / 128; ++mt) tmem_ld16(tacc + Lay::cDk + 64 * mt + lane_addr + 16 * tg, v[mt]);
         tmem_wait_ld();
@@ -933,7 +972,7 @@ token_grad_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_con
 #pragma unroll
             for (int mt = 0; mt < D / 128; ++mt) {
                 const int j = 128 * mt + 32 * quad + lane;
-                const float dkh = __uint_as_float(v[mt][e]) + swk[s_] * (p.dki[ro + j] + sdnb[j]);
+                const float dkh = __uint_as_float(v[mt][e]) + swk[s_] * (x[e][mt] + sdnb[j]);
                 const float kv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(
                     smem + Lay::kK + (j >> 6) * 8192 + s_ * 128 + ((((j & 63) >> 3) ^ (s_ & 7)) << 4) + ((j & 7) << 1)));
                 di += dkh * kv * inv_sqrt;
@@ -944,6 +983,7 @@ token_grad_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_con
             if (lane == 0) red[quad * 64 + s_] = di;
         }
         // dv
+        preload(p.dvi);
 #pragma unroll
         for (int mt = 0; mt < D / 128; ++mt) tmem_ld16(tacc + Lay::cDv + 64 * mt + lane_addr + 16 * tg, v[mt]);
         tmem_wait_ld();
@@ -955,7 +995,7 @@ token_grad_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_con
 #pragma unroll
             for (int mt = 0; mt < D / 128; ++mt) {
                 const int i = 128 * mt + 32 * quad + lane;
-                dv[ro + i] = __float2bfloat16_rn(__uint_as_float(v[mt][e]) + swk[s_] * inv_sqrt * p.dvi[ro + i]);
+                dv[ro + i] = __float2bfloat16_rn(__uint_as_float(v[mt][e]) + swk[s_] * inv_sqrt * x[e][mt]);
             }
         }
     }
