@@ -279,8 +279,11 @@ xlstm_status xlstm_mlstm_state_combine(const float *parts, int count, const floa
  * stabiliser is held fixed, which "xLSTM: Extended Long Short-Term Memory"
  * section 2.2 (appendix A.2) shows leaves the derivatives unchanged; the
  * returned state's own stabiliser m_T is differentiated where the final-state
- * cotangents need it.  fp32 arithmetic on CUDA cores; the chunk-start and
- * reverse states are materialised in the workspace.
+ * cotangents need it.  The chunk-start and reverse states are materialised in
+ * the workspace.  bf16 inputs with DH 128 or 256 run on the tensor cores
+ * (tcgen05, fp32 accumulation; every fp32 operand enters as a bf16 high + low
+ * pair, about 16 significant bits); other arguments run fp32 arithmetic on
+ * CUDA cores.
  *
  *   q, k, v, dh     [B, NH, S, DH]  dtype dt (dh: cotangent of h)
  *   i_pre, f_pre    [B, NH, S]      float
@@ -330,7 +333,11 @@ xlstm_status xlstm_mlstm_bwd(const void *q, const void *k, const void *v,
  *   c_out, n_out, m_out, h_out  [B, NH, DH] float, final state; each nullable
  * Outputs must not be any input or each other (XLSTM_ERR_UNSUPPORTED).
  * DH in [1, 512].  S == 0 copies the initial state to the state outputs.
- * One CTA per (batch, head), fp32; correctness-first (R read from L2 every step).
+ * fp32 throughout.  DH 64, 128, 256 (and 512 where the device can place a
+ * 16-CTA cluster): a cluster of DH/32 CTAs per (batch, head) keeps the
+ * recurrent blocks on chip for the whole sequence and exchanges h_t through
+ * distributed shared memory, one cluster barrier per step; other DH: one CTA
+ * per (batch, head) reading R from L2 at every step.
  */
 xlstm_status xlstm_slstm_fwd(const float *zx, const float *ix, const float *fx, const float *ox,
                              const float *R, float *h,
