@@ -120,6 +120,22 @@ def test_differentiable_op_matches_gradient_oracle(cuda_lib):
     _check(got, ref, "f32", 1e-4)
 
 
+def test_differentiable_op_on_the_tensor_core_path(cuda_lib):
+    """The autograd op with bf16 q/k/v at DH 128 (the tensor-core backward, and
+    the tensor-core forward): gradients of a loss on h and on the final state."""
+    from linear_rnn_mlstm_b200.autograd import mlstm_cell
+    t = _inputs(1, 2, 150, 128, "sigmoid", False, "bf16", seed=21)
+    x = {nm: t[nm].cuda().requires_grad_(True) for nm in NAMES}
+    h, C, n, m = mlstm_cell(*(x[nm] for nm in NAMES), chunk=64)
+    ((h.float() * t["dh"].float().cuda()).sum() + (C * t["dC"].cuda()).sum() +
+     (n * t["dn"].cuda()).sum()).backward()
+    torch.cuda.synchronize()
+    ref = bw.grads(*(t[nm] for nm in NAMES), t["dh"], "sigmoid", dC=t["dC"].numpy(),
+                   dn=t["dn"].numpy())[1]
+    got = {OUT[nm]: x[nm].grad for nm in NAMES}
+    _check(got, ref, "bf16", 1e-4)
+
+
 # Workload-sized shapes: the small workload whole (B4 NH4 S1024 DH64), and one
 # head of the long (S4096, DH256) and block (S1024, DH512, exponential forget
 # gate with i ~ N(0, 3)) workloads at their own gate distributions, bf16 q/k/v
