@@ -725,9 +725,9 @@ size_t bwd_layout(long long BH, long long S, long long DH, long long NC, bool tc
     return off;
 }
 
-// The backward's products with the chunk states run on the tensor cores for
-// bf16 inputs with DH 128 or 256 (the per-chunk token kernels' shapes).
-bool bwd_uses_tc(xlstm_dtype dt, int DH) { return dt == XLSTM_BF16 && (DH == 128 || DH == 256); }
+// The backward runs on the tensor cores for bf16 inputs with DH 64, 128 or
+// 256 (DH 64: one 128-row tile whose upper half is padding).
+bool bwd_uses_tc(xlstm_dtype dt, int DH) { return dt == XLSTM_BF16 && (DH == 64 || DH == 128 || DH == 256); }
 
 bool misaligned16(const void *p) { return ((uintptr_t)p & 15u) != 0; }
 
@@ -757,7 +757,7 @@ cudaError_t launch_state_mma_t(const BwdPtrs &p, const float *states, int slots_
     cudaError_t e = cudaFuncSetAttribute(bwdtc::state_mma_kernel<D, A_T, B_SPLIT>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
     if (e != cudaSuccess) return e;
-    bwdtc::state_mma_kernel<D, A_T, B_SPLIT><<<dim3((unsigned)((long long)p.NC * p.BH), D / 128),
+    bwdtc::state_mma_kernel<D, A_T, B_SPLIT><<<dim3((unsigned)((long long)p.NC * p.BH), bwdtc::kTiles<D>),
                                                bwdtc::kMmaThreads, sm, st>>>(
         m1, m2, reinterpret_cast<const uint8_t *>(states), (size_t)slots_per_head * slot_bytes, slot_bytes, out,
         p.S, p.L, p.NC, device_status_ptr());
@@ -795,7 +795,7 @@ cudaError_t launch_state_recurrence_t(const BwdPtrs &p, cudaStream_t st) {
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
         if (e != cudaSuccess) return e;
         KernelTimer timer(REVERSE ? "bwd_reverse_mma" : "bwd_states_mma", st);
-        bwdtc::delta_mma_kernel<D, REVERSE><<<dim3((unsigned)((long long)nce * p.BH), D / 128), bwdtc::kMmaThreads,
+        bwdtc::delta_mma_kernel<D, REVERSE><<<dim3((unsigned)((long long)nce * p.BH), bwdtc::kTiles<D>), bwdtc::kMmaThreads,
                                               sm, st>>>(ma, ma2, mb, p, c_first, nce, device_status_ptr());
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
@@ -806,6 +806,8 @@ cudaError_t launch_state_recurrence_t(const BwdPtrs &p, cudaStream_t st) {
 }
 
 cudaError_t launch_state_recurrence(const BwdPtrs &p, bool reverse, cudaStream_t st) {
+    if (p.DH == 64)
+        return reverse ? launch_state_recurrence_t<64, true>(p, st) : launch_state_recurrence_t<64, false>(p, st);
     if (p.DH == 128)
         return reverse ? launch_state_recurrence_t<128, true>(p, st) : launch_state_recurrence_t<128, false>(p, st);
     return reverse ? launch_state_recurrence_t<256, true>(p, st) : launch_state_recurrence_t<256, false>(p, st);
@@ -843,7 +845,9 @@ cudaError_t launch_token_grad_tc_t(const BwdPtrs &p, cudaStream_t st) {
 
 cudaError_t launch_state_products(const BwdPtrs &p, int which, cudaStream_t st) {
     KernelTimer timer("bwd_state_mma", st);
-    return p.DH == 128 ? launch_state_mma<128>(p, which, st) : launch_state_mma<256>(p, which, st);
+    return p.DH == 64    ? launch_state_mma<64>(p, which, st)
+           : p.DH == 128 ? launch_state_mma<128>(p, which, st)
+                         : launch_state_mma<256>(p, which, st);
 }
 
 template <typename T>
@@ -864,7 +868,9 @@ cudaError_t launch_bwd(const BwdPtrs &p, cudaStream_t st) {
     }
     if (p.tc) {
         KernelTimer timer("bwd_token_fwd_tc", st);
-        e = p.DH == 128 ? launch_token_fwd_tc_t<128>(p, st) : launch_token_fwd_tc_t<256>(p, st);
+        e = p.DH == 64    ? launch_token_fwd_tc_t<64>(p, st)
+            : p.DH == 128 ? launch_token_fwd_tc_t<128>(p, st)
+                          : launch_token_fwd_tc_t<256>(p, st);
         if (e != cudaSuccess) return e;
     } else {
         KernelTimer timer("bwd_token_fwd", st);
@@ -881,7 +887,9 @@ cudaError_t launch_bwd(const BwdPtrs &p, cudaStream_t st) {
     }
     if (p.tc) {
         KernelTimer timer("bwd_token_grad_tc", st);
-        e = p.DH == 128 ? launch_token_grad_tc_t<128>(p, st) : launch_token_grad_tc_t<256>(p, st);
+        e = p.DH == 64    ? launch_token_grad_tc_t<64>(p, st)
+            : p.DH == 128 ? launch_token_grad_tc_t<128>(p, st)
+                          : launch_token_grad_tc_t<256>(p, st);
         if (e != cudaSuccess) return e;
     } else {
         KernelTimer timer("bwd_token_grad", st);

@@ -40,6 +40,12 @@ __host__ __device__ inline uint32_t plane_offset(int r, int j, int DH) {
 
 constexpr int kMmaThreads = 128;
 
+// 128-row tiles along a DH-long dimension (DH 64: one tile, rows 64-127 of its
+// MMAs are padding, computed and never stored), and the bytes of one 128 x 64
+// plane block in global memory (DH 64: 64 rows).
+template <int D> constexpr int kTiles = D >= 128 ? D / 128 : 1;
+template <int D> constexpr uint32_t kBlkBytes = D >= 128 ? 16384u : (uint32_t)D * 128u;
+
 template <int D, bool B_SPLIT>
 struct MmaLay {
     static constexpr int kAtoms = D / 64;               // 64-wide K blocks
@@ -90,7 +96,7 @@ state_mma_kernel(const __grid_constant__ CUtensorMap map_b, const __grid_constan
 
     bool loaded = true;
     if (threadIdx.x == 0) {
-        mbar_arrive_expect_tx(&bar[0], 2 * Lay::kAPlane + (B_SPLIT ? 2 : 1) * Lay::kBPlane);
+        mbar_arrive_expect_tx(&bar[0], 2 * Lay::kAtoms * kBlkBytes<D> + (B_SPLIT ? 2 : 1) * Lay::kBPlane);
         for (int pl = 0; pl < 2; ++pl)
             for (int a = 0; a < Lay::kAtoms; ++a) {
                 // K-major: this CTA's row tile mt, column blocks a.  MN-major: column
@@ -98,7 +104,7 @@ state_mma_kernel(const __grid_constant__ CUtensorMap map_b, const __grid_constan
                 const uint32_t gblk = A_T ? (uint32_t)((a >> 1) * (D / 64) + 2 * mt + (a & 1))
                                           : (uint32_t)(mt * Lay::kAtoms + a);
                 bulk_load(smem + Lay::kA + pl * Lay::kAPlane + a * 16384, slot + pl * kPlaneBytes + gblk * 16384u,
-                          16384u, &bar[0]);
+                          kBlkBytes<D>, &bar[0]);
             }
         for (int a = 0; a < Lay::kAtoms; ++a) {
             tma_load_3d(smem + Lay::kB + a * 8192, &map_b, &bar[0], 64 * a, a0, bh);
@@ -144,14 +150,16 @@ state_mma_kernel(const __grid_constant__ CUtensorMap map_b, const __grid_constan
 #pragma unroll
         for (int q = 0; q < 4; ++q) tmem_ld16(tacc + ((uint32_t)(32 * warp) << 16) + 16 * q, v[q]);
         tmem_wait_ld();
-        float *dst = out + ((size_t)bh * S + a0) * D + 128 * mt + 32 * warp + lane;
+        const int row = 128 * mt + 32 * warp + lane;
+        float *dst = out + ((size_t)bh * S + a0) * D + row;
+        if (row < D)
 #pragma unroll
-        for (int q = 0; q < 4; ++q)
+            for (int q = 0; q < 4; ++q)
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-                const int t = 16 * q + e;
-                if (t < n) dst[(size_t)t * D] = __uint_as_float(v[q][e]);
-            }
+                for (int e = 0; e < 16; ++e) {
+                    const int t = 16 * q + e;
+                    if (t < n) dst[(size_t)t * D] = __uint_as_float(v[q][e]);
+                }
     }
     tc_fence_before();
     __syncthreads();
@@ -346,9 +354,10 @@ delta_mma_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
     if (tid == 0 && done) {
         uint8_t *slot = reinterpret_cast<uint8_t *>(REVERSE ? p.dCb + ((size_t)bh * NC + c - 1) * DD
                                                             : p.Cst + ((size_t)bh * (NC + 1) + c + 1) * DD);
-        const uint32_t bytes = (uint32_t)(D / 64) * 16384u;
+        // staged as 128-row blocks; in global memory a block holds min(DH, 128) rows
+        const uint32_t sbytes = (uint32_t)(D / 64) * 16384u, gbytes = (uint32_t)(D / 64) * kBlkBytes<D>;
         for (int pl = 0; pl < 2; ++pl)
-            bulk_store(slot + (size_t)pl * DD * 2 + (size_t)mt * bytes, smem + pl * bytes, bytes);
+            bulk_store(slot + (size_t)pl * DD * 2 + (size_t)mt * gbytes, smem + pl * sbytes, gbytes);
         bulk_commit();
         bulk_wait_all();
     }
@@ -622,7 +631,7 @@ token_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_cons
         const uint32_t idesc = idesc_f32acc(kFmtBF16, kFmtBF16, true, false, 128, 64);
         const uint32_t svv = smem_u32(smem + Lay::kV), wh = smem_u32(smem + Lay::kWhi), wl = smem_u32(smem + Lay::kWlo);
 #pragma unroll
-        for (int mt = 0; mt < D / 128; ++mt)
+        for (int mt = 0; mt < kTiles<D>; ++mt)
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks) {
                 const uint64_t ad = sdesc_sw128(svv + 2 * mt * 8192 + ks * 2048, 8192, 1024);
@@ -648,25 +657,26 @@ token_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_cons
         const size_t plane = (size_t)p.BH * S * D;
         {
             const int tg = warp >> 2;
-            uint32_t v[D / 128][16];
+            uint32_t v[kTiles<D>][16];
 #pragma unroll
-            for (int mt = 0; mt < D / 128; ++mt) tmem_ld16(tacc + lane_addr + 64 + 64 * mt + 16 * tg, v[mt]);
+            for (int mt = 0; mt < kTiles<D>; ++mt) tmem_ld16(tacc + lane_addr + 64 + 64 * mt + 16 * tg, v[mt]);
             tmem_wait_ld();
             // eight tokens at a time: every load of the batch is issued before
             // the first store (the stores could alias them otherwise)
 #pragma unroll
             for (int e0 = 0; e0 < 16; e0 += 8) {
-                float xn[8][D / 128], xo[8][D / 128], xd[8][D / 128];
+                float xn[8][kTiles<D>], xo[8][kTiles<D>], xd[8][kTiles<D>];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
                     const int t = 16 * tg + e0 + e;
                     const size_t rowoff = (row0 + (t < n ? t : 0)) * D;
 #pragma unroll
-                    for (int mt = 0; mt < D / 128; ++mt) {
+                    for (int mt = 0; mt < kTiles<D>; ++mt) {
                         const int i = 128 * mt + 32 * quad + lane;
-                        xn[e][mt] = t < n ? p.num[rowoff + i] : 0.f;
-                        xo[e][mt] = t < n ? p.op[rowoff + i] : 0.f;
-                        xd[e][mt] = t < n ? __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(p.dh)[rowoff + i]) : 0.f;
+                        const bool in = t < n && i < D;
+                        xn[e][mt] = in ? p.num[rowoff + i] : 0.f;
+                        xo[e][mt] = in ? p.op[rowoff + i] : 0.f;
+                        xd[e][mt] = in ? __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(p.dh)[rowoff + i]) : 0.f;
                     }
                 }
                 float sd[8], aa[8];
@@ -679,8 +689,9 @@ token_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_cons
                     const float g = sg[t], den = sden[t];
                     const size_t rowoff = (row0 + t) * D;
 #pragma unroll
-                    for (int mt = 0; mt < D / 128; ++mt) {
+                    for (int mt = 0; mt < kTiles<D>; ++mt) {
                         const int i = 128 * mt + 32 * quad + lane;
+                        if (i >= D) continue;                // padding rows of a 64-row head
                         const float num = g * xn[e][mt] + __uint_as_float(v[mt][e0 + e]);
                         const float ht = num / den;
                         const float o = bwd::sigmoid_hd(xo[e][mt]);
@@ -758,7 +769,7 @@ struct GradLay {
     static constexpr int kFloats = 7 * 64 + 4 * 64 + 2 * D;
     static constexpr int kBar = kF + kFloats * 4;
     static constexpr int kBytes = kBar + 64 + 1024;
-    static constexpr int cS = 0, cP = 64, cDq = 128, cDk = 128 + 64 * (D / 128), cDv = 128 + 128 * (D / 128);
+    static constexpr int cS = 0, cP = 64, cDq = 128, cDk = 128 + 64 * (kTiles<D>), cDv = 128 + 128 * (kTiles<D>);
 };
 
 template <int D>
@@ -897,7 +908,7 @@ token_grad_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_con
                        sdl = smem_u32(smem + Lay::kDl), m1h = smem_u32(smem + Lay::kM1h), m1l = smem_u32(smem + Lay::kM1l),
                        m2h = smem_u32(smem + Lay::kM2h), m2l = smem_u32(smem + Lay::kM2l);
 #pragma unroll
-        for (int mt = 0; mt < D / 128; ++mt)
+        for (int mt = 0; mt < kTiles<D>; ++mt)
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks) {
                 const uint32_t ta = 2 * mt * 8192 + ks * 2048;          // 16 token rows of a 128-row tile's two boxes
@@ -926,25 +937,27 @@ token_grad_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_con
     if (done2) {
         tc_fence_after();
         const int tg = warp >> 2;
-        uint32_t v[D / 128][16];
+        uint32_t v[kTiles<D>][16];
         __nv_bfloat16 *dq = reinterpret_cast<__nv_bfloat16 *>(p.dq), *dk = reinterpret_cast<__nv_bfloat16 *>(p.dk),
                       *dv = reinterpret_cast<__nv_bfloat16 *>(p.dv);
         // the state products of the 16 tokens are loaded before the first store
         // (the stores could alias them otherwise)
-        float x[16][D / 128];
+        float x[16][kTiles<D>];
         auto preload = [&](const float *src) {
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
                 const int t = 16 * tg + e;
 #pragma unroll
-                for (int mt = 0; mt < D / 128; ++mt)
-                    x[e][mt] = t < n ? src[(row0 + t) * D + 128 * mt + 32 * quad + lane] : 0.f;
+                for (int mt = 0; mt < kTiles<D>; ++mt) {
+                    const int r = 128 * mt + 32 * quad + lane;
+                    x[e][mt] = t < n && r < D ? src[(row0 + t) * D + r] : 0.f;
+                }
             }
         };
         // dq
         preload(p.num);
 #pragma unroll
-        for (int mt = 0; mt < D / 128; ++mt) tmem_ld16(tacc + Lay::cDq + 64 * mt + lane_addr + 16 * tg, v[mt]);
+        for (int mt = 0; mt < kTiles<D>; ++mt) tmem_ld16(tacc + Lay::cDq + 64 * mt + lane_addr + 16 * tg, v[mt]);
         tmem_wait_ld();
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
@@ -952,8 +965,9 @@ token_grad_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_con
             if (t >= n) continue;
             const size_t ro = (row0 + t) * D;
 #pragma unroll
-            for (int mt = 0; mt < D / 128; ++mt) {
+            for (int mt = 0; mt < kTiles<D>; ++mt) {
                 const int j = 128 * mt + 32 * quad + lane;
+                if (j >= D) continue;
                 dq[ro + j] = __float2bfloat16_rn(__uint_as_float(v[mt][e]) * inv_sqrt +
                                                  sg[t] * (x[e][mt] + sdnq[t] * snp[j]));
             }
@@ -961,7 +975,7 @@ token_grad_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_con
         // dk, ditilde
         preload(p.dki);
 #pragma unroll
-        for (int mt = 0; mt < D / 128; ++mt) tmem_ld16(tacc + Lay::cDk + 64 * mt + lane_addr + 16 * tg, v[mt]);
+        for (int mt = 0; mt < kTiles<D>; ++mt) tmem_ld16(tacc + Lay::cDk + 64 * mt + lane_addr + 16 * tg, v[mt]);
         tmem_wait_ld();
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
@@ -970,8 +984,9 @@ token_grad_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_con
             const size_t ro = (row0 + s_) * D;
             float di = 0.f;
 #pragma unroll
-            for (int mt = 0; mt < D / 128; ++mt) {
+            for (int mt = 0; mt < kTiles<D>; ++mt) {
                 const int j = 128 * mt + 32 * quad + lane;
+                if (j >= D) continue;
                 const float dkh = __uint_as_float(v[mt][e]) + swk[s_] * (x[e][mt] + sdnb[j]);
                 const float kv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(
                     smem + Lay::kK + (j >> 6) * 8192 + s_ * 128 + ((((j & 63) >> 3) ^ (s_ & 7)) << 4) + ((j & 7) << 1)));
@@ -985,7 +1000,7 @@ token_grad_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_con
         // dv
         preload(p.dvi);
 #pragma unroll
-        for (int mt = 0; mt < D / 128; ++mt) tmem_ld16(tacc + Lay::cDv + 64 * mt + lane_addr + 16 * tg, v[mt]);
+        for (int mt = 0; mt < kTiles<D>; ++mt) tmem_ld16(tacc + Lay::cDv + 64 * mt + lane_addr + 16 * tg, v[mt]);
         tmem_wait_ld();
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
@@ -993,8 +1008,9 @@ token_grad_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_con
             if (s_ >= n) continue;
             const size_t ro = (row0 + s_) * D;
 #pragma unroll
-            for (int mt = 0; mt < D / 128; ++mt) {
+            for (int mt = 0; mt < kTiles<D>; ++mt) {
                 const int i = 128 * mt + 32 * quad + lane;
+                if (i >= D) continue;
                 dv[ro + i] = __float2bfloat16_rn(__uint_as_float(v[mt][e]) + swk[s_] * inv_sqrt * x[e][mt]);
             }
         }

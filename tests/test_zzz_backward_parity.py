@@ -69,6 +69,7 @@ CASES = [
     (1, 2, 70, 128, 32, "exp", True, True, "bf16"),
     (1, 1, 100, 256, 64, "sigmoid", False, True, "bf16"),
     (1, 1, 3, 128, 1, "sigmoid", False, True, "bf16"),      # one-token chunks
+    (1, 2, 90, 64, 32, "exp", True, True, "bf16"),          # DH 64 (padded 128-row tiles)
     (1, 1, 1, 16, 1, "sigmoid", False, True, "f32"),
 ]
 
