@@ -280,7 +280,7 @@ xlstm_status xlstm_mlstm_state_combine(const float *parts, int count, const floa
  * section 2.2 (appendix A.2) shows leaves the derivatives unchanged; the
  * returned state's own stabiliser m_T is differentiated where the final-state
  * cotangents need it.  The chunk-start and reverse states are materialised in
- * the workspace.  bf16 inputs with DH 128 or 256 run on the tensor cores
+ * the workspace.  bf16 inputs with DH 64, 128 or 256 run on the tensor cores
  * (tcgen05, fp32 accumulation; every fp32 operand enters as a bf16 high + low
  * pair, about 16 significant bits); other arguments run fp32 arithmetic on
  * CUDA cores.
