@@ -1,5 +1,6 @@
-// Tensor-core products of the backward with the chunk states (included by
-// bwd.cu; bf16 inputs, DH 128 or 256).
+// The backward's tensor-core kernels (included by bwd.cu; bf16 inputs, DH 64,
+// 128 or 256): the state increments and scans, the products with the states,
+// and the two per-token passes.
 //
 // The chunkwise backward of "xLSTM: Extended Long Short-Term Memory" (section
 // 2.3's recurrence, stabiliser held fixed per section 2.2) multiplies every
