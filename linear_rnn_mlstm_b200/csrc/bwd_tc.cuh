@@ -505,7 +505,7 @@ token_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_cons
     uint8_t *smem = align1k(tok_smem_raw);
     float *fb = reinterpret_cast<float *>(smem + Lay::kF);
     float *sb = fb, *sip = fb + 64, *smt = fb + 128, *sg = fb + 192, *sden = fb + 256, *snq = fb + 320,
-          *srs = fb + 448, *red = fb + 512, *snp = fb + 512 + 1024;
+          *red = fb + 512, *snp = fb + 512 + 1024;
     uint64_t *bar = reinterpret_cast<uint64_t *>(smem + Lay::kBar);
     uint32_t *tslot = reinterpret_cast<uint32_t *>(smem + Lay::kBar + 32);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + Lay::kBar + 36);
@@ -584,31 +584,27 @@ token_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_cons
     if (ok && lane == 0) done1 = mbar_wait(&bar[1], 0, abort_flag, status) ? 1 : 0;
     __syncwarp();
     done1 = __shfl_sync(0xffffffffu, done1, 0);
-    if (done1 && warp < 4) {
+    if (done1) {
         tc_fence_after();
-        uint32_t sa[64];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) tmem_ld16(tacc + lane_addr + 16 * q, *reinterpret_cast<uint32_t(*)[16]>(&sa[16 * q]));
+        // all 16 warps: warp w reads TMEM lane quadrant w % 4 (M = 64 layout: rows
+        // t = 16 (w % 4) + (lane & 15) in the quadrant's lanes 0-15) at columns
+        // 16 (w / 4) .. + 15; lanes 16-31 take their row's upper 8 of those columns
+        const int cg = warp >> 2, t = 16 * quad + (lane & 15), hh = lane >> 4;
+        uint32_t sa[16];
+        tmem_ld16(tacc + lane_addr + 16 * cg, sa);
         tmem_wait_ld();
-        // M = 64 layout: row t = 16 warp + (lane & 15) in TMEM lanes 0-15 of the
-        // warp's quadrant; lanes 16-31 take that row's columns 32-63
-        const int t = 16 * warp + (lane & 15), hh = lane >> 4;
-        float sv[32];
-#pragma unroll
-        for (int e = 0; e < 32; ++e) {
-            const uint32_t up = __shfl_sync(0xffffffffu, sa[32 + e], lane & 15);
-            sv[e] = __uint_as_float(hh ? up : sa[e]);
-        }
-        float rs = 0.f;
         const float bt = sb[t], mtt = smt[t];
-        uint32_t hi[16], lo[16];
+        float rs = 0.f;
+        uint32_t hi[4], lo[4];
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) {
+        for (int e = 0; e < 8; e += 2) {
             float w2[2];
 #pragma unroll
             for (int u = 0; u < 2; ++u) {
-                const int s_ = 32 * hh + e + u;
-                w2[u] = (t < n && s_ <= t) ? expf(bt - sb[s_] + sip[s_] - mtt) * sv[e + u] * inv_sqrt : 0.f;
+                const uint32_t up = __shfl_sync(0xffffffffu, sa[8 + e + u], lane & 15);
+                const float sv = __uint_as_float(hh ? up : sa[e + u]);
+                const int s_ = 16 * cg + 8 * hh + e + u;
+                w2[u] = (t < n && s_ <= t) ? expf(bt - sb[s_] + sip[s_] - mtt) * sv * inv_sqrt : 0.f;
                 rs += w2[u];
             }
             hi[e / 2] = cvt_bf16x2(w2[0], w2[1]);
@@ -616,13 +612,10 @@ token_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_cons
             lo[e / 2] = cvt_bf16x2(w2[0] - __low2float(h2), w2[1] - __high2float(h2));
         }
         rs += __shfl_xor_sync(0xffffffffu, rs, 16);
-        if (hh == 0) srs[t] = rs;
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {                 // pieces 4 hh + q of row t
-            const uint32_t off = (uint32_t)t * 128u + ((uint32_t)((4 * hh + q) ^ (t & 7)) << 4);
-            *reinterpret_cast<uint4 *>(smem + Lay::kWhi + off) = make_uint4(hi[4 * q], hi[4 * q + 1], hi[4 * q + 2], hi[4 * q + 3]);
-            *reinterpret_cast<uint4 *>(smem + Lay::kWlo + off) = make_uint4(lo[4 * q], lo[4 * q + 1], lo[4 * q + 2], lo[4 * q + 3]);
-        }
+        if (hh == 0) red[256 + cg * 64 + t] = rs;     // this warp's 16 columns of row t's sum
+        const uint32_t off = (uint32_t)t * 128u + ((uint32_t)((2 * cg + hh) ^ (t & 7)) << 4);
+        *reinterpret_cast<uint4 *>(smem + Lay::kWhi + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+        *reinterpret_cast<uint4 *>(smem + Lay::kWlo + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
         fence_async_smem();
     }
     tc_fence_before();
@@ -643,7 +636,8 @@ token_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_cons
     }
     if (done1 && tid < 64) {                          // normaliser and floor per token
         const int t = tid;
-        const float nq = sg[t] * red[t] + srs[t];
+        const float rsum = red[256 + t] + red[320 + t] + red[384 + t] + red[448 + t];
+        const float nq = sg[t] * red[t] + rsum;
         snq[t] = nq;
         sden[t] = t < n ? fmaxf(fabsf(nq), expf(-smt[t])) : 1.f;
     }
@@ -658,14 +652,14 @@ token_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_cons
         const size_t plane = (size_t)p.BH * S * D;
         {
             const int tg = warp >> 2;
-            uint32_t v[kTiles<D>][16];
-#pragma unroll
-            for (int mt = 0; mt < kTiles<D>; ++mt) tmem_ld16(tacc + lane_addr + 64 + 64 * mt + 16 * tg, v[mt]);
-            tmem_wait_ld();
             // eight tokens at a time: every load of the batch is issued before
             // the first store (the stores could alias them otherwise)
 #pragma unroll
             for (int e0 = 0; e0 < 16; e0 += 8) {
+                uint32_t v[kTiles<D>][8];
+#pragma unroll
+                for (int mt = 0; mt < kTiles<D>; ++mt) tmem_ld8(tacc + lane_addr + 64 + 64 * mt + 16 * tg + e0, v[mt]);
+                tmem_wait_ld();
                 float xn[8][kTiles<D>], xo[8][kTiles<D>], xd[8][kTiles<D>];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
@@ -693,7 +687,7 @@ token_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_cons
                     for (int mt = 0; mt < kTiles<D>; ++mt) {
                         const int i = 128 * mt + 32 * quad + lane;
                         if (i >= D) continue;                // padding rows of a 64-row head
-                        const float num = g * xn[e][mt] + __uint_as_float(v[mt][e0 + e]);
+                        const float num = g * xn[e][mt] + __uint_as_float(v[mt][e]);
                         const float ht = num / den;
                         const float o = bwd::sigmoid_hd(xo[e][mt]);
                         const float dhr = xd[e][mt];
@@ -858,45 +852,44 @@ token_grad_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_con
     if (ok && lane == 0) done1 = mbar_wait(&bar[1], 0, abort_flag, status) ? 1 : 0;
     __syncwarp();
     done1 = __shfl_sync(0xffffffffu, done1, 0);
-    if (done1 && warp < 4) {
+    if (done1) {
         tc_fence_after();
-        const int t = 16 * warp + (lane & 15), hh = lane >> 4;
+        // all 16 warps: warp w reads TMEM lane quadrant w % 4 (M = 64 layout: rows
+        // t = 16 (w % 4) + (lane & 15) in the quadrant's lanes 0-15) at columns
+        // 16 (w / 4) .. + 15 of S and dP0; lanes 16-31 take their row's upper 8
+        const int cg = warp >> 2, t = 16 * quad + (lane & 15), hh = lane >> 4;
         const float bt = sb[t], mtt = smt[t], dnqt = sdnq[t];
-#pragma unroll 1
-        for (int ph = 0; ph < 2; ++ph) {              // 0: S -> M2; 1: dP0 -> M1
-            const uint32_t base = tacc + (ph ? Lay::cP : Lay::cS) + lane_addr;
-            const int ho = ph ? Lay::kM1h : Lay::kM2h, lo_ = ph ? Lay::kM1l : Lay::kM2l;
+        uint32_t ss[16], sp[16];
+        tmem_ld16(tacc + Lay::cS + lane_addr + 16 * cg, ss);
+        tmem_ld16(tacc + Lay::cP + lane_addr + 16 * cg, sp);
+        tmem_wait_ld();
+        uint32_t h1[4], l1[4], h2_[4], l2_[4];
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {    // columns 32 hh + 16 half + [0, 16)
-                uint32_t ra[16], rb[16];
-                tmem_ld16(base + 16 * half, ra);
-                tmem_ld16(base + 32 + 16 * half, rb);
-                tmem_wait_ld();
-                uint32_t hi[8], lo[8];
+        for (int e = 0; e < 8; e += 2) {
+            float m1[2], m2[2];
 #pragma unroll
-                for (int e = 0; e < 16; e += 2) {
-                    float x[2];
-#pragma unroll
-                    for (int u = 0; u < 2; ++u) {
-                        const uint32_t up = __shfl_sync(0xffffffffu, rb[e + u], lane & 15);
-                        const float val = __uint_as_float(hh ? up : ra[e + u]);
-                        const int s_ = 32 * hh + 16 * half + e + u;
-                        const float w = (t < n && s_ <= t) ? expf(bt - sb[s_] + sip[s_] - mtt) : 0.f;
-                        x[u] = ph ? w * (val + dnqt) : w * val * inv_sqrt;
-                    }
-                    hi[e / 2] = cvt_bf16x2(x[0], x[1]);
-                    const __nv_bfloat162 h2 = *reinterpret_cast<const __nv_bfloat162 *>(&hi[e / 2]);
-                    lo[e / 2] = cvt_bf16x2(x[0] - __low2float(h2), x[1] - __high2float(h2));
-                }
-#pragma unroll
-                for (int q = 0; q < 2; ++q) {
-                    const int piece = 4 * hh + 2 * half + q;
-                    const uint32_t off = (uint32_t)t * 128u + ((uint32_t)(piece ^ (t & 7)) << 4);
-                    *reinterpret_cast<uint4 *>(smem + ho + off) = make_uint4(hi[4 * q], hi[4 * q + 1], hi[4 * q + 2], hi[4 * q + 3]);
-                    *reinterpret_cast<uint4 *>(smem + lo_ + off) = make_uint4(lo[4 * q], lo[4 * q + 1], lo[4 * q + 2], lo[4 * q + 3]);
-                }
+            for (int u = 0; u < 2; ++u) {
+                const uint32_t us = __shfl_sync(0xffffffffu, ss[8 + e + u], lane & 15);
+                const uint32_t up = __shfl_sync(0xffffffffu, sp[8 + e + u], lane & 15);
+                const float sv = __uint_as_float(hh ? us : ss[e + u]);
+                const float dp = __uint_as_float(hh ? up : sp[e + u]);
+                const int s_ = 16 * cg + 8 * hh + e + u;
+                const float w = (t < n && s_ <= t) ? expf(bt - sb[s_] + sip[s_] - mtt) : 0.f;
+                m2[u] = w * sv * inv_sqrt;
+                m1[u] = w * (dp + dnqt);
             }
+            h1[e / 2] = cvt_bf16x2(m1[0], m1[1]);
+            const __nv_bfloat162 a1 = *reinterpret_cast<const __nv_bfloat162 *>(&h1[e / 2]);
+            l1[e / 2] = cvt_bf16x2(m1[0] - __low2float(a1), m1[1] - __high2float(a1));
+            h2_[e / 2] = cvt_bf16x2(m2[0], m2[1]);
+            const __nv_bfloat162 a2 = *reinterpret_cast<const __nv_bfloat162 *>(&h2_[e / 2]);
+            l2_[e / 2] = cvt_bf16x2(m2[0] - __low2float(a2), m2[1] - __high2float(a2));
         }
+        const uint32_t off = (uint32_t)t * 128u + ((uint32_t)((2 * cg + hh) ^ (t & 7)) << 4);
+        *reinterpret_cast<uint4 *>(smem + Lay::kM1h + off) = make_uint4(h1[0], h1[1], h1[2], h1[3]);
+        *reinterpret_cast<uint4 *>(smem + Lay::kM1l + off) = make_uint4(l1[0], l1[1], l1[2], l1[3]);
+        *reinterpret_cast<uint4 *>(smem + Lay::kM2h + off) = make_uint4(h2_[0], h2_[1], h2_[2], h2_[3]);
+        *reinterpret_cast<uint4 *>(smem + Lay::kM2l + off) = make_uint4(l2_[0], l2_[1], l2_[2], l2_[3]);
         fence_async_smem();
     }
     tc_fence_before();
