@@ -838,7 +838,8 @@ cudaError_t launch_token_grad_tc_t(const BwdPtrs &p, cudaStream_t st) {
     const int sm = bwdtc::GradLay<D>::kBytes;
     cudaError_t e = cudaFuncSetAttribute(bwdtc::token_grad_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
     if (e != cudaSuccess) return e;
-    bwdtc::token_grad_tc_kernel<D><<<(unsigned)((long long)p.NC * p.BH), bwdtc::kTokThreads, sm, st>>>(
+    const long long items = (long long)p.NC * p.BH, sms = num_sms_current_device();
+    bwdtc::token_grad_tc_kernel<D><<<(unsigned)(items < sms ? items : sms), bwdtc::kTokThreads, sm, st>>>(
         mq, mk, mv, mdh, mdl, p, device_status_ptr());
     return cudaGetLastError();
 }

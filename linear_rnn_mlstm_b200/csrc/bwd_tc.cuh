@@ -767,6 +767,9 @@ struct GradLay {
     static constexpr int cS = 0, cP = 64, cDq = 128, cDk = 128 + 64 * (kTiles<D>), cDv = 128 + 128 * (kTiles<D>);
 };
 
+// Persistent: one CTA per SM walks (chunk, head) items; the next item's tiles
+// are loaded while this item's epilogue runs (all but k at its start, k, which
+// the epilogue still reads, after it).
 template <int D>
 __global__ void __launch_bounds__(kTokThreads, 1)
 token_grad_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
@@ -783,27 +786,45 @@ token_grad_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_con
     uint32_t *tslot = reinterpret_cast<uint32_t *>(smem + Lay::kBar + 32);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + Lay::kBar + 36);
     const int NC = p.NC, S = p.S, L = p.L;
-    const int c = (int)(blockIdx.x % (unsigned)NC), bh = (int)(blockIdx.x / (unsigned)NC);
+    const long long items = (long long)NC * p.BH;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, quad = warp & 3;
-    const int a0 = c * L, n = min(S, a0 + L) - a0;
-    const size_t row0 = (size_t)bh * S + a0, hc = (size_t)bh * NC + c;
     const float inv_sqrt = rsqrtf((float)D);
-
+    // the tiles of item `item` (all five, or all but k / only k)
+    auto load_tiles = [&](long long item, bool arm, bool k_tile, bool others) {
+        const int ci = (int)(item % NC), bhi = (int)(item / NC), ai = ci * L;
+        if (arm) mbar_arrive_expect_tx(&bar[0], 5 * Lay::kTile);
+        for (int a = 0; a < D / 64; ++a) {
+            if (others) {
+                tma_load_3d(smem + Lay::kQ + a * 8192, &map_q, &bar[0], 64 * a, ai, bhi);
+                tma_load_3d(smem + Lay::kV + a * 8192, &map_v, &bar[0], 64 * a, ai, bhi);
+                tma_load_3d(smem + Lay::kDh + a * 8192, &map_dh, &bar[0], 64 * a, ai, bhi);
+                tma_load_3d(smem + Lay::kDl + a * 8192, &map_dl, &bar[0], 64 * a, ai, bhi);
+            }
+            if (k_tile) tma_load_3d(smem + Lay::kK + a * 8192, &map_k, &bar[0], 64 * a, ai, bhi);
+        }
+    };
     if (tid == 0) {
         for (int i = 0; i < 3; ++i) mbar_init(&bar[i], 1);
         *abort_flag = 0;
         fence_mbar_init();
-        mbar_arrive_expect_tx(&bar[0], 5 * Lay::kTile);
-        for (int a = 0; a < D / 64; ++a) {
-            tma_load_3d(smem + Lay::kQ + a * 8192, &map_q, &bar[0], 64 * a, a0, bh);
-            tma_load_3d(smem + Lay::kK + a * 8192, &map_k, &bar[0], 64 * a, a0, bh);
-            tma_load_3d(smem + Lay::kV + a * 8192, &map_v, &bar[0], 64 * a, a0, bh);
-            tma_load_3d(smem + Lay::kDh + a * 8192, &map_dh, &bar[0], 64 * a, a0, bh);
-            tma_load_3d(smem + Lay::kDl + a * 8192, &map_dl, &bar[0], 64 * a, a0, bh);
-        }
+        if ((long long)blockIdx.x < items) load_tiles(blockIdx.x, true, true, true);
     }
     __syncwarp();
     if (warp == 0) tmem_alloc(tslot, 512);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tacc = *tslot;
+    const uint32_t lane_addr = ((uint32_t)(32 * quad)) << 16;
+    // thread 0: a fill of the tiles armed and not yet waited for, and its parity
+    bool loads_pending = (long long)blockIdx.x < items;
+    uint32_t pend_par = 0;
+    int it = 0;
+    for (long long item = blockIdx.x; item < items; item += gridDim.x, ++it) {
+    const int c = (int)(item % NC), bh = (int)(item / NC);
+    const int a0 = c * L, n = min(S, a0 + L) - a0;
+    const size_t row0 = (size_t)bh * S + a0, hc = (size_t)bh * NC + c;
+    const uint32_t par = (uint32_t)it & 1u;
     if (tid < 64) {
         const int t = tid;
         float b = 0.f, ip = -INFINITY, mt = 0.f, dnq = 0.f, A = 0.f, g = 0.f, wk = 0.f;
@@ -825,10 +846,9 @@ token_grad_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_con
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const uint32_t tacc = *tslot;
-    const uint32_t lane_addr = ((uint32_t)(32 * quad)) << 16;
     int ok = 0;
-    if (lane == 0) ok = mbar_wait(&bar[0], 0, abort_flag, status) ? 1 : 0;
+    if (lane == 0) ok = mbar_wait(&bar[0], par, abort_flag, status) ? 1 : 0;
+    if (tid == 0 && ok) loads_pending = false;
     __syncwarp();
     ok = __shfl_sync(0xffffffffu, ok, 0);
     if (ok && tid == 0) {
@@ -849,7 +869,7 @@ token_grad_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_con
     }
     // ---- M1, M2 tiles (warps 0-3: M = 64 layout, row t = 16 quad + (lane & 15))
     int done1 = 0;
-    if (ok && lane == 0) done1 = mbar_wait(&bar[1], 0, abort_flag, status) ? 1 : 0;
+    if (ok && lane == 0) done1 = mbar_wait(&bar[1], par, abort_flag, status) ? 1 : 0;
     __syncwarp();
     done1 = __shfl_sync(0xffffffffu, done1, 0);
     if (done1) {
@@ -925,9 +945,15 @@ token_grad_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_con
         mma_commit(&bar[2]);
     }
     int done2 = 0;
-    if (done1 && lane == 0) done2 = mbar_wait(&bar[2], 0, abort_flag, status) ? 1 : 0;
+    if (done1 && lane == 0) done2 = mbar_wait(&bar[2], par, abort_flag, status) ? 1 : 0;
     __syncwarp();
     done2 = __shfl_sync(0xffffffffu, done2, 0);
+    const long long next = item + gridDim.x;
+    if (done2 && tid == 0 && next < items) {     // the MMAs are done with the tiles: next item's, but k
+        load_tiles(next, true, false, true);
+        loads_pending = true;
+        pend_par = par ^ 1u;
+    }
     if (done2) {
         tc_fence_after();
         const int tg = warp >> 2;
@@ -1011,14 +1037,20 @@ token_grad_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_con
     }
     tc_fence_before();
     __syncthreads();
+    if (done2 && tid == 0 && next < items) load_tiles(next, false, true, false);   // k, read by the epilogue until here
     if (done2 && tid < n) {
         const int s_ = tid;
         const float di = red[s_] + red[64 + s_] + red[128 + s_] + red[192 + s_];
         p.di[row0 + s_] = di;
         p.dF[row0 + s_] = sA[s_] - di;
     }
-    if (tid == 0 && !ok) mbar_wait(&bar[0], 0, nullptr, nullptr);     // no copy left in flight
-    __syncwarp();
+    __syncthreads();
+    if (*abort_flag) break;                          // every thread reads the flag after the barrier
+    }
+    // no copy left in flight into shared memory
+    if (tid == 0 && loads_pending) mbar_wait(&bar[0], pend_par, nullptr, nullptr);
+    tc_fence_before();
+    __syncthreads();
     if (warp == 0) {
         tc_fence_after();
         tmem_dealloc(tacc, 512);
