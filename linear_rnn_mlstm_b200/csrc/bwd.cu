@@ -706,13 +706,14 @@ size_t bwd_layout(long long BH, long long S, long long DH, long long NC, bool tc
                             (size_t)BH * (NC + 1) * DD, (size_t)BH * (NC + 1) * DH,
                             ng * DH, ng * DH,                               // num', dnum'
                             (size_t)BH * NC * DD, (size_t)BH * NC * DH,
-                            xt, xt, xt};                                    // dnum' planes, dk / dv products
+                            xt, xt, xt,                                     // dnum' planes, dk / dv products
+                            tc ? nc * 128 : 0, tc ? nc : 0};                // walk records, decays
     BwdPtrs unused;
     BwdPtrs *t = p ? p : &unused;
     float *dnhl = nullptr;
     float **dst[] = {&t->logf, &t->b, &t->mt, &t->den, &t->nq, &t->A, &t->dF, &t->dnq,
                      &t->mprev, &t->mend, &t->Bsum, &t->Cst, &t->nst, &t->num, &t->dnum,
-                     &t->dCb, &t->dnb, &dnhl, &t->dki, &t->dvi};
+                     &t->dCb, &t->dnb, &dnhl, &t->dki, &t->dvi, &t->wrec, &t->decay};
     static_assert(sizeof(sizes) / sizeof(sizes[0]) == sizeof(dst) / sizeof(dst[0]),
                   "one size per workspace array");
     size_t off = 0;
@@ -777,31 +778,26 @@ cudaError_t launch_state_mma(const BwdPtrs &p, int which, cudaStream_t st) {
     }
 }
 
-// The state recurrences on the tensor cores (bwd_tc.cuh): every chunk's
-// increment at once, then the scan over chunks.
+// The state recurrences on the tensor cores (bwd_tc.cuh): one walk over the
+// chunks per (head, 128-row tile, 64-column block), writing every slot once.
 template <int D, bool REVERSE>
 cudaError_t launch_state_recurrence_t(const BwdPtrs &p, cudaStream_t st) {
-    const int c_first = REVERSE ? 1 : 0, nce = REVERSE ? p.NC - 1 : p.NC;
-    if (nce > 0) {
-        CUtensorMap ma, ma2, mb;
-        const __nv_bfloat16 *dn_hi = reinterpret_cast<const __nv_bfloat16 *>(p.dnhl);
-        const void *a1 = REVERSE ? (const void *)dn_hi : p.v;
-        const void *a2 = REVERSE ? (const void *)(dn_hi + (size_t)p.BH * p.S * D) : p.v;
-        if (!make_map_bf16(&ma, a1, p.BH, p.S, D, true, 64) || !make_map_bf16(&ma2, a2, p.BH, p.S, D, true, 64) ||
-            !make_map_bf16(&mb, REVERSE ? p.q : p.k, p.BH, p.S, D, true, 64))
-            return cudaErrorInvalidValue;
-        const int sm = bwdtc::DeltaLay<D, REVERSE>::kBytes;
-        cudaError_t e = cudaFuncSetAttribute(bwdtc::delta_mma_kernel<D, REVERSE>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
-        if (e != cudaSuccess) return e;
-        KernelTimer timer(REVERSE ? "bwd_reverse_mma" : "bwd_states_mma", st);
-        bwdtc::delta_mma_kernel<D, REVERSE><<<dim3((unsigned)((long long)nce * p.BH), bwdtc::kTiles<D>), bwdtc::kMmaThreads,
-                                              sm, st>>>(ma, ma2, mb, p, c_first, nce, device_status_ptr());
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    }
-    KernelTimer timer(REVERSE ? "bwd_reverse_scan" : "bwd_states_scan", st);
-    const size_t threads = (size_t)D * D / 2 + D / 2;
-    bwdtc::state_scan_kernel<D, REVERSE><<<dim3((unsigned)((threads + 255) / 256), (unsigned)p.BH), 256, 0, st>>>(p);
+    CUtensorMap ma, ma2, mb;
+    const __nv_bfloat16 *dn_hi = reinterpret_cast<const __nv_bfloat16 *>(p.dnhl);
+    const void *a1 = REVERSE ? (const void *)dn_hi : p.v;
+    const void *a2 = REVERSE ? (const void *)(dn_hi + (size_t)p.BH * p.S * D) : p.v;
+    if (!make_map_bf16(&ma, a1, p.BH, p.S, D, true, 64) || !make_map_bf16(&ma2, a2, p.BH, p.S, D, true, 64) ||
+        !make_map_bf16(&mb, REVERSE ? p.q : p.k, p.BH, p.S, D, true, 64))
+        return cudaErrorInvalidValue;
+    const int sm = bwdtc::WalkLay<D, REVERSE>::kBytes;
+    cudaError_t e = cudaFuncSetAttribute(bwdtc::state_walk_kernel<D, REVERSE>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
+    if (e != cudaSuccess) return e;
+    KernelTimer timer(REVERSE ? "bwd_reverse_walk" : "bwd_states_walk", st);
+    const long long slots = (long long)p.BH * p.NC * 64;
+    bwdtc::walk_weights_kernel<REVERSE><<<(unsigned)((slots + 255) / 256), 256, 0, st>>>(p);
+    bwdtc::state_walk_kernel<D, REVERSE><<<dim3((unsigned)p.BH, bwdtc::kTiles<D>, D / 64), bwdtc::kWalkThreads, sm,
+                                           st>>>(ma, ma2, mb, p, device_status_ptr());
     return cudaGetLastError();
 }
 

@@ -91,6 +91,7 @@ struct BwdPtrs {
     // fp32, and the per-token kernels take the state products from:
     void *dnhl;                       // [2][BH, S, DH] bf16: dnum' high, then low part
     float *dki, *dvi;                 // [BH, S, DH]: v_s^T dC~ and dC~ k_s per token
+    float *wrec, *decay;              // [BH, NC, 128] token weights of the state walks, [BH, NC] decays
     int tc;
 };
 

@@ -1,6 +1,6 @@
 // The backward's tensor-core kernels (included by bwd.cu; bf16 inputs, DH 64,
-// 128 or 256): the state increments and scans, the products with the states,
-// and the two per-token passes.
+// 128 or 256): the walks that form the chunk states, the products with the
+// states, and the two per-token passes.
 //
 // The chunkwise backward of "xLSTM: Extended Long Short-Term Memory" (section
 // 2.3's recurrence, stabiliser held fixed per section 2.2) multiplies every
@@ -12,7 +12,7 @@
 // Each runs here as tcgen05 MMAs with an fp32 accumulator in tensor memory:
 // one CTA per (chunk, 128 output columns, head) forms out^T[m][t] = sum_k
 // A[m][k] B[t][k] with M = 128, N = 64 tokens, K = DH.  The state is A, stored
-// by the state kernels as two bf16 planes (x = high + low, 16 significant bits)
+// by the state walks as two bf16 planes (x = high + low, 16 significant bits)
 // in 128 x 64 blocks with 128-byte swizzle, and read by bulk copies: as a
 // K-major operand for C'_c q and dC~_c k, as an MN-major one (the same bytes)
 // for C'_c^T dnum' and dC~_c^T v.  B is the chunk's 64 token rows of q, k, v
@@ -170,299 +170,360 @@ state_mma_kernel(const __grid_constant__ CUtensorMap map_b, const __grid_constan
     }
 }
 
-// ------------------------------------------------------------ state increments
-// The chunk recurrences of the states, C'_{c+1} = decay_c C'_c + dC_c (forward)
-// and dC~_{c-1} = decay_c dC~_c + ddC_c (reverse), split into a parallel part
-// and a scan.  The increments, for every chunk at once on the tensor cores:
-//   dC_c[r][j]  = sum_{s in c} w_s v_s[r] k_s[j],  w_s = e^{B_c - b_s + itilde_s - m_end,c} / sqrt(d)
-//   ddC_c[r][j] = sum_{t in c} g_t dnum'_t[r] q_t[j],  g_t = e^{b_t + m_prev,c - m_t}
-// as one M = 128 (rows r), N = DH (columns j), K = 64 (tokens) product per
-// (chunk, row tile, head): A = (w v)^T, MN-major, formed in shared memory from
-// the TMA-loaded v (or dnum' high + low) tile scaled per token and split into
-// bf16 high and low parts; B = k (or q) as loaded, MN-major.  The fp32
-// accumulator leaves tensor memory as bf16 high / low planes staged in shared
-// memory in the state planes' tile order and stored by two bulk copies into
-// the slot the scan turns into the state (forward: slot c + 1; reverse: slot
-// c - 1).  The normaliser's increment (w_s k_s, or g_t dnq'_t q_t, summed)
-// is formed on the CUDA cores from the same B tile.
-template <int D, bool REVERSE>
-struct DeltaLay {
-    static constexpr int kRaw = 0;                                   // v: 2 boxes; dnum': 2 planes x 2 boxes
-    static constexpr int kRawBytes = REVERSE ? 32768 : 16384;
-    static constexpr int kA = kRaw + kRawBytes;                      // A high, then low: 2 x 16 KB
-    static constexpr int kB = kA + 32768;                            // D / 64 boxes of 64 tokens
-    static constexpr int kIn = kB + D / 64 * 8192;
-    static constexpr int kOut = 2 * (D / 64) * 16384;                // staged planes (over the inputs)
-    static constexpr int kRegion = kIn > kOut ? kIn : kOut;
-    static constexpr int kW = kRegion;                               // w[64], wn[64]
-    static constexpr int kBar = kW + 512;
-    static constexpr int kBytes = kBar + 64 + 1024;
-};
-
+// ------------------------------------------------------------ bulk store
 __device__ __forceinline__ void bulk_store(void *gdst, const void *ssrc, uint32_t bytes) {
     asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst),
                  "r"(tc::smem_u32(ssrc)), "r"(bytes)
                  : "memory");
 }
 
-// grid (chunks x heads, D / 128); chunk c = c_first + blockIdx.x % nce.
+// ------------------------------------------------------------ state walk
+// The chunk recurrences of the states, C'_{c+1} = decay_c C'_c + dC_c (forward)
+// and dC~_{c-1} = decay_c dC~_c + ddC_c (reverse), walked chunk by chunk with
+// the running state in fp32 registers, so that every slot is written once and
+// no increment leaves the chip: one CTA per (head, 128-row tile, 64-column
+// block).  Per chunk the
+// increment is one M = 128 (rows r), N = 64 (columns j), K = 64 (tokens)
+// product on the tensor cores with the token weight moved onto B:
+//   dC_c[r][j]  = sum_{s in c} v_s[r] (w_s k_s[j])
+//   ddC_c[r][j] = sum_{t in c} dnum'_t[r] (g_t q_t[j])
+// A = v (or dnum' as its high and low planes) as loaded by TMA, MN-major; B =
+// the weighted k (or q) tile, split in place into bf16 high and low parts.
+// The token weights (w_s or g_t, and the normaliser's: 1 or dnq'_t) arrive
+// with the tiles as the chunk's 512-byte record, written beforehand by
+// walk_weights_kernel with the chunk decays.  Four warp roles, a ring of
+// stages apart:
+//   warp 13 (loads): refills a stage with a later chunk's tiles and record
+//     once the MMAs that read it completed;
+//   warps 9-12 (transform): form B as soon as a chunk's tiles land and, in
+//     row tile 0, the normaliser's 64 column sums and its walk;
+//   warp 8 (MMA): issues the chunk's MMAs into one of four tensor-memory
+//     buffers;
+//   warps 0-7 (consumers): read the increment out of tensor memory, update
+//     their 32 state elements (row 32 (warp & 3) + lane, columns
+//     32 (warp >> 2) ...) and stage them as bf16 high / low rows; each pair of
+//     warps sharing 32 rows stores them with two 4 KB bulk copies.
+// Walk step i holds the state after i increments: forward slot i (slot 0 =
+// 0), reverse slot NC - 1 - i (slot NC - 1 = the final-state cotangent, or 0).
 template <int D, bool REVERSE>
-__global__ void __launch_bounds__(kMmaThreads, 1)
-delta_mma_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_a2,
-                 const __grid_constant__ CUtensorMap map_b, bwd::BwdPtrs p, int c_first, int nce,
-                 unsigned int *status) {
-    using Lay = DeltaLay<D, REVERSE>;
+struct WalkLay {
+    static constexpr int kStages = REVERSE ? 3 : 4;
+    static constexpr int kBufs = 4;                                  // tensor-memory buffers, 64 columns each
+    static constexpr int kRawA = REVERSE ? 32768 : 16384;            // v: 2 boxes; dnum': 2 planes x 2 boxes
+    static constexpr int kRec = kRawA + 16384;                       // after the B box (high in place) + low part
+    static constexpr int kStage = kRec + 1024;                       // + the chunk's weight record (512 B)
+    static constexpr int kOut = kStages * kStage;                    // 2 x (high 16 KB + low 16 KB) staging
+    static constexpr int kRed = kOut + 65536;                        // column partial sums [2][16][64]
+    static constexpr int kBar = kRed + 8192;
+    static constexpr int kBytes = kBar + 256 + 1024;
+    static constexpr uint32_t kTx = (uint32_t)kRawA + 8192u + 512u;
+};
+constexpr int kWalkThreads = 448;
+
+// The walk's inputs per chunk c of head bh: record [bh, c] = w[64], wn[64]
+// (0 past the chunk's tokens) and decay[bh, c] = e^{B_c + m_prev,c - m_end,c}.
+// Forward: w_s = e^{B_c - b_s + itilde_s - m_end,c} / sqrt(d), wn_s = 1;
+// reverse: g_t = e^{b_t + m_prev,c - m_t}, wn_t = dnq'_t (B_c: the chunk's
+// sum of log f, b: its cumulative sum up to the token).
+// One thread per (chunk, token slot).
+template <bool REVERSE>
+__global__ void __launch_bounds__(256) walk_weights_kernel(bwd::BwdPtrs p) {
+    const size_t g = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const size_t rc = g >> 6;                                        // bh * NC + c
+    if (rc >= (size_t)p.BH * p.NC) return;
+    const int t = (int)(g & 63), c = (int)(rc % (size_t)p.NC), bh = (int)(rc / (size_t)p.NC);
+    const int a0 = c * p.L, n = min(p.S, a0 + p.L) - a0;
+    float w = 0.f, wn = 0.f;
+    if (t < n) {
+        const size_t ts = (size_t)bh * p.S + a0 + t;
+        if (REVERSE) {
+            w = expf(p.b[ts] + p.mprev[rc] - p.mt[ts]);
+            wn = p.dnq[ts];
+        } else {
+            w = expf(p.Bsum[rc] - p.b[ts] + p.ip[ts] - p.mend[rc]) * rsqrtf((float)p.DH);
+            wn = 1.f;
+        }
+    }
+    p.wrec[rc * 128 + t] = w;
+    p.wrec[rc * 128 + 64 + t] = wn;
+    if (t == 0) p.decay[rc] = expf(p.Bsum[rc] + p.mprev[rc] - p.mend[rc]);
+}
+
+template <int D, bool REVERSE>
+__global__ void __launch_bounds__(kWalkThreads, 1)
+state_walk_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_a2,
+                  const __grid_constant__ CUtensorMap map_b, bwd::BwdPtrs p, unsigned int *status) {
+    using Lay = WalkLay<D, REVERSE>;
     using namespace tc;
-    extern __shared__ uint8_t delta_smem_raw[];
-    uint8_t *smem = align1k(delta_smem_raw);
-    float *sw = reinterpret_cast<float *>(smem + Lay::kW), *swn = sw + 64;
-    uint64_t *bar = reinterpret_cast<uint64_t *>(smem + Lay::kBar);
-    uint32_t *tslot = reinterpret_cast<uint32_t *>(smem + Lay::kBar + 16);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + Lay::kBar + 20);
-    const int c = c_first + (int)(blockIdx.x % (unsigned)nce), bh = (int)(blockIdx.x / (unsigned)nce);
-    const int mt = blockIdx.y, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int S = p.S, L = p.L, NC = p.NC;
-    const int a0 = c * L, n = min(S, a0 + L) - a0;
-    const size_t DD = (size_t)D * D, hc = (size_t)bh * NC + c, row0 = (size_t)bh * S + a0;
+    constexpr int NS = Lay::kStages, NB = Lay::kBufs;
+    extern __shared__ uint8_t walk_smem_raw[];
+    uint8_t *smem = align1k(walk_smem_raw);
+    float *red = reinterpret_cast<float *>(smem + Lay::kRed);
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + Lay::kBar);   // [NS] tiles landed
+    uint64_t *bready = full + 4;                                       // [NS] B formed
+    uint64_t *mma_done = full + 8, *tmem_free = full + 12;             // [NB] each
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(smem + Lay::kBar + 128);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + Lay::kBar + 132);
+    const int bh = blockIdx.x, mt = blockIdx.y, kb = blockIdx.z;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int L = p.L, NC = p.NC;
+    const int steps = REVERSE ? NC - 1 : NC;                         // increments walked
+    const size_t DD = (size_t)D * D, hbase = (size_t)bh * NC;
+    uint8_t *slots = reinterpret_cast<uint8_t *>(REVERSE ? p.dCb + hbase * DD : p.Cst + (size_t)bh * (NC + 1) * DD);
+    float *nslots = REVERSE ? p.dnb + hbase * D : p.nst + (size_t)bh * (NC + 1) * D;
+    auto chunk_of = [&](int i) { return REVERSE ? NC - 1 - i : i; };
+    auto slot_of = [&](int i) { return REVERSE ? NC - 1 - i : i; };
+    // the chunk decays, 32 steps to a warp register (lane l: step 32 k + l), the
+    // next block in flight a block ahead
+    auto decay_block = [&](int blk) {
+        const int i = 32 * blk + lane;
+        return i < steps ? p.decay[hbase + chunk_of(i)] : 0.f;
+    };
 
     if (tid == 0) {
-        mbar_init(&bar[0], 1);
-        mbar_init(&bar[1], 1);
+        for (int s = 0; s < NS; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&bready[s], 4);
+        }
+        for (int b = 0; b < NB; ++b) {
+            mbar_init(&mma_done[b], 1);
+            mbar_init(&tmem_free[b], 8);
+        }
         *abort_flag = 0;
         fence_mbar_init();
-        mbar_arrive_expect_tx(&bar[0], (uint32_t)(Lay::kRawBytes + D / 64 * 8192));
-        for (int h = 0; h < 2; ++h) {
-            tma_load_3d(smem + Lay::kRaw + h * 8192, &map_a, &bar[0], 128 * mt + 64 * h, a0, bh);
-            if (REVERSE) tma_load_3d(smem + Lay::kRaw + 16384 + h * 8192, &map_a2, &bar[0], 128 * mt + 64 * h, a0, bh);
-        }
-        for (int a = 0; a < D / 64; ++a) tma_load_3d(smem + Lay::kB + a * 8192, &map_b, &bar[0], 64 * a, a0, bh);
     }
     __syncwarp();
-    if (warp == 0) tmem_alloc(tslot, D);
-    if (tid < 64) {                                  // per-token weights; 0 past the chunk
-        float w = 0.f, wn = 0.f;
-        if (tid < n) {
-            const size_t ts = row0 + tid;
-            if (REVERSE) {
-                w = expf(p.b[ts] + p.mprev[hc] - p.mt[ts]);
-                wn = w * p.dnq[ts];
-            } else {
-                w = expf(p.Bsum[hc] - p.b[ts] + p.ip[ts] - p.mend[hc]) * rsqrtf((float)D);
-                wn = w;
-            }
-        }
-        sw[tid] = w;
-        swn[tid] = wn;
-    }
+    if (warp == 0) tmem_alloc(tslot, 64 * NB);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const uint32_t tacc = *tslot;
-    int ok = 0;
-    if (lane == 0) ok = mbar_wait(&bar[0], 0, abort_flag, status) ? 1 : 0;
-    __syncwarp();                                    // orders the loaded tiles for the whole warp
-    ok = __shfl_sync(0xffffffffu, ok, 0);
-    if (ok) {
-        // A = (w v)^T: every 16-byte piece of the raw tile is scaled by its row's
-        // (token's) weight and split, in place of the same piece in both planes
-        for (int e = tid; e < 16384 / 16; e += kMmaThreads) {
-            const int s = (e * 16 % 8192) / 128;
-            const float w = sw[s];
-            uint4 raw = reinterpret_cast<const uint4 *>(smem + Lay::kRaw)[e];
-            float x[8];
-            const __nv_bfloat16 *rb = reinterpret_cast<const __nv_bfloat16 *>(&raw);
+    const uint32_t tbase = *tslot;
+
+    if (warp < 8) {
+        // ------------------------------------------------ consumers
+        constexpr int kRows = D >= 128 ? 128 : D;                    // rows of a plane block in global memory
+        const int rr = 32 * (warp & 3) + lane, cg = warp >> 2;
+        const int r = 128 * mt + rr, j0 = 64 * kb + 32 * cg;
+        float x[32];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) x[i] = __bfloat162float(rb[i]);
-            if (REVERSE) {
-                const uint4 low = reinterpret_cast<const uint4 *>(smem + Lay::kRaw + 16384)[e];
-                const __nv_bfloat16 *lb = reinterpret_cast<const __nv_bfloat16 *>(&low);
+        for (int e = 0; e < 32; ++e) x[e] = 0.f;
+        if (REVERSE && p.dC && r < D) {
+            const float4 *src = reinterpret_cast<const float4 *>(p.dC + (size_t)bh * DD + (size_t)r * D + j0);
 #pragma unroll
-                for (int i = 0; i < 8; ++i) x[i] += __bfloat162float(lb[i]);
+            for (int e = 0; e < 8; ++e) {
+                const float4 f = src[e];
+                x[4 * e] = f.x; x[4 * e + 1] = f.y; x[4 * e + 2] = f.z; x[4 * e + 3] = f.w;
             }
-            uint32_t hi[4], lo[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const float x0 = w * x[2 * i], x1 = w * x[2 * i + 1];
-                hi[i] = cvt_bf16x2(x0, x1);
-                const __nv_bfloat162 h2 = *reinterpret_cast<const __nv_bfloat162 *>(&hi[i]);
-                lo[i] = cvt_bf16x2(x0 - __low2float(h2), x1 - __high2float(h2));
-            }
-            reinterpret_cast<uint4 *>(smem + Lay::kA)[e] = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-            reinterpret_cast<uint4 *>(smem + Lay::kA + 16384)[e] = make_uint4(lo[0], lo[1], lo[2], lo[3]);
         }
-        fence_async_smem();
-    }
-    __syncthreads();
-    if (ok && tid == 0) {
-        tc_fence_after();
-        const uint32_t idesc = idesc_f32acc(kFmtBF16, kFmtBF16, true, true, 128, D);
-        const uint32_t sa = smem_u32(smem + Lay::kA), sb = smem_u32(smem + Lay::kB);
+        // the 32 rows of this warp pair: staged at row rr, stored from the pair's
+        // first warp by two bulk copies of (up to) 4 KB
+        const int q = warp & 3, nrows = min(32, kRows - 32 * q);
+        const bool issuer = cg == 0 && lane == 0 && nrows > 0;
+        const size_t blk_off = (size_t)(mt * (D / 64) + kb) * kBlkBytes<D> + (size_t)(32 * q) * 128u;
+        auto stage = [&](int buf) {
+            uint8_t *hi = smem + Lay::kOut + buf * 32768;
 #pragma unroll
-        for (int ks = 0; ks < 4; ++ks) {
-            const uint64_t bdesc = sdesc_sw128(sb + ks * 2048, 8192, 1024);
-            mma_bf16_ss(tacc, sdesc_sw128(sa + ks * 2048, 8192, 1024), bdesc, idesc, ks > 0 ? 1u : 0u);
-            mma_bf16_ss(tacc, sdesc_sw128(sa + 16384 + ks * 2048, 8192, 1024), bdesc, idesc, 1u);
-        }
-        mma_commit(&bar[1]);
-    }
-    if (ok && mt == 0) {                             // the normaliser's increment
-        float *dn = REVERSE ? p.dnb + ((size_t)bh * NC + c - 1) * D : p.nst + ((size_t)bh * (NC + 1) + c + 1) * D;
-        for (int j = tid; j < D; j += kMmaThreads) {
-            const uint8_t *box = smem + Lay::kB + (j >> 6) * 8192;
-            float acc = 0.f;
-            for (int s = 0; s < n; ++s) {
-                const uint32_t off = (uint32_t)s * 128u + ((uint32_t)(((j & 63) >> 3) ^ (s & 7)) << 4) +
-                                     ((uint32_t)(j & 7) << 1);
-                acc += swn[s] * __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(box + off));
-            }
-            dn[j] = acc;
-        }
-    }
-    __syncthreads();                                 // the B tile is read: the inputs may be overwritten
-    int done = 0;
-    if (ok && lane == 0) done = mbar_wait(&bar[1], 0, abort_flag, status) ? 1 : 0;
-    __syncwarp();
-    done = __shfl_sync(0xffffffffu, done, 0);
-    if (done) {
-        tc_fence_after();
-        const int rr = 32 * warp + lane;             // this thread's row of the tile
-#pragma unroll 1
-        for (int q = 0; q < D / 16; ++q) {
-            uint32_t v[16];
-            tmem_ld16(tacc + ((uint32_t)(32 * warp) << 16) + 16 * q, v);
-            tmem_wait_ld();
+            for (int pp = 0; pp < 4; ++pp) {
+                uint32_t h[4], l[4];
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                uint32_t hi[4], lo[4];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const float x0 = __uint_as_float(v[8 * half + 2 * i]), x1 = __uint_as_float(v[8 * half + 2 * i + 1]);
-                    hi[i] = cvt_bf16x2(x0, x1);
-                    const __nv_bfloat162 h2 = *reinterpret_cast<const __nv_bfloat162 *>(&hi[i]);
-                    lo[i] = cvt_bf16x2(x0 - __low2float(h2), x1 - __high2float(h2));
+                for (int k = 0; k < 4; ++k) {
+                    const float x0 = x[8 * pp + 2 * k], x1 = x[8 * pp + 2 * k + 1];
+                    h[k] = cvt_bf16x2(x0, x1);
+                    const __nv_bfloat162 h2 = *reinterpret_cast<const __nv_bfloat162 *>(&h[k]);
+                    l[k] = cvt_bf16x2(x0 - __low2float(h2), x1 - __high2float(h2));
                 }
-                const int j0 = 16 * q + 8 * half;
-                const uint32_t off = (uint32_t)(j0 >> 6) * 16384u + (uint32_t)rr * 128u +
-                                     ((uint32_t)(((j0 & 63) >> 3) ^ (rr & 7)) << 4);
-                *reinterpret_cast<uint4 *>(smem + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-                *reinterpret_cast<uint4 *>(smem + (D / 64) * 16384 + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+                const uint32_t off = (uint32_t)rr * 128u + ((uint32_t)((4 * cg + pp) ^ (rr & 7)) << 4);
+                *reinterpret_cast<uint4 *>(hi + off) = make_uint4(h[0], h[1], h[2], h[3]);
+                *reinterpret_cast<uint4 *>(hi + 16384 + off) = make_uint4(l[0], l[1], l[2], l[3]);
+            }
+            fence_async_smem();
+        };
+        auto put = [&](int i) {                      // the pair's issuer: walk step i from buffer i & 1
+            uint8_t *dst = slots + (size_t)slot_of(i) * DD * 4 + blk_off;
+            const uint8_t *src = smem + Lay::kOut + (i & 1) * 32768 + (32 * q) * 128;
+            bulk_store(dst, src, (uint32_t)nrows * 128u);
+            bulk_store(dst + DD * 2, src + 16384, (uint32_t)nrows * 128u);
+            bulk_commit();
+        };
+        // named barrier 2 + q: the 64 threads of warps q and q + 4
+        auto pair_sync = [&]() { asm volatile("bar.sync %0, 64;" ::"r"(2 + q) : "memory"); };
+        stage(0);
+        pair_sync();
+        if (issuer) put(0);
+        float dcur = decay_block(0), dnxt = decay_block(1);
+#pragma unroll 1
+        for (int i = 0; i < steps; ++i) {
+            const float dec = __shfl_sync(0xffffffffu, dcur, i & 31);
+            if ((i & 31) == 31) {
+                dcur = dnxt;
+                dnxt = decay_block((i >> 5) + 2);
+            }
+            const int b = i % NB;
+            int got = 0;
+            if (lane == 0) got = mbar_wait(&mma_done[b], (uint32_t)((i / NB) & 1), abort_flag, status) ? 1 : 0;
+            __syncwarp();
+            got = __shfl_sync(0xffffffffu, got, 0);
+            if (got) {
+                tc_fence_after();
+                uint32_t v0[16], v1[16];
+                const uint32_t ta = tbase + ((uint32_t)(32 * q) << 16) + (uint32_t)(64 * b + 32 * cg);
+                tmem_ld16(ta, v0);
+                tmem_ld16(ta + 16, v1);
+                tmem_wait_ld();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&tmem_free[b]);
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    x[e] = fmaf(x[e], dec, __uint_as_float(v0[e]));
+                    x[16 + e] = fmaf(x[16 + e], dec, __uint_as_float(v1[e]));
+                }
+                stage((i + 1) & 1);
+            }
+            if (issuer) bulk_wait_read_all();        // step i's copies have read their buffer
+            __syncwarp();
+            // both warps' verdicts: a pair leaves together
+            int both;
+            asm volatile("{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
+                         "bar.red.and.pred q, %2, 64, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+                         : "=r"(both) : "r"(got), "r"(2 + q) : "memory");
+            if (!both) break;
+            if (issuer) put(i + 1);
+        }
+        if (issuer) bulk_wait_all();
+    } else if (warp == 8) {
+        // ------------------------------------------------ MMA issue
+        if (lane == 0) {
+            int mmas = 0;
+            const uint32_t idesc = idesc_f32acc(kFmtBF16, kFmtBF16, true, true, 128, 64);
+#pragma unroll 1
+            for (int i = 0; i < steps; ++i) {
+                const int s = i % NS, b = i % NB;
+                if (!mbar_wait(&bready[s], (uint32_t)((i / NS) & 1), abort_flag, status)) break;
+                if (i >= NB && !mbar_wait(&tmem_free[b], (uint32_t)((i / NB - 1) & 1), abort_flag, status)) break;
+                tc_fence_after();
+                const uint32_t sa = smem_u32(smem + s * Lay::kStage), sb = sa + (uint32_t)Lay::kRawA;
+                const uint32_t td = tbase + (uint32_t)(64 * b);
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks) {
+                    const uint64_t ahi = sdesc_sw128(sa + ks * 2048, 8192, 1024);
+                    const uint64_t bhi = sdesc_sw128(sb + ks * 2048, 8192, 1024);
+                    mma_bf16_ss(td, ahi, bhi, idesc, ks > 0 ? 1u : 0u);
+                    mma_bf16_ss(td, ahi, sdesc_sw128(sb + 8192 + ks * 2048, 8192, 1024), idesc, 1u);
+                    if (REVERSE) mma_bf16_ss(td, sdesc_sw128(sa + 16384 + ks * 2048, 8192, 1024), bhi, idesc, 1u);
+                }
+                mma_commit(&mma_done[b]);
+                ++mmas;
+            }
+            // no MMA left in flight
+            if (mmas > 0) mbar_wait(&mma_done[(mmas - 1) % NB], (uint32_t)(((mmas - 1) / NB) & 1), nullptr, nullptr);
+        }
+        __syncwarp();
+    } else if (warp == 13) {
+        // ------------------------------------------------ loads
+        if (lane == 0) {
+            int issued = 0;
+            auto issue = [&](int k) {                // the tiles and weights of walk step k's chunk
+                const int s = k % NS, c = chunk_of(k), a0 = c * L;
+                uint8_t *st = smem + s * Lay::kStage;
+                mbar_arrive_expect_tx(&full[s], Lay::kTx);
+                for (int h = 0; h < 2; ++h) {
+                    tma_load_3d(st + h * 8192, &map_a, &full[s], 128 * mt + 64 * h, a0, bh);
+                    if (REVERSE) tma_load_3d(st + 16384 + h * 8192, &map_a2, &full[s], 128 * mt + 64 * h, a0, bh);
+                }
+                tma_load_3d(st + Lay::kRawA, &map_b, &full[s], 64 * kb, a0, bh);
+                bulk_load(st + Lay::kRec, p.wrec + (hbase + c) * 128, 512, &full[s]);
+            };
+            for (; issued < min(NS, steps); ++issued) issue(issued);
+            // the stage of step k is free once step k's MMAs completed
+#pragma unroll 1
+            for (int k = 0; issued < steps; ++k) {
+                if (!mbar_wait(&mma_done[k % NB], (uint32_t)((k / NB) & 1), abort_flag, status)) break;
+                issue(issued++);
+            }
+            // no copy left in flight (the last copy into each stage)
+            for (int k = max(0, issued - NS); k < issued; ++k)
+                mbar_wait(&full[k % NS], (uint32_t)((k / NS) & 1), nullptr, nullptr);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------ transform
+        // Thread tt forms the pieces 8 t + pp of the B box for the tokens
+        // t = t0 + 16 m (m = 0..3); with the 128-byte swizzle those four pieces
+        // hold the same 8 columns, 8 lp ... 8 lp + 7.
+        const int tt = tid - 288;
+        const bool norm = mt == 0;
+        const int pp = tt & 7, t0 = tt >> 3, lp = pp ^ (t0 & 7);
+        float n_run = 0.f;
+        float dcur = decay_block(0), dnxt = decay_block(1);
+        if (norm && tt < 64) {
+            if (REVERSE && p.dn) n_run = p.dn[(size_t)bh * D + 64 * kb + tt];
+            nslots[(size_t)slot_of(0) * D + 64 * kb + tt] = n_run;
+        }
+#pragma unroll 1
+        for (int i = 0; i < steps; ++i) {
+            const int s = i % NS;
+            uint8_t *bt = smem + s * Lay::kStage + Lay::kRawA;
+            const float *rec = reinterpret_cast<const float *>(smem + s * Lay::kStage + Lay::kRec);
+            const float dec = __shfl_sync(0xffffffffu, dcur, i & 31);
+            if ((i & 31) == 31) {
+                dcur = dnxt;
+                dnxt = decay_block((i >> 5) + 2);
+            }
+            int got = 0;
+            if (lane == 0) got = mbar_wait(&full[s], (uint32_t)((i / NS) & 1), abort_flag, status) ? 1 : 0;
+            __syncwarp();
+            got = __shfl_sync(0xffffffffu, got, 0);
+            float acc[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) acc[k] = 0.f;
+            if (got) {
+#pragma unroll
+                for (int m = 0; m < 4; ++m) {
+                    const int t = t0 + 16 * m, e = 8 * t + pp;
+                    const float wt = rec[t], wn = rec[64 + t];
+                    const uint4 raw = reinterpret_cast<const uint4 *>(bt)[e];
+                    const __nv_bfloat16 *rb = reinterpret_cast<const __nv_bfloat16 *>(&raw);
+                    uint32_t h[4], l[4];
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const float x0 = wt * __bfloat162float(rb[2 * k]), x1 = wt * __bfloat162float(rb[2 * k + 1]);
+                        acc[2 * k] = fmaf(wn, x0, acc[2 * k]);
+                        acc[2 * k + 1] = fmaf(wn, x1, acc[2 * k + 1]);
+                        h[k] = cvt_bf16x2(x0, x1);
+                        const __nv_bfloat162 h2 = *reinterpret_cast<const __nv_bfloat162 *>(&h[k]);
+                        l[k] = cvt_bf16x2(x0 - __low2float(h2), x1 - __high2float(h2));
+                    }
+                    reinterpret_cast<uint4 *>(bt)[e] = make_uint4(h[0], h[1], h[2], h[3]);
+                    reinterpret_cast<uint4 *>(bt + 8192)[e] = make_uint4(l[0], l[1], l[2], l[3]);
+                }
+                fence_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bready[s]);
+            }
+            if (norm) {                              // the normaliser: column sums over the 16 token groups
+                float *rd = red + (i & 1) * 1024 + t0 * 64 + lp * 8;
+                reinterpret_cast<float4 *>(rd)[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+                reinterpret_cast<float4 *>(rd)[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+                if (!group_all<1, 128>(got != 0)) break;
+                if (tt < 64) {
+                    const float *rs = red + (i & 1) * 1024 + tt;
+                    float dn = 0.f;
+#pragma unroll
+                    for (int g = 0; g < 16; ++g) dn += rs[g * 64];
+                    n_run = fmaf(n_run, dec, dn);
+                    nslots[(size_t)slot_of(i + 1) * D + 64 * kb + tt] = n_run;
+                }
+            } else if (!got) {
+                break;
             }
         }
-        fence_async_smem();
     }
     tc_fence_before();
     __syncthreads();
-    if (tid == 0 && done) {
-        uint8_t *slot = reinterpret_cast<uint8_t *>(REVERSE ? p.dCb + ((size_t)bh * NC + c - 1) * DD
-                                                            : p.Cst + ((size_t)bh * (NC + 1) + c + 1) * DD);
-        // staged as 128-row blocks; in global memory a block holds min(DH, 128) rows
-        const uint32_t sbytes = (uint32_t)(D / 64) * 16384u, gbytes = (uint32_t)(D / 64) * kBlkBytes<D>;
-        for (int pl = 0; pl < 2; ++pl)
-            bulk_store(slot + (size_t)pl * DD * 2 + (size_t)mt * gbytes, smem + pl * sbytes, gbytes);
-        bulk_commit();
-        bulk_wait_all();
-    }
-    if (tid == 0 && !ok) mbar_wait(&bar[0], 0, nullptr, nullptr);    // no copy left in flight
-    __syncwarp();
     if (warp == 0) {
         tc_fence_after();
-        tmem_dealloc(tacc, D);
-    }
-}
-
-// The scans: one thread per pair of state elements (one 32-bit word of each
-// bf16 plane; the planes' tile order is the same in every slot, so the
-// recurrence is elementwise on words) or per pair of normaliser elements,
-// walking the chunks with the running values in fp32 registers.  Forward:
-// slot 0 = 0, slot c + 1 = decay_c slot c + increment (read from slot c + 1).
-// Reverse: slot NC - 1 = the final-state cotangent (or 0), slot c - 1 =
-// decay_c slot c + increment (read from slot c - 1).
-template <int D, bool REVERSE>
-__global__ void __launch_bounds__(256) state_scan_kernel(bwd::BwdPtrs p) {
-    const int bh = blockIdx.y, NC = p.NC;
-    const size_t DD = (size_t)D * D;
-    const size_t wi = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
-    const size_t nwords = DD / 2;
-    if (wi >= nwords + D / 2) return;
-    const size_t hbase = (size_t)bh * NC;
-    float x0 = 0.f, x1 = 0.f;
-    if (wi < nwords) {
-        uint8_t *st = reinterpret_cast<uint8_t *>(REVERSE ? p.dCb + hbase * DD : p.Cst + (size_t)bh * (NC + 1) * DD);
-        const size_t slot_bytes = DD * 4;
-        auto put = [&](int slot) {
-            uint32_t *w = reinterpret_cast<uint32_t *>(st + (size_t)slot * slot_bytes) + wi;
-            const uint32_t hi = tc::cvt_bf16x2(x0, x1);
-            const __nv_bfloat162 h2 = *reinterpret_cast<const __nv_bfloat162 *>(&hi);
-            w[0] = hi;
-            w[DD / 2] = tc::cvt_bf16x2(x0 - __low2float(h2), x1 - __high2float(h2));
-        };
-        auto get = [&](int slot, float &d0, float &d1) {
-            const uint32_t *w = reinterpret_cast<const uint32_t *>(st + (size_t)slot * slot_bytes) + wi;
-            const uint32_t hw = w[0], lw = w[DD / 2];
-            const __nv_bfloat162 h2 = *reinterpret_cast<const __nv_bfloat162 *>(&hw);
-            const __nv_bfloat162 l2 = *reinterpret_cast<const __nv_bfloat162 *>(&lw);
-            d0 = __low2float(h2) + __low2float(l2);
-            d1 = __high2float(h2) + __high2float(l2);
-        };
-        if (REVERSE) {
-            if (p.dC) {                                  // (r, j), (r, j + 1) of this word
-                const uint32_t o = (uint32_t)wi * 4u, blk = o >> 14, rem = o & 16383u;
-                const uint32_t rr = rem >> 7, pc = (rem & 127u) >> 4, e = (rem & 15u) >> 1;
-                const int j = (int)((blk % (D / 64)) * 64 + ((pc ^ (rr & 7u)) << 3) + e);
-                const int r = (int)((blk / (D / 64)) * 128 + rr);
-                x0 = p.dC[(size_t)bh * DD + (size_t)r * D + j];
-                x1 = p.dC[(size_t)bh * DD + (size_t)r * D + j + 1];
-            }
-            put(NC - 1);
-            for (int c = NC - 1; c >= 1; --c) {
-                const float decay = expf(p.Bsum[hbase + c] + p.mprev[hbase + c] - p.mend[hbase + c]);
-                float d0, d1;
-                get(c - 1, d0, d1);
-                x0 = x0 * decay + d0;
-                x1 = x1 * decay + d1;
-                put(c - 1);
-            }
-        } else {
-            put(0);
-            for (int c = 0; c < NC; ++c) {
-                const float decay = expf(p.Bsum[hbase + c] + p.mprev[hbase + c] - p.mend[hbase + c]);
-                float d0, d1;
-                get(c + 1, d0, d1);
-                x0 = x0 * decay + d0;
-                x1 = x1 * decay + d1;
-                put(c + 1);
-            }
-        }
-    } else {
-        const int j = 2 * (int)(wi - nwords);
-        float *nv = REVERSE ? p.dnb + hbase * D : p.nst + (size_t)bh * (NC + 1) * D;
-        if (REVERSE) {
-            if (p.dn) {
-                x0 = p.dn[(size_t)bh * D + j];
-                x1 = p.dn[(size_t)bh * D + j + 1];
-            }
-            nv[(size_t)(NC - 1) * D + j] = x0;
-            nv[(size_t)(NC - 1) * D + j + 1] = x1;
-            for (int c = NC - 1; c >= 1; --c) {
-                const float decay = expf(p.Bsum[hbase + c] + p.mprev[hbase + c] - p.mend[hbase + c]);
-                float *d = nv + (size_t)(c - 1) * D + j;
-                x0 = x0 * decay + d[0];
-                x1 = x1 * decay + d[1];
-                d[0] = x0;
-                d[1] = x1;
-            }
-        } else {
-            nv[j] = 0.f;
-            nv[j + 1] = 0.f;
-            for (int c = 0; c < NC; ++c) {
-                const float decay = expf(p.Bsum[hbase + c] + p.mprev[hbase + c] - p.mend[hbase + c]);
-                float *d = nv + (size_t)(c + 1) * D + j;
-                x0 = x0 * decay + d[0];
-                x1 = x1 * decay + d[1];
-                d[0] = x0;
-                d[1] = x1;
-            }
-        }
+        tmem_dealloc(tbase, 64 * NB);
     }
 }
 

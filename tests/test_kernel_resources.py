@@ -20,12 +20,12 @@ STACK_LIMIT = 1024             # default per-thread stack, bytes
 HOT = ("segment_output_tc_kernel", "segment_summary_tc_kernel", "segment_scan_kernel",
        "gate_prologue_kernel", "step_stream_kernel", "step_rows_kernel", "step_state_kernel",
        "headnorm_gate_kernel", "combine_keysplit_kernel", "slstm_cluster_kernel", "state_mma_kernel",
-       "state_fold_kernel", "delta_mma_kernel", "token_fwd_tc_kernel",
+       "state_fold_kernel", "state_walk_kernel", "token_fwd_tc_kernel",
        "token_grad_tc_kernel")
 # threads per CTA the launchers use for the tensor-core and streamed kernels
 LAUNCH_THREADS = {"segment_output_tc_kernel": 448, "segment_summary_tc_kernel": 320,
                   "slstm_cluster_kernel": 256, "state_mma_kernel": 128,
-                  "delta_mma_kernel": 128, "token_fwd_tc_kernel": 512, "token_grad_tc_kernel": 512}
+                  "state_walk_kernel": 384, "token_fwd_tc_kernel": 512, "token_grad_tc_kernel": 512}
 
 
 def _ptxas_report(src):
