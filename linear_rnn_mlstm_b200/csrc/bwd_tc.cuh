@@ -415,8 +415,9 @@ state_walk_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
                 mma_commit(&mma_done[b]);
                 ++mmas;
             }
-            // no MMA left in flight
-            if (mmas > 0) mbar_wait(&mma_done[(mmas - 1) % NB], (uint32_t)(((mmas - 1) / NB) & 1), nullptr, nullptr);
+            // no MMA left in flight (a short bound: this only runs after a timeout)
+            if (mmas > 0)
+                mbar_wait(&mma_done[(mmas - 1) % NB], (uint32_t)(((mmas - 1) / NB) & 1), nullptr, nullptr, 200000000ull);
         }
         __syncwarp();
     } else if (warp == 13) {
@@ -441,9 +442,13 @@ state_walk_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
                 if (!mbar_wait(&mma_done[k % NB], (uint32_t)((k / NB) & 1), abort_flag, status)) break;
                 issue(issued++);
             }
-            // no copy left in flight (the last copy into each stage)
-            for (int k = max(0, issued - NS); k < issued; ++k)
-                mbar_wait(&full[k % NS], (uint32_t)((k / NS) & 1), nullptr, nullptr);
+            // no copy left in flight (the last copy into each stage); one 200 ms
+            // deadline for the whole drain, which only waits after a timeout
+            const uint64_t deadline = globaltimer_ns() + 200000000ull;
+            for (int k = max(0, issued - NS); k < issued; ++k) {
+                const uint64_t now = globaltimer_ns();
+                mbar_wait(&full[k % NS], (uint32_t)((k / NS) & 1), nullptr, nullptr, now < deadline ? deadline - now : 0ull);
+            }
         }
         __syncwarp();
     } else {
