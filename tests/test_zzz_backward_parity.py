@@ -70,6 +70,9 @@ CASES = [
     (1, 1, 100, 256, 64, "sigmoid", False, True, "bf16"),
     (1, 1, 3, 128, 1, "sigmoid", False, True, "bf16"),      # one-token chunks
     (1, 2, 90, 64, 32, "exp", True, True, "bf16"),          # DH 64 (padded 128-row tiles)
+    (1, 2, 50, 128, 64, "sigmoid", False, True, "bf16"),    # one chunk: the reverse walk takes no step
+    (1, 1, 200, 64, 2, "exp", False, True, "bf16"),         # 100 chunks: walks past the stage rings and
+                                                            # the 32-step decay blocks
     (1, 1, 1, 16, 1, "sigmoid", False, True, "f32"),
 ]
 
