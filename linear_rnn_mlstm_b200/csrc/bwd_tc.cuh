@@ -219,6 +219,8 @@ struct WalkLay {
     static constexpr uint32_t kTx = (uint32_t)kRawA + 8192u + 512u;
 };
 constexpr int kWalkThreads = 448;
+static_assert(WalkLay<256, true>::kBytes <= 232448 && WalkLay<256, false>::kBytes <= 232448,
+              "state walk shared memory (227 KB per CTA)");
 
 // The walk's inputs per chunk c of head bh: record [bh, c] = w[64], wn[64]
 // (0 past the chunk's tokens) and decay[bh, c] = e^{B_c + m_prev,c - m_end,c}.
