@@ -704,7 +704,7 @@ size_t bwd_layout(long long BH, long long S, long long DH, long long NC, bool tc
     const size_t sizes[] = {ng, ng, ng, ng, ng, ng, ng, ng,                 // per token
                             nc, nc, nc,                                     // per chunk
                             (size_t)BH * (NC + 1) * DD, (size_t)BH * (NC + 1) * DH,
-                            ng * DH, ng * DH,                               // num', dnum'
+                            ng * DH, tc ? 0 : ng * DH,                      // num', dnum' (fp32 kernels)
                             (size_t)BH * NC * DD, (size_t)BH * NC * DH,
                             xt, xt, xt,                                     // dnum' planes, dk / dv products
                             tc ? nc * 128 : 0, tc ? nc : 0};                // walk records, decays

@@ -81,7 +81,7 @@ struct BwdPtrs {
     float *mprev, *mend, *Bsum;                         // [BH, NC]
     float *Cst;                       // [BH, NC + 1, DH, DH] chunk-start C' (slot NC: final)
     float *nst;                       // [BH, NC + 1, DH]
-    float *num, *dnum;                // [BH, S, DH]
+    float *num, *dnum;                // [BH, S, DH]; dnum on the fp32 kernels only
     float *dCb;                       // [BH, NC, DH, DH] reverse state at the end of chunk c
     float *dnb;                       // [BH, NC, DH]
     int BH, S, DH, L, NC, fgate_exp;

@@ -761,8 +761,7 @@ token_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_cons
                         const float dhr = xd[e][mt];
                         const float dht = dhr * o;
                         p.dO[rowoff + i] = dhr * ht * o * (1.f - o);
-                        const float dn = dht / den;
-                        p.dnum[rowoff + i] = dn;
+                        const float dn = dht / den;      // kept as its high / low planes only
                         const __nv_bfloat16 h16 = __float2bfloat16_rn(dn);
                         hl[rowoff + i] = h16;
                         hl[plane + rowoff + i] = __float2bfloat16_rn(dn - __bfloat162float(h16));
